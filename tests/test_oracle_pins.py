@@ -1,0 +1,413 @@
+"""Pins of the CPU oracle against facts fixed outside it.
+
+No page prints a test vector (no prime list, NTT output, key or ciphertext),
+so each oracle function is pinned by closed forms, invariants, brute force on
+small inputs and by decryption against float64 plaintext arithmetic.  Each
+check is chosen so that a plausible slip (a wrong twiddle or index, a dropped
+term, a sign, a transposed operand) fails at least one of them.
+"""
+import random
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from rns_ckks_polynomial_b200 import synth
+
+from .helpers import N, SCALE, SLOTS, Params, Scheme, galois_for_rotation, rot_left, u64
+
+SEED = synth.config_seed(0)
+
+
+# ------------------------------------------------------------------ helpers
+def _sprp(m, a):
+    """Strong probable-prime test to base a (independent of the oracle)."""
+    d, s = m - 1, 0
+    while d % 2 == 0:
+        d //= 2
+        s += 1
+    x = pow(a, d, m)
+    if x in (1, m - 1):
+        return True
+    for _ in range(s - 1):
+        x = x * x % m
+        if x == m - 1:
+            return True
+    return False
+
+
+def _probably_prime(m):
+    if m < 2:
+        return False
+    for p in (2, 3, 5, 7, 11, 13, 17, 19, 23, 29, 31, 37, 41, 43, 47):
+        if m % p == 0:
+            return m == p
+    rng = random.Random(m)
+    bases = [2, 3, 5, 7, 11, 13] + [rng.randrange(2, m - 1) for _ in range(16)]
+    return all(_sprp(m, a) for a in bases)
+
+
+def _brv(x, bits):
+    return int(format(x, "0%db" % bits)[::-1], 2)
+
+
+def _rand_res(shape, mods, stream):
+    return u64(synth.uniform_residues(shape, mods, SEED, stream))
+
+
+# ------------------------------------------------------------------ primes, psi
+def test_primes_follow_the_scan_rule(orc):
+    P = [int(x) for x in orc.gen_primes(N, 16)]
+    # independent downward scan from 2^60 over candidates 1 mod 2n
+    c = (2**60 - 1) // (2 * N) * (2 * N) + 1
+    expect = []
+    while len(expect) < 16:
+        if _probably_prime(c):
+            expect.append(c)
+        c -= 2 * N
+    assert P == expect
+    for q in P:
+        assert q % (2 * N) == 1 and 2**59 < q < 2**60
+    assert P == sorted(P, reverse=True)
+
+
+def test_first_prime_value(orc):
+    # the largest prime below 2^60 that is 1 mod 4096
+    q0 = int(orc.gen_primes(N, 1)[0])
+    assert q0 == 1152921504606830593
+    for c in range(q0 + 2 * N, 2**60, 2 * N):
+        assert not _probably_prime(c)
+
+
+def test_psi_is_smallest_primitive_root(orc):
+    for q in [int(x) for x in orc.gen_primes(N, 3)]:
+        psi = orc.find_psi(q, N)
+        assert pow(psi, N, q) == q - 1
+        assert pow(psi, 2 * N, q) == 1
+        # independent root: first base g (from 3 upward) whose power has order 2n
+        g = 3
+        while True:
+            x = pow(g, (q - 1) // (2 * N), q)
+            if pow(x, N, q) == q - 1:
+                break
+            g += 1
+        roots = [pow(x, k, q) for k in range(1, 2 * N, 2)]
+        assert psi == min(roots)
+    assert orc.find_psi(1152921504606830593, N) == 459811883340678
+
+
+# ------------------------------------------------------------------ NTT
+def test_ntt_of_monomials_is_the_evaluation_vector(orc):
+    """NTT(1) = all ones and NTT(X) = (psi^(2 brv(k) + 1))_k: fixes the
+    output ordering without using any code under test."""
+    q = int(orc.gen_primes(N, 1)[0])
+    psi = orc.find_psi(q, N)
+    one = np.zeros(N, dtype=np.uint64)
+    one[0] = 1
+    x = np.zeros(N, dtype=np.uint64)
+    x[1] = 1
+    out = orc.ntt_fwd(np.stack([one, x])[:, None, :], [q])
+    assert np.all(out[0, 0] == 1)
+    bits = N.bit_length() - 1
+    expect = [pow(psi, 2 * _brv(k, bits) + 1, q) for k in range(N)]
+    assert [int(v) for v in out[1, 0]] == expect
+
+
+def test_fast_ntt_equals_definition(orc):
+    mods = orc.gen_primes(N, 3)
+    a = _rand_res((3, N), mods, 1)
+    fast = orc.ntt_fwd(a, mods)
+    bits = N.bit_length() - 1
+    for l, q in enumerate(mods):
+        slow = orc.ntt_naive(a[l], q, N)
+        assert np.array_equal(fast[l], slow)
+        # a few outputs straight from the definition with Python integers
+        psi, qq = orc.find_psi(q, N), int(q)
+        coeffs = [int(v) for v in a[l]]
+        for k in (0, 1, 7, 1000, N - 1):
+            w = pow(psi, 2 * _brv(k, bits) + 1, qq)
+            acc = 0
+            for c in reversed(coeffs):
+                acc = (acc * w + c) % qq
+            assert int(fast[l, k]) == acc
+
+
+def test_ntt_roundtrip_identity(orc):
+    mods = orc.gen_primes(N, 3)
+    x = _rand_res((2, 3, N), mods, 2)
+    y = orc.ntt_fwd(x, mods)
+    assert not np.array_equal(x, y)
+    assert np.array_equal(orc.ntt_inv(y, mods), x)
+
+
+def test_negacyclic_schoolbook_tiny(orc):
+    """oracle schoolbook vs numpy full convolution folded by X^n = -1."""
+    n = 16
+    q = int(orc.gen_primes(n, 1)[0])
+    rng = np.random.default_rng(3)
+    a = rng.integers(0, 1000, n)
+    b = rng.integers(0, 1000, n)
+    full = np.convolve(a, b)
+    fold = full[:n].copy()
+    fold[: len(full) - n] -= full[n:]
+    expect = [int(v) % q for v in fold]
+    got = orc.negacyclic_mul(a.astype(np.uint64), b.astype(np.uint64), q)
+    assert [int(v) for v in got] == expect
+
+
+@pytest.mark.parametrize("n", [16, N])
+def test_convolution_theorem(orc, n):
+    q = orc.gen_primes(n, 1)
+    a = _rand_res((1, n), q, 4)
+    b = _rand_res((1, n), q, 5)
+    prod = orc.ntt_inv(orc.pointwise("mul", orc.ntt_fwd(a, q), orc.ntt_fwd(b, q), q), q)
+    assert np.array_equal(prod[0], orc.negacyclic_mul(a[0], b[0], q[0]))
+
+
+# ------------------------------------------------------------------ automorphism
+def test_automorph_coeff_monomials(orc):
+    q = int(orc.gen_primes(N, 1)[0])
+    for j, g in [(1, 5), (500, 5), (3, 4095), (2047, 25)]:
+        x = np.zeros(N, dtype=np.uint64)
+        x[j] = 1
+        out = orc.automorph_coeff(x, q, g)
+        e = j * g % (2 * N)
+        expect = np.zeros(N, dtype=np.uint64)
+        if e < N:
+            expect[e] = 1
+        else:
+            expect[e - N] = q - 1
+        assert np.array_equal(out, expect)
+
+
+@pytest.mark.parametrize("g", [5, 25, 625, 1505, 4095])
+def test_automorph_ntt_permutation_matches_coefficients(orc, g):
+    mods = orc.gen_primes(N, 2)
+    x = _rand_res((2, N), mods, 6)
+    via_ntt = orc.automorph_ntt(orc.ntt_fwd(x, mods), g)
+    coef = np.stack([orc.automorph_coeff(x[l], mods[l], g) for l in range(2)])
+    assert np.array_equal(via_ntt, orc.ntt_fwd(coef, mods))
+    ginv = pow(g, -1, 2 * N)
+    assert np.array_equal(orc.automorph_ntt(via_ntt, ginv), orc.ntt_fwd(x, mods))
+
+
+# ------------------------------------------------------------------ encoding
+def test_encode_constant_closed_form(orc):
+    m = orc.encode(np.full(SLOTS, 0.25), N, SCALE)
+    assert int(m[0]) == SCALE // 4
+    assert np.all(m[1:] == 0)
+
+
+def test_encode_decode_roundtrip_and_rotation(orc):
+    mods = orc.gen_primes(N, 2)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 7).numpy()
+    m = orc.encode(z, N, SCALE)
+    res = np.stack([np.array([int(v) % int(q) for v in m], dtype=np.uint64) for q in mods])
+    back = orc.decode(res, mods, SCALE)
+    assert np.max(np.abs(back - z)) < 1e-12
+    # X -> X^5 rotates slots left by one; X -> X^(5^3) by three
+    for r in (1, 3):
+        g = galois_for_rotation(r)
+        rot = np.stack([orc.automorph_coeff(res[l], mods[l], g) for l in range(2)])
+        assert np.max(np.abs(orc.decode(rot, mods, SCALE) - rot_left(z, r))) < 1e-12
+    # conjugation (g = -1): complex conjugate of every slot
+    zc = z + 1j * synth.uniform_real((SLOTS,), -1, 1, SEED, 8).numpy()
+    mc = orc.encode(zc, N, SCALE)
+    rc = np.stack([np.array([int(v) % int(q) for v in mc], dtype=np.uint64) for q in mods])
+    conj = np.stack([orc.automorph_coeff(rc[l], mods[l], 2 * N - 1) for l in range(2)])
+    assert np.max(np.abs(orc.decode(conj, mods, SCALE) - np.conj(zc))) < 1e-12
+
+
+def test_encoding_is_multiplicative(orc):
+    mods = orc.gen_primes(N, 3)
+    z1 = synth.uniform_real((SLOTS,), -1, 1, SEED, 9).numpy()
+    z2 = synth.uniform_real((SLOTS,), -1, 1, SEED, 10).numpy()
+    m1, m2 = orc.encode(z1, N, SCALE), orc.encode(z2, N, SCALE)
+    r1 = np.stack([np.array([int(v) % int(q) for v in m1], dtype=np.uint64) for q in mods])
+    r2 = np.stack([np.array([int(v) % int(q) for v in m2], dtype=np.uint64) for q in mods])
+    prod = np.stack([orc.negacyclic_mul(r1[l], r2[l], mods[l]) for l in range(3)])
+    assert np.max(np.abs(orc.decode(prod, mods, SCALE * SCALE) - z1 * z2)) < 1e-12
+
+
+# ------------------------------------------------------------------ basis conversion
+def test_basis_conversion_crt_identity(orc):
+    mods = [int(x) for x in orc.gen_primes(N, 8)]
+    src, dst = mods[:3], mods[3:]
+    S = 1
+    for q in src:
+        S *= q
+    rng = random.Random(11)
+    n = 64
+    X = [rng.randrange(S) for _ in range(n)] + [0, S - 1]
+    n = len(X)
+    x = np.array([[v % q for v in X] for q in src], dtype=np.uint64)
+    out = orc.basis_convert(x, np.array(src, dtype=np.uint64), np.array(dst, dtype=np.uint64))
+    for k in range(n):
+        t0 = dst[0]
+        u = (int(out[0, k]) - X[k]) * pow(S, -1, t0) % t0
+        assert 0 <= u < len(src)
+        for t_i, t in enumerate(dst):
+            assert int(out[t_i, k]) == (X[k] + u * S) % t
+
+
+def _crt(res_cols, mods):
+    Q = 1
+    for q in mods:
+        Q *= q
+    x = 0
+    for r, q in zip(res_cols, mods):
+        qh = Q // q
+        x += int(r) * qh * pow(qh % q, -1, q)
+    return x % Q, Q
+
+
+@pytest.mark.parametrize("L,K,alpha", [(6, 2, 2), (5, 2, 2), (4, 1, 1)])
+def test_modup_crt_identity(orc, L, K, alpha):
+    p = Params(L, K, alpha)
+    mods = [int(x) for x in orc.gen_primes(N, L + K)]
+    m64 = np.array(mods, dtype=np.uint64)
+    c = _rand_res((1, L, N), m64[:L], 12)
+    dig = orc.modup(c, m64, L, K, alpha)
+    assert dig.shape == (1, p.dnum, L + K, N)
+    coef_in = orc.ntt_inv(c[0], m64[:L])
+    for j in range(p.dnum):
+        lo, hi = j * alpha, min(L, (j + 1) * alpha)
+        assert np.array_equal(dig[0, j, lo:hi], c[0, lo:hi])
+        coef = orc.ntt_inv(dig[0, j], m64)
+        for k in (0, 5, N - 1):
+            X, Qj = _crt([coef_in[i, k] for i in range(lo, hi)], mods[lo:hi])
+            tgt = [t for t in range(L + K) if not lo <= t < hi]
+            t0 = mods[tgt[0]]
+            u = (int(coef[tgt[0], k]) - X) * pow(Qj, -1, t0) % t0
+            assert 0 <= u < hi - lo
+            for t in tgt:
+                assert int(coef[t, k]) == (X + u * Qj) % mods[t]
+
+
+def test_moddown_floor_identity(orc):
+    L, K = 4, 2
+    mods = [int(x) for x in orc.gen_primes(N, L + K)]
+    m64 = np.array(mods, dtype=np.uint64)
+    acc_coef = _rand_res((1, 2, L + K, N), m64, 13)
+    acc = orc.ntt_fwd(acc_coef, m64)
+    out = orc.moddown(acc, m64, L, K)
+    out_coef = orc.ntt_inv(out, m64[:L])
+    P = 1
+    for q in mods[L:]:
+        P *= q
+    for c in range(2):
+        for k in (0, 9, N - 1):
+            X, _ = _crt([acc_coef[0, c, t, k] for t in range(L + K)], mods)
+            F = X // P
+            v = (F - int(out_coef[0, c, 0, k])) % mods[0]
+            assert 0 <= v < K
+            for i in range(L):
+                assert int(out_coef[0, c, i, k]) == (F - v) % mods[i]
+
+
+def test_rescale_is_exact_floor(orc):
+    lp1 = 5
+    mods = [int(x) for x in orc.gen_primes(N, lp1)]
+    m64 = np.array(mods, dtype=np.uint64)
+    coef = _rand_res((1, 2, lp1, N), m64, 14)
+    out = orc.rescale(orc.ntt_fwd(coef, m64), m64)
+    out_coef = orc.ntt_inv(out, m64[: lp1 - 1])
+    for c in range(2):
+        for k in (0, 3, N - 1):
+            C, _ = _crt([coef[0, c, i, k] for i in range(lp1)], mods)
+            F = C // mods[-1]
+            for i in range(lp1 - 1):
+                assert int(out_coef[0, c, i, k]) == F % mods[i]
+
+
+# ------------------------------------------------------------------ scheme level
+def test_rotation_decrypts_to_slot_rotation_config1(orc):
+    """Tiny RNS-CKKS parameters: 4 ciphertext primes, 1 special, alpha = 1."""
+    sch = Scheme(orc, Params(4, 1, 1), SEED + 1)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 20).numpy()
+    ct = sch.encrypt_slots(z)
+    assert np.max(np.abs(sch.decrypt_slots(ct) - z)) < 1e-8
+    key = sch.keygen_galois(5)
+    out = orc.rotate(ct[None], [key], np.array([5], dtype=np.uint64), sch.mods, 4, 1, 1)
+    err = np.max(np.abs(sch.decrypt_slots(out[0, 0]) - rot_left(z, 1)))
+    assert err < 1e-8
+
+
+def test_hoisted_rotations_small_digits(orc):
+    """Ragged digits (L = 5, alpha = 2) and several keys on one ModUp."""
+    p = Params(5, 2, 2)
+    sch = Scheme(orc, p, SEED + 2)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 21).numpy()
+    ct = sch.encrypt_slots(z)
+    rs = [1, 2, 7]
+    keys = [sch.keygen_galois(galois_for_rotation(r)) for r in rs]
+    gal = np.array([galois_for_rotation(r) for r in rs], dtype=np.uint64)
+    out = orc.rotate(ct[None], keys, gal, sch.mods, p.L, p.K, p.alpha)
+    for i, r in enumerate(rs):
+        assert np.max(np.abs(sch.decrypt_slots(out[i, 0]) - rot_left(z, r))) < 1e-8
+
+
+@pytest.mark.slow
+def test_rotation_and_relin_config3_params(orc):
+    """Layer-shaped parameters: 112 primes, alpha = 8, 8 special primes."""
+    p = Params(112, 8, 8)
+    sch = Scheme(orc, p, SEED + 3)
+    za = synth.uniform_real((SLOTS,), -1, 1, SEED, 30).numpy()
+    zb = synth.uniform_real((SLOTS,), -1, 1, SEED, 31).numpy()
+    ca, cb = sch.encrypt_slots(za), sch.encrypt_slots(zb)
+    g = galois_for_rotation(2)
+    key = sch.keygen_galois(g)
+    out = orc.rotate(ca[None], [key], np.array([g], dtype=np.uint64), sch.mods, 112, 8, 8)
+    assert np.max(np.abs(sch.decrypt_slots(out[0, 0]) - rot_left(za, 2))) < 1e-8
+    rlk = sch.keygen_relin()
+    prod = orc.mul_relin_rescale(ca[None], cb[None], rlk, sch.mods, 112, 8, 8)
+    assert prod.shape == (1, 2, 111, N)
+    sc = sch.rescaled_scale(SCALE * SCALE, 112)
+    assert np.max(np.abs(sch.decrypt_slots(prod[0], sc) - za * zb)) < 1e-8
+
+
+def test_relin_small(orc):
+    p = Params(6, 2, 2)
+    sch = Scheme(orc, p, SEED + 4)
+    za = synth.uniform_real((SLOTS,), -1, 1, SEED, 40).numpy()
+    zb = synth.uniform_real((SLOTS,), -1, 1, SEED, 41).numpy()
+    ca, cb = sch.encrypt_slots(za), sch.encrypt_slots(zb)
+    rlk = sch.keygen_relin()
+    prod = orc.mul_relin_rescale(ca[None], cb[None], rlk, sch.mods, p.L, p.K, p.alpha)
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    assert np.max(np.abs(sch.decrypt_slots(prod[0], sc) - za * zb)) < 1e-8
+
+
+def bsgs_plaintexts(orc, M, bb, gg, mods, scale=SCALE):
+    """pt_{g,b} = Encode(rot_{-bb g}(diag_{bb g + b})), diag_k[i] = M[i][(i+k) mod S]."""
+    S = M.shape[0]
+    idx = np.arange(S)
+    out = []
+    for g in range(gg):
+        row = []
+        for b in range(bb):
+            k = bb * g + b
+            diag = M[idx, (idx + k) % S]
+            row.append(orc.encode_ntt(np.roll(diag, bb * g), mods, scale, N))
+        out.append(np.stack(row))
+    return np.stack(out)
+
+
+def test_bsgs_banded_matvec(orc):
+    """bb = gg = 4 over a matrix with 16 nonzero diagonals: decrypts to M x."""
+    p = Params(6, 2, 2)
+    bb = gg = 4
+    sch = Scheme(orc, p, SEED + 5)
+    rng_m = synth.uniform_real((SLOTS, SLOTS), -1 / 32, 1 / 32, SEED, 50).numpy()
+    idx = np.arange(SLOTS)
+    M = np.zeros((SLOTS, SLOTS))
+    for k in range(bb * gg):
+        M[idx, (idx + k) % SLOTS] = rng_m[idx, (idx + k) % SLOTS]
+    x = synth.uniform_real((SLOTS,), -1, 1, SEED, 51).numpy()
+    ct = sch.encrypt_slots(x)
+    diags = bsgs_plaintexts(orc, M, bb, gg, sch.q)
+    baby = [sch.keygen_galois(galois_for_rotation(b)) for b in range(1, bb)]
+    giant = [sch.keygen_galois(galois_for_rotation(bb * g)) for g in range(1, gg)]
+    y = orc.bsgs(ct[None], diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    assert np.max(np.abs(sch.decrypt_slots(y[0], sc) - M @ x)) < 1e-8
