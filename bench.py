@@ -1,0 +1,524 @@
+#!/usr/bin/env python
+"""Benchmark of the RNS-CKKS hot path on B200.
+
+Workload (one step): the NTT/INTT throughput sweep at n = 2048 -- a batch of
+16 polynomials with seeded uniform residues at each of 3, 112, 512 and 2100
+limbs of 60-bit NTT-friendly primes, forward NTT then inverse NTT, in place;
+the round trip is checked to be the identity after the timed steps.  The
+metric is limb-NTTs per second (forward and inverse both count).
+
+Next to it, the key-switch rates of the three key-switching workloads are
+measured once in the same run (not part of the step): the layer-shaped
+ct x ct multiply (112 primes, alpha 8, 8 pairs), the BSGS matrix-vector
+product (112 primes, bb = gg = 32, 8 ciphertexts) and the boot-level hoisted
+rotation (2100 primes, alpha 60, 4 Galois keys, 8 ciphertexts).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--no-ks]
+
+Under torchrun each rank runs its own batch (weak scaling, no data-path
+collective); the step time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N = 2048
+SWEEP = (3, 112, 512, 2100)
+BATCH = 16
+METRIC = "limb-NTTs/s at n=2048 (NTT+INTT sweep, limbs 3/112/512/2100, batch 16)"
+WORKLOAD = "ntt_sweep_n2048_b16_limbs3-112-512-2100"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-ks", action="store_true", help="skip the key-switch measurements")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi every 200 ms while active."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 6:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if s[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_init(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def max_over_ranks(value, pg):
+    if pg is None:
+        return value
+    import torch
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ---------------------------------------------------------------- roofline bits
+def ntt_launch_work(limbs, batch=BATCH):
+    """Algorithmic bytes and Shoup multiplies of one forward-NTT launch."""
+    jobs = limbs * batch
+    bytes_ = jobs * 2 * N * 8 + limbs * N * 16  # data in+out, {w, w'} per prime
+    mm = jobs * (N // 2) * 11
+    return bytes_, mm
+
+
+def traffic_for(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel_key)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if h != e.get("source_sha256_16"):
+        return None
+    return e["dram_bytes_per_launch"]
+
+
+def intpipe_peaks(ctx):
+    """Same-run integer-pipe microbenchmarks: Shoup multiplies/s and
+    64x64->128 MACs/s over the whole GPU."""
+    out = {}
+    for kind, name in ((0, "shoup_mulmod_per_s"), (1, "mac128_per_s"), (2, "mulhi64_per_s")):
+        best = 0.0
+        for _ in range(3):
+            ms, ops = ctx.bench_intpipe(kind, 148 * 8, 2048)
+            best = max(best, ops / (ms * 1e-3))
+        out[name] = best
+    return out
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_b200(args):
+    import torch
+
+    from rns_ckks_polynomial_b200 import Context, primes, synth
+
+    rank, world, local, pg = dist_init(args)
+    dev = torch.device("cuda", local)
+    hbm_peak, peak_src = peaks()
+    seed = synth.config_seed(2) + 1000 * rank
+    mods = primes(max(SWEEP) + 60)
+    ctx = Context(mods[:max(SWEEP)], mods[max(SWEEP):max(SWEEP) + 60], 60, device=local)
+
+    xs = [synth.uniform_residues((BATCH, l, N), mods[:l], seed, l, device=dev) for l in SWEEP]
+    refs = [x.clone() for x in xs]
+    flush = torch.empty(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        for i, x in enumerate(xs):
+            if ev is not None and i == len(xs) - 1:
+                ev[0].record(stream)
+            ctx.ntt_fwd(x)
+            if ev is not None and i == len(xs) - 1:
+                ev[1].record(stream)
+            ctx.ntt_inv(x)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    ipeak = intpipe_peaks(ctx)
+    barrier(pg)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.zero_()  # L2 flush between steps, outside the timed events
+            starts[s].record(stream)
+            step(kev[s])
+            ends[s].record(stream)
+        torch.cuda.synchronize()
+    barrier(pg)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), pg)
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    # round trip must be the identity after W + K steps
+    ok = all(torch.equal(x, r) for x, r in zip(xs, refs))
+    ok = bool(max_over_ranks(0.0 if ok else 1.0, pg) == 0.0)
+
+    per_step = 2 * BATCH * sum(SWEEP)
+    value = per_step * args.steps * world / (total_ms * 1e-3)
+
+    # roofline of the dominant kernel: forward NTT at 2100 limbs
+    bytes_, mm = ntt_launch_work(2100)
+    t = k_ms * 1e-3
+    t_hbm = bytes_ / (hbm_peak * 1e9)
+    t_alu = mm / ipeak["shoup_mulmod_per_s"]
+    if t_alu > t_hbm:
+        roof = {"bound": "alu", "achieved": mm / t / 1e9, "peak": ipeak["shoup_mulmod_per_s"] / 1e9,
+                "unit": "G Shoup-mulmod/s", "peak_source": "same-run microbenchmark (kind 0)"}
+    else:
+        roof = {"bound": "hbm", "achieved": bytes_ / t / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "peak_source": "%s MEASURED_PEAKS.json hbm_gbs" % peak_src}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for("ntt_fwd_2100")
+    roof["kernel"] = "ntt_fwd_kernel<BatchJob> (16 x 2100 limbs)"
+    roof["launch_ms"] = k_ms
+    roof["hbm_frac_of_measured"] = (bytes_ / t / 1e9) / hbm_peak
+    roof["alu_frac_of_microbench"] = (mm / t) / ipeak["shoup_mulmod_per_s"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "limb-NTTs/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+        "data": "synthetic (seeded uniform residues)",
+        "config": {"workload": WORKLOAD, "n": N, "batch_per_gpu": BATCH, "limbs": list(SWEEP),
+                   "primes": "60-bit, q = 1 mod 4096, descending from 2^60",
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roundtrip_identity": ok,
+        "gpu_launches": 2 * len(SWEEP) * args.steps,
+        "roofline": roof,
+        "intpipe_peaks": ipeak,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(ctx, xs, refs, args, dev, stream, pg, world)
+    if not args.no_ks and rank == 0:
+        del xs, refs
+        torch.cuda.empty_cache()
+        line["keyswitch"] = run_keyswitch(dev, hbm_peak, ipeak)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def run_e2e(ctx, xs, refs, args, dev, stream, pg, world):
+    """Same metric through the public API from pinned host buffers: each step
+    copies its inputs host->device, runs NTT then INTT, and reads the result
+    back."""
+    import torch
+    hosts = [r.cpu().pin_memory() for r in refs]
+    backs = [torch.empty_like(h).pin_memory() for h in hosts]
+    steps = max(3, min(args.steps, 10))
+
+    def step():
+        for h, x, b in zip(hosts, xs, backs):
+            x.copy_(h, non_blocking=True)
+            ctx.ntt_fwd(x)
+            ctx.ntt_inv(x)
+            b.copy_(x, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(pg)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), pg)
+    ok = all(torch.equal(bk, h) for bk, h in zip(backs, hosts))
+    nbytes = sum(h.numel() * 8 for h in hosts)
+    return {"value": 2 * BATCH * sum(SWEEP) * steps * world / (ms * 1e-3), "unit": "limb-NTTs/s",
+            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "steps": steps,
+            "roundtrip_identity": ok}
+
+
+def _time_call(fn, reps, stream):
+    import torch
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_keyswitch(dev, hbm_peak, ipeak):
+    """Key switches per second of the three key-switching workloads."""
+    import torch
+
+    from rns_ckks_polynomial_b200 import Context, primes, synth
+    stream = torch.cuda.current_stream(dev)
+    mm_peak, mac_peak = ipeak["shoup_mulmod_per_s"], ipeak["mac128_per_s"]
+    out = {}
+    # boot-level hoisted rotation: L = 2100, K = 60, alpha = 60, 4 keys, 8 cts
+    seed = synth.config_seed(5)
+    mods = primes(2160)
+    ctx = Context(mods[:2100], mods[2100:], 60, device=dev.index)
+    ct = synth.uniform_residues((8, 2, 2100, N), mods[:2100], seed, 1, device=dev)
+    keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device=dev) for r in range(4)]
+    gal = [5, 25, 625, 1505]
+    res = torch.empty((4, 8, 2, 2100, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(4, 8, 4), dtype=torch.uint8, device=dev)
+    ms = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 3, stream)
+    out["boot_rotation_L2100"] = ks_entry(32, ms, ks_work_rotation(2100, 60, 60, 8, 4), hbm_peak,
+                                          mm_peak, mac_peak)
+    del ct, keys, res, ws, ctx
+    torch.cuda.empty_cache()
+    # layer ct x ct multiply: L = 112, K = 8, alpha = 8, 8 pairs
+    seed = synth.config_seed(3)
+    mods = primes(120)
+    ctx = Context(mods[:112], mods[112:], 8, device=dev.index)
+    a = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 1, device=dev)
+    b = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 2, device=dev)
+    rlk = synth.uniform_residues((14, 2, 120, N), mods, seed, 3, device=dev)
+    res = torch.empty((8, 2, 111, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(6, 8), dtype=torch.uint8, device=dev)
+    ms = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 10, stream)
+    out["layer_mul_relin_L112"] = ks_entry(8, ms, ks_work_mrr(112, 8, 8, 8), hbm_peak, mm_peak, mac_peak)
+    # BSGS: bb = gg = 32, 62 keys, 8 cts
+    seed = synth.config_seed(4)
+    x = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 1, device=dev)
+    diags = synth.uniform_residues((32, 32, 112, N), mods[:112], seed, 2, device=dev)
+    bk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 100 + i, device=dev) for i in range(31)]
+    gk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 200 + i, device=dev) for i in range(31)]
+    y = torch.empty((8, 2, 111, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(7, 8, 32032), dtype=torch.uint8, device=dev)
+    ms = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 3, stream)
+    out["bsgs_L112_32x32"] = ks_entry(8 * 62, ms, ks_work_bsgs(112, 8, 8, 8, 32, 32), hbm_peak,
+                                      mm_peak, mac_peak)
+    return out
+
+
+def ks_work_keyswitch_parts(L, K, alpha):
+    """(MM, MAC) of the parts of one key switch, hybrid method, n = 2048."""
+    dnum = (L + alpha - 1) // alpha
+    LK = L + K
+    ntt = (N // 2) * 11
+    new_limbs = dnum * LK - L
+    modup = {"mm": L * ntt + L * N + new_limbs * ntt, "mac": sum(
+        min(alpha, L - j * alpha) * (LK - min(alpha, L - j * alpha)) for j in range(dnum)) * N}
+    inner = {"mm": 0, "mac": 2 * dnum * LK * N}
+    moddown = {"mm": 2 * (K * ntt + K * N + L * ntt + L * N), "mac": 2 * K * L * N}
+    return modup, inner, moddown
+
+
+def ks_work_rotation(L, K, alpha, B, nkeys):
+    up, inner, down = ks_work_keyswitch_parts(L, K, alpha)
+    mm = B * (up["mm"] + nkeys * (inner["mm"] + down["mm"]))
+    mac = B * (up["mac"] + nkeys * (inner["mac"] + down["mac"]))
+    dnum = (L + alpha - 1) // alpha
+    keyb = nkeys * dnum * 2 * (L + K) * N * 8
+    io = B * 2 * L * N * 8 * (1 + nkeys)
+    return mm, mac, keyb + io
+
+
+def ks_work_mrr(L, K, alpha, B):
+    up, inner, down = ks_work_keyswitch_parts(L, K, alpha)
+    ntt = (N // 2) * 11
+    mm = B * (up["mm"] + down["mm"] + 4 * L * N + 2 * (ntt + (L - 1) * (ntt + N)))
+    mac = B * (up["mac"] + inner["mac"] + down["mac"])
+    dnum = (L + alpha - 1) // alpha
+    keyb = dnum * 2 * (L + K) * N * 8
+    io = B * (4 * L + 2 * (L - 1)) * N * 8
+    return mm, mac, keyb + io
+
+
+def ks_work_bsgs(L, K, alpha, B, bb, gg):
+    up, inner, down = ks_work_keyswitch_parts(L, K, alpha)
+    ntt = (N // 2) * 11
+    baby = up["mm"] + (bb - 1) * down["mm"], up["mac"] + (bb - 1) * (inner["mac"] + down["mac"])
+    giant = (gg - 1) * (up["mm"] + down["mm"]), (gg - 1) * (up["mac"] + inner["mac"] + down["mac"])
+    pt = 0, gg * bb * 2 * L * N
+    resc = 2 * (ntt + (L - 1) * (ntt + N)), 0
+    mm = B * (baby[0] + giant[0] + pt[0] + resc[0])
+    mac = B * (baby[1] + giant[1] + pt[1] + resc[1])
+    dnum = (L + alpha - 1) // alpha
+    keyb = (bb - 1 + gg - 1) * dnum * 2 * (L + K) * N * 8
+    io = gg * bb * L * N * 8 + B * (2 * L + 2 * (L - 1)) * N * 8
+    return mm, mac, keyb + io
+
+
+def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak):
+    mm, mac, bytes_ = work
+    t = ms * 1e-3
+    t_alu = mm / mm_peak + mac / mac_peak
+    t_hbm = bytes_ / (hbm_peak * 1e9)
+    bound = "alu" if t_alu >= t_hbm else "hbm"
+    return {"keyswitches_per_s": nks / t, "ms_per_call": ms, "keyswitches_per_call": nks,
+            "mulmods": mm, "macs": mac, "min_bytes": bytes_, "bound": bound,
+            "roofline_frac": max(t_alu, t_hbm) / t,
+            "alu_frac": t_alu / t, "hbm_frac": t_hbm / t}
+
+
+# ---------------------------------------------------------------- CPU baselines
+def cpu_baseline(min_seconds=10.0):
+    """The oracle as it stands, timed on this host's cores on a bounded sample
+    of the sweep: the 112-limb entry (16 polynomials) forward + inverse,
+    repeated until at least `min_seconds` have elapsed."""
+    import numpy as np
+
+    import oracle
+    from rns_ckks_polynomial_b200 import synth
+    mods = oracle.gen_primes(N, 112)
+    a = synth.uniform_residues((BATCH, 112, N), mods, synth.config_seed(2), 112).numpy()
+    a = a.astype(np.uint64)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        y = oracle.ntt_fwd(a, mods)
+        oracle.ntt_inv(y, mods)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    ntts = reps * 2 * BATCH * 112
+    return {"value": ntts / el, "unit": "limb-NTTs/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d repetitions of 16 x 112-limb NTT + INTT (%.1f s)" % (reps, el)}
+
+
+def run_reference(args):
+    """The CPU oracle as it stands, on the same workload, metric and unit;
+    each step a bounded sample of the sweep (16 x 112-limb NTT + INTT)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from rns_ckks_polynomial_b200 import synth
+    mods = oracle.gen_primes(N, 112)
+    a = synth.uniform_residues((BATCH, 112, N), mods, synth.config_seed(2), 112).numpy()
+    a = a.astype(np.uint64)
+    for _ in range(args.warmup):
+        oracle.ntt_inv(oracle.ntt_fwd(a, mods), mods)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        y = oracle.ntt_fwd(a, mods)
+        oracle.ntt_inv(y, mods)
+    el = time.perf_counter() - t0
+    per_step = 2 * BATCH * 112
+    value = per_step * args.steps / el
+    cores = oracle.num_threads()
+    sample = "16 x 112-limb NTT + INTT per step (the sweep's 112-limb entry)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "limb-NTTs/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u64", "data": "synthetic (seeded uniform residues)",
+        "config": {"workload": WORKLOAD, "n": N, "batch_per_gpu": BATCH, "limbs": list(SWEEP),
+                   "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "limb-NTTs/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "limb-NTTs/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_b200(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,245 @@
+/*
+ * ckks.h -- C ABI of the B200 RNS-CKKS hot-path library (libckks_b200.so).
+ *
+ * What the library computes.  The pages describe a CPU RNS-CKKS engine with
+ * ring degree n = 2048, 1024 slots, scale 2^60 and chains of 112 (layer) and
+ * 2100 (bootstrapping) 60-bit primes (Kestrel FHE relay README, section 1;
+ * Kestrel engine write-up, section 4.1).  Its cost sits in NTT/INTT, RNS basis
+ * conversion, Galois rotation and the baby-step giant-step matmul (Kestrel
+ * engine write-up, section 3 table and the boot profile in section 2 "wall 3",
+ * where coeff_to_slot + slot_to_coeff take 79.1 %); a rotation is a transform
+ * plus a key switch and relinearisation consumes an evaluation key
+ * (EncryptedLLM GPU article, section 2.5).  This header exposes exactly those
+ * operations, each as a hand-written sm_100a CUDA kernel sequence.
+ *
+ * Conventions (apply to every call below):
+ *  - Residues are uint64 in [0, q) for the limb's prime q.  Inputs outside
+ *    that range give unspecified (but memory-safe) results.
+ *  - Tensors are limb-major and contiguous: [batch][component][limb][n],
+ *    n = 2048 coefficients of 8 bytes (16 KiB per limb).
+ *  - Primes: the context holds L ciphertext primes q_0..q_{L-1} followed by K
+ *    special primes p_0..p_{K-1}; "prime index" t < L means q_t, t >= L means
+ *    p_{t-L}.  Digit j of the hybrid key switch is the contiguous block
+ *    q_{j alpha} .. q_{min((j+1) alpha, L) - 1}; dnum = ceil(L / alpha).
+ *  - NTT domain: slot k holds a(psi^(2 brv(k) + 1)), brv = 11-bit reversal,
+ *    psi = the smallest primitive 2n-th root of unity mod the limb's prime.
+ *  - Every tensor pointer is DEVICE memory owned by the caller, 16-byte
+ *    aligned, on the context's device.  The library never frees caller memory.
+ *    Key-pointer arrays (const uint64_t *const *) are HOST arrays of device
+ *    pointers.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Outputs are valid once the stream has synchronised.
+ *  - Outputs may not alias inputs unless a call says so.
+ *  - `ws` is a device workspace of at least ckks_workspace_bytes(...) bytes,
+ *    16-byte aligned, used only for the duration of the call's stream work.
+ *    Passing NULL makes the context allocate (and keep) its own workspace;
+ *    that path calls cudaMalloc and synchronises the device.
+ *  - Status: CKKS_OK (0) or a negative code.  Argument checks run on the host
+ *    before any launch; a failed check launches nothing.  CUDA launch errors
+ *    map to CKKS_ECUDA.  ckks_last_error() returns a thread-local message.
+ *  - A context may be used from several host threads concurrently as long as
+ *    their calls use distinct workspaces.
+ */
+#ifndef CKKS_B200_H
+#define CKKS_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ckks_ctx ckks_ctx;
+typedef void *ckks_stream_t; /* cudaStream_t */
+
+enum ckks_status {
+    CKKS_OK = 0,
+    CKKS_EINVAL = -1,       /* bad argument (null, size, alignment, prime) */
+    CKKS_EUNSUPPORTED = -2, /* valid but outside what the kernels support */
+    CKKS_ECUDA = -3,        /* a CUDA runtime call or launch failed */
+    CKKS_ENOMEM = -4        /* device allocation failed */
+};
+
+/* Operation codes for ckks_workspace_bytes. */
+enum ckks_op {
+    CKKS_OP_MODUP = 1,
+    CKKS_OP_MODDOWN = 2,
+    CKKS_OP_KEYSWITCH = 3,
+    CKKS_OP_ROTATE = 4,
+    CKKS_OP_RESCALE = 5,
+    CKKS_OP_MUL_RELIN_RESCALE = 6,
+    CKKS_OP_BSGS = 7
+};
+
+/* Pointwise operation codes for ckks_pointwise. */
+enum ckks_pointwise_op { CKKS_PW_MUL = 0, CKKS_PW_ADD = 1, CKKS_PW_SUB = 2 };
+
+/* ---------------------------------------------------------------- set-up */
+
+/* Host-only.  Writes the first `count` primes q = 1 (mod 2n), 2^59 < q < 2^60,
+ * scanning downward from 2^60 (largest first).  The pages ask for 60-bit
+ * NTT-friendly primes (Kestrel engine write-up, section 2 "wall 2": "112
+ * 60-bit primes"); the scan order is this library's reading.
+ * Returns CKKS_EINVAL if out is NULL, n is not a power of two in [2, 2^16]
+ * or count < 0, CKKS_EUNSUPPORTED if the interval runs out of primes. */
+int ckks_primes(int n, int count, uint64_t *out);
+
+/* Creates a context on CUDA device `device`: validates the primes (each
+ * prime, distinct, q = 1 mod 2n, q < 2^60), uploads NTT twiddles with Shoup
+ * constants, basis-conversion matrices for ModUp/ModDown and the rescale
+ * constants of the top level.  q: L host values, p: K host values.
+ * Supported: n = 2048, 1 <= L <= 4096, 1 <= K <= 64, 1 <= alpha <= 64,
+ * alpha <= L.  Returns CKKS_EINVAL / CKKS_EUNSUPPORTED / CKKS_ECUDA /
+ * CKKS_ENOMEM with *out untouched on failure. */
+int ckks_ctx_create(const uint64_t *q, int L, const uint64_t *p, int K, int alpha,
+                    int n, int device, ckks_ctx **out);
+
+/* Frees the context's device tables and its own workspace (if any).  Waits
+ * for the device.  NULL is a no-op. */
+void ckks_ctx_destroy(ckks_ctx *ctx);
+
+/* Message for the last non-OK status returned on this host thread. */
+const char *ckks_last_error(void);
+
+/* Context parameters: writes L, K, alpha, dnum, n (any pointer may be NULL). */
+int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n);
+
+/* Bytes of workspace that `op` needs for `batch` inputs.  aux: number of keys
+ * for CKKS_OP_ROTATE, input limb count (level + 1) for CKKS_OP_RESCALE,
+ * bb * 1000 + gg for CKKS_OP_BSGS, ignored otherwise.  Returns 0 for an
+ * unknown op or a null context. */
+size_t ckks_workspace_bytes(const ckks_ctx *ctx, int op, int batch, int aux);
+
+/* ---------------------------------------------------------------- a1/a2: NTT */
+
+/* Forward negacyclic NTT, in place, over x[batch][limbs][n]; local limb l
+ * uses prime index limb_begin + l (0 <= limb_begin, limb_begin + limbs <= L+K).
+ * Natural coefficient order in, bit-reversed evaluation order out.
+ * (Kestrel engine write-up, section 3 table: NTT/INTT turn the O(n^2)
+ * polynomial product into O(n log n).)  batch = 0 or limbs = 0 is a no-op. */
+int ckks_ntt_fwd(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin,
+                 int limbs, ckks_stream_t stream);
+
+/* Exact inverse of ckks_ntt_fwd (includes the factor n^-1), in place. */
+int ckks_ntt_inv(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin,
+                 int limbs, ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a3: pointwise */
+
+/* out = a (op) b mod q per limb, NTT domain, arrays [batch][limbs][n]
+ * (limb l uses prime index limb_begin + l).  op: CKKS_PW_MUL/ADD/SUB.
+ * out may alias a or b.  (ct x pt products of the diagonal method and the
+ * ct x ct tensor product, EncryptedLLM GPU article, section 2.1.) */
+int ckks_pointwise(const ckks_ctx *ctx, int op, const uint64_t *a, const uint64_t *b,
+                   uint64_t *out, int batch, int limb_begin, int limbs,
+                   ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a4: automorphism */
+
+/* Galois automorphism a(X) -> a(X^g) in the NTT domain, a pure index
+ * permutation identical for every limb: out[.][l][k] = in[.][l][k'] with
+ * 2 brv(k') + 1 = g (2 brv(k) + 1) mod 2n.  arrays [rows][n], rows = batch *
+ * limbs.  galois must be odd.  out must not alias in.  (Galois rotation /
+ * conjugation as slot permutation, Kestrel engine write-up, section 3.) */
+int ckks_automorph(const ckks_ctx *ctx, const uint64_t *in, uint64_t *out, int batch,
+                   int limbs, uint32_t galois, ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a5-a7: key switching */
+
+/* ModUp (hybrid key switching, approximate fast basis conversion):
+ * c_ntt[batch][L][n] (NTT over q) -> digits[batch][dnum][L+K][n] (NTT over
+ * q and p).  Digit j's own limbs are copies of the input; every other limb t
+ * holds NTT_t( sum_{i in D_j} [c_i (Q_j/q_i)^-1]_{q_i} [Q_j/q_i]_t ).
+ * (RNS basis conversion as the core of bootstrapping, Kestrel engine
+ * write-up, section 3 table; basis conversion kernel, EncryptedLLM GPU
+ * article, section 3.4.)  ws: CKKS_OP_MODUP bytes. */
+int ckks_modup(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int batch,
+               void *ws, ckks_stream_t stream);
+
+/* Key inner product with the automorphism fused into the digit load:
+ * acc[batch][2][L+K][n] with acc[b][c][t][k] = sum_j phi_g(D_j)[t][k] *
+ * key[j][c][t][k] mod t.  digits [batch][dnum][L+K][n], key
+ * [dnum][2][L+K][n] (component 0 = b, 1 = a).  galois = 1 means no
+ * automorphism. */
+int ckks_key_inner(const ckks_ctx *ctx, const uint64_t *digits, const uint64_t *key,
+                   uint32_t galois, uint64_t *acc, int batch, ckks_stream_t stream);
+
+/* ModDown: acc[batch][2][L+K][n] -> out[batch][2][L][n],
+ * out_i = (acc_i - NTT_i(sum_k [INTT(acc_{p_k}) (P/p_k)^-1]_{p_k} [P/p_k]_{q_i}))
+ *         * P^-1 mod q_i.  ws: CKKS_OP_MODDOWN bytes. */
+int ckks_moddown(const ckks_ctx *ctx, const uint64_t *acc, uint64_t *out, int batch,
+                 void *ws, ckks_stream_t stream);
+
+/* KeySwitch(d) = ModDown(<ModUp(d), key>): d[batch][L][n] (NTT),
+ * key[dnum][2][L+K][n], out[batch][2][L][n].  ws: CKKS_OP_KEYSWITCH bytes. */
+int ckks_keyswitch(const ckks_ctx *ctx, const uint64_t *d, const uint64_t *key,
+                   uint64_t *out, int batch, void *ws, ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a8: rotation */
+
+/* Hoisted rotations: for every key r, out[r][b] = (phi_g(c0) + KS0, KS1)
+ * with KS = ModDown(<phi_g(ModUp(c1)), keys[r]>) and g = galois[r].  ModUp
+ * runs once per ciphertext and is shared by all keys.  ct[batch][2][L][n],
+ * keys: host array of nkeys device pointers to [dnum][2][L+K][n], galois:
+ * host array of nkeys odd elements, out[nkeys][batch][2][L][n].  (Rotation =
+ * transform + key switch, EncryptedLLM GPU article, section 2.5.)
+ * ws: ckks_workspace_bytes(CKKS_OP_ROTATE, batch, nkeys). */
+int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
+                const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
+                ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a10: rescale */
+
+/* Rescale by the last prime of the input level: ct[batch][2][lp1][n] ->
+ * out[batch][2][lp1-1][n], c'_i = (c_i - NTT_i([c]_{q_l})) q_l^-1 mod q_i with
+ * l = lp1 - 1 (floor form).  2 <= lp1 <= L.  (One prime dropped per
+ * multiplication, Kestrel engine write-up, section 2 "wall 2".)
+ * ws: ckks_workspace_bytes(CKKS_OP_RESCALE, batch, lp1). */
+int ckks_rescale(const ckks_ctx *ctx, const uint64_t *ct, uint64_t *out, int lp1,
+                 int batch, void *ws, ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a9: ct x ct */
+
+/* Tensor product, relinearisation and rescale at the top level:
+ * d0 = a0 b0, d1 = a0 b1 + a1 b0, d2 = a1 b1; (d0, d1) + KeySwitch(d2, rlk);
+ * then rescale by q_{L-1}.  a, b [batch][2][L][n], rlk [dnum][2][L+K][n],
+ * out [batch][2][L-1][n].  (Relinearisation after ct x ct multiply,
+ * EncryptedLLM GPU article, section 2.5.)  Requires L >= 2.
+ * ws: CKKS_OP_MUL_RELIN_RESCALE bytes. */
+int ckks_mul_relin_rescale(const ckks_ctx *ctx, const uint64_t *a, const uint64_t *b,
+                           const uint64_t *rlk, uint64_t *out, int batch, void *ws,
+                           ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- a11: BSGS */
+
+/* Baby-step giant-step diagonal matrix-vector product (the engine's matmul2
+ * with BB = GG = 32, Kestrel engine write-up, sections 3 and 4.4):
+ * y = Rescale( sum_{g<gg} Rot_{bb g}( sum_{b<bb} diags[g][b] * Rot_b(x) ) ),
+ * Rot_r with Galois element 5^r mod 2n, baby rotations sharing one ModUp.
+ * x [batch][2][L][n], diags [gg][bb][L][n] (plaintexts in the NTT domain),
+ * baby_keys: bb-1 host pointers (rotation b = 1..bb-1), giant_keys: gg-1
+ * host pointers (rotation bb g, g = 1..gg-1), y [batch][2][L-1][n].
+ * Requires L >= 2, bb >= 1, gg >= 1.
+ * ws: ckks_workspace_bytes(CKKS_OP_BSGS, batch, bb * 1000 + gg). */
+int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                       const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
+                       int bb, int gg, uint64_t *y, int batch, void *ws,
+                       ckks_stream_t stream);
+
+/* ---------------------------------------------------------------- measurement */
+
+/* Integer-pipe microbenchmarks on the context's device (no page counterpart:
+ * they give the roofline denominators).  Each runs `iters` dependency-free
+ * iterations in every thread of a grid of `blocks` x 256 threads and writes
+ * the elapsed milliseconds (CUDA events) to *ms and the operation count to
+ * *ops.  kind 0: 64-bit Shoup modular multiply; kind 1: 64x64->128
+ * multiply-accumulate; kind 2: 64x64 high-half multiply.  Synchronous. */
+int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int iters, double *ms,
+                       double *ops);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKKS_B200_H */

@@ -41,6 +41,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 typedef uint64_t u64;
 typedef int64_t i64;
@@ -810,4 +813,14 @@ void oracle_negacyclic_mul(const u64 *a, const u64 *b, u64 *out, u64 q, int n)
             if (k < n) out[k] = addmod(out[k], p, q);
             else out[k - n] = submod(out[k - n], p, q);
         }
+}
+
+/* Threads an OpenMP parallel-for of this library uses (1 without OpenMP). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }

@@ -63,6 +63,7 @@ def _lib():
                                      C.c_int, C.c_int]
         L.oracle_decrypt.argtypes = [_u64p, _i64p, _u64p, _u64p, C.c_int, C.c_int]
         L.oracle_negacyclic_mul.argtypes = [_u64p, _u64p, _u64p, C.c_uint64, C.c_int]
+        L.oracle_num_threads.restype = C.c_int
     return _LIB
 
 
@@ -80,6 +81,11 @@ def _ptr_array(arrs):
     kept = [_u(a) for a in arrs]
     arr = (_u64p * max(1, len(kept)))(*[p for _, p in kept])
     return kept, arr
+
+
+def num_threads():
+    """Threads the oracle's OpenMP loops use."""
+    return int(_lib().oracle_num_threads())
 
 
 def digit_count(L, alpha):

@@ -1,0 +1,227 @@
+"""Python binding of the C ABI: argument marshalling only.
+
+Tensors are torch int64 (or uint64) CUDA tensors holding uint64 residues in
+the limb-major layout of include/ckks.h; every call runs on the current torch
+CUDA stream of the tensor's device.  Outputs and workspaces are allocated with
+torch when the caller does not pass them.  All arithmetic happens in the CUDA
+library; nothing here computes on the data.
+"""
+import ctypes as C
+
+import torch
+
+from .native import check, lib
+
+N = 2048
+
+PW = {"mul": 0, "add": 1, "sub": 2}
+OP_MODUP, OP_MODDOWN, OP_KEYSWITCH, OP_ROTATE, OP_RESCALE, OP_MRR, OP_BSGS = 1, 2, 3, 4, 5, 6, 7
+
+
+def primes(count, n=N):
+    """First `count` primes q = 1 mod 2n in (2^59, 2^60), largest first (host)."""
+    out = (C.c_uint64 * max(1, count))()
+    check("ckks_primes", lib().ckks_primes(n, count, out))
+    return [int(out[i]) for i in range(count)]
+
+
+def _ptr(t, name, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch tensor" % name)
+    if t.dtype not in (torch.int64, torch.uint64):
+        raise TypeError("%s must be int64/uint64 residues" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(t):
+    return C.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+class Context:
+    """Owns a ckks_ctx: primes q (L) and p (K), digit size alpha."""
+
+    def __init__(self, q, p, alpha, device=0, n=N):
+        self.q, self.p = [int(x) for x in q], [int(x) for x in p]
+        self.L, self.K, self.alpha, self.n = len(self.q), len(self.p), int(alpha), n
+        self.dnum = (self.L + self.alpha - 1) // self.alpha
+        self.device = torch.device("cuda", device)
+        qa = (C.c_uint64 * self.L)(*self.q)
+        pa = (C.c_uint64 * max(1, self.K))(*self.p)
+        h = C.c_void_p()
+        check("ckks_ctx_create",
+              lib().ckks_ctx_create(qa, self.L, pa, self.K, self.alpha, n, device, C.byref(h)))
+        self._h = h
+
+    @property
+    def mods(self):
+        return self.q + self.p
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().ckks_ctx_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------ helpers
+    def _empty(self, *shape):
+        return torch.empty(shape, dtype=torch.int64, device=self.device)
+
+    def workspace_bytes(self, op, batch, aux=0):
+        return int(lib().ckks_workspace_bytes(self._h, op, batch, aux))
+
+    def _ws(self, ws, op, batch, aux=0):
+        need = self.workspace_bytes(op, batch, aux)
+        if ws is None:
+            ws = torch.empty(max(need, 16), dtype=torch.uint8, device=self.device)
+        elif ws.numel() * ws.element_size() < need:
+            raise ValueError("workspace too small: %d < %d bytes" % (ws.numel() * ws.element_size(), need))
+        return ws, C.c_void_p(ws.data_ptr())
+
+    # ------------------------------------------------------------ a1/a2
+    def ntt_fwd(self, x, limb_begin=0):
+        """In place over x[..., limbs, n]."""
+        limbs = x.shape[-2]
+        batch = x.numel() // (limbs * self.n) if x.numel() else 0
+        check("ckks_ntt_fwd", lib().ckks_ntt_fwd(self._h, _ptr(x, "x"), batch, limb_begin, limbs,
+                                                 _stream(x)))
+        return x
+
+    def ntt_inv(self, x, limb_begin=0):
+        limbs = x.shape[-2]
+        batch = x.numel() // (limbs * self.n) if x.numel() else 0
+        check("ckks_ntt_inv", lib().ckks_ntt_inv(self._h, _ptr(x, "x"), batch, limb_begin, limbs,
+                                                 _stream(x)))
+        return x
+
+    # ------------------------------------------------------------ a3/a4
+    def pointwise(self, op, a, b, out=None, limb_begin=0):
+        out = torch.empty_like(a) if out is None else out
+        limbs = a.shape[-2]
+        batch = a.numel() // (limbs * self.n) if a.numel() else 0
+        for t, nm in ((b, "b"), (out, "out")):
+            if t.shape != a.shape:
+                raise ValueError("%s shape mismatch" % nm)
+        check("ckks_pointwise", lib().ckks_pointwise(self._h, PW[op], _ptr(a, "a"), _ptr(b, "b"),
+                                                     _ptr(out, "out"), batch, limb_begin, limbs,
+                                                     _stream(a)))
+        return out
+
+    def automorph(self, x, galois, out=None):
+        out = torch.empty_like(x) if out is None else out
+        limbs = x.shape[-2]
+        batch = x.numel() // (limbs * self.n) if x.numel() else 0
+        check("ckks_automorph", lib().ckks_automorph(self._h, _ptr(x, "in"), _ptr(out, "out"), batch,
+                                                     limbs, int(galois), _stream(x)))
+        return out
+
+    # ------------------------------------------------------------ a5-a7
+    def modup(self, c, out=None, ws=None):
+        B = c.shape[0]
+        _ptr(c, "c_ntt", (B, self.L, self.n))
+        out = self._empty(B, self.dnum, self.L + self.K, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_MODUP, B)
+        check("ckks_modup", lib().ckks_modup(self._h, _ptr(c, "c"), _ptr(out, "digits"), B, wp,
+                                             _stream(c)))
+        return out
+
+    def key_inner(self, digits, key, galois=1, out=None):
+        B = digits.shape[0]
+        LK = self.L + self.K
+        _ptr(digits, "digits", (B, self.dnum, LK, self.n))
+        _ptr(key, "key", (self.dnum, 2, LK, self.n))
+        out = self._empty(B, 2, LK, self.n) if out is None else out
+        check("ckks_key_inner", lib().ckks_key_inner(self._h, _ptr(digits, "digits"), _ptr(key, "key"),
+                                                     int(galois), _ptr(out, "acc"), B,
+                                                     _stream(digits)))
+        return out
+
+    def moddown(self, acc, out=None, ws=None):
+        B = acc.shape[0]
+        _ptr(acc, "acc", (B, 2, self.L + self.K, self.n))
+        out = self._empty(B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_MODDOWN, B)
+        check("ckks_moddown", lib().ckks_moddown(self._h, _ptr(acc, "acc"), _ptr(out, "out"), B, wp,
+                                                 _stream(acc)))
+        return out
+
+    def keyswitch(self, d, key, out=None, ws=None):
+        B = d.shape[0]
+        _ptr(d, "d", (B, self.L, self.n))
+        _ptr(key, "key", (self.dnum, 2, self.L + self.K, self.n))
+        out = self._empty(B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_KEYSWITCH, B)
+        check("ckks_keyswitch", lib().ckks_keyswitch(self._h, _ptr(d, "d"), _ptr(key, "key"),
+                                                     _ptr(out, "out"), B, wp, _stream(d)))
+        return out
+
+    # ------------------------------------------------------------ a8
+    def rotate(self, ct, keys, galois, out=None, ws=None):
+        B = ct.shape[0]
+        nk = len(keys)
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", (self.dnum, 2, self.L + self.K, self.n)).value
+                                        for k in keys])
+        gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
+        out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_ROTATE, B, nk)
+        check("ckks_rotate", lib().ckks_rotate(self._h, _ptr(ct, "ct"), kp, gp, nk, _ptr(out, "out"),
+                                               B, wp, _stream(ct)))
+        return out
+
+    # ------------------------------------------------------------ a9/a10
+    def rescale(self, ct, out=None, ws=None):
+        B, _, lp1, _ = ct.shape
+        out = self._empty(B, 2, lp1 - 1, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_RESCALE, B, lp1)
+        check("ckks_rescale", lib().ckks_rescale(self._h, _ptr(ct, "ct"), _ptr(out, "out"), lp1, B, wp,
+                                                 _stream(ct)))
+        return out
+
+    def mul_relin_rescale(self, a, b, rlk, out=None, ws=None):
+        B = a.shape[0]
+        _ptr(a, "a", (B, 2, self.L, self.n))
+        _ptr(b, "b", (B, 2, self.L, self.n))
+        _ptr(rlk, "rlk", (self.dnum, 2, self.L + self.K, self.n))
+        out = self._empty(B, 2, self.L - 1, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_MRR, B)
+        check("ckks_mul_relin_rescale",
+              lib().ckks_mul_relin_rescale(self._h, _ptr(a, "a"), _ptr(b, "b"), _ptr(rlk, "rlk"),
+                                           _ptr(out, "out"), B, wp, _stream(a)))
+        return out
+
+    # ------------------------------------------------------------ a11
+    def bsgs_lintrans(self, x, diags, baby_keys, giant_keys, bb, gg, out=None, ws=None):
+        B = x.shape[0]
+        _ptr(x, "x", (B, 2, self.L, self.n))
+        _ptr(diags, "diags", (gg, bb, self.L, self.n))
+        kshape = (self.dnum, 2, self.L + self.K, self.n)
+        if len(baby_keys) != bb - 1 or len(giant_keys) != gg - 1:
+            raise ValueError("need bb-1 baby keys and gg-1 giant keys")
+        bk = (C.c_void_p * max(1, bb - 1))(*[_ptr(k, "baby key", kshape).value for k in baby_keys])
+        gk = (C.c_void_p * max(1, gg - 1))(*[_ptr(k, "giant key", kshape).value for k in giant_keys])
+        out = self._empty(B, 2, self.L - 1, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_BSGS, B, bb * 1000 + gg)
+        check("ckks_bsgs_lintrans",
+              lib().ckks_bsgs_lintrans(self._h, _ptr(x, "x"), _ptr(diags, "diags"), bk, gk, bb, gg,
+                                       _ptr(out, "y"), B, wp, _stream(x)))
+        return out
+
+    # ------------------------------------------------------------ measurement
+    def bench_intpipe(self, kind, blocks, iters):
+        """(ms, ops) of the integer-pipe microbenchmark `kind` (0 Shoup mulmod,
+        1 64x64->128 MAC, 2 64-bit high multiply)."""
+        ms, ops = C.c_double(), C.c_double()
+        check("ckks_bench_intpipe",
+              lib().ckks_bench_intpipe(self._h, kind, blocks, iters, C.byref(ms), C.byref(ops)))
+        return ms.value, ops.value

@@ -1,0 +1,155 @@
+// Internal declarations of libckks_b200: context layout, device modular
+// arithmetic, error plumbing.  Not part of the public ABI (see include/ckks.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/ckks.h"
+
+typedef uint64_t u64;
+typedef uint32_t u32;
+
+namespace ckks {
+
+constexpr int kN = 2048;       // ring degree (the only one the kernels support)
+constexpr int kLogN = 11;
+constexpr int kMaxDigit = 64;  // alpha and K bound: sources of one basis conversion
+
+// ---------------------------------------------------------------- per-prime constants
+// 64 bytes per prime, read once per thread per job.
+struct __align__(16) PrimeConst {
+    u64 q;
+    u64 r64, r64p;    // 2^64 mod q and its Shoup constant floor(r64 2^64 / q)
+    u64 mu64;         // floor(2^64 / q)
+    u64 ninv, ninvp;  // n^-1 mod q and its Shoup constant
+    u64 two_q;
+    u64 pad;
+};
+
+// Device tables owned by a context (struct of device pointers, passed by value).
+struct Tables {
+    int L, K, alpha, dnum, LK;
+    const PrimeConst *pc;       // [L+K]
+    const ulonglong2 *tw_fwd;   // [L+K][n]: {psi^brv(k), Shoup}; k = 0 unused
+    const ulonglong2 *tw_inv;   // [L+K][n]: {psi^-brv(k), Shoup}; k = 0 holds psi^-brv(1) n^-1
+    // ModUp: source i (global ciphertext prime index) of its digit
+    const ulonglong2 *up_hatinv;  // [L]: {[(Q_j/q_i)^-1]_{q_i}, Shoup}
+    const u64 *up_mat;            // [dnum][alpha][L+K]: [Q_j/q_i]_t
+    // ModDown
+    const ulonglong2 *dn_hatinv;  // [K]: {[(P/p_k)^-1]_{p_k}, Shoup}
+    const u64 *dn_mat;            // [K][L]: [P/p_k]_{q_i}
+    const ulonglong2 *dn_pinv;    // [L]: {[P^-1]_{q_i}, Shoup}
+};
+
+}  // namespace ckks
+
+struct ckks_ctx {
+    int device = 0;
+    int n = ckks::kN, L = 0, K = 0, alpha = 0, dnum = 0;
+    std::vector<u64> mods;  // L+K host copy
+    ckks::Tables t{};
+    std::vector<void *> allocations;
+    // rescale constants per input level lp1: device [lp1-1] of {q_l^-1 mod q_i, Shoup}
+    std::map<int, ulonglong2 *> rescale_tab;
+    std::mutex mu;
+    void *own_ws = nullptr;
+    size_t own_ws_bytes = 0;
+};
+
+namespace ckks {
+
+// ---------------------------------------------------------------- errors
+int set_error(int code, const std::string &msg);
+int cuda_status(cudaError_t e, const char *what);
+#define CKKS_CHECK_LAUNCH(what)                                        \
+    do {                                                               \
+        cudaError_t _e = cudaGetLastError();                           \
+        if (_e != cudaSuccess) return ::ckks::cuda_status(_e, what);   \
+    } while (0)
+#define CKKS_TRY(expr)              \
+    do {                            \
+        int _rc = (expr);           \
+        if (_rc != CKKS_OK) return _rc; \
+    } while (0)
+
+int check_ctx(const ckks_ctx *ctx);
+int check_ptr(const void *p, const char *name);
+int set_device(const ckks_ctx *ctx);
+// Resolves a workspace: the caller's, or the context's own grown to `bytes`.
+int resolve_ws(ckks_ctx *ctx, void *ws, size_t bytes, void **out);
+const ulonglong2 *rescale_table(ckks_ctx *ctx, int lp1, int *rc);
+
+// ---------------------------------------------------------------- device arithmetic
+// All primes satisfy q < 2^60, so 4q < 2^62 and lazy values never overflow.
+
+__device__ __forceinline__ u64 mulhi(u64 a, u64 b) { return __umul64hi(a, b); }
+
+// a * w mod q up to one extra q: result in [0, 2q) for any 64-bit a, given
+// w < q and wp = floor(w 2^64 / q) (Shoup's precomputed quotient).
+__device__ __forceinline__ u64 shoup_lazy(u64 a, u64 w, u64 wp, u64 q)
+{
+    return a * w - mulhi(a, wp) * q;
+}
+
+__device__ __forceinline__ u64 csub(u64 a, u64 m) { return a >= m ? a - m : a; }
+
+__device__ __forceinline__ u64 shoup(u64 a, u64 w, u64 wp, u64 q)
+{
+    return csub(shoup_lazy(a, w, wp, q), q);
+}
+
+// x = hi 2^64 + lo (any 128-bit value) reduced mod q into [0, q).
+// hi 2^64 mod q comes from Shoup on r64 = 2^64 mod q, lo from a one-step
+// Barrett with mu64 = floor(2^64 / q); each part lies in [0, 2q).
+__device__ __forceinline__ u64 reduce128(u64 hi, u64 lo, const PrimeConst &c)
+{
+    u64 a = shoup_lazy(hi, c.r64, c.r64p, c.q);
+    u64 b = lo - mulhi(lo, c.mu64) * c.q;
+    u64 s = a + b;
+    s = csub(s, c.two_q);
+    return csub(s, c.q);
+}
+
+__device__ __forceinline__ u64 mulmod(u64 a, u64 b, const PrimeConst &c)
+{
+    return reduce128(mulhi(a, b), a * b, c);
+}
+
+__device__ __forceinline__ u64 addmod(u64 a, u64 b, u64 q) { return csub(a + b, q); }
+__device__ __forceinline__ u64 submod(u64 a, u64 b, u64 q) { return a >= b ? a - b : a + q - b; }
+
+// 128-bit accumulator: (hi, lo) += a * b.
+__device__ __forceinline__ void mac128(u64 &hi, u64 &lo, u64 a, u64 b)
+{
+    asm("mad.lo.cc.u64 %0, %2, %3, %0;\n\t"
+        "madc.hi.u64 %1, %2, %3, %1;"
+        : "+l"(lo), "+l"(hi)
+        : "l"(a), "l"(b));
+}
+
+// 11-bit reversal.
+__device__ __forceinline__ u32 brv11(u32 k) { return __brev(k) >> (32 - kLogN); }
+
+// NTT-domain Galois source index: slot k of phi_g(a) reads slot k' of a with
+// 2 brv(k') + 1 = g (2 brv(k) + 1) mod 2n.
+__device__ __forceinline__ u32 galois_src(u32 k, u32 g)
+{
+    u32 e = (g * (2u * brv11(k) + 1u)) & (2u * kN - 1u);
+    return brv11((e - 1u) >> 1);
+}
+
+// ---------------------------------------------------------------- host arithmetic
+u64 host_mulmod(u64 a, u64 b, u64 q);
+u64 host_powmod(u64 a, u64 e, u64 q);
+u64 host_invmod(u64 a, u64 q);
+u64 host_shoup(u64 w, u64 q);
+bool host_is_prime(u64 m);
+u64 host_find_psi(u64 q, int n);
+
+}  // namespace ckks

@@ -1,0 +1,527 @@
+// Hybrid key switching: ModUp, key inner product, ModDown, and the key
+// switch / hoisted rotation entry points built from them.
+//
+// The pages name the operations (RNS basis conversion as the core of the
+// coeff<->slot transforms, Kestrel engine write-up, section 3 table; rotation
+// = transform + key switch and relinearisation with an evaluation key,
+// EncryptedLLM GPU article, section 2.5; the basis-conversion index mapping as
+// the error-prone GPU kernel, same article, section 3.4) but not their
+// formulas.  This file implements the standard full-RNS hybrid method with
+// contiguous digits: approximate ModUp without overflow correction, floor
+// ModDown, and rotation with ModUp hoisted before the automorphism.
+//
+// Kernels:
+//  - INTT of the input limbs with the digit copy and the factor
+//    [(Q_j/q_i)^-1]_{q_i} fused into its load/store (ntt.cuh);
+//  - conv_kernel: the basis-conversion product out_t = sum_s y_s M[s][t],
+//    a (targets x sources) x (sources x coefficients) matrix product with
+//    exact 128-bit accumulation and one reduction per output, on the integer
+//    pipes;
+//  - forward NTT of the new limbs in place;
+//  - key_inner_kernel: the dnum-term inner product with the key, the Galois
+//    permutation applied as a gather on the digit load;
+//  - ModDown: INTT of the special limbs (times [(P/p_k)^-1]), conversion,
+//    forward NTT whose store computes (acc - conv) P^-1 and any fused extra
+//    term (phi_g(c0) for a rotation, the tensor terms for relinearisation).
+#include <algorithm>
+
+#include "internal.cuh"
+#include "ntt.cuh"
+
+namespace ckks {
+
+// ---------------------------------------------------------------- basis conversion
+constexpr int kConvThreads = 128;
+constexpr int kConvTT = 16;  // targets per thread (and per CTA)
+
+template <class Map>
+__global__ void __launch_bounds__(kConvThreads) conv_kernel(Map m, const PrimeConst *__restrict__ pc)
+{
+    __shared__ __align__(16) u64 msm[kMaxDigit * kConvTT];
+    const int z = blockIdx.z;
+    const int S = m.sources(z), T = m.targets(z);
+    const int t0 = blockIdx.y * kConvTT;
+    if (t0 >= T) return;
+    for (int i = threadIdx.x; i < S * kConvTT; i += kConvThreads) {
+        const int s = i / kConvTT, tt = i - s * kConvTT;
+        msm[i] = (t0 + tt < T) ? m.mat(z, s, t0 + tt) : 0;
+    }
+    __syncthreads();
+    const int c = blockIdx.x * kConvThreads + threadIdx.x;
+    const u64 *y = m.src(z) + c;
+    u64 hi[kConvTT], lo[kConvTT];
+#pragma unroll
+    for (int tt = 0; tt < kConvTT; ++tt) hi[tt] = lo[tt] = 0;
+    for (int s = 0; s < S; ++s) {
+        const u64 ys = __ldg(y + (size_t)s * kN);
+        const u64 *mr = msm + s * kConvTT;
+#pragma unroll
+        for (int tt = 0; tt < kConvTT; ++tt) mac128(hi[tt], lo[tt], ys, mr[tt]);
+    }
+#pragma unroll
+    for (int tt = 0; tt < kConvTT; ++tt) {
+        const int ti = t0 + tt;
+        if (ti < T) m.dst(z, ti)[c] = reduce128(hi[tt], lo[tt], pc[m.prime(z, ti)]);
+    }
+}
+
+// ModUp conversion: job z = (b, digit jd); sources are the digit's primes,
+// targets every other prime (ciphertext and special), in index order.
+struct UpConvMap {
+    const u64 *y;
+    u64 *digits;
+    const u64 *matp;
+    int L, LK, alpha, dnum;
+    __device__ __forceinline__ int lo(int z) const { return (z % dnum) * alpha; }
+    __device__ __forceinline__ int sources(int z) const { return min(alpha, L - lo(z)); }
+    __device__ __forceinline__ int targets(int z) const { return LK - sources(z); }
+    __device__ __forceinline__ const u64 *src(int z) const
+    {
+        return y + ((size_t)(z / dnum) * L + lo(z)) * kN;
+    }
+    __device__ __forceinline__ int prime(int z, int ti) const
+    {
+        const int l = lo(z);
+        return ti < l ? ti : ti + sources(z);
+    }
+    __device__ __forceinline__ u64 mat(int z, int s, int ti) const
+    {
+        return matp[(size_t)((z % dnum) * alpha + s) * LK + prime(z, ti)];
+    }
+    __device__ __forceinline__ u64 *dst(int z, int ti) const
+    {
+        return digits + ((size_t)z * LK + prime(z, ti)) * kN;
+    }
+};
+
+// ModDown conversion: job z = (J, component); sources the K special primes,
+// targets the L ciphertext primes.
+struct DownConvMap {
+    const u64 *zsrc;
+    u64 *cv;
+    const u64 *matp;
+    int L, K;
+    __device__ __forceinline__ int sources(int) const { return K; }
+    __device__ __forceinline__ int targets(int) const { return L; }
+    __device__ __forceinline__ const u64 *src(int z) const { return zsrc + (size_t)z * K * kN; }
+    __device__ __forceinline__ int prime(int, int ti) const { return ti; }
+    __device__ __forceinline__ u64 mat(int, int s, int ti) const { return matp[(size_t)s * L + ti]; }
+    __device__ __forceinline__ u64 *dst(int z, int ti) const { return cv + ((size_t)z * L + ti) * kN; }
+};
+
+template <class Map>
+static int launch_conv(const Map &m, int max_targets, int jobs, const Tables &T, cudaStream_t s)
+{
+    if (jobs <= 0 || max_targets <= 0) return CKKS_OK;
+    dim3 grid(kN / kConvThreads, (max_targets + kConvTT - 1) / kConvTT, jobs);
+    conv_kernel<Map><<<grid, kConvThreads, 0, s>>>(m, T.pc);
+    CKKS_CHECK_LAUNCH("conv_kernel");
+    return CKKS_OK;
+}
+
+// ---------------------------------------------------------------- ModUp
+// INTT of source limb i of polynomial b; the load also writes the input limb
+// (NTT domain) into its own digit, the store multiplies by [(Q_j/q_i)^-1].
+template <bool kProduct>
+struct UpInttJob {
+    const u64 *in, *in2;
+    size_t in_bstride;
+    u64 *digits, *y;
+    const ulonglong2 *hatinv;
+    const PrimeConst *pc;
+    int L, LK, alpha, dnum, batch, count;
+    __device__ __forceinline__ int prime(int j) const { return j / batch; }
+    __device__ __forceinline__ void load4(int j, int e, u64 *v) const
+    {
+        const int i = j / batch, b = j - i * batch;
+        const size_t off = (size_t)b * in_bstride + (size_t)i * kN + e;
+        ld4(in + off, v);
+        if (kProduct) {
+            u64 w[4];
+            ld4(in2 + off, w);
+            const PrimeConst c = pc[i];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = mulmod(v[k], w[k], c);
+        }
+        st4(digits + (((size_t)b * dnum + i / alpha) * LK + i) * kN + e, v);
+    }
+    __device__ __forceinline__ void store(int j, int e, u64 v) const
+    {
+        const int i = j / batch, b = j - i * batch;
+        const ulonglong2 h = hatinv[i];
+        y[((size_t)b * L + i) * kN + e] = shoup(v, h.x, h.y, pc[i].q);
+    }
+};
+
+// Forward NTT of the converted limbs, in place.  Jobs are ordered by target
+// prime: for a ciphertext prime t the dnum-1 digits not containing it, for a
+// special prime all dnum digits; batch entries innermost.
+struct UpNttJob {
+    u64 *digits;
+    int L, LK, alpha, dnum, batch, count;
+    __device__ __forceinline__ u64 *row(int j, int *tp) const
+    {
+        const int b = j % batch;
+        int r = j / batch, t, jd;
+        const int per_q = dnum - 1;
+        if (r < L * per_q) {
+            t = r / per_q;
+            const int d = r - t * per_q, own = t / alpha;
+            jd = d < own ? d : d + 1;
+        } else {
+            r -= L * per_q;
+            t = L + r / dnum;
+            jd = r - (t - L) * dnum;
+        }
+        *tp = t;
+        return digits + (((size_t)b * dnum + jd) * LK + t) * kN;
+    }
+    __device__ __forceinline__ int prime(int j) const
+    {
+        int t;
+        row(j, &t);
+        return t;
+    }
+    __device__ __forceinline__ u64 load(int j, int e) const
+    {
+        int t;
+        return row(j, &t)[e];
+    }
+    __device__ __forceinline__ void store4(int j, int e, const u64 *v) const
+    {
+        int t;
+        st4(row(j, &t) + e, v);
+    }
+};
+
+size_t modup_ws_bytes(const ckks_ctx *ctx, int batch) { return limbs_bytes((size_t)batch * ctx->L); }
+
+int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bstride, u64 *digits,
+                int batch, void *ws, cudaStream_t s)
+{
+    if (batch <= 0) return CKKS_OK;
+    const Tables &T = ctx->t;
+    Carve cv(ws);
+    u64 *y = cv.take<u64>((size_t)batch * T.L * kN);
+    if (in2) {
+        UpInttJob<true> j{in, in2, in_bstride, digits, y, T.up_hatinv, T.pc,
+                          T.L, T.LK, T.alpha, T.dnum, batch, T.L * batch};
+        CKKS_TRY(launch_ntt_inv(j, T, s));
+    } else {
+        UpInttJob<false> j{in, nullptr, in_bstride, digits, y, T.up_hatinv, T.pc,
+                           T.L, T.LK, T.alpha, T.dnum, batch, T.L * batch};
+        CKKS_TRY(launch_ntt_inv(j, T, s));
+    }
+    UpConvMap m{y, digits, T.up_mat, T.L, T.LK, T.alpha, T.dnum};
+    CKKS_TRY(launch_conv(m, T.LK - 1, batch * T.dnum, T, s));
+    UpNttJob nj{digits, T.L, T.LK, T.alpha, T.dnum, batch, batch * (T.dnum * T.LK - T.L)};
+    return launch_ntt_fwd(nj, T, s);
+}
+
+// ---------------------------------------------------------------- key inner product
+__global__ void __launch_bounds__(256) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
+                                                        int per_key, int hoisted,
+                                                        u64 *__restrict__ acc, Tables T)
+{
+    const int t = blockIdx.y, z = blockIdx.z;
+    const int k = blockIdx.x * 256 + threadIdx.x;
+    const int r = z / per_key;
+    const int dset = hoisted ? z - r * per_key : z;
+    const u32 g = kl.galois[r];
+    const int src = g == 1u ? k : (int)galois_src((u32)k, g);
+    const size_t LKn = (size_t)T.LK * kN;
+    const u64 *dg = digits + (size_t)dset * T.dnum * LKn + (size_t)t * kN + src;
+    const u64 *kp = kl.key[r] + (size_t)t * kN + k;
+    u64 h0 = 0, l0 = 0, h1 = 0, l1 = 0;
+    for (int j = 0; j < T.dnum; ++j) {
+        const u64 d = __ldg(dg + (size_t)j * LKn);
+        mac128(h0, l0, d, __ldg(kp + (size_t)(2 * j) * LKn));
+        mac128(h1, l1, d, __ldg(kp + (size_t)(2 * j + 1) * LKn));
+    }
+    const PrimeConst pc = T.pc[t];
+    u64 *o = acc + ((size_t)z * 2 * T.LK + t) * kN + k;
+    o[0] = reduce128(h0, l0, pc);
+    o[LKn] = reduce128(h1, l1, pc);
+}
+
+int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, int per_key,
+                    bool hoisted, u64 *acc, int jobs, cudaStream_t s)
+{
+    if (jobs <= 0) return CKKS_OK;
+    const Tables &T = ctx->t;
+    dim3 grid(kN / 256, T.LK, jobs);
+    key_inner_kernel<<<grid, 256, 0, s>>>(digits, kl, per_key, hoisted ? 1 : 0, acc, T);
+    CKKS_CHECK_LAUNCH("key_inner_kernel");
+    return CKKS_OK;
+}
+
+// ---------------------------------------------------------------- ModDown
+struct DownInttJob {
+    const u64 *acc;
+    u64 *zdst;
+    const ulonglong2 *hatinv;
+    const PrimeConst *pc;
+    int L, K, LK, jobs2, count;
+    __device__ __forceinline__ int prime(int j) const { return L + j / jobs2; }
+    __device__ __forceinline__ void load4(int j, int e, u64 *v) const
+    {
+        const int k = j / jobs2, zz = j - k * jobs2;
+        ld4(acc + ((size_t)zz * LK + L + k) * kN + e, v);
+    }
+    __device__ __forceinline__ void store(int j, int e, u64 v) const
+    {
+        const int k = j / jobs2, zz = j - k * jobs2;
+        const ulonglong2 h = hatinv[k];
+        zdst[((size_t)zz * K + k) * kN + e] = shoup(v, h.x, h.y, pc[L + k].q);
+    }
+};
+
+template <int kKind>
+struct DownFinalJob {
+    u64 *cv;
+    const u64 *acc;
+    u64 *out;
+    const ulonglong2 *pinv;
+    const PrimeConst *pc;
+    int L, LK, jobs2, count;
+    DownExtra ex;
+    __device__ __forceinline__ int prime(int j) const { return j / jobs2; }
+    __device__ __forceinline__ u64 load(int j, int e) const
+    {
+        const int i = j / jobs2, zz = j - i * jobs2;
+        return cv[((size_t)zz * L + i) * kN + e];
+    }
+    __device__ __forceinline__ void store4(int j, int e, const u64 *v) const
+    {
+        const int i = j / jobs2, zz = j - i * jobs2;
+        const int z = zz >> 1, comp = zz & 1;
+        const u64 q = pc[i].q;
+        const ulonglong2 pv = pinv[i];
+        u64 a[4], o[4];
+        ld4(acc + ((size_t)zz * LK + i) * kN + e, a);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = shoup(submod(a[c], v[c], q), pv.x, pv.y, q);
+        if (kKind == 1 && comp == 0) {
+            const int ci = ex.ct_mod ? z % ex.ct_mod : z;
+            const u64 *c0 = ex.ct + (size_t)ci * ex.ct_bstride + (size_t)i * kN;
+            const u32 g = ex.gal[z / ex.per];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[c] = addmod(o[c], __ldg(c0 + galois_src((u32)(e + c), g)), q);
+        }
+        if (kKind == 2) {
+            const PrimeConst pcc = pc[i];
+            const size_t base = (size_t)z * 2 * L * kN + (size_t)i * kN + e, Ln = (size_t)L * kN;
+            u64 a0[4], b0[4], a1[4], b1[4];
+            ld4(ex.a + base, a0);
+            ld4(ex.b + base, b0);
+            if (comp == 0) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) o[c] = addmod(o[c], mulmod(a0[c], b0[c], pcc), q);
+            } else {
+                ld4(ex.a + base + Ln, a1);
+                ld4(ex.b + base + Ln, b1);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    u64 hi = 0, lo = 0;
+                    mac128(hi, lo, a0[c], b1[c]);
+                    mac128(hi, lo, a1[c], b0[c]);
+                    o[c] = addmod(o[c], reduce128(hi, lo, pcc), q);
+                }
+            }
+        }
+        st4(out + ((size_t)zz * L + i) * kN + e, o);
+    }
+};
+
+size_t moddown_ws_bytes(const ckks_ctx *ctx, int jobs)
+{
+    return limbs_bytes((size_t)jobs * 2 * ctx->K) + limbs_bytes((size_t)jobs * 2 * ctx->L);
+}
+
+int moddown_stage(const ckks_ctx *ctx, const u64 *acc, u64 *out, int jobs, const DownExtra &ex,
+                  void *ws, cudaStream_t s)
+{
+    if (jobs <= 0) return CKKS_OK;
+    const Tables &T = ctx->t;
+    const int jobs2 = 2 * jobs;
+    Carve c(ws);
+    u64 *zb = c.take<u64>((size_t)jobs2 * T.K * kN);
+    u64 *cvb = c.take<u64>((size_t)jobs2 * T.L * kN);
+    DownInttJob ij{acc, zb, T.dn_hatinv, T.pc, T.L, T.K, T.LK, jobs2, T.K * jobs2};
+    CKKS_TRY(launch_ntt_inv(ij, T, s));
+    DownConvMap m{zb, cvb, T.dn_mat, T.L, T.K};
+    CKKS_TRY(launch_conv(m, T.L, jobs2, T, s));
+    switch (ex.kind) {
+    case 1: {
+        DownFinalJob<1> fj{cvb, acc, out, T.dn_pinv, T.pc, T.L, T.LK, jobs2, T.L * jobs2, ex};
+        return launch_ntt_fwd(fj, T, s);
+    }
+    case 2: {
+        DownFinalJob<2> fj{cvb, acc, out, T.dn_pinv, T.pc, T.L, T.LK, jobs2, T.L * jobs2, ex};
+        return launch_ntt_fwd(fj, T, s);
+    }
+    default: {
+        DownFinalJob<0> fj{cvb, acc, out, T.dn_pinv, T.pc, T.L, T.LK, jobs2, T.L * jobs2, ex};
+        return launch_ntt_fwd(fj, T, s);
+    }
+    }
+}
+
+}  // namespace ckks
+
+// ---------------------------------------------------------------- entry points
+using namespace ckks;
+
+namespace {
+
+int check_batch(int batch)
+{
+    if (batch < 0) return set_error(CKKS_EINVAL, "negative batch");
+    if (batch > 65535) return set_error(CKKS_EUNSUPPORTED, "batch above 65535");
+    return CKKS_OK;
+}
+
+size_t keyswitch_ws(const ckks_ctx *ctx, int batch)
+{
+    return limbs_bytes((size_t)batch * ctx->dnum * (ctx->L + ctx->K)) +
+           limbs_bytes((size_t)batch * 2 * (ctx->L + ctx->K)) +
+           std::max(modup_ws_bytes(ctx, batch), moddown_ws_bytes(ctx, batch));
+}
+
+size_t rotate_ws(const ckks_ctx *ctx, int batch, int nkeys)
+{
+    const int chunk = std::min(std::max(nkeys, 1), kMaxKeys);
+    return limbs_bytes((size_t)batch * ctx->dnum * (ctx->L + ctx->K)) +
+           limbs_bytes((size_t)chunk * batch * 2 * (ctx->L + ctx->K)) +
+           std::max(modup_ws_bytes(ctx, batch), moddown_ws_bytes(ctx, chunk * batch));
+}
+
+}  // namespace
+
+namespace ckks {
+size_t keyswitch_ws_bytes(const ckks_ctx *ctx, int batch) { return keyswitch_ws(ctx, batch); }
+size_t rotate_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys) { return rotate_ws(ctx, batch, nkeys); }
+}  // namespace ckks
+
+extern "C" int ckks_modup(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int batch,
+                          void *ws, ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(c_ntt, "c_ntt"));
+    CKKS_TRY(check_ptr(digits, "digits"));
+    CKKS_TRY(set_device(ctx));
+    void *w;
+    ckks_ctx *mctx = const_cast<ckks_ctx *>(ctx);
+    CKKS_TRY(resolve_ws(mctx, ws, modup_ws_bytes(ctx, batch), &w));
+    return modup_stage(ctx, c_ntt, nullptr, (size_t)ctx->L * kN, digits, batch, w,
+                       (cudaStream_t)stream);
+}
+
+extern "C" int ckks_key_inner(const ckks_ctx *ctx, const uint64_t *digits, const uint64_t *key,
+                              uint32_t galois, uint64_t *acc, int batch, ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if ((galois & 1u) == 0) return set_error(CKKS_EINVAL, "galois element must be odd");
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(digits, "digits"));
+    CKKS_TRY(check_ptr(key, "key"));
+    CKKS_TRY(check_ptr(acc, "acc"));
+    CKKS_TRY(set_device(ctx));
+    KeyList kl{};
+    kl.key[0] = key;
+    kl.galois[0] = galois & (2u * kN - 1u);
+    return key_inner_stage(ctx, digits, kl, batch, true, acc, batch, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_moddown(const ckks_ctx *ctx, const uint64_t *acc, uint64_t *out, int batch,
+                            void *ws, ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(acc, "acc"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    void *w;
+    CKKS_TRY(resolve_ws(const_cast<ckks_ctx *>(ctx), ws, moddown_ws_bytes(ctx, batch), &w));
+    DownExtra ex;
+    return moddown_stage(ctx, acc, out, batch, ex, w, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_keyswitch(const ckks_ctx *ctx, const uint64_t *d, const uint64_t *key,
+                              uint64_t *out, int batch, void *ws, ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(d, "d"));
+    CKKS_TRY(check_ptr(key, "key"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    void *w;
+    CKKS_TRY(resolve_ws(const_cast<ckks_ctx *>(ctx), ws, keyswitch_ws(ctx, batch), &w));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int LK = ctx->L + ctx->K;
+    Carve c(w);
+    u64 *digits = c.take<u64>((size_t)batch * ctx->dnum * LK * kN);
+    u64 *acc = c.take<u64>((size_t)batch * 2 * LK * kN);
+    void *scratch = c.base + c.off;
+    CKKS_TRY(modup_stage(ctx, d, nullptr, (size_t)ctx->L * kN, digits, batch, scratch, s));
+    KeyList kl{};
+    kl.key[0] = key;
+    kl.galois[0] = 1;
+    CKKS_TRY(key_inner_stage(ctx, digits, kl, batch, true, acc, batch, s));
+    DownExtra ex;
+    return moddown_stage(ctx, acc, out, batch, ex, scratch, s);
+}
+
+extern "C" int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
+                           const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
+                           ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (nkeys < 0) return set_error(CKKS_EINVAL, "negative key count");
+    if (batch == 0 || nkeys == 0) return CKKS_OK;
+    if (!keys || !galois) return set_error(CKKS_EINVAL, "null key or galois array");
+    for (int r = 0; r < nkeys; ++r) {
+        CKKS_TRY(check_ptr(keys[r], "keys[r]"));
+        if ((galois[r] & 1u) == 0) return set_error(CKKS_EINVAL, "galois element must be odd");
+    }
+    if ((size_t)nkeys * batch > 32767) return set_error(CKKS_EUNSUPPORTED, "nkeys * batch above 32767");
+    CKKS_TRY(check_ptr(ct, "ct"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    void *w;
+    CKKS_TRY(resolve_ws(const_cast<ckks_ctx *>(ctx), ws, rotate_ws(ctx, batch, nkeys), &w));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int L = ctx->L, LK = L + ctx->K;
+    const size_t ct_elems = (size_t)2 * L * kN;
+    const int chunk = std::min(nkeys, kMaxKeys);
+    Carve c(w);
+    u64 *digits = c.take<u64>((size_t)batch * ctx->dnum * LK * kN);
+    u64 *acc = c.take<u64>((size_t)chunk * batch * 2 * LK * kN);
+    void *scratch = c.base + c.off;
+    CKKS_TRY(modup_stage(ctx, ct + (size_t)L * kN, nullptr, ct_elems, digits, batch, scratch, s));
+    for (int r0 = 0; r0 < nkeys; r0 += chunk) {
+        const int nk = std::min(chunk, nkeys - r0);
+        KeyList kl{};
+        DownExtra ex;
+        ex.kind = 1;
+        ex.ct = ct;
+        ex.ct_bstride = ct_elems;
+        ex.ct_mod = batch;
+        ex.per = batch;
+        for (int r = 0; r < nk; ++r) {
+            kl.key[r] = keys[r0 + r];
+            kl.galois[r] = ex.gal[r] = galois[r0 + r] & (2u * kN - 1u);
+        }
+        CKKS_TRY(key_inner_stage(ctx, digits, kl, batch, true, acc, nk * batch, s));
+        CKKS_TRY(moddown_stage(ctx, acc, out + (size_t)r0 * batch * ct_elems, nk * batch, ex,
+                               scratch, s));
+    }
+    return CKKS_OK;
+}

@@ -1,0 +1,539 @@
+// NTT entry points, pointwise arithmetic, the Galois automorphism, rescale,
+// ct x ct multiply with relinearisation, the BSGS linear transform, workspace
+// sizing and the integer-pipe microbenchmarks.
+#include <algorithm>
+
+#include "internal.cuh"
+#include "ntt.cuh"
+
+namespace ckks {
+
+size_t keyswitch_ws_bytes(const ckks_ctx *ctx, int batch);
+size_t rotate_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys);
+
+static int check_batch(int batch)
+{
+    if (batch < 0) return set_error(CKKS_EINVAL, "negative batch");
+    if (batch > 65535) return set_error(CKKS_EUNSUPPORTED, "batch above 65535");
+    return CKKS_OK;
+}
+
+static int check_limbs(const ckks_ctx *ctx, int limb_begin, int limbs)
+{
+    if (limb_begin < 0 || limbs < 0 || limb_begin + limbs > ctx->L + ctx->K)
+        return set_error(CKKS_EINVAL, "limb range outside the context's primes");
+    return CKKS_OK;
+}
+
+// ---------------------------------------------------------------- pointwise
+__global__ void pointwise_kernel(int op, const u64 *__restrict__ a, const u64 *__restrict__ b,
+                                 u64 *__restrict__ out, int limbs, int limb_begin, size_t pairs,
+                                 const PrimeConst *__restrict__ pc)
+{
+    for (size_t p = blockIdx.x * (size_t)blockDim.x + threadIdx.x; p < pairs;
+         p += (size_t)gridDim.x * blockDim.x) {
+        const size_t e = 2 * p;
+        const int limb = (int)((e / kN) % limbs);
+        const PrimeConst c = pc[limb_begin + limb];
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(a + e);
+        const ulonglong2 y = *reinterpret_cast<const ulonglong2 *>(b + e);
+        ulonglong2 r;
+        if (op == CKKS_PW_MUL) {
+            r.x = mulmod(x.x, y.x, c);
+            r.y = mulmod(x.y, y.y, c);
+        } else if (op == CKKS_PW_ADD) {
+            r.x = addmod(x.x, y.x, c.q);
+            r.y = addmod(x.y, y.y, c.q);
+        } else {
+            r.x = submod(x.x, y.x, c.q);
+            r.y = submod(x.y, y.y, c.q);
+        }
+        *reinterpret_cast<ulonglong2 *>(out + e) = r;
+    }
+}
+
+static int grid_for(size_t work, int threads)
+{
+    size_t blocks = (work + threads - 1) / threads;
+    return (int)std::min<size_t>(std::max<size_t>(blocks, 1), 148 * 32);
+}
+
+// ---------------------------------------------------------------- automorphism
+// One CTA per limb row: stage the row in shared memory with coalesced loads,
+// gather through the Galois index map, store coalesced.
+__global__ void __launch_bounds__(256) automorph_kernel(const u64 *__restrict__ in,
+                                                        u64 *__restrict__ out, u32 g)
+{
+    __shared__ u64 row[kN];
+    const size_t base = (size_t)blockIdx.x * kN;
+    for (int k = threadIdx.x; k < kN / 2; k += 256) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(in + base + 2 * k);
+        row[2 * k] = v.x;
+        row[2 * k + 1] = v.y;
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < kN / 2; k += 256) {
+        ulonglong2 v;
+        v.x = row[galois_src(2 * k, g)];
+        v.y = row[galois_src(2 * k + 1, g)];
+        *reinterpret_cast<ulonglong2 *>(out + base + 2 * k) = v;
+    }
+}
+
+// ---------------------------------------------------------------- rescale
+// INTT of the dropped limb of every (ciphertext, component) into w[.][n].
+struct RescInttJob {
+    const u64 *ct;
+    u64 *w;
+    int lp1, count;
+    __device__ __forceinline__ int prime(int) const { return lp1 - 1; }
+    __device__ __forceinline__ void load4(int j, int e, u64 *v) const
+    {
+        ld4(ct + ((size_t)j * lp1 + lp1 - 1) * kN + e, v);
+    }
+    __device__ __forceinline__ void store(int j, int e, u64 v) const { w[(size_t)j * kN + e] = v; }
+};
+
+// Forward NTT of [w]_{q_i} for every kept limb i; the store forms
+// (c_i - NTT([w]_{q_i})) q_l^-1.
+struct RescFwdJob {
+    const u64 *w, *ct;
+    u64 *out;
+    const ulonglong2 *qinv;
+    const PrimeConst *pc;
+    int lp1, jobs2, count;
+    __device__ __forceinline__ int prime(int j) const { return j / jobs2; }
+    __device__ __forceinline__ u64 load(int j, int e) const
+    {
+        const int i = j / jobs2, zz = j - i * jobs2;
+        const u64 v = w[(size_t)zz * kN + e];
+        const PrimeConst &c = pc[i];
+        return v - mulhi(v, c.mu64) * c.q;  // [0, 2 q_i)
+    }
+    __device__ __forceinline__ void store4(int j, int e, const u64 *v) const
+    {
+        const int i = j / jobs2, zz = j - i * jobs2;
+        const u64 q = pc[i].q;
+        const ulonglong2 qi = qinv[i];
+        u64 c[4], o[4];
+        ld4(ct + ((size_t)zz * lp1 + i) * kN + e, c);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k] = shoup(submod(c[k], v[k], q), qi.x, qi.y, q);
+        st4(out + ((size_t)zz * (lp1 - 1) + i) * kN + e, o);
+    }
+};
+
+size_t rescale_ws_bytes(int batch) { return limbs_bytes((size_t)batch * 2); }
+
+int rescale_stage(ckks_ctx *ctx, const u64 *ct, u64 *out, int lp1, int batch, void *ws, cudaStream_t s)
+{
+    if (batch <= 0) return CKKS_OK;
+    int rc;
+    const ulonglong2 *qinv = rescale_table(ctx, lp1, &rc);
+    if (!qinv) return rc;
+    const Tables &T = ctx->t;
+    Carve c(ws);
+    u64 *w = c.take<u64>((size_t)batch * 2 * kN);
+    RescInttJob ij{ct, w, lp1, 2 * batch};
+    CKKS_TRY(launch_ntt_inv(ij, T, s));
+    RescFwdJob fj{w, ct, out, qinv, T.pc, lp1, 2 * batch, (lp1 - 1) * 2 * batch};
+    return launch_ntt_fwd(fj, T, s);
+}
+
+// ---------------------------------------------------------------- BSGS pieces
+// inner[g][b][c][i][e] = sum_r diags[g][r][i][e] * baby_r[b][c][i][e], where
+// baby_0 = x and baby_r (r >= 1) = baby[r-1].  One CTA per (32 coefficients,
+// limb i, ciphertext-component bc): the bb baby values sit in shared memory,
+// 8 warps split the giant index g.
+constexpr int kMaxBaby = 64;
+
+__global__ void __launch_bounds__(256) bsgs_inner_kernel(const u64 *__restrict__ diags,
+                                                         const u64 *__restrict__ x,
+                                                         const u64 *__restrict__ baby,
+                                                         u64 *__restrict__ inner, int bb, int gg,
+                                                         int B, int L, const PrimeConst *__restrict__ pc)
+{
+    __shared__ u64 sb[kMaxBaby][32];
+    const int lane = threadIdx.x & 31, gw = threadIdx.x >> 5;
+    const int i = blockIdx.y, bc = blockIdx.z;
+    const int e = blockIdx.x * 32 + lane;
+    const size_t Ln = (size_t)L * kN;
+    const size_t off = (size_t)bc * Ln + (size_t)i * kN + e;  // within one [B][2][L][n] block
+    for (int r = gw; r < bb; r += 8)
+        sb[r][lane] = r == 0 ? x[off] : baby[(size_t)(r - 1) * B * 2 * Ln + off];
+    __syncthreads();
+    const PrimeConst c = pc[i];
+    for (int g = gw; g < gg; g += 8) {
+        const u64 *d = diags + ((size_t)g * bb * L + i) * kN + e;
+        u64 hi = 0, lo = 0;
+        for (int r = 0; r < bb; ++r) mac128(hi, lo, __ldg(d + (size_t)r * Ln), sb[r][lane]);
+        inner[(size_t)g * B * 2 * Ln + off] = reduce128(hi, lo, c);
+    }
+}
+
+// total[b] = (first ? first[b] : total[b]) + sum_{t < nterms} terms[t B + b],
+// arrays of ciphertexts [.][2][L][n].
+__global__ void accum_kernel(u64 *__restrict__ total, const u64 *__restrict__ first,
+                             const u64 *__restrict__ terms, int nterms, int B, int L,
+                             const PrimeConst *__restrict__ pc)
+{
+    const size_t ct = (size_t)2 * L * kN, n_all = (size_t)B * ct;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n_all;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const int i = (int)((idx / kN) % L);
+        const u64 q = pc[i].q;
+        u64 v = first ? first[idx] : total[idx];
+        for (int t = 0; t < nterms; ++t) v = addmod(v, terms[(size_t)t * n_all + idx], q);
+        total[idx] = v;
+    }
+}
+
+static u32 galois_pow5(long long r)
+{
+    u32 g = 1;
+    const u32 m = 2 * kN;
+    r %= kN / 2;  // 5 has order n/2 modulo 2n
+    if (r < 0) r += kN / 2;
+    for (long long k = 0; k < r; ++k) g = (g * 5u) % m;
+    return g;
+}
+
+struct BsgsLayout {
+    int gchunk;
+    size_t digits, acc, baby, inner, rot, total, scratch;
+};
+
+static BsgsLayout bsgs_layout(const ckks_ctx *ctx, int B, int bb, int gg)
+{
+    BsgsLayout l{};
+    const size_t LK = ctx->L + ctx->K, L = ctx->L;
+    l.gchunk = std::max(1, std::min(std::min(gg - 1, kMaxKeys), std::max(1, 64 / std::max(B, 1))));
+    const int babyk = std::min(std::max(bb - 1, 1), kMaxKeys);
+    const size_t up_batch = std::max<size_t>(B, (size_t)l.gchunk * B);
+    const size_t acc_jobs = std::max<size_t>((size_t)babyk * B, (size_t)l.gchunk * B);
+    l.digits = limbs_bytes(up_batch * ctx->dnum * LK);
+    l.acc = limbs_bytes(acc_jobs * 2 * LK);
+    l.baby = limbs_bytes((size_t)std::max(bb - 1, 0) * B * 2 * L);
+    l.inner = limbs_bytes((size_t)gg * B * 2 * L);
+    l.rot = limbs_bytes((size_t)l.gchunk * B * 2 * L);
+    l.total = limbs_bytes((size_t)B * 2 * L);
+    l.scratch = std::max({modup_ws_bytes(ctx, (int)up_batch), moddown_ws_bytes(ctx, (int)acc_jobs),
+                          rescale_ws_bytes(B)});
+    return l;
+}
+
+static size_t bsgs_ws(const ckks_ctx *ctx, int B, int bb, int gg)
+{
+    BsgsLayout l = bsgs_layout(ctx, B, bb, gg);
+    return l.digits + l.acc + l.baby + l.inner + l.rot + l.total + l.scratch;
+}
+
+static size_t mrr_ws(const ckks_ctx *ctx, int B)
+{
+    const size_t LK = ctx->L + ctx->K;
+    return limbs_bytes((size_t)B * ctx->dnum * LK) + limbs_bytes((size_t)B * 2 * LK) +
+           limbs_bytes((size_t)B * 2 * ctx->L) +
+           std::max({modup_ws_bytes(ctx, B), moddown_ws_bytes(ctx, B), rescale_ws_bytes(B)});
+}
+
+}  // namespace ckks
+
+using namespace ckks;
+
+// ---------------------------------------------------------------- entry points
+extern "C" size_t ckks_workspace_bytes(const ckks_ctx *ctx, int op, int batch, int aux)
+{
+    if (!ctx || batch < 0) return 0;
+    switch (op) {
+    case CKKS_OP_MODUP: return modup_ws_bytes(ctx, batch);
+    case CKKS_OP_MODDOWN: return moddown_ws_bytes(ctx, batch);
+    case CKKS_OP_KEYSWITCH: return keyswitch_ws_bytes(ctx, batch);
+    case CKKS_OP_ROTATE: return rotate_ws_bytes(ctx, batch, aux);
+    case CKKS_OP_RESCALE: return rescale_ws_bytes(batch);
+    case CKKS_OP_MUL_RELIN_RESCALE: return mrr_ws(ctx, batch);
+    case CKKS_OP_BSGS: {
+        const int bb = aux / 1000, gg = aux % 1000;
+        if (bb < 1 || gg < 1) return 0;
+        return bsgs_ws(ctx, batch, bb, gg);
+    }
+    default: return 0;
+    }
+}
+
+static int ntt_common(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin, int limbs)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_limbs(ctx, limb_begin, limbs));
+    if (batch < 0) return set_error(CKKS_EINVAL, "negative batch");
+    if ((long long)batch * limbs > (1LL << 30)) return set_error(CKKS_EUNSUPPORTED, "too many limbs");
+    if (batch == 0 || limbs == 0) return 1;
+    CKKS_TRY(check_ptr(x, "x"));
+    CKKS_TRY(set_device(ctx));
+    return CKKS_OK;
+}
+
+extern "C" int ckks_ntt_fwd(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin, int limbs,
+                            ckks_stream_t stream)
+{
+    int rc = ntt_common(ctx, x, batch, limb_begin, limbs);
+    if (rc != CKKS_OK) return rc > 0 ? CKKS_OK : rc;
+    BatchJob j{x, limbs, batch, limb_begin, limbs * batch};
+    return launch_ntt_fwd(j, ctx->t, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_ntt_inv(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin, int limbs,
+                            ckks_stream_t stream)
+{
+    int rc = ntt_common(ctx, x, batch, limb_begin, limbs);
+    if (rc != CKKS_OK) return rc > 0 ? CKKS_OK : rc;
+    BatchJob j{x, limbs, batch, limb_begin, limbs * batch};
+    return launch_ntt_inv(j, ctx->t, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_pointwise(const ckks_ctx *ctx, int op, const uint64_t *a, const uint64_t *b,
+                              uint64_t *out, int batch, int limb_begin, int limbs,
+                              ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    if (op != CKKS_PW_MUL && op != CKKS_PW_ADD && op != CKKS_PW_SUB)
+        return set_error(CKKS_EINVAL, "unknown pointwise op");
+    CKKS_TRY(check_limbs(ctx, limb_begin, limbs));
+    CKKS_TRY(check_batch(batch));
+    if (batch == 0 || limbs == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(a, "a"));
+    CKKS_TRY(check_ptr(b, "b"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    const size_t pairs = (size_t)batch * limbs * kN / 2;
+    pointwise_kernel<<<grid_for(pairs, 256), 256, 0, (cudaStream_t)stream>>>(
+        op, a, b, out, limbs, limb_begin, pairs, ctx->t.pc);
+    CKKS_CHECK_LAUNCH("pointwise_kernel");
+    return CKKS_OK;
+}
+
+extern "C" int ckks_automorph(const ckks_ctx *ctx, const uint64_t *in, uint64_t *out, int batch,
+                              int limbs, uint32_t galois, ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (limbs < 0) return set_error(CKKS_EINVAL, "negative limb count");
+    if ((galois & 1u) == 0) return set_error(CKKS_EINVAL, "galois element must be odd");
+    const long long rows = (long long)batch * limbs;
+    if (rows == 0) return CKKS_OK;
+    if (rows > 0x7fffffffLL) return set_error(CKKS_EUNSUPPORTED, "too many rows");
+    CKKS_TRY(check_ptr(in, "in"));
+    CKKS_TRY(check_ptr(out, "out"));
+    if (in == out) return set_error(CKKS_EINVAL, "automorphism cannot run in place");
+    CKKS_TRY(set_device(ctx));
+    automorph_kernel<<<(unsigned)rows, 256, 0, (cudaStream_t)stream>>>(in, out, galois & (2u * kN - 1u));
+    CKKS_CHECK_LAUNCH("automorph_kernel");
+    return CKKS_OK;
+}
+
+extern "C" int ckks_rescale(const ckks_ctx *ctx, const uint64_t *ct, uint64_t *out, int lp1, int batch,
+                            void *ws, ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (lp1 < 2 || lp1 > ctx->L) return set_error(CKKS_EINVAL, "lp1 must be in [2, L]");
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(ct, "ct"));
+    CKKS_TRY(check_ptr(out, "out"));
+    if (ct == out) return set_error(CKKS_EINVAL, "rescale cannot run in place");
+    CKKS_TRY(set_device(ctx));
+    ckks_ctx *m = const_cast<ckks_ctx *>(ctx);
+    void *w;
+    CKKS_TRY(resolve_ws(m, ws, rescale_ws_bytes(batch), &w));
+    return rescale_stage(m, ct, out, lp1, batch, w, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_mul_relin_rescale(const ckks_ctx *ctx, const uint64_t *a, const uint64_t *b,
+                                      const uint64_t *rlk, uint64_t *out, int batch, void *ws,
+                                      ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (ctx->L < 2) return set_error(CKKS_EUNSUPPORTED, "rescale needs L >= 2");
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(a, "a"));
+    CKKS_TRY(check_ptr(b, "b"));
+    CKKS_TRY(check_ptr(rlk, "rlk"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    ckks_ctx *m = const_cast<ckks_ctx *>(ctx);
+    void *w;
+    CKKS_TRY(resolve_ws(m, ws, mrr_ws(ctx, batch), &w));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int L = ctx->L, LK = L + ctx->K;
+    const size_t Ln = (size_t)L * kN;
+    Carve c(w);
+    u64 *digits = c.take<u64>((size_t)batch * ctx->dnum * LK * kN);
+    u64 *acc = c.take<u64>((size_t)batch * 2 * LK * kN);
+    u64 *cr = c.take<u64>((size_t)batch * 2 * Ln);
+    void *scratch = c.base + c.off;
+    // d2 = a1 b1 is formed inside ModUp's first transform
+    CKKS_TRY(modup_stage(ctx, a + Ln, b + Ln, 2 * Ln, digits, batch, scratch, s));
+    KeyList kl{};
+    kl.key[0] = rlk;
+    kl.galois[0] = 1;
+    CKKS_TRY(key_inner_stage(ctx, digits, kl, batch, true, acc, batch, s));
+    DownExtra ex;
+    ex.kind = 2;  // + (a0 b0, a0 b1 + a1 b0)
+    ex.a = a;
+    ex.b = b;
+    CKKS_TRY(moddown_stage(ctx, acc, cr, batch, ex, scratch, s));
+    return rescale_stage(m, cr, out, L, batch, scratch, s);
+}
+
+extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                                  const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
+                                  int bb, int gg, uint64_t *y, int batch, void *ws,
+                                  ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (ctx->L < 2) return set_error(CKKS_EUNSUPPORTED, "rescale needs L >= 2");
+    if (bb < 1 || gg < 1 || bb > kMaxBaby || gg > 999)
+        return set_error(CKKS_EINVAL, "need 1 <= bb <= 64 and 1 <= gg <= 999");
+    if ((size_t)batch * std::max(bb - 1, 1) > 32767)
+        return set_error(CKKS_EUNSUPPORTED, "batch * (bb - 1) above 32767");
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(x, "x"));
+    CKKS_TRY(check_ptr(diags, "diags"));
+    CKKS_TRY(check_ptr(y, "y"));
+    if (bb > 1 && !baby_keys) return set_error(CKKS_EINVAL, "null baby key array");
+    if (gg > 1 && !giant_keys) return set_error(CKKS_EINVAL, "null giant key array");
+    for (int r = 0; r + 1 < bb; ++r) CKKS_TRY(check_ptr(baby_keys[r], "baby_keys[r]"));
+    for (int g = 0; g + 1 < gg; ++g) CKKS_TRY(check_ptr(giant_keys[g], "giant_keys[g]"));
+    CKKS_TRY(set_device(ctx));
+    ckks_ctx *m = const_cast<ckks_ctx *>(ctx);
+    void *w;
+    CKKS_TRY(resolve_ws(m, ws, bsgs_ws(ctx, batch, bb, gg), &w));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const Tables &T = ctx->t;
+    const int L = ctx->L, B = batch;
+    const size_t Ln = (size_t)L * kN, ctn = 2 * Ln;
+    const BsgsLayout lay = bsgs_layout(ctx, B, bb, gg);
+    char *base = static_cast<char *>(w);
+    u64 *digits = reinterpret_cast<u64 *>(base);
+    u64 *acc = reinterpret_cast<u64 *>(base + lay.digits);
+    u64 *baby = reinterpret_cast<u64 *>(base + lay.digits + lay.acc);
+    u64 *inner = reinterpret_cast<u64 *>(base + lay.digits + lay.acc + lay.baby);
+    u64 *rot = reinterpret_cast<u64 *>(base + lay.digits + lay.acc + lay.baby + lay.inner);
+    u64 *total = reinterpret_cast<u64 *>(base + lay.digits + lay.acc + lay.baby + lay.inner + lay.rot);
+    void *scratch = base + lay.digits + lay.acc + lay.baby + lay.inner + lay.rot + lay.total;
+
+    // baby steps: Rot_r(x), r = 1..bb-1, on one hoisted ModUp
+    if (bb > 1) {
+        CKKS_TRY(modup_stage(ctx, x + Ln, nullptr, ctn, digits, B, scratch, s));
+        for (int r0 = 1; r0 < bb; r0 += kMaxKeys) {
+            const int nk = std::min(kMaxKeys, bb - r0);
+            KeyList kl{};
+            DownExtra ex;
+            ex.kind = 1;
+            ex.ct = x;
+            ex.ct_bstride = ctn;
+            ex.ct_mod = B;
+            ex.per = B;
+            for (int r = 0; r < nk; ++r) {
+                kl.key[r] = baby_keys[r0 + r - 1];
+                kl.galois[r] = ex.gal[r] = galois_pow5(r0 + r);
+            }
+            CKKS_TRY(key_inner_stage(ctx, digits, kl, B, true, acc, nk * B, s));
+            CKKS_TRY(moddown_stage(ctx, acc, baby + (size_t)(r0 - 1) * B * ctn, nk * B, ex, scratch, s));
+        }
+    }
+    // inner sums for every giant index
+    {
+        dim3 grid(kN / 32, L, 2 * B);
+        bsgs_inner_kernel<<<grid, 256, 0, s>>>(diags, x, baby, inner, bb, gg, B, L, T.pc);
+        CKKS_CHECK_LAUNCH("bsgs_inner_kernel");
+    }
+    // giant steps: total = inner_0 + sum_{g >= 1} Rot_{bb g}(inner_g)
+    const size_t all = (size_t)B * ctn;
+    accum_kernel<<<grid_for(all, 256), 256, 0, s>>>(total, inner, nullptr, 0, B, L, T.pc);
+    CKKS_CHECK_LAUNCH("accum_kernel");
+    for (int g0 = 1; g0 < gg; g0 += lay.gchunk) {
+        const int ng = std::min(lay.gchunk, gg - g0);
+        const u64 *src = inner + (size_t)g0 * B * ctn;
+        CKKS_TRY(modup_stage(ctx, src + Ln, nullptr, ctn, digits, ng * B, scratch, s));
+        KeyList kl{};
+        DownExtra ex;
+        ex.kind = 1;
+        ex.ct = src;
+        ex.ct_bstride = ctn;
+        ex.ct_mod = 0;
+        ex.per = B;
+        for (int g = 0; g < ng; ++g) {
+            kl.key[g] = giant_keys[g0 + g - 1];
+            kl.galois[g] = ex.gal[g] = galois_pow5((long long)bb * (g0 + g));
+        }
+        CKKS_TRY(key_inner_stage(ctx, digits, kl, B, false, acc, ng * B, s));
+        CKKS_TRY(moddown_stage(ctx, acc, rot, ng * B, ex, scratch, s));
+        accum_kernel<<<grid_for(all, 256), 256, 0, s>>>(total, nullptr, rot, ng, B, L, T.pc);
+        CKKS_CHECK_LAUNCH("accum_kernel");
+    }
+    return rescale_stage(m, total, y, L, B, scratch, s);
+}
+
+// ---------------------------------------------------------------- microbenchmarks
+__global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, u64 *sink)
+{
+    u64 x[8], h[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        x[k] = (threadIdx.x * 8 + k + 1) * 0x9E3779B97F4A7C15ull % q;
+        h[k] = 0;
+    }
+    if (kind == 0) {
+        for (int it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) x[k] = shoup(x[k], w, wp, q);
+        }
+    } else if (kind == 1) {
+        for (int it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mac128(h[k], x[k], x[(k + 1) & 7], w);
+        }
+    } else {
+        for (int it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) x[k] = mulhi(x[k], wp) + w;
+        }
+    }
+    u64 acc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc ^= x[k] ^ h[k];
+    if (acc == 0x1234567ull) sink[threadIdx.x] = acc;  // keeps the loops alive
+}
+
+extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int iters, double *ms,
+                                  double *ops)
+{
+    CKKS_TRY(check_ctx(ctx));
+    if (kind < 0 || kind > 2 || blocks < 1 || iters < 1 || !ms || !ops)
+        return set_error(CKKS_EINVAL, "bad microbenchmark arguments");
+    CKKS_TRY(set_device(ctx));
+    const u64 q = ctx->mods[0];
+    const u64 w = 0x0123456789abcdefull % q, wp = host_shoup(w, q);
+    u64 *sink = nullptr;
+    cudaError_t e = cudaMalloc(&sink, 256 * sizeof(u64));
+    if (e != cudaSuccess) return cuda_status(e, "cudaMalloc(sink)");
+    cudaEvent_t a, b;
+    cudaEventCreate(&a);
+    cudaEventCreate(&b);
+    intpipe_kernel<<<blocks, 256>>>(kind, std::max(1, iters / 16), q, w, wp, sink);  // warm-up
+    cudaEventRecord(a);
+    intpipe_kernel<<<blocks, 256>>>(kind, iters, q, w, wp, sink);
+    cudaEventRecord(b);
+    e = cudaEventSynchronize(b);
+    float t = 0;
+    cudaEventElapsedTime(&t, a, b);
+    cudaEventDestroy(a);
+    cudaEventDestroy(b);
+    cudaFree(sink);
+    if (e != cudaSuccess) return cuda_status(e, "intpipe_kernel");
+    *ms = t;
+    *ops = (double)blocks * 256.0 * iters * 8.0;
+    return CKKS_OK;
+}

@@ -1,0 +1,327 @@
+"""Bit-exact parity of every C-ABI call against the CPU oracle, on the GPU.
+
+All integer RNS tensors must match word for word.  Keys and ciphertexts for
+the small and layer-shaped cases come from the oracle's keygen/encryption so
+that decryption can be checked too; at the full boot-level sizes keys and
+ciphertexts are seeded uniform residues (the integer function is the same,
+and the decryption pins run at the smaller sizes).
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from rns_ckks_polynomial_b200 import native, synth
+from rns_ckks_polynomial_b200.native import CkksError
+
+from .gpu_common import assert_bits_equal, context, ctx_for, dev, gpu, host, need_gpu
+from .helpers import N, SCALE, SLOTS, Params, Scheme, galois_for_rotation, rot_left, u64
+
+pytestmark = gpu
+
+SEED = synth.config_seed(1)
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    need_gpu()
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _res(shape, mods, stream, seed=SEED):
+    return u64(synth.uniform_residues(shape, mods, seed, stream))
+
+
+# ------------------------------------------------------------------ config 1
+def test_config1_tiny_pipeline(orc):
+    """4 + 1 primes, alpha = 1: 8 polynomials -> NTT -> pairwise product ->
+    INTT, and one rotation key switch with the Galois-5 key."""
+    p = Params(4, 1, 1)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED)
+    q = sch.q
+    polys = _res((8, 4, N), q, 1)
+    x = dev(polys)
+    ctx.ntt_fwd(x)
+    want = orc.ntt_fwd(polys, q)
+    assert_bits_equal(host(x), want, "ntt_fwd")
+    prod = ctx.pointwise("mul", x[0::2].contiguous(), x[1::2].contiguous())
+    want_p = orc.pointwise("mul", want[0::2], want[1::2], q)
+    assert_bits_equal(host(prod), want_p, "pointwise mul")
+    ctx.ntt_inv(prod)
+    assert_bits_equal(host(prod), orc.ntt_inv(want_p, q), "ntt_inv")
+    # rotation key switch on (P0, P1) in the NTT domain
+    key = sch.keygen_galois(5)
+    ct = want[0:2][None]
+    out = ctx.rotate(dev(ct), [dev(key)], [5])
+    want_r = orc.rotate(ct, [key], np.array([5], dtype=np.uint64), sch.mods, 4, 1, 1)
+    assert_bits_equal(host(out), want_r, "rotate")
+
+
+def test_config1_rotation_decrypts(orc):
+    p = Params(4, 1, 1)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 1)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 3).numpy()
+    ct = sch.encrypt_slots(z)
+    key = sch.keygen_galois(5)
+    out = host(ctx.rotate(dev(ct[None]), [dev(key)], [5]))
+    assert np.max(np.abs(sch.decrypt_slots(out[0, 0]) - rot_left(z, 1))) < 1e-8
+
+
+# ------------------------------------------------------------------ NTT (config 2)
+@pytest.mark.parametrize("limbs,batch,begin", [(3, 16, 0), (112, 16, 0), (5, 3, 7), (1, 1, 2159),
+                                               (512, 16, 0)])
+def test_ntt_roundtrip_and_parity(orc, limbs, batch, begin):
+    ctx = context(2100, 60, 60)
+    mods = np.array(ctx.mods[begin:begin + limbs], dtype=np.uint64)
+    a = _res((batch, limbs, N), mods, 10 + limbs)
+    x = dev(a)
+    ctx.ntt_fwd(x, limb_begin=begin)
+    assert_bits_equal(host(x), orc.ntt_fwd(a, mods), "ntt_fwd")
+    ctx.ntt_inv(x, limb_begin=begin)
+    assert_bits_equal(host(x), a, "ntt round trip")
+    y = dev(a)
+    ctx.ntt_inv(y, limb_begin=begin)
+    assert_bits_equal(host(y), orc.ntt_inv(a, mods), "ntt_inv")
+
+
+def test_ntt_full_sweep_2100(orc):
+    """The bench's largest sweep entry: 16 x 2100 limbs, every limb checked."""
+    ctx = context(2100, 60, 60)
+    mods = np.array(ctx.q, dtype=np.uint64)
+    a = synth.uniform_residues((16, 2100, N), mods, SEED, 20, device="cuda")
+    x = a.clone()
+    ctx.ntt_fwd(x)
+    want = orc.ntt_fwd(host(a), mods)
+    assert_bits_equal(host(x), want, "ntt_fwd 2100")
+    ctx.ntt_inv(x)
+    assert torch.equal(x, a)
+
+
+def test_ntt_empty_and_errors():
+    ctx = context(4, 1, 1)
+    e = torch.empty((0, 4, N), dtype=torch.int64, device="cuda")
+    ctx.ntt_fwd(e)
+    x = torch.zeros((1, 4, N), dtype=torch.int64, device="cuda")
+    with pytest.raises(CkksError) as err:
+        ctx.ntt_fwd(x, limb_begin=2)  # 2 + 4 > L + K = 5
+    assert err.value.code == -1
+    buf = torch.zeros(4 * N + 1, dtype=torch.int64, device="cuda")
+    lib = native.lib()
+    rc = lib.ckks_ntt_fwd(ctx._h, C.c_void_p(buf.data_ptr() + 8), 1, 0, 4, None)
+    assert rc == -1 and "aligned" in lib.ckks_last_error().decode()
+
+
+# ------------------------------------------------------------------ pointwise / automorphism
+@pytest.mark.parametrize("op", ["mul", "add", "sub"])
+def test_pointwise(orc, op):
+    ctx = context(112, 8, 8)
+    mods = np.array(ctx.mods[:112], dtype=np.uint64)
+    a, b = _res((3, 112, N), mods, 30), _res((3, 112, N), mods, 31)
+    out = ctx.pointwise(op, dev(a), dev(b))
+    assert_bits_equal(host(out), orc.pointwise(op, a, b, mods), op)
+
+
+@pytest.mark.parametrize("g", [5, 25, 625, 1505, 4095, 3])
+def test_automorph(orc, g):
+    ctx = context(112, 8, 8)
+    mods = np.array(ctx.mods[:7], dtype=np.uint64)
+    a = _res((2, 7, N), mods, 40)
+    out = ctx.automorph(dev(a), g)
+    assert_bits_equal(host(out), orc.automorph_ntt(a, g), "automorph %d" % g)
+
+
+def test_automorph_rejects_even_and_in_place():
+    ctx = context(4, 1, 1)
+    x = torch.zeros((1, 4, N), dtype=torch.int64, device="cuda")
+    with pytest.raises(CkksError):
+        ctx.automorph(x, 4)
+    with pytest.raises(CkksError):
+        ctx.automorph(x, 5, out=x)
+
+
+# ------------------------------------------------------------------ key switching stages
+@pytest.mark.parametrize("L,K,alpha", [(4, 1, 1), (6, 2, 2), (5, 2, 2), (112, 8, 8), (20, 3, 7)])
+def test_modup_inner_moddown_stages(orc, L, K, alpha):
+    p = Params(L, K, alpha)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    c = _res((2, L, N), mods[:L], 50)
+    dig = ctx.modup(dev(c))
+    want_d = orc.modup(c, mods, L, K, alpha)
+    assert_bits_equal(host(dig), want_d, "modup")
+    key = _res((p.dnum, 2, L + K, N), mods, 51)
+    for g in (1, 5, 4095):
+        acc = ctx.key_inner(dig, dev(key), g)
+        want_a = orc.key_inner(want_d, key, g, mods, L, K, alpha)
+        assert_bits_equal(host(acc), want_a, "key_inner g=%d" % g)
+    out = ctx.moddown(acc)
+    assert_bits_equal(host(out), orc.moddown(want_a, mods, L, K), "moddown")
+    ks = ctx.keyswitch(dev(c), dev(key))
+    assert_bits_equal(host(ks), orc.keyswitch(c, key, mods, L, K, alpha), "keyswitch")
+
+
+def test_hoisted_rotations_match_and_decrypt(orc):
+    p = Params(5, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 2)
+    zs = [synth.uniform_real((SLOTS,), -1, 1, SEED, 60 + i).numpy() for i in range(3)]
+    cts = np.stack([sch.encrypt_slots(z) for z in zs])
+    rs = [1, 2, 5, 33]
+    keys = [sch.keygen_galois(galois_for_rotation(r)) for r in rs]
+    gal = [galois_for_rotation(r) for r in rs]
+    out = host(ctx.rotate(dev(cts), [dev(k) for k in keys], gal))
+    want = orc.rotate(cts, keys, np.array(gal, dtype=np.uint64), sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(out, want, "rotate")
+    for i, r in enumerate(rs):
+        for b in range(3):
+            assert np.max(np.abs(sch.decrypt_slots(out[i, b]) - rot_left(zs[b], r))) < 1e-8
+
+
+def test_rotate_context_owned_workspace(orc):
+    """ws = NULL makes the context allocate its own workspace."""
+    p = Params(4, 1, 1)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    ct = _res((2, 2, 4, N), mods[:4], 70)
+    key = _res((4, 2, 5, N), mods, 71)
+    ref = host(ctx.rotate(dev(ct), [dev(key)], [25]))
+    out = torch.empty((1, 2, 2, 4, N), dtype=torch.int64, device="cuda")
+    keep = dev(key)
+    kp = (C.c_void_p * 1)(keep.data_ptr())
+    gp = (C.c_uint32 * 1)(25)
+    ctd = dev(ct)
+    lib = native.lib()
+    rc = lib.ckks_rotate(ctx._h, C.c_void_p(ctd.data_ptr()), kp, gp, 1, C.c_void_p(out.data_ptr()),
+                         2, None, None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert_bits_equal(host(out), ref, "rotate (own workspace)")
+
+
+# ------------------------------------------------------------------ rescale, ct x ct
+@pytest.mark.parametrize("lp1,batch", [(5, 3), (112, 2), (2, 1)])
+def test_rescale(orc, lp1, batch):
+    ctx = context(112, 8, 8)
+    mods = np.array(ctx.mods[:lp1], dtype=np.uint64)
+    ct = _res((batch, 2, lp1, N), mods, 80 + lp1)
+    out = ctx.rescale(dev(ct))
+    assert_bits_equal(host(out), orc.rescale(ct, mods), "rescale")
+
+
+def test_mul_relin_rescale_small_decrypts(orc):
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 3)
+    za = [synth.uniform_real((SLOTS,), -1, 1, SEED, 90 + i).numpy() for i in range(2)]
+    zb = [synth.uniform_real((SLOTS,), -1, 1, SEED, 95 + i).numpy() for i in range(2)]
+    ca = np.stack([sch.encrypt_slots(z) for z in za])
+    cb = np.stack([sch.encrypt_slots(z) for z in zb])
+    rlk = sch.keygen_relin()
+    out = host(ctx.mul_relin_rescale(dev(ca), dev(cb), dev(rlk)))
+    assert_bits_equal(out, orc.mul_relin_rescale(ca, cb, rlk, sch.mods, p.L, p.K, p.alpha), "mrr")
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    for i in range(2):
+        assert np.max(np.abs(sch.decrypt_slots(out[i], sc) - za[i] * zb[i])) < 1e-8
+
+
+def test_config3_layer_multiply(orc):
+    """112 primes, alpha = 8, 8 special primes; 8 ciphertext pairs."""
+    p = Params(112, 8, 8)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, synth.config_seed(3))
+    za = [synth.uniform_real((SLOTS,), -1, 1, synth.config_seed(3), 100 + i).numpy() for i in range(8)]
+    zb = [synth.uniform_real((SLOTS,), -1, 1, synth.config_seed(3), 200 + i).numpy() for i in range(8)]
+    ca = np.stack([sch.encrypt_slots(z) for z in za])
+    cb = np.stack([sch.encrypt_slots(z) for z in zb])
+    rlk = sch.keygen_relin()
+    out = host(ctx.mul_relin_rescale(dev(ca), dev(cb), dev(rlk)))
+    want = orc.mul_relin_rescale(ca, cb, rlk, sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(out, want, "config 3")
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    for i in (0, 7):
+        assert np.max(np.abs(sch.decrypt_slots(out[i], sc) - za[i] * zb[i])) < 1e-8
+
+
+# ------------------------------------------------------------------ BSGS
+def test_bsgs_banded_decrypts(orc):
+    from .test_oracle_pins import bsgs_plaintexts
+    p = Params(6, 2, 2)
+    bb = gg = 4
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 5)
+    rng_m = synth.uniform_real((SLOTS, SLOTS), -1 / 32, 1 / 32, SEED, 110).numpy()
+    idx = np.arange(SLOTS)
+    M = np.zeros((SLOTS, SLOTS))
+    for k in range(bb * gg):
+        M[idx, (idx + k) % SLOTS] = rng_m[idx, (idx + k) % SLOTS]
+    xs = [synth.uniform_real((SLOTS,), -1, 1, SEED, 111 + i).numpy() for i in range(2)]
+    ct = np.stack([sch.encrypt_slots(x) for x in xs])
+    diags = bsgs_plaintexts(orc, M, bb, gg, sch.q)
+    baby = [sch.keygen_galois(galois_for_rotation(b)) for b in range(1, bb)]
+    giant = [sch.keygen_galois(galois_for_rotation(bb * g)) for g in range(1, gg)]
+    y = host(ctx.bsgs_lintrans(dev(ct), dev(diags), [dev(k) for k in baby],
+                               [dev(k) for k in giant], bb, gg))
+    want = orc.bsgs(ct, diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(y, want, "bsgs")
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    for i in range(2):
+        assert np.max(np.abs(sch.decrypt_slots(y[i], sc) - M @ xs[i])) < 1e-8
+
+
+@pytest.mark.parametrize("bb,gg", [(3, 5), (1, 2), (2, 1)])
+def test_bsgs_shapes(orc, bb, gg):
+    p = Params(5, 2, 2)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    x = _res((2, 2, 5, N), mods[:5], 120)
+    diags = _res((gg, bb, 5, N), mods[:5], 121)
+    baby = [_res((3, 2, 7, N), mods, 122 + i) for i in range(bb - 1)]
+    giant = [_res((3, 2, 7, N), mods, 140 + i) for i in range(gg - 1)]
+    y = host(ctx.bsgs_lintrans(dev(x), dev(diags), [dev(k) for k in baby], [dev(k) for k in giant],
+                               bb, gg))
+    assert_bits_equal(y, orc.bsgs(x, diags, baby, giant, bb, gg, mods, 5, 2, 2), "bsgs %dx%d" % (bb, gg))
+
+
+def test_config4_bsgs_full_size_sampled(orc):
+    """112 primes, alpha = 8, bb = gg = 32, 62 keys, 8 ciphertexts: the GPU
+    runs the full batch; the oracle recomputes ciphertext 5."""
+    p = Params(112, 8, 8)
+    ctx = ctx_for(p)
+    seed = synth.config_seed(4)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    kshape = (p.dnum, 2, 120, N)
+    x = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 1, device="cuda")
+    diags = synth.uniform_residues((32, 32, 112, N), mods[:112], seed, 2, device="cuda")
+    baby = [synth.uniform_residues(kshape, mods, seed, 100 + i, device="cuda") for i in range(31)]
+    giant = [synth.uniform_residues(kshape, mods, seed, 200 + i, device="cuda") for i in range(31)]
+    y = ctx.bsgs_lintrans(x, diags, baby, giant, 32, 32)
+    want = orc.bsgs(host(x[5:6]), host(diags), [host(k) for k in baby], [host(k) for k in giant],
+                    32, 32, mods, 112, 8, 8)
+    assert_bits_equal(host(y[5:6]), want, "config 4 ct 5")
+
+
+# ------------------------------------------------------------------ config 5
+def test_config5_boot_rotation_full_size_sampled(orc):
+    """2100 primes, alpha = 60, 60 special primes, 4 Galois keys (5^k,
+    k in {1, 2, 4, 8}), 8 ciphertexts: the GPU runs all 32 key switches with
+    one hoisted ModUp per ciphertext; the oracle recomputes ciphertext 3
+    under key 2 (g = 625)."""
+    p = Params(2100, 60, 60)
+    ctx = ctx_for(p)
+    seed = synth.config_seed(5)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    gal = [galois_for_rotation(k) for k in (1, 2, 4, 8)]
+    assert gal == [5, 25, 625, 1505]
+    ct = synth.uniform_residues((8, 2, 2100, N), mods[:2100], seed, 1, device="cuda")
+    keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device="cuda")
+            for r in range(4)]
+    out = ctx.rotate(ct, keys, gal)
+    got = host(out[2, 3])
+    want = orc.rotate(host(ct[3:4]), [host(keys[2])], np.array([gal[2]], dtype=np.uint64), mods,
+                      2100, 60, 60)
+    assert_bits_equal(got, want[0, 0], "config 5 ct 3 key 2")
