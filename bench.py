@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-ks", action="store_true", help="skip the key-switch measurements")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--sweep", default=",".join(str(x) for x in SWEEP),
+                    help="limb counts of the step (a smaller case for profiling only)")
     return ap.parse_args()
 
 
@@ -197,8 +199,9 @@ def run_b200(args):
     dev = torch.device("cuda", local)
     hbm_peak, peak_src = peaks()
     seed = synth.config_seed(2) + 1000 * rank
-    mods = primes(max(SWEEP) + 60)
-    ctx = Context(mods[:max(SWEEP)], mods[max(SWEEP):max(SWEEP) + 60], 60, device=local)
+    top = max(max(SWEEP), 60)
+    mods = primes(top + 60)
+    ctx = Context(mods[:top], mods[top:top + 60], 60, device=local)
 
     xs = [synth.uniform_residues((BATCH, l, N), mods[:l], seed, l, device=dev) for l in SWEEP]
     refs = [x.clone() for x in xs]
@@ -244,8 +247,8 @@ def run_b200(args):
     per_step = 2 * BATCH * sum(SWEEP)
     value = per_step * args.steps * world / (total_ms * 1e-3)
 
-    # roofline of the dominant kernel: forward NTT at 2100 limbs
-    bytes_, mm = ntt_launch_work(2100)
+    # roofline of the dominant kernel: forward NTT on the largest sweep entry
+    bytes_, mm = ntt_launch_work(SWEEP[-1])
     t = k_ms * 1e-3
     t_hbm = bytes_ / (hbm_peak * 1e9)
     t_alu = mm / ipeak["shoup_mulmod_per_s"]
@@ -256,8 +259,8 @@ def run_b200(args):
         roof = {"bound": "hbm", "achieved": bytes_ / t / 1e9, "peak": hbm_peak, "unit": "GB/s",
                 "peak_source": "%s MEASURED_PEAKS.json hbm_gbs" % peak_src}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for("ntt_fwd_2100")
-    roof["kernel"] = "ntt_fwd_kernel<BatchJob> (16 x 2100 limbs)"
+    roof["traffic"] = traffic_for("ntt_fwd_%d" % SWEEP[-1])
+    roof["kernel"] = "ntt_fwd_kernel<BatchJob> (16 x %d limbs)" % SWEEP[-1]
     roof["launch_ms"] = k_ms
     roof["hbm_frac_of_measured"] = (bytes_ / t / 1e9) / hbm_peak
     roof["alu_frac_of_microbench"] = (mm / t) / ipeak["shoup_mulmod_per_s"]
@@ -514,6 +517,8 @@ def run_reference(args):
 
 def main():
     args = parse()
+    global SWEEP
+    SWEEP = tuple(int(x) for x in args.sweep.split(","))
     if args.impl == "reference":
         run_reference(args)
     else:

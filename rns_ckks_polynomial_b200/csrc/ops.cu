@@ -491,9 +491,12 @@ __global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, u64 *s
             for (int k = 0; k < 8; ++k) x[k] = shoup(x[k], w, wp, q);
         }
     } else if (kind == 1) {
+        u64 y[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[k] = x[k] ^ 0x5555555555ull;
         for (int it = 0; it < iters; ++it) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mac128(h[k], x[k], x[(k + 1) & 7], w);
+            for (int k = 0; k < 8; ++k) mac128(h[k], x[k], y[k], w);  // 8 independent chains
         }
     } else {
         for (int it = 0; it < iters; ++it) {
