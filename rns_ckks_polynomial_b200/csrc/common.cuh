@@ -29,12 +29,13 @@ struct __align__(16) PrimeConst {
     u64 mu64;         // floor(2^64 / q)
     u64 ninv, ninvp;  // n^-1 mod q and its Shoup constant
     u64 two_q;
-    u64 pad;
+    u64 delta;        // 2^60 - q when that is below 2^32 (every prime of the pages' chain), else 0
 };
 
 // Device tables owned by a context (struct of device pointers, passed by value).
 struct Tables {
     int L, K, alpha, dnum, LK;
+    bool special;               // every prime is 2^60 - delta with delta < 2^32
     const PrimeConst *pc;       // [L+K]
     const ulonglong2 *tw_fwd;   // [L+K][n]: {psi^brv(k), Shoup}; k = 0 unused
     const ulonglong2 *tw_inv;   // [L+K][n]: {psi^-brv(k), Shoup}; k = 0 holds psi^-brv(1) n^-1
@@ -98,6 +99,27 @@ __device__ __forceinline__ u64 shoup_lazy(u64 a, u64 w, u64 wp, u64 q)
 }
 
 __device__ __forceinline__ u64 csub(u64 a, u64 m) { return a >= m ? a - m : a; }
+
+// High half of a 64x64-bit product, approximated from three 32x32 partial
+// products: the low-by-low product and the carries out of the two cross
+// products are dropped, so the result is at most 2 below floor(a b / 2^64).
+__device__ __forceinline__ u64 mulhi_approx(u64 a, u64 b)
+{
+    const u32 a0 = (u32)a, a1 = (u32)(a >> 32), b0 = (u32)b, b1 = (u32)(b >> 32);
+    return (u64)a1 * b1 + __umulhi(a0, b1) + __umulhi(a1, b0);
+}
+
+// Shoup product with the approximate quotient: a w - qh q with qh at most 3
+// below floor(a w / q), so the result lies in [0, 4q) for any 64-bit a.
+// kSpecial: q = 2^60 - delta with delta < 2^32, so qh q = qh 2^60 - qh delta
+// costs a shift and one 64x32 product instead of a full 64x64 low product.
+template <bool kSpecial>
+__device__ __forceinline__ u64 shoup4(u64 a, u64 w, u64 wp, u64 q, u64 delta)
+{
+    const u64 qh = mulhi_approx(a, wp);
+    if (kSpecial) return a * w + qh * (u32)delta - (qh << 60);
+    return a * w - qh * q;
+}
 
 __device__ __forceinline__ u64 shoup(u64 a, u64 w, u64 wp, u64 q)
 {

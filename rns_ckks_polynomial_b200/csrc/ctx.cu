@@ -243,7 +243,7 @@ static int build_tables(ckks_ctx *ctx)
         c.ninv = host_invmod((u64)n, q);
         c.ninvp = host_shoup(c.ninv, q);
         c.two_q = 2 * q;
-        c.pad = 0;
+        c.delta = (((u64)1 << 60) - q) < ((u64)1 << 32) ? ((u64)1 << 60) - q : 0;
         const u64 psi = host_find_psi(q, n), psi_inv = host_invmod(psi, q);
         std::vector<u64> pw(n), pwi(n);
         pw[0] = pwi[0] = 1;
@@ -309,6 +309,8 @@ static int build_tables(ckks_ctx *ctx)
         dn_pinv[i] = make_ulonglong2(pinv, host_shoup(pinv, qi));
     });
 
+    T.special = true;
+    for (const PrimeConst &c : pc) T.special = T.special && c.delta != 0;
     CKKS_TRY(upload(ctx, pc, &T.pc));
     CKKS_TRY(upload(ctx, fw, &T.tw_fwd));
     CKKS_TRY(upload(ctx, iw, &T.tw_inv));

@@ -7,10 +7,13 @@
 // exchanged between passes through a swizzled 32 KiB shared-memory tile
 // (two alternating 16 KiB buffers), so every exchange is bank-conflict free.
 //
-// Arithmetic: Harvey's lazy butterflies with Shoup twiddles.  The forward
-// (Cooley-Tukey) pass keeps values in [0, 4q), the inverse (Gentleman-Sande)
-// pass in [0, 2q); both end fully reduced to [0, q).  The inverse folds n^-1
-// into its last stage.
+// Arithmetic: Harvey-style lazy butterflies with Shoup twiddles whose
+// quotient comes from a three-product approximation of the high half
+// (shoup4: result in [0, 4q)).  The forward (Cooley-Tukey) pass keeps values
+// in [0, 8q), the inverse (Gentleman-Sande) pass in [0, 4q); 8q < 2^63 for
+// q < 2^60.  Both end fully reduced to [0, q).  The inverse folds n^-1 into
+// its last stage.  kS selects the cheaper quotient product for primes of the
+// form 2^60 - delta, delta < 2^32.
 //
 // Ordering (the library's reading of the pages, which name NTT/INTT but not
 // the convention): forward output slot k holds a(psi^(2 brv(k) + 1)); the
@@ -23,9 +26,9 @@
 // loads and stores.  A Job provides:
 //   int count;                                  number of limb jobs
 //   __device__ int prime(int j) const;          prime index of job j
-//   fwd:  __device__ u64  load(int j, int e)    element e (value < 4q)
+//   fwd:  __device__ u64  load(int j, int e)    element e (value < 8q)
 //         __device__ void store4(int j, int e, const u64 v[4])   e % 4 == 0
-//   inv:  __device__ void load4(int j, int e, u64 v[4])           values < 2q
+//   inv:  __device__ void load4(int j, int e, u64 v[4])           values < 4q
 //         __device__ void store(int j, int e, u64 v)
 #pragma once
 
@@ -42,86 +45,95 @@ __device__ __forceinline__ int swz(int e) { return e ^ ((e >> 4) & 3) ^ (((e >> 
 
 __device__ __forceinline__ ulonglong2 ldtw(const ulonglong2 *tw, int i) { return __ldg(tw + i); }
 
-// Cooley-Tukey butterfly, inputs and outputs in [0, 4q).
-__device__ __forceinline__ void ct_bfly(u64 &x, u64 &y, ulonglong2 w, u64 q, u64 q2)
+struct Mod {
+    u64 q, q2, q4, delta;
+};
+
+// Cooley-Tukey butterfly, inputs and outputs in [0, 8q).
+template <bool kS>
+__device__ __forceinline__ void ct_bfly(u64 &x, u64 &y, ulonglong2 w, const Mod &m)
 {
-    u64 a = csub(x, q2);
-    u64 t = shoup_lazy(y, w.x, w.y, q);
+    const u64 a = csub(x, m.q4);
+    const u64 t = shoup4<kS>(y, w.x, w.y, m.q, m.delta);
     x = a + t;
-    y = a - t + q2;
+    y = a - t + m.q4;
 }
 
-// Gentleman-Sande butterfly, inputs and outputs in [0, 2q).
-__device__ __forceinline__ void gs_bfly(u64 &x, u64 &y, ulonglong2 w, u64 q, u64 q2)
+// Gentleman-Sande butterfly, inputs and outputs in [0, 4q).
+template <bool kS>
+__device__ __forceinline__ void gs_bfly(u64 &x, u64 &y, ulonglong2 w, const Mod &m)
 {
-    u64 s = x + y;
-    u64 d = x - y + q2;
-    x = csub(s, q2);
-    y = shoup_lazy(d, w.x, w.y, q);
+    const u64 s = x + y;
+    const u64 d = x - y + m.q4;
+    x = csub(s, m.q4);
+    y = shoup4<kS>(d, w.x, w.y, m.q, m.delta);
 }
 
 // Three forward stages (half-sizes 4S, 2S, S) on v[k] = a[base + r + S k],
 // base a multiple of 8S; m1 = (n + base) / (8S).
-__device__ __forceinline__ void fwd_radix8(u64 v[8], int m1, const ulonglong2 *tw, u64 q, u64 q2)
+template <bool kS>
+__device__ __forceinline__ void fwd_radix8(u64 v[8], int m1, const ulonglong2 *tw, const Mod &m)
 {
-    ulonglong2 w = ldtw(tw, m1);
+    const ulonglong2 w = ldtw(tw, m1);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) ct_bfly(v[k], v[k + 4], w, q, q2);
-    ulonglong2 w0 = ldtw(tw, 2 * m1), w1 = ldtw(tw, 2 * m1 + 1);
-    ct_bfly(v[0], v[2], w0, q, q2);
-    ct_bfly(v[1], v[3], w0, q, q2);
-    ct_bfly(v[4], v[6], w1, q, q2);
-    ct_bfly(v[5], v[7], w1, q, q2);
+    for (int k = 0; k < 4; ++k) ct_bfly<kS>(v[k], v[k + 4], w, m);
+    const ulonglong2 w0 = ldtw(tw, 2 * m1), w1 = ldtw(tw, 2 * m1 + 1);
+    ct_bfly<kS>(v[0], v[2], w0, m);
+    ct_bfly<kS>(v[1], v[3], w0, m);
+    ct_bfly<kS>(v[4], v[6], w1, m);
+    ct_bfly<kS>(v[5], v[7], w1, m);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) ct_bfly(v[2 * k], v[2 * k + 1], ldtw(tw, 4 * m1 + k), q, q2);
+    for (int k = 0; k < 4; ++k) ct_bfly<kS>(v[2 * k], v[2 * k + 1], ldtw(tw, 4 * m1 + k), m);
 }
 
 // Two forward stages (half-sizes 2, 1) on four consecutive elements 4g..4g+3.
-__device__ __forceinline__ void fwd_radix4(u64 *v, int g, const ulonglong2 *tw, u64 q, u64 q2)
+template <bool kS>
+__device__ __forceinline__ void fwd_radix4(u64 *v, int g, const ulonglong2 *tw, const Mod &m)
 {
     const int m1 = (kN >> 2) + g;
-    ulonglong2 w = ldtw(tw, m1);
-    ct_bfly(v[0], v[2], w, q, q2);
-    ct_bfly(v[1], v[3], w, q, q2);
-    ct_bfly(v[0], v[1], ldtw(tw, 2 * m1), q, q2);
-    ct_bfly(v[2], v[3], ldtw(tw, 2 * m1 + 1), q, q2);
+    const ulonglong2 w = ldtw(tw, m1);
+    ct_bfly<kS>(v[0], v[2], w, m);
+    ct_bfly<kS>(v[1], v[3], w, m);
+    ct_bfly<kS>(v[0], v[1], ldtw(tw, 2 * m1), m);
+    ct_bfly<kS>(v[2], v[3], ldtw(tw, 2 * m1 + 1), m);
 }
 
-__device__ __forceinline__ void inv_radix4(u64 *v, int g, const ulonglong2 *tw, u64 q, u64 q2)
+template <bool kS>
+__device__ __forceinline__ void inv_radix4(u64 *v, int g, const ulonglong2 *tw, const Mod &m)
 {
     const int m1 = (kN >> 2) + g;
-    gs_bfly(v[0], v[1], ldtw(tw, 2 * m1), q, q2);
-    gs_bfly(v[2], v[3], ldtw(tw, 2 * m1 + 1), q, q2);
-    ulonglong2 w = ldtw(tw, m1);
-    gs_bfly(v[0], v[2], w, q, q2);
-    gs_bfly(v[1], v[3], w, q, q2);
+    gs_bfly<kS>(v[0], v[1], ldtw(tw, 2 * m1), m);
+    gs_bfly<kS>(v[2], v[3], ldtw(tw, 2 * m1 + 1), m);
+    const ulonglong2 w = ldtw(tw, m1);
+    gs_bfly<kS>(v[0], v[2], w, m);
+    gs_bfly<kS>(v[1], v[3], w, m);
 }
 
 // Three inverse stages (half-sizes S, 2S, 4S).  kLast folds n^-1 into the
 // final stage (half-size n/2): tw[0] holds psi^-brv(1) n^-1.
-template <bool kLast>
-__device__ __forceinline__ void inv_radix8(u64 v[8], int m1, const ulonglong2 *tw, u64 q, u64 q2,
+template <bool kS, bool kLast>
+__device__ __forceinline__ void inv_radix8(u64 v[8], int m1, const ulonglong2 *tw, const Mod &m,
                                            u64 ninv, u64 ninvp)
 {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) gs_bfly(v[2 * k], v[2 * k + 1], ldtw(tw, 4 * m1 + k), q, q2);
-    ulonglong2 w0 = ldtw(tw, 2 * m1), w1 = ldtw(tw, 2 * m1 + 1);
-    gs_bfly(v[0], v[2], w0, q, q2);
-    gs_bfly(v[1], v[3], w0, q, q2);
-    gs_bfly(v[4], v[6], w1, q, q2);
-    gs_bfly(v[5], v[7], w1, q, q2);
+    for (int k = 0; k < 4; ++k) gs_bfly<kS>(v[2 * k], v[2 * k + 1], ldtw(tw, 4 * m1 + k), m);
+    const ulonglong2 w0 = ldtw(tw, 2 * m1), w1 = ldtw(tw, 2 * m1 + 1);
+    gs_bfly<kS>(v[0], v[2], w0, m);
+    gs_bfly<kS>(v[1], v[3], w0, m);
+    gs_bfly<kS>(v[4], v[6], w1, m);
+    gs_bfly<kS>(v[5], v[7], w1, m);
     if (kLast) {
-        ulonglong2 w = ldtw(tw, 0);
+        const ulonglong2 w = ldtw(tw, 0);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            u64 x = v[k], y = v[k + 4];
-            v[k] = shoup_lazy(x + y, ninv, ninvp, q);
-            v[k + 4] = shoup_lazy(x - y + q2, w.x, w.y, q);
+            const u64 x = v[k], y = v[k + 4];
+            v[k] = shoup4<kS>(x + y, ninv, ninvp, m.q, m.delta);
+            v[k + 4] = shoup4<kS>(x - y + m.q4, w.x, w.y, m.q, m.delta);
         }
     } else {
-        ulonglong2 w = ldtw(tw, m1);
+        const ulonglong2 w = ldtw(tw, m1);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) gs_bfly(v[k], v[k + 4], w, q, q2);
+        for (int k = 0; k < 4; ++k) gs_bfly<kS>(v[k], v[k + 4], w, m);
     }
 }
 
@@ -141,7 +153,7 @@ __device__ __forceinline__ void exchange(u64 v[8], u64 *buf, int tid)
     for (int k = 0; k < 8; ++k) v[k] = buf[swz(G::at(tid, k))];
 }
 
-template <class Job>
+template <class Job, bool kS>
 __global__ void __launch_bounds__(kNttThreads) ntt_fwd_kernel(Job job, Tables T, int per_block)
 {
     __shared__ u64 sm[2][kN];
@@ -152,28 +164,28 @@ __global__ void __launch_bounds__(kNttThreads) ntt_fwd_kernel(Job job, Tables T,
         if (j >= job.count) break;
         const int p = job.prime(j);
         const PrimeConst &pc = T.pc[p];
-        const u64 q = pc.q, q2 = pc.two_q;
+        const Mod m{pc.q, pc.two_q, 2 * pc.two_q, pc.delta};
         const ulonglong2 *tw = T.tw_fwd + (size_t)p * kN;
         u64 v[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = job.load(j, IdxA::at(tid, k));
-        fwd_radix8(v, 1, tw, q, q2);
+        fwd_radix8<kS>(v, 1, tw, m);
         exchange<IdxA, IdxB>(v, sm[0], tid);
-        fwd_radix8(v, 8 + (tid >> 5), tw, q, q2);
+        fwd_radix8<kS>(v, 8 + (tid >> 5), tw, m);
         exchange<IdxB, IdxC>(v, sm[1], tid);
-        fwd_radix8(v, 64 + (tid >> 2), tw, q, q2);
+        fwd_radix8<kS>(v, 64 + (tid >> 2), tw, m);
         exchange<IdxC, IdxD>(v, sm[0], tid);
-        fwd_radix4(v, tid, tw, q, q2);
-        fwd_radix4(v + 4, tid + 256, tw, q, q2);
+        fwd_radix4<kS>(v, tid, tw, m);
+        fwd_radix4<kS>(v + 4, tid + 256, tw, m);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = csub(csub(v[k], q2), q);
+        for (int k = 0; k < 8; ++k) v[k] = csub(csub(csub(v[k], m.q4), m.q2), m.q);
         job.store4(j, 4 * tid, v);
         job.store4(j, 4 * (tid + 256), v + 4);
         if (jj + 1 < per_block) __syncthreads();
     }
 }
 
-template <class Job>
+template <class Job, bool kS>
 __global__ void __launch_bounds__(kNttThreads) ntt_inv_kernel(Job job, Tables T, int per_block)
 {
     __shared__ u64 sm[2][kN];
@@ -184,21 +196,21 @@ __global__ void __launch_bounds__(kNttThreads) ntt_inv_kernel(Job job, Tables T,
         if (j >= job.count) break;
         const int p = job.prime(j);
         const PrimeConst &pc = T.pc[p];
-        const u64 q = pc.q, q2 = pc.two_q;
+        const Mod m{pc.q, pc.two_q, 2 * pc.two_q, pc.delta};
         const ulonglong2 *tw = T.tw_inv + (size_t)p * kN;
         u64 v[8];
         job.load4(j, 4 * tid, v);
         job.load4(j, 4 * (tid + 256), v + 4);
-        inv_radix4(v, tid, tw, q, q2);
-        inv_radix4(v + 4, tid + 256, tw, q, q2);
+        inv_radix4<kS>(v, tid, tw, m);
+        inv_radix4<kS>(v + 4, tid + 256, tw, m);
         exchange<IdxD, IdxC>(v, sm[0], tid);
-        inv_radix8<false>(v, 64 + (tid >> 2), tw, q, q2, 0, 0);
+        inv_radix8<kS, false>(v, 64 + (tid >> 2), tw, m, 0, 0);
         exchange<IdxC, IdxB>(v, sm[1], tid);
-        inv_radix8<false>(v, 8 + (tid >> 5), tw, q, q2, 0, 0);
+        inv_radix8<kS, false>(v, 8 + (tid >> 5), tw, m, 0, 0);
         exchange<IdxB, IdxA>(v, sm[0], tid);
-        inv_radix8<true>(v, 1, tw, q, q2, pc.ninv, pc.ninvp);
+        inv_radix8<kS, true>(v, 1, tw, m, pc.ninv, pc.ninvp);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) job.store(j, IdxA::at(tid, k), csub(v[k], q));
+        for (int k = 0; k < 8; ++k) job.store(j, IdxA::at(tid, k), csub(csub(v[k], m.q2), m.q));
         if (jj + 1 < per_block) __syncthreads();
     }
 }
@@ -218,7 +230,10 @@ inline int launch_ntt_fwd(const Job &job, const Tables &T, cudaStream_t s)
     if (job.count <= 0) return CKKS_OK;
     int per = ntt_per_block(job.count);
     int blocks = (job.count + per - 1) / per;
-    ntt_fwd_kernel<Job><<<blocks, kNttThreads, 0, s>>>(job, T, per);
+    if (T.special)
+        ntt_fwd_kernel<Job, true><<<blocks, kNttThreads, 0, s>>>(job, T, per);
+    else
+        ntt_fwd_kernel<Job, false><<<blocks, kNttThreads, 0, s>>>(job, T, per);
     CKKS_CHECK_LAUNCH("ntt_fwd_kernel");
     return CKKS_OK;
 }
@@ -229,7 +244,10 @@ inline int launch_ntt_inv(const Job &job, const Tables &T, cudaStream_t s)
     if (job.count <= 0) return CKKS_OK;
     int per = ntt_per_block(job.count);
     int blocks = (job.count + per - 1) / per;
-    ntt_inv_kernel<Job><<<blocks, kNttThreads, 0, s>>>(job, T, per);
+    if (T.special)
+        ntt_inv_kernel<Job, true><<<blocks, kNttThreads, 0, s>>>(job, T, per);
+    else
+        ntt_inv_kernel<Job, false><<<blocks, kNttThreads, 0, s>>>(job, T, per);
     CKKS_CHECK_LAUNCH("ntt_inv_kernel");
     return CKKS_OK;
 }
