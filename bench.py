@@ -24,7 +24,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -43,12 +42,14 @@ L2_FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-ks", action="store_true", help="skip the key-switch measurements")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--ks-only", action="store_true",
+                    help="run only the key-switch measurements (for profiling)")
     ap.add_argument("--sweep", default=",".join(str(x) for x in SWEEP),
                     help="limb counts of the step (a smaller case for profiling only)")
     return ap.parse_args()
@@ -64,54 +65,65 @@ def peaks():
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples nvidia-smi every 200 ms while active."""
+    """Samples the SM clock and the clock-event reasons through NVML every
+    `period` seconds while active (the same counters nvidia-smi reports)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, torch_device, period=0.002):
+        self.dev = torch_device
+        self.period = period
         self.samples = []
-        self.proc = None
+        self.max_mhz = None
+        self.handle = None
+        self._stop = threading.Event()
+
+    def _open(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.dev)
+        bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        return pynvml
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            nv = self._open()
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unsampled
+            self.error = repr(e)
+            return self
+
+        def run():
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                    self.samples.append((mhz, int(get_reasons(self.handle))))
+                except Exception:  # noqa: BLE001
+                    pass
+                time.sleep(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) == 6:
-                self.samples.append(parts)
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if getattr(self, "thread", None):
+            self.thread.join(timeout=2)
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[2 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.samples)}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"],
+                    "error": getattr(self, "error", None)}
+        reasons = sorted({name for _, r in self.samples for bit, name in self.REASONS.items()
+                          if r & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -229,7 +241,7 @@ def run_b200(args):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         for s in range(args.steps):
             flush.zero_()  # L2 flush between steps, outside the timed events
             starts[s].record(stream)
@@ -515,8 +527,21 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_ks_only():
+    import torch
+    dev = torch.device("cuda", 0)
+    hbm_peak, _ = peaks()
+    from rns_ckks_polynomial_b200 import Context, primes
+    ctx = Context(primes(60), primes(61)[60:], 60)
+    ipeak = intpipe_peaks(ctx)
+    print(json.dumps({"keyswitch": run_keyswitch(dev, hbm_peak, ipeak)}), flush=True)
+
+
 def main():
     args = parse()
+    if args.ks_only:
+        run_ks_only()
+        return
     global SWEEP
     SWEEP = tuple(int(x) for x in args.sweep.split(","))
     if args.impl == "reference":

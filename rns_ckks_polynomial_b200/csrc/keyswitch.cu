@@ -32,7 +32,7 @@ namespace ckks {
 
 // ---------------------------------------------------------------- basis conversion
 constexpr int kConvThreads = 128;
-constexpr int kConvTT = 16;  // targets per thread (and per CTA)
+constexpr int kConvTT = 8;  // targets per thread (and per CTA)
 
 template <class Map>
 __global__ void __launch_bounds__(kConvThreads) conv_kernel(Map m, const PrimeConst *__restrict__ pc)
@@ -219,14 +219,27 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 }
 
 // ---------------------------------------------------------------- key inner product
+// One thread per output coefficient k of one (prime t, key r, ciphertext b)
+// job.  The 1-D grid is ordered coefficient tile fastest, then ciphertext,
+// then key, then prime, so the CTAs that read the same key rows (all
+// ciphertexts of one key at one prime) run back to back: a key row crosses
+// HBM once and is re-served from L2, and the gathered digit row of one job is
+// shared by its eight coefficient-tile CTAs through L1/L2.  The Galois
+// permutation is the gather on the digit load.
 __global__ void __launch_bounds__(256) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
-                                                        int per_key, int hoisted,
+                                                        int per_key, int nkeys, int hoisted,
                                                         u64 *__restrict__ acc, Tables T)
 {
-    const int t = blockIdx.y, z = blockIdx.z;
-    const int k = blockIdx.x * 256 + threadIdx.x;
-    const int r = z / per_key;
-    const int dset = hoisted ? z - r * per_key : z;
+    int id = blockIdx.x;
+    const int tile = id % (kN / 256);
+    id /= kN / 256;
+    const int b = id % per_key;
+    id /= per_key;
+    const int r = id % nkeys;
+    const int t = id / nkeys;
+    const int k = tile * 256 + threadIdx.x;
+    const int z = r * per_key + b;
+    const int dset = hoisted ? b : z;
     const u32 g = kl.galois[r];
     const int src = g == 1u ? k : (int)galois_src((u32)k, g);
     const size_t LKn = (size_t)T.LK * kN;
@@ -249,8 +262,10 @@ int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, i
 {
     if (jobs <= 0) return CKKS_OK;
     const Tables &T = ctx->t;
-    dim3 grid(kN / 256, T.LK, jobs);
-    key_inner_kernel<<<grid, 256, 0, s>>>(digits, kl, per_key, hoisted ? 1 : 0, acc, T);
+    const int nkeys = jobs / per_key;
+    const size_t blocks = (size_t)(kN / 256) * jobs * T.LK;
+    if (blocks > 0x7fffffffull) return set_error(CKKS_EUNSUPPORTED, "key inner product grid too large");
+    key_inner_kernel<<<(unsigned)blocks, 256, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T);
     CKKS_CHECK_LAUNCH("key_inner_kernel");
     return CKKS_OK;
 }

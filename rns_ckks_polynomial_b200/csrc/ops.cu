@@ -495,8 +495,9 @@ __global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, u64 *s
 #pragma unroll
         for (int k = 0; k < 8; ++k) y[k] = x[k] ^ 0x5555555555ull;
         for (int it = 0; it < iters; ++it) {
+            const u64 m = w ^ (u64)it;  // a new multiplier every iteration: nothing to hoist
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mac128(h[k], x[k], y[k], w);  // 8 independent chains
+            for (int k = 0; k < 8; ++k) mac128(h[k], x[k], y[k], m);  // 8 independent chains
         }
     } else {
         for (int it = 0; it < iters; ++it) {
