@@ -157,6 +157,27 @@ int ckks_automorph(const ckks_ctx *ctx, const uint64_t *in, uint64_t *out, int b
 int ckks_modup(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int batch,
                void *ws, ckks_stream_t stream);
 
+/* ModUp that allocates nothing.  The paper has no counterpart: this entry point
+ * exists for callers that cannot call cudaMalloc.  Examples are a host
+ * framework whose caching allocator already owns the device memory under a
+ * fixed budget, and a latency-critical loop that cannot absorb the device-wide
+ * synchronisation that cudaMalloc/cudaFree can imply.
+ * Same arguments, layouts and result as ckks_modup, without a workspace
+ * argument.  Its scratch is a 32 MiB static device array inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ * Limit: batch * L <= 2048.  Larger requests return CKKS_EUNSUPPORTED and
+ * launch nothing.
+ * The first call on a device resolves the array's device address
+ * (cudaGetSymbolAddress, once per device); make that first call before any
+ * stream capture.
+ * Every call shares the one array, so calls that overlap on the GPU (other
+ * streams, other host threads, the same device) race: serialise them.  No
+ * part of the array needs clearing between calls, because every word a call
+ * reads was written earlier in the same call.  Calls no cudaMalloc, cudaFree
+ * or allocating library routine. */
+int ckks_modup_noalloc(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int batch,
+                       ckks_stream_t stream);
+
 /* Key inner product with the automorphism fused into the digit load:
  * acc[batch][2][L+K][n] with acc[b][c][t][k] = sum_j phi_g(D_j)[t][k] *
  * key[j][c][t][k] mod t.  digits [batch][dnum][L+K][n], key

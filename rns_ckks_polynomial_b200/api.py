@@ -135,6 +135,17 @@ class Context:
                                              _stream(c)))
         return out
 
+    def modup_noalloc(self, c, out):
+        """ModUp whose scratch is the library's static device array: nothing
+        is allocated (the caller provides `out`, [B][dnum][L+K][n]).  Limit:
+        B * L <= 2048."""
+        B = c.shape[0]
+        _ptr(c, "c_ntt", (B, self.L, self.n))
+        _ptr(out, "digits", (B, self.dnum, self.L + self.K, self.n))
+        check("ckks_modup_noalloc", lib().ckks_modup_noalloc(self._h, _ptr(c, "c"), _ptr(out, "digits"),
+                                                             B, _stream(c)))
+        return out
+
     def key_inner(self, digits, key, galois=1, out=None):
         B = digits.shape[0]
         LK = self.L + self.K

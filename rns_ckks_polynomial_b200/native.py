@@ -27,6 +27,7 @@ SIGNATURES = {
     "ckks_pointwise": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_automorph": (C.c_int, [_vp, _vp, _vp, C.c_int, C.c_int, C.c_uint32, _vp]),
     "ckks_modup": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp, _vp]),
+    "ckks_modup_noalloc": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp]),
     "ckks_key_inner": (C.c_int, [_vp, _vp, _vp, C.c_uint32, _vp, C.c_int, _vp]),
     "ckks_moddown": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp, _vp]),
     "ckks_keyswitch": (C.c_int, [_vp, _vp, _vp, _vp, C.c_int, _vp, _vp]),

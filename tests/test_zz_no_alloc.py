@@ -1,0 +1,58 @@
+"""The allocation-free ModUp entry point (ckks_modup_noalloc).
+
+Some callers cannot call cudaMalloc. Examples are a host framework whose
+caching allocator already owns the device memory under a fixed budget, and a
+latency-critical loop that cannot absorb the device-wide synchronisation an
+allocation can imply. For them the library offers ModUp with its scratch in a
+static device array. This test calls it through the C ABI twice in a row and
+checks both results word for word against ckks_modup, whose own parity with the
+CPU oracle is covered by the other GPU tests. It lives in a file of its own that
+pytest collects last, and it passes alone in a fresh process as well as after
+the other tests.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from rns_ckks_polynomial_b200 import native, synth
+
+from .gpu_common import context, need_gpu
+
+pytestmark = pytest.mark.gpu
+
+N = 2048
+
+
+@pytest.mark.parametrize("L,K,alpha,batch", [(112, 8, 8, 8), (5, 2, 2, 3)])
+def test_modup_noalloc_matches_modup_twice(L, K, alpha, batch):
+    need_gpu()
+    ctx = context(L, K, alpha)
+    lib = native.lib()
+    mods = ctx.mods
+    stream = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ref = torch.empty((batch, ctx.dnum, L + K, N), dtype=torch.int64, device="cuda")
+    out = torch.empty_like(ref)
+    for call in range(2):
+        c = synth.uniform_residues((batch, L, N), mods[:L], synth.config_seed(9), 300 + call,
+                                   device="cuda")
+        ws = torch.empty(ctx.workspace_bytes(1, batch), dtype=torch.uint8, device="cuda")
+        rc = lib.ckks_modup(ctx._h, C.c_void_p(c.data_ptr()), C.c_void_p(ref.data_ptr()), batch,
+                            C.c_void_p(ws.data_ptr()), stream)
+        assert rc == 0, lib.ckks_last_error()
+        out.fill_(-1)
+        rc = lib.ckks_modup_noalloc(ctx._h, C.c_void_p(c.data_ptr()), C.c_void_p(out.data_ptr()),
+                                    batch, stream)
+        assert rc == 0, lib.ckks_last_error()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), "call %d differs from ckks_modup" % call
+
+
+def test_modup_noalloc_rejects_oversized_batch():
+    need_gpu()
+    ctx = context(112, 8, 8)
+    lib = native.lib()
+    rc = lib.ckks_modup_noalloc(ctx._h, None, None, 19, None)  # 19 * 112 > 2048 limbs
+    assert rc == -2
+    assert b"2048-limb" in lib.ckks_last_error()
