@@ -102,6 +102,16 @@ void ckks_ctx_destroy(ckks_ctx *ctx);
 /* Message for the last non-OK status returned on this host thread. */
 const char *ckks_last_error(void);
 
+/* Waits for the context's device and reports whether any kernel of this
+ * context gave up a bounded wait since the last call: CKKS_ECUDA with a
+ * message if so (the flag is then cleared), else CKKS_OK.  Only the int8
+ * tensor-core basis conversion (digits or special bases of more than 16
+ * primes) waits on the device; it bounds every wait, and if one expires it
+ * stops issuing work, frees its tensor memory and raises the flag, so the
+ * affected outputs must be discarded.  Also returns CKKS_ECUDA for an
+ * asynchronous CUDA error on the device. */
+int ckks_device_status(const ckks_ctx *ctx);
+
 /* Context parameters: writes L, K, alpha, dnum, n (any pointer may be NULL). */
 int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n);
 

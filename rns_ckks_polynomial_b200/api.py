@@ -73,6 +73,10 @@ class Context:
         except Exception:
             pass
 
+    def device_status(self):
+        """Synchronise the device and raise if a bounded device wait expired."""
+        check("ckks_device_status", lib().ckks_device_status(self._h))
+
     # ------------------------------------------------------------ helpers
     def _empty(self, *shape):
         return torch.empty(shape, dtype=torch.int64, device=self.device)

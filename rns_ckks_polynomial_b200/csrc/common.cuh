@@ -46,6 +46,11 @@ struct Tables {
     const ulonglong2 *dn_hatinv;  // [K]: {[(P/p_k)^-1]_{p_k}, Shoup}
     const u64 *dn_mat;            // [K][L]: [P/p_k]_{q_i}
     const ulonglong2 *dn_pinv;    // [L]: {[P^-1]_{q_i}, Shoup}
+    // Byte planes of the conversion matrices for the int8 tensor-core path (null when the digit /
+    // special basis is small enough for the CUDA-core kernel)
+    const uint8_t *tc_up;         // [dnum][tb_per_digit][8][128 x 64]
+    const uint8_t *tc_dn;         // [ceil(L/128)][8][128 x 64]
+    int tc_tb_per_digit;
 };
 
 }  // namespace ckks
@@ -61,6 +66,7 @@ struct ckks_ctx {
     std::mutex mu;
     void *own_ws = nullptr;
     size_t own_ws_bytes = 0;
+    int *tc_err = nullptr;  // device flag: a bounded wait of the tensor-core kernel expired
 };
 
 namespace ckks {

@@ -10,7 +10,7 @@
 #include <functional>
 #include <thread>
 
-#include "common.cuh"
+#include "internal.cuh"
 
 namespace ckks {
 
@@ -319,7 +319,7 @@ static int build_tables(ckks_ctx *ctx)
     CKKS_TRY(upload(ctx, dn_hatinv, &T.dn_hatinv));
     CKKS_TRY(upload(ctx, dn_mat, &T.dn_mat));
     CKKS_TRY(upload(ctx, dn_pinv, &T.dn_pinv));
-    return CKKS_OK;
+    return build_tc_tables(ctx, up_mat, dn_mat);
 }
 
 static void free_ctx(ckks_ctx *ctx)
@@ -403,6 +403,23 @@ extern "C" void ckks_ctx_destroy(ckks_ctx *ctx)
     cudaSetDevice(ctx->device);
     cudaDeviceSynchronize();
     free_ctx(ctx);
+}
+
+extern "C" int ckks_device_status(const ckks_ctx *ctx)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(set_device(ctx));
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e, "cudaDeviceSynchronize");
+    if (!ctx->tc_err) return CKKS_OK;
+    int flag = 0;
+    e = cudaMemcpy(&flag, ctx->tc_err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e, "cudaMemcpy(flag)");
+    if (flag) {
+        cudaMemset(ctx->tc_err, 0, sizeof(int));
+        return set_error(CKKS_ECUDA, "a tensor-core conversion gave up waiting for its matrix products");
+    }
+    return CKKS_OK;
 }
 
 extern "C" int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n)

@@ -29,6 +29,13 @@ struct Carve {
 
 inline size_t limbs_bytes(size_t rows) { return ((rows * kN * sizeof(u64)) + 255) & ~(size_t)255; }
 
+// ---- int8 tensor-core basis conversion (conv_tc.cu)
+constexpr int kTcMinSources = 16;  // conversions with more sources use the tensor cores
+bool tc_wanted(int sources);
+int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::vector<u64> &dn_mat);
+int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
+int launch_conv_tc_down(const ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);
+
 // ---- sizes of internal stages (bytes)
 size_t modup_ws_bytes(const ckks_ctx *ctx, int batch);
 size_t moddown_ws_bytes(const ckks_ctx *ctx, int jobs);

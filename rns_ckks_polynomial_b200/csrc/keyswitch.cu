@@ -212,8 +212,12 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
                            T.L, T.LK, T.alpha, T.dnum, batch, T.L * batch};
         CKKS_TRY(launch_ntt_inv(j, T, s));
     }
-    UpConvMap m{y, digits, T.up_mat, T.L, T.LK, T.alpha, T.dnum};
-    CKKS_TRY(launch_conv(m, T.LK - 1, batch * T.dnum, T, s));
+    if (T.tc_up) {
+        CKKS_TRY(launch_conv_tc_up(ctx, y, digits, batch, s));
+    } else {
+        UpConvMap m{y, digits, T.up_mat, T.L, T.LK, T.alpha, T.dnum};
+        CKKS_TRY(launch_conv(m, T.LK - 1, batch * T.dnum, T, s));
+    }
     UpNttJob nj{digits, T.L, T.LK, T.alpha, T.dnum, batch, batch * (T.dnum * T.LK - T.L)};
     return launch_ntt_fwd(nj, T, s);
 }
@@ -364,8 +368,12 @@ int moddown_stage(const ckks_ctx *ctx, const u64 *acc, u64 *out, int jobs, const
     u64 *cvb = c.take<u64>((size_t)jobs2 * T.L * kN);
     DownInttJob ij{acc, zb, T.dn_hatinv, T.pc, T.L, T.K, T.LK, jobs2, T.K * jobs2};
     CKKS_TRY(launch_ntt_inv(ij, T, s));
-    DownConvMap m{zb, cvb, T.dn_mat, T.L, T.K};
-    CKKS_TRY(launch_conv(m, T.L, jobs2, T, s));
+    if (T.tc_dn) {
+        CKKS_TRY(launch_conv_tc_down(ctx, zb, cvb, jobs2, s));
+    } else {
+        DownConvMap m{zb, cvb, T.dn_mat, T.L, T.K};
+        CKKS_TRY(launch_conv(m, T.L, jobs2, T, s));
+    }
     switch (ex.kind) {
     case 1: {
         DownFinalJob<1> fj{cvb, acc, out, T.dn_pinv, T.pc, T.L, T.LK, jobs2, T.L * jobs2, ex};

@@ -145,8 +145,11 @@ def test_automorph_rejects_even_and_in_place():
 
 
 # ------------------------------------------------------------------ key switching stages
-@pytest.mark.parametrize("L,K,alpha", [(4, 1, 1), (6, 2, 2), (5, 2, 2), (112, 8, 8), (20, 3, 7)])
+@pytest.mark.parametrize("L,K,alpha", [(4, 1, 1), (6, 2, 2), (5, 2, 2), (112, 8, 8), (20, 3, 7),
+                                       (40, 20, 20), (70, 33, 33), (130, 64, 64)])
 def test_modup_inner_moddown_stages(orc, L, K, alpha):
+    """Digits / special bases above 16 primes run the int8 tensor-core
+    conversion; (70, 33, 33) has a ragged 4-prime last digit."""
     p = Params(L, K, alpha)
     ctx = ctx_for(p)
     mods = np.array(ctx.mods, dtype=np.uint64)
@@ -163,6 +166,7 @@ def test_modup_inner_moddown_stages(orc, L, K, alpha):
     assert_bits_equal(host(out), orc.moddown(want_a, mods, L, K), "moddown")
     ks = ctx.keyswitch(dev(c), dev(key))
     assert_bits_equal(host(ks), orc.keyswitch(c, key, mods, L, K, alpha), "keyswitch")
+    ctx.device_status()
 
 
 def test_hoisted_rotations_match_and_decrypt(orc):
@@ -180,6 +184,23 @@ def test_hoisted_rotations_match_and_decrypt(orc):
     for i, r in enumerate(rs):
         for b in range(3):
             assert np.max(np.abs(sch.decrypt_slots(out[i, b]) - rot_left(zs[b], r))) < 1e-8
+
+
+def test_tensor_core_rotation_decrypts(orc):
+    """Rotation with 20-prime digits and 20 special primes (tensor-core ModUp
+    and ModDown) decrypts to the slot rotation."""
+    p = Params(40, 20, 20)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 7)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 77).numpy()
+    ct = sch.encrypt_slots(z)
+    g = galois_for_rotation(3)
+    key = sch.keygen_galois(g)
+    out = host(ctx.rotate(dev(ct[None]), [dev(key)], [g]))
+    ctx.device_status()
+    assert_bits_equal(out, orc.rotate(ct[None], [key], np.array([g], dtype=np.uint64), sch.mods,
+                                      p.L, p.K, p.alpha), "rotate")
+    assert np.max(np.abs(sch.decrypt_slots(out[0, 0]) - rot_left(z, 3))) < 1e-8
 
 
 def test_rotate_context_owned_workspace(orc):
@@ -321,6 +342,7 @@ def test_config5_boot_rotation_full_size_sampled(orc):
     keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device="cuda")
             for r in range(4)]
     out = ctx.rotate(ct, keys, gal)
+    ctx.device_status()
     got = host(out[2, 3])
     want = orc.rotate(host(ct[3:4]), [host(keys[2])], np.array([gal[2]], dtype=np.uint64), mods,
                       2100, 60, 60)
