@@ -50,6 +50,10 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--ks-only", action="store_true",
                     help="run only the key-switch measurements (for profiling)")
+    ap.add_argument("--ks-batch", type=int, default=8,
+                    help="ciphertexts per key-switch workload (8 = the configs; smaller only for profiling)")
+    ap.add_argument("--ks-keys", type=int, default=4,
+                    help="Galois keys of the boot-level rotation (4 = the config; smaller only for profiling)")
     ap.add_argument("--sweep", default=",".join(str(x) for x in SWEEP),
                     help="limb counts of the step (a smaller case for profiling only)")
     return ap.parse_args()
@@ -355,8 +359,9 @@ def _time_call(fn, reps, stream):
     return a.elapsed_time(b) / reps
 
 
-def run_keyswitch(dev, hbm_peak, ipeak):
-    """Key switches per second of the three key-switching workloads."""
+def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
+    """Key switches per second of the three key-switching workloads (B ciphertexts each; the
+    boot-level rotation with R Galois keys)."""
     import torch
 
     from rns_ckks_polynomial_b200 import Context, primes, synth
@@ -367,15 +372,15 @@ def run_keyswitch(dev, hbm_peak, ipeak):
     seed = synth.config_seed(5)
     mods = primes(2160)
     ctx = Context(mods[:2100], mods[2100:], 60, device=dev.index)
-    ct = synth.uniform_residues((8, 2, 2100, N), mods[:2100], seed, 1, device=dev)
-    keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device=dev) for r in range(4)]
-    gal = [5, 25, 625, 1505]
-    res = torch.empty((4, 8, 2, 2100, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(4, 8, 4), dtype=torch.uint8, device=dev)
+    ct = synth.uniform_residues((B, 2, 2100, N), mods[:2100], seed, 1, device=dev)
+    keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device=dev) for r in range(R)]
+    gal = [5, 25, 625, 1505][:R]
+    res = torch.empty((R, B, 2, 2100, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(4, B, R), dtype=torch.uint8, device=dev)
     ms = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 3, stream)
     up, _, down = ks_work_keyswitch_parts(2100, 60, 60)
-    conv = 8 * (up["mac"] + 4 * down["mac"])
-    out["boot_rotation_L2100"] = ks_entry(32, ms, ks_work_rotation(2100, 60, 60, 8, 4), hbm_peak,
+    conv = B * (up["mac"] + R * down["mac"])
+    out["boot_rotation_L2100"] = ks_entry(B * R, ms, ks_work_rotation(2100, 60, 60, B, R), hbm_peak,
                                           mm_peak, mac_peak, conv_macs=conv, tensor=True)
     ctx.device_status()
     del ct, keys, res, ws, ctx
@@ -384,23 +389,23 @@ def run_keyswitch(dev, hbm_peak, ipeak):
     seed = synth.config_seed(3)
     mods = primes(120)
     ctx = Context(mods[:112], mods[112:], 8, device=dev.index)
-    a = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 1, device=dev)
-    b = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 2, device=dev)
+    a = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
+    b = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 2, device=dev)
     rlk = synth.uniform_residues((14, 2, 120, N), mods, seed, 3, device=dev)
-    res = torch.empty((8, 2, 111, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(6, 8), dtype=torch.uint8, device=dev)
+    res = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
     ms = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 10, stream)
-    out["layer_mul_relin_L112"] = ks_entry(8, ms, ks_work_mrr(112, 8, 8, 8), hbm_peak, mm_peak, mac_peak)
+    out["layer_mul_relin_L112"] = ks_entry(B, ms, ks_work_mrr(112, 8, 8, B), hbm_peak, mm_peak, mac_peak)
     # BSGS: bb = gg = 32, 62 keys, 8 cts
     seed = synth.config_seed(4)
-    x = synth.uniform_residues((8, 2, 112, N), mods[:112], seed, 1, device=dev)
+    x = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
     diags = synth.uniform_residues((32, 32, 112, N), mods[:112], seed, 2, device=dev)
     bk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 100 + i, device=dev) for i in range(31)]
     gk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 200 + i, device=dev) for i in range(31)]
-    y = torch.empty((8, 2, 111, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(7, 8, 32032), dtype=torch.uint8, device=dev)
+    y = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(7, B, 32032), dtype=torch.uint8, device=dev)
     ms = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 3, stream)
-    out["bsgs_L112_32x32"] = ks_entry(8 * 62, ms, ks_work_bsgs(112, 8, 8, 8, 32, 32), hbm_peak,
+    out["bsgs_L112_32x32"] = ks_entry(B * 62, ms, ks_work_bsgs(112, 8, 8, B, 32, 32), hbm_peak,
                                       mm_peak, mac_peak)
     return out
 
@@ -547,20 +552,21 @@ def run_reference(args):
     }), flush=True)
 
 
-def run_ks_only():
+def run_ks_only(args):
     import torch
     dev = torch.device("cuda", 0)
     hbm_peak, _ = peaks()
     from rns_ckks_polynomial_b200 import Context, primes
     ctx = Context(primes(60), primes(61)[60:], 60)
     ipeak = intpipe_peaks(ctx)
-    print(json.dumps({"keyswitch": run_keyswitch(dev, hbm_peak, ipeak)}), flush=True)
+    print(json.dumps({"keyswitch": run_keyswitch(dev, hbm_peak, ipeak, args.ks_batch, args.ks_keys)}),
+          flush=True)
 
 
 def main():
     args = parse()
     if args.ks_only:
-        run_ks_only()
+        run_ks_only(args)
         return
     global SWEEP
     SWEEP = tuple(int(x) for x in args.sweep.split(","))

@@ -9,6 +9,9 @@
 // 16 coefficients it stages the y bytes in shared memory, one thread issues the 64 plane pairs x 1 or
 // 2 K-steps of 32 sources as tcgen05.mma into 15 accumulators (240 TMEM columns), and the four warps
 // read their 32 TMEM lanes back, rebuild the exact 128-bit sum and reduce it once mod q_t.
+// 256 threads: every thread stages 4 sources of one coefficient per tile, with the next tile's loads
+// issued before the wait for the current tile's products; warps w and w + 4 share TMEM lane quadrant
+// w and split its 16 columns in the epilogue.
 //
 // Operand layout in shared memory: K-major, no swizzle, 8-row x 16-byte core matrices; the K-direction
 // core-matrix stride (LBO) is 128 bytes and the 8-row-group stride (SBO) 512 bytes, for a K extent of
@@ -159,8 +162,22 @@ struct TcJobs {
     }
 };
 
-__global__ void __launch_bounds__(128, 2) conv_tc_kernel(TcJobs jobs, const PrimeConst *__restrict__ pc,
-                                                          int *err)
+constexpr int kThreads = 256;
+
+// Byte planes of 4 sources (s0 .. s0+3) of one coefficient into every B plane.
+__device__ __forceinline__ void stage4(uint8_t *bplanes, const u64 *vals, int n, int s0)
+{
+#pragma unroll
+    for (int v = 0; v < kPlanes; ++v) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w |= (uint32_t)((vals[i] >> (8 * v)) & 0xff) << (8 * i);
+        *reinterpret_cast<uint32_t *>(bplanes + v * kBPlane + cm_off(n, s0)) = w;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) conv_tc_kernel(TcJobs jobs, const PrimeConst *__restrict__ pc,
+                                                               int *err)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, tb = blockIdx.x, z = blockIdx.y;
@@ -174,7 +191,7 @@ __global__ void __launch_bounds__(128, 2) conv_tc_kernel(TcJobs jobs, const Prim
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(abase + (size_t)tb * kPlanes * kAPlane);
         uint4 *dst = reinterpret_cast<uint4 *>(sm);
-        for (int i = tid; i < kPlanes * kAPlane / 16; i += 128) dst[i] = src[i];
+        for (int i = tid; i < kPlanes * kAPlane / 16; i += kThreads) dst[i] = src[i];
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -185,6 +202,12 @@ __global__ void __launch_bounds__(128, 2) conv_tc_kernel(TcJobs jobs, const Prim
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(smem_u32(bar)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    // staging task of this thread: coefficient n of the tile, sources s0 .. s0+3
+    const int n = tid & 15, s0 = (tid >> 4) * 4;
+    const u64 *ysrc = ybase + (size_t)s0 * kN + n;
+    u64 pre[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pre[i] = s0 + i < S ? __ldg(ysrc + (size_t)i * kN) : 0;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -192,32 +215,18 @@ __global__ void __launch_bounds__(128, 2) conv_tc_kernel(TcJobs jobs, const Prim
     const uint32_t tmem = *tslot;
     const u64 adesc0 = smem_desc(smem_u32(sm)), bdesc0 = smem_desc(smem_u32(sm + kSmemB));
     const bool two_k = S > 32;
-    const int ti = tb * kTM + tid;
+    const int quad = warp & 3, row = quad * 32 + (tid & 31);
+    const int ti = tb * kTM + row;
     const bool valid = ti < T;
     const int t = valid ? jobs.prime(ti, lo, S) : 0;
     const PrimeConst p = pc[t];
     u64 *row_out = jobs.row(z, t);
-    // staging task of this thread: coefficient n of the tile, sources s0 .. s0+7
-    const int n = tid & 15, s0 = (tid >> 4) * 8;
-    const u64 *ysrc = ybase + (size_t)s0 * kN + n;
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
+    const bool high_cols = warp >= 4;
     uint32_t parity = 0;
     bool ok = true;
     for (int c0 = 0; c0 < kN && ok; c0 += kTN) {
-        {
-            uint32_t w[kPlanes][2];
-#pragma unroll
-            for (int v = 0; v < kPlanes; ++v) w[v][0] = w[v][1] = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const u64 val = s0 + i < S ? __ldg(ysrc + (size_t)i * kN + c0) : 0;
-#pragma unroll
-                for (int v = 0; v < kPlanes; ++v) w[v][i >> 2] |= (uint32_t)((val >> (8 * v)) & 0xff) << (8 * (i & 3));
-            }
-#pragma unroll
-            for (int v = 0; v < kPlanes; ++v)
-                *reinterpret_cast<uint2 *>(sm + kSmemB + v * kBPlane + cm_off(n, s0)) = make_uint2(w[v][0], w[v][1]);
-        }
+        stage4(sm + kSmemB, pre, n, s0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
         if (tid == 0) {
@@ -235,15 +244,23 @@ __global__ void __launch_bounds__(128, 2) conv_tc_kernel(TcJobs jobs, const Prim
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          :: "r"(smem_u32(bar)) : "memory");
         }
+        // next tile's sources, in flight while the products are formed
+        if (c0 + kTN < kN) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pre[i] = s0 + i < S ? __ldg(ysrc + (size_t)i * kN + c0 + kTN) : 0;
+        }
         ok = mbar_wait(smem_u32(bar), parity);
         parity ^= 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (ok) {
             u64 *o = row_out + c0;
-            epilogue4<0>(taddr, o, p, valid);
-            epilogue4<1>(taddr, o, p, valid);
-            epilogue4<2>(taddr, o, p, valid);
-            epilogue4<3>(taddr, o, p, valid);
+            if (high_cols) {
+                epilogue4<2>(taddr, o, p, valid);
+                epilogue4<3>(taddr, o, p, valid);
+            } else {
+                epilogue4<0>(taddr, o, p, valid);
+                epilogue4<1>(taddr, o, p, valid);
+            }
         } else if (tid == 0) {
             atomicExch(err, 1);
         }
@@ -335,7 +352,7 @@ int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch,
     const Tables &T = ctx->t;
     TcJobs j{0, y, digits, T.tc_up, T.L, T.LK, T.alpha, T.dnum, T.K, T.tc_tb_per_digit};
     dim3 grid(T.tc_tb_per_digit, batch * T.dnum);
-    conv_tc_kernel<<<grid, 128, kSmemBytes, s>>>(j, T.pc, ctx->tc_err);
+    conv_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(j, T.pc, ctx->tc_err);
     CKKS_CHECK_LAUNCH("conv_tc_kernel");
     return CKKS_OK;
 }
@@ -345,7 +362,7 @@ int launch_conv_tc_down(const ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2
     const Tables &T = ctx->t;
     TcJobs j{1, zsrc, cv, T.tc_dn, T.L, T.LK, T.alpha, T.dnum, T.K, 0};
     dim3 grid((T.L + kTM - 1) / kTM, jobs2);
-    conv_tc_kernel<<<grid, 128, kSmemBytes, s>>>(j, T.pc, ctx->tc_err);
+    conv_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(j, T.pc, ctx->tc_err);
     CKKS_CHECK_LAUNCH("conv_tc_kernel");
     return CKKS_OK;
 }
