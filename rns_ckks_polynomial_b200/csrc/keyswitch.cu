@@ -130,26 +130,42 @@ struct UpInttJob {
     const ulonglong2 *hatinv;
     const PrimeConst *pc;
     int L, LK, alpha, dnum, batch, count;
-    __device__ __forceinline__ int prime(int j) const { return j / batch; }
-    __device__ __forceinline__ void load4(int j, int e, u64 *v) const
+    struct Ref {
+        const u64 *src, *src2;
+        u64 *copy, *yrow;
+        ulonglong2 h;
+        u64 q;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
     {
         const int i = j / batch, b = j - i * batch;
-        const size_t off = (size_t)b * in_bstride + (size_t)i * kN + e;
-        ld4(in + off, v);
+        const size_t off = (size_t)b * in_bstride + (size_t)i * kN;
+        Ref r;
+        r.src = in + off;
+        r.src2 = kProduct ? in2 + off : nullptr;
+        r.copy = digits + (((size_t)b * dnum + i / alpha) * LK + i) * kN;
+        r.yrow = y + ((size_t)b * L + i) * kN;
+        r.h = hatinv[i];
+        r.q = pc[i].q;
+        r.prime = i;
+        return r;
+    }
+    __device__ __forceinline__ void load4(const Ref &r, int e, u64 *v) const
+    {
+        ld4(r.src + e, v);
         if (kProduct) {
             u64 w[4];
-            ld4(in2 + off, w);
-            const PrimeConst c = pc[i];
+            ld4(r.src2 + e, w);
+            const PrimeConst c = pc[r.prime];
 #pragma unroll
             for (int k = 0; k < 4; ++k) v[k] = mulmod(v[k], w[k], c);
         }
-        st4(digits + (((size_t)b * dnum + i / alpha) * LK + i) * kN + e, v);
+        st4(r.copy + e, v);
     }
-    __device__ __forceinline__ void store(int j, int e, u64 v) const
+    __device__ __forceinline__ void store(const Ref &r, int e, u64 v) const
     {
-        const int i = j / batch, b = j - i * batch;
-        const ulonglong2 h = hatinv[i];
-        y[((size_t)b * L + i) * kN + e] = shoup(v, h.x, h.y, pc[i].q);
+        r.yrow[e] = shoup(v, r.h.x, r.h.y, r.q);
     }
 };
 
@@ -159,7 +175,11 @@ struct UpInttJob {
 struct UpNttJob {
     u64 *digits;
     int L, LK, alpha, dnum, batch, count;
-    __device__ __forceinline__ u64 *row(int j, int *tp) const
+    struct Ref {
+        u64 *row;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
     {
         const int b = j % batch;
         int r = j / batch, t, jd;
@@ -173,25 +193,10 @@ struct UpNttJob {
             t = L + r / dnum;
             jd = r - (t - L) * dnum;
         }
-        *tp = t;
-        return digits + (((size_t)b * dnum + jd) * LK + t) * kN;
+        return {digits + (((size_t)b * dnum + jd) * LK + t) * kN, t};
     }
-    __device__ __forceinline__ int prime(int j) const
-    {
-        int t;
-        row(j, &t);
-        return t;
-    }
-    __device__ __forceinline__ u64 load(int j, int e) const
-    {
-        int t;
-        return row(j, &t)[e];
-    }
-    __device__ __forceinline__ void store4(int j, int e, const u64 *v) const
-    {
-        int t;
-        st4(row(j, &t) + e, v);
-    }
+    __device__ __forceinline__ u64 load(const Ref &r, int e) const { return r.row[e]; }
+    __device__ __forceinline__ void store4(const Ref &r, int e, const u64 *v) const { st4(r.row + e, v); }
 };
 
 size_t modup_ws_bytes(const ckks_ctx *ctx, int batch) { return limbs_bytes((size_t)batch * ctx->L); }
@@ -281,17 +286,23 @@ struct DownInttJob {
     const ulonglong2 *hatinv;
     const PrimeConst *pc;
     int L, K, LK, jobs2, count;
-    __device__ __forceinline__ int prime(int j) const { return L + j / jobs2; }
-    __device__ __forceinline__ void load4(int j, int e, u64 *v) const
+    struct Ref {
+        const u64 *src;
+        u64 *dst;
+        ulonglong2 h;
+        u64 q;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
     {
         const int k = j / jobs2, zz = j - k * jobs2;
-        ld4(acc + ((size_t)zz * LK + L + k) * kN + e, v);
+        return {acc + ((size_t)zz * LK + L + k) * kN, zdst + ((size_t)zz * K + k) * kN, hatinv[k],
+                pc[L + k].q, L + k};
     }
-    __device__ __forceinline__ void store(int j, int e, u64 v) const
+    __device__ __forceinline__ void load4(const Ref &r, int e, u64 *v) const { ld4(r.src + e, v); }
+    __device__ __forceinline__ void store(const Ref &r, int e, u64 v) const
     {
-        const int k = j / jobs2, zz = j - k * jobs2;
-        const ulonglong2 h = hatinv[k];
-        zdst[((size_t)zz * K + k) * kN + e] = shoup(v, h.x, h.y, pc[L + k].q);
+        r.dst[e] = shoup(v, r.h.x, r.h.y, r.q);
     }
 };
 
@@ -304,41 +315,65 @@ struct DownFinalJob {
     const PrimeConst *pc;
     int L, LK, jobs2, count;
     DownExtra ex;
-    __device__ __forceinline__ int prime(int j) const { return j / jobs2; }
-    __device__ __forceinline__ u64 load(int j, int e) const
+    struct Ref {
+        const u64 *cv, *acc, *c0, *a, *b;
+        u64 *out;
+        ulonglong2 pv;
+        u64 q;
+        u32 g;
+        int prime, comp;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
     {
         const int i = j / jobs2, zz = j - i * jobs2;
-        return cv[((size_t)zz * L + i) * kN + e];
-    }
-    __device__ __forceinline__ void store4(int j, int e, const u64 *v) const
-    {
-        const int i = j / jobs2, zz = j - i * jobs2;
-        const int z = zz >> 1, comp = zz & 1;
-        const u64 q = pc[i].q;
-        const ulonglong2 pv = pinv[i];
-        u64 a[4], o[4];
-        ld4(acc + ((size_t)zz * LK + i) * kN + e, a);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) o[c] = shoup(submod(a[c], v[c], q), pv.x, pv.y, q);
-        if (kKind == 1 && comp == 0) {
+        const int z = zz >> 1;
+        Ref r;
+        r.cv = cv + ((size_t)zz * L + i) * kN;
+        r.acc = acc + ((size_t)zz * LK + i) * kN;
+        r.out = out + ((size_t)zz * L + i) * kN;
+        r.pv = pinv[i];
+        r.q = pc[i].q;
+        r.prime = i;
+        r.comp = zz & 1;
+        r.c0 = nullptr;
+        r.a = r.b = nullptr;
+        r.g = 1;
+        if (kKind == 1) {
             const int ci = ex.ct_mod ? z % ex.ct_mod : z;
-            const u64 *c0 = ex.ct + (size_t)ci * ex.ct_bstride + (size_t)i * kN;
-            const u32 g = ex.gal[z / ex.per];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) o[c] = addmod(o[c], __ldg(c0 + galois_src((u32)(e + c), g)), q);
+            r.c0 = ex.ct + (size_t)ci * ex.ct_bstride + (size_t)i * kN;
+            r.g = ex.gal[z / ex.per];
         }
         if (kKind == 2) {
-            const PrimeConst pcc = pc[i];
-            const size_t base = (size_t)z * 2 * L * kN + (size_t)i * kN + e, Ln = (size_t)L * kN;
+            const size_t base = (size_t)z * 2 * L * kN + (size_t)i * kN;
+            r.a = ex.a + base;
+            r.b = ex.b + base;
+        }
+        return r;
+    }
+    __device__ __forceinline__ u64 load(const Ref &r, int e) const { return r.cv[e]; }
+    __device__ __forceinline__ void store4(const Ref &r, int e, const u64 *v) const
+    {
+        const u64 q = r.q;
+        u64 a[4], o[4];
+        ld4(r.acc + e, a);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = shoup(submod(a[c], v[c], q), r.pv.x, r.pv.y, q);
+        if (kKind == 1 && r.comp == 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[c] = addmod(o[c], __ldg(r.c0 + galois_src((u32)(e + c), r.g)), q);
+        }
+        if (kKind == 2) {
+            const PrimeConst pcc = pc[r.prime];
+            const size_t Ln = (size_t)L * kN;
             u64 a0[4], b0[4], a1[4], b1[4];
-            ld4(ex.a + base, a0);
-            ld4(ex.b + base, b0);
-            if (comp == 0) {
+            ld4(r.a + e, a0);
+            ld4(r.b + e, b0);
+            if (r.comp == 0) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) o[c] = addmod(o[c], mulmod(a0[c], b0[c], pcc), q);
             } else {
-                ld4(ex.a + base + Ln, a1);
-                ld4(ex.b + base + Ln, b1);
+                ld4(r.a + Ln + e, a1);
+                ld4(r.b + Ln + e, b1);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     u64 hi = 0, lo = 0;
@@ -348,7 +383,7 @@ struct DownFinalJob {
                 }
             }
         }
-        st4(out + ((size_t)zz * L + i) * kN + e, o);
+        st4(r.out + e, o);
     }
 };
 

@@ -86,12 +86,17 @@ struct RescInttJob {
     const u64 *ct;
     u64 *w;
     int lp1, count;
-    __device__ __forceinline__ int prime(int) const { return lp1 - 1; }
-    __device__ __forceinline__ void load4(int j, int e, u64 *v) const
+    struct Ref {
+        const u64 *src;
+        u64 *dst;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
     {
-        ld4(ct + ((size_t)j * lp1 + lp1 - 1) * kN + e, v);
+        return {ct + ((size_t)j * lp1 + lp1 - 1) * kN, w + (size_t)j * kN, lp1 - 1};
     }
-    __device__ __forceinline__ void store(int j, int e, u64 v) const { w[(size_t)j * kN + e] = v; }
+    __device__ __forceinline__ void load4(const Ref &r, int e, u64 *v) const { ld4(r.src + e, v); }
+    __device__ __forceinline__ void store(const Ref &r, int e, u64 v) const { r.dst[e] = v; }
 };
 
 // Forward NTT of [w]_{q_i} for every kept limb i; the store forms
@@ -102,24 +107,31 @@ struct RescFwdJob {
     const ulonglong2 *qinv;
     const PrimeConst *pc;
     int lp1, jobs2, count;
-    __device__ __forceinline__ int prime(int j) const { return j / jobs2; }
-    __device__ __forceinline__ u64 load(int j, int e) const
+    struct Ref {
+        const u64 *w, *ct;
+        u64 *out;
+        ulonglong2 qi;
+        u64 q, mu;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
     {
         const int i = j / jobs2, zz = j - i * jobs2;
-        const u64 v = w[(size_t)zz * kN + e];
-        const PrimeConst &c = pc[i];
-        return v - mulhi(v, c.mu64) * c.q;  // [0, 2 q_i)
+        return {w + (size_t)zz * kN, ct + ((size_t)zz * lp1 + i) * kN, out + ((size_t)zz * (lp1 - 1) + i) * kN,
+                qinv[i], pc[i].q, pc[i].mu64, i};
     }
-    __device__ __forceinline__ void store4(int j, int e, const u64 *v) const
+    __device__ __forceinline__ u64 load(const Ref &r, int e) const
     {
-        const int i = j / jobs2, zz = j - i * jobs2;
-        const u64 q = pc[i].q;
-        const ulonglong2 qi = qinv[i];
+        const u64 v = r.w[e];
+        return v - mulhi(v, r.mu) * r.q;  // [0, 2 q_i)
+    }
+    __device__ __forceinline__ void store4(const Ref &r, int e, const u64 *v) const
+    {
         u64 c[4], o[4];
-        ld4(ct + ((size_t)zz * lp1 + i) * kN + e, c);
+        ld4(r.ct + e, c);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) o[k] = shoup(submod(c[k], v[k], q), qi.x, qi.y, q);
-        st4(out + ((size_t)zz * (lp1 - 1) + i) * kN + e, o);
+        for (int k = 0; k < 4; ++k) o[k] = shoup(submod(c[k], v[k], r.q), r.qi.x, r.qi.y, r.q);
+        st4(r.out + e, o);
     }
 };
 
