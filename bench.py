@@ -383,6 +383,13 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
     out["boot_rotation_L2100"] = ks_entry(B * R, ms, ks_work_rotation(2100, 60, 60, B, R), hbm_peak,
                                           mm_peak, mac_peak, conv_macs=conv, tensor=True)
     ctx.device_status()
+    # the same call with both conversions on the integer pipes (bit-identical output)
+    ctx.set_conversion("integer")
+    ms = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 2, stream)
+    out["boot_rotation_L2100_integer_pipes"] = ks_entry(B * R, ms, ks_work_rotation(2100, 60, 60, B, R),
+                                                        hbm_peak, mm_peak, mac_peak)
+    ctx.set_conversion("auto")
+    ctx.device_status()
     del ct, keys, res, ws, ctx
     torch.cuda.empty_cache()
     # layer ct x ct multiply: L = 112, K = 8, alpha = 8, 8 pairs

@@ -112,6 +112,23 @@ const char *ckks_last_error(void);
  * asynchronous CUDA error on the device. */
 int ckks_device_status(const ckks_ctx *ctx);
 
+/* Where the basis conversions of ModUp and ModDown run.  The conversion is
+ * the exact product out_t = sum_s y_s [Q_j/q_s]_t (mod t), the step named
+ * "RNS basis conversion" in the Kestrel engine write-up, section 3 table.
+ *  CKKS_CONV_AUTO     int8 tensor cores when the conversion has more than 16
+ *                     source primes (ModUp: alpha; ModDown: K), the integer
+ *                     pipes otherwise (the default);
+ *  CKKS_CONV_INTEGER  always the integer pipes (64x64->128-bit multiply-adds);
+ *  CKKS_CONV_TENSOR   always the int8 tensor cores (byte-plane products).
+ * Every engine computes the same exact sum before the one final reduction, so
+ * results are bit-identical; this is a performance switch only.  The pages
+ * have no counterpart (their engine runs on CPU threads).  Takes effect for
+ * calls issued after it returns; do not change it while another host thread
+ * issues calls on the same context.  CKKS_EINVAL for a null context or an
+ * unknown engine. */
+enum { CKKS_CONV_AUTO = 0, CKKS_CONV_INTEGER = 1, CKKS_CONV_TENSOR = 2 };
+int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine);
+
 /* Context parameters: writes L, K, alpha, dnum, n (any pointer may be NULL). */
 int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n);
 

@@ -77,6 +77,15 @@ class Context:
         """Synchronise the device and raise if a bounded device wait expired."""
         check("ckks_device_status", lib().ckks_device_status(self._h))
 
+    CONVERSION = {"auto": 0, "integer": 1, "tensor": 2}
+
+    def set_conversion(self, engine):
+        """Where ModUp/ModDown basis conversions run: "auto", "integer" (integer
+        pipes) or "tensor" (int8 tensor cores).  Results are bit-identical."""
+        check("ckks_ctx_set_conversion",
+              lib().ckks_ctx_set_conversion(self._h, self.CONVERSION.get(engine, -1)
+                                            if isinstance(engine, str) else int(engine)))
+
     # ------------------------------------------------------------ helpers
     def _empty(self, *shape):
         return torch.empty(shape, dtype=torch.int64, device=self.device)

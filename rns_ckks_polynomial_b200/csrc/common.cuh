@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <string>
@@ -67,6 +68,7 @@ struct ckks_ctx {
     void *own_ws = nullptr;
     size_t own_ws_bytes = 0;
     int *tc_err = nullptr;  // device flag: a bounded wait of the tensor-core kernel expired
+    std::atomic<int> conv_engine{CKKS_CONV_AUTO};
 };
 
 namespace ckks {

@@ -291,7 +291,14 @@ void build_planes(std::vector<uint8_t> &dst, size_t base, int T, int S, F at)
 
 }  // namespace
 
-bool tc_wanted(int sources) { return sources > kTcMinSources; }
+bool conv_on_tensor(const ckks_ctx *ctx, int sources)
+{
+    switch (ctx->conv_engine.load(std::memory_order_relaxed)) {
+    case CKKS_CONV_INTEGER: return false;
+    case CKKS_CONV_TENSOR: return true;
+    default: return sources > kTcMinSources;
+    }
+}
 
 int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::vector<u64> &dn_mat)
 {
@@ -300,7 +307,7 @@ int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::ve
     T.tc_up = nullptr;
     T.tc_dn = nullptr;
     T.tc_tb_per_digit = (LK - 1 + kTM - 1) / kTM;
-    if (tc_wanted(alpha)) {
+    {
         const size_t per_digit = (size_t)T.tc_tb_per_digit * kPlanes * kAPlane;
         std::vector<uint8_t> h(per_digit * dnum, 0);
         for (int j = 0; j < dnum; ++j) {
@@ -320,7 +327,7 @@ int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::ve
         if (e != cudaSuccess) return cuda_status(e, "cudaMemcpy(tensor-core tables)");
         T.tc_up = static_cast<const uint8_t *>(d);
     }
-    if (tc_wanted(K)) {
+    {
         const size_t bytes = (size_t)((L + kTM - 1) / kTM) * kPlanes * kAPlane;
         std::vector<uint8_t> h(bytes, 0);
         build_planes(h, 0, L, K, [&](int ti, int s) { return dn_mat[(size_t)s * L + ti]; });

@@ -422,6 +422,15 @@ extern "C" int ckks_device_status(const ckks_ctx *ctx)
     return CKKS_OK;
 }
 
+extern "C" int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine)
+{
+    CKKS_TRY(check_ctx(ctx));
+    if (engine != CKKS_CONV_AUTO && engine != CKKS_CONV_INTEGER && engine != CKKS_CONV_TENSOR)
+        return set_error(CKKS_EINVAL, "unknown conversion engine");
+    ctx->conv_engine.store(engine, std::memory_order_relaxed);
+    return CKKS_OK;
+}
+
 extern "C" int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n)
 {
     CKKS_TRY(check_ctx(ctx));

@@ -217,7 +217,7 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
                            T.L, T.LK, T.alpha, T.dnum, batch, T.L * batch};
         CKKS_TRY(launch_ntt_inv(j, T, s));
     }
-    if (T.tc_up) {
+    if (conv_on_tensor(ctx, T.alpha)) {
         CKKS_TRY(launch_conv_tc_up(ctx, y, digits, batch, s));
     } else {
         UpConvMap m{y, digits, T.up_mat, T.L, T.LK, T.alpha, T.dnum};
@@ -403,7 +403,7 @@ int moddown_stage(const ckks_ctx *ctx, const u64 *acc, u64 *out, int jobs, const
     u64 *cvb = c.take<u64>((size_t)jobs2 * T.L * kN);
     DownInttJob ij{acc, zb, T.dn_hatinv, T.pc, T.L, T.K, T.LK, jobs2, T.K * jobs2};
     CKKS_TRY(launch_ntt_inv(ij, T, s));
-    if (T.tc_dn) {
+    if (conv_on_tensor(ctx, T.K)) {
         CKKS_TRY(launch_conv_tc_down(ctx, zb, cvb, jobs2, s));
     } else {
         DownConvMap m{zb, cvb, T.dn_mat, T.L, T.K};

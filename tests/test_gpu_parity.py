@@ -148,25 +148,41 @@ def test_automorph_rejects_even_and_in_place():
 @pytest.mark.parametrize("L,K,alpha", [(4, 1, 1), (6, 2, 2), (5, 2, 2), (112, 8, 8), (20, 3, 7),
                                        (40, 20, 20), (70, 33, 33), (130, 64, 64)])
 def test_modup_inner_moddown_stages(orc, L, K, alpha):
-    """Digits / special bases above 16 primes run the int8 tensor-core
-    conversion; (70, 33, 33) has a ragged 4-prime last digit."""
+    """Every stage on every conversion engine (integer pipes, int8 tensor cores,
+    and the automatic choice, which takes the tensor cores above 16 source
+    primes); (70, 33, 33) has a ragged 4-prime last digit."""
     p = Params(L, K, alpha)
     ctx = ctx_for(p)
     mods = np.array(ctx.mods, dtype=np.uint64)
     c = _res((2, L, N), mods[:L], 50)
-    dig = ctx.modup(dev(c))
-    want_d = orc.modup(c, mods, L, K, alpha)
-    assert_bits_equal(host(dig), want_d, "modup")
     key = _res((p.dnum, 2, L + K, N), mods, 51)
-    for g in (1, 5, 4095):
-        acc = ctx.key_inner(dig, dev(key), g)
-        want_a = orc.key_inner(want_d, key, g, mods, L, K, alpha)
-        assert_bits_equal(host(acc), want_a, "key_inner g=%d" % g)
-    out = ctx.moddown(acc)
-    assert_bits_equal(host(out), orc.moddown(want_a, mods, L, K), "moddown")
-    ks = ctx.keyswitch(dev(c), dev(key))
-    assert_bits_equal(host(ks), orc.keyswitch(c, key, mods, L, K, alpha), "keyswitch")
-    ctx.device_status()
+    want_d = orc.modup(c, mods, L, K, alpha)
+    want_a = {g: orc.key_inner(want_d, key, g, mods, L, K, alpha) for g in (1, 5, 4095)}
+    want_m = orc.moddown(want_a[4095], mods, L, K)
+    want_k = orc.keyswitch(c, key, mods, L, K, alpha)
+    try:
+        for engine in ("integer", "tensor", "auto"):
+            ctx.set_conversion(engine)
+            dig = ctx.modup(dev(c))
+            assert_bits_equal(host(dig), want_d, "modup (%s)" % engine)
+            for g in (1, 5, 4095):
+                acc = ctx.key_inner(dig, dev(key), g)
+                assert_bits_equal(host(acc), want_a[g], "key_inner g=%d" % g)
+            out = ctx.moddown(acc)
+            assert_bits_equal(host(out), want_m, "moddown (%s)" % engine)
+            ks = ctx.keyswitch(dev(c), dev(key))
+            assert_bits_equal(host(ks), want_k, "keyswitch (%s)" % engine)
+            ctx.device_status()
+    finally:
+        ctx.set_conversion("auto")
+
+
+def test_set_conversion_rejects_unknown_engine():
+    ctx = ctx_for(Params(4, 1, 1))
+    with pytest.raises(CkksError):
+        ctx.set_conversion(7)
+    with pytest.raises(CkksError):
+        ctx.set_conversion("fast")
 
 
 def test_hoisted_rotations_match_and_decrypt(orc):
@@ -347,3 +363,11 @@ def test_config5_boot_rotation_full_size_sampled(orc):
     want = orc.rotate(host(ct[3:4]), [host(keys[2])], np.array([gal[2]], dtype=np.uint64), mods,
                       2100, 60, 60)
     assert_bits_equal(got, want[0, 0], "config 5 ct 3 key 2")
+    # the integer-pipe conversion gives the same words for all 32 key switches
+    try:
+        ctx.set_conversion("integer")
+        out_int = ctx.rotate(ct, keys, gal)
+        ctx.device_status()
+    finally:
+        ctx.set_conversion("auto")
+    assert torch.equal(out_int, out)
