@@ -47,11 +47,12 @@ struct Tables {
     const ulonglong2 *dn_hatinv;  // [K]: {[(P/p_k)^-1]_{p_k}, Shoup}
     const u64 *dn_mat;            // [K][L]: [P/p_k]_{q_i}
     const ulonglong2 *dn_pinv;    // [L]: {[P^-1]_{q_i}, Shoup}
-    // Byte planes of the conversion matrices for the int8 tensor-core path (null when the digit /
-    // special basis is small enough for the CUDA-core kernel)
-    const uint8_t *tc_up;         // [dnum][tb_per_digit][8][128 x 64]
-    const uint8_t *tc_dn;         // [ceil(L/128)][8][128 x 64]
+    // Byte planes of the conversion matrices for the int8 tensor-core path: per target row its
+    // 8 planes of 64 source bytes, targets in blocks of 128
+    const uint8_t *tc_up;         // [dnum][tb_per_digit][128][8][64]
+    const uint8_t *tc_dn;         // [ceil(L/128)][128][8][64]
     int tc_tb_per_digit;
+    bool tc_special;              // every prime is 2^60 - delta with delta < 2^28
 };
 
 }  // namespace ckks
