@@ -228,42 +228,61 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 }
 
 // ---------------------------------------------------------------- key inner product
-// One thread per output coefficient k of one (prime t, key r, ciphertext b)
-// job.  The 1-D grid is ordered coefficient tile fastest, then ciphertext,
-// then key, then prime, so the CTAs that read the same key rows (all
-// ciphertexts of one key at one prime) run back to back: a key row crosses
-// HBM once and is re-served from L2, and the gathered digit row of one job is
-// shared by its eight coefficient-tile CTAs through L1/L2.  The Galois
-// permutation is the gather on the digit load.
-__global__ void __launch_bounds__(256) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
+// One thread per output coefficient k of one (prime t, key r) pair and a chunk of up to kKiB
+// ciphertexts b: per digit j it loads the two key words once and the chunk's gathered digit words,
+// and keeps 2 kKiB exact 128-bit sums.  The 1-D grid is ordered coefficient tile fastest, then key,
+// then ciphertext chunk, then prime, so the CTAs that read the same digit rows (all keys of one
+// chunk at one prime) run back to back and re-read them from L2.  The Galois permutation is the
+// gather on the digit load (it maps each aligned tile of 32 coefficients onto one, so a warp's
+// gathered loads stay within one 256-byte segment).
+constexpr int kKiB = 4;       // ciphertexts per thread
+constexpr int kKiThreads = 128;
+
+__global__ void __launch_bounds__(kKiThreads, 4) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
                                                         int per_key, int nkeys, int hoisted,
                                                         u64 *__restrict__ acc, Tables T)
 {
+    const int nchunks = (per_key + kKiB - 1) / kKiB;
     int id = blockIdx.x;
-    const int tile = id % (kN / 256);
-    id /= kN / 256;
-    const int b = id % per_key;
-    id /= per_key;
+    const int tile = id % (kN / kKiThreads);
+    id /= kN / kKiThreads;
     const int r = id % nkeys;
-    const int t = id / nkeys;
-    const int k = tile * 256 + threadIdx.x;
-    const int z = r * per_key + b;
-    const int dset = hoisted ? b : z;
+    id /= nkeys;
+    const int chunk = id % nchunks;
+    const int t = id / nchunks;
+    const int b0 = chunk * kKiB, nb = min(kKiB, per_key - b0);
+    const int k = tile * kKiThreads + threadIdx.x;
     const u32 g = kl.galois[r];
     const int src = g == 1u ? k : (int)galois_src((u32)k, g);
     const size_t LKn = (size_t)T.LK * kN;
-    const u64 *dg = digits + (size_t)dset * T.dnum * LKn + (size_t)t * kN + src;
+    const size_t bstride = (size_t)T.dnum * LKn;  // between the digit sets of consecutive ciphertexts
+    const u64 *dg = digits + (size_t)(hoisted ? b0 : r * per_key + b0) * bstride + (size_t)t * kN + src;
     const u64 *kp = kl.key[r] + (size_t)t * kN + k;
-    u64 h0 = 0, l0 = 0, h1 = 0, l1 = 0;
+    u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
+#pragma unroll
+    for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
+#pragma unroll 2
     for (int j = 0; j < T.dnum; ++j) {
-        const u64 d = __ldg(dg + (size_t)j * LKn);
-        mac128(h0, l0, d, __ldg(kp + (size_t)(2 * j) * LKn));
-        mac128(h1, l1, d, __ldg(kp + (size_t)(2 * j + 1) * LKn));
+        const u64 kb = __ldg(kp + (size_t)(2 * j) * LKn), ka = __ldg(kp + (size_t)(2 * j + 1) * LKn);
+        const u64 *dj = dg + (size_t)j * LKn;
+        u64 d[kKiB];
+#pragma unroll
+        for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
+#pragma unroll
+        for (int b = 0; b < kKiB; ++b) {
+            mac128(h0[b], l0[b], d[b], kb);
+            mac128(h1[b], l1[b], d[b], ka);
+        }
     }
     const PrimeConst pc = T.pc[t];
-    u64 *o = acc + ((size_t)z * 2 * T.LK + t) * kN + k;
-    o[0] = reduce128(h0, l0, pc);
-    o[LKn] = reduce128(h1, l1, pc);
+#pragma unroll
+    for (int b = 0; b < kKiB; ++b) {
+        if (b < nb) {
+            u64 *o = acc + ((size_t)(r * per_key + b0 + b) * 2 * T.LK + t) * kN + k;
+            o[0] = reduce128(h0[b], l0[b], pc);
+            o[LKn] = reduce128(h1[b], l1[b], pc);
+        }
+    }
 }
 
 int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, int per_key,
@@ -272,9 +291,9 @@ int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, i
     if (jobs <= 0) return CKKS_OK;
     const Tables &T = ctx->t;
     const int nkeys = jobs / per_key;
-    const size_t blocks = (size_t)(kN / 256) * jobs * T.LK;
+    const size_t blocks = (size_t)(kN / kKiThreads) * nkeys * ((per_key + kKiB - 1) / kKiB) * T.LK;
     if (blocks > 0x7fffffffull) return set_error(CKKS_EUNSUPPORTED, "key inner product grid too large");
-    key_inner_kernel<<<(unsigned)blocks, 256, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T);
+    key_inner_kernel<<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T);
     CKKS_CHECK_LAUNCH("key_inner_kernel");
     return CKKS_OK;
 }
