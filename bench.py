@@ -176,30 +176,36 @@ def ntt_launch_work(limbs, batch=BATCH):
 
 
 def traffic_for(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    source is unchanged since the capture."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    sources are unchanged since the capture (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    e = d.get(kernel_key)
+    e = json.load(open(p)).get(kernel_key)
     if not e:
         return None
-    src = os.path.join(ROOT, e["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if h != e.get("source_sha256_16"):
+    blob = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in e["sources"])
+    if hashlib.sha256(blob).hexdigest()[:16] != e.get("sources_sha256_16"):
         return None
     return e["dram_bytes_per_launch"]
 
 
 def intpipe_peaks(ctx):
-    """Same-run integer-pipe microbenchmarks: Shoup multiplies/s and
-    64x64->128 MACs/s over the whole GPU."""
+    """Same-run microbenchmarks over the whole GPU: Shoup multiplies/s,
+    64x64->128 MACs/s and 64-bit high multiplies/s on the integer pipes, and
+    int8 tcgen05.mma ops/s at N = 256 (dense rate) and N = 32 (the basis
+    conversion's tile), one issuing thread per SM."""
     out = {}
     for kind, name in ((0, "shoup_mulmod_per_s"), (1, "mac128_per_s"), (2, "mulhi64_per_s")):
         best = 0.0
         for _ in range(3):
             ms, ops = ctx.bench_intpipe(kind, 148 * 8, 2048)
+            best = max(best, ops / (ms * 1e-3))
+        out[name] = best
+    for kind, name in ((3, "int8_mma_n256_ops_per_s"), (4, "int8_mma_n32_ops_per_s")):
+        best = 0.0
+        for _ in range(3):
+            ms, ops = ctx.bench_intpipe(kind, 148, 4096)
             best = max(best, ops / (ms * 1e-3))
         out[name] = best
     return out
@@ -381,7 +387,8 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
     up, _, down = ks_work_keyswitch_parts(2100, 60, 60)
     conv = B * (up["mac"] + R * down["mac"])
     out["boot_rotation_L2100"] = ks_entry(B * R, ms, ks_work_rotation(2100, 60, 60, B, R), hbm_peak,
-                                          mm_peak, mac_peak, conv_macs=conv, tensor=True)
+                                          mm_peak, mac_peak, conv_macs=conv,
+                                          int8_peak=int8_mac_peak(ipeak))
     ctx.device_status()
     # the same call with both conversions on the integer pipes (bit-identical output)
     ctx.set_conversion("integer")
@@ -466,19 +473,17 @@ def ks_work_bsgs(L, K, alpha, B, bb, gg):
     return mm, mac, keyb + io
 
 
-def int8_peak():
-    """Dense int8 MAC/s: the measured bf16 GEMM peak x the nominal int8/bf16 ratio (2)."""
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    tf = json.load(open(p))["bf16_tflops"] if os.path.exists(p) else 1590.0
-    return 2 * tf * 1e12 / 2  # ops/s -> MAC/s
+def int8_mac_peak(ipeak):
+    """Dense int8 MAC/s: the same-run tcgen05 int8 rate at N = 256."""
+    return ipeak["int8_mma_n256_ops_per_s"] / 2
 
 
-def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak, conv_macs=0, tensor=False):
+def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak, conv_macs=0, int8_peak=None):
     """roofline_frac follows the problem statement: modular multiplies and 64-bit MACs at the
     same-run integer-pipe peaks, bytes at the HBM peak.  When the basis conversion runs on the
     int8 tensor cores (digits above 16 primes) that model can be exceeded; tensor_model_frac then
     charges the conversion's int8 byte-plane products (64 per 60-bit MAC, sources padded to 64)
-    at the int8 peak instead."""
+    at the same-run int8 tensor-core peak (`int8_peak`, MAC/s) instead."""
     mm, mac, bytes_ = work
     t = ms * 1e-3
     t_alu = mm / mm_peak + mac / mac_peak
@@ -488,9 +493,9 @@ def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak, conv_macs=0, tensor=Fal
            "mulmods": mm, "macs": mac, "min_bytes": bytes_, "bound": bound,
            "roofline_frac": max(t_alu, t_hbm) / t,
            "alu_frac": t_alu / t, "hbm_frac": t_hbm / t,
-           "conversion": "int8 tensor cores" if tensor else "integer pipes"}
-    if tensor:
-        t_tc = mm / mm_peak + (mac - conv_macs) / mac_peak + conv_macs * 64 * 64 / 60 / int8_peak()
+           "conversion": "int8 tensor cores" if int8_peak else "integer pipes"}
+    if int8_peak:
+        t_tc = mm / mm_peak + (mac - conv_macs) / mac_peak + conv_macs * 64 * 64 / 60 / int8_peak
         out["tensor_model_frac"] = max(t_tc, t_hbm) / t
     return out
 

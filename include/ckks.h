@@ -282,7 +282,11 @@ int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *d
  * iterations in every thread of a grid of `blocks` x 256 threads and writes
  * the elapsed milliseconds (CUDA events) to *ms and the operation count to
  * *ops.  kind 0: 64-bit Shoup modular multiply; kind 1: 64x64->128
- * multiply-accumulate; kind 2: 64x64 high-half multiply.  Synchronous. */
+ * multiply-accumulate; kind 2: 64x64 high-half multiply.
+ * Tensor-pipe kinds (one issuing thread per CTA of 128 threads, `iters`
+ * back-to-back int8 tcgen05.mma of M = 128, K = 32; *ops counts 2 M N K per
+ * MMA): kind 3: N = 256 (the dense int8 rate); kind 4: N = 32 (the basis
+ * conversion's tile).  blocks <= 148 * 64.  Synchronous. */
 int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int iters, double *ms,
                        double *ops);
 

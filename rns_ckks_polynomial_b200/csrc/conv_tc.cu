@@ -443,6 +443,57 @@ int launch(const ckks_ctx *ctx, TcJobs j, int tbs, int jobs, cudaStream_t s)
     return CKKS_OK;
 }
 
+// ---------------------------------------------------------------- tensor-pipe microbenchmark
+// Back-to-back tcgen05.mma (kind::i8, M = 128, K = 32, both operands in shared memory) from one
+// thread per CTA, one CTA per SM: the fixed cost per MMA at a given N (the conversion's own tile is
+// N = 32) and the dense int8 rate (N = 256).  Operand values do not matter; the products accumulate
+// into one TMEM region.
+constexpr int kBenchSmem = kTM * kKP + 256 * kKP + 64;  // A 8 KiB, B up to 16 KiB, barrier, slot
+
+template <int N>
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, int *err)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kTM * kKP + 256 * kKP);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kTM * kKP + 256 * kKP + 8);
+    for (int i = threadIdx.x; i < (kTM + 256) * kKP / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t *>(sm)[i] = 0x01010101u;
+    if (threadIdx.x < 32) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tslot)), "r"(256));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = *tslot;
+    if (threadIdx.x == 0) {
+        constexpr uint32_t idesc = (2u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
+        const u64 ad = smem_desc(smem_u32(sm)), bd = smem_desc(smem_u32(sm + kTM * kKP));
+        for (int r = 0; r < iters; r += 8) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+                    :: "r"(tmem), "l"(ad + ((k & 1) * 256 >> 4)), "l"(bd + ((k & 1) * 256 >> 4)), "r"(idesc),
+                       "r"(k | r), "r"(0), "r"(0), "r"(0), "r"(0));
+        }
+        commit(bar);
+        if (!mbar_wait(bar, 0)) atomicExch(err, 1);
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (threadIdx.x < 32)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(256));
+}
+
 }  // namespace
 
 bool conv_on_tensor(const ckks_ctx *ctx, int sources)
@@ -509,6 +560,38 @@ int launch_conv_tc_down(const ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2
     const Tables &T = ctx->t;
     TcJobs j{1, zsrc, cv, T.tc_dn, T.L, T.LK, T.alpha, T.dnum, T.K, 0, 1};
     return launch(ctx, j, (T.L + kTM - 1) / kTM, jobs2, s);
+}
+
+int bench_mma(const ckks_ctx *ctx, int n, int blocks, int iters, double *ms, double *ops)
+{
+    iters = (iters + 7) / 8 * 8;
+    cudaError_t e = n == 32 ? cudaFuncSetAttribute(mma_rate_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kBenchSmem)
+                            : cudaFuncSetAttribute(mma_rate_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kBenchSmem);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(mma_rate_kernel)");
+    auto launch_n = [&](int it) {
+        if (n == 32)
+            mma_rate_kernel<32><<<blocks, 128, kBenchSmem>>>(it, ctx->tc_err);
+        else
+            mma_rate_kernel<256><<<blocks, 128, kBenchSmem>>>(it, ctx->tc_err);
+    };
+    cudaEvent_t a, b;
+    cudaEventCreate(&a);
+    cudaEventCreate(&b);
+    launch_n(8);  // warm-up
+    cudaEventRecord(a);
+    launch_n(iters);
+    cudaEventRecord(b);
+    e = cudaEventSynchronize(b);
+    float t = 0;
+    cudaEventElapsedTime(&t, a, b);
+    cudaEventDestroy(a);
+    cudaEventDestroy(b);
+    if (e != cudaSuccess) return cuda_status(e, "mma_rate_kernel");
+    *ms = t;
+    *ops = 2.0 * kTM * n * 32 * (double)blocks * iters;
+    return CKKS_OK;
 }
 
 }  // namespace ckks

@@ -35,6 +35,8 @@ bool conv_on_tensor(const ckks_ctx *ctx, int sources);
 int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::vector<u64> &dn_mat);
 int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
 int launch_conv_tc_down(const ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);
+// tcgen05 int8 MMA rate (M = 128, N = n in {32, 256}, K = 32), synchronous: elapsed ms and int8 ops
+int bench_mma(const ckks_ctx *ctx, int n, int blocks, int iters, double *ms, double *ops);
 
 // ---- sizes of internal stages (bytes)
 size_t modup_ws_bytes(const ckks_ctx *ctx, int batch);

@@ -371,3 +371,17 @@ def test_config5_boot_rotation_full_size_sampled(orc):
     finally:
         ctx.set_conversion("auto")
     assert torch.equal(out_int, out)
+
+
+def test_microbenchmarks_report_counts():
+    """The roofline denominators: every kind runs, reports its own operation
+    count and leaves the device flag clear; bad kinds are rejected."""
+    ctx = ctx_for(Params(4, 1, 1))
+    for kind, blocks, iters, per in ((0, 16, 64, 256 * 8), (1, 16, 64, 256 * 8), (2, 16, 64, 256 * 8),
+                                     (3, 4, 64, 2 * 128 * 256 * 32), (4, 4, 64, 2 * 128 * 32 * 32)):
+        ms, ops = ctx.bench_intpipe(kind, blocks, iters)
+        assert ms > 0
+        assert ops == blocks * iters * per
+    ctx.device_status()
+    with pytest.raises(CkksError):
+        ctx.bench_intpipe(5, 1, 1)
