@@ -13,17 +13,20 @@
 //  - the 15 accumulators P_d take TMEM columns 32 d .. 32 d + 31, in two groups: X = P_0..P_7
 //    (36 plane pairs) and Y = P_8..P_14 (28 pairs);
 //  - the y bytes of a tile are staged in one of two shared-memory buffers, two tiles ahead.
-// Every tcgen05.mma costs the SM a fixed issue time of a few dozen cycles up to N = 64, so the tile
-// is as wide as the 15 accumulators allow (15 x 32 of the 512 columns).
-// Warp roles: 16 epilogue warps and one MMA warp, synchronised by mbarriers only.
-//  - MMA warp (one elected lane): for tile i, waits until the tile's y bytes are staged and the
-//    epilogue has read group X of tile i - 1, issues group X and commits; then waits until the
-//    epilogue has read group Y of tile i - 1, issues group Y and commits.
+// Every tcgen05.mma costs a fixed issue time of a few dozen SM cycles up to N = 64, so the tile is as
+// wide as the 15 accumulators allow (15 x 32 of the 512 columns), and four warps issue: separate
+// issuing threads overlap their issue costs.
+// Warp roles: 16 epilogue warps and 4 MMA warps, synchronised by mbarriers only.
+//  - MMA warps (one elected lane each) own disjoint sets of accumulators: two split group X (P_d sets
+//    {0, 1, 6, 7} and {2, 3, 4, 5}, 18 plane pairs each), two split group Y ({8, 11, 12} and
+//    {9, 10, 13, 14}, 14 pairs each).  For tile i an issuer waits until the tile's y bytes are
+//    staged and the epilogue has read its group of tile i - 1, issues its products and commits to
+//    its group's barrier (which completes after both of the group's issuers commit).
 //  - Epilogue warps: wait for group X of tile i, fold it and release it (the tensor cores meanwhile
-//    form group Y); wait for group Y, release it, rebuild the exact 128-bit sums, reduce them once
-//    mod q_t and store (the tensor cores meanwhile run group X of tile i + 1); then stage tile i + 2
-//    into the buffer tile i used.  Warp w reads TMEM lane quadrant w & 3 (targets 32 (w & 3) ..) and
-//    columns 8 (w >> 2) .. of each accumulator: eight coefficients of one target per thread.
+//    form group Y); wait for group Y, fold it, rebuild the exact 128-bit sums, reduce them once mod
+//    q_t, release Y and store (the tensor cores meanwhile run group X of tile i + 1); then stage
+//    tile i + 2 into the buffer tile i used.  Warp w reads TMEM lane quadrant w & 3 (targets
+//    32 (w & 3) ..) and columns 8 (w >> 2) .. of each accumulator: eight coefficients of one target.
 //
 // Operand layout in shared memory (A and B): K-major, no swizzle, 8-row x 16-byte core matrices,
 // K-direction core-matrix stride (LBO) 128 bytes, 8-row-group stride (SBO) 512 bytes, for a K extent
@@ -31,8 +34,8 @@
 // on the host at context creation in exactly this layout; the y planes are packed by the threads.
 //
 // Every mbarrier wait is bounded: on expiry a thread records an error flag and leaves its loop (the
-// others then run out of arrivals and leave theirs), the MMA warp waits (bounded again) for the
-// products it issued, the CTA frees its tensor memory and returns; the host reports CKKS_ECUDA.
+// others then run out of arrivals and leave theirs), the MMA warps wait (bounded again) for the
+// products they issued, the CTA frees its tensor memory and returns; the host reports CKKS_ECUDA.
 #include "internal.cuh"
 
 namespace ckks {
@@ -44,12 +47,12 @@ constexpr int kATile = kPlanes * kAPlane;  // 64 KiB per block of 128 targets
 constexpr int kBPlane = kTN * kKP;         // 2 KiB per staged B byte plane
 constexpr int kBTile = kPlanes * kBPlane;  // 16 KiB per staged coefficient tile
 constexpr int kEpiWarps = 16, kEpiThreads = 32 * kEpiWarps;  // epilogue and staging
-constexpr int kThreads = kEpiThreads + 32;                    // plus one MMA-issue warp
+constexpr int kThreads = kEpiThreads + 128;                   // plus four MMA-issue warps
 constexpr int kTmemCols = 512;
 constexpr int kSmemB = kATile;             // two B buffers follow the A planes
 constexpr int kSmemBar = kSmemB + 2 * kBTile;
 constexpr int kSmemBytes = 116 * 1024;     // keeps one CTA per SM (it owns all of TMEM)
-static_assert(kSmemBar + 64 <= kSmemBytes, "shared-memory layout");
+static_assert(kSmemBar + 8 * 8 + 4 <= kSmemBytes, "shared-memory layout");
 
 __host__ __device__ __forceinline__ int cm_off(int row, int k)
 {
@@ -103,22 +106,24 @@ __device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity)
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// One accumulator group for the y tile at `bdesc`: X (kGroup 0) holds P_0..P_7, Y (kGroup 1)
-// P_8..P_14.  The first product into each P_d overwrites it.
-template <int kGroup>
-__device__ __forceinline__ void issue_group(uint32_t tmem, u64 adesc, u64 bdesc, bool two_k)
+// The products of the y tile at `bdesc` into the accumulators P_d whose bit d is set in kMask.  The
+// first product into each P_d (u = max(0, d - 7), K-step 0) overwrites it.
+template <int kMask>
+__device__ __forceinline__ void issue_set(uint32_t tmem, u64 adesc, u64 bdesc, bool two_k)
 {
 #pragma unroll
     for (int u = 0; u < kPlanes; ++u)
 #pragma unroll
-        for (int v = 0; v < kPlanes; ++v) {
-            const int d = u + v;
-            if ((d < 8) != (kGroup == 0)) continue;
-            const uint32_t acc = (u == (d > 7 ? d - 7 : 0)) ? 0u : 1u;
-            const uint32_t dcol = tmem + d * kTN;
-            const u64 ad = adesc + ((u * kAPlane) >> 4), bd = bdesc + ((v * kBPlane) >> 4);
-            mma_ss(dcol, ad, bd, acc);
-            if (two_k) mma_ss(dcol, ad + (256 >> 4), bd + (256 >> 4), 1u);
+        for (int h = 0; h < 2; ++h) {
+            if (h == 1 && !two_k) break;
+            const u64 ad = adesc + ((u * kAPlane + h * 256) >> 4);
+#pragma unroll
+            for (int v = 0; v < kPlanes; ++v) {
+                const int d = u + v;
+                if (!((kMask >> d) & 1)) continue;
+                const uint32_t acc = (h == 0 && u == (d > 7 ? d - 7 : 0)) ? 0u : 1u;
+                mma_ss(tmem + d * kTN, ad, bdesc + ((v * kBPlane + h * 256) >> 4), acc);
+            }
         }
 }
 
@@ -277,7 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1) conv_tc_kernel(TcJobs jobs, const
     const int cbase = run * ntiles * kTN;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSmemBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kSmemBar + 8 * kNumBars);
-    const bool mma_warp = warp == kEpiWarps;
+    const bool mma_warp = warp >= kEpiWarps;
+    const int issuer = warp - kEpiWarps;  // 0, 1: group X; 2, 3: group Y
+    const bool y_issuer = issuer >= 2;
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -285,13 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) conv_tc_kernel(TcJobs jobs, const
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
-        mbar_init(bar + kBarMmaX, 1);
-        mbar_init(bar + kBarMmaY, 1);
+        mbar_init(bar + kBarMmaX, 2);
+        mbar_init(bar + kBarMmaY, 2);
         mbar_init(bar + kBarFreeX, kEpiThreads);
         mbar_init(bar + kBarFreeY, kEpiThreads);
         mbar_init(bar + kBarFull0, kEpiThreads);
         mbar_init(bar + kBarFull1, kEpiThreads);
-        mbar_init(bar + kBarDrain, 1);
+        mbar_init(bar + kBarDrain, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // Staging share of an epilogue thread: coefficient n of each tile, sources s0 .. s0 + 3.
@@ -321,26 +328,22 @@ __global__ void __launch_bounds__(kThreads, 1) conv_tc_kernel(TcJobs jobs, const
     bool ok = true;
 
     if (mma_warp) {
-        // ------------------------------------------------ MMA issue (one elected lane)
+        // ------------------------------------------------ MMA issue (one elected lane per warp)
         const bool two_k = S > 32;
         const u64 adesc = smem_desc(smem_u32(sm)), bdesc0 = smem_desc(smem_u32(sm + kSmemB));
         for (int i = 0; i < ntiles && ok; ++i) {
             const u64 bdesc = bdesc0 + (((i & 1) * kBTile) >> 4);
             ok = __all_sync(0xffffffffu, mbar_wait(bar + kBarFull0 + (i & 1), (i >> 1) & 1));
-            if (ok && i > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar + kBarFreeX, (i - 1) & 1));
+            if (ok && i > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar + (y_issuer ? kBarFreeY : kBarFreeX), (i - 1) & 1));
             if (!ok) break;
             fence_after();
             if (lane == 0) {
-                issue_group<0>(tmem, adesc, bdesc, two_k);
-                commit(bar + kBarMmaX);
-            }
-            __syncwarp();
-            if (i > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar + kBarFreeY, (i - 1) & 1));
-            if (!ok) break;
-            fence_after();
-            if (lane == 0) {
-                issue_group<1>(tmem, adesc, bdesc, two_k);
-                commit(bar + kBarMmaY);
+                // P_d sets of 18, 18, 14 and 14 plane pairs
+                if (issuer == 0) issue_set<(1 << 0) | (1 << 1) | (1 << 6) | (1 << 7)>(tmem, adesc, bdesc, two_k);
+                if (issuer == 1) issue_set<(1 << 2) | (1 << 3) | (1 << 4) | (1 << 5)>(tmem, adesc, bdesc, two_k);
+                if (issuer == 2) issue_set<(1 << 8) | (1 << 11) | (1 << 12)>(tmem, adesc, bdesc, two_k);
+                if (issuer == 3) issue_set<(1 << 9) | (1 << 10) | (1 << 13) | (1 << 14)>(tmem, adesc, bdesc, two_k);
+                commit(bar + (y_issuer ? kBarMmaY : kBarMmaX));
             }
             __syncwarp();
         }
