@@ -501,10 +501,27 @@ def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak, conv_macs=0, int8_peak=
 
 
 # ---------------------------------------------------------------- CPU baselines
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(min_seconds=10.0):
-    """The oracle as it stands, timed on this host's cores on a bounded sample
-    of the sweep: the 112-limb entry (16 polynomials) forward + inverse,
-    repeated until at least `min_seconds` have elapsed."""
+    """The oracle as it stands, timed on this host's cores on bounded samples.
+
+    - value: the sweep's 112-limb entry (16 polynomials) forward + inverse on
+      all cores, repeated until at least `min_seconds` have elapsed;
+    - single_thread: the same on one thread (one polynomial, >= 3 s);
+    - keyswitch: the key-switching workloads on all cores, each on a subset
+      scaled linearly to the GPU workload: the boot-level rotation from one
+      ciphertext with one and with two keys (separating the hoisted ModUp
+      from the per-key work, then 8 ModUps + 32 key switches), the layer
+      multiply from one ciphertext pair."""
     import numpy as np
 
     import oracle
@@ -520,10 +537,59 @@ def cpu_baseline(min_seconds=10.0):
         el = time.perf_counter() - t0
         if el >= min_seconds:
             break
-    ntts = reps * 2 * BATCH * 112
-    return {"value": ntts / el, "unit": "limb-NTTs/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": "%d repetitions of 16 x 112-limb NTT + INTT (%.1f s)" % (reps, el)}
+    cores = oracle.num_threads()
+    out = {"value": reps * 2 * BATCH * 112 / el, "unit": "limb-NTTs/s", "cores": cores, "kind": "oracle",
+           "sample": "%d repetitions of 16 x 112-limb NTT + INTT (%.1f s)" % (reps, el),
+           "cpu_model": cpu_model()}
+    # one thread
+    oracle.set_num_threads(1)
+    try:
+        a1 = np.ascontiguousarray(a[:1])
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.ntt_inv(oracle.ntt_fwd(a1, mods), mods)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= 3.0:
+                break
+    finally:
+        oracle.set_num_threads(cores)
+    out["single_thread"] = {"value": reps * 2 * 112 / el, "unit": "limb-NTTs/s", "cores": 1,
+                            "sample": "%d repetitions of 1 x 112-limb NTT + INTT (%.1f s)" % (reps, el)}
+    ks = {}
+    # boot-level rotation: L = 2100, K = 60, alpha = 60
+    m5 = np.array(oracle.gen_primes(N, 2160), dtype=np.uint64)
+    seed = synth.config_seed(5)
+    ct = synth.uniform_residues((1, 2, 2100, N), [int(x) for x in m5[:2100]], seed, 1).numpy().astype(np.uint64)
+    keys = [synth.uniform_residues((35, 2, 2160, N), [int(x) for x in m5], seed, 10 + r).numpy().astype(np.uint64)
+            for r in range(2)]
+    t0 = time.perf_counter()
+    oracle.rotate(ct, keys[:1], np.array([5], dtype=np.uint64), m5, 2100, 60, 60)
+    t1 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.rotate(ct, keys, np.array([5, 25], dtype=np.uint64), m5, 2100, 60, 60)
+    t2 = time.perf_counter() - t0
+    per_key = max(t2 - t1, 1e-9)
+    full = 8 * (t1 - per_key) + 32 * per_key
+    ks["boot_rotation_L2100"] = {
+        "keyswitches_per_s": 32 / full, "unit": "key switches/s",
+        "sample": "1 ciphertext with 1 key (%.1f s) and with 2 keys (%.1f s); scaled to 8 hoisted ModUps "
+                  "+ 32 key switches" % (t1, t2)}
+    del keys
+    # layer multiply: L = 112, K = 8, alpha = 8, one ciphertext pair
+    m3 = np.array(oracle.gen_primes(N, 120), dtype=np.uint64)
+    seed = synth.config_seed(3)
+    q3 = [int(x) for x in m3[:112]]
+    ca = synth.uniform_residues((1, 2, 112, N), q3, seed, 1).numpy().astype(np.uint64)
+    cb = synth.uniform_residues((1, 2, 112, N), q3, seed, 2).numpy().astype(np.uint64)
+    rlk = synth.uniform_residues((14, 2, 120, N), [int(x) for x in m3], seed, 3).numpy().astype(np.uint64)
+    t0 = time.perf_counter()
+    oracle.mul_relin_rescale(ca, cb, rlk, m3, 112, 8, 8)
+    t3 = time.perf_counter() - t0
+    ks["layer_mul_relin_L112"] = {"keyswitches_per_s": 1 / t3, "unit": "key switches/s",
+                                  "sample": "1 ciphertext pair (%.2f s)" % t3}
+    out["keyswitch"] = ks
+    return out
 
 
 def run_reference(args):

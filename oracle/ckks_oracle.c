@@ -816,6 +816,16 @@ void oracle_negacyclic_mul(const u64 *a, const u64 *b, u64 *out, u64 q, int n)
 }
 
 /* Threads an OpenMP parallel-for of this library uses (1 without OpenMP). */
+/* Thread count for the parallel loops that follow (t >= 1); for timing only. */
+void oracle_set_num_threads(int t)
+{
+#ifdef _OPENMP
+    if (t >= 1) omp_set_num_threads(t);
+#else
+    (void)t;
+#endif
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

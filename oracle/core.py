@@ -64,6 +64,8 @@ def _lib():
         L.oracle_decrypt.argtypes = [_u64p, _i64p, _u64p, _u64p, C.c_int, C.c_int]
         L.oracle_negacyclic_mul.argtypes = [_u64p, _u64p, _u64p, C.c_uint64, C.c_int]
         L.oracle_num_threads.restype = C.c_int
+        L.oracle_set_num_threads.argtypes = [C.c_int]
+        L.oracle_set_num_threads.restype = None
     return _LIB
 
 
@@ -86,6 +88,11 @@ def _ptr_array(arrs):
 def num_threads():
     """Threads the oracle's OpenMP loops use."""
     return int(_lib().oracle_num_threads())
+
+
+def set_num_threads(t):
+    """Threads for the oracle's following OpenMP loops (timing only)."""
+    _lib().oracle_set_num_threads(int(t))
 
 
 def digit_count(L, alpha):
