@@ -131,7 +131,10 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- distributed plumbing
-def dist_init(args):
+def dist_init(args, backend=None):
+    """One process per GPU: rank, world size, local rank and the process group
+    (None for a single process).  The backend is NCCL when CUDA is present,
+    gloo otherwise (or as given)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -141,7 +144,8 @@ def dist_init(args):
         import datetime
 
         import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
@@ -152,10 +156,12 @@ def dist_init(args):
 
 
 def max_over_ranks(value, pg):
+    """The maximum of a per-rank value over all ranks (device timing is taken
+    as the slowest rank's)."""
     if pg is None:
         return value
     import torch
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
     t = torch.tensor([value], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
@@ -164,6 +170,12 @@ def max_over_ranks(value, pg):
 def barrier(pg):
     if pg is not None:
         pg.barrier()
+
+
+def weak_scaling_value(per_step_units, steps, world, total_ms):
+    """Whole-job throughput: every rank processes per_step_units per step (its
+    own batch), and the job takes the slowest rank's time."""
+    return per_step_units * steps * world / (total_ms * 1e-3)
 
 
 # ---------------------------------------------------------------- roofline bits
@@ -267,7 +279,7 @@ def run_b200(args):
     ok = bool(max_over_ranks(0.0 if ok else 1.0, pg) == 0.0)
 
     per_step = 2 * BATCH * sum(SWEEP)
-    value = per_step * args.steps * world / (total_ms * 1e-3)
+    value = weak_scaling_value(per_step, args.steps, world, total_ms)
 
     # roofline of the dominant kernel: forward NTT on the largest sweep entry
     bytes_, mm = ntt_launch_work(SWEEP[-1])
