@@ -421,7 +421,10 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
     res = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
     ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
     ms = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 10, stream)
-    out["layer_mul_relin_L112"] = ks_entry(B, ms, ks_work_mrr(112, 8, 8, B), hbm_peak, mm_peak, mac_peak)
+    up, _, down = ks_work_keyswitch_parts(112, 8, 8)
+    out["layer_mul_relin_L112"] = ks_entry(B, ms, ks_work_mrr(112, 8, 8, B), hbm_peak, mm_peak, mac_peak,
+                                           conv_macs=B * (up["mac"] + down["mac"]),
+                                           int8_peak=int8_mac_peak(ipeak))
     # BSGS: bb = gg = 32, 62 keys, 8 cts
     seed = synth.config_seed(4)
     x = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
@@ -432,7 +435,9 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
     ws = torch.empty(ctx.workspace_bytes(7, B, 32032), dtype=torch.uint8, device=dev)
     ms = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 3, stream)
     out["bsgs_L112_32x32"] = ks_entry(B * 62, ms, ks_work_bsgs(112, 8, 8, B, 32, 32), hbm_peak,
-                                      mm_peak, mac_peak)
+                                      mm_peak, mac_peak,
+                                      conv_macs=B * (up["mac"] + 31 * down["mac"] + 31 * (up["mac"] + down["mac"])),
+                                      int8_peak=int8_mac_peak(ipeak))
     return out
 
 
@@ -493,7 +498,7 @@ def int8_mac_peak(ipeak):
 def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak, conv_macs=0, int8_peak=None):
     """roofline_frac follows the problem statement: modular multiplies and 64-bit MACs at the
     same-run integer-pipe peaks, bytes at the HBM peak.  When the basis conversion runs on the
-    int8 tensor cores (digits above 16 primes) that model can be exceeded; tensor_model_frac then
+    int8 tensor cores (8 or more source primes) that model can be exceeded; tensor_model_frac then
     charges the conversion's int8 byte-plane products (64 per 60-bit MAC, sources padded to 64)
     at the same-run int8 tensor-core peak (`int8_peak`, MAC/s) instead."""
     mm, mac, bytes_ = work

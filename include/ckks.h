@@ -105,17 +105,17 @@ const char *ckks_last_error(void);
 /* Waits for the context's device and reports whether any kernel of this
  * context gave up a bounded wait since the last call: CKKS_ECUDA with a
  * message if so (the flag is then cleared), else CKKS_OK.  Only the int8
- * tensor-core basis conversion (digits or special bases of more than 16
- * primes) waits on the device; it bounds every wait, and if one expires it
- * stops issuing work, frees its tensor memory and raises the flag, so the
- * affected outputs must be discarded.  Also returns CKKS_ECUDA for an
- * asynchronous CUDA error on the device. */
+ * tensor-core basis conversion (see ckks_ctx_set_conversion) and the
+ * tensor-pipe microbenchmark wait on the device; they bound every wait, and
+ * if one expires the kernel stops issuing work, frees its tensor memory and
+ * raises the flag, so the affected outputs must be discarded.  Also returns
+ * CKKS_ECUDA for an asynchronous CUDA error on the device. */
 int ckks_device_status(const ckks_ctx *ctx);
 
 /* Where the basis conversions of ModUp and ModDown run.  The conversion is
  * the exact product out_t = sum_s y_s [Q_j/q_s]_t (mod t), the step named
  * "RNS basis conversion" in the Kestrel engine write-up, section 3 table.
- *  CKKS_CONV_AUTO     int8 tensor cores when the conversion has more than 16
+ *  CKKS_CONV_AUTO     int8 tensor cores when the conversion has 8 or more
  *                     source primes (ModUp: alpha; ModDown: K), the integer
  *                     pipes otherwise (the default);
  *  CKKS_CONV_INTEGER  always the integer pipes (64x64->128-bit multiply-adds);

@@ -80,8 +80,9 @@ class Context:
     CONVERSION = {"auto": 0, "integer": 1, "tensor": 2}
 
     def set_conversion(self, engine):
-        """Where ModUp/ModDown basis conversions run: "auto", "integer" (integer
-        pipes) or "tensor" (int8 tensor cores).  Results are bit-identical."""
+        """Where ModUp/ModDown basis conversions run: "auto" (tensor cores from 8
+        source primes on), "integer" (integer pipes) or "tensor" (int8 tensor
+        cores).  Results are bit-identical."""
         check("ckks_ctx_set_conversion",
               lib().ckks_ctx_set_conversion(self._h, self.CONVERSION.get(engine, -1)
                                             if isinstance(engine, str) else int(engine)))

@@ -30,7 +30,7 @@ struct Carve {
 inline size_t limbs_bytes(size_t rows) { return ((rows * kN * sizeof(u64)) + 255) & ~(size_t)255; }
 
 // ---- int8 tensor-core basis conversion (conv_tc.cu)
-constexpr int kTcMinSources = 16;  // CKKS_CONV_AUTO: more sources use the tensor cores
+constexpr int kTcMinSources = 7;  // CKKS_CONV_AUTO: more sources (8 or more) use the tensor cores
 bool conv_on_tensor(const ckks_ctx *ctx, int sources);
 int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::vector<u64> &dn_mat);
 int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);

@@ -149,8 +149,8 @@ def test_automorph_rejects_even_and_in_place():
                                        (40, 20, 20), (70, 33, 33), (130, 64, 64)])
 def test_modup_inner_moddown_stages(orc, L, K, alpha):
     """Every stage on every conversion engine (integer pipes, int8 tensor cores,
-    and the automatic choice, which takes the tensor cores above 16 source
-    primes); (70, 33, 33) has a ragged 4-prime last digit."""
+    and the automatic choice, which takes the tensor cores from 8 source
+    primes on); (70, 33, 33) has a ragged 4-prime last digit."""
     p = Params(L, K, alpha)
     ctx = ctx_for(p)
     mods = np.array(ctx.mods, dtype=np.uint64)
