@@ -385,3 +385,48 @@ def test_microbenchmarks_report_counts():
     ctx.device_status()
     with pytest.raises(CkksError):
         ctx.bench_intpipe(5, 1, 1)
+
+
+def _general_primes(orc, count):
+    """Primes q = 1 mod 2n just above 2^59: far from 2^60, so none has the 2^60 - delta form the
+    library's cheaper products use."""
+    out, c = [], (1 << 59) + 1
+    while len(out) < count:
+        if orc.is_prime(c):
+            out.append(c)
+        c += 2 * N
+    return out
+
+
+def test_general_primes_full_stage_parity(orc):
+    """The general-prime code paths (full Shoup quotients in the transforms, the generic 128-bit
+    reduction in both conversion engines) on every stage, against the oracle."""
+    from rns_ckks_polynomial_b200 import Context
+    L, K, alpha = 6, 3, 3
+    mods_l = _general_primes(orc, L + K)
+    assert all((1 << 60) - q >= (1 << 32) for q in mods_l)
+    ctx = Context(mods_l[:L], mods_l[L:], alpha)
+    mods = np.array(mods_l, dtype=np.uint64)
+    x = _res((2, L, N), mods[:L], 300)
+    y = ctx.ntt_fwd(dev(x))
+    assert_bits_equal(host(y), orc.ntt_fwd(x, mods[:L]), "ntt_fwd")
+    assert_bits_equal(host(ctx.ntt_inv(y)), x, "ntt_inv round trip")
+    key = _res((2, 2, L + K, N), mods, 301)
+    want_d = orc.modup(x, mods, L, K, alpha)
+    want_a = orc.key_inner(want_d, key, 5, mods, L, K, alpha)
+    want_m = orc.moddown(want_a, mods, L, K)
+    want_k = orc.keyswitch(x, key, mods, L, K, alpha)
+    try:
+        for engine in ("integer", "tensor"):
+            ctx.set_conversion(engine)
+            dig = ctx.modup(dev(x))
+            assert_bits_equal(host(dig), want_d, "modup (%s)" % engine)
+            acc = ctx.key_inner(dig, dev(key), 5)
+            assert_bits_equal(host(acc), want_a, "key_inner")
+            assert_bits_equal(host(ctx.moddown(acc)), want_m, "moddown (%s)" % engine)
+            assert_bits_equal(host(ctx.keyswitch(dev(x), dev(key))), want_k, "keyswitch (%s)" % engine)
+            ctx.device_status()
+    finally:
+        ctx.set_conversion("auto")
+    ct = _res((2, 2, L, N), mods[:L], 302)
+    assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, mods[:L]), "rescale")
