@@ -386,6 +386,36 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
     stream = torch.cuda.current_stream(dev)
     mm_peak, mac_peak = ipeak["shoup_mulmod_per_s"], ipeak["mac128_per_s"]
     out = {}
+    # tiny pipeline: 4 + 1 primes, alpha = 1; 8 polynomials -> NTT -> pairwise product -> INTT, and
+    # one rotation key switch of (P0, P1) with the Galois-5 key
+    seed = synth.config_seed(1)
+    m1 = primes(5)
+    ctx = Context(m1[:4], m1[4:], 1, device=dev.index)
+    polys = synth.uniform_residues((8, 4, N), m1[:4], seed, 1, device=dev)
+    key = synth.uniform_residues((4, 2, 5, N), m1, seed, 2, device=dev)
+    x = polys.clone()
+    prod = torch.empty((4, 4, N), dtype=torch.int64, device=dev)
+    rot = torch.empty((1, 1, 2, 4, N), dtype=torch.int64, device=dev)
+    ws = torch.empty(ctx.workspace_bytes(4, 1, 1), dtype=torch.uint8, device=dev)
+
+    def tiny():
+        x.copy_(polys)
+        ctx.ntt_fwd(x)
+        ctx.pointwise("mul", x[0::2].contiguous(), x[1::2].contiguous(), out=prod)
+        ctx.ntt_inv(prod)
+        ctx.rotate(x[0:2].reshape(1, 2, 4, N), [key], [5], out=rot, ws=ws)
+
+    ms = _time_call(tiny, 50, stream)
+    ntt = (N // 2) * 11
+    up, inner, down = ks_work_keyswitch_parts(4, 1, 1)
+    mm = (8 + 4) * 4 * ntt + 4 * 4 * N + up["mm"] + down["mm"]
+    mac = up["mac"] + inner["mac"] + down["mac"]
+    io = (8 * 4 + 4 * 4 + 2 * 4) * N * 8 + 4 * 2 * 5 * N * 8
+    out["tiny_pipeline_L4"] = ks_entry(1, ms, (mm, mac, io), hbm_peak, mm_peak, mac_peak)
+    out["tiny_pipeline_L4"]["note"] = ("one call: 8 limb-4 NTTs, 4 products, 4 INTTs and one rotation; "
+                                       "launch-bound at this size")
+    ctx.device_status()
+    del ctx, polys, key, x, prod, rot, ws
     # boot-level hoisted rotation: L = 2100, K = 60, alpha = 60, 4 keys, 8 cts
     seed = synth.config_seed(5)
     mods = primes(2160)
@@ -536,9 +566,9 @@ def cpu_baseline(min_seconds=10.0):
     - single_thread: the same on one thread (one polynomial, >= 3 s);
     - keyswitch: the key-switching workloads on all cores, each on a subset
       scaled linearly to the GPU workload: the boot-level rotation from one
-      ciphertext with one and with two keys (separating the hoisted ModUp
-      from the per-key work, then 8 ModUps + 32 key switches), the layer
-      multiply from one ciphertext pair."""
+      ciphertext's hoisted ModUp and one key's inner product + ModDown (then
+      8 ModUps + 32 key switches), the layer multiply from one ciphertext
+      pair, BSGS from one ciphertext."""
     import numpy as np
 
     import oracle
@@ -574,25 +604,23 @@ def cpu_baseline(min_seconds=10.0):
     out["single_thread"] = {"value": reps * 2 * 112 / el, "unit": "limb-NTTs/s", "cores": 1,
                             "sample": "%d repetitions of 1 x 112-limb NTT + INTT (%.1f s)" % (reps, el)}
     ks = {}
-    # boot-level rotation: L = 2100, K = 60, alpha = 60
+    # boot-level rotation: L = 2100, K = 60, alpha = 60; one ciphertext's hoisted ModUp and one
+    # key's inner product + ModDown, scaled to 8 ModUps + 32 key switches
     m5 = np.array(oracle.gen_primes(N, 2160), dtype=np.uint64)
     seed = synth.config_seed(5)
-    ct = synth.uniform_residues((1, 2, 2100, N), [int(x) for x in m5[:2100]], seed, 1).numpy().astype(np.uint64)
-    keys = [synth.uniform_residues((35, 2, 2160, N), [int(x) for x in m5], seed, 10 + r).numpy().astype(np.uint64)
-            for r in range(2)]
+    c1 = synth.uniform_residues((1, 2100, N), [int(x) for x in m5[:2100]], seed, 1).numpy().astype(np.uint64)
+    key = synth.uniform_residues((35, 2, 2160, N), [int(x) for x in m5], seed, 10).numpy().astype(np.uint64)
     t0 = time.perf_counter()
-    oracle.rotate(ct, keys[:1], np.array([5], dtype=np.uint64), m5, 2100, 60, 60)
-    t1 = time.perf_counter() - t0
+    dig = oracle.modup(c1, m5, 2100, 60, 60)
+    t_up = time.perf_counter() - t0
     t0 = time.perf_counter()
-    oracle.rotate(ct, keys, np.array([5, 25], dtype=np.uint64), m5, 2100, 60, 60)
-    t2 = time.perf_counter() - t0
-    per_key = max(t2 - t1, 1e-9)
-    full = 8 * (t1 - per_key) + 32 * per_key
+    oracle.moddown(oracle.key_inner(dig, key, 5, m5, 2100, 60, 60), m5, 2100, 60)
+    t_key = time.perf_counter() - t0
     ks["boot_rotation_L2100"] = {
-        "keyswitches_per_s": 32 / full, "unit": "key switches/s",
-        "sample": "1 ciphertext with 1 key (%.1f s) and with 2 keys (%.1f s); scaled to 8 hoisted ModUps "
-                  "+ 32 key switches" % (t1, t2)}
-    del keys
+        "keyswitches_per_s": 32 / (8 * t_up + 32 * t_key), "unit": "key switches/s",
+        "sample": "1 ciphertext's ModUp (%.1f s) and one key's inner product + ModDown (%.1f s); scaled "
+                  "to 8 hoisted ModUps + 32 key switches" % (t_up, t_key)}
+    del dig, key
     # layer multiply: L = 112, K = 8, alpha = 8, one ciphertext pair
     m3 = np.array(oracle.gen_primes(N, 120), dtype=np.uint64)
     seed = synth.config_seed(3)
@@ -605,6 +633,19 @@ def cpu_baseline(min_seconds=10.0):
     t3 = time.perf_counter() - t0
     ks["layer_mul_relin_L112"] = {"keyswitches_per_s": 1 / t3, "unit": "key switches/s",
                                   "sample": "1 ciphertext pair (%.2f s)" % t3}
+    # BSGS 32 x 32 at 112 primes: one ciphertext (62 key switches)
+    seed = synth.config_seed(4)
+    x4 = synth.uniform_residues((1, 2, 112, N), q3, seed, 1).numpy().astype(np.uint64)
+    d4 = synth.uniform_residues((32, 32, 112, N), q3, seed, 2).numpy().astype(np.uint64)
+    bk = [synth.uniform_residues((14, 2, 120, N), [int(x) for x in m3], seed, 100 + i).numpy().astype(np.uint64)
+          for i in range(31)]
+    gk = [synth.uniform_residues((14, 2, 120, N), [int(x) for x in m3], seed, 200 + i).numpy().astype(np.uint64)
+          for i in range(31)]
+    t0 = time.perf_counter()
+    oracle.bsgs(x4, d4, bk, gk, 32, 32, m3, 112, 8, 8)
+    t4 = time.perf_counter() - t0
+    ks["bsgs_L112_32x32"] = {"keyswitches_per_s": 62 / t4, "unit": "key switches/s",
+                             "sample": "1 ciphertext (62 key switches, %.1f s)" % t4}
     out["keyswitch"] = ks
     return out
 
