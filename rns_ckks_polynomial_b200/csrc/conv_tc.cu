@@ -301,8 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1) conv_tc_kernel(TcJobs jobs, const
         mbar_init(bar + kBarDrain, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // Staging share of an epilogue thread: coefficient n of each tile, sources s0 .. s0 + 3.
-    const int n = tid & 31, s0 = (tid >> 5) * 4;
+    // Staging share of an epilogue thread: coefficient n of each tile, sources s0 .. s0 + 3.  A warp
+    // covers 8 coefficients x 4 source quads, so its 32-bit stores into the core-matrix layout fall
+    // in 32 different banks (bank = 4 (n & 7) + ((s0 & 15) >> 2)).
+    const int n = ((warp & 3) << 3) | (lane & 7), s0 = ((warp >> 2) << 4) | ((lane >> 3) << 2);
     const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + n;
     auto fetch = [&](int i, u64 (&v)[4]) {
 #pragma unroll
