@@ -155,31 +155,52 @@ int rescale_stage(ckks_ctx *ctx, const u64 *ct, u64 *out, int lp1, int batch, vo
 // ---------------------------------------------------------------- BSGS pieces
 // inner[g][b][c][i][e] = sum_r diags[g][r][i][e] * baby_r[b][c][i][e], where
 // baby_0 = x and baby_r (r >= 1) = baby[r-1].  One CTA per (32 coefficients,
-// limb i, ciphertext-component bc): the bb baby values sit in shared memory,
-// 8 warps split the giant index g.
+// limb i, group of kBC ciphertext-components bc): the group's bb baby values
+// sit in shared memory, 8 warps split the giant index g, and each diagonal
+// word loaded serves the kBC components.  The grid runs the component groups
+// of one (coefficients, limb) back to back, so the diagonals cross HBM once
+// and are re-read from L2 by the other groups.
 constexpr int kMaxBaby = 64;
 
+template <int kBC>
 __global__ void __launch_bounds__(256) bsgs_inner_kernel(const u64 *__restrict__ diags,
                                                          const u64 *__restrict__ x,
                                                          const u64 *__restrict__ baby,
                                                          u64 *__restrict__ inner, int bb, int gg,
                                                          int B, int L, const PrimeConst *__restrict__ pc)
 {
-    __shared__ u64 sb[kMaxBaby][32];
+    extern __shared__ u64 sb[];  // [kBC][bb][32]
     const int lane = threadIdx.x & 31, gw = threadIdx.x >> 5;
-    const int i = blockIdx.y, bc = blockIdx.z;
-    const int e = blockIdx.x * 32 + lane;
+    const int ngrp = (2 * B + kBC - 1) / kBC;
+    const int grp = blockIdx.x % ngrp, ech = blockIdx.x / ngrp, i = blockIdx.y;
+    const int e = ech * 32 + lane;
+    const int bc0 = grp * kBC, nbc = min(kBC, 2 * B - bc0);
     const size_t Ln = (size_t)L * kN;
-    const size_t off = (size_t)bc * Ln + (size_t)i * kN + e;  // within one [B][2][L][n] block
-    for (int r = gw; r < bb; r += 8)
-        sb[r][lane] = r == 0 ? x[off] : baby[(size_t)(r - 1) * B * 2 * Ln + off];
+    const size_t off0 = (size_t)bc0 * Ln + (size_t)i * kN + e;  // within one [B][2][L][n] block
+    for (int idx = gw; idx < kBC * bb; idx += 8) {
+        const int q = idx / bb, r = idx - q * bb;
+        u64 v = 0;
+        if (q < nbc) {
+            const size_t off = off0 + (size_t)q * Ln;
+            v = r == 0 ? x[off] : baby[(size_t)(r - 1) * B * 2 * Ln + off];
+        }
+        sb[(q * bb + r) * 32 + lane] = v;
+    }
     __syncthreads();
     const PrimeConst c = pc[i];
     for (int g = gw; g < gg; g += 8) {
         const u64 *d = diags + ((size_t)g * bb * L + i) * kN + e;
-        u64 hi = 0, lo = 0;
-        for (int r = 0; r < bb; ++r) mac128(hi, lo, __ldg(d + (size_t)r * Ln), sb[r][lane]);
-        inner[(size_t)g * B * 2 * Ln + off] = reduce128(hi, lo, c);
+        u64 hi[kBC], lo[kBC];
+#pragma unroll
+        for (int q = 0; q < kBC; ++q) hi[q] = lo[q] = 0;
+        for (int r = 0; r < bb; ++r) {
+            const u64 dv = __ldg(d + (size_t)r * Ln);
+#pragma unroll
+            for (int q = 0; q < kBC; ++q) mac128(hi[q], lo[q], dv, sb[(q * bb + r) * 32 + lane]);
+        }
+#pragma unroll
+        for (int q = 0; q < kBC; ++q)
+            if (q < nbc) inner[(size_t)g * B * 2 * Ln + off0 + (size_t)q * Ln] = reduce128(hi[q], lo[q], c);
     }
 }
 
@@ -457,8 +478,16 @@ extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const 
     }
     // inner sums for every giant index
     {
-        dim3 grid(kN / 32, L, 2 * B);
-        bsgs_inner_kernel<<<grid, 256, 0, s>>>(diags, x, baby, inner, bb, gg, B, L, T.pc);
+        // 4 components per CTA while the baby values fit 32 KiB of shared memory, else 2
+        if (bb <= 32) {
+            const dim3 grid((kN / 32) * ((2 * B + 3) / 4), L);
+            bsgs_inner_kernel<4><<<grid, 256, (size_t)4 * bb * 32 * sizeof(u64), s>>>(diags, x, baby, inner, bb,
+                                                                                       gg, B, L, T.pc);
+        } else {
+            const dim3 grid((kN / 32) * ((2 * B + 1) / 2), L);
+            bsgs_inner_kernel<2><<<grid, 256, (size_t)2 * bb * 32 * sizeof(u64), s>>>(diags, x, baby, inner, bb,
+                                                                                       gg, B, L, T.pc);
+        }
         CKKS_CHECK_LAUNCH("bsgs_inner_kernel");
     }
     // giant steps: total = inner_0 + sum_{g >= 1} Rot_{bb g}(inner_g)
