@@ -13,10 +13,11 @@
 // Kernels:
 //  - INTT of the input limbs with the digit copy and the factor
 //    [(Q_j/q_i)^-1]_{q_i} fused into its load/store (ntt.cuh);
-//  - conv_kernel: the basis-conversion product out_t = sum_s y_s M[s][t],
-//    a (targets x sources) x (sources x coefficients) matrix product with
-//    exact 128-bit accumulation and one reduction per output, on the integer
-//    pipes;
+//  - the basis-conversion product out_t = sum_s y_s M[s][t], a (targets x
+//    sources) x (sources x coefficients) matrix product reduced once per
+//    output: conv_kernel below on the integer pipes (exact 128-bit
+//    accumulation), or conv_tc_kernel (conv_tc.cu) on the int8 tensor cores,
+//    as the context's conversion engine selects;
 //  - forward NTT of the new limbs in place;
 //  - key_inner_kernel: the dnum-term inner product with the key, the Galois
 //    permutation applied as a gather on the digit load;
