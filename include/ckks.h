@@ -112,6 +112,14 @@ const char *ckks_last_error(void);
  * CKKS_ECUDA for an asynchronous CUDA error on the device. */
 int ckks_device_status(const ckks_ctx *ctx);
 
+/* Failure-path self-test of the bounded device waits (no page counterpart):
+ * launches, on the context's device and default stream, one kernel that waits
+ * with the library's bound on a barrier nothing completes, so the wait expires
+ * and the context's device flag is raised.  The next ckks_device_status then
+ * returns CKKS_ECUDA and clears the flag; the context stays usable.  Takes up
+ * to about a second of device time.  CKKS_EINVAL for a null context. */
+int ckks_selftest_wait_expiry(const ckks_ctx *ctx);
+
 /* Where the basis conversions of ModUp and ModDown run.  The conversion is
  * the exact product out_t = sum_s y_s [Q_j/q_s]_t (mod t), the step named
  * "RNS basis conversion" in the Kestrel engine write-up, section 3 table.

@@ -77,6 +77,10 @@ class Context:
         """Synchronise the device and raise if a bounded device wait expired."""
         check("ckks_device_status", lib().ckks_device_status(self._h))
 
+    def selftest_wait_expiry(self):
+        """Launch the bounded-wait expiry self-test; device_status() then raises."""
+        check("ckks_selftest_wait_expiry", lib().ckks_selftest_wait_expiry(self._h))
+
     CONVERSION = {"auto": 0, "integer": 1, "tensor": 2}
 
     def set_conversion(self, engine):

@@ -499,6 +499,18 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, int *err)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(256));
 }
 
+// Failure-path self-test: one thread waits, with the same bound as every other wait in this file, on
+// an mbarrier that nothing ever completes, and raises the context's flag when the bound expires.
+__global__ void wait_expiry_kernel(int *err)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (!mbar_wait(&bar, 0)) atomicExch(err, 1);
+    }
+}
+
 }  // namespace
 
 bool conv_on_tensor(const ckks_ctx *ctx, int sources)
@@ -596,6 +608,13 @@ int bench_mma(const ckks_ctx *ctx, int n, int blocks, int iters, double *ms, dou
     if (e != cudaSuccess) return cuda_status(e, "mma_rate_kernel");
     *ms = t;
     *ops = 2.0 * kTM * n * 32 * (double)blocks * iters;
+    return CKKS_OK;
+}
+
+int selftest_wait_expiry(const ckks_ctx *ctx)
+{
+    wait_expiry_kernel<<<1, 32>>>(ctx->tc_err);
+    CKKS_CHECK_LAUNCH("wait_expiry_kernel");
     return CKKS_OK;
 }
 

@@ -422,6 +422,13 @@ extern "C" int ckks_device_status(const ckks_ctx *ctx)
     return CKKS_OK;
 }
 
+extern "C" int ckks_selftest_wait_expiry(const ckks_ctx *ctx)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(set_device(ctx));
+    return selftest_wait_expiry(ctx);
+}
+
 extern "C" int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine)
 {
     CKKS_TRY(check_ctx(ctx));

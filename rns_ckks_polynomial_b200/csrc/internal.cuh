@@ -37,6 +37,8 @@ int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch,
 int launch_conv_tc_down(const ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);
 // tcgen05 int8 MMA rate (M = 128, N = n in {32, 256}, K = 32), synchronous: elapsed ms and int8 ops
 int bench_mma(const ckks_ctx *ctx, int n, int blocks, int iters, double *ms, double *ops);
+// launches the bounded-wait expiry self-test (asynchronous)
+int selftest_wait_expiry(const ckks_ctx *ctx);
 
 // ---- sizes of internal stages (bytes)
 size_t modup_ws_bytes(const ckks_ctx *ctx, int batch);

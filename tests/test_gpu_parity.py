@@ -430,3 +430,19 @@ def test_general_primes_full_stage_parity(orc):
         ctx.set_conversion("auto")
     ct = _res((2, 2, L, N), mods[:L], 302)
     assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, mods[:L]), "rescale")
+
+
+def test_bounded_wait_expiry_is_reported_and_recoverable(orc):
+    """A device wait that runs out (on a barrier nothing completes) raises the
+    context's flag; device_status reports it once, clears it, and the context
+    keeps computing correctly."""
+    ctx = ctx_for(Params(4, 1, 1))
+    ctx.device_status()
+    ctx.selftest_wait_expiry()
+    with pytest.raises(CkksError) as e:
+        ctx.device_status()
+    assert e.value.code == -3 and "waiting" in str(e.value)
+    ctx.device_status()
+    q = np.array(ctx.q, dtype=np.uint64)
+    x = _res((2, 4, N), q, 400)
+    assert_bits_equal(host(ctx.ntt_fwd(dev(x))), orc.ntt_fwd(x, q), "ntt_fwd after the expiry")
