@@ -547,6 +547,44 @@ void oracle_rotate(const u64 *ct /*[B][2][L][n]*/, const u64 *const *keys,
     ptabs_free(tabs, LK);
 }
 
+/* The other rotation order (automorphism first, no hoisting): for every key,
+ * phi_g(c1) is key-switched with the Galois key -- ModUp of the rotated c1,
+ * inner product without a gather, ModDown -- and phi_g(c0) is added.  The
+ * Galois key is the same (it switches from phi_g(s) to s); the approximate
+ * ModUp of phi_g(c1) is not phi_g of the ModUp of c1, so the low bits differ
+ * from oracle_rotate while both decrypt to the rotated slots. */
+void oracle_rotate_unhoisted(const u64 *ct /*[B][2][L][n]*/, const u64 *const *keys,
+                             const u64 *galois, int nkeys, u64 *out /*[nkeys][B][2][L][n]*/,
+                             const u64 *mods, int L, int K, int alpha, int batch, int n)
+{
+    const int dnum = digit_count(L, alpha), LK = L + K;
+    ptab *tabs = ptabs_make(mods, LK, n);
+    u64 *dig = (u64 *)malloc(sizeof(u64) * (size_t)dnum * LK * n);
+    u64 *acc = (u64 *)malloc(sizeof(u64) * (size_t)2 * LK * n);
+    u64 *ks = (u64 *)malloc(sizeof(u64) * (size_t)2 * L * n);
+    u64 *rot0 = (u64 *)malloc(sizeof(u64) * (size_t)L * n);
+    u64 *rot1 = (u64 *)malloc(sizeof(u64) * (size_t)L * n);
+    for (int b = 0; b < batch; ++b) {
+        const u64 *c0 = ct + (size_t)b * 2 * L * n, *c1 = c0 + (size_t)L * n;
+        for (int r = 0; r < nkeys; ++r) {
+            oracle_automorph_ntt(c1, rot1, L, 1, n, galois[r]);
+            modup_one(rot1, dig, mods, tabs, L, K, alpha, n);
+            inner_one(dig, keys[r], 1, acc, mods, L, K, alpha, n);
+            moddown_one(acc, ks, mods, tabs, L, K, n);
+            oracle_automorph_ntt(c0, rot0, L, 1, n, galois[r]);
+            u64 *o = out + ((size_t)r * batch + b) * 2 * L * n;
+            for (int i = 0; i < L; ++i)
+                for (int k = 0; k < n; ++k) {
+                    size_t at = (size_t)i * n + k;
+                    o[at] = addmod(rot0[at], ks[at], mods[i]);
+                    o[(size_t)L * n + at] = ks[(size_t)L * n + at];
+                }
+        }
+    }
+    free(dig); free(acc); free(ks); free(rot0); free(rot1);
+    ptabs_free(tabs, LK);
+}
+
 /* ------------------------------------------------------------------ */
 /* R9: rescale                                                         */
 /* ------------------------------------------------------------------ */

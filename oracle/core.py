@@ -47,6 +47,7 @@ def _lib():
                                        C.c_int, C.c_int, C.c_int]
         L.oracle_rotate.argtypes = [_u64p, C.POINTER(_u64p), _u64p, C.c_int, _u64p,
                                     _u64p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.oracle_rotate_unhoisted.argtypes = L.oracle_rotate.argtypes
         L.oracle_rescale.argtypes = [_u64p, _u64p, _u64p, C.c_int, C.c_int, C.c_int]
         L.oracle_mul_relin_rescale.argtypes = [_u64p, _u64p, _u64p, _u64p, _u64p,
                                                C.c_int, C.c_int, C.c_int, C.c_int,
@@ -251,6 +252,19 @@ def rotate(ct, keys, galois, mods, L, K, alpha):
     m, pm = _u(mods)
     _lib().oracle_rotate(pc, karr, pg, len(keys), out.ctypes.data_as(_u64p), pm, L, K,
                          alpha, B, n)
+    return out
+
+
+def rotate_unhoisted(ct, keys, galois, mods, L, K, alpha):
+    """ct[B][2][L][n] -> out[nkeys][B][2][L][n], automorphism before the key switch."""
+    c, pc = _u(ct)
+    B, n = c.shape[0], c.shape[-1]
+    kept, karr = _ptr_array(keys)
+    g, pg = _u(galois)
+    out = np.zeros((len(keys), B, 2, L, n), dtype=np.uint64)
+    m, pm = _u(mods)
+    _lib().oracle_rotate_unhoisted(pc, karr, pg, len(keys), out.ctypes.data_as(_u64p), pm, L, K,
+                                   alpha, B, n)
     return out
 
 

@@ -347,6 +347,28 @@ def test_hoisted_rotations_small_digits(orc):
         assert np.max(np.abs(sch.decrypt_slots(out[i, 0]) - rot_left(z, r))) < 1e-8
 
 
+def test_unhoisted_rotation_order_decrypts_and_differs_in_low_bits(orc):
+    """The automorphism-first order (no hoisting) decrypts to the same slot rotation as the hoisted
+    order, with different low bits (the approximate ModUp does not commute with phi_g)."""
+    p = Params(5, 2, 2)
+    sch = Scheme(orc, p, SEED + 5)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 23).numpy()
+    ct = sch.encrypt_slots(z)
+    rs = [1, 3]
+    keys = [sch.keygen_galois(galois_for_rotation(r)) for r in rs]
+    gal = np.array([galois_for_rotation(r) for r in rs], dtype=np.uint64)
+    a = orc.rotate_unhoisted(ct[None], keys, gal, sch.mods, p.L, p.K, p.alpha)
+    h = orc.rotate(ct[None], keys, gal, sch.mods, p.L, p.K, p.alpha)
+    for i, r in enumerate(rs):
+        assert np.max(np.abs(sch.decrypt_slots(a[i, 0]) - rot_left(z, r))) < 1e-8
+    assert not np.array_equal(a, h)
+    # with g = 1 there is no automorphism, so the two orders coincide
+    k1 = sch.keygen_galois(1)
+    one = np.array([1], dtype=np.uint64)
+    assert np.array_equal(orc.rotate_unhoisted(ct[None], [k1], one, sch.mods, p.L, p.K, p.alpha),
+                          orc.rotate(ct[None], [k1], one, sch.mods, p.L, p.K, p.alpha))
+
+
 @pytest.mark.slow
 def test_rotation_and_relin_config3_params(orc):
     """Layer-shaped parameters: 112 primes, alpha = 8, 8 special primes."""
