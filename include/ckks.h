@@ -69,7 +69,8 @@ enum ckks_op {
     CKKS_OP_ROTATE = 4,
     CKKS_OP_RESCALE = 5,
     CKKS_OP_MUL_RELIN_RESCALE = 6,
-    CKKS_OP_BSGS = 7
+    CKKS_OP_BSGS = 7,
+    CKKS_OP_ROTATE_UNHOISTED = 8
 };
 
 /* Pointwise operation codes for ckks_pointwise. */
@@ -244,6 +245,20 @@ int ckks_keyswitch(const ckks_ctx *ctx, const uint64_t *d, const uint64_t *key,
 int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
                 const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
                 ckks_stream_t stream);
+
+/* a8, the other order: Rot_g(c) = (phi_g(c0) + KS_0, KS_1) with KS the key
+ * switch of phi_g(c1) -- the automorphism applied before ModUp, one ModUp per
+ * key (no hoisting) -- using the same Galois keys as ckks_rotate.  This is the
+ * textbook order without hoisting; the pages fix neither order (Galois
+ * rotation: Kestrel engine write-up, section 3 table; rotation = transform +
+ * key switch: EncryptedLLM GPU article, section 2.5).  Its low bits differ
+ * from ckks_rotate's (the approximate
+ * ModUp does not commute with phi_g); both decrypt to the rotated slots.
+ * Arguments, layouts and errors as ckks_rotate; ws:
+ * ckks_workspace_bytes(CKKS_OP_ROTATE_UNHOISTED, batch, 0). */
+int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
+                          const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
+                          ckks_stream_t stream);
 
 /* ---------------------------------------------------------------- a10: rescale */
 

@@ -16,6 +16,7 @@ N = 2048
 
 PW = {"mul": 0, "add": 1, "sub": 2}
 OP_MODUP, OP_MODDOWN, OP_KEYSWITCH, OP_ROTATE, OP_RESCALE, OP_MRR, OP_BSGS = 1, 2, 3, 4, 5, 6, 7
+OP_ROTATE_UNHOISTED = 8
 
 
 def primes(count, n=N):
@@ -206,6 +207,21 @@ class Context:
         ws, wp = self._ws(ws, OP_ROTATE, B, nk)
         check("ckks_rotate", lib().ckks_rotate(self._h, _ptr(ct, "ct"), kp, gp, nk, _ptr(out, "out"),
                                                B, wp, _stream(ct)))
+        return out
+
+    def rotate_unhoisted(self, ct, keys, galois, out=None, ws=None):
+        """Rotations in the other order: phi_g before ModUp, one ModUp per key."""
+        B = ct.shape[0]
+        nk = len(keys)
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", (self.dnum, 2, self.L + self.K, self.n)).value
+                                        for k in keys])
+        gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
+        out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_ROTATE_UNHOISTED, B)
+        check("ckks_rotate_unhoisted",
+              lib().ckks_rotate_unhoisted(self._h, _ptr(ct, "ct"), kp, gp, nk, _ptr(out, "out"), B, wp,
+                                          _stream(ct)))
         return out
 
     # ------------------------------------------------------------ a9/a10

@@ -10,6 +10,7 @@ namespace ckks {
 
 size_t keyswitch_ws_bytes(const ckks_ctx *ctx, int batch);
 size_t rotate_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys);
+size_t rotate_unhoisted_ws(const ckks_ctx *ctx, int batch);
 
 static int check_batch(int batch)
 {
@@ -282,6 +283,7 @@ extern "C" size_t ckks_workspace_bytes(const ckks_ctx *ctx, int op, int batch, i
     case CKKS_OP_MODDOWN: return moddown_ws_bytes(ctx, batch);
     case CKKS_OP_KEYSWITCH: return keyswitch_ws_bytes(ctx, batch);
     case CKKS_OP_ROTATE: return rotate_ws_bytes(ctx, batch, aux);
+    case CKKS_OP_ROTATE_UNHOISTED: return rotate_unhoisted_ws(ctx, batch);
     case CKKS_OP_RESCALE: return rescale_ws_bytes(batch);
     case CKKS_OP_MUL_RELIN_RESCALE: return mrr_ws(ctx, batch);
     case CKKS_OP_BSGS: {
@@ -360,6 +362,64 @@ extern "C" int ckks_automorph(const ckks_ctx *ctx, const uint64_t *in, uint64_t 
     CKKS_TRY(set_device(ctx));
     automorph_kernel<<<(unsigned)rows, 256, 0, (cudaStream_t)stream>>>(in, out, galois & (2u * kN - 1u));
     CKKS_CHECK_LAUNCH("automorph_kernel");
+    return CKKS_OK;
+}
+
+namespace ckks {
+size_t rotate_unhoisted_ws(const ckks_ctx *ctx, int batch)
+{
+    return limbs_bytes((size_t)batch * 2 * ctx->L) + rotate_ws_bytes(ctx, batch, 1);
+}
+}  // namespace ckks
+
+// The other rotation order: for each key, phi_g of the whole ciphertext batch (one automorphism
+// launch over both components), then a key switch of the rotated c1 with the Galois key (ModUp,
+// inner product without a gather, ModDown) whose final store adds the rotated c0.
+extern "C" int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
+                                     const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
+                                     ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (nkeys < 0) return set_error(CKKS_EINVAL, "negative key count");
+    if (batch == 0 || nkeys == 0) return CKKS_OK;
+    if (!keys || !galois) return set_error(CKKS_EINVAL, "null key or galois array");
+    for (int r = 0; r < nkeys; ++r) {
+        CKKS_TRY(check_ptr(keys[r], "keys[r]"));
+        if ((galois[r] & 1u) == 0) return set_error(CKKS_EINVAL, "galois element must be odd");
+    }
+    if (batch > 32767) return set_error(CKKS_EUNSUPPORTED, "batch above 32767");
+    CKKS_TRY(check_ptr(ct, "ct"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    void *w;
+    CKKS_TRY(resolve_ws(const_cast<ckks_ctx *>(ctx), ws, rotate_unhoisted_ws(ctx, batch), &w));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int L = ctx->L, LK = L + ctx->K;
+    const size_t ct_elems = (size_t)2 * L * kN;
+    Carve c(w);
+    u64 *rct = c.take<u64>((size_t)batch * 2 * L * kN);
+    u64 *digits = c.take<u64>((size_t)batch * ctx->dnum * LK * kN);
+    u64 *acc = c.take<u64>((size_t)batch * 2 * LK * kN);
+    void *scratch = c.base + c.off;
+    for (int r = 0; r < nkeys; ++r) {
+        const u32 g = galois[r] & (2u * kN - 1u);
+        automorph_kernel<<<(unsigned)((size_t)batch * 2 * L), 256, 0, s>>>(ct, rct, g);
+        CKKS_CHECK_LAUNCH("automorph_kernel");
+        CKKS_TRY(modup_stage(ctx, rct + (size_t)L * kN, nullptr, ct_elems, digits, batch, scratch, s));
+        KeyList kl{};
+        kl.key[0] = keys[r];
+        kl.galois[0] = 1;
+        CKKS_TRY(key_inner_stage(ctx, digits, kl, batch, true, acc, batch, s));
+        DownExtra ex;
+        ex.kind = 1;
+        ex.ct = rct;
+        ex.ct_bstride = ct_elems;
+        ex.ct_mod = batch;
+        ex.per = batch;
+        ex.gal[0] = 1;
+        CKKS_TRY(moddown_stage(ctx, acc, out + (size_t)r * batch * ct_elems, batch, ex, scratch, s));
+    }
     return CKKS_OK;
 }
 

@@ -446,3 +446,31 @@ def test_bounded_wait_expiry_is_reported_and_recoverable(orc):
     q = np.array(ctx.q, dtype=np.uint64)
     x = _res((2, 4, N), q, 400)
     assert_bits_equal(host(ctx.ntt_fwd(dev(x))), orc.ntt_fwd(x, q), "ntt_fwd after the expiry")
+
+
+def test_unhoisted_rotation_order(orc):
+    """The automorphism-before-ModUp order: bit-exact against the oracle and decrypting to the
+    rotated slots (small scheme), and bit-exact with 20-prime digits on the tensor-core path."""
+    p = Params(5, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 9)
+    zs = [synth.uniform_real((SLOTS,), -1, 1, SEED, 90 + i).numpy() for i in range(2)]
+    cts = np.stack([sch.encrypt_slots(z) for z in zs])
+    rs = [1, 5]
+    keys = [sch.keygen_galois(galois_for_rotation(r)) for r in rs]
+    gal = [galois_for_rotation(r) for r in rs]
+    out = host(ctx.rotate_unhoisted(dev(cts), [dev(k) for k in keys], gal))
+    want = orc.rotate_unhoisted(cts, keys, np.array(gal, dtype=np.uint64), sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(out, want, "rotate_unhoisted")
+    for i, r in enumerate(rs):
+        for b in range(2):
+            assert np.max(np.abs(sch.decrypt_slots(out[i, b]) - rot_left(zs[b], r))) < 1e-8
+    p2 = Params(40, 20, 20)
+    ctx2 = ctx_for(p2)
+    mods = np.array(ctx2.mods, dtype=np.uint64)
+    ct = _res((2, 2, 40, N), mods[:40], 91)
+    key = _res((2, 2, 60, N), mods, 92)
+    got = host(ctx2.rotate_unhoisted(dev(ct), [dev(key)], [25]))
+    ctx2.device_status()
+    assert_bits_equal(got, orc.rotate_unhoisted(ct, [key], np.array([25], dtype=np.uint64), mods, 40, 20, 20),
+                      "rotate_unhoisted, tensor-core conversion")
