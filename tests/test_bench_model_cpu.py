@@ -1,0 +1,37 @@
+"""The algorithmic-work model behind the key-switch roofline fractions, checked
+against an independent derivation of the same counts (the per-configuration
+totals worked out by hand from the algorithm: hybrid key switching with
+contiguous digits, n = 2048, 11 264 modular products per limb transform)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_boot_rotation_counts():
+    up, inner, down = bench.ks_work_keyswitch_parts(2100, 60, 60)
+    # ModUp of one ciphertext: 35 digits x 60 sources x 2100 targets x 2048 multiply-adds
+    assert up["mac"] == 35 * 60 * 2100 * 2048
+    assert up["mm"] + up["mac"] == pytest.approx(9.89e9, rel=0.01)
+    assert inner["mm"] + inner["mac"] + down["mm"] + down["mac"] == pytest.approx(8.88e8, rel=0.01)
+    mm, mac, _ = bench.ks_work_rotation(2100, 60, 60, 1, 4)
+    assert mm + mac == pytest.approx(1.344e10, rel=0.01)
+
+
+def test_layer_and_bsgs_counts():
+    mm, mac, _ = bench.ks_work_mrr(112, 8, 8, 1)
+    assert mm + mac == pytest.approx(6.30e7, rel=0.02)
+    mm, mac, _ = bench.ks_work_bsgs(112, 8, 8, 1, 32, 32)
+    assert mm + mac == pytest.approx(2.78e9, rel=0.02)
+
+
+def test_ntt_launch_bytes_and_products():
+    bytes_, mm = bench.ntt_launch_work(2100)
+    assert bytes_ == 33600 * 2 * 2048 * 8 + 2100 * 2048 * 16
+    assert mm == 33600 * 1024 * 11
