@@ -80,8 +80,8 @@ enum ckks_pointwise_op { CKKS_PW_MUL = 0, CKKS_PW_ADD = 1, CKKS_PW_SUB = 2 };
 
 /* Host-only.  Writes the first `count` primes q = 1 (mod 2n), 2^59 < q < 2^60,
  * scanning downward from 2^60 (largest first).  The pages ask for 60-bit
- * NTT-friendly primes (Kestrel engine write-up, section 2 "wall 2": "112
- * 60-bit primes"); the scan order is this library's reading.
+ * NTT-friendly primes (Kestrel engine write-up, section 2 "wall 2", a chain of
+ * 112 of them); the scan order is this library's reading.
  * Returns CKKS_EINVAL if out is NULL, n is not a power of two in [2, 2^16]
  * or count < 0, CKKS_EUNSUPPORTED if the interval runs out of primes. */
 int ckks_primes(int n, int count, uint64_t *out);
