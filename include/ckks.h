@@ -252,8 +252,8 @@ int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *
  * textbook order without hoisting; the pages fix neither order (Galois
  * rotation: Kestrel engine write-up, section 3 table; rotation = transform +
  * key switch: EncryptedLLM GPU article, section 2.5).  Its low bits differ
- * from ckks_rotate's (the approximate
- * ModUp does not commute with phi_g); both decrypt to the rotated slots.
+ * from ckks_rotate's (the approximate ModUp does not commute with phi_g);
+ * both decrypt to the rotated slots.
  * Arguments, layouts and errors as ckks_rotate; ws:
  * ckks_workspace_bytes(CKKS_OP_ROTATE_UNHOISTED, batch, 0). */
 int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
