@@ -310,7 +310,7 @@ def test_bsgs_banded_decrypts(orc):
         assert np.max(np.abs(sch.decrypt_slots(y[i], sc) - M @ xs[i])) < 1e-8
 
 
-@pytest.mark.parametrize("bb,gg", [(3, 5), (1, 2), (2, 1)])
+@pytest.mark.parametrize("bb,gg", [(3, 5), (1, 2), (2, 1), (33, 2)])
 def test_bsgs_shapes(orc, bb, gg):
     p = Params(5, 2, 2)
     ctx = ctx_for(p)
