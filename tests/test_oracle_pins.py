@@ -7,7 +7,6 @@ check is chosen so that a plausible slip (a wrong twiddle or index, a dropped
 term, a sign, a transposed operand) fails at least one of them.
 """
 import random
-from fractions import Fraction
 
 import numpy as np
 import pytest

@@ -12,7 +12,6 @@ the other tests.
 """
 import ctypes as C
 
-import numpy as np
 import pytest
 import torch
 
