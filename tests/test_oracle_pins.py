@@ -163,6 +163,32 @@ def test_convolution_theorem(orc, n):
     assert np.array_equal(prod[0], orc.negacyclic_mul(a[0], b[0], q[0]))
 
 
+def test_pointwise_sum_and_difference_by_linearity(orc):
+    """The NTT is linear, so evaluation-domain sums and differences come back
+    as coefficient sums and differences mod q, taken here with Python integers.
+    Operands include 0 and q - 1 so both wrap directions are hit; a swapped
+    operand in 'sub' flips every nonzero difference."""
+    mods = orc.gen_primes(N, 3)
+    a = _rand_res((2, 3, N), mods, 6)
+    b = _rand_res((2, 3, N), mods, 7)
+    for l, m in enumerate(mods):
+        a[0, l, :4] = [0, int(m) - 1, 0, int(m) - 1]
+        b[0, l, :4] = [0, int(m) - 1, int(m) - 1, 0]
+    fa, fb = orc.ntt_fwd(a, mods), orc.ntt_fwd(b, mods)
+    s = orc.ntt_inv(orc.pointwise("add", fa, fb, mods), mods)
+    d = orc.ntt_inv(orc.pointwise("sub", fa, fb, mods), mods)
+    for l, m in enumerate(int(v) for v in mods):
+        for bi in range(2):
+            av = [int(v) for v in a[bi, l]]
+            bv = [int(v) for v in b[bi, l]]
+            assert [int(v) for v in s[bi, l]] == [(x + y) % m for x, y in zip(av, bv)]
+            assert [int(v) for v in d[bi, l]] == [(x - y) % m for x, y in zip(av, bv)]
+    # directly in the evaluation domain: every output is a reduced residue
+    for op in ("add", "sub", "mul"):
+        r = orc.pointwise(op, fa, fb, mods)
+        assert all(int(r[:, l].max()) < int(m) for l, m in enumerate(mods))
+
+
 # ------------------------------------------------------------------ automorphism
 def test_automorph_coeff_monomials(orc):
     q = int(orc.gen_primes(N, 1)[0])
