@@ -32,11 +32,14 @@
  *     the first L are the ciphertext primes, the next K the special primes.
  *  R2 psi: the smallest primitive 2n-th root of unity mod q.
  *  R3 NTT: ahat[k] = sum_j a_j psi^(j (2 brv(k) + 1)), bit-reversed order.
+ *  R4 automorphism: X -> X^g; slot j sits at zeta^(5^j), so g = 5^r rotates
+ *     the slots left by r.
  *  R5 hybrid key switching with contiguous digits, approximate ModUp,
- *     floor ModDown, key b_j = -a_j s + e_j + g_j s'.
+ *     floor ModDown.
+ *  R6 keys: b_j = -a_j s + e_j + g_j s', stored [dnum][2][L+K][n].
  *  R7 rotation: ModUp(c1) first, the automorphism is applied to the
  *     extended digits, then inner product, ModDown, plus phi_g(c0).
- *  R9 rescale: floor form (c - [c]_{q_l}) / q_l.
+ *  R8 rescale: floor form (c - [c]_{q_l}) / q_l.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -586,7 +589,7 @@ void oracle_rotate_unhoisted(const u64 *ct /*[B][2][L][n]*/, const u64 *const *k
 }
 
 /* ------------------------------------------------------------------ */
-/* R9: rescale                                                         */
+/* R8: rescale                                                         */
 /* ------------------------------------------------------------------ */
 
 /* ct[B][2][l+1][n] -> out[B][2][l][n]: c'_i = (c_i - NTT_{q_i}([c]_{q_l})) q_l^{-1}.
@@ -736,7 +739,7 @@ static void small_to_ntt(const i64 *v, u64 *out, const u64 *mods,
     }
 }
 
-/* Switching key from s' to s (R5):  key[j][0] = -a_j s + e_j + g_j s',
+/* Switching key from s' to s (R6):  key[j][0] = -a_j s + e_j + g_j s',
  * key[j][1] = a_j over all L+K primes, NTT domain.  g_j is P on the limbs of
  * digit j and 0 elsewhere (0 on every special prime).
  * s: ternary secret coefficients [n]; sprime_ntt: s' as NTT residues
