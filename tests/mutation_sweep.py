@@ -1,0 +1,196 @@
+"""Mutation sweep over the CPU oracle: plants one plausible slip at a time in
+a temporary copy of `oracle/` and runs the pin suite (test_oracle_pins.py)
+against that copy.  A pin set that is independent of the oracle must fail on
+every slip; a slip that passes every pin would mark a step left unpinned.
+
+Each entry is (what the slip is, file, text, replacement, which occurrence,
+the pin expected to catch it).  The replacement is applied to the copy only;
+the repository's oracle is never touched.
+
+    python tests/mutation_sweep.py            # every slip, full pin suite each
+    python tests/mutation_sweep.py 0 15 21    # chosen slips
+    python tests/mutation_sweep.py --targeted # run only each slip's own pin
+"""
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+C = "ckks_oracle.c"
+
+MUTATIONS = [
+    ("NTT twiddle index", C,
+     "u64 w = t->fw[m + i];", "u64 w = t->fw[i + 1];", 0,
+     "test_ntt_of_monomials_is_the_evaluation_vector"),
+    ("INTT without n^-1", C,
+     "a[j] = mulmod(a[j], t->n_inv, q);", "a[j] = a[j] % q;", 0,
+     "test_ntt_roundtrip_identity"),
+    ("psi: largest root instead of smallest", C,
+     "if (cur < best) best = cur;", "if (cur > best) best = cur;", 0,
+     "test_psi_is_smallest_primitive_root"),
+    ("prime scan steps by 4n", C,
+     "        c -= m;\n    }", "        c -= 2 * m;\n    }", 0,
+     "test_primes_follow_the_scan_rule"),
+    ("Miller-Rabin squaring loop one short", C,
+     "for (int r = 1; r < s; ++r) {", "for (int r = 2; r < s; ++r) {", 0,
+     "test_primes_follow_the_scan_rule"),
+    ("NTT-domain automorphism without bit reversal", C,
+     "return (int)bitrev((e - 1) / 2, lg);", "return (int)((e - 1) / 2);", 0,
+     "test_automorph_ntt_permutation_matches_coefficients"),
+    ("coefficient automorphism drops the X^n = -1 sign", C,
+     "else out[e - n] = submod(out[e - n], in[j], q);",
+     "else out[e - n] = addmod(out[e - n], in[j], q);", 0,
+     "test_automorph_coeff_monomials"),
+    ("basis conversion skips the q-hat inverse", C,
+     "mulmod(x[(size_t)i * n + k], hat_inv[i], src[i])", "(x[(size_t)i * n + k] % src[i])", 0,
+     "test_basis_conversion_crt_identity"),
+    ("basis conversion: q-hat reduced by the wrong prime", C,
+     "pt = mulmod(pt, src[i2] % dst[t], dst[t]);", "pt = mulmod(pt, src[i2] % src[i], dst[t]);", 0,
+     "test_basis_conversion_crt_identity"),
+    ("ModUp leaves the digit's own limbs empty", C,
+     "for (int t = lo; t < hi; ++t)\n            memcpy(dj",
+     "for (int t = lo; t < lo; ++t)\n            memcpy(dj", 0,
+     "test_modup_crt_identity"),
+    ("ModUp converts NTT values (no INTT)", C,
+     "for (int l = 0; l < L; ++l) ntt_inv_one(coef", "for (int l = 0; l < 0; ++l) ntt_inv_one(coef", 0,
+     "test_modup_crt_identity"),
+    ("ModUp output left in the coefficient domain", C,
+     "ntt_fwd_one(row, &tabs[dst_idx[c]], n);", "(void)row;", 0,
+     "test_modup_crt_identity"),
+    ("key inner product: key halves swapped", C,
+     "key[(((size_t)j * 2 + c) * LK + t) * n + k];",
+     "key[(((size_t)j * 2 + (1 - c)) * LK + t) * n + k];", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("key inner product without the automorphism", C,
+     "digits[((size_t)j * LK + t) * n + src[k]];", "digits[((size_t)j * LK + t) * n + k];", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("key inner product drops the last digit", C,
+     "for (int j = 0; j < dnum; ++j) {\n                    u64 d",
+     "for (int j = 0; j + 1 < dnum; ++j) {\n                    u64 d", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("ModDown without P^-1", C,
+     "mulmod(submod(a[(size_t)i * n + k], ci[k], mods[i]), pinv[i], mods[i]);",
+     "submod(a[(size_t)i * n + k], ci[k], mods[i]);", 0,
+     "test_moddown_floor_identity"),
+    ("ModDown adds the conversion", C,
+     "mulmod(submod(a[(size_t)i * n + k], ci[k], mods[i]), pinv[i], mods[i]);",
+     "mulmod(addmod(a[(size_t)i * n + k], ci[k], mods[i]), pinv[i], mods[i]);", 0,
+     "test_moddown_floor_identity"),
+    ("ModDown subtracts coefficients from NTT values", C,
+     "ntt_fwd_one(ci, &tabs[i], n);", "(void)ci;", 0,
+     "test_moddown_floor_identity"),
+    ("hoisted rotation adds c0 unrotated", C,
+     "o[at] = addmod(rot0[at], ks[at], mods[i]);", "o[at] = addmod(c0[at], ks[at], mods[i]);", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("unhoisted rotation adds c0 unrotated", C,
+     "o[at] = addmod(rot0[at], ks[at], mods[i]);", "o[at] = addmod(c0[at], ks[at], mods[i]);", 1,
+     "test_unhoisted_rotation_order_decrypts_and_differs_in_low_bits"),
+    ("unhoisted rotation applies the automorphism twice", C,
+     "inner_one(dig, keys[r], 1, acc", "inner_one(dig, keys[r], galois[r], acc", 0,
+     "test_unhoisted_rotation_order_decrypts_and_differs_in_low_bits"),
+    ("rescale by the wrong prime's inverse on limb 0", C,
+     "u64 inv = invmod(mods[l] % qi, qi);",
+     "u64 inv = invmod(mods[l] % qi, qi); inv = i ? inv : invmod(mods[l - 1] % qi, qi);", 0,
+     "test_rescale_is_exact_floor"),
+    ("rescale subtracts the wrong way", C,
+     "row[k] = mulmod(submod(in[(size_t)i * n + k], row[k], qi), inv, qi);",
+     "row[k] = mulmod(submod(row[k], in[(size_t)i * n + k], qi), inv, qi);", 0,
+     "test_rescale_is_exact_floor"),
+    ("tensor product drops a cross term", C,
+     "addmod(mulmod(a0[at], b1[at], q), mulmod(a1[at], b0[at], q), q);",
+     "mulmod(a0[at], b1[at], q);", 0,
+     "test_rotation_and_relin_config3_params"),
+    ("tensor product: d2 from a transposed operand", C,
+     "d[2 * Ln + at] = mulmod(a1[at], b1[at], q);", "d[2 * Ln + at] = mulmod(a1[at], b0[at], q);", 0,
+     "test_rotation_and_relin_config3_params"),
+    ("relinearisation drops the second key-switch output", C,
+     "c[Ln + at] = addmod(d[Ln + at], ks[Ln + at], mods[i]);", "c[Ln + at] = d[Ln + at];", 0,
+     "test_rotation_and_relin_config3_params"),
+    ("BSGS giant step rotates by g instead of bb*g", C,
+     "u64 gal = galois_power((u64)bb * g, n);", "u64 gal = galois_power((u64)g, n);", 0,
+     "test_bsgs_banded_matvec"),
+    ("BSGS plaintext diagonals transposed", C,
+     "diags + ((size_t)g * bb + r) * Ln;", "diags + ((size_t)r * gg + g) * Ln;", 0,
+     "test_bsgs_banded_matvec"),
+    ("BSGS baby step rotation off by one", C,
+     "galb[r - 1] = galois_power((u64)r, n);", "galb[r - 1] = galois_power((u64)r - 1, n);", 0,
+     "test_bsgs_banded_matvec"),
+    ("key generation puts P on the next digit's first limb", C,
+     "if (t >= lo && t < hi) {\n                gj = 1;", "if (t >= lo && t <= hi) {\n                gj = 1;", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("key generation sign of a*s", C,
+     "u64 bv = submod(e_ntt[at], mulmod(av, s_ntt[at], q), q);",
+     "u64 bv = addmod(e_ntt[at], mulmod(av, s_ntt[at], q), q);", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("encryption sign of a*s", C,
+     "u64 v = submod(e_ntt[at], mulmod(a[at], s_ntt[at], q), q);",
+     "u64 v = addmod(e_ntt[at], mulmod(a[at], s_ntt[at], q), q);", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("Galois secret built with the wrong element", C,
+     "oracle_automorph_coeff(tmp, out + (size_t)l * n, mods[l], n, g);",
+     "oracle_automorph_coeff(tmp, out + (size_t)l * n, mods[l], n, (g * g) % (2 * (u64)n));", 0,
+     "test_rotation_decrypts_to_slot_rotation_config1"),
+    ("schoolbook product wraps cyclically", C,
+     "else out[k - n] = submod(out[k - n], p, q);", "else out[k - n] = addmod(out[k - n], p, q);", 0,
+     "test_negacyclic_schoolbook_tiny"),
+    ("encoder conjugates the slots", "encoding.py",
+     "idx = _angle_matrix(n, -1)", "idx = _angle_matrix(n, 1)", 0,
+     "test_encode_decode_roundtrip_and_rotation"),
+    ("modular addition wraps one too high", C,
+     "static u64 addmod(u64 a, u64 b, u64 q) { return (a + b) % q; }",
+     "static u64 addmod(u64 a, u64 b, u64 q) { u64 s = a + b; return s >= q ? s - q + 1 : s; }", 0,
+     "test_fast_ntt_equals_definition"),
+]
+
+
+def plant(index, dest):
+    """Copy oracle/ into dest with slip `index` applied; returns the copy's path."""
+    name, fname, old, new, occ, _ = MUTATIONS[index]
+    copy = os.path.join(dest, "oracle")
+    shutil.copytree(os.path.join(ROOT, "oracle"), copy,
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    path = os.path.join(copy, fname)
+    with open(path) as f:
+        text = f.read()
+    parts = text.split(old)
+    if len(parts) <= occ + 1:
+        raise ValueError("slip %r: text not found in %s" % (name, fname))
+    text = old.join(parts[:occ + 1]) + new + old.join(parts[occ + 1:])
+    with open(path, "w") as f:
+        f.write(text)
+    return copy
+
+
+def run(index, targeted=False, timeout=1800):
+    """Run the pins against a copy with slip `index`; return (caught, first failure)."""
+    with tempfile.TemporaryDirectory(prefix="oracle_slip_") as d:
+        plant(index, d)
+        cmd = [sys.executable, "-m", "pytest", PINS, "-x", "-q", "--import-mode=append",
+               "-p", "no:cacheprovider"]
+        if targeted:
+            cmd += ["-k", MUTATIONS[index][5]]
+        # `python -m pytest` puts its working directory first on sys.path, so
+        # `import oracle` finds the planted copy ahead of the repository's one
+        r = subprocess.run(cmd, cwd=d, capture_output=True, text=True, timeout=timeout)
+    failed = [ln.split("::")[-1].split(" - ")[0] for ln in r.stdout.splitlines()
+              if ln.startswith(("FAILED", "ERROR"))]
+    return r.returncode != 0, (failed[0] if failed else "")
+
+
+def main(argv):
+    targeted = "--targeted" in argv
+    picks = [int(a) for a in argv if not a.startswith("--")] or range(len(MUTATIONS))
+    missed = 0
+    for i in picks:
+        caught, first = run(i, targeted)
+        missed += not caught
+        print("%2d  %-7s %-55s %s" % (i, "caught" if caught else "MISSED", MUTATIONS[i][0], first),
+              flush=True)
+    return 1 if missed else 0
+
+
+if __name__ == "__main__":
+    sys.exit(main(sys.argv[1:]))
