@@ -40,6 +40,11 @@
  *  R7 rotation: ModUp(c1) first, the automorphism is applied to the
  *     extended digits, then inner product, ModDown, plus phi_g(c0).
  *  R8 rescale: floor form (c - [c]_{q_l}) / q_l.
+ *  R14 bootstrapping steps (Kestrel engine write-up, the boot profile in
+ *     section 5.3, names them; the forms are the textbook ones): modraise is
+ *     the centred lift of each coefficient from q_0..q_{l-1} to the longer
+ *     chain; conj_extract gives (ct + conj ct, X^{n/2}(conj ct - ct));
+ *     restore_merge gives re + X^{n/2} im.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -721,6 +726,162 @@ void oracle_bsgs(const u64 *x, const u64 *diags, const u64 *const *baby_keys,
         oracle_rescale(acc, y + (size_t)b * 2 * (L - 1) * n, mods, L, 1, n);
     }
     free(baby); free(inner); free(acc); free(rot); free(galb);
+}
+
+/* ------------------------------------------------------------------ */
+/* R14: the bootstrapping steps around the two linear transforms       */
+/* ------------------------------------------------------------------ */
+
+/* Multiplication by the monomial X^e, 0 <= e < 2n, in Z_q[X]/(X^n + 1),
+ * coefficient domain, one limb: X^j goes to X^{j+e}, negated once for every
+ * time the exponent passes n (X^n = -1). */
+static void monomial_coeff(const u64 *in, u64 *out, u64 q, int n, int e)
+{
+    for (int j = 0; j < n; ++j) {
+        int t = j + e;
+        int neg = 0;
+        while (t >= n) { t -= n; neg ^= 1; }
+        out[t] = neg ? submod(0, in[j], q) : in[j] % q;
+    }
+}
+
+/* x[batch][limbs][n] NTT domain -> X^e * x, NTT domain: INTT, the
+ * coefficient shift above, NTT. */
+void oracle_mul_monomial(const u64 *in, u64 *out, const u64 *mods, int limbs,
+                         int batch, int n, int e)
+{
+    ptab *tabs = ptabs_make(mods, limbs, n);
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < batch; ++b)
+        for (int l = 0; l < limbs; ++l) {
+            size_t off = ((size_t)b * limbs + l) * n;
+            u64 *tmp = (u64 *)malloc(sizeof(u64) * n);
+            memcpy(tmp, in + off, sizeof(u64) * n);
+            ntt_inv_one(tmp, &tabs[l], n);
+            monomial_coeff(tmp, out + off, mods[l], n, e);
+            ntt_fwd_one(out + off, &tabs[l], n);
+            free(tmp);
+        }
+    ptabs_free(tabs, limbs);
+}
+
+/* ModRaise: polynomials x[P][l][n] over q_0..q_{l-1} (NTT domain) ->
+ * out[P][Lf][n] over q_0..q_{Lf-1} (NTT domain), Lf >= l.  Each coefficient
+ * is read as the centred integer X in (-Q/2, Q/2], Q = q_0 ... q_{l-1}, and
+ * X is reduced modulo every prime of the longer chain.
+ *
+ * X is found in Garner's mixed-radix form X = d_0 + d_1 q_0 + d_2 q_0 q_1 +
+ * ..., with digits d_i in [0, q_i): d_i = (...((x_i - d_0) q_0^{-1} - d_1)
+ * q_1^{-1} ... - d_{i-1}) q_{i-1}^{-1} mod q_i.  H = (Q - 1) / 2 has residue
+ * (q_i - 1) / 2 at every q_i (2H = -1 mod q_i); X > H is decided by comparing
+ * the two digit strings from the most significant digit down, and in that
+ * case Q is subtracted.  X mod p is evaluated from the digits by Horner's
+ * rule.  Only word-size modular arithmetic is involved. */
+void oracle_modraise(const u64 *x, u64 *out, const u64 *mods, int l, int Lf,
+                     int P, int n)
+{
+    ptab *tabs = ptabs_make(mods, Lf, n);
+    /* inv[i][k] = q_k^{-1} mod q_i, k < i */
+    u64 *inv = (u64 *)malloc(sizeof(u64) * (size_t)l * l);
+    for (int i = 0; i < l; ++i)
+        for (int k = 0; k < i; ++k) inv[(size_t)i * l + k] = invmod(mods[k] % mods[i], mods[i]);
+    /* Garner digits of H = (Q - 1) / 2 */
+    u64 *hd = (u64 *)malloc(sizeof(u64) * l);
+    for (int i = 0; i < l; ++i) {
+        u64 t = (mods[i] - 1) / 2;
+        for (int k = 0; k < i; ++k)
+            t = mulmod(submod(t, hd[k] % mods[i], mods[i]), inv[(size_t)i * l + k], mods[i]);
+        hd[i] = t;
+    }
+    /* Q mod p for every prime of the longer chain */
+    u64 *qmod = (u64 *)malloc(sizeof(u64) * Lf);
+    for (int t = 0; t < Lf; ++t) {
+        u64 r = 1 % mods[t];
+        for (int i = 0; i < l; ++i) r = mulmod(r, mods[i] % mods[t], mods[t]);
+        qmod[t] = r;
+    }
+    for (int pi = 0; pi < P; ++pi) {
+        const u64 *src = x + (size_t)pi * l * n;
+        u64 *dst = out + (size_t)pi * Lf * n;
+        u64 *coef = (u64 *)malloc(sizeof(u64) * (size_t)l * n);
+        memcpy(coef, src, sizeof(u64) * (size_t)l * n);
+        #pragma omp parallel for schedule(static)
+        for (int i = 0; i < l; ++i) ntt_inv_one(coef + (size_t)i * n, &tabs[i], n);
+        #pragma omp parallel for schedule(static)
+        for (int k = 0; k < n; ++k) {
+            u64 d[l > 0 ? l : 1];
+            for (int i = 0; i < l; ++i) {
+                u64 t = coef[(size_t)i * n + k];
+                for (int j = 0; j < i; ++j)
+                    t = mulmod(submod(t, d[j] % mods[i], mods[i]), inv[(size_t)i * l + j], mods[i]);
+                d[i] = t;
+            }
+            int neg = 0;
+            for (int i = l - 1; i >= 0; --i)
+                if (d[i] != hd[i]) { neg = d[i] > hd[i]; break; }
+            for (int t = l; t < Lf; ++t) {
+                u64 p = mods[t], r = 0;
+                for (int i = l - 1; i >= 0; --i)
+                    r = addmod(mulmod(r, mods[i] % p, p), d[i] % p, p);
+                if (neg) r = submod(r, qmod[t], p);
+                dst[(size_t)t * n + k] = r;
+            }
+        }
+        #pragma omp parallel for schedule(static)
+        for (int t = l; t < Lf; ++t) ntt_fwd_one(dst + (size_t)t * n, &tabs[t], n);
+        /* below q_l the centred integer keeps its residues */
+        memcpy(dst, src, sizeof(u64) * (size_t)l * n);
+        free(coef);
+    }
+    free(inv); free(hd); free(qmod);
+    ptabs_free(tabs, Lf);
+}
+
+/* conj_extract: ct[B][2][L][n] with slots w -> re, im [B][2][L][n] with
+ * slots 2 Re(w) and 2 Im(w), at the input's scale:
+ *     c* = the conjugate of ct (hoisted rotation by g = 2n - 1, key conj_key),
+ *     re = ct + c*,   im = X^{n/2} (c* - ct).
+ * X^{n/2} multiplies every slot by i (slot j sits at zeta^{5^j} and 5^j = 1
+ * mod 4), so im's slots are i (conj(w) - w) = 2 Im(w). */
+void oracle_conj_extract(const u64 *ct, const u64 *conj_key, u64 *re, u64 *im,
+                         const u64 *mods, int L, int K, int alpha, int batch, int n)
+{
+    const size_t csz = (size_t)2 * L * n;
+    u64 *cj = (u64 *)malloc(sizeof(u64) * csz);
+    u64 *dif = (u64 *)malloc(sizeof(u64) * csz);
+    const u64 g = 2 * (u64)n - 1;
+    for (int b = 0; b < batch; ++b) {
+        const u64 *c = ct + (size_t)b * csz;
+        const u64 *keys[1] = {conj_key};
+        oracle_rotate(c, keys, &g, 1, cj, mods, L, K, alpha, 1, n);
+        for (size_t at = 0; at < csz; ++at) {
+            u64 q = mods[(at / n) % L];
+            re[(size_t)b * csz + at] = addmod(c[at], cj[at], q);
+            dif[at] = submod(cj[at], c[at], q);
+        }
+        for (int comp = 0; comp < 2; ++comp)
+            oracle_mul_monomial(dif + (size_t)comp * L * n,
+                                im + (size_t)b * csz + (size_t)comp * L * n, mods, L, 1, n, n / 2);
+    }
+    free(cj); free(dif);
+}
+
+/* restore_merge: re, im [B][2][L][n] with slots a, b -> re + X^{n/2} im,
+ * whose slots are a + i b. */
+void oracle_restore_merge(const u64 *re, const u64 *im, u64 *out, const u64 *mods,
+                          int L, int batch, int n)
+{
+    const size_t csz = (size_t)2 * L * n;
+    u64 *sh = (u64 *)malloc(sizeof(u64) * csz);
+    for (int b = 0; b < batch; ++b) {
+        for (int comp = 0; comp < 2; ++comp)
+            oracle_mul_monomial(im + (size_t)b * csz + (size_t)comp * L * n,
+                                sh + (size_t)comp * L * n, mods, L, 1, n, n / 2);
+        for (size_t at = 0; at < csz; ++at)
+            out[(size_t)b * csz + at] = addmod(re[(size_t)b * csz + at], sh[at],
+                                               mods[(at / n) % L]);
+    }
+    free(sh);
 }
 
 /* ------------------------------------------------------------------ */

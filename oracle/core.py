@@ -64,6 +64,13 @@ def _lib():
                                      C.c_int, C.c_int]
         L.oracle_decrypt.argtypes = [_u64p, _i64p, _u64p, _u64p, C.c_int, C.c_int]
         L.oracle_negacyclic_mul.argtypes = [_u64p, _u64p, _u64p, C.c_uint64, C.c_int]
+        L.oracle_mul_monomial.argtypes = [_u64p, _u64p, _u64p, C.c_int, C.c_int, C.c_int,
+                                          C.c_int]
+        L.oracle_modraise.argtypes = [_u64p, _u64p, _u64p, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.oracle_conj_extract.argtypes = [_u64p, _u64p, _u64p, _u64p, _u64p, C.c_int,
+                                          C.c_int, C.c_int, C.c_int, C.c_int]
+        L.oracle_restore_merge.argtypes = [_u64p, _u64p, _u64p, _u64p, C.c_int, C.c_int,
+                                           C.c_int]
         L.oracle_num_threads.restype = C.c_int
         L.oracle_set_num_threads.argtypes = [C.c_int]
         L.oracle_set_num_threads.restype = None
@@ -301,6 +308,56 @@ def bsgs(x, diags, baby_keys, giant_keys, bb, gg, mods, L, K, alpha):
     m, pm = _u(mods)
     _lib().oracle_bsgs(px, pd, ab, ag, bb, gg, out.ctypes.data_as(_u64p), pm, L, K,
                        alpha, B, n)
+    return out
+
+
+# ---------------------------------------------------------------- bootstrapping steps
+
+def mul_monomial(x, e, mods):
+    """x[..., limbs, n] (NTT domain) times X^e in Z_q[X]/(X^n + 1), NTT domain."""
+    x, px = _u(x)
+    out = np.zeros_like(x)
+    limbs, n = x.shape[-2], x.shape[-1]
+    m, pm = _u(mods)
+    _lib().oracle_mul_monomial(px, out.ctypes.data_as(_u64p), pm, limbs,
+                               x.size // (limbs * n), n, int(e))
+    return out
+
+
+def modraise(x, mods_full):
+    """x[..., l, n] over mods_full[:l] (NTT domain) -> [..., Lf, n] over all of
+    mods_full: each coefficient lifted to its centred value and reduced."""
+    x, px = _u(x)
+    l, n = x.shape[-2], x.shape[-1]
+    Lf = len(mods_full)
+    P = x.size // (l * n)
+    out = np.zeros(x.shape[:-2] + (Lf, n), dtype=np.uint64)
+    m, pm = _u(mods_full)
+    _lib().oracle_modraise(px, out.ctypes.data_as(_u64p), pm, l, Lf, P, n)
+    return out
+
+
+def conj_extract(ct, conj_key, mods, L, K, alpha):
+    """ct[B][2][L][n] -> (re, im), each [B][2][L][n], slots 2 Re w and 2 Im w."""
+    c, pc = _u(ct)
+    k, pk = _u(conj_key)
+    B, n = c.shape[0], c.shape[-1]
+    re = np.zeros((B, 2, L, n), dtype=np.uint64)
+    im = np.zeros((B, 2, L, n), dtype=np.uint64)
+    m, pm = _u(mods)
+    _lib().oracle_conj_extract(pc, pk, re.ctypes.data_as(_u64p), im.ctypes.data_as(_u64p),
+                               pm, L, K, alpha, B, n)
+    return re, im
+
+
+def restore_merge(re, im, mods):
+    """re, im [B][2][L][n] with slots a, b -> [B][2][L][n] with slots a + i b."""
+    r, pr = _u(re)
+    i, pi = _u(im)
+    B, L, n = r.shape[0], r.shape[2], r.shape[-1]
+    out = np.zeros_like(r)
+    m, pm = _u(mods)
+    _lib().oracle_restore_merge(pr, pi, out.ctypes.data_as(_u64p), pm, L, B, n)
     return out
 
 

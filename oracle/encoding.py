@@ -98,5 +98,49 @@ def encode_ntt(z, mods, scale, n):
     return ntt_fwd(res, mods)
 
 
+def embedding_matrix(n):
+    """U[j][k] = zeta^(k e_j), j, k < n/2, zeta = exp(i pi / n), e_j = 5^j mod 2n.
+
+    Slot j of a polynomial with real coefficients m is sum_k m_k zeta^(k e_j);
+    since zeta^(n/2 e_j) = i (e_j = 1 mod 4), the slots are U (m_lo + i m_hi)
+    with m_lo = m[:n/2] and m_hi = m[n/2:].  slot_to_coeff applies U to the
+    slots, coeff_to_slot applies U^-1 = (2/n) U^H (the rows of U are orthogonal:
+    the e_j are distinct mod 2n, so every off-diagonal row product is a full
+    sum over the powers of a non-trivial root of unity)."""
+    e = slot_exponents(n)
+    k = np.arange(n // 2, dtype=np.int64)
+    idx = np.outer(e, k) % (2 * n)
+    ang = _PI * idx.astype(np.longdouble) / np.longdouble(n)
+    return (np.cos(ang) + 1j * np.sin(ang)).astype(np.complex128)
+
+
+def coeff_to_slot_matrix(n):
+    """(2/n) U^H: slots U v -> slots v."""
+    return (2.0 / n) * embedding_matrix(n).conj().T
+
+
+def slot_to_coeff_matrix(n):
+    """U: slots v -> slots U v, i.e. the encoding of the coefficients (Re v, Im v)."""
+    return embedding_matrix(n)
+
+
+def lintrans_plaintexts(M, bb, gg, mods, scale, n):
+    """BSGS plaintexts of a slot matrix M (S x S, S = n/2, S = bb gg):
+    pt_{g,b} = Encode(rot_{-bb g}(diag_{bb g + b})), diag_k[i] = M[i][(i + k) mod S],
+    NTT residues [gg][bb][L][n]."""
+    S = M.shape[0]
+    if S != n // 2 or bb * gg != S:
+        raise ValueError("need an (n/2) x (n/2) matrix and bb * gg = n/2")
+    idx = np.arange(S)
+    out = np.zeros((gg, bb, len(mods), n), dtype=np.uint64)
+    for g in range(gg):
+        for b in range(bb):
+            k = bb * g + b
+            diag = M[idx, (idx + k) % S]
+            out[g, b] = encode_ntt(np.roll(diag, bb * g), mods, scale, n)
+    return out
+
+
 __all__ = ["slot_exponents", "encode", "crt_centered", "decode", "decode_coeffs_float",
-           "encode_ntt"]
+           "encode_ntt", "embedding_matrix", "coeff_to_slot_matrix", "slot_to_coeff_matrix",
+           "lintrans_plaintexts"]

@@ -1,7 +1,8 @@
 """Mutation sweep over the CPU oracle: plants one plausible slip at a time in
-a temporary copy of `oracle/` and runs the pin suite (test_oracle_pins.py)
-against that copy.  A pin set that is independent of the oracle must fail on
-every slip; a slip that passes every pin would mark a step left unpinned.
+a temporary copy of `oracle/` and runs the pin suites (test_oracle_pins.py,
+test_oracle_boot_pins.py) against that copy.  A pin set that is independent
+of the oracle must fail on every slip; a slip that passes every pin would
+mark a step left unpinned.
 
 Each entry is (what the slip is, file, text, replacement, which occurrence,
 the pin expected to catch it).  The replacement is applied to the copy only;
@@ -18,7 +19,7 @@ import sys
 import tempfile
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+PINS = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_boot_pins.py")]
 C = "ckks_oracle.c"
 
 MUTATIONS = [
@@ -143,6 +144,41 @@ MUTATIONS = [
      "static u64 addmod(u64 a, u64 b, u64 q) { return (a + b) % q; }",
      "static u64 addmod(u64 a, u64 b, u64 q) { u64 s = a + b; return s >= q ? s - q + 1 : s; }", 0,
      "test_fast_ntt_equals_definition"),
+    ("monomial product never negates", C,
+     "out[t] = neg ? submod(0, in[j], q) : in[j] % q;", "out[t] = in[j] % q;", 0,
+     "test_mul_monomial_on_monomials"),
+    ("modraise without centring", C,
+     "if (d[i] != hd[i]) { neg = d[i] > hd[i]; break; }", "if (d[i] != hd[i]) { neg = 0; break; }", 0,
+     "test_modraise_is_the_centred_crt_lift"),
+    ("modraise centres (Q-1)/2 itself", C,
+     "int neg = 0;\n            for (int i = l - 1;", "int neg = 1;\n            for (int i = l - 1;", 0,
+     "test_modraise_is_the_centred_crt_lift"),
+    ("modraise Garner digit with the first inverse only", C,
+     "t = mulmod(submod(t, d[j] % mods[i], mods[i]), inv[(size_t)i * l + j], mods[i]);",
+     "t = mulmod(submod(t, d[j] % mods[i], mods[i]), inv[(size_t)i * l], mods[i]);", 0,
+     "test_modraise_is_the_centred_crt_lift"),
+    ("modraise Horner from the wrong end", C,
+     "for (int i = l - 1; i >= 0; --i)\n                    r = addmod(",
+     "for (int i = 0; i < l; ++i)\n                    r = addmod(", 0,
+     "test_modraise_is_the_centred_crt_lift"),
+    ("conj_extract: imaginary part with the wrong sign", C,
+     "dif[at] = submod(cj[at], c[at], q);", "dif[at] = submod(c[at], cj[at], q);", 0,
+     "test_conj_extract_gives_real_and_imaginary_parts"),
+    ("conj_extract with the wrong Galois element", C,
+     "const u64 g = 2 * (u64)n - 1;", "const u64 g = (u64)n - 1;", 0,
+     "test_conj_extract_gives_real_and_imaginary_parts"),
+    ("restore_merge multiplies by -i", C,
+     "mods, L, 1, n, n / 2);", "mods, L, 1, n, 3 * n / 2);", 1,
+     "test_restore_merge_and_round_trip"),
+    ("embedding matrix transposed", "encoding.py",
+     "idx = np.outer(e, k) % (2 * n)", "idx = np.outer(k, e) % (2 * n)", 0,
+     "test_embedding_matrix_rows_are_orthogonal"),
+    ("coeff_to_slot matrix without the conjugate", "encoding.py",
+     "return (2.0 / n) * embedding_matrix(n).conj().T", "return (2.0 / n) * embedding_matrix(n).T", 0,
+     "test_embedding_matrix_rows_are_orthogonal"),
+    ("BSGS plaintexts pre-rotated the wrong way", "encoding.py",
+     "encode_ntt(np.roll(diag, bb * g), mods, scale, n)", "encode_ntt(np.roll(diag, -bb * g), mods, scale, n)", 0,
+     "test_coeff_to_slot_gives_the_coefficients_as_slots"),
 ]
 
 
@@ -168,7 +204,7 @@ def run(index, targeted=False, timeout=1800):
     """Run the pins against a copy with slip `index`; return (caught, first failure)."""
     with tempfile.TemporaryDirectory(prefix="oracle_slip_") as d:
         plant(index, d)
-        cmd = [sys.executable, "-m", "pytest", PINS, "-x", "-q", "--import-mode=append",
+        cmd = [sys.executable, "-m", "pytest", *PINS, "-x", "-q", "--import-mode=append",
                "-p", "no:cacheprovider"]
         if targeted:
             cmd += ["-k", MUTATIONS[index][5]]

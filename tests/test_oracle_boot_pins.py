@@ -1,0 +1,246 @@
+"""Pins of the oracle's bootstrapping steps: modraise, the monomial product,
+conj_extract, restore_merge and the coeff_to_slot / slot_to_coeff transforms.
+
+The pages name these steps (Kestrel engine write-up, the boot profile in
+section 5.3) but give no formulas; the oracle follows the textbook forms.
+Each pin checks a fact fixed outside the oracle: the centred CRT lift written
+with Python integers, the closed form of X^e on monomials, X^{n/2} acting as i
+on the slots, and decryption of each step against float64 arithmetic on the
+plaintext (its real and imaginary parts, or its coefficients)."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from rns_ckks_polynomial_b200 import synth
+
+from .helpers import N, SCALE, Params, Scheme, galois_for_rotation, u64
+
+SEED = synth.config_seed(0) + 0x100
+
+
+def _complex_slots(n, stream):
+    re = synth.uniform_real((n // 2,), -1, 1, SEED, stream).numpy()
+    im = synth.uniform_real((n // 2,), -1, 1, SEED, stream + 1).numpy()
+    return re + 1j * im
+
+
+def _centred_coeffs(sch, ct):
+    """Decryption of ct as centred Python integers (CRT over the ct's primes)."""
+    L = ct.shape[-2]
+    res = sch.orc.decrypt(ct, sch.s, sch.mods[:L])
+    return sch.orc.crt_centered(res, sch.mods[:L])
+
+
+# ------------------------------------------------------------------ X^e
+@pytest.mark.parametrize("n", [16, N])
+def test_mul_monomial_on_monomials(orc, n):
+    """X^j X^e = (-1)^floor((j+e)/n) X^((j+e) mod n), for e in [0, 2n)."""
+    mods = orc.gen_primes(n, 2)
+    for j, e in [(0, 0), (1, n // 2), (n - 1, 1), (3, n - 3), (5, n + 2), (n - 1, 2 * n - 1)]:
+        x = np.zeros((2, n), dtype=np.uint64)
+        x[:, j] = 1
+        y = orc.ntt_inv(orc.mul_monomial(orc.ntt_fwd(x, mods), e, mods), mods)
+        t, sign = (j + e) % n, (-1) ** ((j + e) // n)
+        for l, q in enumerate(int(v) for v in mods):
+            want = np.zeros(n, dtype=object)
+            want[t] = sign % q
+            assert [int(v) for v in y[l]] == list(want)
+
+
+def test_mul_monomial_half_is_i_on_slots(orc):
+    """zeta^(n/2 * 5^j) = i for every slot j, so X^{n/2} multiplies each slot
+    by i; applied twice it negates the polynomial."""
+    mods = orc.gen_primes(N, 3)
+    z = _complex_slots(N, 10)
+    pt = orc.encode_ntt(z, mods, SCALE, N)
+    out = orc.mul_monomial(pt, N // 2, mods)
+    got = orc.decode(orc.ntt_inv(out, mods), mods, SCALE)
+    assert np.max(np.abs(got - 1j * z)) < 1e-12
+    twice = orc.mul_monomial(out, N // 2, mods)
+    neg = np.array([[(int(q) - int(v)) % int(q) for v in pt[l]] for l, q in enumerate(mods)],
+                   dtype=np.uint64)
+    assert np.array_equal(twice, neg)
+
+
+# ------------------------------------------------------------------ modraise
+def test_modraise_is_the_centred_crt_lift(orc):
+    """Coefficients over q_0..q_2 -> their centred integer X in (-Q/2, Q/2],
+    reduced modulo all six primes; the residues below q_3 are unchanged.
+    The boundary values 0, 1, (Q-1)/2, (Q+1)/2, Q-1 are included."""
+    mods = orc.gen_primes(N, 6)
+    l = 3
+    q = [int(v) for v in mods]
+    Q = q[0] * q[1] * q[2]
+    x = u64(synth.uniform_residues((2, l, N), mods[:l], SEED, 20))
+    specials = [0, 1, (Q - 1) // 2, (Q + 1) // 2, Q - 1, Q // 3]
+    for k, X in enumerate(specials):
+        for i in range(l):
+            x[0, i, k] = X % q[i]
+    y = orc.ntt_inv(orc.modraise(orc.ntt_fwd(x, mods[:l]), mods), mods)
+    assert y.shape == (2, 6, N)
+    for p in range(2):
+        X = orc.crt_centered(x[p], mods[:l])
+        for t in range(6):
+            assert [int(v) for v in y[p, t]] == [v % q[t] for v in X]
+    # the centring decision at the boundary
+    assert orc.crt_centered(y[0, :, :5], mods)[:5] == [0, 1, (Q - 1) // 2, -(Q - 1) // 2, -1]
+
+
+def test_modraise_decrypts_to_message_plus_small_multiple_of_q(orc):
+    """A ciphertext kept on q_0, q_1 and raised to six primes decrypts to
+    m + e + Q_2 I with an integer polynomial I, |I_k| <= (h + 1) / 2 + 1 for a
+    secret of Hamming weight h."""
+    p = Params(6, 2, 2)
+    sch = Scheme(orc, p, SEED + 1)
+    z = _complex_slots(N, 30)
+    ct = sch.encrypt_slots(z)
+    low = np.ascontiguousarray(ct[:, :2])
+    Q2 = int(sch.mods[0]) * int(sch.mods[1])
+    raised = orc.modraise(low, sch.q)
+    assert np.array_equal(raised[:, :2], low)
+    v_low = _centred_coeffs(sch, low)
+    v_full = _centred_coeffs(sch, raised)
+    h = int(np.count_nonzero(sch.s))
+    I = []
+    for a, b in zip(v_full, v_low):
+        assert (a - b) % Q2 == 0
+        I.append((a - b) // Q2)
+    assert max(abs(v) for v in I) <= (h + 1) // 2 + 1
+    assert any(I)
+    # the low decryption is the message: it decodes to z
+    got = sch.decrypt_slots(low)
+    assert np.max(np.abs(got - z)) < 1e-8
+
+
+# ------------------------------------------------------------------ conj_extract, restore_merge
+def _conj_scheme(orc):
+    p = Params(6, 2, 2)
+    sch = Scheme(orc, p, SEED + 2)
+    return sch, sch.keygen_galois(2 * N - 1)
+
+
+def test_conj_extract_gives_real_and_imaginary_parts(orc):
+    sch, ck = _conj_scheme(orc)
+    p = sch.p
+    w = _complex_slots(N, 40)
+    ct = sch.encrypt_slots(w)
+    re, im = orc.conj_extract(ct[None], ck, sch.mods, p.L, p.K, p.alpha)
+    got_re = sch.decrypt_slots(re[0], 2 * SCALE)
+    got_im = sch.decrypt_slots(im[0], 2 * SCALE)
+    assert np.max(np.abs(got_re - w.real)) < 1e-8
+    assert np.max(np.abs(got_im - w.imag)) < 1e-8
+
+
+def test_restore_merge_and_round_trip(orc):
+    sch, ck = _conj_scheme(orc)
+    p = sch.p
+    a = synth.uniform_real((N // 2,), -1, 1, SEED, 50).numpy()
+    b = synth.uniform_real((N // 2,), -1, 1, SEED, 51).numpy()
+    ca, cb = sch.encrypt_slots(a), sch.encrypt_slots(b)
+    merged = orc.restore_merge(ca[None], cb[None], sch.q)
+    assert np.max(np.abs(sch.decrypt_slots(merged[0]) - (a + 1j * b))) < 1e-8
+    # merge(extract(ct)) has slots 2w
+    w = _complex_slots(N, 52)
+    ct = sch.encrypt_slots(w)
+    re, im = orc.conj_extract(ct[None], ck, sch.mods, p.L, p.K, p.alpha)
+    back = orc.restore_merge(re, im, sch.q)
+    assert np.max(np.abs(sch.decrypt_slots(back[0], 2 * SCALE) - w)) < 1e-8
+
+
+# ------------------------------------------------------------------ coeff_to_slot / slot_to_coeff
+def _transform_scheme(orc, n, bb, gg):
+    p = Params(6, 2, 2, n=n)
+    sch = Scheme(orc, p, SEED + 3 + n)
+    baby = [sch.keygen_galois(galois_for_rotation(b, n)) for b in range(1, bb)]
+    giant = [sch.keygen_galois(galois_for_rotation(bb * g, n)) for g in range(1, gg)]
+    return sch, baby, giant
+
+
+def _at_level(sch, L, keys):
+    """Moduli and keys for a ciphertext on q_0..q_{L-1}: the special primes
+    follow the ciphertext primes, and each key keeps the limbs of those primes
+    and the first ceil(L / alpha) digits (a key reduced modulo a divisor of
+    its modulus is a key for that modulus)."""
+    p = sch.p
+    keep = list(range(L)) + list(range(p.L, p.L + p.K))
+    mods = np.ascontiguousarray(sch.mods[keep])
+    dn = (L + p.alpha - 1) // p.alpha
+    return mods, [np.ascontiguousarray(k[:dn][:, :, keep]) for k in keys]
+
+
+def _lintrans(orc, sch, ct, M, bb, gg, baby, giant):
+    p = sch.p
+    L = ct.shape[-2]
+    mods, keys = _at_level(sch, L, baby + giant)
+    diags = orc.lintrans_plaintexts(M, bb, gg, mods[:L], SCALE, p.n)
+    y = orc.bsgs(ct[None], diags, keys[: bb - 1], keys[bb - 1:], bb, gg, mods, L, p.K, p.alpha)
+    return y[0]
+
+
+def test_embedding_matrix_rows_are_orthogonal(orc):
+    """U U^H = (n/2) I, and U applied to (m_lo + i m_hi) / scale equals the
+    decoder's slots of m."""
+    n = 64
+    U = orc.embedding_matrix(n)
+    assert np.max(np.abs(U @ U.conj().T - (n // 2) * np.eye(n // 2))) < 1e-12
+    assert np.max(np.abs(orc.coeff_to_slot_matrix(n) @ orc.slot_to_coeff_matrix(n)
+                         - np.eye(n // 2))) < 1e-12
+    m = synth.uniform_real((n,), -1, 1, SEED, 60).numpy()
+    v = m[: n // 2] + 1j * m[n // 2:]
+    assert np.max(np.abs(U @ v - orc.decode_coeffs_float(m, n))) < 1e-12
+
+
+@pytest.mark.parametrize("n,bb,gg", [(64, 8, 4), (256, 16, 8)])
+def test_coeff_to_slot_gives_the_coefficients_as_slots(orc, n, bb, gg):
+    """coeff_to_slot of an encryption of polynomial m decrypts to slots
+    (m_k + i m_{k+n/2}) / scale, read off the decrypted input's coefficients."""
+    sch, baby, giant = _transform_scheme(orc, n, bb, gg)
+    z = _complex_slots(n, 70)
+    ct = sch.encrypt_slots(z)
+    m = _centred_coeffs(sch, ct)
+    want = np.array([(Fraction(m[k]) / SCALE) for k in range(n // 2)], dtype=float) + \
+        1j * np.array([(Fraction(m[k + n // 2]) / SCALE) for k in range(n // 2)], dtype=float)
+    y = _lintrans(orc, sch, ct, orc.coeff_to_slot_matrix(n), bb, gg, baby, giant)
+    sc = sch.rescaled_scale(SCALE * SCALE, sch.p.L)
+    assert np.max(np.abs(sch.decrypt_slots(y, sc) - want)) < 1e-8
+
+
+@pytest.mark.parametrize("n,bb,gg", [(64, 8, 4), (256, 16, 8)])
+def test_slot_to_coeff_puts_the_slots_into_the_coefficients(orc, n, bb, gg):
+    """slot_to_coeff of an encryption of slots v decrypts to a polynomial with
+    coefficients scale * Re v_k (k < n/2) and scale * Im v_{k-n/2} (k >= n/2)."""
+    sch, baby, giant = _transform_scheme(orc, n, bb, gg)
+    v = _complex_slots(n, 80)
+    ct = sch.encrypt_slots(v)
+    y = _lintrans(orc, sch, ct, orc.slot_to_coeff_matrix(n), bb, gg, baby, giant)
+    sc = sch.rescaled_scale(SCALE * SCALE, sch.p.L)
+    got = np.array([float(Fraction(c) / sc) for c in _centred_coeffs(sch, y)])
+    assert np.max(np.abs(got - np.concatenate([v.real, v.imag]))) < 1e-8
+
+
+def test_linear_part_of_bootstrapping(orc):
+    """modraise -> coeff_to_slot -> conj_extract -> restore_merge ->
+    slot_to_coeff on a ciphertext kept on two primes: the result decrypts to
+    2 t, where t = m + e + Q_2 I is the raised plaintext (no evaluation of the
+    modular reduction in between, so nothing removes Q_2 I)."""
+    n, bb, gg = 64, 8, 4
+    sch, baby, giant = _transform_scheme(orc, n, bb, gg)
+    p = sch.p
+    ck = sch.keygen_galois(2 * n - 1)
+    z = _complex_slots(n, 90)
+    low = np.ascontiguousarray(sch.encrypt_slots(z)[:, :2])
+    ct = orc.modraise(low, sch.q)
+    t = _centred_coeffs(sch, ct)
+    a = _lintrans(orc, sch, ct, orc.coeff_to_slot_matrix(n), bb, gg, baby, giant)
+    mods5, (ck5,) = _at_level(sch, p.L - 1, [ck])
+    re, im = orc.conj_extract(a[None], ck5, mods5, p.L - 1, p.K, p.alpha)
+    merged = orc.restore_merge(re, im, sch.mods[: p.L - 1])[0]
+    out = _lintrans(orc, sch, merged, orc.slot_to_coeff_matrix(n), bb, gg, baby, giant)
+    assert out.shape == (2, p.L - 2, n)
+    sc = (Fraction(SCALE * SCALE, int(sch.mods[p.L - 1])) * SCALE) / int(sch.mods[p.L - 2])
+    got = [Fraction(c) / sc for c in _centred_coeffs(sch, out)]
+    want = [Fraction(2 * v, SCALE) for v in t]
+    big = max(abs(w) for w in want)
+    assert big > 2**50  # the lift really added multiples of Q_2
+    assert max(abs(float(g - w)) for g, w in zip(got, want)) < 1e-9 * float(big)
