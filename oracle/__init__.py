@@ -9,6 +9,8 @@ The integer arithmetic lives in ``ckks_oracle.c`` (plain C, ``unsigned
 __int128``, each operation written as its definition).  This module adds the
 ctypes bindings and the parts of the scheme that need big integers or complex
 numbers: the canonical-embedding encoder/decoder and CRT reconstruction.
+``oracle.boot`` composes those operations into sin_fold and the whole
+bootstrapping refresh.
 """
 from .core import *  # noqa: F401,F403
 from .encoding import *  # noqa: F401,F403

@@ -179,6 +179,25 @@ MUTATIONS = [
     ("BSGS plaintexts pre-rotated the wrong way", "encoding.py",
      "encode_ntt(np.roll(diag, bb * g), mods, scale, n)", "encode_ntt(np.roll(diag, -bb * g), mods, scale, n)", 0,
      "test_coeff_to_slot_gives_the_coefficients_as_slots"),
+    ("sin_fold: Taylor series of cosh instead of cos", "boot.py",
+     "a_k = (-1) ** k / math.factorial(2 * k)", "a_k = 1 / math.factorial(2 * k)", 0,
+     "test_sin_fold_is_sine_of_two_pi_x"),
+    ("sin_fold: double-angle step without the factor 2", "boot.py",
+     "        c = mul_int(c, 2, chain)\n", "", 0,
+     "test_sin_fold_is_sine_of_two_pi_x"),
+    ("sin_fold: quarter-turn shift the wrong way", "boot.py",
+     "th = add_const(th, -w / 4, s_th, chain)", "th = add_const(th, w / 4, s_th, chain)", 0,
+     "test_sin_fold_is_sine_of_two_pi_x"),
+    ("constants added to c1 instead of c0", "boot.py",
+     'out[0] = core.pointwise("add", ct[0], c, chain.mods[:l])',
+     'out[1] = core.pointwise("add", ct[1], c, chain.mods[:l])', 0,
+     "test_sin_fold_is_sine_of_two_pi_x"),
+    ("coeff_to_slot without the 1/2 that conj_extract doubles", "boot.py",
+     "lintrans_plaintexts(0.5 * coeff_to_slot_matrix(n)", "lintrans_plaintexts(coeff_to_slot_matrix(n)", 0,
+     "test_bootstrap_removes_the_multiple_of_q0"),
+    ("slot_to_coeff factor q0 / (pi Delta)", "boot.py",
+     "f = q0 / (2 * math.pi * delta)", "f = q0 / (math.pi * delta)", 0,
+     "test_bootstrap_removes_the_multiple_of_q0"),
 ]
 
 

@@ -244,3 +244,61 @@ def test_linear_part_of_bootstrapping(orc):
     big = max(abs(w) for w in want)
     assert big > 2**50  # the lift really added multiples of Q_2
     assert max(abs(float(g - w)) for g, w in zip(got, want)) < 1e-9 * float(big)
+
+
+# ------------------------------------------------------------------ sin_fold and the whole refresh
+def _boot_scheme(orc, n, bb, gg, seed):
+    p = Params(20, 4, 4, n=n)
+    sch = Scheme(orc, p, seed)
+    keys = {"relin": sch.keygen_relin(), "conj": sch.keygen_galois(2 * n - 1),
+            "baby": [sch.keygen_galois(galois_for_rotation(b, n)) for b in range(1, bb)],
+            "giant": [sch.keygen_galois(galois_for_rotation(bb * g, n)) for g in range(1, gg)]}
+    return sch, keys
+
+
+def test_sin_fold_is_sine_of_two_pi_x(orc):
+    """Slots x = I + f, integers |I| <= 20 and |f| <= 0.01: sin_fold with r = 8
+    consumes 6 + 8 levels and decrypts to sin(2 pi x), to 1e-9."""
+    from oracle import boot
+    n, r = 64, 8
+    sch = Scheme(orc, Params(20, 4, 4, n=n), SEED + 7)
+    chain = boot.Chain(sch.mods, 20, 4, 4)
+    rlk = sch.keygen_relin()
+    x = (synth.uniform_below((n // 2,), 41, SEED, 100).numpy() - 20
+         + synth.uniform_real((n // 2,), -0.01, 0.01, SEED, 101).numpy())
+    ct = sch.encrypt_slots(x)
+    out, s = boot.sin_fold(ct, Fraction(SCALE), r, rlk, chain)
+    assert out.shape == (2, 20 - 6 - r, n)
+    got = sch.decrypt_slots(out, s)
+    assert np.max(np.abs(got - np.sin(2 * np.pi * x))) < 1e-9
+
+
+def test_bootstrap_removes_the_multiple_of_q0(orc):
+    """A ciphertext on q_0 holding slots z at scale 2^50, refreshed onto the
+    20-prime chain: modraise adds q_0 I, and the refresh returns a ciphertext
+    2 + 6 + 8 levels down whose coefficients are
+    (q_0 / 2 pi) sin(2 pi m_k / q_0) / Delta (to 1e-7), i.e. m_k / Delta up to
+    the sine's own cubic term, and whose slots are z to within that term."""
+    import math
+
+    from oracle import boot
+    n, bb, gg, r = 64, 8, 4, 8
+    delta = 2**50
+    sch, keys = _boot_scheme(orc, n, bb, gg, SEED + 8)
+    chain = boot.Chain(sch.mods, 20, 4, 4)
+    z = _complex_slots(n, 110)
+    low = np.ascontiguousarray(sch.encrypt_slots(z, delta)[:, :1])
+    q0 = int(sch.mods[0])
+    m = _centred_coeffs(sch, low)
+    t = _centred_coeffs(sch, orc.modraise(low, sch.q))
+    assert any((a - b) // q0 for a, b in zip(t, m))
+    out, s = boot.bootstrap(low, delta, r, keys, chain, bb, gg)
+    assert out.shape == (2, 20 - 2 - 6 - r, n)
+    got = np.array([float(Fraction(c) / s) for c in _centred_coeffs(sch, out)])
+    sine = np.array([q0 / (2 * math.pi) * math.sin(2 * math.pi * v / q0) / delta for v in m])
+    assert np.max(np.abs(got - sine)) < 1e-7
+    mm = np.array(m, dtype=float) / delta
+    cubic = np.max(np.abs(mm) * (2 * np.pi * np.abs(mm) * delta / q0) ** 2 / 6)
+    assert np.max(np.abs(got - mm)) < cubic + 1e-7
+    slots = sch.decrypt_slots(out, s)
+    assert np.max(np.abs(slots - z)) < n * (cubic + 1e-7)
