@@ -33,7 +33,9 @@
  *  - `ws` is a device workspace of at least ckks_workspace_bytes(...) bytes,
  *    16-byte aligned, used only for the duration of the call's stream work.
  *    Passing NULL makes the context allocate (and keep) its own workspace;
- *    that path calls cudaMalloc and synchronises the device.
+ *    that path calls cudaMalloc and synchronises the device.  All NULL-
+ *    workspace calls on one context share that one buffer, so they must be
+ *    serialised: issue them on one stream from one host thread at a time.
  *  - Status: CKKS_OK (0) or a negative code.  Argument checks run on the host
  *    before any launch; a failed check launches nothing.  CUDA launch errors
  *    map to CKKS_ECUDA.  ckks_last_error() returns a thread-local message.

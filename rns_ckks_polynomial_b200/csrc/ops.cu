@@ -21,7 +21,9 @@ static int check_batch(int batch)
 
 static int check_limbs(const ckks_ctx *ctx, int limb_begin, int limbs)
 {
-    if (limb_begin < 0 || limbs < 0 || limb_begin + limbs > ctx->L + ctx->K)
+    // compared without forming limb_begin + limbs, which could overflow an int
+    const int total = ctx->L + ctx->K;
+    if (limb_begin < 0 || limbs < 0 || limb_begin > total || limbs > total - limb_begin)
         return set_error(CKKS_EINVAL, "limb range outside the context's primes");
     return CKKS_OK;
 }
