@@ -167,6 +167,102 @@ def lintrans(ct, scale, diags, pt_scale, bb, gg, baby, giant, chain):
     return y, Fraction(scale) * Fraction(pt_scale) / chain.q(l - 1)
 
 
+def rotation_amounts(plan, S):
+    """Left-rotation amounts a BSGS plan needs keys for (Galois 5^r each)."""
+    stride, t0, bb, gg = plan
+    amounts = {(stride * b) % S for b in range(1, bb)}
+    amounts |= {(stride * (t0 + bb * g)) % S for g in range(gg)}
+    return sorted(a for a in amounts if a)
+
+
+def lintrans_planned(ct, scale, Dg, plan, pt_scale, keys, chain):
+    """y = sum_g Rot_{G_g}( sum_b pt_{g,b} * Rot_{stride b}(x) ), then one
+    rescale, for a matrix in diagonal form with plan (stride, t0, bb, gg)
+    (encoding.bsgs_plan).  keys: {r: Galois key of 5^r} over the full chain.
+    The baby rotations share one ModUp (hoisted); a giant step with G_g = 0
+    is not rotated; absent diagonals are skipped."""
+    from .encoding import plan_plaintexts
+    n = ct.shape[-1]
+    S = n // 2
+    l = level(ct)
+    stride, t0, bb, gg = plan
+    pts, giants = plan_plaintexts(Dg, plan, S, chain.mods[:l], pt_scale, n)
+    mods_l = chain.mods_at(l)
+    qs = chain.mods[:l]
+    babies = [ct]
+    if bb > 1:
+        amounts = [(stride * b) % S for b in range(1, bb)]
+        gal = np.array([pow(5, a, 2 * n) for a in amounts], dtype=np.uint64)
+        rot = core.rotate(ct[None], [chain.key_at(keys[a], l) for a in amounts], gal, mods_l, l,
+                          chain.K, chain.alpha)
+        babies += [rot[i, 0] for i in range(len(amounts))]
+    acc = None
+    for g in range(gg):
+        inner = None
+        for b in range(bb):
+            pt = pts[g][b]
+            if pt is None:
+                continue
+            prod = core.pointwise("mul", babies[b], np.broadcast_to(pt, babies[b].shape).copy(), qs)
+            inner = prod if inner is None else core.pointwise("add", inner, prod, qs)
+        if inner is None:
+            continue
+        G = giants[g]
+        if G:
+            gal = np.array([pow(5, G, 2 * n)], dtype=np.uint64)
+            inner = core.rotate(inner[None], [chain.key_at(keys[G], l)], gal, mods_l, l, chain.K,
+                                chain.alpha)[0, 0]
+        acc = inner if acc is None else core.pointwise("add", acc, inner, qs)
+    out = core.rescale(acc[None], qs)[0]
+    return out, Fraction(scale) * Fraction(pt_scale) / chain.q(l - 1)
+
+
+def lintrans_factored(ct, scale, factors, pt_scale, keys, chain, first_factor_scalar=1.0):
+    """Apply diagonal forms F_1, F_2, ... in turn (one level each); the scalar
+    multiplies F_1's diagonals."""
+    from .encoding import bsgs_plan
+    S = ct.shape[-1] // 2
+    for i, F in enumerate(factors):
+        if i == 0 and first_factor_scalar != 1.0:
+            F = {k: first_factor_scalar * d for k, d in F.items()}
+        ct, scale = lintrans_planned(ct, scale, F, bsgs_plan(F, S), pt_scale, keys, chain)
+    return ct, scale
+
+
+def factored_rotation_amounts(n, depth):
+    """Every rotation the factored coeff_to_slot and slot_to_coeff of this
+    depth use (the two share their diagonal offsets)."""
+    from .encoding import bsgs_plan, factored_coeff_to_slot, factored_slot_to_coeff
+    S = n // 2
+    out = set()
+    for F in factored_coeff_to_slot(n, depth) + factored_slot_to_coeff(n, depth):
+        out |= set(rotation_amounts(bsgs_plan(F, S), S))
+    return sorted(out)
+
+
+def bootstrap_factored(ct_q0, delta, r, depth, keys, chain):
+    """bootstrap() with coeff_to_slot and slot_to_coeff as `depth` factored
+    levels each (slots in bit-reversed order in between, which the slot-wise
+    steps do not mind).  keys: 'rot' {r: key of 5^r} for
+    factored_rotation_amounts(n, depth), 'conj', 'relin'.  Uses
+    2 depth + 6 + r levels."""
+    from .encoding import factored_coeff_to_slot, factored_slot_to_coeff
+    n = ct_q0.shape[-1]
+    q0 = chain.q(0)
+    ct = core.modraise(ct_q0, chain.mods[: chain.L])
+    ct, scale = lintrans_factored(ct, Fraction(q0), factored_coeff_to_slot(n, depth), 2**60,
+                                  keys["rot"], chain, first_factor_scalar=0.5)
+    l = level(ct)
+    re, im = core.conj_extract(ct[None], chain.key_at(keys["conj"], l), chain.mods_at(l), l,
+                               chain.K, chain.alpha)
+    sre, s_out = sin_fold(re[0], scale, r, keys["relin"], chain)
+    sim, _ = sin_fold(im[0], scale, r, keys["relin"], chain)
+    merged = core.restore_merge(sre[None], sim[None], chain.mods[: level(sre)])[0]
+    f = q0 / (2 * math.pi * delta)
+    return lintrans_factored(merged, s_out, factored_slot_to_coeff(n, depth), 2**50, keys["rot"],
+                             chain, first_factor_scalar=f)
+
+
 def bootstrap(ct_q0, delta, r, keys, chain, bb, gg):
     """Refresh a ciphertext on q_0 holding slots z at scale `delta`
     (delta well below q_0).  `keys` holds 'baby', 'giant' (Galois keys for
@@ -194,4 +290,5 @@ def bootstrap(ct_q0, delta, r, keys, chain, bb, gg):
 
 __all__ = ["Chain", "drop", "mul_int", "add_const", "mul_const", "mul", "add", "sin_fold",
            "coeff_to_slot_plaintexts", "slot_to_coeff_plaintexts", "lintrans", "bootstrap",
-           "TAYLOR_TERMS"]
+           "rotation_amounts", "lintrans_planned", "lintrans_factored",
+           "factored_rotation_amounts", "bootstrap_factored", "TAYLOR_TERMS"]

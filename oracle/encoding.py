@@ -141,6 +141,150 @@ def lintrans_plaintexts(M, bb, gg, mods, scale, n):
     return out
 
 
+# ---------------------------------------------------------------- factored transforms
+#
+# U evaluates V(X) = sum_k v_k X^k at the S = n/2 points w_j = zeta^(5^j).  Split
+# V(X) = E(X^2) + X O(X^2).  The squares w_j^2 are the points of the same problem
+# for S/2 (zeta^2, 5^j mod n), and w_{j+S/2} = -w_j because 5^(S/2) = 1 + n
+# (mod 2n).  Hence z_j = E_j + w_j O_j and z_{j+S/2} = E_j - w_j O_j: a
+# butterfly stage over a half-size transform of the even and of the odd
+# coefficients.  Unrolled, U = G_m ... G_1 R with m = log2 S, R the bit-reversal
+# permutation and G_s (block length len = 2^s) acting on each block of len
+# slots as [[I, D], [I, -D]], D = diag(zeta_len^(5^j)), j < len/2, zeta_len a
+# primitive (4 len)-th root of unity.  Every G_s has three slot diagonals
+# (offsets 0, len/2, -len/2), so a group of consecutive stages a..b has at
+# most 2^(b-a+2) - 1 diagonals, all multiples of 2^(a-1).
+#
+# A matrix is held in diagonal form {k: d_k}, d_k[i] = M[i][(i + k) mod S], so
+# (M x)_i = sum_k d_k[i] x[(i + k) mod S].
+
+
+def bit_reverse_indices(S):
+    bits = S.bit_length() - 1
+    return np.array([int(format(i, "0%db" % bits)[::-1], 2) if bits else 0 for i in range(S)])
+
+
+def _stage_diagonals(n, s, inverse=False):
+    """G_s (or its inverse) in diagonal form."""
+    S = n // 2
+    ln = 1 << s
+    h = ln // 2
+    e = np.array([pow(5, j, 4 * ln) for j in range(h)], dtype=np.int64)
+    ang = 2 * _PI * e.astype(np.longdouble) / np.longdouble(4 * ln)
+    D = (np.cos(ang) + 1j * np.sin(ang)).astype(np.complex128)
+    pos = np.arange(S) % ln
+    top = pos < h
+    j = np.where(top, pos, pos - h)
+    d0, dp, dm = np.zeros(S, complex), np.zeros(S, complex), np.zeros(S, complex)
+    if not inverse:
+        # top rows: u + D v;  bottom rows: u - D v
+        d0[top], dp[top] = 1, D[j[top]]
+        dm[~top], d0[~top] = 1, -D[j[~top]]
+    else:
+        # [[I, D], [I, -D]]^-1 = 1/2 [[I, I], [D^-1, -D^-1]]
+        d0[top], dp[top] = 0.5, 0.5
+        dm[~top], d0[~top] = 0.5 / D[j[~top]], -0.5 / D[j[~top]]
+    out = {0: d0}
+    if h == S // 2 and S > 1:
+        out[h] = dp + dm               # +h and -h are the same offset mod S
+    else:
+        out[h] = dp
+        out[(S - h) % S] = dm
+    return out
+
+
+def diag_product(A, B, S):
+    """Diagonal form of A B: d_{a+b}[i] += A_a[i] B_b[i + a]."""
+    out = {}
+    for a, da in A.items():
+        for b, db in B.items():
+            k = (a + b) % S
+            out[k] = out.get(k, 0) + da * np.roll(db, -a)
+    return out
+
+
+def diag_to_dense(Dg, S):
+    M = np.zeros((S, S), dtype=complex)
+    i = np.arange(S)
+    for k, d in Dg.items():
+        M[i, (i + k) % S] += d
+    return M
+
+
+def stage_groups(n, depth):
+    """Split the log2(n/2) butterfly stages into `depth` consecutive groups,
+    the later groups at least as long as the earlier ones."""
+    m = (n // 2).bit_length() - 1
+    base, extra = divmod(m, depth)
+    sizes = [base + (1 if g >= depth - extra else 0) for g in range(depth)]
+    out, s = [], 1
+    for sz in sizes:
+        out.append(list(range(s, s + sz)))
+        s += sz
+    return out
+
+
+def factored_slot_to_coeff(n, depth):
+    """Diagonal forms F_1..F_depth with U = F_depth ... F_1 R (F_1 applied first)."""
+    S = n // 2
+    mats = []
+    for grp in stage_groups(n, depth):
+        F = {0: np.ones(S, complex)}
+        for s in grp:
+            F = diag_product(_stage_diagonals(n, s), F, S)
+        mats.append(F)
+    return mats
+
+
+def factored_coeff_to_slot(n, depth):
+    """Diagonal forms H_1..H_depth with R U^-1 = H_depth ... H_1 (H_1 applied
+    first): the inverse stages in reverse order; the output slots come out in
+    bit-reversed order, which factored_slot_to_coeff takes back."""
+    S = n // 2
+    mats = []
+    for grp in reversed(stage_groups(n, depth)):
+        F = {0: np.ones(S, complex)}
+        for s in reversed(grp):
+            F = diag_product(_stage_diagonals(n, s, inverse=True), F, S)
+        mats.append(F)
+    return mats
+
+
+def bsgs_plan(Dg, S, tol=0.0):
+    """Baby-step giant-step plan for a diagonal form whose nonzero offsets are
+    stride * t, t in a window [t0, t0 + T): offsets stride (t0 + bb g + b),
+    g < gg, b < bb, with bb the power of two nearest sqrt(T).  Returns
+    (stride, t0, bb, gg)."""
+    ks = sorted(k for k, d in Dg.items() if np.max(np.abs(d)) > tol)
+    if ks == [0]:
+        return 1, 0, 1, 1
+    stride = int(np.gcd.reduce([k for k in ks if k] + [S]))
+    ts = sorted(((k // stride) + S // stride // 2) % (S // stride) - S // stride // 2 for k in ks)
+    t0, T = ts[0], ts[-1] - ts[0] + 1
+    bb = 1 << max(0, round(np.log2(np.sqrt(T))))
+    gg = -(-T // bb)
+    return stride, t0, bb, gg
+
+
+def plan_plaintexts(Dg, plan, S, mods, scale, n):
+    """pt_{g,b} = Encode(rot_{-G_g}(d_{G_g + stride b})) with G_g = stride (t0 + bb g);
+    None where that diagonal is absent.  Also returns the giant offsets G_g."""
+    stride, t0, bb, gg = plan
+    pts, giants = [], []
+    for g in range(gg):
+        G = (stride * (t0 + bb * g)) % S
+        giants.append(G)
+        row = []
+        for b in range(bb):
+            k = (G + stride * b) % S
+            d = Dg.get(k)
+            row.append(None if d is None else encode_ntt(np.roll(d, G), mods, scale, n))
+        pts.append(row)
+    return pts, giants
+
+
 __all__ = ["slot_exponents", "encode", "crt_centered", "decode", "decode_coeffs_float",
            "encode_ntt", "embedding_matrix", "coeff_to_slot_matrix", "slot_to_coeff_matrix",
-           "lintrans_plaintexts"]
+           "lintrans_plaintexts", "bit_reverse_indices", "diag_product", "diag_to_dense",
+           "stage_groups", "factored_slot_to_coeff", "factored_coeff_to_slot", "bsgs_plan",
+           "plan_plaintexts"]

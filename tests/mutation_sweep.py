@@ -198,6 +198,23 @@ MUTATIONS = [
     ("slot_to_coeff factor q0 / (pi Delta)", "boot.py",
      "f = q0 / (2 * math.pi * delta)", "f = q0 / (math.pi * delta)", 0,
      "test_bootstrap_removes_the_multiple_of_q0"),
+    ("butterfly twiddles from the (2 len)-th root", "encoding.py",
+     "ang = 2 * _PI * e.astype(np.longdouble) / np.longdouble(4 * ln)",
+     "ang = 2 * _PI * e.astype(np.longdouble) / np.longdouble(2 * ln)", 0,
+     "test_special_fft_factorization"),
+    ("inverse butterfly multiplies by D instead of D^-1", "encoding.py",
+     "dm[~top], d0[~top] = 0.5 / D[j[~top]], -0.5 / D[j[~top]]",
+     "dm[~top], d0[~top] = 0.5 * D[j[~top]], -0.5 * D[j[~top]]", 0,
+     "test_special_fft_factorization"),
+    ("diagonal product shifts the wrong way", "encoding.py",
+     "out[k] = out.get(k, 0) + da * np.roll(db, -a)", "out[k] = out.get(k, 0) + da * np.roll(db, a)", 0,
+     "test_special_fft_factorization"),
+    ("bit reversal left out", "encoding.py",
+     'int(format(i, "0%db" % bits)[::-1], 2)', 'int(format(i, "0%db" % bits), 2)', 0,
+     "test_special_fft_factorization"),
+    ("planned BSGS plaintexts pre-rotated the wrong way", "encoding.py",
+     "encode_ntt(np.roll(d, G), mods, scale, n)", "encode_ntt(np.roll(d, -G), mods, scale, n)", 0,
+     "test_factored_transforms_decrypt"),
 ]
 
 

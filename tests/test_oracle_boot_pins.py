@@ -302,3 +302,79 @@ def test_bootstrap_removes_the_multiple_of_q0(orc):
     assert np.max(np.abs(got - mm)) < cubic + 1e-7
     slots = sch.decrypt_slots(out, s)
     assert np.max(np.abs(slots - z)) < n * (cubic + 1e-7)
+
+
+# ------------------------------------------------------------------ factored transforms
+@pytest.mark.parametrize("n", [16, 64, 256])
+@pytest.mark.parametrize("depth", [1, 2, 3])
+def test_special_fft_factorization(orc, n, depth):
+    """F_depth ... F_1 R = U and H_depth ... H_1 = R U^-1 against the dense
+    embedding matrix; a group of k butterfly stages has at most 2^(k+1) - 1
+    diagonals, all multiples of its stride, and its BSGS plan covers them."""
+    S = n // 2
+    U = orc.embedding_matrix(n)
+    R = np.eye(S)[orc.bit_reverse_indices(S)]
+    assert sorted(orc.bit_reverse_indices(S)) == list(range(S))
+    P, Q = np.eye(S, dtype=complex), np.eye(S, dtype=complex)
+    for F in orc.factored_slot_to_coeff(n, depth):
+        P = orc.diag_to_dense(F, S) @ P
+    for H in orc.factored_coeff_to_slot(n, depth):
+        Q = orc.diag_to_dense(H, S) @ Q
+    assert np.max(np.abs(P @ R - U)) < 1e-12
+    assert np.max(np.abs(Q @ U - R)) < 1e-12
+    for grp, F in zip(orc.stage_groups(n, depth), orc.factored_slot_to_coeff(n, depth)):
+        assert len(F) <= 2 ** (len(grp) + 1) - 1
+        stride, t0, bb, gg = orc.bsgs_plan(F, S)
+        assert all(k % stride == 0 for k in F)
+        covered = {(stride * (t0 + bb * g + b)) % S for g in range(gg) for b in range(bb)}
+        assert set(F) <= covered
+
+
+def _factored_scheme(orc, n, depth, seed):
+    from oracle import boot
+    sch = Scheme(orc, Params(20, 4, 4, n=n), seed)
+    keys = {"rot": {a: sch.keygen_galois(galois_for_rotation(a, n))
+                    for a in boot.factored_rotation_amounts(n, depth)},
+            "conj": sch.keygen_galois(2 * n - 1), "relin": sch.keygen_relin()}
+    return sch, boot.Chain(sch.mods, 20, 4, 4), keys
+
+
+def test_factored_transforms_decrypt(orc):
+    """Two-level coeff_to_slot puts (m_k + i m_{k+n/2}) / scale into slot
+    brv(k); two-level slot_to_coeff of those bit-reversed slots gives U v."""
+    from oracle import boot
+    n, depth = 64, 2
+    S = n // 2
+    sch, chain, keys = _factored_scheme(orc, n, depth, SEED + 9)
+    ct = sch.encrypt_slots(_complex_slots(n, 120))
+    m = _centred_coeffs(sch, ct)
+    v = np.array([float(Fraction(m[k], SCALE)) + 1j * float(Fraction(m[k + S], SCALE))
+                  for k in range(S)])
+    w = v[orc.bit_reverse_indices(S)]
+    y, sc = boot.lintrans_factored(ct, Fraction(SCALE), orc.factored_coeff_to_slot(n, depth), SCALE,
+                                   keys["rot"], chain)
+    assert y.shape == (2, 20 - depth, n)
+    assert np.max(np.abs(sch.decrypt_slots(y, sc) - w)) < 1e-8
+    y2, sc2 = boot.lintrans_factored(sch.encrypt_slots(w), Fraction(SCALE),
+                                     orc.factored_slot_to_coeff(n, depth), SCALE, keys["rot"], chain)
+    assert np.max(np.abs(sch.decrypt_slots(y2, sc2) - orc.embedding_matrix(n) @ v)) < 1e-8
+
+
+def test_bootstrap_with_factored_transforms(orc):
+    """The refresh with two-level transforms: 2 * 2 + 6 + 8 levels, and the
+    same sine form of the coefficients as the dense refresh."""
+    import math
+
+    from oracle import boot
+    n, depth, r = 64, 2, 8
+    delta = 2**50
+    sch, chain, keys = _factored_scheme(orc, n, depth, SEED + 10)
+    z = _complex_slots(n, 130)
+    low = np.ascontiguousarray(sch.encrypt_slots(z, delta)[:, :1])
+    q0 = int(sch.mods[0])
+    m = _centred_coeffs(sch, low)
+    out, s = boot.bootstrap_factored(low, delta, r, depth, keys, chain)
+    assert out.shape == (2, 20 - 2 * depth - 6 - r, n)
+    got = np.array([float(Fraction(c) / s) for c in _centred_coeffs(sch, out)])
+    sine = np.array([q0 / (2 * math.pi) * math.sin(2 * math.pi * v / q0) / delta for v in m])
+    assert np.max(np.abs(got - sine)) < 1e-7
