@@ -378,3 +378,30 @@ def test_bootstrap_with_factored_transforms(orc):
     got = np.array([float(Fraction(c) / s) for c in _centred_coeffs(sch, out)])
     sine = np.array([q0 / (2 * math.pi) * math.sin(2 * math.pi * v / q0) / delta for v in m])
     assert np.max(np.abs(got - sine)) < 1e-7
+
+
+@pytest.mark.slow
+@pytest.mark.skipif(not __import__("os").environ.get("CKKS_SLOW_PINS"),
+                    reason="about 90 s of CPU; set CKKS_SLOW_PINS=1")
+def test_bootstrap_at_ring_degree_2048(orc):
+    """The refresh at n = 2048 with a dense ternary secret, three-level
+    factored transforms and r = 9: 2 * 3 + 6 + 9 = 21 levels (23 primes down
+    to 2), and the sine form of the coefficients within 1e-5."""
+    import math
+
+    from oracle import boot
+    n, depth, r, L = N, 3, 9, 23
+    delta = 2**50
+    sch = Scheme(orc, Params(L, 4, 4), SEED + 11)
+    chain = boot.Chain(sch.mods, L, 4, 4)
+    keys = {"rot": {a: sch.keygen_galois(galois_for_rotation(a, n))
+                    for a in boot.factored_rotation_amounts(n, depth)},
+            "conj": sch.keygen_galois(2 * n - 1), "relin": sch.keygen_relin()}
+    low = np.ascontiguousarray(sch.encrypt_slots(_complex_slots(n, 140), delta)[:, :1])
+    q0 = int(sch.mods[0])
+    m = _centred_coeffs(sch, low)
+    out, s = boot.bootstrap_factored(low, delta, r, depth, keys, chain)
+    assert out.shape == (2, L - 2 * depth - 6 - r, n)
+    got = np.array([float(Fraction(c) / s) for c in _centred_coeffs(sch, out)])
+    sine = np.array([q0 / (2 * math.pi) * math.sin(2 * math.pi * v / q0) / delta for v in m])
+    assert np.max(np.abs(got - sine)) < 1e-5
