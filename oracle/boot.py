@@ -185,7 +185,7 @@ def lintrans_planned(ct, scale, Dg, plan, pt_scale, keys, chain):
     n = ct.shape[-1]
     S = n // 2
     l = level(ct)
-    stride, t0, bb, gg = plan
+    stride, _, bb, gg = plan
     pts, giants = plan_plaintexts(Dg, plan, S, chain.mods[:l], pt_scale, n)
     mods_l = chain.mods_at(l)
     qs = chain.mods[:l]

@@ -77,6 +77,9 @@ def _lib():
     return _LIB
 
 
+# _u / _i / _ptr_array return the (possibly copied) arrays with their
+# pointers; callers keep those arrays bound to a local (named with a leading
+# underscore where nothing else reads it) so the memory outlives the C call.
 def _u(a):
     a = np.ascontiguousarray(a, dtype=np.uint64)
     return a, a.ctypes.data_as(_u64p)
@@ -140,7 +143,7 @@ def ntt_fwd(x, mods):
     x = np.array(x, dtype=np.uint64, copy=True, order="C")
     limbs, n = x.shape[-2], x.shape[-1]
     batch = x.size // (limbs * n) if x.size else 0
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_ntt_fwd(x.ctypes.data_as(_u64p), pm, limbs, batch, n)
     return x
 
@@ -149,7 +152,7 @@ def ntt_inv(x, mods):
     x = np.array(x, dtype=np.uint64, copy=True, order="C")
     limbs, n = x.shape[-2], x.shape[-1]
     batch = x.size // (limbs * n) if x.size else 0
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_ntt_inv(x.ctypes.data_as(_u64p), pm, limbs, batch, n)
     return x
 
@@ -161,7 +164,7 @@ def pointwise(op, a, b, mods):
     b, pb = _u(b)
     out = np.zeros_like(a)
     limbs, n = a.shape[-2], a.shape[-1]
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_pointwise(code, pa, pb, out.ctypes.data_as(_u64p), pm, limbs,
                             a.size // (limbs * n), n)
     return out
@@ -211,7 +214,7 @@ def modup(c_ntt, mods, L, K, alpha):
     B, n = c.shape[0], c.shape[-1]
     dn = digit_count(L, alpha)
     out = np.zeros((B, dn, L + K, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_modup(pc, out.ctypes.data_as(_u64p), pm, L, K, alpha, B, n)
     return out
 
@@ -219,10 +222,10 @@ def modup(c_ntt, mods, L, K, alpha):
 def key_inner(digits, key, galois, mods, L, K, alpha):
     """digits[B][dnum][L+K][n], key[dnum][2][L+K][n] -> acc[B][2][L+K][n]."""
     d, pd = _u(digits)
-    k, pk = _u(key)
+    _k, pk = _u(key)
     B, n = d.shape[0], d.shape[-1]
     out = np.zeros((B, 2, L + K, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_key_inner(pd, pk, int(galois), out.ctypes.data_as(_u64p), pm, L, K,
                             alpha, B, n)
     return out
@@ -233,7 +236,7 @@ def moddown(acc, mods, L, K):
     a, pa = _u(acc)
     B, n = a.shape[0], a.shape[-1]
     out = np.zeros((B, 2, L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_moddown(pa, out.ctypes.data_as(_u64p), pm, L, K, B, n)
     return out
 
@@ -241,10 +244,10 @@ def moddown(acc, mods, L, K):
 def keyswitch(d, key, mods, L, K, alpha):
     """d[B][L][n] (NTT) -> out[B][2][L][n]."""
     d, pd = _u(d)
-    k, pk = _u(key)
+    _k, pk = _u(key)
     B, n = d.shape[0], d.shape[-1]
     out = np.zeros((B, 2, L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_keyswitch(pd, pk, out.ctypes.data_as(_u64p), pm, L, K, alpha, B, n)
     return out
 
@@ -253,10 +256,10 @@ def rotate(ct, keys, galois, mods, L, K, alpha):
     """ct[B][2][L][n] -> out[nkeys][B][2][L][n] with hoisted ModUp."""
     c, pc = _u(ct)
     B, n = c.shape[0], c.shape[-1]
-    kept, karr = _ptr_array(keys)
-    g, pg = _u(galois)
+    _kept, karr = _ptr_array(keys)
+    _g, pg = _u(galois)
     out = np.zeros((len(keys), B, 2, L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_rotate(pc, karr, pg, len(keys), out.ctypes.data_as(_u64p), pm, L, K,
                          alpha, B, n)
     return out
@@ -266,10 +269,10 @@ def rotate_unhoisted(ct, keys, galois, mods, L, K, alpha):
     """ct[B][2][L][n] -> out[nkeys][B][2][L][n], automorphism before the key switch."""
     c, pc = _u(ct)
     B, n = c.shape[0], c.shape[-1]
-    kept, karr = _ptr_array(keys)
-    g, pg = _u(galois)
+    _kept, karr = _ptr_array(keys)
+    _g, pg = _u(galois)
     out = np.zeros((len(keys), B, 2, L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_rotate_unhoisted(pc, karr, pg, len(keys), out.ctypes.data_as(_u64p), pm, L, K,
                                    alpha, B, n)
     return out
@@ -280,7 +283,7 @@ def rescale(ct, mods):
     c, pc = _u(ct)
     B, lp1, n = c.shape[0], c.shape[2], c.shape[-1]
     out = np.zeros((B, 2, lp1 - 1, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_rescale(pc, out.ctypes.data_as(_u64p), pm, lp1, B, n)
     return out
 
@@ -288,10 +291,10 @@ def rescale(ct, mods):
 def mul_relin_rescale(a, b, rlk, mods, L, K, alpha):
     a, pa = _u(a)
     b, pb = _u(b)
-    r, pr = _u(rlk)
+    _r, pr = _u(rlk)
     B, n = a.shape[0], a.shape[-1]
     out = np.zeros((B, 2, L - 1, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_mul_relin_rescale(pa, pb, pr, out.ctypes.data_as(_u64p), pm, L, K,
                                     alpha, B, n)
     return out
@@ -300,12 +303,12 @@ def mul_relin_rescale(a, b, rlk, mods, L, K, alpha):
 def bsgs(x, diags, baby_keys, giant_keys, bb, gg, mods, L, K, alpha):
     """x[B][2][L][n], diags[gg][bb][L][n] -> y[B][2][L-1][n]."""
     xx, px = _u(x)
-    dg, pd = _u(diags)
-    kb, ab = _ptr_array(baby_keys)
-    kg, ag = _ptr_array(giant_keys)
+    _dg, pd = _u(diags)
+    _kb, ab = _ptr_array(baby_keys)
+    _kg, ag = _ptr_array(giant_keys)
     B, n = xx.shape[0], xx.shape[-1]
     out = np.zeros((B, 2, L - 1, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_bsgs(px, pd, ab, ag, bb, gg, out.ctypes.data_as(_u64p), pm, L, K,
                        alpha, B, n)
     return out
@@ -318,7 +321,7 @@ def mul_monomial(x, e, mods):
     x, px = _u(x)
     out = np.zeros_like(x)
     limbs, n = x.shape[-2], x.shape[-1]
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_mul_monomial(px, out.ctypes.data_as(_u64p), pm, limbs,
                                x.size // (limbs * n), n, int(e))
     return out
@@ -332,7 +335,7 @@ def modraise(x, mods_full):
     Lf = len(mods_full)
     P = x.size // (l * n)
     out = np.zeros(x.shape[:-2] + (Lf, n), dtype=np.uint64)
-    m, pm = _u(mods_full)
+    _m, pm = _u(mods_full)
     _lib().oracle_modraise(px, out.ctypes.data_as(_u64p), pm, l, Lf, P, n)
     return out
 
@@ -340,11 +343,11 @@ def modraise(x, mods_full):
 def conj_extract(ct, conj_key, mods, L, K, alpha):
     """ct[B][2][L][n] -> (re, im), each [B][2][L][n], slots 2 Re w and 2 Im w."""
     c, pc = _u(ct)
-    k, pk = _u(conj_key)
+    _k, pk = _u(conj_key)
     B, n = c.shape[0], c.shape[-1]
     re = np.zeros((B, 2, L, n), dtype=np.uint64)
     im = np.zeros((B, 2, L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_conj_extract(pc, pk, re.ctypes.data_as(_u64p), im.ctypes.data_as(_u64p),
                                pm, L, K, alpha, B, n)
     return re, im
@@ -353,10 +356,10 @@ def conj_extract(ct, conj_key, mods, L, K, alpha):
 def restore_merge(re, im, mods):
     """re, im [B][2][L][n] with slots a, b -> [B][2][L][n] with slots a + i b."""
     r, pr = _u(re)
-    i, pi = _u(im)
+    _im, pi = _u(im)
     B, L, n = r.shape[0], r.shape[2], r.shape[-1]
     out = np.zeros_like(r)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_restore_merge(pr, pi, out.ctypes.data_as(_u64p), pm, L, B, n)
     return out
 
@@ -367,8 +370,8 @@ def secret_galois(s, g, mods):
     s, ps = _i(s)
     n = s.shape[-1]
     out = np.zeros((len(mods), n), dtype=np.uint64)
-    m, pm = _u(mods)
-    _lib().oracle_secret_galois(ps, int(g), out.ctypes.data_as(_u64p), pm, len(m), n)
+    _m, pm = _u(mods)
+    _lib().oracle_secret_galois(ps, int(g), out.ctypes.data_as(_u64p), pm, len(_m), n)
     return out
 
 
@@ -376,8 +379,8 @@ def secret_square(s, mods):
     s, ps = _i(s)
     n = s.shape[-1]
     out = np.zeros((len(mods), n), dtype=np.uint64)
-    m, pm = _u(mods)
-    _lib().oracle_secret_square(ps, out.ctypes.data_as(_u64p), pm, len(m), n)
+    _m, pm = _u(mods)
+    _lib().oracle_secret_square(ps, out.ctypes.data_as(_u64p), pm, len(_m), n)
     return out
 
 
@@ -385,13 +388,13 @@ def keygen(s, sprime_ntt, a, e, mods, L, K, alpha):
     """Switching key s' -> s: [dnum][2][L+K][n]. a[dnum][L+K][n] uniform NTT
     residues, e[dnum][n] small error coefficients."""
     s, ps = _i(s)
-    sp, psp = _u(sprime_ntt)
+    _sp, psp = _u(sprime_ntt)
     a, pa = _u(a)
     e, pe = _i(e)
     n = s.shape[-1]
     dn = digit_count(L, alpha)
     out = np.zeros((dn, 2, L + K, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_keygen(ps, psp, pa, pe, out.ctypes.data_as(_u64p), pm, L, K, alpha, n)
     return out
 
@@ -412,7 +415,7 @@ def encrypt(m_coeffs, s, a, e, mods):
     e, pe = _i(e)
     L, n = len(mods), mm.shape[-1]
     out = np.zeros((2, L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_encrypt(pm_, ps, pa, pe, out.ctypes.data_as(_u64p), pm, L, n)
     return out
 
@@ -423,7 +426,7 @@ def decrypt(ct, s, mods):
     s, ps = _i(s)
     L, n = len(mods), c.shape[-1]
     out = np.zeros((L, n), dtype=np.uint64)
-    m, pm = _u(mods)
+    _m, pm = _u(mods)
     _lib().oracle_decrypt(pc, ps, out.ctypes.data_as(_u64p), pm, L, n)
     return out
 
