@@ -317,7 +317,9 @@ def run_b200(args):
 
     if not args.no_e2e:
         line["e2e"] = run_e2e(ctx, xs, refs, args, dev, stream, pg, world)
-    if not args.no_ks and rank == 0:
+    # the key-switch rates come from the single-GPU run; under torchrun every
+    # rank leaves together instead of waiting on rank 0's extra minutes
+    if not args.no_ks and rank == 0 and world == 1:
         del xs, refs
         torch.cuda.empty_cache()
         line["keyswitch"] = run_keyswitch(dev, hbm_peak, ipeak)
