@@ -63,6 +63,20 @@ def test_mul_monomial_half_is_i_on_slots(orc):
     assert np.array_equal(twice, neg)
 
 
+def test_mul_monomial_half_in_the_ntt_domain(orc):
+    """NTT(X^{n/2})[k] = psi^{(n/2)(2 brv(k) + 1)} = i_q (-1)^{brv(k)} with
+    i_q = psi^{n/2}: +i_q on the first n/2 evaluation slots, -i_q on the rest.
+    So X^{n/2} x is a pointwise product by those constants."""
+    mods = orc.gen_primes(N, 3)
+    x = u64(synth.uniform_residues((2, 3, N), mods, SEED, 15))
+    iq = [pow(int(orc.find_psi(int(q), N)), N // 2, int(q)) for q in mods]
+    assert all(v * v % int(q) == int(q) - 1 for v, q in zip(iq, mods))
+    c = np.array([[v] * (N // 2) + [int(q) - v] * (N // 2) for v, q in zip(iq, mods)],
+                 dtype=np.uint64)
+    want = orc.pointwise("mul", x, np.broadcast_to(c, x.shape).copy(), mods)
+    assert np.array_equal(orc.mul_monomial(x, N // 2, mods), want)
+
+
 # ------------------------------------------------------------------ modraise
 def test_modraise_is_the_centred_crt_lift(orc):
     """Coefficients over q_0..q_2 -> their centred integer X in (-Q/2, Q/2],
