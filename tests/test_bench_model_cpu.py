@@ -35,3 +35,26 @@ def test_ntt_launch_bytes_and_products():
     bytes_, mm = bench.ntt_launch_work(2100)
     assert bytes_ == 33600 * 2 * 2048 * 8 + 2100 * 2048 * 16
     assert mm == 33600 * 1024 * 11
+
+
+def test_traffic_is_reported_only_for_unchanged_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu figure only while the
+    kernel's sources hash to what they were at capture; after any change it
+    is null."""
+    import hashlib
+    import json
+    import os
+
+    src = tmp_path / "k.cu"
+    src.write_bytes(b"kernel v1")
+    (tmp_path / "profiles").mkdir()
+    entry = {"sources": ["k.cu"], "dram_bytes_per_launch": 12345,
+             "sources_sha256_16": hashlib.sha256(b"kernel v1").hexdigest()[:16]}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"k": entry}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("k") == 12345
+    assert bench.traffic_for("other") is None
+    src.write_bytes(b"kernel v2")
+    assert bench.traffic_for("k") is None
+    os.remove(tmp_path / "profiles" / "traffic.json")
+    assert bench.traffic_for("k") is None
