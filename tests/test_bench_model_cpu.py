@@ -58,3 +58,20 @@ def test_traffic_is_reported_only_for_unchanged_sources(tmp_path, monkeypatch):
     assert bench.traffic_for("k") is None
     os.remove(tmp_path / "profiles" / "traffic.json")
     assert bench.traffic_for("k") is None
+
+
+def test_clock_summary_decodes_the_nvml_reasons():
+    """Median SM clock under load and the named clock-event reasons (NVML bit
+    values: sw_power_cap 0x4, hw_slowdown 0x8, sw_thermal 0x20, hw_thermal 0x40,
+    power brake 0x80); idle and application-clock bits are not reasons."""
+    cs = bench.ClockSampler(None)
+    cs.max_mhz = 1965
+    cs.samples = [(1965, 0x0), (1900, 0x4), (1965, 0x4 | 0x8), (1950, 0x1 | 0x2)]
+    s = cs.summary()
+    assert s["sm_mhz"] == 1957.5 and s["sm_max_mhz"] == 1965 and s["samples"] == 4
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    cs.samples = [(1965, 0x20 | 0x40 | 0x80)]
+    assert cs.summary()["reasons"] == ["hw_power_brake_slowdown", "hw_thermal_slowdown",
+                                       "sw_thermal_slowdown"]
+    empty = bench.ClockSampler(None)
+    assert empty.summary()["reasons"] == ["unsampled"]
