@@ -11,6 +11,7 @@ the repository's oracle is never touched.
     python tests/mutation_sweep.py            # every slip, full pin suite each
     python tests/mutation_sweep.py 0 15 21    # chosen slips
     python tests/mutation_sweep.py --targeted # run only each slip's own pin
+    python tests/mutation_sweep.py --jobs 4   # four slips at a time, threads split between them
 """
 import os
 import shutil
@@ -236,8 +237,11 @@ def plant(index, dest):
     return copy
 
 
-def run(index, targeted=False, timeout=1800):
+def run(index, targeted=False, timeout=1800, threads=None):
     """Run the pins against a copy with slip `index`; return (caught, first failure)."""
+    env = dict(os.environ)
+    if threads:
+        env["OMP_NUM_THREADS"] = str(threads)
     with tempfile.TemporaryDirectory(prefix="oracle_slip_") as d:
         plant(index, d)
         cmd = [sys.executable, "-m", "pytest", *PINS, "-x", "-q", "--import-mode=append",
@@ -246,21 +250,30 @@ def run(index, targeted=False, timeout=1800):
             cmd += ["-k", MUTATIONS[index][5]]
         # `python -m pytest` puts its working directory first on sys.path, so
         # `import oracle` finds the planted copy ahead of the repository's one
-        r = subprocess.run(cmd, cwd=d, capture_output=True, text=True, timeout=timeout)
+        r = subprocess.run(cmd, cwd=d, capture_output=True, text=True, timeout=timeout, env=env)
     failed = [ln.split("::")[-1].split(" - ")[0] for ln in r.stdout.splitlines()
               if ln.startswith(("FAILED", "ERROR"))]
     return r.returncode != 0, (failed[0] if failed else "")
 
 
 def main(argv):
+    from concurrent.futures import ThreadPoolExecutor
+
     targeted = "--targeted" in argv
-    picks = [int(a) for a in argv if not a.startswith("--")] or range(len(MUTATIONS))
+    jobs = 1
+    if "--jobs" in argv:
+        k = argv.index("--jobs")
+        jobs = int(argv[k + 1])
+        argv = argv[:k] + argv[k + 2:]
+    picks = [int(a) for a in argv if not a.startswith("--")] or list(range(len(MUTATIONS)))
+    threads = max(1, (os.cpu_count() or 1) // jobs) if jobs > 1 else None
     missed = 0
-    for i in picks:
-        caught, first = run(i, targeted)
-        missed += not caught
-        print("%2d  %-7s %-55s %s" % (i, "caught" if caught else "MISSED", MUTATIONS[i][0], first),
-              flush=True)
+    with ThreadPoolExecutor(max_workers=jobs) as pool:
+        results = pool.map(lambda i: (i, run(i, targeted, threads=threads)), picks)
+        for i, (caught, first) in results:
+            missed += not caught
+            print("%2d  %-7s %-55s %s" % (i, "caught" if caught else "MISSED", MUTATIONS[i][0],
+                                          first), flush=True)
     return 1 if missed else 0
 
 
