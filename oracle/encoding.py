@@ -99,7 +99,8 @@ def encode_ntt(z, mods, scale, n):
 
 
 def embedding_matrix(n):
-    """U[j][k] = zeta^(k e_j), j, k < n/2, zeta = exp(i pi / n), e_j = 5^j mod 2n.
+    """U[j][k] = zeta^(k e_j), j, k < n/2, zeta = exp(i pi / n), e_j = 5^j mod 2n
+    (reading R14 of the design notes).
 
     Slot j of a polynomial with real coefficients m is sum_k m_k zeta^(k e_j);
     since zeta^(n/2 e_j) = i (e_j = 1 mod 4), the slots are U (m_lo + i m_hi)
@@ -142,6 +143,10 @@ def lintrans_plaintexts(M, bb, gg, mods, scale, n):
 
 
 # ---------------------------------------------------------------- factored transforms
+#
+# Reading R16 of the design notes: the pages time coeff_to_slot and
+# slot_to_coeff (Kestrel engine write-up, boot profile in section 5.3) but give
+# no factorization; this is the textbook special-FFT one.
 #
 # U evaluates V(X) = sum_k v_k X^k at the S = n/2 points w_j = zeta^(5^j).  Split
 # V(X) = E(X^2) + X O(X^2).  The squares w_j^2 are the points of the same problem
