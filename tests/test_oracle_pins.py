@@ -286,8 +286,11 @@ def _crt(res_cols, mods):
     return x % Q, Q
 
 
-@pytest.mark.parametrize("L,K,alpha", [(6, 2, 2), (5, 2, 2), (4, 1, 1)])
+@pytest.mark.parametrize("L,K,alpha", [(6, 2, 2), (5, 2, 2), (4, 1, 1), (7, 2, 3), (1, 1, 1),
+                                       (1, 3, 1)])
 def test_modup_crt_identity(orc, L, K, alpha):
+    """Including the single-prime chain L = 1 (the level a refresh starts
+    from) and a ragged last digit (7 = 3 + 3 + 1)."""
     p = Params(L, K, alpha)
     mods = [int(x) for x in orc.gen_primes(N, L + K)]
     m64 = np.array(mods, dtype=np.uint64)
@@ -309,8 +312,8 @@ def test_modup_crt_identity(orc, L, K, alpha):
                 assert int(coef[t, k]) == (X + u * Qj) % mods[t]
 
 
-def test_moddown_floor_identity(orc):
-    L, K = 4, 2
+@pytest.mark.parametrize("L,K", [(4, 2), (1, 1), (1, 3), (3, 1)])
+def test_moddown_floor_identity(orc, L, K):
     mods = [int(x) for x in orc.gen_primes(N, L + K)]
     m64 = np.array(mods, dtype=np.uint64)
     acc_coef = _rand_res((1, 2, L + K, N), m64, 13)
@@ -356,6 +359,23 @@ def test_rotation_decrypts_to_slot_rotation_config1(orc):
     out = orc.rotate(ct[None], [key], np.array([5], dtype=np.uint64), sch.mods, 4, 1, 1)
     err = np.max(np.abs(sch.decrypt_slots(out[0, 0]) - rot_left(z, 1)))
     assert err < 1e-8
+
+
+@pytest.mark.parametrize("K", [1, 2])
+def test_rotation_on_a_single_prime_chain(orc, K):
+    """L = 1, the level a refresh starts from: one digit, K special primes,
+    the message at scale 2^40 below q_0.  Rotation by 3 and conjugation
+    decrypt to the rotated and conjugated slots."""
+    scale = 2**40
+    sch = Scheme(orc, Params(1, K, 1), SEED + 12 + K)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 25).numpy() + \
+        1j * synth.uniform_real((SLOTS,), -1, 1, SEED, 26).numpy()
+    ct = sch.encrypt_slots(z, scale)
+    gal = [galois_for_rotation(3), 2 * N - 1]
+    keys = [sch.keygen_galois(g) for g in gal]
+    out = orc.rotate(ct[None], keys, np.array(gal, dtype=np.uint64), sch.mods, 1, K, 1)
+    assert np.max(np.abs(sch.decrypt_slots(out[0, 0], scale) - rot_left(z, 3))) < 1e-6
+    assert np.max(np.abs(sch.decrypt_slots(out[1, 0], scale) - np.conj(z))) < 1e-6
 
 
 def test_hoisted_rotations_small_digits(orc):
