@@ -378,6 +378,23 @@ def test_rotation_on_a_single_prime_chain(orc, K):
     assert np.max(np.abs(sch.decrypt_slots(out[1, 0], scale) - np.conj(z))) < 1e-6
 
 
+def test_rotation_at_the_boot_chain_size(orc):
+    """The boot chain itself: 2100 ciphertext primes, 60 special, 35 digits of
+    60 (about 20 s).  Rotation by 8 with config 5's Galois element 1505 = 5^8
+    decrypts to the rotated slots; the decryption reads q_0..q_2 only, where
+    m + e is far below Q/2."""
+    assert galois_for_rotation(8) == 1505
+    p = Params(2100, 60, 60)
+    sch = Scheme(orc, p, SEED + 15)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 27).numpy()
+    ct = sch.encrypt_slots(z)
+    key = sch.keygen_galois(1505)
+    out = orc.rotate(ct[None], [key], np.array([1505], dtype=np.uint64), sch.mods, 2100, 60, 60)
+    assert out.shape == (1, 1, 2, 2100, N)
+    low = np.ascontiguousarray(out[0, 0][:, :3])
+    assert np.max(np.abs(sch.decrypt_slots(low) - rot_left(z, 8))) < 1e-8
+
+
 def test_hoisted_rotations_small_digits(orc):
     """Ragged digits (L = 5, alpha = 2) and several keys on one ModUp."""
     p = Params(5, 2, 2)
