@@ -495,3 +495,30 @@ def test_bsgs_banded_matvec(orc):
     y = orc.bsgs(ct[None], diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
     sc = sch.rescaled_scale(SCALE * SCALE, p.L)
     assert np.max(np.abs(sch.decrypt_slots(y[0], sc) - M @ x)) < 1e-8
+
+
+def test_bsgs_at_the_layer_chain_size(orc):
+    """Config 4's shape: 112 + 8 primes, bb = gg = 32, 31 baby and 31 giant
+    keys (about 30 s).  M has nonzero diagonals at offsets spread over the
+    32 x 32 (giant, baby) grid, including both ends and both sides of a giant
+    boundary; absent diagonals are zero plaintexts.  Decrypts (through
+    q_0..q_2) to M x."""
+    p = Params(112, 8, 8)
+    bb = gg = 32
+    sch = Scheme(orc, p, SEED + 16)
+    offs = [0, 1, 31, 32, 33, 100, 511, 1000, 1023]
+    vals = synth.uniform_real((len(offs), SLOTS), -1 / 8, 1 / 8, SEED, 60).numpy()
+    idx = np.arange(SLOTS)
+    M = np.zeros((SLOTS, SLOTS))
+    diags = np.zeros((gg, bb, p.L, N), dtype=np.uint64)
+    for v, k in zip(vals, offs):
+        M[idx, (idx + k) % SLOTS] = v
+        g, b = divmod(k, bb)
+        diags[g, b] = orc.encode_ntt(np.roll(v, bb * g), sch.q, SCALE, N)
+    baby = [sch.keygen_galois(galois_for_rotation(b)) for b in range(1, bb)]
+    giant = [sch.keygen_galois(galois_for_rotation(bb * g)) for g in range(1, gg)]
+    x = synth.uniform_real((SLOTS,), -1, 1, SEED, 61).numpy()
+    y = orc.bsgs(sch.encrypt_slots(x)[None], diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    low = np.ascontiguousarray(y[0][:, :3])
+    assert np.max(np.abs(sch.decrypt_slots(low, sc) - M @ x)) < 1e-8
