@@ -45,6 +45,8 @@ def test_library_path_is_in_tree():
 
 def test_product_primes_match_oracle(orc):
     assert primes(300) == [int(x) for x in orc.gen_primes(N, 300)]
+    # the whole boot chain: 2100 ciphertext and 60 special primes
+    assert primes(2160) == [int(x) for x in orc.gen_primes(N, 2160)]
 
 
 def test_primes_argument_checks():
