@@ -97,3 +97,18 @@ def test_calls_reject_null_context():
     assert "null context" in lib.ckks_last_error().decode()
     assert lib.ckks_ctx_set_conversion(None, 1) == EINVAL
     assert lib.ckks_selftest_wait_expiry(None) == EINVAL
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the compiled library every call raises; nothing falls back to
+    a CPU path."""
+    from rns_ckks_polynomial_b200 import Context
+    ps = primes(4)
+    monkeypatch.setattr(native, "_LIB", None)
+    monkeypatch.setattr(native._build, "LIB", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        native.lib()
+    with pytest.raises(RuntimeError, match="not built"):
+        Context(ps[:3], ps[3:], 1)
+    with pytest.raises(RuntimeError, match="not built"):
+        primes(4)
