@@ -140,6 +140,20 @@ int ckks_selftest_wait_expiry(const ckks_ctx *ctx);
 enum { CKKS_CONV_AUTO = 0, CKKS_CONV_INTEGER = 1, CKKS_CONV_TENSOR = 2 };
 int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine);
 
+/* Declares that the switching keys passed to this context's calls were made
+ * for a chain of key_L >= L ciphertext primes q_0..q_{key_L-1} (and the same
+ * special primes): layout [dnum_key][2][key_L + K][n] with dnum_key =
+ * ceil(key_L / alpha).  The calls then read ciphertext prime t < L at key row
+ * t, special prime k at row key_L + k, and only the first ceil(L / alpha)
+ * digits.  A key reduced modulo a divisor of its modulus is a key for that
+ * divisor, so one key set made at the top of a chain serves the context of
+ * every level below it; the digits must be the same contiguous blocks of
+ * alpha primes.  The default is key_L = L.  Takes effect for calls issued
+ * after it returns; do not change it while another host thread issues calls
+ * on the same context.  CKKS_EINVAL for a null context or key_L outside
+ * [L, 4096]. */
+int ckks_ctx_set_key_chain(ckks_ctx *ctx, int key_L);
+
 /* Context parameters: writes L, K, alpha, dnum, n (any pointer may be NULL). */
 int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n);
 

@@ -84,6 +84,20 @@ class Context:
 
     CONVERSION = {"auto": 0, "integer": 1, "tensor": 2}
 
+    @property
+    def _kshape(self):
+        """Shape of a switching key for this context: [dnum][2][L+K][n], or the
+        longer chain's layout after set_key_chain."""
+        kl = getattr(self, "key_L", self.L)
+        return ((kl + self.alpha - 1) // self.alpha, 2, kl + self.K, self.n)
+
+    def set_key_chain(self, key_L):
+        """Keys passed from now on were made for a chain of key_L >= L
+        ciphertext primes (the same special primes and digits): one key set
+        made at the top level serves the context of every lower level."""
+        check("ckks_ctx_set_key_chain", lib().ckks_ctx_set_key_chain(self._h, int(key_L)))
+        self.key_L = int(key_L)
+
     def set_conversion(self, engine):
         """Where ModUp/ModDown basis conversions run: "auto" (tensor cores from 8
         source primes on), "integer" (integer pipes) or "tensor" (int8 tensor
@@ -169,7 +183,7 @@ class Context:
         B = digits.shape[0]
         LK = self.L + self.K
         _ptr(digits, "digits", (B, self.dnum, LK, self.n))
-        _ptr(key, "key", (self.dnum, 2, LK, self.n))
+        _ptr(key, "key", self._kshape)
         out = self._empty(B, 2, LK, self.n) if out is None else out
         check("ckks_key_inner", lib().ckks_key_inner(self._h, _ptr(digits, "digits"), _ptr(key, "key"),
                                                      int(galois), _ptr(out, "acc"), B,
@@ -188,7 +202,7 @@ class Context:
     def keyswitch(self, d, key, out=None, ws=None):
         B = d.shape[0]
         _ptr(d, "d", (B, self.L, self.n))
-        _ptr(key, "key", (self.dnum, 2, self.L + self.K, self.n))
+        _ptr(key, "key", self._kshape)
         out = self._empty(B, 2, self.L, self.n) if out is None else out
         ws, wp = self._ws(ws, OP_KEYSWITCH, B)
         check("ckks_keyswitch", lib().ckks_keyswitch(self._h, _ptr(d, "d"), _ptr(key, "key"),
@@ -200,7 +214,7 @@ class Context:
         B = ct.shape[0]
         nk = len(keys)
         _ptr(ct, "ct", (B, 2, self.L, self.n))
-        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", (self.dnum, 2, self.L + self.K, self.n)).value
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", self._kshape).value
                                         for k in keys])
         gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
         out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
@@ -214,7 +228,7 @@ class Context:
         B = ct.shape[0]
         nk = len(keys)
         _ptr(ct, "ct", (B, 2, self.L, self.n))
-        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", (self.dnum, 2, self.L + self.K, self.n)).value
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", self._kshape).value
                                         for k in keys])
         gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
         out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
@@ -237,7 +251,7 @@ class Context:
         B = a.shape[0]
         _ptr(a, "a", (B, 2, self.L, self.n))
         _ptr(b, "b", (B, 2, self.L, self.n))
-        _ptr(rlk, "rlk", (self.dnum, 2, self.L + self.K, self.n))
+        _ptr(rlk, "rlk", self._kshape)
         out = self._empty(B, 2, self.L - 1, self.n) if out is None else out
         ws, wp = self._ws(ws, OP_MRR, B)
         check("ckks_mul_relin_rescale",
@@ -250,7 +264,7 @@ class Context:
         B = x.shape[0]
         _ptr(x, "x", (B, 2, self.L, self.n))
         _ptr(diags, "diags", (gg, bb, self.L, self.n))
-        kshape = (self.dnum, 2, self.L + self.K, self.n)
+        kshape = self._kshape
         if len(baby_keys) != bb - 1 or len(giant_keys) != gg - 1:
             raise ValueError("need bb-1 baby keys and gg-1 giant keys")
         bk = (C.c_void_p * max(1, bb - 1))(*[_ptr(k, "baby key", kshape).value for k in baby_keys])

@@ -36,6 +36,11 @@ struct __align__(16) PrimeConst {
 // Device tables owned by a context (struct of device pointers, passed by value).
 struct Tables {
     int L, K, alpha, dnum, LK;
+    // Switching keys may be made for a longer chain of key_L >= L ciphertext
+    // primes (one key set serving the contexts of every lower level): ciphertext
+    // prime t sits at key row t, special prime k at key row key_L + k, and
+    // each (digit, component) block holds key_LK = key_L + K rows.
+    int key_L, key_LK;
     bool special;               // every prime is 2^60 - delta with delta < 2^32
     const PrimeConst *pc;       // [L+K]
     const ulonglong2 *tw_fwd;   // [L+K][n]: {psi^brv(k), Shoup}; k = 0 unused

@@ -230,6 +230,7 @@ static int build_tables(ckks_ctx *ctx)
     const std::vector<u64> &m = ctx->mods;
     Tables &T = ctx->t;
     T.L = L; T.K = K; T.alpha = alpha; T.dnum = dnum; T.LK = LK;
+    T.key_L = L; T.key_LK = LK;
 
     std::vector<PrimeConst> pc(LK);
     std::vector<ulonglong2> fw((size_t)LK * n), iw((size_t)LK * n);
@@ -435,6 +436,16 @@ extern "C" int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine)
     if (engine != CKKS_CONV_AUTO && engine != CKKS_CONV_INTEGER && engine != CKKS_CONV_TENSOR)
         return set_error(CKKS_EINVAL, "unknown conversion engine");
     ctx->conv_engine.store(engine, std::memory_order_relaxed);
+    return CKKS_OK;
+}
+
+extern "C" int ckks_ctx_set_key_chain(ckks_ctx *ctx, int key_L)
+{
+    CKKS_TRY(check_ctx(ctx));
+    if (key_L < ctx->L || key_L > 4096)
+        return set_error(CKKS_EINVAL, "key_L must be in [L, 4096]");
+    ctx->t.key_L = key_L;
+    ctx->t.key_LK = key_L + ctx->K;
     return CKKS_OK;
 }
 

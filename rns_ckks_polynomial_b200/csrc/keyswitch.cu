@@ -258,13 +258,15 @@ __global__ void __launch_bounds__(kKiThreads, 4) key_inner_kernel(const u64 *__r
     const size_t LKn = (size_t)T.LK * kN;
     const size_t bstride = (size_t)T.dnum * LKn;  // between the digit sets of consecutive ciphertexts
     const u64 *dg = digits + (size_t)(hoisted ? b0 : r * per_key + b0) * bstride + (size_t)t * kN + src;
-    const u64 *kp = kl.key[r] + (size_t)t * kN + k;
+    const size_t kLKn = (size_t)T.key_LK * kN;  // key rows per (digit, component)
+    const int kt = t < T.L ? t : t - T.L + T.key_L;
+    const u64 *kp = kl.key[r] + (size_t)kt * kN + k;
     u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
 #pragma unroll
     for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
 #pragma unroll 2
     for (int j = 0; j < T.dnum; ++j) {
-        const u64 kb = __ldg(kp + (size_t)(2 * j) * LKn), ka = __ldg(kp + (size_t)(2 * j + 1) * LKn);
+        const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
         const u64 *dj = dg + (size_t)j * LKn;
         u64 d[kKiB];
 #pragma unroll

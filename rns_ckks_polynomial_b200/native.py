@@ -23,6 +23,7 @@ SIGNATURES = {
     "ckks_ctx_params": (C.c_int, [_vp] + [C.POINTER(C.c_int)] * 5),
     "ckks_device_status": (C.c_int, [_vp]),
     "ckks_ctx_set_conversion": (C.c_int, [_vp, C.c_int]),
+    "ckks_ctx_set_key_chain": (C.c_int, [_vp, C.c_int]),
     "ckks_selftest_wait_expiry": (C.c_int, [_vp]),
     "ckks_workspace_bytes": (C.c_size_t, [_vp, C.c_int, C.c_int, C.c_int]),
     "ckks_ntt_fwd": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),

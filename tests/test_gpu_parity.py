@@ -474,3 +474,41 @@ def test_unhoisted_rotation_order(orc):
     ctx2.device_status()
     assert_bits_equal(got, orc.rotate_unhoisted(ct, [key], np.array([25], dtype=np.uint64), mods, 40, 20, 20),
                       "rotate_unhoisted, tensor-core conversion")
+
+
+# ------------------------------------------------------------------ keys of a longer chain
+@pytest.mark.parametrize("L,K,alpha,l", [(6, 2, 2, 3), (7, 2, 3, 4), (20, 3, 7, 13), (5, 1, 1, 1)])
+def test_key_chain_serves_lower_levels(orc, L, K, alpha, l):
+    """A context on q_0..q_{l-1} (with the top chain's special primes) given
+    keys made for all L primes (set_key_chain(L)): key switch, rotation and
+    relinearised product bit-exact against the oracle run with the keys cut
+    down to level l.  (5, 1, 1, 1) is the single-prime chain a refresh starts
+    from."""
+    from oracle.boot import Chain
+
+    from rns_ckks_polynomial_b200 import Context
+    mods = [int(x) for x in orc.gen_primes(N, L + K)]
+    m64 = np.array(mods, dtype=np.uint64)
+    chain = Chain(m64, L, K, alpha)
+    m_l = chain.mods_at(l)
+    ctx = Context(mods[:l], mods[L:], alpha)
+    try:
+        ctx.set_key_chain(L)
+        key = _res((Params(L, K, alpha).dnum, 2, L + K, N), m64, 300)
+        key_l = chain.key_at(key, l)
+        d = _res((2, l, N), m_l[:l], 301)
+        assert_bits_equal(host(ctx.keyswitch(dev(d), dev(key))),
+                          orc.keyswitch(d, key_l, m_l, l, K, alpha), "keyswitch, level %d" % l)
+        ct = _res((2, 2, l, N), m_l[:l], 302)
+        assert_bits_equal(host(ctx.rotate(dev(ct), [dev(key)], [5])),
+                          orc.rotate(ct, [key_l], np.array([5], dtype=np.uint64), m_l, l, K, alpha),
+                          "rotate, level %d" % l)
+        if l >= 2:
+            a, b = _res((1, 2, l, N), m_l[:l], 303), _res((1, 2, l, N), m_l[:l], 304)
+            assert_bits_equal(host(ctx.mul_relin_rescale(dev(a), dev(b), dev(key))),
+                              orc.mul_relin_rescale(a, b, key_l, m_l, l, K, alpha),
+                              "mul_relin_rescale, level %d" % l)
+        with pytest.raises(CkksError):
+            ctx.set_key_chain(l - 1)
+    finally:
+        ctx.close()
