@@ -17,6 +17,7 @@ N = 2048
 PW = {"mul": 0, "add": 1, "sub": 2}
 OP_MODUP, OP_MODDOWN, OP_KEYSWITCH, OP_ROTATE, OP_RESCALE, OP_MRR, OP_BSGS = 1, 2, 3, 4, 5, 6, 7
 OP_ROTATE_UNHOISTED = 8
+OP_MODRAISE, OP_CONJ_EXTRACT = 9, 10
 
 
 def primes(count, n=N):
@@ -274,6 +275,69 @@ class Context:
         check("ckks_bsgs_lintrans",
               lib().ckks_bsgs_lintrans(self._h, _ptr(x, "x"), _ptr(diags, "diags"), bk, gk, bb, gg,
                                        _ptr(out, "y"), B, wp, _stream(x)))
+        return out
+
+    # ------------------------------------------------------------ refresh building blocks
+    def pointwise_scalar(self, op, a, k, out=None, limb_begin=0):
+        """out = a op k[limb] over a[..., limbs, n]; k: device int64 tensor of
+        `limbs` residues."""
+        out = torch.empty_like(a) if out is None else out
+        limbs = a.shape[-2]
+        batch = a.numel() // (limbs * self.n) if a.numel() else 0
+        _ptr(k, "k", (limbs,))
+        check("ckks_pointwise_scalar",
+              lib().ckks_pointwise_scalar(self._h, PW[op], _ptr(a, "a"), _ptr(k, "k"), _ptr(out, "out"),
+                                          batch, limb_begin, limbs, _stream(a)))
+        return out
+
+    def add_const_c0(self, ct, k):
+        """In place: component 0 of every ciphertext of ct[B][2][L][n] plus k[limb]."""
+        B = ct.shape[0]
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        _ptr(k, "k", (self.L,))
+        check("ckks_add_const_c0", lib().ckks_add_const_c0(self._h, _ptr(ct, "ct"), _ptr(k, "k"), B,
+                                                           _stream(ct)))
+        return ct
+
+    def mul_i(self, x, out=None, limb_begin=0):
+        """X^{n/2} x (every slot times i) over x[..., limbs, n], NTT domain."""
+        out = torch.empty_like(x) if out is None else out
+        limbs = x.shape[-2]
+        batch = x.numel() // (limbs * self.n) if x.numel() else 0
+        check("ckks_mul_i", lib().ckks_mul_i(self._h, _ptr(x, "in"), _ptr(out, "out"), batch, limb_begin,
+                                             limbs, _stream(x)))
+        return out
+
+    def conj_extract(self, ct, conj_key, ws=None):
+        """ct[B][2][L][n] -> (re, im) with slots 2 Re w and 2 Im w."""
+        B = ct.shape[0]
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        _ptr(conj_key, "conj_key", self._kshape)
+        re, im = self._empty(B, 2, self.L, self.n), self._empty(B, 2, self.L, self.n)
+        ws, wp = self._ws(ws, OP_CONJ_EXTRACT, B)
+        check("ckks_conj_extract",
+              lib().ckks_conj_extract(self._h, _ptr(ct, "ct"), _ptr(conj_key, "conj_key"), _ptr(re, "re"),
+                                      _ptr(im, "im"), B, wp, _stream(ct)))
+        return re, im
+
+    def restore_merge(self, re, im, out=None):
+        """re + X^{n/2} im over [B][2][L][n]: slots a + i b."""
+        B = re.shape[0]
+        _ptr(re, "re", (B, 2, self.L, self.n))
+        _ptr(im, "im", (B, 2, self.L, self.n))
+        out = torch.empty_like(re) if out is None else out
+        check("ckks_restore_merge", lib().ckks_restore_merge(self._h, _ptr(re, "re"), _ptr(im, "im"),
+                                                             _ptr(out, "out"), B, _stream(re)))
+        return out
+
+    def modraise(self, x, out=None, ws=None):
+        """x[B][2][l][n] over q_0..q_{l-1} -> [B][2][L][n], each coefficient
+        lifted to its centred value and reduced modulo every prime."""
+        B, _, l, _ = x.shape
+        out = self._empty(B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_MODRAISE, B, l)
+        check("ckks_modraise", lib().ckks_modraise(self._h, _ptr(x, "in"), l, _ptr(out, "out"), B, wp,
+                                                   _stream(x)))
         return out
 
     # ------------------------------------------------------------ measurement

@@ -120,6 +120,28 @@ static int launch_conv(const Map &m, int max_targets, int jobs, const Tables &T,
     return CKKS_OK;
 }
 
+// modraise conversion: job z = polynomial; sources its l Garner digits and the
+// sign row; targets the primes l..L-1.  matp[s][t] = [q_0..q_{s-1}]_{q_t} for
+// s < l and [-Q]_{q_t} for s = l, so the exact sum is the centred lift.
+struct RaiseConvMap {
+    const u64 *dg;
+    u64 *out;
+    const u64 *matp;  // [l+1][L]
+    int l, L;
+    __device__ __forceinline__ int sources(int) const { return l + 1; }
+    __device__ __forceinline__ int targets(int) const { return L - l; }
+    __device__ __forceinline__ const u64 *src(int z) const { return dg + (size_t)z * (l + 1) * kN; }
+    __device__ __forceinline__ u64 mat(int, int s, int t) const { return matp[(size_t)s * L + l + t]; }
+    __device__ __forceinline__ u64 *dst(int z, int t) const { return out + ((size_t)z * L + l + t) * kN; }
+    __device__ __forceinline__ int prime(int, int t) const { return l + t; }
+};
+
+int raise_conv(const Tables &T, const u64 *dg, u64 *out, const u64 *matp, int l, int P, cudaStream_t s)
+{
+    RaiseConvMap m{dg, out, matp, l, T.L};
+    return launch_conv(m, T.L - l, P, T, s);
+}
+
 // ---------------------------------------------------------------- ModUp
 // INTT of source limb i of polynomial b; the load also writes the input limb
 // (NTT domain) into its own digit, the store multiplies by [(Q_j/q_i)^-1].

@@ -29,6 +29,12 @@ SIGNATURES = {
     "ckks_ntt_fwd": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_ntt_inv": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_pointwise": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_pointwise_scalar": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_add_const_c0": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp]),
+    "ckks_mul_i": (C.c_int, [_vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_conj_extract": (C.c_int, [_vp, _vp, _vp, _vp, _vp, C.c_int, _vp, _vp]),
+    "ckks_restore_merge": (C.c_int, [_vp, _vp, _vp, _vp, C.c_int, _vp]),
+    "ckks_modraise": (C.c_int, [_vp, _vp, C.c_int, _vp, C.c_int, _vp, _vp]),
     "ckks_automorph": (C.c_int, [_vp, _vp, _vp, C.c_int, C.c_int, C.c_uint32, _vp]),
     "ckks_modup": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp, _vp]),
     "ckks_modup_noalloc": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp]),

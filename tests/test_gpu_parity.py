@@ -512,3 +512,68 @@ def test_key_chain_serves_lower_levels(orc, L, K, alpha, l):
             ctx.set_key_chain(l - 1)
     finally:
         ctx.close()
+
+
+# ------------------------------------------------------------------ refresh building blocks
+def test_mul_i_scalar_ops_and_c0_constant(orc):
+    """X^{n/2} (slots times i) against the oracle's coefficient-domain
+    monomial product; products and sums with a per-limb constant; a constant
+    added to component 0 only."""
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    LK = p.L + p.K
+    x = _res((3, LK, N), mods, 400)
+    assert_bits_equal(host(ctx.mul_i(dev(x))), orc.mul_monomial(x, N // 2, mods), "mul_i")
+    k = np.ascontiguousarray(_res((LK, 1), mods, 401)[:, 0])
+    kb = np.ascontiguousarray(np.broadcast_to(k[:, None], x.shape))
+    for op in ("mul", "add", "sub"):
+        assert_bits_equal(host(ctx.pointwise_scalar(op, dev(x), dev(k))),
+                          orc.pointwise(op, x, kb, mods), "pointwise_scalar %s" % op)
+    ct = _res((2, 2, p.L, N), mods[:p.L], 402)
+    want = ct.copy()
+    want[:, 0] = orc.pointwise("add", ct[:, 0], np.ascontiguousarray(
+        np.broadcast_to(k[:p.L, None], ct[:, 0].shape)), mods[:p.L])
+    assert_bits_equal(host(ctx.add_const_c0(dev(ct), dev(np.ascontiguousarray(k[:p.L])))), want,
+                      "add_const_c0")
+
+
+def test_conj_extract_and_restore_merge(orc):
+    """Bit-exact against the oracle, and the slots decrypt to 2 Re w, 2 Im w,
+    then to 2 w after the merge."""
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 40)
+    w = synth.uniform_real((SLOTS,), -1, 1, SEED, 410).numpy() + \
+        1j * synth.uniform_real((SLOTS,), -1, 1, SEED, 411).numpy()
+    ct = sch.encrypt_slots(w)[None]
+    ck = sch.keygen_galois(2 * N - 1)
+    re, im = ctx.conj_extract(dev(ct), dev(ck))
+    want_re, want_im = orc.conj_extract(ct, ck, sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(host(re), want_re, "conj_extract re")
+    assert_bits_equal(host(im), want_im, "conj_extract im")
+    merged = ctx.restore_merge(re, im)
+    assert_bits_equal(host(merged), orc.restore_merge(want_re, want_im, sch.q), "restore_merge")
+    assert np.max(np.abs(sch.decrypt_slots(host(re)[0], 2 * SCALE) - w.real)) < 1e-8
+    assert np.max(np.abs(sch.decrypt_slots(host(merged)[0], 2 * SCALE) - w)) < 1e-8
+
+
+@pytest.mark.parametrize("L,K,alpha,l", [(6, 2, 2, 1), (6, 2, 2, 3), (6, 2, 2, 6), (40, 4, 4, 19),
+                                         (80, 4, 4, 63)])
+def test_modraise(orc, L, K, alpha, l):
+    """The centred lift onto the whole chain, bit-exact against the oracle;
+    coefficients 0, 1, (Q-1)/2, (Q+1)/2 and Q-1 sit at the start of the
+    first polynomial, where the sign decision is tightest."""
+    ctx = context(L, K, alpha)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    q = [int(v) for v in mods[:l]]
+    Q = 1
+    for v in q:
+        Q *= v
+    coef = _res((2, 2, l, N), mods[:l], 420)
+    for j, X in enumerate([0, 1, (Q - 1) // 2, (Q + 1) // 2, Q - 1]):
+        for i in range(l):
+            coef[0, 0, i, j] = X % q[i]
+    x = orc.ntt_fwd(coef, mods[:l])
+    got = host(ctx.modraise(dev(x)))
+    assert_bits_equal(got, orc.modraise(x, mods[:L]), "modraise l=%d" % l)
