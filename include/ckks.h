@@ -316,6 +316,23 @@ int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *d
                        int bb, int gg, uint64_t *y, int batch, void *ws,
                        ckks_stream_t stream);
 
+/* The same transform for a matrix whose nonzero diagonals sit at the offsets
+ * stride (t0 + bb g + b), g < gg, b < bb (a group of butterfly stages of a
+ * factored coeff_to_slot / slot_to_coeff):
+ *   y = Rescale( sum_g Rot_{G_g}( sum_b diags[g][b] * Rot_{stride b}(x) ) ),
+ *   G_g = stride (t0 + bb g) mod n/2,
+ * with diags[g][b] = Encode(rot_{-G_g}(diag_{G_g + stride b})) (zeros where
+ * the diagonal is absent).  baby_keys[b-1] rotates by stride b (Galois
+ * 5^{stride b}); giant_keys has gg entries, giant_keys[g] rotating by G_g
+ * (it may be NULL where G_g = 0, which is not rotated).  stride = 1, t0 = 0
+ * is ckks_bsgs_lintrans.  Limits as ckks_bsgs_lintrans, plus stride >= 1,
+ * stride (bb - 1) < n/2, |t0| <= n/2.
+ * ws: ckks_workspace_bytes(CKKS_OP_BSGS, batch, bb * 1000 + gg). */
+int ckks_bsgs_lintrans_plan(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                            const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
+                            int stride, int t0, int bb, int gg, uint64_t *y, int batch, void *ws,
+                            ckks_stream_t stream);
+
 /* ---- building blocks of the bootstrapping refresh (Kestrel engine write-up,
  * the boot profile in section 5.3; the forms are the textbook ones, as the
  * oracle reads them). */

@@ -277,6 +277,27 @@ class Context:
                                        _ptr(out, "y"), B, wp, _stream(x)))
         return out
 
+    def bsgs_lintrans_plan(self, x, diags, baby_keys, giant_keys, plan, out=None, ws=None):
+        """The BSGS transform over a strided window of diagonals, plan =
+        (stride, t0, bb, gg): baby_keys rotate by stride b (b = 1..bb-1),
+        giant_keys[g] by stride (t0 + bb g) mod n/2 (None where that is 0)."""
+        stride, t0, bb, gg = (int(v) for v in plan)
+        B = x.shape[0]
+        _ptr(x, "x", (B, 2, self.L, self.n))
+        _ptr(diags, "diags", (gg, bb, self.L, self.n))
+        kshape = self._kshape
+        if len(baby_keys) != bb - 1 or len(giant_keys) != gg:
+            raise ValueError("need bb-1 baby keys and gg giant keys")
+        bk = (C.c_void_p * max(1, bb - 1))(*[_ptr(k, "baby key", kshape).value for k in baby_keys])
+        gk = (C.c_void_p * gg)(*[None if k is None else _ptr(k, "giant key", kshape).value
+                                 for k in giant_keys])
+        out = self._empty(B, 2, self.L - 1, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_BSGS, B, bb * 1000 + gg)
+        check("ckks_bsgs_lintrans_plan",
+              lib().ckks_bsgs_lintrans_plan(self._h, _ptr(x, "x"), _ptr(diags, "diags"), bk, gk, stride,
+                                            t0, bb, gg, _ptr(out, "y"), B, wp, _stream(x)))
+        return out
+
     # ------------------------------------------------------------ refresh building blocks
     def pointwise_scalar(self, op, a, k, out=None, limb_begin=0):
         """out = a op k[limb] over a[..., limbs, n]; k: device int64 tensor of

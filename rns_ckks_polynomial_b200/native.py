@@ -49,6 +49,8 @@ SIGNATURES = {
     "ckks_mul_relin_rescale": (C.c_int, [_vp, _vp, _vp, _vp, _vp, C.c_int, _vp, _vp]),
     "ckks_bsgs_lintrans": (C.c_int, [_vp, _vp, _vp, C.POINTER(_vp), C.POINTER(_vp), C.c_int,
                                      C.c_int, _vp, C.c_int, _vp, _vp]),
+    "ckks_bsgs_lintrans_plan": (C.c_int, [_vp, _vp, _vp, C.POINTER(_vp), C.POINTER(_vp), C.c_int,
+                                          C.c_int, C.c_int, C.c_int, _vp, C.c_int, _vp, _vp]),
     "ckks_bench_intpipe": (C.c_int, [_vp, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_double),
                                      C.POINTER(C.c_double)]),
 }

@@ -577,3 +577,29 @@ def test_modraise(orc, L, K, alpha, l):
     x = orc.ntt_fwd(coef, mods[:l])
     got = host(ctx.modraise(dev(x)))
     assert_bits_equal(got, orc.modraise(x, mods[:L]), "modraise l=%d" % l)
+
+
+@pytest.mark.parametrize("plan", [(64, -8, 4, 4), (8, -7, 4, 4), (1, -7, 4, 4), (1, 0, 4, 3),
+                                  (3, 5, 2, 1)])
+def test_bsgs_plan_matches_oracle(orc, plan):
+    """Strided-window BSGS (the groups of a three-level factored transform at
+    n = 2048, the dense window, and a single rotated giant step) bit-exact
+    against the oracle on seeded residues, with the oracle's Galois keys."""
+    from oracle.boot import Chain, bsgs_plan_apply
+    stride, t0, bb, gg = plan
+    S = SLOTS
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 50)
+    chain = Chain(sch.mods, p.L, p.K, p.alpha)
+    amounts = {(stride * b) % S for b in range(1, bb)} | {(stride * (t0 + bb * g)) % S for g in range(gg)}
+    keys = {a: sch.keygen_galois(galois_for_rotation(a)) for a in amounts if a}
+    x = _res((2, 2, p.L, N), sch.q, 430)
+    pts = _res((gg, bb, p.L, N), sch.q, 431)
+    giants = [(stride * (t0 + bb * g)) % S for g in range(gg)]
+    y = host(ctx.bsgs_lintrans_plan(dev(x), dev(pts), [dev(keys[(stride * b) % S]) for b in range(1, bb)],
+                                    [dev(keys[G]) if G else None for G in giants], plan))
+    for i in range(2):
+        want, _ = bsgs_plan_apply(x[i], SCALE, [[pts[g, b] for b in range(bb)] for g in range(gg)],
+                                  plan, SCALE, keys, chain)
+        assert_bits_equal(y[i], want, "bsgs plan %s, ct %d" % (plan, i))
