@@ -144,10 +144,11 @@ int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine);
 
 /* Declares that the switching keys passed to this context's calls were made
  * for a chain of key_L >= L ciphertext primes q_0..q_{key_L-1} (and the same
- * special primes): layout [dnum_key][2][key_L + K][n] with dnum_key =
- * ceil(key_L / alpha).  The calls then read ciphertext prime t < L at key row
+ * special primes): layout [dnum_key][2][key_L + K][n] with dnum_key at least
+ * ceil(L / alpha).  The calls then read ciphertext prime t < L at key row
  * t, special prime k at row key_L + k, and only the first ceil(L / alpha)
- * digits.  A key reduced modulo a divisor of its modulus is a key for that
+ * digits, which must cover the same primes as this context's digits (a
+ * context below alpha primes has one digit, the start of the key's first).  A key reduced modulo a divisor of its modulus is a key for that
  * divisor, so one key set made at the top of a chain serves the context of
  * every level below it; the digits must be the same contiguous blocks of
  * alpha primes.  The default is key_L = L.  Takes effect for calls issued

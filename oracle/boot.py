@@ -274,6 +274,29 @@ def bootstrap_factored(ct_q0, delta, r, depth, keys, chain):
                              chain, first_factor_scalar=f)
 
 
+def refresh_with_levels(ct_q0, r, cts_levels, stc_levels, keys, chain):
+    """The refresh of bootstrap_factored with every transform level given as
+    (plan, pts), pts[g][b] the level's plaintexts as NTT residues over its
+    primes (zeros where a diagonal is absent): coeff_to_slot's at scale 2^60,
+    slot_to_coeff's at 2^50.  The integer function of the refresh for any
+    plaintexts, so a parity test can feed seeded residues.  Returns
+    (ct, scale)."""
+    ct = core.modraise(ct_q0, chain.mods[: chain.L])
+    scale = Fraction(chain.q(0))
+    for plan, pts in cts_levels:
+        ct, scale = bsgs_plan_apply(ct, scale, pts, plan, 2**60, keys["rot"], chain)
+    l = level(ct)
+    re, im = core.conj_extract(ct[None], chain.key_at(keys["conj"], l), chain.mods_at(l), l,
+                               chain.K, chain.alpha)
+    sre, s_out = sin_fold(re[0], scale, r, keys["relin"], chain)
+    sim, _ = sin_fold(im[0], scale, r, keys["relin"], chain)
+    ct = core.restore_merge(sre[None], sim[None], chain.mods[: level(sre)])[0]
+    scale = s_out
+    for plan, pts in stc_levels:
+        ct, scale = bsgs_plan_apply(ct, scale, pts, plan, 2**50, keys["rot"], chain)
+    return ct, scale
+
+
 def bootstrap(ct_q0, delta, r, keys, chain, bb, gg):
     """Refresh a ciphertext on q_0 holding slots z at scale `delta`
     (delta well below q_0).  `keys` holds 'baby', 'giant' (Galois keys for
@@ -302,4 +325,5 @@ def bootstrap(ct_q0, delta, r, keys, chain, bb, gg):
 __all__ = ["Chain", "drop", "mul_int", "add_const", "mul_const", "mul", "add", "sin_fold",
            "coeff_to_slot_plaintexts", "slot_to_coeff_plaintexts", "lintrans", "bootstrap",
            "rotation_amounts", "bsgs_plan_apply", "lintrans_planned", "lintrans_factored",
-           "factored_rotation_amounts", "bootstrap_factored", "TAYLOR_TERMS"]
+           "factored_rotation_amounts", "bootstrap_factored", "refresh_with_levels",
+           "TAYLOR_TERMS"]

@@ -90,14 +90,18 @@ class Context:
         """Shape of a switching key for this context: [dnum][2][L+K][n], or the
         longer chain's layout after set_key_chain."""
         kl = getattr(self, "key_L", self.L)
-        return ((kl + self.alpha - 1) // self.alpha, 2, kl + self.K, self.n)
+        dn = getattr(self, "key_dnum", None) or (kl + self.alpha - 1) // self.alpha
+        return (dn, 2, kl + self.K, self.n)
 
-    def set_key_chain(self, key_L):
+    def set_key_chain(self, key_L, key_dnum=None):
         """Keys passed from now on were made for a chain of key_L >= L
-        ciphertext primes (the same special primes and digits): one key set
-        made at the top level serves the context of every lower level."""
+        ciphertext primes with the same special primes, in key_dnum digits
+        (default ceil(key_L / alpha)) whose first blocks cover this context's
+        digits: one key set made at the top level serves the context of every
+        lower level."""
         check("ckks_ctx_set_key_chain", lib().ckks_ctx_set_key_chain(self._h, int(key_L)))
         self.key_L = int(key_L)
+        self.key_dnum = None if key_dnum is None else int(key_dnum)
 
     def set_conversion(self, engine):
         """Where ModUp/ModDown basis conversions run: "auto" (tensor cores from 8

@@ -603,3 +603,45 @@ def test_bsgs_plan_matches_oracle(orc, plan):
         want, _ = bsgs_plan_apply(x[i], SCALE, [[pts[g, b] for b in range(bb)] for g in range(gg)],
                                   plan, SCALE, keys, chain)
         assert_bits_equal(y[i], want, "bsgs plan %s, ct %d" % (plan, i))
+
+
+def test_refresh_matches_oracle(orc):
+    """The whole refresh at n = 2048 (16 primes, the plans of two-level
+    factored transforms, r = 4: 2 * 2 + 6 + 4 levels) through the per-level
+    contexts and one top-level key set, bit-exact against the oracle's
+    refresh with the same seeded plaintext residues, and the same tracked
+    scale.  (Decryption of the refresh is pinned on the CPU.)"""
+    from oracle import boot
+
+    from rns_ckks_polynomial_b200.refresh import Refresh
+    L, K, alpha, depth, r = 16, 4, 4, 2, 4
+    p = Params(L, K, alpha)
+    sch = Scheme(orc, p, SEED + 60)
+    chain = boot.Chain(sch.mods, L, K, alpha)
+    keys = {"rot": {a: sch.keygen_galois(galois_for_rotation(a))
+                    for a in boot.factored_rotation_amounts(N, depth)},
+            "conj": sch.keygen_galois(2 * N - 1), "relin": sch.keygen_relin()}
+    low = np.ascontiguousarray(_res((2, 1, N), sch.q[:1], 440))
+
+    def levels(factors, top, stream):
+        out = []
+        for i, F in enumerate(factors):
+            plan = orc.bsgs_plan(F, SLOTS)
+            _, _, bb, gg = plan
+            out.append((plan, _res((gg, bb, top - i, N), sch.q[:top - i], stream + i)))
+        return out
+
+    cts = levels(orc.factored_coeff_to_slot(N, depth), L, 450)
+    stc = levels(orc.factored_slot_to_coeff(N, depth), L - depth - 6 - r, 460)
+    want, s_want = boot.refresh_with_levels(low, r, [(pl, list(a)) for pl, a in cts],
+                                            [(pl, list(a)) for pl, a in stc], keys, chain)
+    dkeys = {"rot": {a: dev(k) for a, k in keys["rot"].items()}, "conj": dev(keys["conj"]),
+             "relin": dev(keys["relin"])}
+    rf = Refresh(sch.q, sch.mods[L:], alpha, dkeys)
+    try:
+        got, s_got = rf.refresh(dev(low[None]), r, [(pl, dev(a)) for pl, a in cts],
+                                [(pl, dev(a)) for pl, a in stc])
+        assert s_got == s_want
+        assert_bits_equal(host(got)[0], want, "refresh")
+    finally:
+        rf.close()
