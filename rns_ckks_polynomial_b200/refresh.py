@@ -25,13 +25,15 @@ are the textbook ones:
 
 Each level l runs on its own context (primes q_0..q_{l-1} and the chain's
 special primes), all sharing one key set made for the whole chain
-(ckks_ctx_set_key_chain)."""
+(ckks_ctx_set_key_chain) and one workspace, grown to the largest call's need
+(the calls run in order on one stream, so reuse is safe; per-context
+workspaces would cost tens of GB per level at 2100 primes)."""
 import math
 from fractions import Fraction
 
 import torch
 
-from .api import Context
+from .api import OP_BSGS, OP_CONJ_EXTRACT, OP_MODRAISE, OP_MRR, OP_RESCALE, Context
 
 TAYLOR_TERMS = 8
 
@@ -46,6 +48,14 @@ class Refresh:
         self.keys = keys
         self.device = device
         self._ctx = {}
+        self._buf = None
+
+    def _ws(self, ctx, op, batch, aux=0):
+        need = max(ctx.workspace_bytes(op, batch, aux), 16)
+        if self._buf is None or self._buf.numel() < need:
+            self._buf = None
+            self._buf = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda", self.device))
+        return self._buf
 
     def ctx(self, l):
         c = self._ctx.get(l)
@@ -60,6 +70,7 @@ class Refresh:
         for c in self._ctx.values():
             c.close()
         self._ctx.clear()
+        self._buf = None
 
     # ------------------------------------------------------------ constants
     def _kvec(self, value, l):
@@ -87,12 +98,15 @@ class Refresh:
     def mul_const(self, ct, scale, c, target):
         l = self.level(ct)
         k = round(Fraction(c) * target * self.q[l - 1] / scale)
-        return self.ctx(l).rescale(self.mul_int(ct, k)), Fraction(target)
+        cx = self.ctx(l)
+        prod = self.mul_int(ct, k)
+        return cx.rescale(prod, ws=self._ws(cx, OP_RESCALE, ct.shape[0], l)), Fraction(target)
 
     def mul(self, a, sa, b, sb):
         l = min(self.level(a), self.level(b))
         a, b = self.drop(a, l), self.drop(b, l)
-        out = self.ctx(l).mul_relin_rescale(a, b, self.keys["relin"])
+        cx = self.ctx(l)
+        out = cx.mul_relin_rescale(a, b, self.keys["relin"], ws=self._ws(cx, OP_MRR, a.shape[0]))
         return out, Fraction(sa) * Fraction(sb) / self.q[l - 1]
 
     def add(self, a, sa, b, sb):
@@ -142,7 +156,9 @@ class Refresh:
             baby = [rot[(stride * b) % S] for b in range(1, bb)]
             giant = [None if G == 0 else rot[G] for G in
                      ((stride * (t0 + bb * g)) % S for g in range(gg))]
-            ct = self.ctx(l).bsgs_lintrans_plan(ct, pts, baby, giant, plan)
+            cx = self.ctx(l)
+            ct = cx.bsgs_lintrans_plan(ct, pts, baby, giant, plan,
+                                       ws=self._ws(cx, OP_BSGS, ct.shape[0], bb * 1000 + gg))
             scale = Fraction(scale) * Fraction(pt_scale) / self.q[l - 1]
         return ct, scale
 
@@ -150,10 +166,12 @@ class Refresh:
         """A ciphertext [B][2][1][n] on q_0 -> (ciphertext, scale), the slots
         back at the message scale.  cts_levels / stc_levels as for lintrans,
         encoded at 2^60 and 2^50."""
-        ct = self.ctx(self.L).modraise(ct_q0)
+        top = self.ctx(self.L)
+        ct = top.modraise(ct_q0, ws=self._ws(top, OP_MODRAISE, ct_q0.shape[0], ct_q0.shape[2]))
         ct, scale = self.lintrans(ct, Fraction(self.q[0]), cts_levels, 2**60)
         l = self.level(ct)
-        re, im = self.ctx(l).conj_extract(ct, self.keys["conj"])
+        cx = self.ctx(l)
+        re, im = cx.conj_extract(ct, self.keys["conj"], ws=self._ws(cx, OP_CONJ_EXTRACT, ct.shape[0]))
         sre, s_out = self.sin_fold(re, scale, r)
         sim, _ = self.sin_fold(im, scale, r)
         merged = self.ctx(self.level(sre)).restore_merge(sre, sim)
