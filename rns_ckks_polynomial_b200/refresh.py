@@ -38,6 +38,53 @@ from .api import OP_BSGS, OP_CONJ_EXTRACT, OP_MODRAISE, OP_MRR, OP_RESCALE, Cont
 TAYLOR_TERMS = 8
 
 
+def stage_groups(n, depth):
+    """The log2(n/2) butterfly stages of the special FFT in `depth`
+    consecutive groups, the later groups at least as long as the earlier."""
+    m = (n // 2).bit_length() - 1
+    base, extra = divmod(m, depth)
+    out, s = [], 1
+    for g in range(depth):
+        size = base + (1 if g >= depth - extra else 0)
+        out.append(list(range(s, s + size)))
+        s += size
+    return out
+
+
+def group_plan(n, grp):
+    """BSGS plan (stride, t0, bb, gg) of a group of butterfly stages a..b:
+    its diagonals sit at stride t, stride = 2^(a-1), |t| <= 2^(b-a+1) - 1,
+    taken modulo M = (n/2) / stride (every residue once the window wraps)."""
+    S = n // 2
+    stride = 1 << (grp[0] - 1)
+    M = S // stride
+    k = len(grp)
+    if 2 ** (k + 1) - 1 >= M:
+        t0, T = -(M // 2), M
+    else:
+        t0, T = -(2 ** k - 1), 2 ** (k + 1) - 1
+    bb = 1 << max(0, round(math.log2(math.sqrt(T))))
+    return stride, t0, bb, -(-T // bb)
+
+
+def factored_plans(n, depth):
+    """Plans of the coeff_to_slot levels (inverse stages, last group first)
+    and of the slot_to_coeff levels (first group first)."""
+    groups = stage_groups(n, depth)
+    stc = [group_plan(n, g) for g in groups]
+    return stc[::-1], stc
+
+
+def plan_rotations(plans, n):
+    """The left-rotation amounts whose Galois keys the plans use."""
+    S = n // 2
+    out = set()
+    for stride, t0, bb, gg in plans:
+        out |= {(stride * b) % S for b in range(1, bb)}
+        out |= {(stride * (t0 + bb * g)) % S for g in range(gg)}
+    return sorted(a for a in out if a)
+
+
 class Refresh:
     def __init__(self, q, p, alpha, keys, device=0):
         """q: the chain's ciphertext primes q_0..q_{L-1}; p: its special primes;
