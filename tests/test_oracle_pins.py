@@ -378,6 +378,23 @@ def test_rotation_on_a_single_prime_chain(orc, K):
     assert np.max(np.abs(sch.decrypt_slots(out[1, 0], scale) - np.conj(z))) < 1e-6
 
 
+def test_rotation_at_the_boot_chain_size(orc):
+    """The boot chain itself: 2100 ciphertext primes, 60 special, 35 digits of
+    60 (about 20 s).  Rotation by 8 with config 5's Galois element 1505 = 5^8
+    decrypts to the rotated slots; the decryption reads q_0..q_2 only, where
+    m + e is far below Q/2."""
+    assert galois_for_rotation(8) == 1505
+    p = Params(2100, 60, 60)
+    sch = Scheme(orc, p, SEED + 15)
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 27).numpy()
+    ct = sch.encrypt_slots(z)
+    key = sch.keygen_galois(1505)
+    out = orc.rotate(ct[None], [key], np.array([1505], dtype=np.uint64), sch.mods, 2100, 60, 60)
+    assert out.shape == (1, 1, 2, 2100, N)
+    low = np.ascontiguousarray(out[0, 0][:, :3])
+    assert np.max(np.abs(sch.decrypt_slots(low) - rot_left(z, 8))) < 1e-8
+
+
 def test_hoisted_rotations_small_digits(orc):
     """Ragged digits (L = 5, alpha = 2) and several keys on one ModUp."""
     p = Params(5, 2, 2)
@@ -478,3 +495,96 @@ def test_bsgs_banded_matvec(orc):
     y = orc.bsgs(ct[None], diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
     sc = sch.rescaled_scale(SCALE * SCALE, p.L)
     assert np.max(np.abs(sch.decrypt_slots(y[0], sc) - M @ x)) < 1e-8
+
+
+def test_bsgs_at_the_layer_chain_size(orc):
+    """Config 4's shape: 112 + 8 primes, bb = gg = 32, 31 baby and 31 giant
+    keys (about 30 s).  M has nonzero diagonals at offsets spread over the
+    32 x 32 (giant, baby) grid, including both ends and both sides of a giant
+    boundary; absent diagonals are zero plaintexts.  Decrypts (through
+    q_0..q_2) to M x."""
+    p = Params(112, 8, 8)
+    bb = gg = 32
+    sch = Scheme(orc, p, SEED + 16)
+    offs = [0, 1, 31, 32, 33, 100, 511, 1000, 1023]
+    vals = synth.uniform_real((len(offs), SLOTS), -1 / 8, 1 / 8, SEED, 60).numpy()
+    idx = np.arange(SLOTS)
+    M = np.zeros((SLOTS, SLOTS))
+    diags = np.zeros((gg, bb, p.L, N), dtype=np.uint64)
+    for v, k in zip(vals, offs):
+        M[idx, (idx + k) % SLOTS] = v
+        g, b = divmod(k, bb)
+        diags[g, b] = orc.encode_ntt(np.roll(v, bb * g), sch.q, SCALE, N)
+    baby = [sch.keygen_galois(galois_for_rotation(b)) for b in range(1, bb)]
+    giant = [sch.keygen_galois(galois_for_rotation(bb * g)) for g in range(1, gg)]
+    x = synth.uniform_real((SLOTS,), -1, 1, SEED, 61).numpy()
+    y = orc.bsgs(sch.encrypt_slots(x)[None], diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    low = np.ascontiguousarray(y[0][:, :3])
+    assert np.max(np.abs(sch.decrypt_slots(low, sc) - M @ x)) < 1e-8
+
+
+def test_every_input_is_read(orc):
+    """Flipping one residue of any input changes the output, for every
+    oracle operation and every one of its inputs (an operation that ignored
+    an input, or part of it, would pass tests whose inputs happen not to
+    matter)."""
+    p = Params(6, 2, 2)
+    L, K, alpha = p.L, p.K, p.alpha
+    mods = orc.gen_primes(N, L + K)
+    q = mods[:L]
+
+    def flip(a, at, m):
+        b = a.copy()
+        b[at] = (int(b[at]) + 1) % int(m)
+        return b
+
+    def check(fn, args, idx, at, m):
+        base = fn(*args)
+        args2 = list(args)
+        args2[idx] = flip(args[idx], at, m)
+        got = fn(*args2)
+        base = base if isinstance(base, tuple) else (base,)
+        got = got if isinstance(got, tuple) else (got,)
+        assert any(not np.array_equal(x, y) for x, y in zip(base, got)), (fn.__name__, idx, at)
+
+    a, b = _rand_res((2, L, N), q, 70), _rand_res((2, L, N), q, 71)
+    key, key2 = _rand_res((p.dnum, 2, L + K, N), mods, 72), _rand_res((p.dnum, 2, L + K, N), mods, 73)
+    ct = _rand_res((1, 2, L, N), q, 74)
+    gal = np.array([5], dtype=np.uint64)
+    check(lambda x: orc.ntt_fwd(x, q), [a], 0, (1, 5, 7), q[5])
+    check(lambda x: orc.ntt_inv(x, q), [a], 0, (0, 0, N - 1), q[0])
+    for i in range(2):
+        check(lambda x, y: orc.pointwise("mul", x, y, q), [a, b], i, (1, 3, 9), q[3])
+    check(lambda x: orc.automorph_ntt(x, 5), [a], 0, (0, 2, 100), q[2])
+    check(lambda x: orc.modup(x, mods, L, K, alpha), [a], 0, (1, 5, 11), q[5])
+    dig = orc.modup(a, mods, L, K, alpha)
+    check(lambda d, k: orc.key_inner(d, k, 5, mods, L, K, alpha), [dig, key], 0, (0, 2, L + 1, 3),
+          mods[L + 1])
+    check(lambda d, k: orc.key_inner(d, k, 5, mods, L, K, alpha), [dig, key], 1, (1, 1, 4, 8), mods[4])
+    acc = orc.key_inner(dig, key, 1, mods, L, K, alpha)
+    check(lambda x: orc.moddown(x, mods, L, K), [acc], 0, (0, 1, L, 17), mods[L])
+    check(lambda x: orc.moddown(x, mods, L, K), [acc], 0, (1, 0, 2, 17), mods[2])
+    for idx, at, m in ((0, (0, 4, 5), q[4]), (1, (2, 0, L + 1, 6), mods[L + 1])):
+        check(lambda d, k: orc.keyswitch(d, k, mods, L, K, alpha), [a, key], idx, at, m)
+    for fn in (orc.rotate, orc.rotate_unhoisted):
+        for at in ((0, 0, 1, 4), (0, 1, 3, 4)):
+            check(lambda c: fn(c, [key], gal, mods, L, K, alpha), [ct], 0, at, q[at[2]])
+        check(lambda k: fn(ct, [k], gal, mods, L, K, alpha), [key], 0, (1, 0, L, 5), mods[L])
+    check(lambda c: orc.rescale(c, q), [ct], 0, (0, 1, L - 1, 2), q[L - 1])
+    check(lambda c: orc.rescale(c, q), [ct], 0, (0, 0, 0, 2), q[0])
+    ct2 = _rand_res((1, 2, L, N), q, 75)
+    for idx, at, m in ((0, (0, 1, 1, 1), q[1]), (1, (0, 0, 5, 1), q[5]),
+                       (2, (0, 1, L, 9), mods[L])):
+        check(lambda x, y, k: orc.mul_relin_rescale(x, y, k, mods, L, K, alpha), [ct, ct2, key], idx,
+              at, m)
+    diags = _rand_res((2, 2, L, N), q, 76)
+    bs = lambda x, d, kb, kg: orc.bsgs(x, d, [kb], [kg], 2, 2, mods, L, K, alpha)
+    for idx, at, m in ((0, (0, 1, 2, 3), q[2]), (1, (1, 1, 0, 3), q[0]), (2, (0, 0, 1, 3), q[1]),
+                       (3, (1, 1, L, 3), mods[L])):
+        check(bs, [ct, diags, key, key2], idx, at, m)
+    check(lambda x: orc.modraise(x, q), [a[:, :3].copy()], 0, (1, 2, 7), q[2])
+    check(lambda c, k: orc.conj_extract(c, k, mods, L, K, alpha), [ct, key], 0, (0, 1, 0, 0), q[0])
+    check(lambda c, k: orc.conj_extract(c, k, mods, L, K, alpha), [ct, key], 1, (2, 1, 3, 0), mods[3])
+    for idx in range(2):
+        check(lambda r, i: orc.restore_merge(r, i, q), [ct, ct2], idx, (0, idx, 4, 4), q[4])
