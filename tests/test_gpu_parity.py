@@ -645,3 +645,28 @@ def test_refresh_matches_oracle(orc):
         assert_bits_equal(host(got)[0], want, "refresh")
     finally:
         rf.close()
+
+
+def test_extreme_residues(orc):
+    """Inputs at the ends of [0, q): all zeros, all q - 1, and q - 1
+    alternating with 0, through the NTT both ways, a key switch and a rescale
+    (the lazy butterflies and 128-bit sums see their largest operands)."""
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    q = mods[:p.L]
+    top = np.broadcast_to((q - 1)[:, None], (p.L, N))
+    alt = np.where(np.arange(N) % 2 == 0, top, 0).astype(np.uint64)
+    cases = [np.zeros((p.L, N), np.uint64), np.ascontiguousarray(top, dtype=np.uint64), alt]
+    x = np.stack(cases)
+    y = dev(x)
+    ctx.ntt_fwd(y)
+    assert_bits_equal(host(y), orc.ntt_fwd(x, q), "ntt_fwd extremes")
+    ctx.ntt_inv(y)
+    assert_bits_equal(host(y), x, "ntt round trip extremes")
+    kt = np.broadcast_to((mods - 1)[None, None, :, None], (p.dnum, 2, p.L + p.K, N))
+    key = np.ascontiguousarray(kt, dtype=np.uint64)
+    assert_bits_equal(host(ctx.keyswitch(dev(x), dev(key))), orc.keyswitch(x, key, mods, p.L, p.K, p.alpha),
+                      "keyswitch extremes")
+    ct = np.stack([np.stack([c, c]) for c in cases])
+    assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, q), "rescale extremes")
