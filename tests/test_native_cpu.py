@@ -45,6 +45,8 @@ def test_library_path_is_in_tree():
 
 def test_product_primes_match_oracle(orc):
     assert primes(300) == [int(x) for x in orc.gen_primes(N, 300)]
+    # the whole boot chain: 2100 ciphertext and 60 special primes
+    assert primes(2160) == [int(x) for x in orc.gen_primes(N, 2160)]
 
 
 def test_primes_argument_checks():
@@ -96,3 +98,18 @@ def test_calls_reject_null_context():
     assert lib.ckks_ctx_set_conversion(None, 1) == EINVAL
     assert lib.ckks_ctx_set_key_chain(None, 5) == EINVAL
     assert lib.ckks_selftest_wait_expiry(None) == EINVAL
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the compiled library every call raises; nothing falls back to
+    a CPU path."""
+    from rns_ckks_polynomial_b200 import Context
+    ps = primes(4)
+    monkeypatch.setattr(native, "_LIB", None)
+    monkeypatch.setattr(native._build, "LIB", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        native.lib()
+    with pytest.raises(RuntimeError, match="not built"):
+        Context(ps[:3], ps[3:], 1)
+    with pytest.raises(RuntimeError, match="not built"):
+        primes(4)
