@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-ks", action="store_true", help="skip the key-switch measurements")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--refresh-only", action="store_true",
+                    help="time only the bootstrapping refresh at 2100 + 60 primes")
     ap.add_argument("--ks-only", action="store_true",
                     help="run only the key-switch measurements (for profiling)")
     ap.add_argument("--ks-batch", type=int, default=8,
@@ -707,6 +709,56 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_refresh(dev, B=8, L=2100, K=60, alpha=60, depth=3, r=9, reps=2):
+    """The bootstrapping refresh of B ciphertexts on the boot chain (2100 + 60
+    primes): modraise from q_0, `depth`-level factored coeff_to_slot and
+    slot_to_coeff, conj_extract, two sin_folds of 6 + r levels, restore_merge.
+    Keys and plaintext diagonals are seeded uniform residues: the kernels'
+    time does not depend on the values (the parity test runs the same schedule
+    on the oracle's keys)."""
+    import torch
+
+    from rns_ckks_polynomial_b200 import primes, synth
+    from rns_ckks_polynomial_b200.refresh import Refresh, factored_plans, plan_rotations
+    seed = synth.config_seed(5) + 77
+    mods = primes(L + K)
+    q, p = mods[:L], mods[L:]
+    dnum = (L + alpha - 1) // alpha
+    cts_plans, stc_plans = factored_plans(N, depth)
+    amounts = plan_rotations(cts_plans + stc_plans, N)
+
+    def key(stream):
+        return synth.uniform_residues((dnum, 2, L + K, N), mods, seed, stream, device=dev)
+
+    keys = {"rot": {a: key(100 + i) for i, a in enumerate(amounts)}, "conj": key(90), "relin": key(91)}
+
+    def levels(plans, top, stream):
+        return [(pl, synth.uniform_residues((pl[3], pl[2], top - i, N), q[:top - i], seed, stream + i,
+                                            device=dev)) for i, pl in enumerate(plans)]
+
+    cts = levels(cts_plans, L, 200)
+    stc = levels(stc_plans, L - depth - 6 - r, 300)
+    ct = synth.uniform_residues((B, 2, 1, N), q[:1], seed, 1, device=dev)
+    rf = Refresh(q, p, alpha, keys, device=dev.index)
+    stream = torch.cuda.current_stream(dev)
+    try:
+        ms = _time_call(lambda: rf.refresh(ct, r, cts, stc), reps, stream)
+    finally:
+        rf.close()
+    S = N // 2
+    per_ct = 1 + 2 * (7 + r)
+    for stride, t0, bb, gg in cts_plans + stc_plans:
+        rotated = sum(1 for g in range(gg) if (stride * (t0 + bb * g)) % S)
+        per_ct += (bb - 1) + rotated
+    return {"workload": "refresh of %d ciphertexts, %d + %d primes, alpha %d, factored transforms of "
+                        "depth %d, sin_fold r = %d (%d levels)" % (B, L, K, alpha, depth, r,
+                                                                  2 * depth + 6 + r),
+            "ms_per_call": ms, "ciphertext_refreshes_per_s": B / (ms * 1e-3),
+            "key_switches_per_ciphertext": per_ct, "keys": len(amounts) + 2,
+            "pages_cpu_s_for_8_ciphertexts": 4393.5,
+            "data": "seeded uniform residues for keys, plaintexts and the input ciphertexts"}
+
+
 def run_ks_only(args):
     import torch
     dev = torch.device("cuda", 0)
@@ -720,6 +772,10 @@ def run_ks_only(args):
 
 def main():
     args = parse()
+    if args.refresh_only:
+        import torch
+        print(json.dumps({"refresh": run_refresh(torch.device("cuda", 0))}), flush=True)
+        return
     if args.ks_only:
         run_ks_only(args)
         return

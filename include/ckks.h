@@ -72,7 +72,9 @@ enum ckks_op {
     CKKS_OP_RESCALE = 5,
     CKKS_OP_MUL_RELIN_RESCALE = 6,
     CKKS_OP_BSGS = 7,
-    CKKS_OP_ROTATE_UNHOISTED = 8
+    CKKS_OP_ROTATE_UNHOISTED = 8,
+    CKKS_OP_MODRAISE = 9,       /* aux: l, the input's prime count */
+    CKKS_OP_CONJ_EXTRACT = 10
 };
 
 /* Pointwise operation codes for ckks_pointwise. */
@@ -139,6 +141,21 @@ int ckks_selftest_wait_expiry(const ckks_ctx *ctx);
  * unknown engine. */
 enum { CKKS_CONV_AUTO = 0, CKKS_CONV_INTEGER = 1, CKKS_CONV_TENSOR = 2 };
 int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine);
+
+/* Declares that the switching keys passed to this context's calls were made
+ * for a chain of key_L >= L ciphertext primes q_0..q_{key_L-1} (and the same
+ * special primes): layout [dnum_key][2][key_L + K][n] with dnum_key at least
+ * ceil(L / alpha).  The calls then read ciphertext prime t < L at key row
+ * t, special prime k at row key_L + k, and only the first ceil(L / alpha)
+ * digits, which must cover the same primes as this context's digits (a
+ * context below alpha primes has one digit, the start of the key's first).  A key reduced modulo a divisor of its modulus is a key for that
+ * divisor, so one key set made at the top of a chain serves the context of
+ * every level below it; the digits must be the same contiguous blocks of
+ * alpha primes.  The default is key_L = L.  Takes effect for calls issued
+ * after it returns; do not change it while another host thread issues calls
+ * on the same context.  CKKS_EINVAL for a null context or key_L outside
+ * [L, 4096]. */
+int ckks_ctx_set_key_chain(ckks_ctx *ctx, int key_L);
 
 /* Context parameters: writes L, K, alpha, dnum, n (any pointer may be NULL). */
 int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n);
@@ -299,6 +316,73 @@ int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *d
                        const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
                        int bb, int gg, uint64_t *y, int batch, void *ws,
                        ckks_stream_t stream);
+
+/* The same transform for a matrix whose nonzero diagonals sit at the offsets
+ * stride (t0 + bb g + b), g < gg, b < bb (a group of butterfly stages of a
+ * factored coeff_to_slot / slot_to_coeff):
+ *   y = Rescale( sum_g Rot_{G_g}( sum_b diags[g][b] * Rot_{stride b}(x) ) ),
+ *   G_g = stride (t0 + bb g) mod n/2,
+ * with diags[g][b] = Encode(rot_{-G_g}(diag_{G_g + stride b})) (zeros where
+ * the diagonal is absent).  baby_keys[b-1] rotates by stride b (Galois
+ * 5^{stride b}); giant_keys has gg entries, giant_keys[g] rotating by G_g
+ * (it may be NULL where G_g = 0, which is not rotated).  stride = 1, t0 = 0
+ * is ckks_bsgs_lintrans.  Limits as ckks_bsgs_lintrans, plus stride >= 1,
+ * stride (bb - 1) < n/2, |t0| <= n/2.
+ * ws: ckks_workspace_bytes(CKKS_OP_BSGS, batch, bb * 1000 + gg). */
+int ckks_bsgs_lintrans_plan(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                            const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
+                            int stride, int t0, int bb, int gg, uint64_t *y, int batch, void *ws,
+                            ckks_stream_t stream);
+
+/* ---- building blocks of the bootstrapping refresh (Kestrel engine write-up,
+ * the boot profile in section 5.3; the forms are the textbook ones, as the
+ * oracle reads them). */
+
+/* out[p][l][k] = a[p][l][k] op k[l] over [batch][limbs][n]; k is a DEVICE
+ * array of `limbs` residues, k[l] in [0, q) of prime limb_begin + l (a
+ * constant polynomial's NTT is the constant).  op: CKKS_PW_MUL/ADD/SUB.
+ * out may alias a.  Limit: batch <= 65535. */
+int ckks_pointwise_scalar(const ckks_ctx *ctx, int op, const uint64_t *a, const uint64_t *k,
+                          uint64_t *out, int batch, int limb_begin, int limbs,
+                          ckks_stream_t stream);
+
+/* In place on ct[batch][2][L][n]: component 0 of every ciphertext gets k[l]
+ * added at limb l (k: DEVICE array of L residues), i.e. every slot gets the
+ * constant whose scaled value k encodes. */
+int ckks_add_const_c0(const ckks_ctx *ctx, uint64_t *ct, const uint64_t *k, int batch,
+                      ckks_stream_t stream);
+
+/* out = X^{n/2} in over [batch][limbs][n] (NTT domain, limb l with prime
+ * limb_begin + l): every slot times i.  In the NTT domain this is the
+ * pointwise product by psi^{n/2} on the first n/2 evaluation slots and by
+ * -psi^{n/2} on the others.  out may alias in. */
+int ckks_mul_i(const ckks_ctx *ctx, const uint64_t *in, uint64_t *out, int batch, int limb_begin,
+               int limbs, ckks_stream_t stream);
+
+/* conj_extract: ct[batch][2][L][n] with slots w -> re, im [batch][2][L][n]
+ * with slots 2 Re w and 2 Im w (same scale): re = ct + conj(ct),
+ * im = X^{n/2} (conj(ct) - ct), conj being the hoisted rotation by the
+ * Galois element 2n - 1 with conj_key ([dnum][2][L+K][n], or the layout
+ * ckks_ctx_set_key_chain declares).  Limit: batch <= 32767.
+ * ws: ckks_workspace_bytes(CKKS_OP_CONJ_EXTRACT, batch, 0). */
+int ckks_conj_extract(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *conj_key, uint64_t *re,
+                      uint64_t *im, int batch, void *ws, ckks_stream_t stream);
+
+/* restore_merge: re, im [batch][2][L][n] with slots a, b -> out = re +
+ * X^{n/2} im, slots a + i b. */
+int ckks_restore_merge(const ckks_ctx *ctx, const uint64_t *re, const uint64_t *im, uint64_t *out,
+                       int batch, ckks_stream_t stream);
+
+/* modraise: in[batch][2][l][n] over q_0..q_{l-1} (NTT domain) ->
+ * out[batch][2][L][n] over the context's L primes.  Each coefficient is read
+ * as its centred integer X in (-Q/2, Q/2], Q = q_0 ... q_{l-1}, and reduced
+ * modulo every q_t (exact: Garner's mixed-radix digits, then a conversion
+ * whose sign row subtracts Q where X > (Q-1)/2).  Limbs below l are copied.
+ * Limits: 1 <= l <= min(L, 63), batch <= 32767.  Tables for each l are built
+ * on first use and kept by the context.
+ * ws: ckks_workspace_bytes(CKKS_OP_MODRAISE, batch, l). */
+int ckks_modraise(const ckks_ctx *ctx, const uint64_t *in, int l, uint64_t *out, int batch, void *ws,
+                  ckks_stream_t stream);
 
 /* ---------------------------------------------------------------- measurement */
 

@@ -175,18 +175,17 @@ def rotation_amounts(plan, S):
     return sorted(a for a in amounts if a)
 
 
-def lintrans_planned(ct, scale, Dg, plan, pt_scale, keys, chain):
-    """y = sum_g Rot_{G_g}( sum_b pt_{g,b} * Rot_{stride b}(x) ), then one
-    rescale, for a matrix in diagonal form with plan (stride, t0, bb, gg)
-    (encoding.bsgs_plan).  keys: {r: Galois key of 5^r} over the full chain.
-    The baby rotations share one ModUp (hoisted); a giant step with G_g = 0
-    is not rotated; absent diagonals are skipped."""
-    from .encoding import plan_plaintexts
+def bsgs_plan_apply(ct, scale, pts, plan, pt_scale, keys, chain):
+    """The integer part of lintrans_planned: pts[g][b] NTT residues over the
+    ciphertext's primes (zeros where a diagonal is absent),
+    y = Rescale( sum_g Rot_{G_g}( sum_b pts[g][b] * Rot_{stride b}(x) ) ),
+    G_g = stride (t0 + bb g) mod n/2.  keys: {r: Galois key of 5^r} over the
+    full chain.  The baby rotations share one ModUp (hoisted); a giant step
+    with G_g = 0 is not rotated."""
     n = ct.shape[-1]
     S = n // 2
     l = level(ct)
-    stride, _, bb, gg = plan
-    pts, giants = plan_plaintexts(Dg, plan, S, chain.mods[:l], pt_scale, n)
+    stride, t0, bb, gg = plan
     mods_l = chain.mods_at(l)
     qs = chain.mods[:l]
     babies = [ct]
@@ -207,7 +206,7 @@ def lintrans_planned(ct, scale, Dg, plan, pt_scale, keys, chain):
             inner = prod if inner is None else core.pointwise("add", inner, prod, qs)
         if inner is None:
             continue
-        G = giants[g]
+        G = (stride * (t0 + bb * g)) % S
         if G:
             gal = np.array([pow(5, G, 2 * n)], dtype=np.uint64)
             inner = core.rotate(inner[None], [chain.key_at(keys[G], l)], gal, mods_l, l, chain.K,
@@ -215,6 +214,18 @@ def lintrans_planned(ct, scale, Dg, plan, pt_scale, keys, chain):
         acc = inner if acc is None else core.pointwise("add", acc, inner, qs)
     out = core.rescale(acc[None], qs)[0]
     return out, Fraction(scale) * Fraction(pt_scale) / chain.q(l - 1)
+
+
+def lintrans_planned(ct, scale, Dg, plan, pt_scale, keys, chain):
+    """y = sum_g Rot_{G_g}( sum_b pt_{g,b} * Rot_{stride b}(x) ), then one
+    rescale, for a matrix in diagonal form with plan (stride, t0, bb, gg)
+    (encoding.bsgs_plan); the plaintexts come from encoding.plan_plaintexts
+    and absent diagonals are skipped."""
+    from .encoding import plan_plaintexts
+    n = ct.shape[-1]
+    l = level(ct)
+    pts, _ = plan_plaintexts(Dg, plan, n // 2, chain.mods[:l], pt_scale, n)
+    return bsgs_plan_apply(ct, scale, pts, plan, pt_scale, keys, chain)
 
 
 def lintrans_factored(ct, scale, factors, pt_scale, keys, chain, first_factor_scalar=1.0):
@@ -263,6 +274,29 @@ def bootstrap_factored(ct_q0, delta, r, depth, keys, chain):
                              chain, first_factor_scalar=f)
 
 
+def refresh_with_levels(ct_q0, r, cts_levels, stc_levels, keys, chain):
+    """The refresh of bootstrap_factored with every transform level given as
+    (plan, pts), pts[g][b] the level's plaintexts as NTT residues over its
+    primes (zeros where a diagonal is absent): coeff_to_slot's at scale 2^60,
+    slot_to_coeff's at 2^50.  The integer function of the refresh for any
+    plaintexts, so a parity test can feed seeded residues.  Returns
+    (ct, scale)."""
+    ct = core.modraise(ct_q0, chain.mods[: chain.L])
+    scale = Fraction(chain.q(0))
+    for plan, pts in cts_levels:
+        ct, scale = bsgs_plan_apply(ct, scale, pts, plan, 2**60, keys["rot"], chain)
+    l = level(ct)
+    re, im = core.conj_extract(ct[None], chain.key_at(keys["conj"], l), chain.mods_at(l), l,
+                               chain.K, chain.alpha)
+    sre, s_out = sin_fold(re[0], scale, r, keys["relin"], chain)
+    sim, _ = sin_fold(im[0], scale, r, keys["relin"], chain)
+    ct = core.restore_merge(sre[None], sim[None], chain.mods[: level(sre)])[0]
+    scale = s_out
+    for plan, pts in stc_levels:
+        ct, scale = bsgs_plan_apply(ct, scale, pts, plan, 2**50, keys["rot"], chain)
+    return ct, scale
+
+
 def bootstrap(ct_q0, delta, r, keys, chain, bb, gg):
     """Refresh a ciphertext on q_0 holding slots z at scale `delta`
     (delta well below q_0).  `keys` holds 'baby', 'giant' (Galois keys for
@@ -290,5 +324,6 @@ def bootstrap(ct_q0, delta, r, keys, chain, bb, gg):
 
 __all__ = ["Chain", "drop", "mul_int", "add_const", "mul_const", "mul", "add", "sin_fold",
            "coeff_to_slot_plaintexts", "slot_to_coeff_plaintexts", "lintrans", "bootstrap",
-           "rotation_amounts", "lintrans_planned", "lintrans_factored",
-           "factored_rotation_amounts", "bootstrap_factored", "TAYLOR_TERMS"]
+           "rotation_amounts", "bsgs_plan_apply", "lintrans_planned", "lintrans_factored",
+           "factored_rotation_amounts", "bootstrap_factored", "refresh_with_levels",
+           "TAYLOR_TERMS"]

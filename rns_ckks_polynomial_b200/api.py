@@ -17,6 +17,7 @@ N = 2048
 PW = {"mul": 0, "add": 1, "sub": 2}
 OP_MODUP, OP_MODDOWN, OP_KEYSWITCH, OP_ROTATE, OP_RESCALE, OP_MRR, OP_BSGS = 1, 2, 3, 4, 5, 6, 7
 OP_ROTATE_UNHOISTED = 8
+OP_MODRAISE, OP_CONJ_EXTRACT = 9, 10
 
 
 def primes(count, n=N):
@@ -83,6 +84,24 @@ class Context:
         check("ckks_selftest_wait_expiry", lib().ckks_selftest_wait_expiry(self._h))
 
     CONVERSION = {"auto": 0, "integer": 1, "tensor": 2}
+
+    @property
+    def _kshape(self):
+        """Shape of a switching key for this context: [dnum][2][L+K][n], or the
+        longer chain's layout after set_key_chain."""
+        kl = getattr(self, "key_L", self.L)
+        dn = getattr(self, "key_dnum", None) or (kl + self.alpha - 1) // self.alpha
+        return (dn, 2, kl + self.K, self.n)
+
+    def set_key_chain(self, key_L, key_dnum=None):
+        """Keys passed from now on were made for a chain of key_L >= L
+        ciphertext primes with the same special primes, in key_dnum digits
+        (default ceil(key_L / alpha)) whose first blocks cover this context's
+        digits: one key set made at the top level serves the context of every
+        lower level."""
+        check("ckks_ctx_set_key_chain", lib().ckks_ctx_set_key_chain(self._h, int(key_L)))
+        self.key_L = int(key_L)
+        self.key_dnum = None if key_dnum is None else int(key_dnum)
 
     def set_conversion(self, engine):
         """Where ModUp/ModDown basis conversions run: "auto" (tensor cores from 8
@@ -169,7 +188,7 @@ class Context:
         B = digits.shape[0]
         LK = self.L + self.K
         _ptr(digits, "digits", (B, self.dnum, LK, self.n))
-        _ptr(key, "key", (self.dnum, 2, LK, self.n))
+        _ptr(key, "key", self._kshape)
         out = self._empty(B, 2, LK, self.n) if out is None else out
         check("ckks_key_inner", lib().ckks_key_inner(self._h, _ptr(digits, "digits"), _ptr(key, "key"),
                                                      int(galois), _ptr(out, "acc"), B,
@@ -188,7 +207,7 @@ class Context:
     def keyswitch(self, d, key, out=None, ws=None):
         B = d.shape[0]
         _ptr(d, "d", (B, self.L, self.n))
-        _ptr(key, "key", (self.dnum, 2, self.L + self.K, self.n))
+        _ptr(key, "key", self._kshape)
         out = self._empty(B, 2, self.L, self.n) if out is None else out
         ws, wp = self._ws(ws, OP_KEYSWITCH, B)
         check("ckks_keyswitch", lib().ckks_keyswitch(self._h, _ptr(d, "d"), _ptr(key, "key"),
@@ -200,7 +219,7 @@ class Context:
         B = ct.shape[0]
         nk = len(keys)
         _ptr(ct, "ct", (B, 2, self.L, self.n))
-        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", (self.dnum, 2, self.L + self.K, self.n)).value
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", self._kshape).value
                                         for k in keys])
         gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
         out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
@@ -214,7 +233,7 @@ class Context:
         B = ct.shape[0]
         nk = len(keys)
         _ptr(ct, "ct", (B, 2, self.L, self.n))
-        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", (self.dnum, 2, self.L + self.K, self.n)).value
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", self._kshape).value
                                         for k in keys])
         gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
         out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
@@ -237,7 +256,7 @@ class Context:
         B = a.shape[0]
         _ptr(a, "a", (B, 2, self.L, self.n))
         _ptr(b, "b", (B, 2, self.L, self.n))
-        _ptr(rlk, "rlk", (self.dnum, 2, self.L + self.K, self.n))
+        _ptr(rlk, "rlk", self._kshape)
         out = self._empty(B, 2, self.L - 1, self.n) if out is None else out
         ws, wp = self._ws(ws, OP_MRR, B)
         check("ckks_mul_relin_rescale",
@@ -250,7 +269,7 @@ class Context:
         B = x.shape[0]
         _ptr(x, "x", (B, 2, self.L, self.n))
         _ptr(diags, "diags", (gg, bb, self.L, self.n))
-        kshape = (self.dnum, 2, self.L + self.K, self.n)
+        kshape = self._kshape
         if len(baby_keys) != bb - 1 or len(giant_keys) != gg - 1:
             raise ValueError("need bb-1 baby keys and gg-1 giant keys")
         bk = (C.c_void_p * max(1, bb - 1))(*[_ptr(k, "baby key", kshape).value for k in baby_keys])
@@ -260,6 +279,90 @@ class Context:
         check("ckks_bsgs_lintrans",
               lib().ckks_bsgs_lintrans(self._h, _ptr(x, "x"), _ptr(diags, "diags"), bk, gk, bb, gg,
                                        _ptr(out, "y"), B, wp, _stream(x)))
+        return out
+
+    def bsgs_lintrans_plan(self, x, diags, baby_keys, giant_keys, plan, out=None, ws=None):
+        """The BSGS transform over a strided window of diagonals, plan =
+        (stride, t0, bb, gg): baby_keys rotate by stride b (b = 1..bb-1),
+        giant_keys[g] by stride (t0 + bb g) mod n/2 (None where that is 0)."""
+        stride, t0, bb, gg = (int(v) for v in plan)
+        B = x.shape[0]
+        _ptr(x, "x", (B, 2, self.L, self.n))
+        _ptr(diags, "diags", (gg, bb, self.L, self.n))
+        kshape = self._kshape
+        if len(baby_keys) != bb - 1 or len(giant_keys) != gg:
+            raise ValueError("need bb-1 baby keys and gg giant keys")
+        bk = (C.c_void_p * max(1, bb - 1))(*[_ptr(k, "baby key", kshape).value for k in baby_keys])
+        gk = (C.c_void_p * gg)(*[None if k is None else _ptr(k, "giant key", kshape).value
+                                 for k in giant_keys])
+        out = self._empty(B, 2, self.L - 1, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_BSGS, B, bb * 1000 + gg)
+        check("ckks_bsgs_lintrans_plan",
+              lib().ckks_bsgs_lintrans_plan(self._h, _ptr(x, "x"), _ptr(diags, "diags"), bk, gk, stride,
+                                            t0, bb, gg, _ptr(out, "y"), B, wp, _stream(x)))
+        return out
+
+    # ------------------------------------------------------------ refresh building blocks
+    def pointwise_scalar(self, op, a, k, out=None, limb_begin=0):
+        """out = a op k[limb] over a[..., limbs, n]; k: device int64 tensor of
+        `limbs` residues."""
+        out = torch.empty_like(a) if out is None else out
+        limbs = a.shape[-2]
+        batch = a.numel() // (limbs * self.n) if a.numel() else 0
+        _ptr(k, "k", (limbs,))
+        check("ckks_pointwise_scalar",
+              lib().ckks_pointwise_scalar(self._h, PW[op], _ptr(a, "a"), _ptr(k, "k"), _ptr(out, "out"),
+                                          batch, limb_begin, limbs, _stream(a)))
+        return out
+
+    def add_const_c0(self, ct, k):
+        """In place: component 0 of every ciphertext of ct[B][2][L][n] plus k[limb]."""
+        B = ct.shape[0]
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        _ptr(k, "k", (self.L,))
+        check("ckks_add_const_c0", lib().ckks_add_const_c0(self._h, _ptr(ct, "ct"), _ptr(k, "k"), B,
+                                                           _stream(ct)))
+        return ct
+
+    def mul_i(self, x, out=None, limb_begin=0):
+        """X^{n/2} x (every slot times i) over x[..., limbs, n], NTT domain."""
+        out = torch.empty_like(x) if out is None else out
+        limbs = x.shape[-2]
+        batch = x.numel() // (limbs * self.n) if x.numel() else 0
+        check("ckks_mul_i", lib().ckks_mul_i(self._h, _ptr(x, "in"), _ptr(out, "out"), batch, limb_begin,
+                                             limbs, _stream(x)))
+        return out
+
+    def conj_extract(self, ct, conj_key, ws=None):
+        """ct[B][2][L][n] -> (re, im) with slots 2 Re w and 2 Im w."""
+        B = ct.shape[0]
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        _ptr(conj_key, "conj_key", self._kshape)
+        re, im = self._empty(B, 2, self.L, self.n), self._empty(B, 2, self.L, self.n)
+        ws, wp = self._ws(ws, OP_CONJ_EXTRACT, B)
+        check("ckks_conj_extract",
+              lib().ckks_conj_extract(self._h, _ptr(ct, "ct"), _ptr(conj_key, "conj_key"), _ptr(re, "re"),
+                                      _ptr(im, "im"), B, wp, _stream(ct)))
+        return re, im
+
+    def restore_merge(self, re, im, out=None):
+        """re + X^{n/2} im over [B][2][L][n]: slots a + i b."""
+        B = re.shape[0]
+        _ptr(re, "re", (B, 2, self.L, self.n))
+        _ptr(im, "im", (B, 2, self.L, self.n))
+        out = torch.empty_like(re) if out is None else out
+        check("ckks_restore_merge", lib().ckks_restore_merge(self._h, _ptr(re, "re"), _ptr(im, "im"),
+                                                             _ptr(out, "out"), B, _stream(re)))
+        return out
+
+    def modraise(self, x, out=None, ws=None):
+        """x[B][2][l][n] over q_0..q_{l-1} -> [B][2][L][n], each coefficient
+        lifted to its centred value and reduced modulo every prime."""
+        B, _, l, _ = x.shape
+        out = self._empty(B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_MODRAISE, B, l)
+        check("ckks_modraise", lib().ckks_modraise(self._h, _ptr(x, "in"), l, _ptr(out, "out"), B, wp,
+                                                   _stream(x)))
         return out
 
     # ------------------------------------------------------------ measurement

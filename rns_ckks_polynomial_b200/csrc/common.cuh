@@ -36,6 +36,12 @@ struct __align__(16) PrimeConst {
 // Device tables owned by a context (struct of device pointers, passed by value).
 struct Tables {
     int L, K, alpha, dnum, LK;
+    // Switching keys may be made for a longer chain of key_L >= L ciphertext
+    // primes (one key set serving the contexts of every lower level): ciphertext
+    // prime t sits at key row t, special prime k at key row key_L + k, and
+    // each (digit, component) block holds key_LK = key_L + K rows.
+    int key_L, key_LK;
+    const ulonglong2 *mul_i;      // [L+K][2]: {psi^{n/2}, Shoup}, {-psi^{n/2}, Shoup} (X^{n/2} in NTT form)
     bool special;               // every prime is 2^60 - delta with delta < 2^32
     const PrimeConst *pc;       // [L+K]
     const ulonglong2 *tw_fwd;   // [L+K][n]: {psi^brv(k), Shoup}; k = 0 unused
@@ -65,6 +71,8 @@ struct ckks_ctx {
     std::vector<void *> allocations;
     // rescale constants per input level lp1: device [lp1-1] of {q_l^-1 mod q_i, Shoup}
     std::map<int, ulonglong2 *> rescale_tab;
+    // modraise tables per input level l (boot.cu)
+    std::map<int, void *> raise_tab;
     std::mutex mu;
     void *own_ws = nullptr;
     size_t own_ws_bytes = 0;

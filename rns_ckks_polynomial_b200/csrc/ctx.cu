@@ -230,9 +230,10 @@ static int build_tables(ckks_ctx *ctx)
     const std::vector<u64> &m = ctx->mods;
     Tables &T = ctx->t;
     T.L = L; T.K = K; T.alpha = alpha; T.dnum = dnum; T.LK = LK;
+    T.key_L = L; T.key_LK = LK;
 
     std::vector<PrimeConst> pc(LK);
-    std::vector<ulonglong2> fw((size_t)LK * n), iw((size_t)LK * n);
+    std::vector<ulonglong2> fw((size_t)LK * n), iw((size_t)LK * n), iq((size_t)2 * LK);
     parallel_for(LK, [&](int t) {
         const u64 q = m[t];
         PrimeConst &c = pc[t];
@@ -258,6 +259,8 @@ static int build_tables(ckks_ctx *ctx)
             v[k] = make_ulonglong2(pwi[e], host_shoup(pwi[e], q));
         }
         f[0] = make_ulonglong2(1, host_shoup(1, q));
+        iq[2 * t] = make_ulonglong2(pw[n / 2], host_shoup(pw[n / 2], q));
+        iq[2 * t + 1] = make_ulonglong2(q - pw[n / 2], host_shoup(q - pw[n / 2], q));
         u64 last = host_mulmod(v[1].x, c.ninv, q);  // psi^-brv(1) n^-1
         v[0] = make_ulonglong2(last, host_shoup(last, q));
     });
@@ -314,6 +317,7 @@ static int build_tables(ckks_ctx *ctx)
     CKKS_TRY(upload(ctx, pc, &T.pc));
     CKKS_TRY(upload(ctx, fw, &T.tw_fwd));
     CKKS_TRY(upload(ctx, iw, &T.tw_inv));
+    CKKS_TRY(upload(ctx, iq, &T.mul_i));
     CKKS_TRY(upload(ctx, up_hatinv, &T.up_hatinv));
     CKKS_TRY(upload(ctx, up_mat, &T.up_mat));
     CKKS_TRY(upload(ctx, dn_hatinv, &T.dn_hatinv));
@@ -326,6 +330,7 @@ static void free_ctx(ckks_ctx *ctx)
 {
     for (void *p : ctx->allocations) cudaFree(p);
     for (auto &kv : ctx->rescale_tab) cudaFree(kv.second);
+    free_raise_tables(ctx);
     if (ctx->own_ws) cudaFree(ctx->own_ws);
     delete ctx;
 }
@@ -435,6 +440,16 @@ extern "C" int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine)
     if (engine != CKKS_CONV_AUTO && engine != CKKS_CONV_INTEGER && engine != CKKS_CONV_TENSOR)
         return set_error(CKKS_EINVAL, "unknown conversion engine");
     ctx->conv_engine.store(engine, std::memory_order_relaxed);
+    return CKKS_OK;
+}
+
+extern "C" int ckks_ctx_set_key_chain(ckks_ctx *ctx, int key_L)
+{
+    CKKS_TRY(check_ctx(ctx));
+    if (key_L < ctx->L || key_L > 4096)
+        return set_error(CKKS_EINVAL, "key_L must be in [L, 4096]");
+    ctx->t.key_L = key_L;
+    ctx->t.key_LK = key_L + ctx->K;
     return CKKS_OK;
 }
 

@@ -40,6 +40,14 @@ int bench_mma(const ckks_ctx *ctx, int n, int blocks, int iters, double *ms, dou
 // launches the bounded-wait expiry self-test (asynchronous)
 int selftest_wait_expiry(const ckks_ctx *ctx);
 
+// ---- bootstrapping building blocks (boot.cu)
+// conv_kernel over the Garner digits and sign rows dg[P][l+1][n] into rows l..L-1 of out[P][L][n]
+int raise_conv(const Tables &T, const u64 *dg, u64 *out, const u64 *matp, int l, int P, cudaStream_t s);
+void free_raise_tables(ckks_ctx *ctx);
+size_t modraise_ws_bytes(const ckks_ctx *ctx, int batch, int l);
+size_t conj_extract_ws_bytes(const ckks_ctx *ctx, int batch);
+size_t rotate_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys);
+
 // ---- sizes of internal stages (bytes)
 size_t modup_ws_bytes(const ckks_ctx *ctx, int batch);
 size_t moddown_ws_bytes(const ckks_ctx *ctx, int jobs);

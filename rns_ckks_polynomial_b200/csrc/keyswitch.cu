@@ -120,6 +120,28 @@ static int launch_conv(const Map &m, int max_targets, int jobs, const Tables &T,
     return CKKS_OK;
 }
 
+// modraise conversion: job z = polynomial; sources its l Garner digits and the
+// sign row; targets the primes l..L-1.  matp[s][t] = [q_0..q_{s-1}]_{q_t} for
+// s < l and [-Q]_{q_t} for s = l, so the exact sum is the centred lift.
+struct RaiseConvMap {
+    const u64 *dg;
+    u64 *out;
+    const u64 *matp;  // [l+1][L]
+    int l, L;
+    __device__ __forceinline__ int sources(int) const { return l + 1; }
+    __device__ __forceinline__ int targets(int) const { return L - l; }
+    __device__ __forceinline__ const u64 *src(int z) const { return dg + (size_t)z * (l + 1) * kN; }
+    __device__ __forceinline__ u64 mat(int, int s, int t) const { return matp[(size_t)s * L + l + t]; }
+    __device__ __forceinline__ u64 *dst(int z, int t) const { return out + ((size_t)z * L + l + t) * kN; }
+    __device__ __forceinline__ int prime(int, int t) const { return l + t; }
+};
+
+int raise_conv(const Tables &T, const u64 *dg, u64 *out, const u64 *matp, int l, int P, cudaStream_t s)
+{
+    RaiseConvMap m{dg, out, matp, l, T.L};
+    return launch_conv(m, T.L - l, P, T, s);
+}
+
 // ---------------------------------------------------------------- ModUp
 // INTT of source limb i of polynomial b; the load also writes the input limb
 // (NTT domain) into its own digit, the store multiplies by [(Q_j/q_i)^-1].
@@ -258,13 +280,15 @@ __global__ void __launch_bounds__(kKiThreads, 4) key_inner_kernel(const u64 *__r
     const size_t LKn = (size_t)T.LK * kN;
     const size_t bstride = (size_t)T.dnum * LKn;  // between the digit sets of consecutive ciphertexts
     const u64 *dg = digits + (size_t)(hoisted ? b0 : r * per_key + b0) * bstride + (size_t)t * kN + src;
-    const u64 *kp = kl.key[r] + (size_t)t * kN + k;
+    const size_t kLKn = (size_t)T.key_LK * kN;  // key rows per (digit, component)
+    const int kt = t < T.L ? t : t - T.L + T.key_L;
+    const u64 *kp = kl.key[r] + (size_t)kt * kN + k;
     u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
 #pragma unroll
     for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
 #pragma unroll 2
     for (int j = 0; j < T.dnum; ++j) {
-        const u64 kb = __ldg(kp + (size_t)(2 * j) * LKn), ka = __ldg(kp + (size_t)(2 * j + 1) * LKn);
+        const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
         const u64 *dj = dg + (size_t)j * LKn;
         u64 d[kKiB];
 #pragma unroll

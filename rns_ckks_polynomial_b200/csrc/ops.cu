@@ -286,6 +286,8 @@ extern "C" size_t ckks_workspace_bytes(const ckks_ctx *ctx, int op, int batch, i
     case CKKS_OP_KEYSWITCH: return keyswitch_ws_bytes(ctx, batch);
     case CKKS_OP_ROTATE: return rotate_ws_bytes(ctx, batch, aux);
     case CKKS_OP_ROTATE_UNHOISTED: return rotate_unhoisted_ws(ctx, batch);
+    case CKKS_OP_MODRAISE: return aux >= 1 ? modraise_ws_bytes(ctx, batch, aux) : 0;
+    case CKKS_OP_CONJ_EXTRACT: return conj_extract_ws_bytes(ctx, batch);
     case CKKS_OP_RESCALE: return rescale_ws_bytes(batch);
     case CKKS_OP_MUL_RELIN_RESCALE: return mrr_ws(ctx, batch);
     case CKKS_OP_BSGS: {
@@ -480,31 +482,18 @@ extern "C" int ckks_mul_relin_rescale(const ckks_ctx *ctx, const uint64_t *a, co
     return rescale_stage(m, cr, out, L, batch, scratch, s);
 }
 
-extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
-                                  const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
-                                  int bb, int gg, uint64_t *y, int batch, void *ws,
-                                  ckks_stream_t stream)
+// The BSGS transform for diagonals at offsets stride (t0 + bb g + b), g < gg,
+// b < bb (the dense form is stride 1, t0 0):
+//   y = Rescale( sum_g Rot_{G_g}( sum_b diags[g][b] * Rot_{stride b}(x) ) ),
+//   G_g = stride (t0 + bb g) mod n/2.
+// giant_keys[g] serves G_g (unused where G_g = 0, which needs no rotation).
+static int bsgs_core(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                     const uint64_t *const *baby_keys, const uint64_t *const *giant_keys, int stride,
+                     int t0, int bb, int gg, uint64_t *y, int batch, void *ws, cudaStream_t s)
 {
-    CKKS_TRY(check_ctx(ctx));
-    CKKS_TRY(check_batch(batch));
-    if (ctx->L < 2) return set_error(CKKS_EUNSUPPORTED, "rescale needs L >= 2");
-    if (bb < 1 || gg < 1 || bb > kMaxBaby || gg > 999)
-        return set_error(CKKS_EINVAL, "need 1 <= bb <= 64 and 1 <= gg <= 999");
-    if ((size_t)batch * std::max(bb - 1, 1) > 32767)
-        return set_error(CKKS_EUNSUPPORTED, "batch * (bb - 1) above 32767");
-    if (batch == 0) return CKKS_OK;
-    CKKS_TRY(check_ptr(x, "x"));
-    CKKS_TRY(check_ptr(diags, "diags"));
-    CKKS_TRY(check_ptr(y, "y"));
-    if (bb > 1 && !baby_keys) return set_error(CKKS_EINVAL, "null baby key array");
-    if (gg > 1 && !giant_keys) return set_error(CKKS_EINVAL, "null giant key array");
-    for (int r = 0; r + 1 < bb; ++r) CKKS_TRY(check_ptr(baby_keys[r], "baby_keys[r]"));
-    for (int g = 0; g + 1 < gg; ++g) CKKS_TRY(check_ptr(giant_keys[g], "giant_keys[g]"));
-    CKKS_TRY(set_device(ctx));
     ckks_ctx *m = const_cast<ckks_ctx *>(ctx);
     void *w;
     CKKS_TRY(resolve_ws(m, ws, bsgs_ws(ctx, batch, bb, gg), &w));
-    const cudaStream_t s = (cudaStream_t)stream;
     const Tables &T = ctx->t;
     const int L = ctx->L, B = batch;
     const size_t Ln = (size_t)L * kN, ctn = 2 * Ln;
@@ -518,7 +507,7 @@ extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const 
     u64 *total = reinterpret_cast<u64 *>(base + lay.digits + lay.acc + lay.baby + lay.inner + lay.rot);
     void *scratch = base + lay.digits + lay.acc + lay.baby + lay.inner + lay.rot + lay.total;
 
-    // baby steps: Rot_r(x), r = 1..bb-1, on one hoisted ModUp
+    // baby steps: Rot_{stride r}(x), r = 1..bb-1, on one hoisted ModUp
     if (bb > 1) {
         CKKS_TRY(modup_stage(ctx, x + Ln, nullptr, ctn, digits, B, scratch, s));
         for (int r0 = 1; r0 < bb; r0 += kMaxKeys) {
@@ -532,7 +521,7 @@ extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const 
             ex.per = B;
             for (int r = 0; r < nk; ++r) {
                 kl.key[r] = baby_keys[r0 + r - 1];
-                kl.galois[r] = ex.gal[r] = galois_pow5(r0 + r);
+                kl.galois[r] = ex.gal[r] = galois_pow5((long long)stride * (r0 + r));
             }
             CKKS_TRY(key_inner_stage(ctx, digits, kl, B, true, acc, nk * B, s));
             CKKS_TRY(moddown_stage(ctx, acc, baby + (size_t)(r0 - 1) * B * ctn, nk * B, ex, scratch, s));
@@ -552,31 +541,107 @@ extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const 
         }
         CKKS_CHECK_LAUNCH("bsgs_inner_kernel");
     }
-    // giant steps: total = inner_0 + sum_{g >= 1} Rot_{bb g}(inner_g)
+    // giant steps: total = (the unrotated inner sum, if any) + sum of the rotated ones
+    const int S = kN / 2;
+    auto giant = [&](int g) {
+        long long v = (long long)stride * (t0 + (long long)bb * g) % S;
+        return (int)(v < 0 ? v + S : v);
+    };
+    int gz = -1;
+    for (int g = 0; g < gg && gz < 0; ++g)
+        if (giant(g) == 0) gz = g;
     const size_t all = (size_t)B * ctn;
-    accum_kernel<<<grid_for(all, 256), 256, 0, s>>>(total, inner, nullptr, 0, B, L, T.pc);
-    CKKS_CHECK_LAUNCH("accum_kernel");
-    for (int g0 = 1; g0 < gg; g0 += lay.gchunk) {
-        const int ng = std::min(lay.gchunk, gg - g0);
-        const u64 *src = inner + (size_t)g0 * B * ctn;
-        CKKS_TRY(modup_stage(ctx, src + Ln, nullptr, ctn, digits, ng * B, scratch, s));
-        KeyList kl{};
-        DownExtra ex;
-        ex.kind = 1;
-        ex.ct = src;
-        ex.ct_bstride = ctn;
-        ex.ct_mod = 0;
-        ex.per = B;
-        for (int g = 0; g < ng; ++g) {
-            kl.key[g] = giant_keys[g0 + g - 1];
-            kl.galois[g] = ex.gal[g] = galois_pow5((long long)bb * (g0 + g));
-        }
-        CKKS_TRY(key_inner_stage(ctx, digits, kl, B, false, acc, ng * B, s));
-        CKKS_TRY(moddown_stage(ctx, acc, rot, ng * B, ex, scratch, s));
-        accum_kernel<<<grid_for(all, 256), 256, 0, s>>>(total, nullptr, rot, ng, B, L, T.pc);
+    if (gz >= 0) {
+        accum_kernel<<<grid_for(all, 256), 256, 0, s>>>(total, inner + (size_t)gz * B * ctn, nullptr, 0, B, L,
+                                                        T.pc);
         CKKS_CHECK_LAUNCH("accum_kernel");
+    } else {
+        cudaError_t e = cudaMemsetAsync(total, 0, all * sizeof(u64), s);
+        if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync(bsgs total)");
+    }
+    // the rotated giant steps form at most two runs of consecutive g, around gz
+    const int run_lo[2] = {0, gz + 1}, run_hi[2] = {gz < 0 ? gg : gz, gz < 0 ? 0 : gg};
+    for (int run = 0; run < 2; ++run) {
+        for (int g0 = run_lo[run]; g0 < run_hi[run]; g0 += lay.gchunk) {
+            const int ng = std::min(lay.gchunk, run_hi[run] - g0);
+            const u64 *src = inner + (size_t)g0 * B * ctn;
+            CKKS_TRY(modup_stage(ctx, src + Ln, nullptr, ctn, digits, ng * B, scratch, s));
+            KeyList kl{};
+            DownExtra ex;
+            ex.kind = 1;
+            ex.ct = src;
+            ex.ct_bstride = ctn;
+            ex.ct_mod = 0;
+            ex.per = B;
+            for (int g = 0; g < ng; ++g) {
+                kl.key[g] = giant_keys[g0 + g];
+                kl.galois[g] = ex.gal[g] = galois_pow5(giant(g0 + g));
+            }
+            CKKS_TRY(key_inner_stage(ctx, digits, kl, B, false, acc, ng * B, s));
+            CKKS_TRY(moddown_stage(ctx, acc, rot, ng * B, ex, scratch, s));
+            accum_kernel<<<grid_for(all, 256), 256, 0, s>>>(total, nullptr, rot, ng, B, L, T.pc);
+            CKKS_CHECK_LAUNCH("accum_kernel");
+        }
     }
     return rescale_stage(m, total, y, L, B, scratch, s);
+}
+
+static int bsgs_checks(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags, uint64_t *y, int bb,
+                       int gg, int batch)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (ctx->L < 2) return set_error(CKKS_EUNSUPPORTED, "rescale needs L >= 2");
+    if (bb < 1 || gg < 1 || bb > kMaxBaby || gg > 999)
+        return set_error(CKKS_EINVAL, "need 1 <= bb <= 64 and 1 <= gg <= 999");
+    if ((size_t)batch * std::max(bb - 1, 1) > 32767)
+        return set_error(CKKS_EUNSUPPORTED, "batch * (bb - 1) above 32767");
+    if (batch == 0) return CKKS_OK;
+    CKKS_TRY(check_ptr(x, "x"));
+    CKKS_TRY(check_ptr(diags, "diags"));
+    CKKS_TRY(check_ptr(y, "y"));
+    return CKKS_OK;
+}
+
+extern "C" int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                                  const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
+                                  int bb, int gg, uint64_t *y, int batch, void *ws,
+                                  ckks_stream_t stream)
+{
+    CKKS_TRY(bsgs_checks(ctx, x, diags, y, bb, gg, batch));
+    if (batch == 0) return CKKS_OK;
+    if (bb > 1 && !baby_keys) return set_error(CKKS_EINVAL, "null baby key array");
+    if (gg > 1 && !giant_keys) return set_error(CKKS_EINVAL, "null giant key array");
+    for (int r = 0; r + 1 < bb; ++r) CKKS_TRY(check_ptr(baby_keys[r], "baby_keys[r]"));
+    for (int g = 0; g + 1 < gg; ++g) CKKS_TRY(check_ptr(giant_keys[g], "giant_keys[g]"));
+    CKKS_TRY(set_device(ctx));
+    // giant step g >= 1 uses giant_keys[g - 1]; step 0 is unrotated
+    std::vector<const uint64_t *> gk(gg, nullptr);
+    for (int g = 1; g < gg; ++g) gk[g] = giant_keys[g - 1];
+    return bsgs_core(ctx, x, diags, baby_keys, gk.data(), 1, 0, bb, gg, y, batch, ws, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_bsgs_lintrans_plan(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
+                                       const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
+                                       int stride, int t0, int bb, int gg, uint64_t *y, int batch, void *ws,
+                                       ckks_stream_t stream)
+{
+    CKKS_TRY(bsgs_checks(ctx, x, diags, y, bb, gg, batch));
+    if (stride < 1 || (long long)stride * (bb - 1) >= kN / 2)
+        return set_error(CKKS_EINVAL, "need stride >= 1 and stride * (bb - 1) < n/2");
+    if (t0 < -(kN / 2) || t0 > kN / 2) return set_error(CKKS_EINVAL, "t0 outside [-n/2, n/2]");
+    if (batch == 0) return CKKS_OK;
+    if (bb > 1 && !baby_keys) return set_error(CKKS_EINVAL, "null baby key array");
+    if (!giant_keys) return set_error(CKKS_EINVAL, "null giant key array");
+    for (int r = 0; r + 1 < bb; ++r) CKKS_TRY(check_ptr(baby_keys[r], "baby_keys[r]"));
+    const int S = kN / 2;
+    for (int g = 0; g < gg; ++g) {
+        long long v = (long long)stride * (t0 + (long long)bb * g) % S;
+        if (v != 0) CKKS_TRY(check_ptr(giant_keys[g], "giant_keys[g]"));
+    }
+    CKKS_TRY(set_device(ctx));
+    return bsgs_core(ctx, x, diags, baby_keys, giant_keys, stride, t0, bb, gg, y, batch, ws,
+                     (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------- microbenchmarks

@@ -23,11 +23,18 @@ SIGNATURES = {
     "ckks_ctx_params": (C.c_int, [_vp] + [C.POINTER(C.c_int)] * 5),
     "ckks_device_status": (C.c_int, [_vp]),
     "ckks_ctx_set_conversion": (C.c_int, [_vp, C.c_int]),
+    "ckks_ctx_set_key_chain": (C.c_int, [_vp, C.c_int]),
     "ckks_selftest_wait_expiry": (C.c_int, [_vp]),
     "ckks_workspace_bytes": (C.c_size_t, [_vp, C.c_int, C.c_int, C.c_int]),
     "ckks_ntt_fwd": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_ntt_inv": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_pointwise": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_pointwise_scalar": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_add_const_c0": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp]),
+    "ckks_mul_i": (C.c_int, [_vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_conj_extract": (C.c_int, [_vp, _vp, _vp, _vp, _vp, C.c_int, _vp, _vp]),
+    "ckks_restore_merge": (C.c_int, [_vp, _vp, _vp, _vp, C.c_int, _vp]),
+    "ckks_modraise": (C.c_int, [_vp, _vp, C.c_int, _vp, C.c_int, _vp, _vp]),
     "ckks_automorph": (C.c_int, [_vp, _vp, _vp, C.c_int, C.c_int, C.c_uint32, _vp]),
     "ckks_modup": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp, _vp]),
     "ckks_modup_noalloc": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp]),
@@ -42,6 +49,8 @@ SIGNATURES = {
     "ckks_mul_relin_rescale": (C.c_int, [_vp, _vp, _vp, _vp, _vp, C.c_int, _vp, _vp]),
     "ckks_bsgs_lintrans": (C.c_int, [_vp, _vp, _vp, C.POINTER(_vp), C.POINTER(_vp), C.c_int,
                                      C.c_int, _vp, C.c_int, _vp, _vp]),
+    "ckks_bsgs_lintrans_plan": (C.c_int, [_vp, _vp, _vp, C.POINTER(_vp), C.POINTER(_vp), C.c_int,
+                                          C.c_int, C.c_int, C.c_int, _vp, C.c_int, _vp, _vp]),
     "ckks_bench_intpipe": (C.c_int, [_vp, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_double),
                                      C.POINTER(C.c_double)]),
 }

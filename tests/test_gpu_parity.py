@@ -474,3 +474,199 @@ def test_unhoisted_rotation_order(orc):
     ctx2.device_status()
     assert_bits_equal(got, orc.rotate_unhoisted(ct, [key], np.array([25], dtype=np.uint64), mods, 40, 20, 20),
                       "rotate_unhoisted, tensor-core conversion")
+
+
+# ------------------------------------------------------------------ keys of a longer chain
+@pytest.mark.parametrize("L,K,alpha,l", [(6, 2, 2, 3), (7, 2, 3, 4), (20, 3, 7, 13), (5, 1, 1, 1)])
+def test_key_chain_serves_lower_levels(orc, L, K, alpha, l):
+    """A context on q_0..q_{l-1} (with the top chain's special primes) given
+    keys made for all L primes (set_key_chain(L)): key switch, rotation and
+    relinearised product bit-exact against the oracle run with the keys cut
+    down to level l.  (5, 1, 1, 1) is the single-prime chain a refresh starts
+    from."""
+    from oracle.boot import Chain
+
+    from rns_ckks_polynomial_b200 import Context
+    mods = [int(x) for x in orc.gen_primes(N, L + K)]
+    m64 = np.array(mods, dtype=np.uint64)
+    chain = Chain(m64, L, K, alpha)
+    m_l = chain.mods_at(l)
+    ctx = Context(mods[:l], mods[L:], alpha)
+    try:
+        ctx.set_key_chain(L)
+        key = _res((Params(L, K, alpha).dnum, 2, L + K, N), m64, 300)
+        key_l = chain.key_at(key, l)
+        d = _res((2, l, N), m_l[:l], 301)
+        assert_bits_equal(host(ctx.keyswitch(dev(d), dev(key))),
+                          orc.keyswitch(d, key_l, m_l, l, K, alpha), "keyswitch, level %d" % l)
+        ct = _res((2, 2, l, N), m_l[:l], 302)
+        assert_bits_equal(host(ctx.rotate(dev(ct), [dev(key)], [5])),
+                          orc.rotate(ct, [key_l], np.array([5], dtype=np.uint64), m_l, l, K, alpha),
+                          "rotate, level %d" % l)
+        if l >= 2:
+            a, b = _res((1, 2, l, N), m_l[:l], 303), _res((1, 2, l, N), m_l[:l], 304)
+            assert_bits_equal(host(ctx.mul_relin_rescale(dev(a), dev(b), dev(key))),
+                              orc.mul_relin_rescale(a, b, key_l, m_l, l, K, alpha),
+                              "mul_relin_rescale, level %d" % l)
+        with pytest.raises(CkksError):
+            ctx.set_key_chain(l - 1)
+    finally:
+        ctx.close()
+
+
+# ------------------------------------------------------------------ refresh building blocks
+def test_mul_i_scalar_ops_and_c0_constant(orc):
+    """X^{n/2} (slots times i) against the oracle's coefficient-domain
+    monomial product; products and sums with a per-limb constant; a constant
+    added to component 0 only."""
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    LK = p.L + p.K
+    x = _res((3, LK, N), mods, 400)
+    assert_bits_equal(host(ctx.mul_i(dev(x))), orc.mul_monomial(x, N // 2, mods), "mul_i")
+    k = np.ascontiguousarray(_res((LK, 1), mods, 401)[:, 0])
+    kb = np.ascontiguousarray(np.broadcast_to(k[:, None], x.shape))
+    for op in ("mul", "add", "sub"):
+        assert_bits_equal(host(ctx.pointwise_scalar(op, dev(x), dev(k))),
+                          orc.pointwise(op, x, kb, mods), "pointwise_scalar %s" % op)
+    ct = _res((2, 2, p.L, N), mods[:p.L], 402)
+    want = ct.copy()
+    want[:, 0] = orc.pointwise("add", ct[:, 0], np.ascontiguousarray(
+        np.broadcast_to(k[:p.L, None], ct[:, 0].shape)), mods[:p.L])
+    assert_bits_equal(host(ctx.add_const_c0(dev(ct), dev(np.ascontiguousarray(k[:p.L])))), want,
+                      "add_const_c0")
+
+
+def test_conj_extract_and_restore_merge(orc):
+    """Bit-exact against the oracle, and the slots decrypt to 2 Re w, 2 Im w,
+    then to 2 w after the merge."""
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 40)
+    w = synth.uniform_real((SLOTS,), -1, 1, SEED, 410).numpy() + \
+        1j * synth.uniform_real((SLOTS,), -1, 1, SEED, 411).numpy()
+    ct = sch.encrypt_slots(w)[None]
+    ck = sch.keygen_galois(2 * N - 1)
+    re, im = ctx.conj_extract(dev(ct), dev(ck))
+    want_re, want_im = orc.conj_extract(ct, ck, sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(host(re), want_re, "conj_extract re")
+    assert_bits_equal(host(im), want_im, "conj_extract im")
+    merged = ctx.restore_merge(re, im)
+    assert_bits_equal(host(merged), orc.restore_merge(want_re, want_im, sch.q), "restore_merge")
+    assert np.max(np.abs(sch.decrypt_slots(host(re)[0], 2 * SCALE) - w.real)) < 1e-8
+    assert np.max(np.abs(sch.decrypt_slots(host(merged)[0], 2 * SCALE) - w)) < 1e-8
+
+
+@pytest.mark.parametrize("L,K,alpha,l", [(6, 2, 2, 1), (6, 2, 2, 3), (6, 2, 2, 6), (40, 4, 4, 19),
+                                         (80, 4, 4, 63)])
+def test_modraise(orc, L, K, alpha, l):
+    """The centred lift onto the whole chain, bit-exact against the oracle;
+    coefficients 0, 1, (Q-1)/2, (Q+1)/2 and Q-1 sit at the start of the
+    first polynomial, where the sign decision is tightest."""
+    ctx = context(L, K, alpha)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    q = [int(v) for v in mods[:l]]
+    Q = 1
+    for v in q:
+        Q *= v
+    coef = _res((2, 2, l, N), mods[:l], 420)
+    for j, X in enumerate([0, 1, (Q - 1) // 2, (Q + 1) // 2, Q - 1]):
+        for i in range(l):
+            coef[0, 0, i, j] = X % q[i]
+    x = orc.ntt_fwd(coef, mods[:l])
+    got = host(ctx.modraise(dev(x)))
+    assert_bits_equal(got, orc.modraise(x, mods[:L]), "modraise l=%d" % l)
+
+
+@pytest.mark.parametrize("plan", [(64, -8, 4, 4), (8, -7, 4, 4), (1, -7, 4, 4), (1, 0, 4, 3),
+                                  (3, 5, 2, 1)])
+def test_bsgs_plan_matches_oracle(orc, plan):
+    """Strided-window BSGS (the groups of a three-level factored transform at
+    n = 2048, the dense window, and a single rotated giant step) bit-exact
+    against the oracle on seeded residues, with the oracle's Galois keys."""
+    from oracle.boot import Chain, bsgs_plan_apply
+    stride, t0, bb, gg = plan
+    S = SLOTS
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    sch = Scheme(orc, p, SEED + 50)
+    chain = Chain(sch.mods, p.L, p.K, p.alpha)
+    amounts = {(stride * b) % S for b in range(1, bb)} | {(stride * (t0 + bb * g)) % S for g in range(gg)}
+    keys = {a: sch.keygen_galois(galois_for_rotation(a)) for a in amounts if a}
+    x = _res((2, 2, p.L, N), sch.q, 430)
+    pts = _res((gg, bb, p.L, N), sch.q, 431)
+    giants = [(stride * (t0 + bb * g)) % S for g in range(gg)]
+    y = host(ctx.bsgs_lintrans_plan(dev(x), dev(pts), [dev(keys[(stride * b) % S]) for b in range(1, bb)],
+                                    [dev(keys[G]) if G else None for G in giants], plan))
+    for i in range(2):
+        want, _ = bsgs_plan_apply(x[i], SCALE, [[pts[g, b] for b in range(bb)] for g in range(gg)],
+                                  plan, SCALE, keys, chain)
+        assert_bits_equal(y[i], want, "bsgs plan %s, ct %d" % (plan, i))
+
+
+def test_refresh_matches_oracle(orc):
+    """The whole refresh at n = 2048 (16 primes, the plans of two-level
+    factored transforms, r = 4: 2 * 2 + 6 + 4 levels) through the per-level
+    contexts and one top-level key set, bit-exact against the oracle's
+    refresh with the same seeded plaintext residues, and the same tracked
+    scale.  (Decryption of the refresh is pinned on the CPU.)"""
+    from oracle import boot
+
+    from rns_ckks_polynomial_b200.refresh import Refresh
+    L, K, alpha, depth, r = 16, 4, 4, 2, 4
+    p = Params(L, K, alpha)
+    sch = Scheme(orc, p, SEED + 60)
+    chain = boot.Chain(sch.mods, L, K, alpha)
+    keys = {"rot": {a: sch.keygen_galois(galois_for_rotation(a))
+                    for a in boot.factored_rotation_amounts(N, depth)},
+            "conj": sch.keygen_galois(2 * N - 1), "relin": sch.keygen_relin()}
+    low = np.ascontiguousarray(_res((2, 1, N), sch.q[:1], 440))
+
+    def levels(factors, top, stream):
+        out = []
+        for i, F in enumerate(factors):
+            plan = orc.bsgs_plan(F, SLOTS)
+            _, _, bb, gg = plan
+            out.append((plan, _res((gg, bb, top - i, N), sch.q[:top - i], stream + i)))
+        return out
+
+    cts = levels(orc.factored_coeff_to_slot(N, depth), L, 450)
+    stc = levels(orc.factored_slot_to_coeff(N, depth), L - depth - 6 - r, 460)
+    want, s_want = boot.refresh_with_levels(low, r, [(pl, list(a)) for pl, a in cts],
+                                            [(pl, list(a)) for pl, a in stc], keys, chain)
+    dkeys = {"rot": {a: dev(k) for a, k in keys["rot"].items()}, "conj": dev(keys["conj"]),
+             "relin": dev(keys["relin"])}
+    rf = Refresh(sch.q, sch.mods[L:], alpha, dkeys)
+    try:
+        got, s_got = rf.refresh(dev(low[None]), r, [(pl, dev(a)) for pl, a in cts],
+                                [(pl, dev(a)) for pl, a in stc])
+        assert s_got == s_want
+        assert_bits_equal(host(got)[0], want, "refresh")
+    finally:
+        rf.close()
+
+
+def test_extreme_residues(orc):
+    """Inputs at the ends of [0, q): all zeros, all q - 1, and q - 1
+    alternating with 0, through the NTT both ways, a key switch and a rescale
+    (the lazy butterflies and 128-bit sums see their largest operands)."""
+    p = Params(6, 2, 2)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    q = mods[:p.L]
+    top = np.broadcast_to((q - 1)[:, None], (p.L, N))
+    alt = np.where(np.arange(N) % 2 == 0, top, 0).astype(np.uint64)
+    cases = [np.zeros((p.L, N), np.uint64), np.ascontiguousarray(top, dtype=np.uint64), alt]
+    x = np.stack(cases)
+    y = dev(x)
+    ctx.ntt_fwd(y)
+    assert_bits_equal(host(y), orc.ntt_fwd(x, q), "ntt_fwd extremes")
+    ctx.ntt_inv(y)
+    assert_bits_equal(host(y), x, "ntt round trip extremes")
+    kt = np.broadcast_to((mods - 1)[None, None, :, None], (p.dnum, 2, p.L + p.K, N))
+    key = np.ascontiguousarray(kt, dtype=np.uint64)
+    assert_bits_equal(host(ctx.keyswitch(dev(x), dev(key))), orc.keyswitch(x, key, mods, p.L, p.K, p.alpha),
+                      "keyswitch extremes")
+    ct = np.stack([np.stack([c, c]) for c in cases])
+    assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, q), "rescale extremes")

@@ -96,6 +96,7 @@ def test_calls_reject_null_context():
     assert lib.ckks_workspace_bytes(None, 1, 1, 0) == 0
     assert "null context" in lib.ckks_last_error().decode()
     assert lib.ckks_ctx_set_conversion(None, 1) == EINVAL
+    assert lib.ckks_ctx_set_key_chain(None, 5) == EINVAL
     assert lib.ckks_selftest_wait_expiry(None) == EINVAL
 
 

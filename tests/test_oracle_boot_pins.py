@@ -419,3 +419,35 @@ def test_bootstrap_at_ring_degree_2048(orc):
     got = np.array([float(Fraction(c) / s) for c in _centred_coeffs(sch, out)])
     sine = np.array([q0 / (2 * math.pi) * math.sin(2 * math.pi * v / q0) / delta for v in m])
     assert np.max(np.abs(got - sine)) < 1e-5
+
+
+def test_refresh_with_levels_is_the_factored_refresh(orc):
+    """Fed the encoded levels, the plaintext-taking refresh is the factored
+    refresh bit for bit (zeros stand for absent diagonals)."""
+    import math
+
+    from oracle import boot
+    n, depth, r = 64, 2, 8
+    delta = 2**50
+    sch, chain, keys = _factored_scheme(orc, n, depth, SEED + 12)
+    low = np.ascontiguousarray(sch.encrypt_slots(_complex_slots(n, 150), delta)[:, :1])
+    want, s_want = boot.bootstrap_factored(low, delta, r, depth, keys, chain)
+
+    def levels(factors, scalar, top, pt_scale):
+        out = []
+        for i, F in enumerate(factors):
+            if i == 0:
+                F = {k: scalar * d for k, d in F.items()}
+            plan = orc.bsgs_plan(F, n // 2)
+            pts, _ = orc.plan_plaintexts(F, plan, n // 2, sch.mods[:top - i], pt_scale, n)
+            out.append((plan, [[np.zeros((top - i, n), np.uint64) if v is None else v for v in row]
+                               for row in pts]))
+        return out
+
+    q0 = int(sch.mods[0])
+    cts = levels(orc.factored_coeff_to_slot(n, depth), 0.5, 20, 2**60)
+    stc = levels(orc.factored_slot_to_coeff(n, depth), q0 / (2 * math.pi * delta),
+                 20 - depth - 6 - r, 2**50)
+    got, s_got = boot.refresh_with_levels(low, r, cts, stc, keys, chain)
+    assert s_got == s_want
+    assert np.array_equal(got, want)
