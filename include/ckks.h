@@ -224,7 +224,10 @@ int ckks_modup(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int
  * launch nothing.
  * The first call on a device resolves the array's device address
  * (cudaGetSymbolAddress, once per device); make that first call before any
- * stream capture.
+ * stream capture.  The address is cached for the life of the process and
+ * belongs to the device's primary context as it was then: after
+ * cudaDeviceReset, or anything else that tears that context down, do not
+ * call this entry point again in the same process.
  * Every call shares the one array, so calls that overlap on the GPU (other
  * streams, other host threads, the same device) race: serialise them.  No
  * part of the array needs clearing between calls, because every word a call
@@ -237,18 +240,33 @@ int ckks_modup_noalloc(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *dig
  * acc[batch][2][L+K][n] with acc[b][c][t][k] = sum_j phi_g(D_j)[t][k] *
  * key[j][c][t][k] mod t.  digits [batch][dnum][L+K][n], key
  * [dnum][2][L+K][n] (component 0 = b, 1 = a).  galois = 1 means no
- * automorphism. */
+ * automorphism.  This is the step of a key switch that consumes the
+ * evaluation key, which the EncryptedLLM GPU article (section 2.5) sizes at
+ * hundreds of MB to several GB and names, with the rotation it serves, as
+ * the under-rated cost of encrypted inference.  Sums over any number of
+ * digits are exact (reduced once per 256 digits).  CKKS_EINVAL for a null
+ * pointer, a pointer that is not 16-byte aligned or an even galois. */
 int ckks_key_inner(const ckks_ctx *ctx, const uint64_t *digits, const uint64_t *key,
                    uint32_t galois, uint64_t *acc, int batch, ckks_stream_t stream);
 
 /* ModDown: acc[batch][2][L+K][n] -> out[batch][2][L][n],
  * out_i = (acc_i - NTT_i(sum_k [INTT(acc_{p_k}) (P/p_k)^-1]_{p_k} [P/p_k]_{q_i}))
- *         * P^-1 mod q_i.  ws: CKKS_OP_MODDOWN bytes. */
+ *         * P^-1 mod q_i.
+ * The conversion from the special primes back to the q_i is the same "RNS
+ * basis conversion" step that the Kestrel engine write-up (section 3
+ * table) names as the core of bootstrapping, run in the other direction;
+ * dividing by P ends the key switch of the EncryptedLLM GPU article
+ * (section 2.5).  ws: CKKS_OP_MODDOWN bytes. */
 int ckks_moddown(const ckks_ctx *ctx, const uint64_t *acc, uint64_t *out, int batch,
                  void *ws, ckks_stream_t stream);
 
 /* KeySwitch(d) = ModDown(<ModUp(d), key>): d[batch][L][n] (NTT),
- * key[dnum][2][L+K][n], out[batch][2][L][n].  ws: CKKS_OP_KEYSWITCH bytes. */
+ * key[dnum][2][L+K][n], out[batch][2][L][n].  This is the key switch that
+ * every rotation and every relinearisation runs (EncryptedLLM GPU article,
+ * section 2.5: a rotation is a transform plus a key switch, and
+ * relinearisation after a ct x ct product consumes an evaluation key); its
+ * two basis conversions are the "RNS basis conversion" of the Kestrel engine
+ * write-up, section 3 table.  ws: CKKS_OP_KEYSWITCH bytes. */
 int ckks_keyswitch(const ckks_ctx *ctx, const uint64_t *d, const uint64_t *key,
                    uint64_t *out, int batch, void *ws, ckks_stream_t stream);
 

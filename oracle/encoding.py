@@ -98,6 +98,38 @@ def encode_ntt(z, mods, scale, n):
     return ntt_fwd(res, mods)
 
 
+def encode_many(Z, n, scale):
+    """Encode every row of Z ([count][n/2] slots) as encode() does, with the
+    sum over slots written as one long-double matrix product against the
+    table zeta^(-k e_j).  The sums run in another order than encode()'s, so
+    a coefficient can differ from encode()'s by one where scale times the sum
+    falls within long-double rounding of a half-integer; both are
+    round(scale * tau^-1(z)) to within that rounding."""
+    Z = np.atleast_2d(np.asarray(Z, dtype=np.clongdouble))
+    if Z.shape[1] != n // 2:
+        raise ValueError("expected rows of %d slots" % (n // 2))
+    ang = _PI * _angle_matrix(n, -1).astype(np.longdouble) / np.longdouble(n)
+    re = np.cos(ang) @ Z.real.T
+    if np.any(Z.imag != 0):
+        re = re - np.sin(ang) @ Z.imag.T
+    v = (np.longdouble(2) / np.longdouble(n)) * re * np.longdouble(scale)
+    r = np.sign(v) * np.floor(np.abs(v) + np.longdouble(0.5))
+    return np.ascontiguousarray(r.T.astype(np.int64))
+
+
+def encode_ntt_many(Z, mods, scale, n):
+    """encode_many, then the residues of every coefficient modulo each prime
+    and the forward NTT: [count][L][n]."""
+    from .core import ntt_fwd
+    m = encode_many(Z, n, scale)
+    q = np.array([int(v) for v in mods], dtype=np.int64)
+    out = np.empty((m.shape[0], len(q), n), dtype=np.uint64)
+    for c in range(0, m.shape[0], 64):  # bounded temporaries
+        res = np.mod(m[c:c + 64, None, :], q[None, :, None]).astype(np.uint64)
+        out[c:c + 64] = ntt_fwd(res, mods)
+    return out
+
+
 def embedding_matrix(n):
     """U[j][k] = zeta^(k e_j), j, k < n/2, zeta = exp(i pi / n), e_j = 5^j mod 2n
     (reading R14 of the design notes).
@@ -292,4 +324,4 @@ __all__ = ["slot_exponents", "encode", "crt_centered", "decode", "decode_coeffs_
            "encode_ntt", "embedding_matrix", "coeff_to_slot_matrix", "slot_to_coeff_matrix",
            "lintrans_plaintexts", "bit_reverse_indices", "diag_product", "diag_to_dense",
            "stage_groups", "factored_slot_to_coeff", "factored_coeff_to_slot", "bsgs_plan",
-           "plan_plaintexts"]
+           "plan_plaintexts", "encode_many", "encode_ntt_many"]

@@ -260,6 +260,7 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 // gathered loads stay within one 256-byte segment).
 constexpr int kKiB = 4;       // ciphertexts per thread
 constexpr int kKiThreads = 128;
+constexpr int kKiFold = 256;  // digits summed exactly in 128 bits between reductions
 
 __global__ void __launch_bounds__(kKiThreads, 4) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
                                                         int per_key, int nkeys, int hoisted,
@@ -286,20 +287,33 @@ __global__ void __launch_bounds__(kKiThreads, 4) key_inner_kernel(const u64 *__r
     u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
 #pragma unroll
     for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
+    const PrimeConst pc = T.pc[t];
+    // 256 products below 2^120 plus a folded value below 2^60 stay below
+    // 2^128: past 256 digits the sums are reduced once per block of 256
+    for (int j0 = 0; j0 < T.dnum; j0 += kKiFold) {
+        if (j0 > 0) {
+#pragma unroll
+            for (int b = 0; b < kKiB; ++b) {
+                l0[b] = reduce128(h0[b], l0[b], pc);
+                l1[b] = reduce128(h1[b], l1[b], pc);
+                h0[b] = h1[b] = 0;
+            }
+        }
+        const int j1 = min(T.dnum, j0 + kKiFold);
 #pragma unroll 2
-    for (int j = 0; j < T.dnum; ++j) {
-        const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
-        const u64 *dj = dg + (size_t)j * LKn;
-        u64 d[kKiB];
+        for (int j = j0; j < j1; ++j) {
+            const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
+            const u64 *dj = dg + (size_t)j * LKn;
+            u64 d[kKiB];
 #pragma unroll
-        for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
+            for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
 #pragma unroll
-        for (int b = 0; b < kKiB; ++b) {
-            mac128(h0[b], l0[b], d[b], kb);
-            mac128(h1[b], l1[b], d[b], ka);
+            for (int b = 0; b < kKiB; ++b) {
+                mac128(h0[b], l0[b], d[b], kb);
+                mac128(h1[b], l1[b], d[b], ka);
+            }
         }
     }
-    const PrimeConst pc = T.pc[t];
 #pragma unroll
     for (int b = 0; b < kKiB; ++b) {
         if (b < nb) {

@@ -634,10 +634,17 @@ extern "C" int ckks_bsgs_lintrans_plan(const ckks_ctx *ctx, const uint64_t *x, c
     if (bb > 1 && !baby_keys) return set_error(CKKS_EINVAL, "null baby key array");
     if (!giant_keys) return set_error(CKKS_EINVAL, "null giant key array");
     for (int r = 0; r + 1 < bb; ++r) CKKS_TRY(check_ptr(baby_keys[r], "baby_keys[r]"));
+    // only the first giant step with G_g = 0 is summed unrotated; any other
+    // step (including a later one with G_g = 0) is a key switch and needs a key
     const int S = kN / 2;
+    bool unrotated_seen = false;
     for (int g = 0; g < gg; ++g) {
         long long v = (long long)stride * (t0 + (long long)bb * g) % S;
-        if (v != 0) CKKS_TRY(check_ptr(giant_keys[g], "giant_keys[g]"));
+        if (v == 0 && !unrotated_seen) {
+            unrotated_seen = true;
+            continue;
+        }
+        CKKS_TRY(check_ptr(giant_keys[g], "giant_keys[g]"));
     }
     CKKS_TRY(set_device(ctx));
     return bsgs_core(ctx, x, diags, baby_keys, giant_keys, stride, t0, bb, gg, y, batch, ws,

@@ -324,9 +324,10 @@ def test_bsgs_shapes(orc, bb, gg):
     assert_bits_equal(y, orc.bsgs(x, diags, baby, giant, bb, gg, mods, 5, 2, 2), "bsgs %dx%d" % (bb, gg))
 
 
-def test_config4_bsgs_full_size_sampled(orc):
-    """112 primes, alpha = 8, bb = gg = 32, 62 keys, 8 ciphertexts: the GPU
-    runs the full batch; the oracle recomputes ciphertext 5."""
+def test_config4_bsgs_full_size(orc):
+    """112 primes, alpha = 8, bb = gg = 32, 62 keys, 8 ciphertexts of seeded
+    uniform residues: the GPU runs the batch, the oracle recomputes every
+    ciphertext."""
     p = Params(112, 8, 8)
     ctx = ctx_for(p)
     seed = synth.config_seed(4)
@@ -337,17 +338,52 @@ def test_config4_bsgs_full_size_sampled(orc):
     baby = [synth.uniform_residues(kshape, mods, seed, 100 + i, device="cuda") for i in range(31)]
     giant = [synth.uniform_residues(kshape, mods, seed, 200 + i, device="cuda") for i in range(31)]
     y = ctx.bsgs_lintrans(x, diags, baby, giant, 32, 32)
-    want = orc.bsgs(host(x[5:6]), host(diags), [host(k) for k in baby], [host(k) for k in giant],
+    ctx.device_status()
+    want = orc.bsgs(host(x), host(diags), [host(k) for k in baby], [host(k) for k in giant],
                     32, 32, mods, 112, 8, 8)
-    assert_bits_equal(host(y[5:6]), want, "config 4 ct 5")
+    assert_bits_equal(host(y), want, "config 4, all 8 ciphertexts")
+
+
+def test_config4_dense_matrix_decrypts(orc):
+    """Config 4 as stated: a dense 1024 x 1024 matrix with entries uniform in
+    [-1, 1]/32, its 1024 diagonals encoded at scale 2^60 (pre-rotated for the
+    giant steps), 8 encryptions of slots uniform in [-1, 1], and the 62
+    Galois keys of bb = gg = 32 from the oracle's key generation.  All 8
+    outputs decrypt to M x within 1e-8 of the float64 product; ciphertexts 0
+    and 7 are bit-exact against the oracle."""
+    p = Params(112, 8, 8)
+    ctx = ctx_for(p)
+    seed = synth.config_seed(4) + 500
+    sch = Scheme(orc, p, seed)
+    bb = gg = 32
+    M = synth.uniform_real((SLOTS, SLOTS), -1 / 32, 1 / 32, seed, 1).numpy()
+    xs = [synth.uniform_real((SLOTS,), -1, 1, seed, 10 + i).numpy() for i in range(8)]
+    ct = np.stack([sch.encrypt_slots(x) for x in xs])
+    idx = np.arange(SLOTS)
+    rows = np.stack([np.roll(M[idx, (idx + bb * g + b) % SLOTS], bb * g)
+                     for g in range(gg) for b in range(bb)])
+    diags = orc.encode_ntt_many(rows, sch.q, SCALE, N).reshape(gg, bb, p.L, N)
+    baby = [sch.keygen_galois(galois_for_rotation(b)) for b in range(1, bb)]
+    giant = [sch.keygen_galois(galois_for_rotation(bb * g)) for g in range(1, gg)]
+    y = host(ctx.bsgs_lintrans(dev(ct), dev(diags), [dev(k) for k in baby],
+                               [dev(k) for k in giant], bb, gg))
+    ctx.device_status()
+    sc = sch.rescaled_scale(SCALE * SCALE, p.L)
+    for i in range(8):
+        err = np.max(np.abs(sch.decrypt_slots(y[i], sc) - M @ xs[i]))
+        assert err < 1e-8, (i, err)
+    want = orc.bsgs(ct[[0, 7]], diags, baby, giant, bb, gg, sch.mods, p.L, p.K, p.alpha)
+    assert_bits_equal(y[[0, 7]], want, "config 4 dense, ciphertexts 0 and 7")
 
 
 # ------------------------------------------------------------------ config 5
-def test_config5_boot_rotation_full_size_sampled(orc):
+def test_config5_boot_rotation_full_size(orc):
     """2100 primes, alpha = 60, 60 special primes, 4 Galois keys (5^k,
     k in {1, 2, 4, 8}), 8 ciphertexts: the GPU runs all 32 key switches with
-    one hoisted ModUp per ciphertext; the oracle recomputes ciphertext 3
-    under key 2 (g = 625)."""
+    one hoisted ModUp per ciphertext.  The oracle recomputes ciphertexts 1
+    and 6 (one in each chunk of 4 that the key inner product groups) under
+    all four keys, 8 of the 32 key switches; the integer-pipe conversion
+    then gives the same words for all 32."""
     p = Params(2100, 60, 60)
     ctx = ctx_for(p)
     seed = synth.config_seed(5)
@@ -359,11 +395,11 @@ def test_config5_boot_rotation_full_size_sampled(orc):
             for r in range(4)]
     out = ctx.rotate(ct, keys, gal)
     ctx.device_status()
-    got = host(out[2, 3])
-    want = orc.rotate(host(ct[3:4]), [host(keys[2])], np.array([gal[2]], dtype=np.uint64), mods,
+    pick = [1, 6]
+    want = orc.rotate(host(ct[pick]), [host(k) for k in keys], np.array(gal, dtype=np.uint64), mods,
                       2100, 60, 60)
-    assert_bits_equal(got, want[0, 0], "config 5 ct 3 key 2")
-    # the integer-pipe conversion gives the same words for all 32 key switches
+    assert_bits_equal(host(out[:, pick]), want, "config 5, ciphertexts 1 and 6, all keys")
+    del want
     try:
         ctx.set_conversion("integer")
         out_int = ctx.rotate(ct, keys, gal)
@@ -647,26 +683,87 @@ def test_refresh_matches_oracle(orc):
         rf.close()
 
 
-def test_extreme_residues(orc):
-    """Inputs at the ends of [0, q): all zeros, all q - 1, and q - 1
-    alternating with 0, through the NTT both ways, a key switch and a rescale
-    (the lazy butterflies and 128-bit sums see their largest operands)."""
-    p = Params(6, 2, 2)
-    ctx = ctx_for(p)
-    mods = np.array(ctx.mods, dtype=np.uint64)
-    q = mods[:p.L]
-    top = np.broadcast_to((q - 1)[:, None], (p.L, N))
+def _extremes(q):
+    """All zeros, all q - 1, and q - 1 alternating with 0, over limbs with primes q: [3][len(q)][n]."""
+    q = np.asarray(q, dtype=np.uint64)
+    top = np.broadcast_to((q - 1)[:, None], (q.size, N))
     alt = np.where(np.arange(N) % 2 == 0, top, 0).astype(np.uint64)
-    cases = [np.zeros((p.L, N), np.uint64), np.ascontiguousarray(top, dtype=np.uint64), alt]
-    x = np.stack(cases)
+    return np.stack([np.zeros((q.size, N), np.uint64), np.ascontiguousarray(top, dtype=np.uint64), alt])
+
+
+def test_extreme_residues_ntt_2100(orc):
+    """Inputs at the ends of [0, q) through the forward and inverse NTT on all
+    2100 limbs of the boot chain (the lazy butterflies see their largest
+    operands)."""
+    ctx = context(2100, 60, 60)
+    q = np.array(ctx.q, dtype=np.uint64)
+    x = _extremes(q)
     y = dev(x)
     ctx.ntt_fwd(y)
-    assert_bits_equal(host(y), orc.ntt_fwd(x, q), "ntt_fwd extremes")
+    assert_bits_equal(host(y), orc.ntt_fwd(x, q), "ntt_fwd extremes, 2100 limbs")
     ctx.ntt_inv(y)
-    assert_bits_equal(host(y), x, "ntt round trip extremes")
-    kt = np.broadcast_to((mods - 1)[None, None, :, None], (p.dnum, 2, p.L + p.K, N))
-    key = np.ascontiguousarray(kt, dtype=np.uint64)
-    assert_bits_equal(host(ctx.keyswitch(dev(x), dev(key))), orc.keyswitch(x, key, mods, p.L, p.K, p.alpha),
-                      "keyswitch extremes")
-    ct = np.stack([np.stack([c, c]) for c in cases])
-    assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, q), "rescale extremes")
+    assert_bits_equal(host(y), x, "ntt round trip extremes, 2100 limbs")
+    z = dev(x)
+    ctx.ntt_inv(z)
+    assert_bits_equal(host(z), orc.ntt_inv(x, q), "ntt_inv extremes, 2100 limbs")
+
+
+@pytest.mark.parametrize("L,K,alpha", [(6, 2, 2), (24, 8, 8), (120, 60, 60)])
+def test_extreme_residues_key_switch_stages(orc, L, K, alpha):
+    """Extreme inputs (all zeros, all q - 1, alternating) and an all-(q - 1)
+    key through ModUp, the key inner product (g = 1 and 5) and ModDown on
+    both conversion engines, where the exact 128-bit sums and the tensor
+    cores' byte planes reach their largest values; ModDown also on an
+    all-(q - 1) accumulator.  Each stage bit-exact against the oracle."""
+    p = Params(L, K, alpha)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    c = _extremes(mods[:L])
+    key = np.ascontiguousarray(np.broadcast_to((mods - 1)[None, None, :, None], (p.dnum, 2, L + K, N)),
+                               dtype=np.uint64)
+    acc_top = np.ascontiguousarray(np.broadcast_to((mods - 1)[None, None, :, None], (1, 2, L + K, N)),
+                                   dtype=np.uint64)
+    want_d = orc.modup(c, mods, L, K, alpha)
+    want_a = {g: orc.key_inner(want_d, key, g, mods, L, K, alpha) for g in (1, 5)}
+    want_m = orc.moddown(want_a[5], mods, L, K)
+    want_top = orc.moddown(acc_top, mods, L, K)
+    try:
+        for engine in ("integer", "tensor"):
+            ctx.set_conversion(engine)
+            dig = ctx.modup(dev(c))
+            assert_bits_equal(host(dig), want_d, "modup extremes (%s)" % engine)
+            for g in (1, 5):
+                acc = ctx.key_inner(dig, dev(key), g)
+                assert_bits_equal(host(acc), want_a[g], "key_inner extremes g=%d (%s)" % (g, engine))
+            assert_bits_equal(host(ctx.moddown(acc)), want_m, "moddown extremes (%s)" % engine)
+            assert_bits_equal(host(ctx.moddown(dev(acc_top))), want_top, "moddown all q-1 (%s)" % engine)
+            ctx.device_status()
+    finally:
+        ctx.set_conversion("auto")
+
+
+@pytest.mark.parametrize("lp1", [2, 112])
+def test_extreme_residues_rescale(orc, lp1):
+    ctx = context(112, 8, 8)
+    q = np.array(ctx.mods[:lp1], dtype=np.uint64)
+    x = _extremes(q)
+    ct = np.ascontiguousarray(np.stack([x, x[::-1]], axis=1))  # [3][2][lp1][n]
+    assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, q), "rescale extremes, %d limbs" % lp1)
+
+
+def test_key_inner_more_than_256_digits():
+    """260 single-prime digits (L = 260, alpha = 1): with every digit word and
+    key word at q - 1 the exact sum 260 (q - 1)^2 passes 2^128, so the kernel
+    must reduce between blocks of digits.  Each output word is the closed
+    form 260 (q - 1)^2 = 260 mod q."""
+    L, K = 260, 1
+    ctx = context(L, K, 1)
+    mods = torch.tensor(np.array(ctx.mods, dtype=np.uint64).view(np.int64), device="cuda")
+    LK = L + K
+    top = (mods - 1).view(1, 1, LK, 1)
+    digits = top.expand(1, L, LK, N).contiguous()
+    key = top.expand(L, 2, LK, N).contiguous()
+    acc = host(ctx.key_inner(digits, key, 1))
+    ctx.device_status()
+    want = np.broadcast_to((260 % np.array(ctx.mods, dtype=np.uint64))[None, None, :, None], (1, 2, LK, N))
+    assert_bits_equal(acc, want, "key inner product over 260 digits")

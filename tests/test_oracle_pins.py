@@ -254,6 +254,26 @@ def test_encoding_is_multiplicative(orc):
     assert np.max(np.abs(orc.decode(prod, mods, SCALE * SCALE) - z1 * z2)) < 1e-12
 
 
+def test_batch_encoder_matches_encode_and_decodes(orc):
+    """encode_many (one long-double matrix product) against encode() row by
+    row, within one unit per coefficient, on real and complex slots; the
+    residues of encode_ntt_many decode back to the slots; a constant row
+    gives the closed form (c scale, 0, ..., 0)."""
+    mods = orc.gen_primes(N, 2)
+    Z = np.stack([synth.uniform_real((SLOTS,), -1, 1, SEED, 60 + i).numpy() / 32 for i in range(3)])
+    Zc = Z + 1j * np.stack([synth.uniform_real((SLOTS,), -1, 1, SEED, 70 + i).numpy() for i in range(3)])
+    for rows, scale in ((Z, SCALE), (Zc, 2**40)):
+        many = orc.encode_many(rows, N, scale)
+        for i in range(rows.shape[0]):
+            assert np.max(np.abs(many[i] - orc.encode(rows[i], N, scale))) <= 1
+    nt = orc.encode_ntt_many(Zc, mods, 2**40, N)
+    for i in range(Zc.shape[0]):
+        back = orc.decode(orc.ntt_inv(nt[i], mods), mods, 2**40)
+        assert np.max(np.abs(back - Zc[i])) < 1e-9
+    const = orc.encode_many(np.full((1, SLOTS), 0.25), N, SCALE)[0]
+    assert int(const[0]) == SCALE // 4 and np.all(const[1:] == 0)
+
+
 # ------------------------------------------------------------------ basis conversion
 def test_basis_conversion_crt_identity(orc):
     mods = [int(x) for x in orc.gen_primes(N, 8)]

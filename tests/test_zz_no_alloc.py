@@ -46,6 +46,21 @@ def test_modup_noalloc_matches_modup_twice(L, K, alpha, batch):
         assert rc == 0, lib.ckks_last_error()
         torch.cuda.synchronize()
         assert torch.equal(out, ref), "call %d differs from ckks_modup" % call
+    ctx.device_status()
+    # with the address resolved, calls of the entry point alone leave the
+    # device's free memory as it was
+    del ws
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(2):
+        rc = lib.ckks_modup_noalloc(ctx._h, C.c_void_p(c.data_ptr()), C.c_void_p(out.data_ptr()),
+                                    batch, stream)
+        assert rc == 0, lib.ckks_last_error()
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before
+    assert torch.equal(out, ref)
+    ctx.device_status()
 
 
 def test_modup_noalloc_rejects_oversized_batch():
