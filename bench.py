@@ -56,6 +56,8 @@ def parse():
                     help="ciphertexts per key-switch workload (8 = the configs; smaller only for profiling)")
     ap.add_argument("--ks-keys", type=int, default=4,
                     help="Galois keys of the boot-level rotation (4 = the config; smaller only for profiling)")
+    ap.add_argument("--ks-entries", default=",".join(KS_ENTRIES),
+                    help="key-switching workloads to build and time (with --ks-only: only these)")
     ap.add_argument("--sweep", default=",".join(str(x) for x in SWEEP),
                     help="limb counts of the step (a smaller case for profiling only)")
     return ap.parse_args()
@@ -206,11 +208,13 @@ def traffic_for(kernel_key):
 
 def intpipe_peaks(ctx):
     """Same-run microbenchmarks over the whole GPU: Shoup multiplies/s,
-    64x64->128 MACs/s and 64-bit high multiplies/s on the integer pipes, and
-    int8 tcgen05.mma ops/s at N = 256 (dense rate) and N = 32 (the basis
-    conversion's tile), one issuing thread per SM."""
+    64x64->128 MACs/s and 64-bit high multiplies/s on the integer pipes, the
+    forward NTT's own butterfly (kind 5), and int8 tcgen05.mma ops/s at
+    N = 256 (dense rate) and N = 32 (the basis conversion's tile), one
+    issuing thread per SM."""
     out = {}
-    for kind, name in ((0, "shoup_mulmod_per_s"), (1, "mac128_per_s"), (2, "mulhi64_per_s")):
+    for kind, name in ((0, "shoup_mulmod_per_s"), (1, "mac128_per_s"), (2, "mulhi64_per_s"),
+                       (5, "ntt_butterfly_per_s")):
         best = 0.0
         for _ in range(3):
             ms, ops = ctx.bench_intpipe(kind, 148 * 8, 2048)
@@ -223,6 +227,40 @@ def intpipe_peaks(ctx):
             best = max(best, ops / (ms * 1e-3))
         out[name] = best
     return out
+
+
+def rates_from(ipeak):
+    """Per-operation rates of the roofline model (operations per second)."""
+    return {"bfly": ipeak["ntt_butterfly_per_s"], "mm": ipeak["shoup_mulmod_per_s"],
+            "mac": ipeak["mac128_per_s"], "int8_mac": ipeak["int8_mma_n256_ops_per_s"] / 2}
+
+
+def ntt_roofline(limbs, k_ms, hbm_peak, peak_src, ipeak):
+    """Roofline object of one forward-NTT launch over BATCH x limbs: the
+    slower of its bytes at the measured HBM copy rate and its butterflies at
+    the same-run rate of the kernel's own butterfly (microbenchmark kind 5).
+    The generic Shoup rate (kind 0) is reported beside it."""
+    bytes_, mm = ntt_launch_work(limbs)
+    t = k_ms * 1e-3
+    t_hbm = bytes_ / (hbm_peak * 1e9)
+    t_alu = mm / ipeak["ntt_butterfly_per_s"]
+    if t_alu > t_hbm:
+        roof = {"bound": "alu", "achieved": mm / t / 1e9, "peak": ipeak["ntt_butterfly_per_s"] / 1e9,
+                "unit": "G butterflies/s",
+                "peak_source": "same-run microbenchmark of the kernel's own butterfly (kind 5)"}
+    else:
+        roof = {"bound": "hbm", "achieved": bytes_ / t / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "peak_source": "%s MEASURED_PEAKS.json hbm_gbs" % peak_src}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for("ntt_fwd_%d" % limbs)
+    roof["kernel"] = "ntt_fwd_kernel<BatchJob> (%d x %d limbs)" % (BATCH, limbs)
+    roof["launch_ms"] = k_ms
+    roof["algorithmic_bytes"] = bytes_
+    roof["butterflies"] = mm
+    roof["hbm_frac_of_%s" % peak_src] = (bytes_ / t / 1e9) / hbm_peak
+    roof["alu_frac_of_butterfly_microbench"] = (mm / t) / ipeak["ntt_butterfly_per_s"]
+    roof["alu_frac_of_generic_shoup_microbench"] = (mm / t) / ipeak["shoup_mulmod_per_s"]
+    return roof
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -284,22 +322,7 @@ def run_b200(args):
     value = weak_scaling_value(per_step, args.steps, world, total_ms)
 
     # roofline of the dominant kernel: forward NTT on the largest sweep entry
-    bytes_, mm = ntt_launch_work(SWEEP[-1])
-    t = k_ms * 1e-3
-    t_hbm = bytes_ / (hbm_peak * 1e9)
-    t_alu = mm / ipeak["shoup_mulmod_per_s"]
-    if t_alu > t_hbm:
-        roof = {"bound": "alu", "achieved": mm / t / 1e9, "peak": ipeak["shoup_mulmod_per_s"] / 1e9,
-                "unit": "G Shoup-mulmod/s", "peak_source": "same-run microbenchmark (kind 0)"}
-    else:
-        roof = {"bound": "hbm", "achieved": bytes_ / t / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                "peak_source": "%s MEASURED_PEAKS.json hbm_gbs" % peak_src}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for("ntt_fwd_%d" % SWEEP[-1])
-    roof["kernel"] = "ntt_fwd_kernel<BatchJob> (16 x %d limbs)" % SWEEP[-1]
-    roof["launch_ms"] = k_ms
-    roof["hbm_frac_of_measured"] = (bytes_ / t / 1e9) / hbm_peak
-    roof["alu_frac_of_microbench"] = (mm / t) / ipeak["shoup_mulmod_per_s"]
+    roof = ntt_roofline(SWEEP[-1], k_ms, hbm_peak, peak_src, ipeak)
 
     line = {
         "metric": METRIC, "value": value, "unit": "limb-NTTs/s", "n_gpus": world,
@@ -324,7 +347,8 @@ def run_b200(args):
     if not args.no_ks and rank == 0 and world == 1:
         del xs, refs
         torch.cuda.empty_cache()
-        line["keyswitch"] = run_keyswitch(dev, hbm_peak, ipeak)
+        line["keyswitch"] = run_keyswitch(dev, hbm_peak, ipeak,
+                                          entries=tuple(e for e in args.ks_entries.split(",") if e))
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
@@ -384,187 +408,252 @@ def run_e2e(ctx, xs, refs, args, dev, stream, pg, world):
             "roundtrip_identity": ok, "pipelining": "chunks of 2 polynomials on 3 streams"}
 
 
-def _time_call(fn, reps, stream):
+def _time_call(fn, reps, stream, dev=None):
+    """Mean device milliseconds of fn() over `reps` calls after 2 warm-up
+    calls (CUDA events on the launching stream), and the clocks sampled while
+    the timed calls ran."""
     import torch
     for _ in range(2):
         fn()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(reps):
-        fn()
-    b.record(stream)
-    torch.cuda.synchronize()
-    return a.elapsed_time(b) / reps
+    with ClockSampler(dev if dev is not None else torch.device("cuda", torch.cuda.current_device())) as clk:
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps, clk.summary()
 
 
-def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4):
-    """Key switches per second of the three key-switching workloads (B ciphertexts each; the
-    boot-level rotation with R Galois keys)."""
+KS_ENTRIES = ("tiny", "boot_rotation", "boot_rotation_integer", "layer", "bsgs", "refresh")
+
+
+def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_batch=8):
+    """Key switches per second of the key-switching workloads (B ciphertexts
+    each; the boot-level rotation with R Galois keys), each with its roofline
+    fraction and the clocks sampled while it ran.  `entries` selects which
+    workloads are built at all (a smaller set for profiling)."""
     import torch
 
     from rns_ckks_polynomial_b200 import Context, primes, synth
     stream = torch.cuda.current_stream(dev)
-    mm_peak, mac_peak = ipeak["shoup_mulmod_per_s"], ipeak["mac128_per_s"]
+    rates = rates_from(ipeak)
     out = {}
-    # tiny pipeline: 4 + 1 primes, alpha = 1; 8 polynomials -> NTT -> pairwise product -> INTT, and
-    # one rotation key switch of (P0, P1) with the Galois-5 key
-    seed = synth.config_seed(1)
-    m1 = primes(5)
-    ctx = Context(m1[:4], m1[4:], 1, device=dev.index)
-    polys = synth.uniform_residues((8, 4, N), m1[:4], seed, 1, device=dev)
-    key = synth.uniform_residues((4, 2, 5, N), m1, seed, 2, device=dev)
-    x = polys.clone()
-    prod = torch.empty((4, 4, N), dtype=torch.int64, device=dev)
-    rot = torch.empty((1, 1, 2, 4, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(4, 1, 1), dtype=torch.uint8, device=dev)
+    if "tiny" in entries:
+        # 4 + 1 primes, alpha = 1; 8 polynomials -> NTT -> pairwise product -> INTT, and one
+        # rotation key switch of (P0, P1) with the Galois-5 key
+        seed = synth.config_seed(1)
+        m1 = primes(5)
+        ctx = Context(m1[:4], m1[4:], 1, device=dev.index)
+        polys = synth.uniform_residues((8, 4, N), m1[:4], seed, 1, device=dev)
+        key = synth.uniform_residues((4, 2, 5, N), m1, seed, 2, device=dev)
+        x = polys.clone()
+        prod = torch.empty((4, 4, N), dtype=torch.int64, device=dev)
+        rot = torch.empty((1, 1, 2, 4, N), dtype=torch.int64, device=dev)
+        ws = torch.empty(ctx.workspace_bytes(4, 1, 1), dtype=torch.uint8, device=dev)
 
-    def tiny():
-        x.copy_(polys)
-        ctx.ntt_fwd(x)
-        ctx.pointwise("mul", x[0::2].contiguous(), x[1::2].contiguous(), out=prod)
-        ctx.ntt_inv(prod)
-        ctx.rotate(x[0:2].reshape(1, 2, 4, N), [key], [5], out=rot, ws=ws)
+        def tiny():
+            x.copy_(polys)
+            ctx.ntt_fwd(x)
+            ctx.pointwise("mul", x[0::2].contiguous(), x[1::2].contiguous(), out=prod)
+            ctx.ntt_inv(prod)
+            ctx.rotate(x[0:2].reshape(1, 2, 4, N), [key], [5], out=rot, ws=ws)
 
-    ms = _time_call(tiny, 50, stream)
-    ntt = (N // 2) * 11
-    up, inner, down = ks_work_keyswitch_parts(4, 1, 1)
-    mm = (8 + 4) * 4 * ntt + 4 * 4 * N + up["mm"] + down["mm"]
-    mac = up["mac"] + inner["mac"] + down["mac"]
-    io = (8 * 4 + 4 * 4 + 2 * 4) * N * 8 + 4 * 2 * 5 * N * 8
-    out["tiny_pipeline_L4"] = ks_entry(1, ms, (mm, mac, io), hbm_peak, mm_peak, mac_peak)
-    out["tiny_pipeline_L4"]["note"] = ("one call: 8 limb-4 NTTs, 4 products, 4 INTTs and one rotation; "
-                                       "launch-bound at this size")
-    ctx.device_status()
-    del ctx, polys, key, x, prod, rot, ws
-    # boot-level hoisted rotation: L = 2100, K = 60, alpha = 60, 4 keys, 8 cts
-    seed = synth.config_seed(5)
-    mods = primes(2160)
-    ctx = Context(mods[:2100], mods[2100:], 60, device=dev.index)
-    ct = synth.uniform_residues((B, 2, 2100, N), mods[:2100], seed, 1, device=dev)
-    keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device=dev) for r in range(R)]
-    gal = [5, 25, 625, 1505][:R]
-    res = torch.empty((R, B, 2, 2100, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(4, B, R), dtype=torch.uint8, device=dev)
-    ms = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 3, stream)
-    up, _, down = ks_work_keyswitch_parts(2100, 60, 60)
-    conv = B * (up["mac"] + R * down["mac"])
-    out["boot_rotation_L2100"] = ks_entry(B * R, ms, ks_work_rotation(2100, 60, 60, B, R), hbm_peak,
-                                          mm_peak, mac_peak, conv_macs=conv,
-                                          int8_peak=int8_mac_peak(ipeak))
-    ctx.device_status()
-    # the same call with both conversions on the integer pipes (bit-identical output)
-    ctx.set_conversion("integer")
-    ms = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 2, stream)
-    out["boot_rotation_L2100_integer_pipes"] = ks_entry(B * R, ms, ks_work_rotation(2100, 60, 60, B, R),
-                                                        hbm_peak, mm_peak, mac_peak)
-    ctx.set_conversion("auto")
-    ctx.device_status()
-    del ct, keys, res, ws, ctx
-    torch.cuda.empty_cache()
-    # layer ct x ct multiply: L = 112, K = 8, alpha = 8, 8 pairs
-    seed = synth.config_seed(3)
-    mods = primes(120)
-    ctx = Context(mods[:112], mods[112:], 8, device=dev.index)
-    a = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
-    b = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 2, device=dev)
-    rlk = synth.uniform_residues((14, 2, 120, N), mods, seed, 3, device=dev)
-    res = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
-    ms = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 10, stream)
-    up, _, down = ks_work_keyswitch_parts(112, 8, 8)
-    out["layer_mul_relin_L112"] = ks_entry(B, ms, ks_work_mrr(112, 8, 8, B), hbm_peak, mm_peak, mac_peak,
-                                           conv_macs=B * (up["mac"] + down["mac"]),
-                                           int8_peak=int8_mac_peak(ipeak))
-    # BSGS: bb = gg = 32, 62 keys, 8 cts
-    seed = synth.config_seed(4)
-    x = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
-    diags = synth.uniform_residues((32, 32, 112, N), mods[:112], seed, 2, device=dev)
-    bk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 100 + i, device=dev) for i in range(31)]
-    gk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 200 + i, device=dev) for i in range(31)]
-    y = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
-    ws = torch.empty(ctx.workspace_bytes(7, B, 32032), dtype=torch.uint8, device=dev)
-    ms = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 3, stream)
-    out["bsgs_L112_32x32"] = ks_entry(B * 62, ms, ks_work_bsgs(112, 8, 8, B, 32, 32), hbm_peak,
-                                      mm_peak, mac_peak,
-                                      conv_macs=B * (up["mac"] + 31 * down["mac"] + 31 * (up["mac"] + down["mac"])),
-                                      int8_peak=int8_mac_peak(ipeak))
+        ms, clk = _time_call(tiny, 50, stream, dev)
+        w = work_sum(work(bfly=(8 + 4) * 4 * NTT_BFLY, mm=4 * 4 * N + 4 * 4 * N),
+                     work_rotation(4, 1, 1, 1, 1))
+        w["bytes"] = (8 * 4 + 4 * 4 + 2 * 4) * N * 8 + 4 * 2 * 5 * N * 8
+        out["tiny_pipeline_L4"] = ks_entry(1, ms, w, hbm_peak, rates, clk)
+        out["tiny_pipeline_L4"]["note"] = ("one call: 8 limb-4 NTTs, 4 products, 4 INTTs and one rotation; "
+                                           "launch-bound at this size")
+        ctx.device_status()
+        del ctx, polys, key, x, prod, rot, ws
+    if "boot_rotation" in entries or "boot_rotation_integer" in entries:
+        # boot-level hoisted rotation: L = 2100, K = 60, alpha = 60, R keys, B cts
+        seed = synth.config_seed(5)
+        mods = primes(2160)
+        ctx = Context(mods[:2100], mods[2100:], 60, device=dev.index)
+        ct = synth.uniform_residues((B, 2, 2100, N), mods[:2100], seed, 1, device=dev)
+        keys = [synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + r, device=dev) for r in range(R)]
+        gal = [5, 25, 625, 1505][:R]
+        res = torch.empty((R, B, 2, 2100, N), dtype=torch.int64, device=dev)
+        ws = torch.empty(ctx.workspace_bytes(4, B, R), dtype=torch.uint8, device=dev)
+        if "boot_rotation" in entries:
+            ms, clk = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 10, stream, dev)
+            out["boot_rotation_L2100"] = ks_entry(B * R, ms, work_rotation(2100, 60, 60, B, R), hbm_peak,
+                                                  rates, clk)
+            ctx.device_status()
+        if "boot_rotation_integer" in entries:
+            # the same call with both conversions on the integer pipes (bit-identical output)
+            ctx.set_conversion("integer")
+            ms, clk = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 10, stream, dev)
+            out["boot_rotation_L2100_integer_pipes"] = ks_entry(
+                B * R, ms, work_rotation(2100, 60, 60, B, R, engine="integer"), hbm_peak, rates, clk)
+            ctx.set_conversion("auto")
+            ctx.device_status()
+        del ct, keys, res, ws, ctx
+        torch.cuda.empty_cache()
+    if "layer" in entries or "bsgs" in entries:
+        mods = primes(120)
+        ctx = Context(mods[:112], mods[112:], 8, device=dev.index)
+    if "layer" in entries:
+        # layer ct x ct multiply: L = 112, K = 8, alpha = 8, B pairs
+        seed = synth.config_seed(3)
+        a = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
+        b = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 2, device=dev)
+        rlk = synth.uniform_residues((14, 2, 120, N), mods, seed, 3, device=dev)
+        res = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
+        ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
+        ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
+        out["layer_mul_relin_L112"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
+        del a, b, rlk, res, ws
+    if "bsgs" in entries:
+        # BSGS: bb = gg = 32, 62 keys, B cts
+        seed = synth.config_seed(4)
+        x = synth.uniform_residues((B, 2, 112, N), mods[:112], seed, 1, device=dev)
+        diags = synth.uniform_residues((32, 32, 112, N), mods[:112], seed, 2, device=dev)
+        bk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 100 + i, device=dev) for i in range(31)]
+        gk = [synth.uniform_residues((14, 2, 120, N), mods, seed, 200 + i, device=dev) for i in range(31)]
+        y = torch.empty((B, 2, 111, N), dtype=torch.int64, device=dev)
+        ws = torch.empty(ctx.workspace_bytes(7, B, 32032), dtype=torch.uint8, device=dev)
+        ms, clk = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 10, stream, dev)
+        out["bsgs_L112_32x32"] = ks_entry(B * 62, ms, work_bsgs(112, 8, 8, B, 32, 32), hbm_peak, rates, clk)
+        del x, diags, bk, gk, y, ws
+    if "layer" in entries or "bsgs" in entries:
+        ctx.device_status()
+        del ctx
+        torch.cuda.empty_cache()
+    if "refresh" in entries:
+        try:
+            out["refresh_L2100"] = run_refresh(dev, hbm_peak, rates, B=refresh_batch)
+        except Exception as e:  # noqa: BLE001 - reported in the line, the other entries stand
+            out["refresh_L2100"] = {"error": repr(e)[:400]}
+        torch.cuda.empty_cache()
     return out
 
 
-def ks_work_keyswitch_parts(L, K, alpha):
-    """(MM, MAC) of the parts of one key switch, hybrid method, n = 2048."""
+# ---------------------------------------------------------------- algorithmic work model
+NTT_BFLY = (N // 2) * 11  # butterflies per limb transform, one modular product each
+TC_MIN_SOURCES = 8        # conversions with this many source primes run on the int8 tensor cores
+
+
+def work(bfly=0, mm=0, mac=0, conv_tc=0, bytes=0):
+    """Algorithmic work: NTT butterflies, other modular products, 64x64->128
+    multiply-adds (mac) of which conv_tc run as basis conversions on the int8
+    tensor cores, and the minimum bytes that cross HBM."""
+    return {"bfly": bfly, "mm": mm, "mac": mac, "conv_tc": conv_tc, "bytes": bytes}
+
+
+def work_sum(*parts, times=1):
+    out = work()
+    for p in parts:
+        for k in out:
+            out[k] += p[k] * times
+    return out
+
+
+def ks_work_keyswitch_parts(L, K, alpha, engine="auto"):
+    """Work of the parts of one hybrid key switch at n = 2048 (ModUp of one
+    polynomial, the key inner product, ModDown of the two components)."""
     dnum = (L + alpha - 1) // alpha
     LK = L + K
-    ntt = (N // 2) * 11
     new_limbs = dnum * LK - L
-    modup = {"mm": L * ntt + L * N + new_limbs * ntt, "mac": sum(
-        min(alpha, L - j * alpha) * (LK - min(alpha, L - j * alpha)) for j in range(dnum)) * N}
-    inner = {"mm": 0, "mac": 2 * dnum * LK * N}
-    moddown = {"mm": 2 * (K * ntt + K * N + L * ntt + L * N), "mac": 2 * K * L * N}
+    tc = engine != "integer"
+    conv_up = conv_up_tc = 0
+    for j in range(dnum):
+        S = min(alpha, L - j * alpha)
+        conv_up += S * (LK - S) * N
+        if tc and S >= TC_MIN_SOURCES:
+            conv_up_tc += S * (LK - S) * N
+    conv_dn = 2 * K * L * N
+    modup = work(bfly=(L + new_limbs) * NTT_BFLY, mm=L * N, mac=conv_up, conv_tc=conv_up_tc)
+    inner = work(mac=2 * dnum * LK * N)
+    moddown = work(bfly=2 * (K + L) * NTT_BFLY, mm=2 * (K + L) * N, mac=conv_dn,
+                   conv_tc=conv_dn if tc and K >= TC_MIN_SOURCES else 0)
     return modup, inner, moddown
 
 
-def ks_work_rotation(L, K, alpha, B, nkeys):
-    up, inner, down = ks_work_keyswitch_parts(L, K, alpha)
-    mm = B * (up["mm"] + nkeys * (inner["mm"] + down["mm"]))
-    mac = B * (up["mac"] + nkeys * (inner["mac"] + down["mac"]))
+def work_rescale(l, B):
+    """Rescale of B ciphertexts from l primes: INTT of the dropped limb, NTT of
+    the l - 1 kept ones with the subtraction and q_l^-1 in the store."""
+    return work(bfly=B * 2 * l * NTT_BFLY, mm=B * 2 * (l - 1) * N,
+                bytes=B * 2 * (2 * l - 1) * N * 8)
+
+
+def work_rotation(L, K, alpha, B, nkeys, engine="auto"):
+    up, inner, down = ks_work_keyswitch_parts(L, K, alpha, engine)
+    w = work_sum(work_sum(up, times=B), work_sum(inner, down, times=B * nkeys))
     dnum = (L + alpha - 1) // alpha
-    keyb = nkeys * dnum * 2 * (L + K) * N * 8
-    io = B * 2 * L * N * 8 * (1 + nkeys)
-    return mm, mac, keyb + io
+    w["bytes"] = nkeys * dnum * 2 * (L + K) * N * 8 + B * 2 * L * N * 8 * (1 + nkeys)
+    return w
 
 
-def ks_work_mrr(L, K, alpha, B):
+def work_mrr(L, K, alpha, B):
     up, inner, down = ks_work_keyswitch_parts(L, K, alpha)
-    ntt = (N // 2) * 11
-    mm = B * (up["mm"] + down["mm"] + 4 * L * N + 2 * (ntt + (L - 1) * (ntt + N)))
-    mac = B * (up["mac"] + inner["mac"] + down["mac"])
+    w = work_sum(up, inner, down, times=B)
+    w = work_sum(w, work(mm=B * 4 * L * N), work_rescale(L, B))
     dnum = (L + alpha - 1) // alpha
-    keyb = dnum * 2 * (L + K) * N * 8
-    io = B * (4 * L + 2 * (L - 1)) * N * 8
-    return mm, mac, keyb + io
+    w["bytes"] = dnum * 2 * (L + K) * N * 8 + B * (4 * L + 2 * (L - 1)) * N * 8
+    return w
 
 
-def ks_work_bsgs(L, K, alpha, B, bb, gg):
-    up, inner, down = ks_work_keyswitch_parts(L, K, alpha)
-    ntt = (N // 2) * 11
-    baby = up["mm"] + (bb - 1) * down["mm"], up["mac"] + (bb - 1) * (inner["mac"] + down["mac"])
-    giant = (gg - 1) * (up["mm"] + down["mm"]), (gg - 1) * (up["mac"] + inner["mac"] + down["mac"])
-    pt = 0, gg * bb * 2 * L * N
-    resc = 2 * (ntt + (L - 1) * (ntt + N)), 0
-    mm = B * (baby[0] + giant[0] + pt[0] + resc[0])
-    mac = B * (baby[1] + giant[1] + pt[1] + resc[1])
-    dnum = (L + alpha - 1) // alpha
-    keyb = (bb - 1 + gg - 1) * dnum * 2 * (L + K) * N * 8
-    io = gg * bb * L * N * 8 + B * (2 * L + 2 * (L - 1)) * N * 8
-    return mm, mac, keyb + io
+def work_bsgs_plan(l, K, alpha, B, bb, gg, rotated_giants):
+    """BSGS over bb x gg plaintext diagonals at l primes: one hoisted ModUp and
+    bb - 1 baby key switches, the inner sums (one multiply-add per diagonal
+    word and ciphertext component), `rotated_giants` full key switches and a
+    rescale."""
+    up, inner, down = ks_work_keyswitch_parts(l, K, alpha)
+    w = work()
+    if bb > 1:
+        w = work_sum(w, up, work_sum(inner, down, times=bb - 1))
+    w = work_sum(w, work_sum(up, inner, down, times=rotated_giants))
+    w = work_sum(work_sum(w, times=B), work(mac=B * gg * bb * 2 * l * N), work_rescale(l, B))
+    dnum = (l + alpha - 1) // alpha
+    w["bytes"] = ((bb - 1 + rotated_giants) * dnum * 2 * (l + K) * N * 8 + gg * bb * l * N * 8
+                  + B * (2 * l + 2 * (l - 1)) * N * 8)
+    return w
 
 
-def int8_mac_peak(ipeak):
-    """Dense int8 MAC/s: the same-run tcgen05 int8 rate at N = 256."""
-    return ipeak["int8_mma_n256_ops_per_s"] / 2
+def work_bsgs(L, K, alpha, B, bb, gg):
+    return work_bsgs_plan(L, K, alpha, B, bb, gg, gg - 1)
 
 
-def ks_entry(nks, ms, work, hbm_peak, mm_peak, mac_peak, conv_macs=0, int8_peak=None):
-    """roofline_frac follows the problem statement: modular multiplies and 64-bit MACs at the
-    same-run integer-pipe peaks, bytes at the HBM peak.  When the basis conversion runs on the
-    int8 tensor cores (8 or more source primes) that model can be exceeded; tensor_model_frac then
-    charges the conversion's int8 byte-plane products (64 per 60-bit MAC, sources padded to 64)
-    at the same-run int8 tensor-core peak (`int8_peak`, MAC/s) instead."""
-    mm, mac, bytes_ = work
+def model_seconds(w, rates, hbm_peak, engine_tc=True):
+    """(ALU seconds, HBM seconds) of a work dict.  With engine_tc the
+    conversions counted in conv_tc are charged as 64 int8 byte-plane
+    multiply-adds per 60-bit multiply-add at the same-run dense int8 rate;
+    otherwise every multiply-add is charged at the 128-bit MAC rate."""
+    t = w["bfly"] / rates["bfly"] + w["mm"] / rates["mm"]
+    if engine_tc:
+        t += (w["mac"] - w["conv_tc"]) / rates["mac"] + w["conv_tc"] * 64 / rates["int8_mac"]
+    else:
+        t += w["mac"] / rates["mac"]
+    return t, w["bytes"] / (hbm_peak * 1e9)
+
+
+def ks_entry(nks, ms, w, hbm_peak, rates, clocks=None):
+    """One key-switching workload: rate, and roofline_frac = (the slower of
+    its bytes at the measured HBM rate and its operations at the same-run
+    rates of the engines that actually ran) / measured time.  NTT butterflies
+    are charged at the kernel's own butterfly rate, other modular products at
+    the Shoup rate, multiply-adds at the 128-bit MAC rate, and conversions on
+    the tensor cores at the dense int8 rate.  integer_pipe_model_frac charges
+    every multiply-add to the integer pipes instead: a model the tensor-core
+    path can exceed, so it is reported, not used as the bound."""
     t = ms * 1e-3
-    t_alu = mm / mm_peak + mac / mac_peak
-    t_hbm = bytes_ / (hbm_peak * 1e9)
+    t_alu, t_hbm = model_seconds(w, rates, hbm_peak, engine_tc=True)
     bound = "alu" if t_alu >= t_hbm else "hbm"
     out = {"keyswitches_per_s": nks / t, "ms_per_call": ms, "keyswitches_per_call": nks,
-           "mulmods": mm, "macs": mac, "min_bytes": bytes_, "bound": bound,
-           "roofline_frac": max(t_alu, t_hbm) / t,
+           "butterflies": w["bfly"], "mulmods": w["mm"], "macs": w["mac"], "macs_on_tensor_cores": w["conv_tc"],
+           "min_bytes": w["bytes"], "bound": bound, "roofline_frac": max(t_alu, t_hbm) / t,
            "alu_frac": t_alu / t, "hbm_frac": t_hbm / t,
-           "conversion": "int8 tensor cores" if int8_peak else "integer pipes"}
-    if int8_peak:
-        t_tc = mm / mm_peak + (mac - conv_macs) / mac_peak + conv_macs * 64 * 64 / 60 / int8_peak
-        out["tensor_model_frac"] = max(t_tc, t_hbm) / t
+           "conversion": "int8 tensor cores" if w["conv_tc"] else "integer pipes"}
+    if w["conv_tc"]:
+        t_int, _ = model_seconds(w, rates, hbm_peak, engine_tc=False)
+        out["integer_pipe_model_frac"] = max(t_int, t_hbm) / t
+    if clocks is not None:
+        out["clocks"] = clocks
     return out
 
 
@@ -582,9 +671,10 @@ def cpu_model():
 def cpu_baseline(min_seconds=10.0):
     """The oracle as it stands, timed on this host's cores on bounded samples.
 
-    - value: the sweep's 112-limb entry (16 polynomials) forward + inverse on
-      all cores, repeated until at least `min_seconds` have elapsed;
-    - single_thread: the same on one thread (one polynomial, >= 3 s);
+    - value: the bench step itself (16 polynomials at each of the sweep's limb
+      counts, forward + inverse) on all cores, repeated until at least
+      `min_seconds` have elapsed;
+    - single_thread: one polynomial of each limb count on one thread (>= 3 s);
     - keyswitch: the key-switching workloads on all cores, each on a subset
       scaled linearly to the GPU workload: the boot-level rotation from one
       ciphertext's hoisted ModUp and one key's inner product + ModDown (then
@@ -594,36 +684,41 @@ def cpu_baseline(min_seconds=10.0):
 
     import oracle
     from rns_ckks_polynomial_b200 import synth
-    mods = oracle.gen_primes(N, 112)
-    a = synth.uniform_residues((BATCH, 112, N), mods, synth.config_seed(2), 112).numpy()
-    a = a.astype(np.uint64)
+    mods = oracle.gen_primes(N, max(SWEEP))
+    xs = [synth.uniform_residues((BATCH, l, N), mods[:l], synth.config_seed(2), l).numpy().astype(np.uint64)
+          for l in SWEEP]
     reps, t0 = 0, time.perf_counter()
     while True:
-        y = oracle.ntt_fwd(a, mods)
-        oracle.ntt_inv(y, mods)
+        for x in xs:
+            oracle.ntt_inv(oracle.ntt_fwd(x, mods[:x.shape[1]]), mods[:x.shape[1]])
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds:
             break
     cores = oracle.num_threads()
-    out = {"value": reps * 2 * BATCH * 112 / el, "unit": "limb-NTTs/s", "cores": cores, "kind": "oracle",
-           "sample": "%d repetitions of 16 x 112-limb NTT + INTT (%.1f s)" % (reps, el),
+    per_step = 2 * BATCH * sum(SWEEP)
+    out = {"value": reps * per_step / el, "unit": "limb-NTTs/s", "cores": cores, "kind": "oracle",
+           "sample": "%d repetitions of the bench step, 16 x {%s}-limb NTT + INTT (%.1f s)" % (
+               reps, ", ".join(str(l) for l in SWEEP), el),
            "cpu_model": cpu_model()}
     # one thread
     oracle.set_num_threads(1)
     try:
-        a1 = np.ascontiguousarray(a[:1])
+        x1 = [np.ascontiguousarray(x[:1]) for x in xs]
         reps, t0 = 0, time.perf_counter()
         while True:
-            oracle.ntt_inv(oracle.ntt_fwd(a1, mods), mods)
+            for x in x1:
+                oracle.ntt_inv(oracle.ntt_fwd(x, mods[:x.shape[1]]), mods[:x.shape[1]])
             reps += 1
             el = time.perf_counter() - t0
             if el >= 3.0:
                 break
     finally:
         oracle.set_num_threads(cores)
-    out["single_thread"] = {"value": reps * 2 * 112 / el, "unit": "limb-NTTs/s", "cores": 1,
-                            "sample": "%d repetitions of 1 x 112-limb NTT + INTT (%.1f s)" % (reps, el)}
+    out["single_thread"] = {"value": reps * 2 * sum(SWEEP) / el, "unit": "limb-NTTs/s", "cores": 1,
+                            "sample": "%d repetitions of 1 x {%s}-limb NTT + INTT (%.1f s)" % (
+                                reps, ", ".join(str(l) for l in SWEEP), el)}
+    del xs, x1
     ks = {}
     # boot-level rotation: L = 2100, K = 60, alpha = 60; one ciphertext's hoisted ModUp and one
     # key's inner product + ModDown, scaled to 8 ModUps + 32 key switches
@@ -672,8 +767,9 @@ def cpu_baseline(min_seconds=10.0):
 
 
 def run_reference(args):
-    """The CPU oracle as it stands, on the same workload, metric and unit;
-    each step a bounded sample of the sweep (16 x 112-limb NTT + INTT)."""
+    """The CPU oracle as it stands, on the same workload, metric and unit:
+    every step is the bench step itself (16 polynomials at each of the
+    sweep's limb counts, forward NTT then inverse), on the host's cores."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -681,20 +777,24 @@ def run_reference(args):
 
     import oracle
     from rns_ckks_polynomial_b200 import synth
-    mods = oracle.gen_primes(N, 112)
-    a = synth.uniform_residues((BATCH, 112, N), mods, synth.config_seed(2), 112).numpy()
-    a = a.astype(np.uint64)
+    mods = oracle.gen_primes(N, max(SWEEP))
+    xs = [synth.uniform_residues((BATCH, l, N), mods[:l], synth.config_seed(2), l).numpy().astype(np.uint64)
+          for l in SWEEP]
+
+    def step():
+        for x in xs:
+            oracle.ntt_inv(oracle.ntt_fwd(x, mods[:x.shape[1]]), mods[:x.shape[1]])
+
     for _ in range(args.warmup):
-        oracle.ntt_inv(oracle.ntt_fwd(a, mods), mods)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        y = oracle.ntt_fwd(a, mods)
-        oracle.ntt_inv(y, mods)
+        step()
     el = time.perf_counter() - t0
-    per_step = 2 * BATCH * 112
+    per_step = 2 * BATCH * sum(SWEEP)
     value = per_step * args.steps / el
     cores = oracle.num_threads()
-    sample = "16 x 112-limb NTT + INTT per step (the sweep's 112-limb entry)"
+    sample = "the whole bench step per step: 16 x {%s}-limb NTT + INTT" % ", ".join(str(l) for l in SWEEP)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "limb-NTTs/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -703,19 +803,21 @@ def run_reference(args):
         "config": {"workload": WORKLOAD, "n": N, "batch_per_gpu": BATCH, "limbs": list(SWEEP),
                    "sample": sample},
         "cpu_baseline": {"value": value, "unit": "limb-NTTs/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "limb-NTTs/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
-def run_refresh(dev, B=8, L=2100, K=60, alpha=60, depth=3, r=9, reps=2):
+def run_refresh(dev, hbm_peak, rates, B=8, L=2100, K=60, alpha=60, depth=3, r=9, reps=3):
     """The bootstrapping refresh of B ciphertexts on the boot chain (2100 + 60
     primes): modraise from q_0, `depth`-level factored coeff_to_slot and
     slot_to_coeff, conj_extract, two sin_folds of 6 + r levels, restore_merge.
-    Keys and plaintext diagonals are seeded uniform residues: the kernels'
-    time does not depend on the values (the parity test runs the same schedule
-    on the oracle's keys)."""
+    Each step is timed with CUDA events between its calls; coeff_to_slot and
+    slot_to_coeff also get key switches/s and a roofline fraction.  Keys and
+    plaintext diagonals are seeded uniform residues: the kernels' time does
+    not depend on the values (the parity test runs the same schedule on the
+    oracle's keys)."""
     import torch
 
     from rns_ckks_polynomial_b200 import primes, synth
@@ -736,46 +838,87 @@ def run_refresh(dev, B=8, L=2100, K=60, alpha=60, depth=3, r=9, reps=2):
         return [(pl, synth.uniform_residues((pl[3], pl[2], top - i, N), q[:top - i], seed, stream + i,
                                             device=dev)) for i, pl in enumerate(plans)]
 
+    stc_top = L - depth - 6 - r
     cts = levels(cts_plans, L, 200)
-    stc = levels(stc_plans, L - depth - 6 - r, 300)
+    stc = levels(stc_plans, stc_top, 300)
     ct = synth.uniform_residues((B, 2, 1, N), q[:1], seed, 1, device=dev)
     rf = Refresh(q, p, alpha, keys, device=dev.index)
     stream = torch.cuda.current_stream(dev)
+    steps = ["modraise", "coeff_to_slot", "conj_extract", "sin_fold_re", "sin_fold_im", "restore_merge",
+             "slot_to_coeff"]
+    per = {k: 0.0 for k in steps}
     try:
-        ms = _time_call(lambda: rf.refresh(ct, r, cts, stc), reps, stream)
+        for _ in range(2):
+            rf.refresh(ct, r, cts, stc)
+        torch.cuda.synchronize()
+        total = 0.0
+        with ClockSampler(dev) as clk:
+            for _ in range(reps):
+                evs = []
+
+                def mark(name):
+                    e = torch.cuda.Event(enable_timing=True)
+                    e.record(stream)
+                    evs.append((name, e))
+
+                start = torch.cuda.Event(enable_timing=True)
+                start.record(stream)
+                rf.refresh(ct, r, cts, stc, mark=mark)
+                torch.cuda.synchronize()
+                prev = start
+                for name, e in evs:
+                    per[name] += prev.elapsed_time(e) / reps
+                    prev = e
+                total += start.elapsed_time(evs[-1][1]) / reps
     finally:
         rf.close()
     S = N // 2
-    per_ct = 1 + 2 * (7 + r)
-    for stride, t0, bb, gg in cts_plans + stc_plans:
-        rotated = sum(1 for g in range(gg) if (stride * (t0 + bb * g)) % S)
-        per_ct += (bb - 1) + rotated
-    return {"workload": "refresh of %d ciphertexts, %d + %d primes, alpha %d, factored transforms of "
-                        "depth %d, sin_fold r = %d (%d levels)" % (B, L, K, alpha, depth, r,
-                                                                  2 * depth + 6 + r),
-            "ms_per_call": ms, "ciphertext_refreshes_per_s": B / (ms * 1e-3),
-            "key_switches_per_ciphertext": per_ct, "keys": len(amounts) + 2,
-            "pages_cpu_s_for_8_ciphertexts": 4393.5,
-            "data": "seeded uniform residues for keys, plaintexts and the input ciphertexts"}
+
+    def transform(plans, top):
+        ks, w = 0, work()
+        for i, (stride, t0, bb, gg) in enumerate(plans):
+            rotated = sum(1 for g in range(gg) if (stride * (t0 + bb * g)) % S)
+            ks += (bb - 1) + rotated
+            w = work_sum(w, work_bsgs_plan(top - i, K, alpha, B, bb, gg, rotated))
+        return ks, w
+
+    out = {"workload": "refresh of %d ciphertexts, %d + %d primes, alpha %d, factored transforms of "
+                       "depth %d, sin_fold r = %d (%d levels)" % (B, L, K, alpha, depth, r, 2 * depth + 6 + r),
+           "ms_per_call": total, "ciphertext_refreshes_per_s": B / (total * 1e-3),
+           "ms_per_step": per, "share_per_step": {k: v / total for k, v in per.items()},
+           "keys": len(amounts) + 2, "clocks": clk.summary(),
+           "pages_cpu_s_for_8_ciphertexts": 4393.5,
+           "data": "seeded uniform residues for keys, plaintexts and the input ciphertexts"}
+    for name, plans, top in (("coeff_to_slot", cts_plans, L), ("slot_to_coeff", stc_plans, stc_top)):
+        ks, w = transform(plans, top)
+        e = ks_entry(B * ks, per[name], w, hbm_peak, rates)
+        e["plans"] = [list(pl) for pl in plans]
+        e["key_switches_per_ciphertext"] = ks
+        e["pages_cpu_s_for_8_ciphertexts"] = 1737.20 if name == "coeff_to_slot" else 1736.19
+        out[name] = e
+    return out
 
 
 def run_ks_only(args):
+    """Only the selected key-switching workloads (--ks-entries), for
+    profiling: nothing else is built, so a capture holds only that workload's
+    keys and workspace on the device."""
     import torch
     dev = torch.device("cuda", 0)
     hbm_peak, _ = peaks()
     from rns_ckks_polynomial_b200 import Context, primes
     ctx = Context(primes(60), primes(61)[60:], 60)
     ipeak = intpipe_peaks(ctx)
-    print(json.dumps({"keyswitch": run_keyswitch(dev, hbm_peak, ipeak, args.ks_batch, args.ks_keys)}),
-          flush=True)
+    ctx.close()
+    entries = tuple(e for e in args.ks_entries.split(",") if e)
+    print(json.dumps({"keyswitch": run_keyswitch(dev, hbm_peak, ipeak, args.ks_batch, args.ks_keys,
+                                                 entries, refresh_batch=args.ks_batch)}), flush=True)
 
 
 def main():
     args = parse()
     if args.refresh_only:
-        import torch
-        print(json.dumps({"refresh": run_refresh(torch.device("cuda", 0))}), flush=True)
-        return
+        args.ks_only, args.ks_entries = True, "refresh"
     if args.ks_only:
         run_ks_only(args)
         return

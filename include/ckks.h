@@ -409,7 +409,11 @@ int ckks_modraise(const ckks_ctx *ctx, const uint64_t *in, int l, uint64_t *out,
  * iterations in every thread of a grid of `blocks` x 256 threads and writes
  * the elapsed milliseconds (CUDA events) to *ms and the operation count to
  * *ops.  kind 0: 64-bit Shoup modular multiply; kind 1: 64x64->128
- * multiply-accumulate; kind 2: 64x64 high-half multiply.
+ * multiply-accumulate; kind 2: 64x64 high-half multiply; kind 5: the
+ * forward NTT's own butterfly (Shoup product with the three-partial-product
+ * quotient, the cheap quotient-times-q for 2^60 - delta primes when every
+ * prime of the context has that form, and the lazy add/sub; *ops counts
+ * butterflies, one modular product each).
  * Tensor-pipe kinds (one issuing thread per CTA of 128 threads, `iters`
  * back-to-back int8 tcgen05.mma of M = 128, K = 32; *ops counts 2 M N K per
  * MMA): kind 3: N = 256 (the dense int8 rate); kind 4: N = 32 (the basis

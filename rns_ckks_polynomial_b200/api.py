@@ -367,8 +367,9 @@ class Context:
 
     # ------------------------------------------------------------ measurement
     def bench_intpipe(self, kind, blocks, iters):
-        """(ms, ops) of the integer-pipe microbenchmark `kind` (0 Shoup mulmod,
-        1 64x64->128 MAC, 2 64-bit high multiply)."""
+        """(ms, ops) of the microbenchmark `kind`: 0 Shoup mulmod, 1 64x64->128
+        MAC, 2 64-bit high multiply, 3 / 4 int8 tcgen05.mma at N = 256 / 32,
+        5 the forward NTT's butterfly."""
         ms, ops = C.c_double(), C.c_double()
         check("ckks_bench_intpipe",
               lib().ckks_bench_intpipe(self._h, kind, blocks, iters, C.byref(ms), C.byref(ops)))

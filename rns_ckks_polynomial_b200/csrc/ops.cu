@@ -652,7 +652,21 @@ extern "C" int ckks_bsgs_lintrans_plan(const ckks_ctx *ctx, const uint64_t *x, c
 }
 
 // ---------------------------------------------------------------- microbenchmarks
-__global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, u64 *sink)
+// The forward NTT's own butterfly (ct_bfly: the three-partial-product Shoup
+// quotient, the cheap q h product for 2^60 - delta primes when kS, and the
+// lazy add/sub), 4 independent butterflies over 8 registers per iteration.
+template <bool kS>
+__device__ __forceinline__ void bfly_loop(u64 x[8], int iters, u64 q, u64 w, u64 wp)
+{
+    const Mod md{q, 2 * q, 4 * q, (1ull << 60) - q};
+    const ulonglong2 tw = make_ulonglong2(w, wp);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ct_bfly<kS>(x[k], x[k + 4], tw, md);
+    }
+}
+
+__global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, int special, u64 *sink)
 {
     u64 x[8], h[8];
 #pragma unroll
@@ -674,11 +688,15 @@ __global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, u64 *s
 #pragma unroll
             for (int k = 0; k < 8; ++k) mac128(h[k], x[k], y[k], m);  // 8 independent chains
         }
-    } else {
+    } else if (kind == 2) {
         for (int it = 0; it < iters; ++it) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) x[k] = mulhi(x[k], wp) + w;
         }
+    } else if (special) {
+        bfly_loop<true>(x, iters, q, w, wp);
+    } else {
+        bfly_loop<false>(x, iters, q, w, wp);
     }
     u64 acc = 0;
 #pragma unroll
@@ -690,7 +708,7 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
                                   double *ops)
 {
     CKKS_TRY(check_ctx(ctx));
-    if (kind < 0 || kind > 4 || blocks < 1 || blocks > 148 * 64 || iters < 1 || !ms || !ops)
+    if (kind < 0 || kind > 5 || blocks < 1 || blocks > 148 * 64 || iters < 1 || !ms || !ops)
         return set_error(CKKS_EINVAL, "bad microbenchmark arguments");
     CKKS_TRY(set_device(ctx));
     if (kind >= 3) return bench_mma(ctx, kind == 3 ? 256 : 32, blocks, iters, ms, ops);
@@ -702,9 +720,10 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
     cudaEvent_t a, b;
     cudaEventCreate(&a);
     cudaEventCreate(&b);
-    intpipe_kernel<<<blocks, 256>>>(kind, std::max(1, iters / 16), q, w, wp, sink);  // warm-up
+    const int special = ctx->t.special ? 1 : 0;
+    intpipe_kernel<<<blocks, 256>>>(kind, std::max(1, iters / 16), q, w, wp, special, sink);  // warm-up
     cudaEventRecord(a);
-    intpipe_kernel<<<blocks, 256>>>(kind, iters, q, w, wp, sink);
+    intpipe_kernel<<<blocks, 256>>>(kind, iters, q, w, wp, special, sink);
     cudaEventRecord(b);
     e = cudaEventSynchronize(b);
     float t = 0;
@@ -714,6 +733,6 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
     cudaFree(sink);
     if (e != cudaSuccess) return cuda_status(e, "intpipe_kernel");
     *ms = t;
-    *ops = (double)blocks * 256.0 * iters * 8.0;
+    *ops = (double)blocks * 256.0 * iters * (kind == 5 ? 4.0 : 8.0);
     return CKKS_OK;
 }

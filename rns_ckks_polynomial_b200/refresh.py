@@ -209,17 +209,28 @@ class Refresh:
             scale = Fraction(scale) * Fraction(pt_scale) / self.q[l - 1]
         return ct, scale
 
-    def refresh(self, ct_q0, r, cts_levels, stc_levels):
+    def refresh(self, ct_q0, r, cts_levels, stc_levels, mark=None):
         """A ciphertext [B][2][1][n] on q_0 -> (ciphertext, scale), the slots
         back at the message scale.  cts_levels / stc_levels as for lintrans,
-        encoded at 2^60 and 2^50."""
+        encoded at 2^60 and 2^50.  mark, if given, is called with each step's
+        name after its calls are issued (a timing hook: it may record an
+        event on the current stream)."""
+        mark = mark or (lambda name: None)
         top = self.ctx(self.L)
         ct = top.modraise(ct_q0, ws=self._ws(top, OP_MODRAISE, ct_q0.shape[0], ct_q0.shape[2]))
+        mark("modraise")
         ct, scale = self.lintrans(ct, Fraction(self.q[0]), cts_levels, 2**60)
+        mark("coeff_to_slot")
         l = self.level(ct)
         cx = self.ctx(l)
         re, im = cx.conj_extract(ct, self.keys["conj"], ws=self._ws(cx, OP_CONJ_EXTRACT, ct.shape[0]))
+        mark("conj_extract")
         sre, s_out = self.sin_fold(re, scale, r)
+        mark("sin_fold_re")
         sim, _ = self.sin_fold(im, scale, r)
+        mark("sin_fold_im")
         merged = self.ctx(self.level(sre)).restore_merge(sre, sim)
-        return self.lintrans(merged, s_out, stc_levels, 2**50)
+        mark("restore_merge")
+        out = self.lintrans(merged, s_out, stc_levels, 2**50)
+        mark("slot_to_coeff")
+        return out

@@ -14,21 +14,48 @@ if ROOT not in sys.path:
 import bench  # noqa: E402
 
 
+def _ops(w):
+    return w["bfly"] + w["mm"] + w["mac"]
+
+
 def test_boot_rotation_counts():
     up, inner, down = bench.ks_work_keyswitch_parts(2100, 60, 60)
     # ModUp of one ciphertext: 35 digits x 60 sources x 2100 targets x 2048 multiply-adds
     assert up["mac"] == 35 * 60 * 2100 * 2048
-    assert up["mm"] + up["mac"] == pytest.approx(9.89e9, rel=0.01)
-    assert inner["mm"] + inner["mac"] + down["mm"] + down["mac"] == pytest.approx(8.88e8, rel=0.01)
-    mm, mac, _ = bench.ks_work_rotation(2100, 60, 60, 1, 4)
-    assert mm + mac == pytest.approx(1.344e10, rel=0.01)
+    # its transforms: 2100 INTTs and 35 x 2160 - 2100 NTTs of 11 x 1024 butterflies
+    assert up["bfly"] == (2100 + 35 * 2160 - 2100) * 11 * 1024
+    assert _ops(up) == pytest.approx(9.89e9, rel=0.01)
+    assert _ops(inner) + _ops(down) == pytest.approx(8.88e8, rel=0.01)
+    w = bench.work_rotation(2100, 60, 60, 1, 4)
+    assert _ops(w) == pytest.approx(1.344e10, rel=0.01)
+    # 60-prime digits and 60 special primes: every conversion runs on the tensor cores
+    assert w["conv_tc"] == up["mac"] + 4 * down["mac"]
+    assert bench.work_rotation(2100, 60, 60, 1, 4, engine="integer")["conv_tc"] == 0
+    # key bytes: 4 keys of 35 x 2 x 2160 limbs
+    assert w["bytes"] == 4 * 35 * 2 * 2160 * 2048 * 8 + 2 * 2100 * 2048 * 8 * 5
 
 
 def test_layer_and_bsgs_counts():
-    mm, mac, _ = bench.ks_work_mrr(112, 8, 8, 1)
-    assert mm + mac == pytest.approx(6.30e7, rel=0.02)
-    mm, mac, _ = bench.ks_work_bsgs(112, 8, 8, 1, 32, 32)
-    assert mm + mac == pytest.approx(2.78e9, rel=0.02)
+    assert _ops(bench.work_mrr(112, 8, 8, 1)) == pytest.approx(6.30e7, rel=0.02)
+    assert _ops(bench.work_bsgs(112, 8, 8, 1, 32, 32)) == pytest.approx(2.78e9, rel=0.02)
+    # alpha = 1, K = 1: below the tensor cores' 8 sources
+    assert bench.work_rotation(4, 1, 1, 1, 1)["conv_tc"] == 0
+
+
+def test_model_charges_the_engine_that_ran():
+    """With the conversion on the tensor cores the roofline charges it at the
+    int8 rate (64 byte-plane products per multiply-add); the integer-pipe
+    model is reported beside it."""
+    rates = {"bfly": 1e12, "mm": 1e12, "mac": 1e12, "int8_mac": 64e12}
+    w = bench.work(mac=10**12, conv_tc=10**12)
+    t_tc, _ = bench.model_seconds(w, rates, 1e3, engine_tc=True)
+    t_int, _ = bench.model_seconds(w, rates, 1e3, engine_tc=False)
+    assert t_tc == pytest.approx(1.0) and t_int == pytest.approx(1.0)
+    e = bench.ks_entry(1, 2000.0, w, 1e3, rates)
+    assert e["roofline_frac"] == pytest.approx(0.5) and e["integer_pipe_model_frac"] == pytest.approx(0.5)
+    w2 = bench.work(bfly=2 * 10**12, mac=10**12, conv_tc=10**12, bytes=0)
+    e2 = bench.ks_entry(1, 3000.0, w2, 1e3, rates)
+    assert e2["roofline_frac"] == pytest.approx(1.0)
 
 
 def test_ntt_launch_bytes_and_products():

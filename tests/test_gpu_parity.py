@@ -414,13 +414,14 @@ def test_microbenchmarks_report_counts():
     count and leaves the device flag clear; bad kinds are rejected."""
     ctx = ctx_for(Params(4, 1, 1))
     for kind, blocks, iters, per in ((0, 16, 64, 256 * 8), (1, 16, 64, 256 * 8), (2, 16, 64, 256 * 8),
-                                     (3, 4, 64, 2 * 128 * 256 * 32), (4, 4, 64, 2 * 128 * 32 * 32)):
+                                     (3, 4, 64, 2 * 128 * 256 * 32), (4, 4, 64, 2 * 128 * 32 * 32),
+                                     (5, 16, 64, 256 * 4)):
         ms, ops = ctx.bench_intpipe(kind, blocks, iters)
         assert ms > 0
         assert ops == blocks * iters * per
     ctx.device_status()
     with pytest.raises(CkksError):
-        ctx.bench_intpipe(5, 1, 1)
+        ctx.bench_intpipe(6, 1, 1)
 
 
 def _general_primes(orc, count):
@@ -767,3 +768,100 @@ def test_key_inner_more_than_256_digits():
     ctx.device_status()
     want = np.broadcast_to((260 % np.array(ctx.mods, dtype=np.uint64))[None, None, :, None], (1, 2, LK, N))
     assert_bits_equal(acc, want, "key inner product over 260 digits")
+
+
+def test_refresh_n2048_decodes_to_the_sine_form(orc):
+    """The refresh as the oracle's n = 2048 pin runs it (23 + 4 primes, a
+    dense ternary secret, three-level factored transforms with their encoded
+    plaintexts, r = 9: 21 levels) through the per-level contexts on the GPU:
+    bit-exact against the oracle's refresh over the same plaintexts, and the
+    decrypted coefficients within 1e-5 of the sine form
+    (q_0 / 2 pi) sin(2 pi m_k / q_0) / Delta of the input's coefficients m."""
+    import math
+    from fractions import Fraction
+
+    from oracle import boot
+
+    from rns_ckks_polynomial_b200.refresh import Refresh
+    n, depth, r, L, K, alpha = N, 3, 9, 23, 4, 4
+    delta = 2**50
+    p = Params(L, K, alpha)
+    sch = Scheme(orc, p, SEED + 80)
+    chain = boot.Chain(sch.mods, L, K, alpha)
+    keys = {"rot": {a: sch.keygen_galois(galois_for_rotation(a, n))
+                    for a in boot.factored_rotation_amounts(n, depth)},
+            "conj": sch.keygen_galois(2 * n - 1), "relin": sch.keygen_relin()}
+    z = synth.uniform_real((SLOTS,), -1, 1, SEED, 810).numpy() + \
+        1j * synth.uniform_real((SLOTS,), -1, 1, SEED, 811).numpy()
+    low = np.ascontiguousarray(sch.encrypt_slots(z, delta)[:, :1])
+    q0 = int(sch.mods[0])
+
+    def levels(factors, scalar, top, pt_scale):
+        out = []
+        for i, F in enumerate(factors):
+            if i == 0:
+                F = {k: scalar * d for k, d in F.items()}
+            plan = orc.bsgs_plan(F, SLOTS)
+            pts, _ = orc.plan_plaintexts(F, plan, SLOTS, sch.mods[:top - i], pt_scale, n)
+            out.append((plan, np.stack([np.stack([np.zeros((top - i, n), np.uint64) if v is None else v
+                                                  for v in row]) for row in pts])))
+        return out
+
+    cts = levels(orc.factored_coeff_to_slot(n, depth), 0.5, L, 2**60)
+    stc = levels(orc.factored_slot_to_coeff(n, depth), q0 / (2 * math.pi * delta), L - depth - 6 - r, 2**50)
+    want, s_want = boot.refresh_with_levels(low, r, [(pl, list(a)) for pl, a in cts],
+                                            [(pl, list(a)) for pl, a in stc], keys, chain)
+    dkeys = {"rot": {a: dev(k) for a, k in keys["rot"].items()}, "conj": dev(keys["conj"]),
+             "relin": dev(keys["relin"])}
+    rf = Refresh(sch.q, sch.mods[L:], alpha, dkeys)
+    try:
+        got, s_got = rf.refresh(dev(low[None]), r, [(pl, dev(a)) for pl, a in cts],
+                                [(pl, dev(a)) for pl, a in stc])
+        torch.cuda.synchronize()
+    finally:
+        rf.close()
+    assert s_got == s_want
+    out = host(got)[0]
+    assert out.shape == (2, L - 2 * depth - 6 - r, n)
+    assert_bits_equal(out, want, "refresh at n = 2048")
+    res = orc.decrypt(low, sch.s, sch.mods[:1])
+    m = orc.crt_centered(res, sch.mods[:1])
+    res_o = orc.decrypt(out, sch.s, sch.mods[:out.shape[-2]])
+    got_c = np.array([float(Fraction(c) / s_got) for c in orc.crt_centered(res_o, sch.mods[:out.shape[-2]])])
+    sine = np.array([q0 / (2 * math.pi) * math.sin(2 * math.pi * v / q0) / delta for v in m])
+    assert np.max(np.abs(got_c - sine)) < 1e-5
+
+
+def test_coeff_to_slot_level_at_2100_primes(orc):
+    """One level of the three-level factored coeff_to_slot at the boot chain's
+    full size (2100 + 60 primes, alpha = 60): the plan (stride 64, t0 = -8,
+    bb = gg = 4) with its 6 Galois keys over 8 ciphertexts of seeded uniform
+    residues and seeded plaintext diagonals, as the refresh bench runs it.
+    The oracle recomputes ciphertext 5 (3 hoisted baby rotations, 3 rotated
+    giant steps and the unrotated one, rescale)."""
+    import psutil
+
+    from oracle.boot import Chain, bsgs_plan_apply
+    if psutil.virtual_memory().available < 64 << 30:
+        pytest.skip("needs 64 GB of free host memory for the oracle's keys")
+    p = Params(2100, 60, 60)
+    ctx = ctx_for(p)
+    seed = synth.config_seed(5) + 90
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    stride, t0, bb, gg = plan = (64, -8, 4, 4)
+    S = SLOTS
+    amounts = sorted({(stride * b) % S for b in range(1, bb)} |
+                     {(stride * (t0 + bb * g)) % S for g in range(gg)} - {0})
+    assert amounts == [64, 128, 192, 256, 512, 768]
+    keys = {a: synth.uniform_residues((35, 2, 2160, N), mods, seed, 10 + a, device="cuda") for a in amounts}
+    x = synth.uniform_residues((8, 2, 2100, N), mods[:2100], seed, 1, device="cuda")
+    pts = synth.uniform_residues((gg, bb, 2100, N), mods[:2100], seed, 2, device="cuda")
+    giants = [(stride * (t0 + bb * g)) % S for g in range(gg)]
+    y = ctx.bsgs_lintrans_plan(x, pts, [keys[(stride * b) % S] for b in range(1, bb)],
+                               [keys[G] if G else None for G in giants], plan)
+    ctx.device_status()
+    chain = Chain(mods, 2100, 60, 60)
+    hp = host(pts)
+    want, _ = bsgs_plan_apply(host(x[5]), SCALE, [[hp[g, b] for b in range(bb)] for g in range(gg)], plan,
+                              SCALE, {a: host(k) for a, k in keys.items()}, chain)
+    assert_bits_equal(host(y[5]), want, "coeff_to_slot level (64, -8, 4, 4) at 2100 primes, ciphertext 5")
