@@ -132,14 +132,22 @@ int ckks_selftest_wait_expiry(const ckks_ctx *ctx);
  *                     source primes (ModUp: alpha; ModDown: K), the integer
  *                     pipes otherwise (the default);
  *  CKKS_CONV_INTEGER  always the integer pipes (64x64->128-bit multiply-adds);
- *  CKKS_CONV_TENSOR   always the int8 tensor cores (byte-plane products).
+ *  CKKS_CONV_TENSOR   always the int8 tensor cores (byte-plane products of
+ *                     both operands, 15 accumulators per output);
+ *  CKKS_CONV_FOLDED   always the int8 tensor cores in the folded form: the
+ *                     data's byte weights folded into the matrix modulo each
+ *                     target (8 accumulators per output, the data words in
+ *                     tensor memory).  Its tables (8 x 512 bytes per target
+ *                     and digit) are built on the first call that uses it,
+ *                     which is then synchronous; make that call before any
+ *                     stream capture.
  * Every engine computes the same exact sum before the one final reduction, so
  * results are bit-identical; this is a performance switch only.  The pages
  * have no counterpart (their engine runs on CPU threads).  Takes effect for
  * calls issued after it returns; do not change it while another host thread
  * issues calls on the same context.  CKKS_EINVAL for a null context or an
  * unknown engine. */
-enum { CKKS_CONV_AUTO = 0, CKKS_CONV_INTEGER = 1, CKKS_CONV_TENSOR = 2 };
+enum { CKKS_CONV_AUTO = 0, CKKS_CONV_INTEGER = 1, CKKS_CONV_TENSOR = 2, CKKS_CONV_FOLDED = 3 };
 int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine);
 
 /* Declares that the switching keys passed to this context's calls were made

@@ -83,7 +83,7 @@ class Context:
         """Launch the bounded-wait expiry self-test; device_status() then raises."""
         check("ckks_selftest_wait_expiry", lib().ckks_selftest_wait_expiry(self._h))
 
-    CONVERSION = {"auto": 0, "integer": 1, "tensor": 2}
+    CONVERSION = {"auto": 0, "integer": 1, "tensor": 2, "folded": 3}
 
     @property
     def _kshape(self):

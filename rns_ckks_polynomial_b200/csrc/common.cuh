@@ -59,6 +59,11 @@ struct Tables {
     const uint8_t *tc_dn;         // [ceil(L/128)][128][8][64]
     int tc_tb_per_digit;
     bool tc_special;              // every prime is 2^60 - delta with delta < 2^28
+    // Folded byte planes for the int8 tensor-core path with the data in tensor memory
+    // (conv_fold.cu), targets in blocks of 32, built on first use
+    const uint8_t *fold_up;       // [dnum][fold_tb_per_digit][8][32][512]
+    const uint8_t *fold_dn;       // [ceil(L/32)][8][32][512]
+    int fold_tb_per_digit;
 };
 
 }  // namespace ckks
@@ -78,6 +83,9 @@ struct ckks_ctx {
     size_t own_ws_bytes = 0;
     int *tc_err = nullptr;  // device flag: a bounded wait of the tensor-core kernel expired
     std::atomic<int> conv_engine{CKKS_CONV_AUTO};
+    // host copies of the conversion matrices, for the folded tables built on first use
+    std::vector<u64> up_mat_host, dn_mat_host;
+    bool fold_built = false;
 };
 
 namespace ckks {

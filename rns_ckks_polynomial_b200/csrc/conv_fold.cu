@@ -1,0 +1,482 @@
+// RNS basis conversion on the int8 tensor cores, folded form (tcgen05.mma kind::i8 with the data
+// operand in tensor memory).
+//
+// The conversion out[t][c] = (sum_s M[s][t] y[s][c]) mod q_t (the step the Kestrel engine write-up,
+// section 3 table, names "RNS basis conversion") is computed exactly, but with the byte weights of
+// the data folded into the matrix modulo each target prime:
+//     y_s = sum_v y_{s,v} 2^(8v)  (bytes),   F[(s,v)][t] = 2^(8v) M[s][t] mod q_t  (60 bits),
+//     out_t = sum_{s,v} y_{s,v} F[(s,v)][t]  (mod q_t).
+// F is split into byte planes F_u, so that
+//     sum_{s,v} y_{s,v} F = sum_{u<8} 2^(8u) P_u,   P_u = sum_{k'} y_{k'} F_u[k'][t],  k' = 8s + v,
+// an unsigned 8-bit contraction of K' = 8 S terms: P_u <= 512 * 255^2 < 2^25, so eight int32
+// accumulators hold the exact sum, and the epilogue rebuilds the (< 2^82) value and reduces it once.
+// The K' index 8s + v makes the data operand the raw 64-bit words: the four bytes of a 32-bit half
+// of y_s are consecutive K' entries, so staging writes the words unchanged.
+//
+// One CTA (one per SM, owning all 512 TMEM columns) converts one block of 32 targets (the MMA's N)
+// for a run of coefficient tiles of 128 (the MMA's M, the TMEM lanes):
+//  - the block's eight F planes (8 x 32 targets x 512 bytes = 128 KiB) stay in shared memory (the B
+//    operand, K-major core matrices) for the whole run;
+//  - the data tile (128 coefficients x S words) is the A operand in tensor memory, double-buffered
+//    (columns 256..383 and 384..511, two 32-bit columns per source);
+//  - accumulator P_u takes columns 32 u .. 32 u + 31.
+// Warp roles, synchronised by mbarriers only:
+//  - 4 MMA warps (one elected lane each) own planes {2k, 2k+1}: for tile i they wait until its data
+//    is staged and the epilogue has read their planes of tile i - 1, issue the ceil(S / 4) K-steps
+//    of each plane and commit each plane to its own barrier;
+//  - 16 epilogue / staging warps: for tile i they read P_0 .. P_7 as each completes (releasing it to
+//    the next tile's products at once), rebuild and reduce the 32 x 128 outputs and store them, then
+//    write the prefetched words of tile i + 2 into the data buffer tile i used (free once all eight
+//    planes of tile i are complete) and prefetch tile i + 3.  Warp w reads TMEM lane quadrant w & 3
+//    (coefficients 32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight
+//    targets of one coefficient; for staging it owns sources 16 (w >> 2) .. 16 (w >> 2) + 15.
+//
+// Every mbarrier wait is bounded: on expiry a thread records an error flag and leaves its loop, the
+// MMA warps wait (bounded again) for the products they issued, the CTA frees its tensor memory and
+// returns; the host reports CKKS_ECUDA.
+#include "internal.cuh"
+
+namespace ckks {
+namespace {
+
+constexpr int kFM = 128;                          // coefficients per tile (MMA M, TMEM lanes)
+constexpr int kFN = 32;                           // targets per CTA (MMA N)
+constexpr int kFKP = 512;                         // K' extent in bytes: 64 sources x 8 bytes
+constexpr int kFPlanes = 8;
+constexpr int kFPlaneBytes = kFN * kFKP;          // 16 KiB
+constexpr int kFBlock = kFPlanes * kFPlaneBytes;  // 128 KiB per block of 32 targets
+constexpr int kFSbo = (kFKP / 16) * 128;          // 8-row-group stride of the core-matrix layout
+constexpr int kFEpiWarps = 16, kFEpiThreads = 32 * kFEpiWarps;
+constexpr int kFThreads = kFEpiThreads + 128;
+constexpr int kFTmemCols = 512;
+constexpr int kFAcol = 256;                       // first data-buffer column
+constexpr int kFSmemBar = kFBlock;
+constexpr int kFSmemBytes = kFBlock + 256;
+
+enum { kFBarMma = 0, kFBarFree = 8, kFBarFull = 16, kFBarDrain = 18, kFNumBars = 19 };
+static_assert(kFSmemBar + 8 * kFNumBars + 4 <= kFSmemBytes, "shared-memory layout");
+
+__host__ __device__ __forceinline__ int fcm_off(int row, int k)
+{
+    return (row >> 3) * kFSbo + (k >> 4) * 128 + (row & 7) * 16 + (k & 15);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Shared-memory matrix descriptor: start address >> 4, LBO 128 B, SBO kFSbo, version 1, no swizzle.
+__device__ __forceinline__ u64 fsmem_desc(uint32_t addr)
+{
+    return (u64)((addr >> 4) & 0x3FFF) | ((u64)(128 >> 4) << 16) | ((u64)(kFSbo >> 4) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor: int32 accumulate, unsigned 8-bit A and B, both K-major, N = 32, M = 128.
+constexpr uint32_t kFIdesc = (2u << 4) | ((uint32_t)(kFN >> 3) << 17) | ((uint32_t)(kFM >> 4) << 24);
+
+// D[tmem_d] (+)= A[tmem_a] x B[bdesc]: A from tensor memory, B from shared memory.
+__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, u64 bdesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+        :: "r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(kFIdesc), "r"(accumulate), "r"(0), "r"(0), "r"(0),
+           "r"(0));
+}
+
+__device__ __forceinline__ void fcommit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool fbar_wait(const uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    for (int i = 0; i < (1 << 18); ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void fbar_init(uint64_t *bar, int count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fbar_arrive(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" :: "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void ffence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void ffence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Eight columns of one accumulator plane for the warp's 32 lanes.
+__device__ __forceinline__ void fld8(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 columns (16 source words) of the data operand for the warp's 32 lanes.
+__device__ __forceinline__ void fst32(uint32_t taddr, const u64 (&v)[16])
+{
+    uint32_t r[32];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        r[2 * k] = (uint32_t)v[k];
+        r[2 * k + 1] = (uint32_t)(v[k] >> 32);
+    }
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+           "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+           "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+           "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// x = hi 2^64 + lo (x < 2^126) mod q for q = 2^60 - delta, delta < 2^28 (2^60 = delta mod q).
+__device__ __forceinline__ u64 freduce_special(u64 hi, u64 lo, u64 delta, u64 q)
+{
+    constexpr u64 kMask60 = ((u64)1 << 60) - 1;
+    const uint32_t c16 = (uint32_t)delta << 4;
+    const u64 p0 = (u64)(uint32_t)hi * c16, p1 = (u64)(uint32_t)(hi >> 32) * c16;
+    const u64 t = p0 + (p1 << 32);
+    const u64 yl = t + lo;
+    const u64 yh = (p1 >> 32) + (t < p0) + (yl < t);
+    const u64 a = (yh << 4) | (yl >> 60);
+    const u64 z = (yl & kMask60) + a * delta;
+    const u64 w = (z & kMask60) + (z >> 60) * delta;
+    return w >= q ? w - q : w;
+}
+
+// Job geometry (kind 0: ModUp over (ciphertext, digit), the ciphertext fastest in the grid so the
+// CTAs that share a digit's F block run together; kind 1: ModDown over (job, component)).
+struct FoldJobs {
+    int kind;
+    const u64 *y;
+    u64 *out;
+    const uint8_t *fpl;   // F blocks
+    int L, LK, alpha, dnum, K, tb_per_digit, batch;
+    int csplit;
+    __device__ __forceinline__ void geometry(int z, int &S, int &T, int &lo, const u64 *&ybase,
+                                             const uint8_t *&fbase, int &zrow) const
+    {
+        if (kind == 0) {
+            const int b = z % batch, jd = z / batch;
+            lo = jd * alpha;
+            S = min(alpha, L - lo);
+            T = LK - S;
+            ybase = y + ((size_t)b * L + lo) * kN;
+            fbase = fpl + (size_t)jd * tb_per_digit * kFBlock;
+            zrow = b * dnum + jd;
+        } else {
+            lo = 0;
+            S = K;
+            T = L;
+            ybase = y + (size_t)z * K * kN;
+            fbase = fpl;
+            zrow = z;
+        }
+    }
+    __device__ __forceinline__ int prime(int ti, int lo, int S) const
+    {
+        return kind == 0 ? (ti < lo ? ti : ti + S) : ti;
+    }
+    __device__ __forceinline__ u64 *row(int zrow, int t) const
+    {
+        return kind == 0 ? out + ((size_t)zrow * LK + t) * kN : out + ((size_t)zrow * L + t) * kN;
+    }
+};
+
+template <bool kSpecial>
+__global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, const PrimeConst *__restrict__ pc,
+                                                                  int *err)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tb = blockIdx.x / jobs.csplit, run = blockIdx.x - tb * jobs.csplit, z = blockIdx.y;
+    int S, T, lo, zrow;
+    const u64 *ybase;
+    const uint8_t *fbase;
+    jobs.geometry(z, S, T, lo, ybase, fbase, zrow);
+    if (tb * kFN >= T) return;  // uniform per CTA
+    const int ntiles = kN / kFM / jobs.csplit;  // 16, 8 or 4
+    const int cbase = run * ntiles * kFM;
+    const int nks = (S + 3) >> 2;                // K-steps of 32 bytes (4 sources)
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kFSmemBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kFSmemBar + 8 * kFNumBars);
+    const bool mma_warp = warp >= kFEpiWarps;
+    const int issuer = warp - kFEpiWarps;  // planes 2 issuer, 2 issuer + 1
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tslot)), "r"(kFTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        for (int u = 0; u < kFPlanes; ++u) {
+            fbar_init(bar + kFBarMma + u, 1);
+            fbar_init(bar + kFBarFree + u, kFEpiThreads);
+        }
+        fbar_init(bar + kFBarFull + 0, kFEpiThreads);
+        fbar_init(bar + kFBarFull + 1, kFEpiThreads);
+        fbar_init(bar + kFBarDrain, 4);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // staging share: coefficient m of each tile, sources s0 .. s0 + 15
+    const int quad = warp & 3, part = warp >> 2;
+    const int m = quad * 32 + lane, s0 = part * 16;
+    const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + m;
+    auto fetch = [&](int i, u64 (&v)[16]) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? __ldg(ysrc + (size_t)k * kN + i * kFM) : 0;
+    };
+    u64 pre[16];
+    if (!mma_warp) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(fbase + (size_t)tb * kFBlock);
+        uint4 *dst = reinterpret_cast<uint4 *>(sm);
+        for (int i = tid; i < kFBlock / 16; i += kFEpiThreads) dst[i] = __ldg(src + i);
+        fetch(0, pre);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    ffence_before();
+    __syncthreads();
+    ffence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    bool ok = true;
+
+    if (mma_warp) {
+        // ------------------------------------------------ MMA issue (one elected lane per warp)
+        const u64 bdesc0 = fsmem_desc(smem_u32(sm));
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int buf = i & 1;
+            ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFull + buf, (i >> 1) & 1));
+            for (int h = 0; h < 2 && ok; ++h) {
+                const int u = 2 * issuer + h;
+                if (i > 0) ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFree + u, (i - 1) & 1));
+                if (!ok) break;
+                ffence_after();
+                if (lane == 0) {
+                    const u64 bd = bdesc0 + (((size_t)u * kFPlaneBytes) >> 4);
+                    const uint32_t ta = tmem + kFAcol + buf * 128;
+                    for (int ks = 0; ks < nks; ++ks)
+                        mma_ts(tmem + u * kFN, ta + ks * 8, bd + ((ks * 256) >> 4), ks > 0 ? 1u : 0u);
+                    fcommit(bar + kFBarMma + u);
+                }
+                __syncwarp();
+            }
+        }
+        // every product issued here has completed before tensor memory is freed (bounded)
+        if (lane == 0) fcommit(bar + kFBarDrain);
+        __syncwarp();
+        ok = fbar_wait(bar + kFBarDrain, 0) && ok;
+    } else {
+        // ------------------------------------------------ epilogue and staging
+        // tile 0 into buffer 0, tile 1 into buffer 1
+        fst32(tmem + lane_base + kFAcol + 0 * 128 + part * 32, pre);
+        if (ntiles > 1) {
+            fetch(1, pre);
+            fst32(tmem + lane_base + kFAcol + 1 * 128 + part * 32, pre);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        ffence_before();
+        fbar_arrive(bar + kFBarFull + 0);
+        fbar_arrive(bar + kFBarFull + 1);
+        if (ntiles > 2) fetch(2, pre);
+        // the eight targets of this thread: tb * 32 + part * 8 + c
+        int tcol[8];
+        bool tvalid[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int ti = tb * kFN + part * 8 + c;
+            tvalid[c] = ti < T;
+            tcol[c] = tvalid[c] ? jobs.prime(ti, lo, S) : 0;
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            u64 g0[8], g1[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) g0[c] = g1[c] = 0;
+#pragma unroll
+            for (int u = 0; u < kFPlanes; ++u) {
+                ok = fbar_wait(bar + kFBarMma + u, i & 1) && ok;
+                ffence_after();
+                uint32_t r[8];
+                fld8(tmem + lane_base + u * kFN + part * 8, r);
+                ffence_before();
+                fbar_arrive(bar + kFBarFree + u);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (u < 4)
+                        g0[c] += (u64)r[c] << (8 * u);
+                    else
+                        g1[c] += (u64)r[c] << (8 * (u - 4));
+                }
+            }
+            // all eight planes of tile i are complete: its data buffer takes tile i + 2
+            if (i + 2 < ntiles && ok) {
+                fst32(tmem + lane_base + kFAcol + (i & 1) * 128 + part * 32, pre);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                ffence_before();
+                fbar_arrive(bar + kFBarFull + (i & 1));
+                if (i + 3 < ntiles) fetch(i + 3, pre);
+            }
+            if (ok) {
+                const int coef = cbase + i * kFM + m;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (!tvalid[c]) continue;
+                    const u64 lo64 = g0[c] + (g1[c] << 32);
+                    const u64 hi64 = (g1[c] >> 32) + (lo64 < g0[c]);
+                    const PrimeConst &p = pc[tcol[c]];
+                    u64 res;
+                    if constexpr (kSpecial)
+                        res = freduce_special(hi64, lo64, p.delta, p.q);
+                    else
+                        res = reduce128(hi64, lo64, p);
+                    jobs.row(zrow, tcol[c])[coef] = res;
+                }
+            }
+            if (!ok) break;
+        }
+    }
+    if (!ok) atomicExch(err, 1);
+    ffence_before();
+    __syncthreads();
+    ffence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kFTmemCols));
+}
+
+// Host: the F blocks of a (targets x sources) matrix given by `at(ti, s)` over target primes
+// `prime(ti)`, one block of 32 targets after another, each in the shared-memory layout:
+// plane u, row r (target 32 tb + r), byte k' = 8 s + v holds byte u of 2^(8v) at(ti, s) mod q.
+template <class F, class P>
+void build_fold(std::vector<uint8_t> &dst, size_t base, int T, int S, const std::vector<u64> &mods, F at,
+                P prime)
+{
+    const int tbs = (T + kFN - 1) / kFN;
+    parallel_for(tbs, [&](int tb) {
+        for (int r = 0; r < kFN; ++r) {
+            const int ti = tb * kFN + r;
+            if (ti >= T) continue;
+            const u64 q = mods[prime(ti)];
+            for (int s = 0; s < S; ++s) {
+                u64 f = at(ti, s) % q;
+                for (int v = 0; v < 8; ++v) {
+                    const int k = 8 * s + v;
+                    for (int u = 0; u < kFPlanes; ++u)
+                        dst[base + (size_t)tb * kFBlock + (size_t)u * kFPlaneBytes + fcm_off(r, k)] =
+                            (uint8_t)(f >> (8 * u));
+                    f = host_mulmod(f, 256 % q, q);
+                }
+            }
+        }
+    });
+}
+
+int upload_fold(ckks_ctx *ctx, const std::vector<uint8_t> &h, const uint8_t **out)
+{
+    void *d = nullptr;
+    if (cudaMalloc(&d, std::max<size_t>(h.size(), 16)) != cudaSuccess) {
+        cudaGetLastError();
+        return set_error(CKKS_ENOMEM, "folded conversion table allocation failed");
+    }
+    ctx->allocations.push_back(d);
+    cudaError_t e = cudaMemcpy(d, h.data(), h.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_status(e, "cudaMemcpy(folded conversion tables)");
+    *out = static_cast<const uint8_t *>(d);
+    return CKKS_OK;
+}
+
+int launch_fold(const ckks_ctx *ctx, FoldJobs j, int tbs, int jobs, cudaStream_t s)
+{
+    if (jobs <= 0) return CKKS_OK;
+    const long ctas = (long)tbs * jobs;
+    j.csplit = ctas >= 148 * 4 ? 1 : ctas >= 148 * 2 ? 2 : 4;  // 16, 8 or 4 tiles per run
+    const dim3 grid(tbs * j.csplit, jobs);
+    if (ctx->t.tc_special)
+        conv_fold_kernel<true><<<grid, kFThreads, kFSmemBytes, s>>>(j, ctx->t.pc, ctx->tc_err);
+    else
+        conv_fold_kernel<false><<<grid, kFThreads, kFSmemBytes, s>>>(j, ctx->t.pc, ctx->tc_err);
+    CKKS_CHECK_LAUNCH("conv_fold_kernel");
+    return CKKS_OK;
+}
+
+}  // namespace
+
+static int build_fold_tables(ckks_ctx *ctx)
+{
+    Tables &T = ctx->t;
+    const std::vector<u64> &up_mat = ctx->up_mat_host, &dn_mat = ctx->dn_mat_host;
+    const int L = ctx->L, K = ctx->K, LK = L + K, alpha = ctx->alpha, dnum = ctx->dnum;
+    T.fold_tb_per_digit = (LK - 1 + kFN - 1) / kFN;
+    if (alpha > 64 || K > 64) return set_error(CKKS_EUNSUPPORTED, "more than 64 sources per conversion");
+    {
+        const size_t per_digit = (size_t)T.fold_tb_per_digit * kFBlock;
+        std::vector<uint8_t> h(per_digit * dnum, 0);
+        for (int j = 0; j < dnum; ++j) {
+            const int lo = j * alpha, S = std::min(alpha, L - lo);
+            build_fold(h, per_digit * j, LK - S, S, ctx->mods,
+                       [&](int ti, int s) {
+                           const int t = ti < lo ? ti : ti + S;
+                           return up_mat[((size_t)j * alpha + s) * LK + t];
+                       },
+                       [&](int ti) { return ti < lo ? ti : ti + S; });
+        }
+        CKKS_TRY(upload_fold(ctx, h, &T.fold_up));
+    }
+    {
+        std::vector<uint8_t> h((size_t)((L + kFN - 1) / kFN) * kFBlock, 0);
+        build_fold(h, 0, L, K, ctx->mods, [&](int ti, int s) { return dn_mat[(size_t)s * L + ti]; },
+                   [&](int ti) { return ti; });
+        CKKS_TRY(upload_fold(ctx, h, &T.fold_dn));
+    }
+    cudaError_t e = cudaFuncSetAttribute(conv_fold_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kFSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(conv_fold_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kFSmemBytes);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(conv_fold_kernel)");
+    return CKKS_OK;
+}
+
+// The folded tables, built once per context on the first call that needs them.
+static int ensure_fold_tables(ckks_ctx *ctx)
+{
+    std::lock_guard<std::mutex> lock(ctx->mu);
+    if (ctx->fold_built) return CKKS_OK;
+    CKKS_TRY(build_fold_tables(ctx));
+    ctx->fold_built = true;
+    return CKKS_OK;
+}
+
+int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s)
+{
+    CKKS_TRY(ensure_fold_tables(ctx));
+    const Tables &T = ctx->t;
+    FoldJobs j{0, y, digits, T.fold_up, T.L, T.LK, T.alpha, T.dnum, T.K, T.fold_tb_per_digit, batch, 1};
+    return launch_fold(ctx, j, T.fold_tb_per_digit, batch * T.dnum, s);
+}
+
+int launch_conv_fold_down(ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s)
+{
+    CKKS_TRY(ensure_fold_tables(ctx));
+    const Tables &T = ctx->t;
+    FoldJobs j{1, zsrc, cv, T.fold_dn, T.L, T.LK, T.alpha, T.dnum, T.K, 0, 1, 1};
+    return launch_fold(ctx, j, (T.L + kFN - 1) / kFN, jobs2, s);
+}
+
+}  // namespace ckks

@@ -513,12 +513,13 @@ __global__ void wait_expiry_kernel(int *err)
 
 }  // namespace
 
-bool conv_on_tensor(const ckks_ctx *ctx, int sources)
+ConvKind conv_kind(const ckks_ctx *ctx, int sources)
 {
     switch (ctx->conv_engine.load(std::memory_order_relaxed)) {
-    case CKKS_CONV_INTEGER: return false;
-    case CKKS_CONV_TENSOR: return true;
-    default: return sources > kTcMinSources;
+    case CKKS_CONV_INTEGER: return kConvInteger;
+    case CKKS_CONV_TENSOR: return kConvTensor;
+    case CKKS_CONV_FOLDED: return kConvFolded;
+    default: return sources > kTcMinSources ? kConvTensor : kConvInteger;
     }
 }
 

@@ -147,7 +147,7 @@ u64 host_find_psi(u64 q, int n)
     return best;
 }
 
-static void parallel_for(int count, const std::function<void(int)> &fn)
+void parallel_for(int count, const std::function<void(int)> &fn)
 {
     unsigned hw = std::max(1u, std::min(32u, std::thread::hardware_concurrency()));
     int nt = std::min<int>((int)hw, count);
@@ -323,7 +323,10 @@ static int build_tables(ckks_ctx *ctx)
     CKKS_TRY(upload(ctx, dn_hatinv, &T.dn_hatinv));
     CKKS_TRY(upload(ctx, dn_mat, &T.dn_mat));
     CKKS_TRY(upload(ctx, dn_pinv, &T.dn_pinv));
-    return build_tc_tables(ctx, up_mat, dn_mat);
+    CKKS_TRY(build_tc_tables(ctx, up_mat, dn_mat));
+    ctx->up_mat_host = std::move(up_mat);
+    ctx->dn_mat_host = std::move(dn_mat);
+    return CKKS_OK;
 }
 
 static void free_ctx(ckks_ctx *ctx)
@@ -437,7 +440,8 @@ extern "C" int ckks_selftest_wait_expiry(const ckks_ctx *ctx)
 extern "C" int ckks_ctx_set_conversion(ckks_ctx *ctx, int engine)
 {
     CKKS_TRY(check_ctx(ctx));
-    if (engine != CKKS_CONV_AUTO && engine != CKKS_CONV_INTEGER && engine != CKKS_CONV_TENSOR)
+    if (engine != CKKS_CONV_AUTO && engine != CKKS_CONV_INTEGER && engine != CKKS_CONV_TENSOR &&
+        engine != CKKS_CONV_FOLDED)
         return set_error(CKKS_EINVAL, "unknown conversion engine");
     ctx->conv_engine.store(engine, std::memory_order_relaxed);
     return CKKS_OK;

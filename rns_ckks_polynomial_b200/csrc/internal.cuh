@@ -1,6 +1,8 @@
 // Internal building blocks shared by the entry points (not part of the ABI).
 #pragma once
 
+#include <functional>
+
 #include "common.cuh"
 
 namespace ckks {
@@ -29,9 +31,14 @@ struct Carve {
 
 inline size_t limbs_bytes(size_t rows) { return ((rows * kN * sizeof(u64)) + 255) & ~(size_t)255; }
 
-// ---- int8 tensor-core basis conversion (conv_tc.cu)
+void parallel_for(int count, const std::function<void(int)> &fn);
+
+// ---- int8 tensor-core basis conversion (conv_tc.cu: byte planes; conv_fold.cu: folded)
 constexpr int kTcMinSources = 7;  // CKKS_CONV_AUTO: more sources (8 or more) use the tensor cores
-bool conv_on_tensor(const ckks_ctx *ctx, int sources);
+enum ConvKind { kConvInteger = 0, kConvTensor = 1, kConvFolded = 2 };
+ConvKind conv_kind(const ckks_ctx *ctx, int sources);
+int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
+int launch_conv_fold_down(ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);
 int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::vector<u64> &dn_mat);
 int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
 int launch_conv_tc_down(const ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);

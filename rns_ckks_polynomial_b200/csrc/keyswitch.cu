@@ -240,7 +240,10 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
                            T.L, T.LK, T.alpha, T.dnum, batch, T.L * batch};
         CKKS_TRY(launch_ntt_inv(j, T, s));
     }
-    if (conv_on_tensor(ctx, T.alpha)) {
+    const ConvKind ck = conv_kind(ctx, T.alpha);
+    if (ck == kConvFolded) {
+        CKKS_TRY(launch_conv_fold_up(const_cast<ckks_ctx *>(ctx), y, digits, batch, s));
+    } else if (ck == kConvTensor) {
         CKKS_TRY(launch_conv_tc_up(ctx, y, digits, batch, s));
     } else {
         UpConvMap m{y, digits, T.up_mat, T.L, T.LK, T.alpha, T.dnum};
@@ -461,7 +464,10 @@ int moddown_stage(const ckks_ctx *ctx, const u64 *acc, u64 *out, int jobs, const
     u64 *cvb = c.take<u64>((size_t)jobs2 * T.L * kN);
     DownInttJob ij{acc, zb, T.dn_hatinv, T.pc, T.L, T.K, T.LK, jobs2, T.K * jobs2};
     CKKS_TRY(launch_ntt_inv(ij, T, s));
-    if (conv_on_tensor(ctx, T.K)) {
+    const ConvKind ck = conv_kind(ctx, T.K);
+    if (ck == kConvFolded) {
+        CKKS_TRY(launch_conv_fold_down(const_cast<ckks_ctx *>(ctx), zb, cvb, jobs2, s));
+    } else if (ck == kConvTensor) {
         CKKS_TRY(launch_conv_tc_down(ctx, zb, cvb, jobs2, s));
     } else {
         DownConvMap m{zb, cvb, T.dn_mat, T.L, T.K};
