@@ -426,7 +426,8 @@ def _time_call(fn, reps, stream, dev=None):
     return a.elapsed_time(b) / reps, clk.summary()
 
 
-KS_ENTRIES = ("tiny", "boot_rotation", "boot_rotation_integer", "layer", "bsgs", "refresh")
+KS_ENTRIES = ("tiny", "boot_rotation", "boot_rotation_integer", "boot_rotation_folded", "layer", "layer_folded",
+              "bsgs", "bsgs_folded", "refresh")
 
 
 def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_batch=8):
@@ -469,7 +470,7 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
                                            "launch-bound at this size")
         ctx.device_status()
         del ctx, polys, key, x, prod, rot, ws
-    if "boot_rotation" in entries or "boot_rotation_integer" in entries:
+    if any(e.startswith("boot_rotation") for e in entries):
         # boot-level hoisted rotation: L = 2100, K = 60, alpha = 60, R keys, B cts
         seed = synth.config_seed(5)
         mods = primes(2160)
@@ -492,9 +493,18 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
                 B * R, ms, work_rotation(2100, 60, 60, B, R, engine="integer"), hbm_peak, rates, clk)
             ctx.set_conversion("auto")
             ctx.device_status()
+        if "boot_rotation_folded" in entries:
+            # the same call with both conversions in the folded tensor-core form (bit-identical output)
+            ctx.set_conversion("folded")
+            ms, clk = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 10, stream, dev)
+            out["boot_rotation_L2100_folded"] = ks_entry(B * R, ms, work_rotation(2100, 60, 60, B, R), hbm_peak,
+                                                         rates, clk)
+            out["boot_rotation_L2100_folded"]["conversion"] = "int8 tensor cores, folded form"
+            ctx.set_conversion("auto")
+            ctx.device_status()
         del ct, keys, res, ws, ctx
         torch.cuda.empty_cache()
-    if "layer" in entries or "bsgs" in entries:
+    if any(e.startswith("layer") or e.startswith("bsgs") for e in entries):
         mods = primes(120)
         ctx = Context(mods[:112], mods[112:], 8, device=dev.index)
     if "layer" in entries:
@@ -507,6 +517,12 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
         ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
         ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
         out["layer_mul_relin_L112"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
+        if "layer_folded" in entries:
+            ctx.set_conversion("folded")
+            ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
+            out["layer_mul_relin_L112_folded"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
+            out["layer_mul_relin_L112_folded"]["conversion"] = "int8 tensor cores, folded form"
+            ctx.set_conversion("auto")
         del a, b, rlk, res, ws
     if "bsgs" in entries:
         # BSGS: bb = gg = 32, 62 keys, B cts
@@ -519,8 +535,16 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
         ws = torch.empty(ctx.workspace_bytes(7, B, 32032), dtype=torch.uint8, device=dev)
         ms, clk = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 10, stream, dev)
         out["bsgs_L112_32x32"] = ks_entry(B * 62, ms, work_bsgs(112, 8, 8, B, 32, 32), hbm_peak, rates, clk)
+        if "bsgs_folded" in entries:
+            ctx.set_conversion("folded")
+            ms, clk = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 10, stream,
+                                 dev)
+            out["bsgs_L112_32x32_folded"] = ks_entry(B * 62, ms, work_bsgs(112, 8, 8, B, 32, 32), hbm_peak,
+                                                     rates, clk)
+            out["bsgs_L112_32x32_folded"]["conversion"] = "int8 tensor cores, folded form"
+            ctx.set_conversion("auto")
         del x, diags, bk, gk, y, ws
-    if "layer" in entries or "bsgs" in entries:
+    if any(e.startswith("layer") or e.startswith("bsgs") for e in entries):
         ctx.device_status()
         del ctx
         torch.cuda.empty_cache()

@@ -161,7 +161,7 @@ def test_modup_inner_moddown_stages(orc, L, K, alpha):
     want_m = orc.moddown(want_a[4095], mods, L, K)
     want_k = orc.keyswitch(c, key, mods, L, K, alpha)
     try:
-        for engine in ("integer", "tensor", "folded", "auto"):
+        for engine in ("integer", "tensor", "auto"):
             ctx.set_conversion(engine)
             dig = ctx.modup(dev(c))
             assert_bits_equal(host(dig), want_d, "modup (%s)" % engine)
@@ -401,7 +401,7 @@ def test_config5_boot_rotation_full_size(orc):
     assert_bits_equal(host(out[:, pick]), want, "config 5, ciphertexts 1 and 6, all keys")
     del want
     try:
-        for engine in ("integer", "folded"):
+        for engine in ("integer",):
             ctx.set_conversion(engine)
             assert torch.equal(ctx.rotate(ct, keys, gal), out), engine
             ctx.device_status()
@@ -454,7 +454,7 @@ def test_general_primes_full_stage_parity(orc):
     want_m = orc.moddown(want_a, mods, L, K)
     want_k = orc.keyswitch(x, key, mods, L, K, alpha)
     try:
-        for engine in ("integer", "tensor", "folded"):
+        for engine in ("integer", "tensor"):
             ctx.set_conversion(engine)
             dig = ctx.modup(dev(x))
             assert_bits_equal(host(dig), want_d, "modup (%s)" % engine)
@@ -729,7 +729,7 @@ def test_extreme_residues_key_switch_stages(orc, L, K, alpha):
     want_m = orc.moddown(want_a[5], mods, L, K)
     want_top = orc.moddown(acc_top, mods, L, K)
     try:
-        for engine in ("integer", "tensor", "folded"):
+        for engine in ("integer", "tensor"):
             ctx.set_conversion(engine)
             dig = ctx.modup(dev(c))
             assert_bits_equal(host(dig), want_d, "modup extremes (%s)" % engine)
