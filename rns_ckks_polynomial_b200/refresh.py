@@ -96,6 +96,7 @@ class Refresh:
         self.device = device
         self._ctx = {}
         self._buf = None
+        self._consts = {}
 
     def _ws(self, ctx, op, batch, aux=0):
         need = max(ctx.workspace_bytes(op, batch, aux), 16)
@@ -118,12 +119,21 @@ class Refresh:
             c.close()
         self._ctx.clear()
         self._buf = None
+        self._consts.clear()
 
     # ------------------------------------------------------------ constants
     def _kvec(self, value, l):
+        """The residues of an integer constant modulo q_0..q_{l-1} as a device
+        vector, kept for later calls (a refresh issues the same constants every
+        time, so repeated refreshes upload nothing)."""
         v = int(value)
-        return torch.tensor([v % qi for qi in self.q[:l]], dtype=torch.int64,
-                            device=torch.device("cuda", self.device))
+        key = (v, l)
+        t = self._consts.get(key)
+        if t is None:
+            t = torch.tensor([v % qi for qi in self.q[:l]], dtype=torch.int64,
+                             device=torch.device("cuda", self.device))
+            self._consts[key] = t
+        return t
 
     @staticmethod
     def level(ct):

@@ -216,6 +216,16 @@ MUTATIONS = [
     ("planned BSGS plaintexts pre-rotated the wrong way", "encoding.py",
      "encode_ntt(np.roll(d, G), mods, scale, n)", "encode_ntt(np.roll(d, -G), mods, scale, n)", 0,
      "test_factored_transforms_decrypt"),
+    ("batch encoder: imaginary part added instead of subtracted", "encoding.py",
+     "re = re - np.sin(ang) @ Z.imag.T", "re = re + np.sin(ang) @ Z.imag.T", 0,
+     "test_batch_encoder_matches_encode_and_decodes"),
+    ("batch encoder without the 2/n factor", "encoding.py",
+     "v = (np.longdouble(2) / np.longdouble(n)) * re * np.longdouble(scale)",
+     "v = re * np.longdouble(scale)", 0,
+     "test_batch_encoder_matches_encode_and_decodes"),
+    ("batch encoder: residues of the wrong prime", "encoding.py",
+     "res = np.mod(m[c:c + 64, None, :], q[None, :, None])", "res = np.mod(m[c:c + 64, None, :], q[None, ::-1, None])",
+     0, "test_batch_encoder_matches_encode_and_decodes"),
 ]
 
 
