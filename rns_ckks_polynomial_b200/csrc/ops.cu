@@ -711,7 +711,7 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
     if (kind < 0 || kind > 5 || blocks < 1 || blocks > 148 * 64 || iters < 1 || !ms || !ops)
         return set_error(CKKS_EINVAL, "bad microbenchmark arguments");
     CKKS_TRY(set_device(ctx));
-    if (kind >= 3) return bench_mma(ctx, kind == 3 ? 256 : 32, blocks, iters, ms, ops);
+    if (kind == 3 || kind == 4) return bench_mma(ctx, kind == 3 ? 256 : 32, blocks, iters, ms, ops);
     const u64 q = ctx->mods[0];
     const u64 w = 0x0123456789abcdefull % q, wp = host_shoup(w, q);
     u64 *sink = nullptr;
