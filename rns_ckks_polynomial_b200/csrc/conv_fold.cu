@@ -22,14 +22,17 @@
 //  - accumulator P_u takes columns 32 u .. 32 u + 31.
 // Warp roles, synchronised by mbarriers only:
 //  - 4 MMA warps (one elected lane each) own planes {2k, 2k+1}: for tile i they wait until its data
-//    is staged and the epilogue has read their planes of tile i - 1, issue the ceil(S / 4) K-steps
-//    of each plane and commit each plane to its own barrier;
-//  - 16 epilogue / staging warps: for tile i they read P_0 .. P_7 as each completes (releasing it to
-//    the next tile's products at once), rebuild and reduce the 32 x 128 outputs and store them, then
-//    write the prefetched words of tile i + 2 into the data buffer tile i used (free once all eight
-//    planes of tile i are complete) and prefetch tile i + 3.  Warp w reads TMEM lane quadrant w & 3
-//    (coefficients 32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight
-//    targets of one coefficient; for staging it owns sources 16 (w >> 2) .. 16 (w >> 2) + 15.
+//    is staged and the epilogue has read their plane group (P_0..P_3 or P_4..P_7) of tile i - 1,
+//    issue the ceil(S / 4) K-steps of both planes and commit once;
+//  - 16 epilogue / staging warps: for tile i they read plane group 0 as soon as it completes and
+//    release it (the next tile's products into it can start), fold it to the low 50 bits of each
+//    sum; wait for group 1, then write the prefetched words of tile i + 2 into the data buffer tile
+//    i used (every product of tile i is complete by then), read and release group 1, rebuild each
+//    (< 2^83) sum, reduce it once and store it, and prefetch tile i + 3.  Warp w reads TMEM lane
+//    quadrant w & 3 (coefficients 32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each
+//    plane: eight targets of one coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
+// Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
+// 2^60 - delta (delta < 2^28) that is a shift, a 32 x 32 product and one conditional subtraction.
 //
 // Every mbarrier wait is bounded: on expiry a thread records an error flag and leaves its loop, the
 // MMA warps wait (bounded again) for the products they issued, the CTA frees its tensor memory and
@@ -53,7 +56,7 @@ constexpr int kFAcol = 256;                       // first data-buffer column
 constexpr int kFSmemBar = kFBlock;
 constexpr int kFSmemBytes = kFBlock + 256;
 
-enum { kFBarMma = 0, kFBarFree = 8, kFBarFull = 16, kFBarDrain = 18, kFNumBars = 19 };
+enum { kFBarMma = 0, kFBarFree = 4, kFBarFull = 6, kFBarDrain = 8, kFNumBars = 9 };
 static_assert(kFSmemBar + 8 * kFNumBars + 4 <= kFSmemBytes, "shared-memory layout");
 
 __host__ __device__ __forceinline__ int fcm_off(int row, int k)
@@ -117,48 +120,22 @@ __device__ __forceinline__ void fbar_arrive(uint64_t *bar)
 __device__ __forceinline__ void ffence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void ffence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Eight columns of one accumulator plane for the warp's 32 lanes.
-__device__ __forceinline__ void fld8(uint32_t taddr, uint32_t (&r)[8])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7])
-                 : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// 32 columns (16 source words) of the data operand for the warp's 32 lanes.
+// 32 columns (16 source words) of the data operand for the warp's 32 lanes, as two stores of 16.
 __device__ __forceinline__ void fst32(uint32_t taddr, const u64 (&v)[16])
 {
-    uint32_t r[32];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        r[2 * k] = (uint32_t)v[k];
-        r[2 * k + 1] = (uint32_t)(v[k] >> 32);
+    for (int h = 0; h < 2; ++h) {
+        const u64 *w = v + 8 * h;
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16};"
+            :: "r"(taddr + 16 * h), "r"((uint32_t)w[0]), "r"((uint32_t)(w[0] >> 32)), "r"((uint32_t)w[1]),
+               "r"((uint32_t)(w[1] >> 32)), "r"((uint32_t)w[2]), "r"((uint32_t)(w[2] >> 32)), "r"((uint32_t)w[3]),
+               "r"((uint32_t)(w[3] >> 32)), "r"((uint32_t)w[4]), "r"((uint32_t)(w[4] >> 32)), "r"((uint32_t)w[5]),
+               "r"((uint32_t)(w[5] >> 32)), "r"((uint32_t)w[6]), "r"((uint32_t)(w[6] >> 32)), "r"((uint32_t)w[7]),
+               "r"((uint32_t)(w[7] >> 32))
+            : "memory");
     }
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-           "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-           "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-           "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-// x = hi 2^64 + lo (x < 2^126) mod q for q = 2^60 - delta, delta < 2^28 (2^60 = delta mod q).
-__device__ __forceinline__ u64 freduce_special(u64 hi, u64 lo, u64 delta, u64 q)
-{
-    constexpr u64 kMask60 = ((u64)1 << 60) - 1;
-    const uint32_t c16 = (uint32_t)delta << 4;
-    const u64 p0 = (u64)(uint32_t)hi * c16, p1 = (u64)(uint32_t)(hi >> 32) * c16;
-    const u64 t = p0 + (p1 << 32);
-    const u64 yl = t + lo;
-    const u64 yh = (p1 >> 32) + (t < p0) + (yl < t);
-    const u64 a = (yh << 4) | (yl >> 60);
-    const u64 z = (yl & kMask60) + a * delta;
-    const u64 w = (z & kMask60) + (z >> 60) * delta;
-    return w >= q ? w - q : w;
 }
 
 // Job geometry (kind 0: ModUp over (ciphertext, digit), the ciphertext fastest in the grid so the
@@ -200,6 +177,38 @@ struct FoldJobs {
     }
 };
 
+// x = lo + hi 2^64 < 2^82 mod q for q = 2^60 - delta, delta < 2^28: x = a 2^60 + b with
+// a < 2^22, and 2^60 = delta (mod q), so x = a delta + b < 2^60 + 2^50 < 2q.
+__device__ __forceinline__ u64 freduce82(u64 hi, u64 lo, uint32_t delta)
+{
+    constexpr u64 kMask60 = ((u64)1 << 60) - 1;
+    const uint32_t a = (uint32_t)(lo >> 60) | (uint32_t)(hi << 4);
+    const u64 w = (lo & kMask60) + (u64)a * delta;
+    const u64 q = ((u64)1 << 60) - delta;
+    return w >= q ? w - q : w;
+}
+
+// p0 + p1 2^8 + p2 2^16 + p3 2^24 (each p < 2^25, sum < 2^50).
+__device__ __forceinline__ u64 ffold4(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3)
+{
+    const u64 a = (u64)p1 * 256u + p0, b = (u64)p3 * 256u + p2;
+    return a + (b << 16);
+}
+
+// Four planes (P_g4 .. P_g4+3) x four columns of the warp's lanes, one wait for all loads.
+__device__ __forceinline__ void fld4x4(uint32_t taddr, uint32_t (&r)[4][4])
+{
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(r[u][0]), "=r"(r[u][1]), "=r"(r[u][2]), "=r"(r[u][3])
+                     : "r"(taddr + u * kFN));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Barriers: kFBarMma + k (k < 4) completes when MMA warp k's planes 2k, 2k+1 of a tile are done;
+// kFBarFree + g (g < 2) when the epilogue has read plane group g (planes 4g .. 4g+3) of a tile;
+// kFBarFull + b when data buffer b is staged; kFBarDrain when every issued product is done.
 template <bool kSpecial>
 __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, const PrimeConst *__restrict__ pc,
                                                                   int *err)
@@ -226,10 +235,9 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
-        for (int u = 0; u < kFPlanes; ++u) {
-            fbar_init(bar + kFBarMma + u, 1);
-            fbar_init(bar + kFBarFree + u, kFEpiThreads);
-        }
+        for (int k = 0; k < 4; ++k) fbar_init(bar + kFBarMma + k, 1);
+        fbar_init(bar + kFBarFree + 0, kFEpiThreads);
+        fbar_init(bar + kFBarFree + 1, kFEpiThreads);
         fbar_init(bar + kFBarFull + 0, kFEpiThreads);
         fbar_init(bar + kFBarFull + 1, kFEpiThreads);
         fbar_init(bar + kFBarDrain, 4);
@@ -245,10 +253,10 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
     };
     u64 pre[16];
     if (!mma_warp) {
+        fetch(0, pre);
         const uint4 *src = reinterpret_cast<const uint4 *>(fbase + (size_t)tb * kFBlock);
         uint4 *dst = reinterpret_cast<uint4 *>(sm);
         for (int i = tid; i < kFBlock / 16; i += kFEpiThreads) dst[i] = __ldg(src + i);
-        fetch(0, pre);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     ffence_before();
@@ -261,23 +269,25 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
     if (mma_warp) {
         // ------------------------------------------------ MMA issue (one elected lane per warp)
         const u64 bdesc0 = fsmem_desc(smem_u32(sm));
+        const int grp = issuer >> 1;  // plane group read back together by the epilogue
         for (int i = 0; i < ntiles && ok; ++i) {
             const int buf = i & 1;
             ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFull + buf, (i >> 1) & 1));
-            for (int h = 0; h < 2 && ok; ++h) {
-                const int u = 2 * issuer + h;
-                if (i > 0) ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFree + u, (i - 1) & 1));
-                if (!ok) break;
-                ffence_after();
-                if (lane == 0) {
+            if (ok && i > 0) ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFree + grp, (i - 1) & 1));
+            if (!ok) break;
+            ffence_after();
+            if (lane == 0) {
+                const uint32_t ta = tmem + kFAcol + buf * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int u = 2 * issuer + h;
                     const u64 bd = bdesc0 + (((size_t)u * kFPlaneBytes) >> 4);
-                    const uint32_t ta = tmem + kFAcol + buf * 128;
                     for (int ks = 0; ks < nks; ++ks)
                         mma_ts(tmem + u * kFN, ta + ks * 8, bd + ((ks * 256) >> 4), ks > 0 ? 1u : 0u);
-                    fcommit(bar + kFBarMma + u);
                 }
-                __syncwarp();
+                fcommit(bar + kFBarMma + issuer);
             }
+            __syncwarp();
         }
         // every product issued here has completed before tensor memory is freed (bounded)
         if (lane == 0) fcommit(bar + kFBarDrain);
@@ -295,58 +305,64 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         ffence_before();
         fbar_arrive(bar + kFBarFull + 0);
         fbar_arrive(bar + kFBarFull + 1);
-        if (ntiles > 2) fetch(2, pre);
-        // the eight targets of this thread: tb * 32 + part * 8 + c
-        int tcol[8];
-        bool tvalid[8];
+        // the eight targets of this thread: tb * 32 + part * 8 + c (an invalid one has trow = -1)
+        int trow[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const int ti = tb * kFN + part * 8 + c;
-            tvalid[c] = ti < T;
-            tcol[c] = tvalid[c] ? jobs.prime(ti, lo, S) : 0;
+            trow[c] = ti < T ? jobs.prime(ti, lo, S) : -1;
         }
+        const uint32_t tcol = tmem + lane_base + part * 8;
         for (int i = 0; i < ntiles; ++i) {
-            u64 g0[8], g1[8];
+            // plane group 0 (P_0 .. P_3): the low 50 bits of each sum
+            ok = fbar_wait(bar + kFBarMma + 0, i & 1) && ok;
+            ok = fbar_wait(bar + kFBarMma + 1, i & 1) && ok;
+            ffence_after();
+            u64 g0[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) g0[c] = g1[c] = 0;
+            for (int hc = 0; hc < 2; ++hc) {
+                uint32_t r[4][4];
+                fld4x4(tcol + 4 * hc, r);
 #pragma unroll
-            for (int u = 0; u < kFPlanes; ++u) {
-                ok = fbar_wait(bar + kFBarMma + u, i & 1) && ok;
-                ffence_after();
-                uint32_t r[8];
-                fld8(tmem + lane_base + u * kFN + part * 8, r);
-                ffence_before();
-                fbar_arrive(bar + kFBarFree + u);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (u < 4)
-                        g0[c] += (u64)r[c] << (8 * u);
-                    else
-                        g1[c] += (u64)r[c] << (8 * (u - 4));
-                }
+                for (int c = 0; c < 4; ++c) g0[4 * hc + c] = ffold4(r[0][c], r[1][c], r[2][c], r[3][c]);
             }
-            // all eight planes of tile i are complete: its data buffer takes tile i + 2
+            ffence_before();
+            fbar_arrive(bar + kFBarFree + 0);
+            // the words of tile i + 2 load while the products of tile i finish
+            if (i + 2 < ntiles && ok) fetch(i + 2, pre);
+            // plane group 1 (P_4 .. P_7): all products of tile i are then complete, so its data
+            // buffer takes tile i + 2 at once
+            ok = fbar_wait(bar + kFBarMma + 2, i & 1) && ok;
+            ok = fbar_wait(bar + kFBarMma + 3, i & 1) && ok;
+            ffence_after();
             if (i + 2 < ntiles && ok) {
                 fst32(tmem + lane_base + kFAcol + (i & 1) * 128 + part * 32, pre);
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 ffence_before();
                 fbar_arrive(bar + kFBarFull + (i & 1));
-                if (i + 3 < ntiles) fetch(i + 3, pre);
             }
-            if (ok) {
-                const int coef = cbase + i * kFM + m;
+            const int coef = cbase + i * kFM + m;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (!tvalid[c]) continue;
-                    const u64 lo64 = g0[c] + (g1[c] << 32);
-                    const u64 hi64 = (g1[c] >> 32) + (lo64 < g0[c]);
-                    const PrimeConst &p = pc[tcol[c]];
+            for (int hc = 0; hc < 2; ++hc) {
+                uint32_t r[4][4];
+                fld4x4(tcol + 4 * kFN + 4 * hc, r);
+                if (hc == 1) {
+                    ffence_before();
+                    fbar_arrive(bar + kFBarFree + 1);
+                }
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int c = 4 * hc + cc;
+                    const u64 g1 = ffold4(r[0][cc], r[1][cc], r[2][cc], r[3][cc]);
+                    const u64 lo64 = g0[c] + (g1 << 32);
+                    const u64 hi64 = (g1 >> 32) + (lo64 < g0[c]);
+                    if (trow[c] < 0 || !ok) continue;
                     u64 res;
                     if constexpr (kSpecial)
-                        res = freduce_special(hi64, lo64, p.delta, p.q);
+                        res = freduce82(hi64, lo64, (uint32_t)pc[trow[c]].delta);
                     else
-                        res = reduce128(hi64, lo64, p);
-                    jobs.row(zrow, tcol[c])[coef] = res;
+                        res = reduce128(hi64, lo64, pc[trow[c]]);
+                    jobs.row(zrow, trow[c])[coef] = res;
                 }
             }
             if (!ok) break;
