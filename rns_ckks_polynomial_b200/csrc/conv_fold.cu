@@ -17,20 +17,24 @@
 // for a run of coefficient tiles of 128 (the MMA's M, the TMEM lanes):
 //  - the block's eight F planes (8 x 32 targets x 512 bytes = 128 KiB) stay in shared memory (the B
 //    operand, K-major core matrices) for the whole run;
-//  - the data tile (128 coefficients x S words) is the A operand in tensor memory, double-buffered
-//    (columns 256..383 and 384..511, two 32-bit columns per source);
+//  - a data tile (S source rows of 128 words, contiguous 1 KiB each in global memory) arrives in a
+//    64 KiB shared-memory buffer by S bulk copies that complete on an mbarrier, so no thread waits on
+//    a global load for it; the staging threads move it (transposed: one coefficient per TMEM lane)
+//    into the A operand in tensor memory, double-buffered (columns 256..383 and 384..511, two 32-bit
+//    columns per source);
 //  - accumulator P_u takes columns 32 u .. 32 u + 31.
-// Warp roles, synchronised by mbarriers only:
+// Warp roles (20 warps, so that 96 registers fit), synchronised by mbarriers only:
 //  - 4 MMA warps (one elected lane each) own planes {2k, 2k+1}: for tile i they wait until its data
 //    is staged and the epilogue has read their plane group (P_0..P_3 or P_4..P_7) of tile i - 1,
 //    issue the ceil(S / 4) K-steps of both planes and commit once;
 //  - 16 epilogue / staging warps: for tile i they read plane group 0 as soon as it completes and
-//    release it (the next tile's products into it can start), fold it to the low 50 bits of each
-//    sum; wait for group 1, then write the prefetched words of tile i + 2 into the data buffer tile
-//    i used (every product of tile i is complete by then), read and release group 1, rebuild each
-//    (< 2^83) sum, reduce it once and store it, and prefetch tile i + 3.  Warp w reads TMEM lane
-//    quadrant w & 3 (coefficients 32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each
-//    plane: eight targets of one coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
+//    release it (the next tile's products into it can start) and fold it to the low 50 bits of each
+//    sum; wait for group 1, then stage tile i + 2 from shared memory into the data buffer tile i
+//    used (every product of tile i is complete by then); read and release group 1, rebuild each
+//    (< 2^83) sum, reduce it once and store it.  Thread 0 issues the bulk copies of tile t + 1 once
+//    every staging thread has read tile t.  Warp w reads TMEM lane quadrant w & 3 (coefficients
+//    32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight targets of one
+//    coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
 // Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
 // 2^60 - delta (delta < 2^28) that is a shift, a 32 x 32 product and one conditional subtraction.
 //
@@ -50,14 +54,20 @@ constexpr int kFPlaneBytes = kFN * kFKP;          // 16 KiB
 constexpr int kFBlock = kFPlanes * kFPlaneBytes;  // 128 KiB per block of 32 targets
 constexpr int kFSbo = (kFKP / 16) * 128;          // 8-row-group stride of the core-matrix layout
 constexpr int kFEpiWarps = 16, kFEpiThreads = 32 * kFEpiWarps;
-constexpr int kFThreads = kFEpiThreads + 128;
+constexpr int kFMmaWarp0 = kFEpiWarps;
+constexpr int kFThreads = kFEpiThreads + 128;  // 20 warps: at most 5 per SM partition keeps 96 registers
 constexpr int kFTmemCols = 512;
 constexpr int kFAcol = 256;                       // first data-buffer column
-constexpr int kFSmemBar = kFBlock;
-constexpr int kFSmemBytes = kFBlock + 256;
+constexpr int kFRowBytes = kFM * 8;               // one source row of a data tile: 1 KiB
+constexpr int kFSmemY = kFBlock;                  // data tile staged by bulk copies: 64 rows x 1 KiB
+constexpr int kFSmemDelta = kFSmemY + 64 * kFRowBytes;  // 32 target deltas (2^60 - q)
+constexpr int kFSmemBar = kFSmemDelta + 32 * 4;
+constexpr int kFSmemBytes = kFSmemBar + 256;
 
-enum { kFBarMma = 0, kFBarFree = 4, kFBarFull = 6, kFBarDrain = 8, kFNumBars = 9 };
+enum { kFBarMma = 0, kFBarFree = 4, kFBarFull = 6, kFBarDrain = 8, kFBarYFull = 9, kFBarYFree = 10,
+       kFNumBars = 11 };
 static_assert(kFSmemBar + 8 * kFNumBars + 4 <= kFSmemBytes, "shared-memory layout");
+static_assert(kFSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 __host__ __device__ __forceinline__ int fcm_off(int row, int k)
 {
@@ -115,6 +125,21 @@ __device__ __forceinline__ void fbar_arrive(uint64_t *bar)
 {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" :: "r"(smem_u32(bar))
                  : "memory");
+}
+
+__device__ __forceinline__ void fbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+                 :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// Bulk copy (no tensor map, no multicast) of `bytes` from this GPU's global memory into this CTA's
+// shared memory, completing as transaction bytes on `bar`.  Both addresses 16-byte aligned, size a
+// multiple of 16.
+__device__ __forceinline__ void fbulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void ffence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -208,7 +233,9 @@ __device__ __forceinline__ void fld4x4(uint32_t taddr, uint32_t (&r)[4][4])
 
 // Barriers: kFBarMma + k (k < 4) completes when MMA warp k's planes 2k, 2k+1 of a tile are done;
 // kFBarFree + g (g < 2) when the epilogue has read plane group g (planes 4g .. 4g+3) of a tile;
-// kFBarFull + b when data buffer b is staged; kFBarDrain when every issued product is done.
+// kFBarFull + b when tensor-memory data buffer b is staged; kFBarYFull when a tile's words have
+// landed in shared memory; kFBarYFree when the staging threads have read them; kFBarDrain when
+// every issued product is done.
 template <bool kSpecial>
 __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, const PrimeConst *__restrict__ pc,
                                                                   int *err)
@@ -226,8 +253,8 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
     const int nks = (S + 3) >> 2;                // K-steps of 32 bytes (4 sources)
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kFSmemBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kFSmemBar + 8 * kFNumBars);
-    const bool mma_warp = warp >= kFEpiWarps;
-    const int issuer = warp - kFEpiWarps;  // planes 2 issuer, 2 issuer + 1
+    const u64 *ys = reinterpret_cast<const u64 *>(sm + kFSmemY);
+    uint32_t *dsm = reinterpret_cast<uint32_t *>(sm + kFSmemDelta);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -241,33 +268,29 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         fbar_init(bar + kFBarFull + 0, kFEpiThreads);
         fbar_init(bar + kFBarFull + 1, kFEpiThreads);
         fbar_init(bar + kFBarDrain, 4);
+        fbar_init(bar + kFBarYFull, 1);
+        fbar_init(bar + kFBarYFree, kFEpiThreads);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // staging share: coefficient m of each tile, sources s0 .. s0 + 15
-    const int quad = warp & 3, part = warp >> 2;
-    const int m = quad * 32 + lane, s0 = part * 16;
-    const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + m;
-    auto fetch = [&](int i, u64 (&v)[16]) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? __ldg(ysrc + (size_t)k * kN + i * kFM) : 0;
-    };
-    u64 pre[16];
-    if (!mma_warp) {
-        fetch(0, pre);
+    if (warp < kFEpiWarps) {
         const uint4 *src = reinterpret_cast<const uint4 *>(fbase + (size_t)tb * kFBlock);
         uint4 *dst = reinterpret_cast<uint4 *>(sm);
         for (int i = tid; i < kFBlock / 16; i += kFEpiThreads) dst[i] = __ldg(src + i);
+        if (tid < kFN) {
+            const int ti = tb * kFN + tid;
+            dsm[tid] = ti < T ? (uint32_t)pc[jobs.prime(ti, lo, S)].delta : 0u;
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     ffence_before();
     __syncthreads();
     ffence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     bool ok = true;
 
-    if (mma_warp) {
+    if (warp >= kFMmaWarp0) {
         // ------------------------------------------------ MMA issue (one elected lane per warp)
+        const int issuer = warp - kFMmaWarp0;  // planes 2 issuer, 2 issuer + 1
         const u64 bdesc0 = fsmem_desc(smem_u32(sm));
         const int grp = issuer >> 1;  // plane group read back together by the epilogue
         for (int i = 0; i < ntiles && ok; ++i) {
@@ -295,16 +318,47 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         ok = fbar_wait(bar + kFBarDrain, 0) && ok;
     } else {
         // ------------------------------------------------ epilogue and staging
-        // tile 0 into buffer 0, tile 1 into buffer 1
-        fst32(tmem + lane_base + kFAcol + 0 * 128 + part * 32, pre);
-        if (ntiles > 1) {
-            fetch(1, pre);
-            fst32(tmem + lane_base + kFAcol + 1 * 128 + part * 32, pre);
+        const int quad = warp & 3, part = warp >> 2;
+        const int m = quad * 32 + lane, s0 = part * 16;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        // Thread 0 issues the bulk copies of tile t (S source rows of 1 KiB) into the one shared
+        // staging buffer once every staging thread has read tile t - 1 from it.
+        const u64 *ysrc = ybase + cbase;
+        auto issue = [&](int t) {
+            fbar_expect_tx(bar + kFBarYFull, (uint32_t)S * kFRowBytes);
+            for (int s2 = 0; s2 < S; ++s2)
+                fbulk_g2s(sm + kFSmemY + s2 * kFRowBytes, ysrc + (size_t)s2 * kN + t * kFM, kFRowBytes,
+                          bar + kFBarYFull);
+        };
+        int issued = 0;  // thread 0: tiles whose copies are in flight or done
+        // tile t's words: shared memory -> tensor-memory buffer t & 1 (the caller knows it is free)
+        auto stage = [&](int t) -> bool {
+            bool good = __all_sync(0xffffffffu, fbar_wait(bar + kFBarYFull, t & 1));
+            u64 v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? ys[(s0 + k) * kFM + m] : 0;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fbar_arrive(bar + kFBarYFree);
+            if (tid == 0 && good && t + 1 < ntiles) {
+                good = fbar_wait(bar + kFBarYFree, t & 1);
+                if (good) {
+                    issue(t + 1);
+                    ++issued;
+                }
+            }
+            good = __all_sync(0xffffffffu, good);
+            fst32(tmem + lane_base + kFAcol + (t & 1) * 128 + part * 32, v);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            ffence_before();
+            fbar_arrive(bar + kFBarFull + (t & 1));
+            return good;
+        };
+        if (tid == 0) {
+            issue(0);
+            issued = 1;
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        ffence_before();
-        fbar_arrive(bar + kFBarFull + 0);
-        fbar_arrive(bar + kFBarFull + 1);
+        ok = stage(0);
+        if (ok && ntiles > 1) ok = stage(1);
         // the eight targets of this thread: tb * 32 + part * 8 + c (an invalid one has trow = -1)
         int trow[8];
 #pragma unroll
@@ -313,10 +367,11 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             trow[c] = ti < T ? jobs.prime(ti, lo, S) : -1;
         }
         const uint32_t tcol = tmem + lane_base + part * 8;
-        for (int i = 0; i < ntiles; ++i) {
+        for (int i = 0; i < ntiles && ok; ++i) {
             // plane group 0 (P_0 .. P_3): the low 50 bits of each sum
             ok = fbar_wait(bar + kFBarMma + 0, i & 1) && ok;
             ok = fbar_wait(bar + kFBarMma + 1, i & 1) && ok;
+            ok = __all_sync(0xffffffffu, ok);  // warp-uniform: the loads below are warp-collective
             ffence_after();
             u64 g0[8];
 #pragma unroll
@@ -328,19 +383,13 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             }
             ffence_before();
             fbar_arrive(bar + kFBarFree + 0);
-            // the words of tile i + 2 load while the products of tile i finish
-            if (i + 2 < ntiles && ok) fetch(i + 2, pre);
             // plane group 1 (P_4 .. P_7): all products of tile i are then complete, so its data
             // buffer takes tile i + 2 at once
             ok = fbar_wait(bar + kFBarMma + 2, i & 1) && ok;
             ok = fbar_wait(bar + kFBarMma + 3, i & 1) && ok;
+            ok = __all_sync(0xffffffffu, ok);
             ffence_after();
-            if (i + 2 < ntiles && ok) {
-                fst32(tmem + lane_base + kFAcol + (i & 1) * 128 + part * 32, pre);
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                ffence_before();
-                fbar_arrive(bar + kFBarFull + (i & 1));
-            }
+            if (i + 2 < ntiles && ok) ok = stage(i + 2);
             const int coef = cbase + i * kFM + m;
 #pragma unroll
             for (int hc = 0; hc < 2; ++hc) {
@@ -359,14 +408,15 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
                     if (trow[c] < 0 || !ok) continue;
                     u64 res;
                     if constexpr (kSpecial)
-                        res = freduce82(hi64, lo64, (uint32_t)pc[trow[c]].delta);
+                        res = freduce82(hi64, lo64, dsm[part * 8 + c]);
                     else
                         res = reduce128(hi64, lo64, pc[trow[c]]);
                     jobs.row(zrow, trow[c])[coef] = res;
                 }
             }
-            if (!ok) break;
         }
+        // every copy thread 0 issued has landed before the CTA exits (bounded)
+        if (tid == 0 && issued > 0 && !fbar_wait(bar + kFBarYFull, (issued - 1) & 1)) ok = false;
     }
     if (!ok) atomicExch(err, 1);
     ffence_before();
