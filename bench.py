@@ -936,7 +936,8 @@ def run_ks_only(args):
     ctx.close()
     entries = tuple(e for e in args.ks_entries.split(",") if e)
     print(json.dumps({"keyswitch": run_keyswitch(dev, hbm_peak, ipeak, args.ks_batch, args.ks_keys,
-                                                 entries, refresh_batch=args.ks_batch)}), flush=True)
+                                                 entries, refresh_batch=args.ks_batch),
+                      "intpipe_peaks": ipeak}), flush=True)
 
 
 def main():
