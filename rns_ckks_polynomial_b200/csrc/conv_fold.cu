@@ -17,11 +17,10 @@
 // for a run of coefficient tiles of 128 (the MMA's M, the TMEM lanes):
 //  - the block's eight F planes (8 x 32 targets x 512 bytes = 128 KiB) stay in shared memory (the B
 //    operand, K-major core matrices) for the whole run;
-//  - a data tile (S source rows of 128 words, contiguous 1 KiB each in global memory) arrives in a
-//    64 KiB shared-memory buffer by S bulk copies that complete on an mbarrier, so no thread waits on
-//    a global load for it; the staging threads move it (transposed: one coefficient per TMEM lane)
-//    into the A operand in tensor memory, double-buffered (columns 256..383 and 384..511, two 32-bit
-//    columns per source);
+//  - each staging thread copies its 16 words of the next data tile (cp.async, 8 bytes each) into
+//    its own shared-memory slots one tile ahead, and moves them (one coefficient per TMEM lane) into
+//    the A operand in tensor memory when a buffer frees up: double-buffered, columns 256..383 and
+//    384..511, two 32-bit columns per source;
 //  - accumulator P_u takes columns 32 u .. 32 u + 31.
 // Warp roles (20 warps, so that 96 registers fit), synchronised by mbarriers only:
 //  - 4 MMA warps (one elected lane each) own planes {2k, 2k+1}: for tile i they wait until its data
@@ -31,8 +30,7 @@
 //    release it (the next tile's products into it can start) and fold it to the low 50 bits of each
 //    sum; wait for group 1, then stage tile i + 2 from shared memory into the data buffer tile i
 //    used (every product of tile i is complete by then); read and release group 1, rebuild each
-//    (< 2^83) sum, reduce it once and store it.  Thread 0 issues the bulk copies of tile t + 1 once
-//    every staging thread has read tile t.  Warp w reads TMEM lane quadrant w & 3 (coefficients
+//    (< 2^83) sum, reduce it once and store it.  Warp w reads TMEM lane quadrant w & 3 (coefficients
 //    32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight targets of one
 //    coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
 // Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
@@ -58,14 +56,12 @@ constexpr int kFMmaWarp0 = kFEpiWarps;
 constexpr int kFThreads = kFEpiThreads + 128;  // 20 warps: at most 5 per SM partition keeps 96 registers
 constexpr int kFTmemCols = 512;
 constexpr int kFAcol = 256;                       // first data-buffer column
-constexpr int kFRowBytes = kFM * 8;               // one source row of a data tile: 1 KiB
-constexpr int kFSmemY = kFBlock;                  // data tile staged by bulk copies: 64 rows x 1 KiB
-constexpr int kFSmemDelta = kFSmemY + 64 * kFRowBytes;  // 32 target deltas (2^60 - q)
+constexpr int kFSmemY = kFBlock;                  // staging slots: 16 words per epilogue thread (64 KiB)
+constexpr int kFSmemDelta = kFSmemY + 16 * kFEpiThreads * 8;  // 32 target deltas (2^60 - q)
 constexpr int kFSmemBar = kFSmemDelta + 32 * 4;
 constexpr int kFSmemBytes = kFSmemBar + 256;
 
-enum { kFBarMma = 0, kFBarFree = 4, kFBarFull = 6, kFBarDrain = 8, kFBarYFull = 9, kFBarYFree = 10,
-       kFNumBars = 11 };
+enum { kFBarMma = 0, kFBarFree = 4, kFBarFull = 6, kFBarDrain = 8, kFNumBars = 9 };
 static_assert(kFSmemBar + 8 * kFNumBars + 4 <= kFSmemBytes, "shared-memory layout");
 static_assert(kFSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -127,20 +123,15 @@ __device__ __forceinline__ void fbar_arrive(uint64_t *bar)
                  : "memory");
 }
 
-__device__ __forceinline__ void fbar_expect_tx(uint64_t *bar, uint32_t bytes)
+// Asynchronous 8-byte copy from global into this thread's own shared-memory slot (no register
+// holds the word while it is in flight); completion per thread by commit / wait groups.
+__device__ __forceinline__ void fcp8(void *dst, const void *src)
 {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                 :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
-// Bulk copy (no tensor map, no multicast) of `bytes` from this GPU's global memory into this CTA's
-// shared memory, completing as transaction bytes on `bar`.  Both addresses 16-byte aligned, size a
-// multiple of 16.
-__device__ __forceinline__ void fbulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
+__device__ __forceinline__ void fcp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void fcp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void ffence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void ffence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -233,9 +224,8 @@ __device__ __forceinline__ void fld4x4(uint32_t taddr, uint32_t (&r)[4][4])
 
 // Barriers: kFBarMma + k (k < 4) completes when MMA warp k's planes 2k, 2k+1 of a tile are done;
 // kFBarFree + g (g < 2) when the epilogue has read plane group g (planes 4g .. 4g+3) of a tile;
-// kFBarFull + b when tensor-memory data buffer b is staged; kFBarYFull when a tile's words have
-// landed in shared memory; kFBarYFree when the staging threads have read them; kFBarDrain when
-// every issued product is done.
+// kFBarFull + b when tensor-memory data buffer b is staged; kFBarDrain when every issued product
+// is done.
 template <bool kSpecial>
 __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, const PrimeConst *__restrict__ pc,
                                                                   int *err)
@@ -253,7 +243,6 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
     const int nks = (S + 3) >> 2;                // K-steps of 32 bytes (4 sources)
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kFSmemBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kFSmemBar + 8 * kFNumBars);
-    const u64 *ys = reinterpret_cast<const u64 *>(sm + kFSmemY);
     uint32_t *dsm = reinterpret_cast<uint32_t *>(sm + kFSmemDelta);
 
     if (warp == 0) {
@@ -268,8 +257,6 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         fbar_init(bar + kFBarFull + 0, kFEpiThreads);
         fbar_init(bar + kFBarFull + 1, kFEpiThreads);
         fbar_init(bar + kFBarDrain, 4);
-        fbar_init(bar + kFBarYFull, 1);
-        fbar_init(bar + kFBarYFree, kFEpiThreads);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp < kFEpiWarps) {
@@ -321,42 +308,32 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         const int quad = warp & 3, part = warp >> 2;
         const int m = quad * 32 + lane, s0 = part * 16;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        // Thread 0 issues the bulk copies of tile t (S source rows of 1 KiB) into the one shared
-        // staging buffer once every staging thread has read tile t - 1 from it.
-        const u64 *ysrc = ybase + cbase;
+        // Each thread copies its 16 words of a tile (coefficient m, sources s0 .. s0 + 15) into its
+        // own shared-memory slots one tile ahead, so the words are waiting when the tensor-memory
+        // buffer frees up, and no register or other thread is involved while they travel.
+        u64 *slot = reinterpret_cast<u64 *>(sm + kFSmemY) + tid;  // word k at slot[k * 512]
+        const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + m;
         auto issue = [&](int t) {
-            fbar_expect_tx(bar + kFBarYFull, (uint32_t)S * kFRowBytes);
-            for (int s2 = 0; s2 < S; ++s2)
-                fbulk_g2s(sm + kFSmemY + s2 * kFRowBytes, ysrc + (size_t)s2 * kN + t * kFM, kFRowBytes,
-                          bar + kFBarYFull);
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (s0 + k < S) fcp8(slot + k * kFEpiThreads, ysrc + (size_t)k * kN + t * kFM);
+            fcp_commit();
         };
-        int issued = 0;  // thread 0: tiles whose copies are in flight or done
-        // tile t's words: shared memory -> tensor-memory buffer t & 1 (the caller knows it is free)
+        // tile t's words: own slots -> tensor-memory buffer t & 1 (the caller knows it is free); the
+        // copies of tile t + 1 then start into the same slots
         auto stage = [&](int t) -> bool {
-            bool good = __all_sync(0xffffffffu, fbar_wait(bar + kFBarYFull, t & 1));
+            fcp_wait_all();
             u64 v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? ys[(s0 + k) * kFM + m] : 0;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            fbar_arrive(bar + kFBarYFree);
-            if (tid == 0 && good && t + 1 < ntiles) {
-                good = fbar_wait(bar + kFBarYFree, t & 1);
-                if (good) {
-                    issue(t + 1);
-                    ++issued;
-                }
-            }
-            good = __all_sync(0xffffffffu, good);
+            for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? slot[k * kFEpiThreads] : 0;
             fst32(tmem + lane_base + kFAcol + (t & 1) * 128 + part * 32, v);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             ffence_before();
             fbar_arrive(bar + kFBarFull + (t & 1));
-            return good;
+            if (t + 1 < ntiles) issue(t + 1);
+            return true;
         };
-        if (tid == 0) {
-            issue(0);
-            issued = 1;
-        }
+        issue(0);
         ok = stage(0);
         if (ok && ntiles > 1) ok = stage(1);
         // the eight targets of this thread: tb * 32 + part * 8 + c (an invalid one has trow = -1)
@@ -415,8 +392,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
                 }
             }
         }
-        // every copy thread 0 issued has landed before the CTA exits (bounded)
-        if (tid == 0 && issued > 0 && !fbar_wait(bar + kFBarYFull, (issued - 1) & 1)) ok = false;
+        fcp_wait_all();  // no copy of this thread is still in flight when the CTA exits
     }
     if (!ok) atomicExch(err, 1);
     ffence_before();
