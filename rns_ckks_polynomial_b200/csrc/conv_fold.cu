@@ -57,7 +57,8 @@ constexpr int kFThreads = kFEpiThreads + 128;  // 20 warps: at most 5 per SM par
 constexpr int kFTmemCols = 512;
 constexpr int kFAcol = 256;                       // first data-buffer column
 constexpr int kFSmemY = kFBlock;                  // staging slots: 16 words per epilogue thread (64 KiB)
-constexpr int kFSmemDelta = kFSmemY + 16 * kFEpiThreads * 8;  // 32 target deltas (2^60 - q)
+constexpr int kFSmemQ = kFSmemY + 16 * kFEpiThreads * 8;  // 32 target primes q
+constexpr int kFSmemDelta = kFSmemQ + 32 * 8;                 // and their deltas 2^60 - q
 constexpr int kFSmemBar = kFSmemDelta + 32 * 4;
 constexpr int kFSmemBytes = kFSmemBar + 256;
 
@@ -193,22 +194,38 @@ struct FoldJobs {
     }
 };
 
-// x = lo + hi 2^64 < 2^82 mod q for q = 2^60 - delta, delta < 2^28: x = a 2^60 + b with
-// a < 2^22, and 2^60 = delta (mod q), so x = a delta + b < 2^60 + 2^50 < 2q.
-__device__ __forceinline__ u64 freduce82(u64 hi, u64 lo, uint32_t delta)
+// p0 + p1 2^8 + p2 2^16 + p3 2^24 (each p < 2^25, sum < 2^50) as three 32 x 32 -> 64-bit
+// multiply-adds.
+__device__ __forceinline__ u64 ffold4(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3)
 {
-    constexpr u64 kMask60 = ((u64)1 << 60) - 1;
-    const uint32_t a = (uint32_t)(lo >> 60) | (uint32_t)(hi << 4);
-    const u64 w = (lo & kMask60) + (u64)a * delta;
-    const u64 q = ((u64)1 << 60) - delta;
+    u64 g;
+    asm("mad.wide.u32 %0, %1, 256, %2;" : "=l"(g) : "r"(p1), "l"((u64)p0));
+    asm("mad.wide.u32 %0, %1, 65536, %0;" : "+l"(g) : "r"(p2));
+    asm("mad.wide.u32 %0, %1, 16777216, %0;" : "+l"(g) : "r"(p3));
+    return g;
+}
+
+// (g0 + g1 2^32) mod q for g0, g1 < 2^50 and q = 2^60 - delta, delta < 2^28.  The sum x < 2^83 is
+// a 2^60 + b with a < 2^23; 2^60 = delta (mod q), so x = a delta + b < 2^60 + 2^51 < 2q, and one
+// conditional subtraction finishes.
+__device__ __forceinline__ u64 freduce_fold(u64 g0, u64 g1, uint32_t delta, u64 q)
+{
+    uint32_t xm, xh;  // bits 32..63 and 64..95 of x (bits 0..31 are g0's low word)
+    asm("add.cc.u32 %0, %2, %3;\n\taddc.u32 %1, %4, 0;"
+        : "=r"(xm), "=r"(xh) : "r"((uint32_t)(g0 >> 32)), "r"((uint32_t)g1), "r"((uint32_t)(g1 >> 32)));
+    const uint32_t a = __funnelshift_l(xm, xh, 4);                  // x >> 60
+    const u64 b = ((u64)(xm & 0x0FFFFFFFu) << 32) | (uint32_t)g0;  // x mod 2^60
+    u64 w;
+    asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(w) : "r"(a), "r"(delta), "l"(b));
     return w >= q ? w - q : w;
 }
 
-// p0 + p1 2^8 + p2 2^16 + p3 2^24 (each p < 2^25, sum < 2^50).
-__device__ __forceinline__ u64 ffold4(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3)
+// The same sum reduced by the generic 128-bit reduction (primes not of the 2^60 - delta form).
+__device__ __forceinline__ u64 freduce_fold_generic(u64 g0, u64 g1, const PrimeConst &p)
 {
-    const u64 a = (u64)p1 * 256u + p0, b = (u64)p3 * 256u + p2;
-    return a + (b << 16);
+    const u64 lo64 = g0 + (g1 << 32);
+    const u64 hi64 = (g1 >> 32) + (lo64 < g0);
+    return reduce128(hi64, lo64, p);
 }
 
 // Four planes (P_g4 .. P_g4+3) x four columns of the warp's lanes, one wait for all loads.
@@ -244,6 +261,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kFSmemBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kFSmemBar + 8 * kFNumBars);
     uint32_t *dsm = reinterpret_cast<uint32_t *>(sm + kFSmemDelta);
+    u64 *qsm = reinterpret_cast<u64 *>(sm + kFSmemQ);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -265,7 +283,9 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         for (int i = tid; i < kFBlock / 16; i += kFEpiThreads) dst[i] = __ldg(src + i);
         if (tid < kFN) {
             const int ti = tb * kFN + tid;
-            dsm[tid] = ti < T ? (uint32_t)pc[jobs.prime(ti, lo, S)].delta : 0u;
+            const PrimeConst &p = pc[ti < T ? jobs.prime(ti, lo, S) : 0];
+            dsm[tid] = (uint32_t)p.delta;
+            qsm[tid] = p.q;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -336,12 +356,14 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         issue(0);
         ok = stage(0);
         if (ok && ntiles > 1) ok = stage(1);
-        // the eight targets of this thread: tb * 32 + part * 8 + c (an invalid one has trow = -1)
-        int trow[8];
+        // the eight targets of this thread, tb * 32 + part * 8 + c: element offset of its output word
+        // in tile 0 from the job's first output row (-1 for a target past the end)
+        u64 *const jobrow = jobs.row(zrow, 0);
+        int toff[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const int ti = tb * kFN + part * 8 + c;
-            trow[c] = ti < T ? jobs.prime(ti, lo, S) : -1;
+            toff[c] = ti < T ? jobs.prime(ti, lo, S) * kN + cbase + m : -1;
         }
         const uint32_t tcol = tmem + lane_base + part * 8;
         for (int i = 0; i < ntiles && ok; ++i) {
@@ -367,7 +389,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             ok = __all_sync(0xffffffffu, ok);
             ffence_after();
             if (i + 2 < ntiles && ok) ok = stage(i + 2);
-            const int coef = cbase + i * kFM + m;
+            u64 *const out_i = jobrow + i * kFM;
 #pragma unroll
             for (int hc = 0; hc < 2; ++hc) {
                 uint32_t r[4][4];
@@ -380,15 +402,13 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
                 for (int cc = 0; cc < 4; ++cc) {
                     const int c = 4 * hc + cc;
                     const u64 g1 = ffold4(r[0][cc], r[1][cc], r[2][cc], r[3][cc]);
-                    const u64 lo64 = g0[c] + (g1 << 32);
-                    const u64 hi64 = (g1 >> 32) + (lo64 < g0[c]);
-                    if (trow[c] < 0 || !ok) continue;
+                    if (toff[c] < 0 || !ok) continue;
                     u64 res;
                     if constexpr (kSpecial)
-                        res = freduce82(hi64, lo64, dsm[part * 8 + c]);
+                        res = freduce_fold(g0[c], g1, dsm[part * 8 + c], qsm[part * 8 + c]);
                     else
-                        res = reduce128(hi64, lo64, pc[trow[c]]);
-                    jobs.row(zrow, trow[c])[coef] = res;
+                        res = freduce_fold_generic(g0[c], g1, pc[jobs.prime(tb * kFN + part * 8 + c, lo, S)]);
+                    out_i[toff[c]] = res;
                 }
             }
         }
