@@ -99,15 +99,21 @@ __device__ __forceinline__ void fcommit(uint64_t *bar)
                  :: "r"(smem_u32(bar)) : "memory");
 }
 
+// Bounded wait for a phase parity: each poll lets the hardware suspend the thread for up to
+// kFSuspendNs (it resumes as soon as the phase completes), so waiting warps take no issue slots
+// from the working ones; kFPolls polls bound the whole wait to about a second.
+constexpr uint32_t kFSuspendNs = 1000000;
+constexpr int kFPolls = 1024;
+
 __device__ __forceinline__ bool fbar_wait(const uint64_t *bar, uint32_t parity)
 {
     const uint32_t a = smem_u32(bar);
-    for (int i = 0; i < (1 << 18); ++i) {
+    for (int i = 0; i < kFPolls; ++i) {
         uint32_t done;
         asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done) : "r"(a), "r"(parity) : "memory");
+            : "=r"(done) : "r"(a), "r"(parity), "r"(kFSuspendNs) : "memory");
         if (done) return true;
     }
     return false;
