@@ -426,8 +426,8 @@ def _time_call(fn, reps, stream, dev=None):
     return a.elapsed_time(b) / reps, clk.summary()
 
 
-KS_ENTRIES = ("tiny", "boot_rotation", "boot_rotation_integer", "boot_rotation_folded", "layer", "layer_folded",
-              "bsgs", "bsgs_folded", "refresh")
+KS_ENTRIES = ("tiny", "boot_rotation", "boot_rotation_integer", "boot_rotation_byteplanes", "layer",
+              "layer_byteplanes", "bsgs", "bsgs_byteplanes", "refresh")
 
 
 def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_batch=8):
@@ -493,13 +493,13 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
                 B * R, ms, work_rotation(2100, 60, 60, B, R, engine="integer"), hbm_peak, rates, clk)
             ctx.set_conversion("auto")
             ctx.device_status()
-        if "boot_rotation_folded" in entries:
-            # the same call with both conversions in the folded tensor-core form (bit-identical output)
-            ctx.set_conversion("folded")
+        if "boot_rotation_byteplanes" in entries:
+            # the same call with both conversions on the byte-plane tensor-core form (bit-identical output)
+            ctx.set_conversion("tensor")
             ms, clk = _time_call(lambda: ctx.rotate(ct, keys, gal, out=res, ws=ws), 10, stream, dev)
-            out["boot_rotation_L2100_folded"] = ks_entry(B * R, ms, work_rotation(2100, 60, 60, B, R), hbm_peak,
-                                                         rates, clk)
-            out["boot_rotation_L2100_folded"]["conversion"] = "int8 tensor cores, folded form"
+            out["boot_rotation_L2100_byteplanes"] = ks_entry(B * R, ms, work_rotation(2100, 60, 60, B, R),
+                                                             hbm_peak, rates, clk)
+            out["boot_rotation_L2100_byteplanes"]["conversion"] = "int8 tensor cores, byte planes"
             ctx.set_conversion("auto")
             ctx.device_status()
         del ct, keys, res, ws, ctx
@@ -517,11 +517,11 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
         ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
         ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
         out["layer_mul_relin_L112"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
-        if "layer_folded" in entries:
-            ctx.set_conversion("folded")
+        if "layer_byteplanes" in entries:
+            ctx.set_conversion("tensor")
             ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
-            out["layer_mul_relin_L112_folded"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
-            out["layer_mul_relin_L112_folded"]["conversion"] = "int8 tensor cores, folded form"
+            out["layer_mul_relin_L112_byteplanes"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
+            out["layer_mul_relin_L112_byteplanes"]["conversion"] = "int8 tensor cores, byte planes"
             ctx.set_conversion("auto")
         del a, b, rlk, res, ws
     if "bsgs" in entries:
@@ -535,13 +535,13 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
         ws = torch.empty(ctx.workspace_bytes(7, B, 32032), dtype=torch.uint8, device=dev)
         ms, clk = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 10, stream, dev)
         out["bsgs_L112_32x32"] = ks_entry(B * 62, ms, work_bsgs(112, 8, 8, B, 32, 32), hbm_peak, rates, clk)
-        if "bsgs_folded" in entries:
-            ctx.set_conversion("folded")
+        if "bsgs_byteplanes" in entries:
+            ctx.set_conversion("tensor")
             ms, clk = _time_call(lambda: ctx.bsgs_lintrans(x, diags, bk, gk, 32, 32, out=y, ws=ws), 10, stream,
                                  dev)
-            out["bsgs_L112_32x32_folded"] = ks_entry(B * 62, ms, work_bsgs(112, 8, 8, B, 32, 32), hbm_peak,
-                                                     rates, clk)
-            out["bsgs_L112_32x32_folded"]["conversion"] = "int8 tensor cores, folded form"
+            out["bsgs_L112_32x32_byteplanes"] = ks_entry(B * 62, ms, work_bsgs(112, 8, 8, B, 32, 32), hbm_peak,
+                                                         rates, clk)
+            out["bsgs_L112_32x32_byteplanes"]["conversion"] = "int8 tensor cores, byte planes"
             ctx.set_conversion("auto")
         del x, diags, bk, gk, y, ws
     if any(e.startswith("layer") or e.startswith("bsgs") for e in entries):
@@ -672,7 +672,7 @@ def ks_entry(nks, ms, w, hbm_peak, rates, clocks=None):
            "butterflies": w["bfly"], "mulmods": w["mm"], "macs": w["mac"], "macs_on_tensor_cores": w["conv_tc"],
            "min_bytes": w["bytes"], "bound": bound, "roofline_frac": max(t_alu, t_hbm) / t,
            "alu_frac": t_alu / t, "hbm_frac": t_hbm / t,
-           "conversion": "int8 tensor cores" if w["conv_tc"] else "integer pipes"}
+           "conversion": "int8 tensor cores, folded form" if w["conv_tc"] else "integer pipes"}
     if w["conv_tc"]:
         t_int, _ = model_seconds(w, rates, hbm_peak, engine_tc=False)
         out["integer_pipe_model_frac"] = max(t_int, t_hbm) / t

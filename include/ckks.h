@@ -128,9 +128,9 @@ int ckks_selftest_wait_expiry(const ckks_ctx *ctx);
 /* Where the basis conversions of ModUp and ModDown run.  The conversion is
  * the exact product out_t = sum_s y_s [Q_j/q_s]_t (mod t), the step named
  * "RNS basis conversion" in the Kestrel engine write-up, section 3 table.
- *  CKKS_CONV_AUTO     int8 tensor cores when the conversion has 8 or more
- *                     source primes (ModUp: alpha; ModDown: K), the integer
- *                     pipes otherwise (the default);
+ *  CKKS_CONV_AUTO     the folded int8 tensor-core form (below) when the
+ *                     conversion has 8 or more source primes (ModUp: alpha;
+ *                     ModDown: K), the integer pipes otherwise (the default);
  *  CKKS_CONV_INTEGER  always the integer pipes (64x64->128-bit multiply-adds);
  *  CKKS_CONV_TENSOR   always the int8 tensor cores (byte-plane products of
  *                     both operands, 15 accumulators per output);

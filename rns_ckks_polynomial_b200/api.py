@@ -104,9 +104,11 @@ class Context:
         self.key_dnum = None if key_dnum is None else int(key_dnum)
 
     def set_conversion(self, engine):
-        """Where ModUp/ModDown basis conversions run: "auto" (tensor cores from 8
-        source primes on), "integer" (integer pipes) or "tensor" (int8 tensor
-        cores).  Results are bit-identical."""
+        """Where ModUp/ModDown basis conversions run: "auto" (the folded tensor-core
+        form from 8 source primes on, else the integer pipes), "integer" (integer
+        pipes), "tensor" (int8 tensor cores, byte planes of both operands) or
+        "folded" (int8 tensor cores, the data's byte weights folded into the
+        matrix).  Results are bit-identical."""
         check("ckks_ctx_set_conversion",
               lib().ckks_ctx_set_conversion(self._h, self.CONVERSION.get(engine, -1)
                                             if isinstance(engine, str) else int(engine)))

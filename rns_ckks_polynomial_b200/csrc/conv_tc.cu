@@ -519,7 +519,7 @@ ConvKind conv_kind(const ckks_ctx *ctx, int sources)
     case CKKS_CONV_INTEGER: return kConvInteger;
     case CKKS_CONV_TENSOR: return kConvTensor;
     case CKKS_CONV_FOLDED: return kConvFolded;
-    default: return sources > kTcMinSources ? kConvTensor : kConvInteger;
+    default: return sources > kTcMinSources ? kConvFolded : kConvInteger;
     }
 }
 

@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kKiThreads, 4) key_inner_kernel(const u64 *__r
             }
         }
         const int j1 = min(T.dnum, j0 + kKiFold);
-#pragma unroll 2
+#pragma unroll 4
         for (int j = j0; j < j1; ++j) {
             const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
             const u64 *dj = dg + (size_t)j * LKn;
