@@ -28,9 +28,9 @@
 //    issue the ceil(S / 4) K-steps of both planes and commit once;
 //  - 16 epilogue / staging warps: for tile i they read plane group 0 as soon as it completes and
 //    release it (the next tile's products into it can start) and fold it to the low 50 bits of each
-//    sum; wait for group 1, then stage tile i + 2 from shared memory into the data buffer tile i
-//    used (every product of tile i is complete by then); read and release group 1, rebuild each
-//    (< 2^83) sum, reduce it once and store it.  Warp w reads TMEM lane quadrant w & 3 (coefficients
+//    sum; read and release group 1 as soon as it completes, rebuild each (< 2^83) sum, reduce it
+//    once and store it while the tensor cores run the next tile; then stage tile i + 2 from shared
+//    memory into the data buffer tile i used (every product of tile i is complete by then).  Warp w reads TMEM lane quadrant w & 3 (coefficients
 //    32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight targets of one
 //    coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
 // Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
@@ -234,6 +234,18 @@ __device__ __forceinline__ u64 freduce_fold_generic(u64 g0, u64 g1, const PrimeC
     return reduce128(hi64, lo64, p);
 }
 
+// Four planes (P_g4 .. P_g4+3) x eight columns of the warp's lanes, one wait for all loads.
+__device__ __forceinline__ void fld4x8(uint32_t taddr, uint32_t (&r)[4][8])
+{
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[u][0]), "=r"(r[u][1]), "=r"(r[u][2]), "=r"(r[u][3]), "=r"(r[u][4]), "=r"(r[u][5]),
+                       "=r"(r[u][6]), "=r"(r[u][7])
+                     : "r"(taddr + u * kFN));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // Four planes (P_g4 .. P_g4+3) x four columns of the warp's lanes, one wait for all loads.
 __device__ __forceinline__ void fld4x4(uint32_t taddr, uint32_t (&r)[4][4])
 {
@@ -388,35 +400,30 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             }
             ffence_before();
             fbar_arrive(bar + kFBarFree + 0);
-            // plane group 1 (P_4 .. P_7): all products of tile i are then complete, so its data
-            // buffer takes tile i + 2 at once
+            // plane group 1 (P_4 .. P_7), released as soon as it is read: the next tile's products
+            // into both groups then run while this tile's outputs are finished
             ok = fbar_wait(bar + kFBarMma + 2, i & 1) && ok;
             ok = fbar_wait(bar + kFBarMma + 3, i & 1) && ok;
             ok = __all_sync(0xffffffffu, ok);
             ffence_after();
-            if (i + 2 < ntiles && ok) ok = stage(i + 2);
+            uint32_t r1[4][8];
+            fld4x8(tcol + 4 * kFN, r1);
+            ffence_before();
+            fbar_arrive(bar + kFBarFree + 1);
             u64 *const out_i = jobrow + i * kFM;
 #pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-                uint32_t r[4][4];
-                fld4x4(tcol + 4 * kFN + 4 * hc, r);
-                if (hc == 1) {
-                    ffence_before();
-                    fbar_arrive(bar + kFBarFree + 1);
-                }
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int c = 4 * hc + cc;
-                    const u64 g1 = ffold4(r[0][cc], r[1][cc], r[2][cc], r[3][cc]);
-                    if (toff[c] < 0 || !ok) continue;
-                    u64 res;
-                    if constexpr (kSpecial)
-                        res = freduce_fold(g0[c], g1, dsm[part * 8 + c], qsm[part * 8 + c]);
-                    else
-                        res = freduce_fold_generic(g0[c], g1, pc[jobs.prime(tb * kFN + part * 8 + c, lo, S)]);
-                    out_i[toff[c]] = res;
-                }
+            for (int c = 0; c < 8; ++c) {
+                const u64 g1 = ffold4(r1[0][c], r1[1][c], r1[2][c], r1[3][c]);
+                if (toff[c] < 0 || !ok) continue;
+                u64 res;
+                if constexpr (kSpecial)
+                    res = freduce_fold(g0[c], g1, dsm[part * 8 + c], qsm[part * 8 + c]);
+                else
+                    res = freduce_fold_generic(g0[c], g1, pc[jobs.prime(tb * kFN + part * 8 + c, lo, S)]);
+                out_i[toff[c]] = res;
             }
+            // every product of tile i is complete: its data buffer takes tile i + 2
+            if (i + 2 < ntiles && ok) ok = stage(i + 2);
         }
         fcp_wait_all();  // no copy of this thread is still in flight when the CTA exits
     }
