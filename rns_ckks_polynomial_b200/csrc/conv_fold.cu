@@ -34,7 +34,9 @@
 //    32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight targets of one
 //    coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
 // Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
-// 2^60 - delta (delta < 2^28) that is a shift, a 32 x 32 product and one conditional subtraction.
+// 2^60 - delta (delta < 2^28) a funnel shift and one 32 x 32 multiply-add leave the value in
+// [0, 2q), which the forward NTT that consumes every converted limb accepts (it takes inputs below
+// 8q); other primes get the full 128-bit reduction.
 //
 // Every mbarrier wait is bounded: on expiry a thread records an error flag and leaves its loop, the
 // MMA warps wait (bounded again) for the products they issued, the CTA frees its tensor memory and
@@ -57,8 +59,7 @@ constexpr int kFThreads = kFEpiThreads + 128;  // 20 warps: at most 5 per SM par
 constexpr int kFTmemCols = 512;
 constexpr int kFAcol = 256;                       // first data-buffer column
 constexpr int kFSmemY = kFBlock;                  // staging slots: 16 words per epilogue thread (64 KiB)
-constexpr int kFSmemQ = kFSmemY + 16 * kFEpiThreads * 8;  // 32 target primes q
-constexpr int kFSmemDelta = kFSmemQ + 32 * 8;                 // and their deltas 2^60 - q
+constexpr int kFSmemDelta = kFSmemY + 16 * kFEpiThreads * 8;  // 32 target deltas 2^60 - q
 constexpr int kFSmemBar = kFSmemDelta + 32 * 4;
 constexpr int kFSmemBytes = kFSmemBar + 256;
 
@@ -200,21 +201,23 @@ struct FoldJobs {
     }
 };
 
-// p0 + p1 2^8 + p2 2^16 + p3 2^24 (each p < 2^25, sum < 2^50) as three 32 x 32 -> 64-bit
-// multiply-adds.
+// p0 + p1 2^8 + p2 2^16 + p3 2^24 (each p < 2^25, sum < 2^50) as four 32 x 32 -> 64-bit
+// multiply(-add)s on the multiply pipe.
 __device__ __forceinline__ u64 ffold4(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3)
 {
     u64 g;
-    asm("mad.wide.u32 %0, %1, 256, %2;" : "=l"(g) : "r"(p1), "l"((u64)p0));
+    asm("mul.wide.u32 %0, %1, 1;" : "=l"(g) : "r"(p0));
+    asm("mad.wide.u32 %0, %1, 256, %0;" : "+l"(g) : "r"(p1));
     asm("mad.wide.u32 %0, %1, 65536, %0;" : "+l"(g) : "r"(p2));
     asm("mad.wide.u32 %0, %1, 16777216, %0;" : "+l"(g) : "r"(p3));
     return g;
 }
 
-// (g0 + g1 2^32) mod q for g0, g1 < 2^50 and q = 2^60 - delta, delta < 2^28.  The sum x < 2^83 is
-// a 2^60 + b with a < 2^23; 2^60 = delta (mod q), so x = a delta + b < 2^60 + 2^51 < 2q, and one
-// conditional subtraction finishes.
-__device__ __forceinline__ u64 freduce_fold(u64 g0, u64 g1, uint32_t delta, u64 q)
+// A value in [0, 2q) congruent to g0 + g1 2^32 mod q, for g0, g1 < 2^50 and q = 2^60 - delta,
+// delta < 2^28.  The sum x < 2^83 is a 2^60 + b with a < 2^23; 2^60 = delta (mod q), so x = a delta
+// + b < 2^60 + 2^51 < 2q.  The forward NTT that consumes every converted limb (ModUp's new limbs,
+// ModDown's correction) accepts inputs below 8q and returns them fully reduced.
+__device__ __forceinline__ u64 freduce_fold_lazy(u64 g0, u64 g1, uint32_t delta)
 {
     uint32_t xm, xh;  // bits 32..63 and 64..95 of x (bits 0..31 are g0's low word)
     asm("add.cc.u32 %0, %2, %3;\n\taddc.u32 %1, %4, 0;"
@@ -223,7 +226,7 @@ __device__ __forceinline__ u64 freduce_fold(u64 g0, u64 g1, uint32_t delta, u64 
     const u64 b = ((u64)(xm & 0x0FFFFFFFu) << 32) | (uint32_t)g0;  // x mod 2^60
     u64 w;
     asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(w) : "r"(a), "r"(delta), "l"(b));
-    return w >= q ? w - q : w;
+    return w;
 }
 
 // The same sum reduced by the generic 128-bit reduction (primes not of the 2^60 - delta form).
@@ -279,7 +282,6 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kFSmemBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kFSmemBar + 8 * kFNumBars);
     uint32_t *dsm = reinterpret_cast<uint32_t *>(sm + kFSmemDelta);
-    u64 *qsm = reinterpret_cast<u64 *>(sm + kFSmemQ);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -303,7 +305,6 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             const int ti = tb * kFN + tid;
             const PrimeConst &p = pc[ti < T ? jobs.prime(ti, lo, S) : 0];
             dsm[tid] = (uint32_t)p.delta;
-            qsm[tid] = p.q;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -351,10 +352,17 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         // buffer frees up, and no register or other thread is involved while they travel.
         u64 *slot = reinterpret_cast<u64 *>(sm + kFSmemY) + tid;  // word k at slot[k * 512]
         const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + m;
+        const bool full16 = s0 + 16 <= S;  // warp-uniform: all 16 of this thread's sources exist
         auto issue = [&](int t) {
+            const u64 *src = ysrc + t * kFM;
+            if (full16) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (s0 + k < S) fcp8(slot + k * kFEpiThreads, ysrc + (size_t)k * kN + t * kFM);
+                for (int k = 0; k < 16; ++k) fcp8(slot + k * kFEpiThreads, src + (size_t)k * kN);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (s0 + k < S) fcp8(slot + k * kFEpiThreads, src + (size_t)k * kN);
+            }
             fcp_commit();
         };
         // tile t's words: own slots -> tensor-memory buffer t & 1 (the caller knows it is free); the
@@ -362,8 +370,13 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         auto stage = [&](int t) -> bool {
             fcp_wait_all();
             u64 v[16];
+            if (full16) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? slot[k * kFEpiThreads] : 0;
+                for (int k = 0; k < 16; ++k) v[k] = slot[k * kFEpiThreads];
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) v[k] = s0 + k < S ? slot[k * kFEpiThreads] : 0;
+            }
             fst32(tmem + lane_base + kFAcol + (t & 1) * 128 + part * 32, v);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             ffence_before();
@@ -417,7 +430,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
                 if (toff[c] < 0 || !ok) continue;
                 u64 res;
                 if constexpr (kSpecial)
-                    res = freduce_fold(g0[c], g1, dsm[part * 8 + c], qsm[part * 8 + c]);
+                    res = freduce_fold_lazy(g0[c], g1, dsm[part * 8 + c]);
                 else
                     res = freduce_fold_generic(g0[c], g1, pc[jobs.prime(tb * kFN + part * 8 + c, lo, S)]);
                 out_i[toff[c]] = res;
