@@ -169,6 +169,23 @@ __device__ __forceinline__ void inv_radix16(u64 v[16], int m1, const ulonglong2 
     }
 }
 
+// Full reduction of a lazy value v < 8q (forward) or v < 4q (inverse).  For q = 2^60 - delta with
+// delta < 2^32: v = k 2^60 + (v mod 2^60) with k = v >> 60 < 8, and 2^60 = delta (mod q), so
+// r = (v mod 2^60) + k delta < 2^60 + 2^35 < 2q is congruent to v and one conditional subtraction
+// finishes (one shift, one mask and one 32 x 32 multiply-add in place of a chain of subtractions).
+template <bool kS, int kRange>
+__device__ __forceinline__ u64 reduce_lazy(u64 v, const Mod &m)
+{
+    if (kS) {
+        const uint32_t k = (uint32_t)(v >> 60);
+        u64 r;
+        asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(r) : "r"(k), "r"((uint32_t)m.delta), "l"(v & ((1ull << 60) - 1)));
+        return csub(r, m.q);
+    }
+    if (kRange == 8) v = csub(v, m.q4);
+    return csub(csub(v, m.q2), m.q);
+}
+
 // Element index held in register k by thread `t` in each of the three passes.
 struct IdxA { __device__ static __forceinline__ int at(int t, int k) { return t + 128 * k; } };
 struct IdxB { __device__ static __forceinline__ int at(int t, int k) { return (t >> 3) * 128 + (t & 7) + 8 * k; } };
@@ -207,7 +224,7 @@ __global__ void __launch_bounds__(kNttThreads, 4) ntt_fwd_kernel(Job job, Tables
         fwd_radix8c<kS>(v, tid, tw, m);
         fwd_radix8c<kS>(v + 8, tid + 128, tw, m);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = csub(csub(csub(v[k], m.q4), m.q2), m.q);
+        for (int k = 0; k < 16; ++k) v[k] = reduce_lazy<kS, 8>(v[k], m);
         job.store4(r, 8 * tid, v);
         job.store4(r, 8 * tid + 4, v + 4);
         job.store4(r, 8 * (tid + 128), v + 8);
@@ -241,7 +258,7 @@ __global__ void __launch_bounds__(kNttThreads, 4) ntt_inv_kernel(Job job, Tables
         exchange<IdxB, IdxA>(v, sm[1], tid);
         inv_radix16<kS, true>(v, 1, tw, m, pc.ninv, pc.ninvp);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) job.store(r, IdxA::at(tid, k), csub(csub(v[k], m.q2), m.q));
+        for (int k = 0; k < 16; ++k) job.store(r, IdxA::at(tid, k), reduce_lazy<kS, 4>(v[k], m));
         if (jj + 1 < per_block) __syncthreads();
     }
 }
