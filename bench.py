@@ -426,6 +426,23 @@ def _time_call(fn, reps, stream, dev=None):
     return a.elapsed_time(b) / reps, clk.summary()
 
 
+def _time_graph(fn, reps, stream, dev):
+    """The same as _time_call for fn() captured once in a CUDA graph and replayed (the library
+    calls take torch's current stream, which is the capture stream while capturing; their
+    one-time tables are built by the eager warm-up calls first)."""
+    import torch
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    ms, clk = _time_call(g.replay, reps, torch.cuda.current_stream(dev), dev)
+    del g
+    return ms, clk
+
+
 KS_ENTRIES = ("tiny", "boot_rotation", "boot_rotation_integer", "boot_rotation_byteplanes", "layer",
               "layer_byteplanes", "bsgs", "bsgs_byteplanes", "refresh")
 
@@ -468,6 +485,9 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
         out["tiny_pipeline_L4"] = ks_entry(1, ms, w, hbm_peak, rates, clk)
         out["tiny_pipeline_L4"]["note"] = ("one call: 8 limb-4 NTTs, 4 products, 4 INTTs and one rotation; "
                                            "launch-bound at this size")
+        ms, clk = _time_graph(tiny, 200, stream, dev)
+        out["tiny_pipeline_L4_graph"] = ks_entry(1, ms, w, hbm_peak, rates, clk)
+        out["tiny_pipeline_L4_graph"]["note"] = "the same call captured once in a CUDA graph and replayed"
         ctx.device_status()
         del ctx, polys, key, x, prod, rot, ws
     if any(e.startswith("boot_rotation") for e in entries):
@@ -517,6 +537,9 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
         ws = torch.empty(ctx.workspace_bytes(6, B), dtype=torch.uint8, device=dev)
         ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
         out["layer_mul_relin_L112"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
+        ms, clk = _time_graph(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 50, stream, dev)
+        out["layer_mul_relin_L112_graph"] = ks_entry(B, ms, work_mrr(112, 8, 8, B), hbm_peak, rates, clk)
+        out["layer_mul_relin_L112_graph"]["note"] = "the same call captured once in a CUDA graph and replayed"
         if "layer_byteplanes" in entries:
             ctx.set_conversion("tensor")
             ms, clk = _time_call(lambda: ctx.mul_relin_rescale(a, b, rlk, out=res, ws=ws), 20, stream, dev)
