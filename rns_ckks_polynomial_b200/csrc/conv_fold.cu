@@ -26,11 +26,11 @@
 //  - 4 MMA warps (one elected lane each) own planes {2k, 2k+1}: for tile i they wait until its data
 //    is staged and the epilogue has read their plane group (P_0..P_3 or P_4..P_7) of tile i - 1,
 //    issue the ceil(S / 4) K-steps of both planes and commit once;
-//  - 16 epilogue / staging warps, software-pipelined over the tiles: in step i they read and
-//    release plane group 1 of tile i, stage tile i + 2 from shared memory into the data buffer tile i
-//    used (every product of tile i is complete by then), read and release group 0 of tile i + 1,
-//    and only then rebuild each (< 2^83) sum of tile i, reduce it once and store it, while the
-//    tensor cores hold group 1 of tile i + 1 and group 0 of tile i + 2.  Warp w reads TMEM lane quadrant w & 3 (coefficients
+//  - 16 epilogue / staging warps: for tile i they read plane group 0 as soon as it completes and
+//    release it (the next tile's products into it can start) and fold it to the low 50 bits of each
+//    sum; read and release group 1 as soon as it completes, rebuild each (< 2^83) sum, reduce it
+//    once and store it while the tensor cores run the next tile; then stage tile i + 2 from shared
+//    memory into the data buffer tile i used (every product of tile i is complete by then).  Warp w reads TMEM lane quadrant w & 3 (coefficients
 //    32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight targets of one
 //    coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
 // Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
@@ -237,6 +237,18 @@ __device__ __forceinline__ u64 freduce_fold_generic(u64 g0, u64 g1, const PrimeC
     return reduce128(hi64, lo64, p);
 }
 
+// Four planes (P_g4 .. P_g4+3) x eight columns of the warp's lanes, one wait for all loads.
+__device__ __forceinline__ void fld4x8(uint32_t taddr, uint32_t (&r)[4][8])
+{
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[u][0]), "=r"(r[u][1]), "=r"(r[u][2]), "=r"(r[u][3]), "=r"(r[u][4]), "=r"(r[u][5]),
+                       "=r"(r[u][6]), "=r"(r[u][7])
+                     : "r"(taddr + u * kFN));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // Four planes (P_g4 .. P_g4+3) x four columns of the warp's lanes, one wait for all loads.
 __device__ __forceinline__ void fld4x4(uint32_t taddr, uint32_t (&r)[4][4])
 {
@@ -385,12 +397,13 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             toff[c] = ti < T ? jobs.prime(ti, lo, S) * kN + cbase + m : -1;
         }
         const uint32_t tcol = tmem + lane_base + part * 8;
-        // Plane group 0 of tile t: wait, read, release, fold to the low 50 bits of each sum.
-        auto read_g0 = [&](int t, u64 (&g0)[8]) {
-            ok = fbar_wait(bar + kFBarMma + 0, t & 1) && ok;
-            ok = fbar_wait(bar + kFBarMma + 1, t & 1) && ok;
+        for (int i = 0; i < ntiles && ok; ++i) {
+            // plane group 0 (P_0 .. P_3): the low 50 bits of each sum
+            ok = fbar_wait(bar + kFBarMma + 0, i & 1) && ok;
+            ok = fbar_wait(bar + kFBarMma + 1, i & 1) && ok;
             ok = __all_sync(0xffffffffu, ok);  // warp-uniform: the loads below are warp-collective
             ffence_after();
+            u64 g0[8];
 #pragma unroll
             for (int hc = 0; hc < 2; ++hc) {
                 uint32_t r[4][4];
@@ -400,45 +413,30 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             }
             ffence_before();
             fbar_arrive(bar + kFBarFree + 0);
-        };
-        // The loop is software-pipelined so that the output arithmetic of tile i runs while the
-        // tensor cores hold group 1 of tile i + 1 and group 0 of tile i + 2: each iteration reads
-        // and releases group 1 of tile i, stages tile i + 2 into the data buffer tile i used (every
-        // product of tile i is then complete), reads and releases group 0 of tile i + 1, and only
-        // then finishes tile i.
-        u64 g0[8];
-        read_g0(0, g0);
-        for (int i = 0; i < ntiles && ok; ++i) {
+            // plane group 1 (P_4 .. P_7), released as soon as it is read: the next tile's products
+            // into both groups then run while this tile's outputs are finished
             ok = fbar_wait(bar + kFBarMma + 2, i & 1) && ok;
             ok = fbar_wait(bar + kFBarMma + 3, i & 1) && ok;
             ok = __all_sync(0xffffffffu, ok);
             ffence_after();
-            u64 g1[8];
-#pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-                uint32_t r[4][4];
-                fld4x4(tcol + 4 * kFN + 4 * hc, r);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) g1[4 * hc + c] = ffold4(r[0][c], r[1][c], r[2][c], r[3][c]);
-            }
+            uint32_t r1[4][8];
+            fld4x8(tcol + 4 * kFN, r1);
             ffence_before();
             fbar_arrive(bar + kFBarFree + 1);
-            if (i + 2 < ntiles && ok) ok = stage(i + 2);
-            u64 g0n[8];
-            if (i + 1 < ntiles && ok) read_g0(i + 1, g0n);
             u64 *const out_i = jobrow + i * kFM;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
+                const u64 g1 = ffold4(r1[0][c], r1[1][c], r1[2][c], r1[3][c]);
                 if (toff[c] < 0 || !ok) continue;
                 u64 res;
                 if constexpr (kSpecial)
-                    res = freduce_fold_lazy(g0[c], g1[c], dsm[part * 8 + c]);
+                    res = freduce_fold_lazy(g0[c], g1, dsm[part * 8 + c]);
                 else
-                    res = freduce_fold_generic(g0[c], g1[c], pc[jobs.prime(tb * kFN + part * 8 + c, lo, S)]);
+                    res = freduce_fold_generic(g0[c], g1, pc[jobs.prime(tb * kFN + part * 8 + c, lo, S)]);
                 out_i[toff[c]] = res;
             }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) g0[c] = g0n[c];
+            // every product of tile i is complete: its data buffer takes tile i + 2
+            if (i + 2 < ntiles && ok) ok = stage(i + 2);
         }
         fcp_wait_all();  // no copy of this thread is still in flight when the CTA exits
     }
