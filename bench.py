@@ -3,9 +3,11 @@
 
 Workload (one step): the NTT/INTT throughput sweep at n = 2048 -- a batch of
 16 polynomials with seeded uniform residues at each of 3, 112, 512 and 2100
-limbs of 60-bit NTT-friendly primes, forward NTT then inverse NTT, in place;
-the round trip is checked to be the identity after the timed steps.  The
-metric is limb-NTTs per second (forward and inverse both count).
+limbs of 60-bit NTT-friendly primes, forward NTT then inverse NTT, in place,
+each direction one grouped launch over the four tensors (ckks_ntt_fwd_group /
+ckks_ntt_inv_group); the round trip is checked to be the identity after the
+timed steps.  The metric is limb-NTTs per second (forward and inverse both
+count).
 
 Next to it, the key-switch rates of the three key-switching workloads are
 measured once in the same run (not part of the step): the layer-shaped
@@ -184,10 +186,16 @@ def weak_scaling_value(per_step_units, steps, world, total_ms):
 
 # ---------------------------------------------------------------- roofline bits
 def ntt_launch_work(limbs, batch=BATCH):
-    """Algorithmic bytes and Shoup multiplies of one forward-NTT launch."""
-    jobs = limbs * batch
-    bytes_ = jobs * 2 * N * 8 + limbs * N * 16  # data in+out, {w, w'} per prime
-    mm = jobs * (N // 2) * 11
+    """Algorithmic bytes and butterflies of one forward-NTT launch over `batch` polynomials at each
+    limb count in `limbs` (one int, or a tuple for a grouped launch); the twiddle table of a prime
+    is counted once per tensor."""
+    if isinstance(limbs, int):
+        limbs = (limbs,)
+    bytes_ = mm = 0
+    for l in limbs:
+        jobs = l * batch
+        bytes_ += jobs * 2 * N * 8 + l * N * 16  # data in+out, {w, w'} per prime
+        mm += jobs * (N // 2) * 11
     return bytes_, mm
 
 
@@ -236,7 +244,8 @@ def rates_from(ipeak):
 
 
 def ntt_roofline(limbs, k_ms, hbm_peak, peak_src, ipeak):
-    """Roofline object of one forward-NTT launch over BATCH x limbs: the
+    """Roofline object of one forward-NTT launch over BATCH x limbs (or the grouped launch over a
+    tuple of limb counts): the
     slower of its bytes at the measured HBM copy rate and its butterflies at
     the same-run rate of the kernel's own butterfly (microbenchmark kind 5).
     The generic Shoup rate (kind 0) is reported beside it."""
@@ -252,8 +261,10 @@ def ntt_roofline(limbs, k_ms, hbm_peak, peak_src, ipeak):
         roof = {"bound": "hbm", "achieved": bytes_ / t / 1e9, "peak": hbm_peak, "unit": "GB/s",
                 "peak_source": "%s MEASURED_PEAKS.json hbm_gbs" % peak_src}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for("ntt_fwd_%d" % limbs)
-    roof["kernel"] = "ntt_fwd_kernel<BatchJob> (%d x %d limbs)" % (BATCH, limbs)
+    key = "ntt_fwd_group_" + "-".join(str(l) for l in limbs) if isinstance(limbs, tuple) else "ntt_fwd_%d" % limbs
+    roof["traffic"] = traffic_for(key)
+    roof["kernel"] = ("ntt_fwd_kernel<GroupJob> (%d x {%s} limbs, one launch)" % (BATCH, ", ".join(map(str, limbs)))
+                      if isinstance(limbs, tuple) else "ntt_fwd_kernel<BatchJob> (%d x %d limbs)" % (BATCH, limbs))
     roof["launch_ms"] = k_ms
     roof["algorithmic_bytes"] = bytes_
     roof["butterflies"] = mm
@@ -283,13 +294,13 @@ def run_b200(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
-        for i, x in enumerate(xs):
-            if ev is not None and i == len(xs) - 1:
-                ev[0].record(stream)
-            ctx.ntt_fwd(x)
-            if ev is not None and i == len(xs) - 1:
-                ev[1].record(stream)
-            ctx.ntt_inv(x)
+        # every sweep entry in one grouped launch per direction
+        if ev is not None:
+            ev[0].record(stream)
+        ctx.ntt_fwd_group(xs)
+        if ev is not None:
+            ev[1].record(stream)
+        ctx.ntt_inv_group(xs)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -321,8 +332,8 @@ def run_b200(args):
     per_step = 2 * BATCH * sum(SWEEP)
     value = weak_scaling_value(per_step, args.steps, world, total_ms)
 
-    # roofline of the dominant kernel: forward NTT on the largest sweep entry
-    roof = ntt_roofline(SWEEP[-1], k_ms, hbm_peak, peak_src, ipeak)
+    # roofline of the dominant kernel: the grouped forward NTT over every sweep entry
+    roof = ntt_roofline(SWEEP, k_ms, hbm_peak, peak_src, ipeak)
 
     line = {
         "metric": METRIC, "value": value, "unit": "limb-NTTs/s", "n_gpus": world,
@@ -334,7 +345,7 @@ def run_b200(args):
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": "replicas" if world > 1 else "single"},
         "roundtrip_identity": ok,
-        "gpu_launches": 2 * len(SWEEP) * args.steps,
+        "gpu_launches": 2 * args.steps,
         "roofline": roof,
         "intpipe_peaks": ipeak,
         "clocks": clk.summary(),

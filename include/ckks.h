@@ -188,6 +188,22 @@ int ckks_ntt_fwd(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin,
 int ckks_ntt_inv(const ckks_ctx *ctx, uint64_t *x, int batch, int limb_begin,
                  int limbs, ckks_stream_t stream);
 
+/* The same transforms on several tensors in one launch (a batch of
+ * polynomials at several levels, such as the NTT sweep of 16 polynomials at
+ * 3, 112, 512 and 2100 limbs): for g < groups, x[g] (a host array of device
+ * pointers) is [batch[g]][limbs[g]][n] and its local limb l uses prime index
+ * limb_begin[g] + l.  Each tensor gets exactly ckks_ntt_fwd's (or
+ * ckks_ntt_inv's) result; the small tensors no longer need launches of their
+ * own that leave most of the GPU idle.  Tensors must not overlap.
+ * 0 <= groups <= 8; empty groups are skipped.  CKKS_EINVAL for bad ranges,
+ * null or misaligned pointers; CKKS_EUNSUPPORTED past 2^30 limbs in all. */
+int ckks_ntt_fwd_group(const ckks_ctx *ctx, uint64_t *const *x, const int *batch,
+                       const int *limb_begin, const int *limbs, int groups,
+                       ckks_stream_t stream);
+int ckks_ntt_inv_group(const ckks_ctx *ctx, uint64_t *const *x, const int *batch,
+                       const int *limb_begin, const int *limbs, int groups,
+                       ckks_stream_t stream);
+
 /* ---------------------------------------------------------------- a3: pointwise */
 
 /* out = a (op) b mod q per limb, NTT domain, arrays [batch][limbs][n]

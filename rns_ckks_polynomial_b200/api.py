@@ -144,6 +144,28 @@ class Context:
                                                  _stream(x)))
         return x
 
+    def _group(self, name, xs, limb_begins):
+        xs = list(xs)
+        begins = list(limb_begins) if limb_begins is not None else [0] * len(xs)
+        if len(begins) != len(xs):
+            raise ValueError("one limb_begin per tensor")
+        g = len(xs)
+        ptrs = (C.c_void_p * max(1, g))(*[_ptr(x, "x").value for x in xs])
+        limbs = [x.shape[-2] for x in xs]
+        batch = [x.numel() // (l * self.n) if x.numel() else 0 for x, l in zip(xs, limbs)]
+        arr = lambda v: (C.c_int * max(1, g))(*v)  # noqa: E731
+        stream = _stream(xs[0]) if xs else None
+        check(name, getattr(lib(), name)(self._h, ptrs, arr(batch), arr(begins), arr(limbs), g, stream))
+        return xs
+
+    def ntt_fwd_group(self, xs, limb_begins=None):
+        """Forward NTT of every tensor x[..., limbs, n] of `xs` in place, in one launch."""
+        return self._group("ckks_ntt_fwd_group", xs, limb_begins)
+
+    def ntt_inv_group(self, xs, limb_begins=None):
+        """Inverse NTT of every tensor of `xs` in place, in one launch."""
+        return self._group("ckks_ntt_inv_group", xs, limb_begins)
+
     # ------------------------------------------------------------ a3/a4
     def pointwise(self, op, a, b, out=None, limb_begin=0):
         out = torch.empty_like(a) if out is None else out

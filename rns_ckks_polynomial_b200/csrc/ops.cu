@@ -329,6 +329,82 @@ extern "C" int ckks_ntt_inv(const ckks_ctx *ctx, uint64_t *x, int batch, int lim
     return launch_ntt_inv(j, ctx->t, (cudaStream_t)stream);
 }
 
+// Several tensors in one launch: group g is x[g][batch][limbs][n], limb l with prime
+// limb_begin + l; its jobs follow those of the groups before it, limb-major within the group (the
+// order BatchJob uses), so a CTA's consecutive jobs still share a prime.
+constexpr int kMaxNttGroups = 8;
+
+struct GroupJob {
+    u64 *x[kMaxNttGroups];
+    int limbs[kMaxNttGroups], batch[kMaxNttGroups], begin[kMaxNttGroups], start[kMaxNttGroups + 1];
+    int groups, count;
+    struct Ref {
+        u64 *row;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
+    {
+        int g = 0;
+#pragma unroll
+        for (int i = 1; i < kMaxNttGroups; ++i) g += (i < groups && j >= start[i]) ? 1 : 0;
+        const int jj = j - start[g];
+        const int l = jj / batch[g], b = jj - l * batch[g];
+        return {x[g] + ((size_t)b * limbs[g] + l) * kN, begin[g] + l};
+    }
+    __device__ __forceinline__ u64 load(const Ref &r, int e) const { return r.row[e]; }
+    __device__ __forceinline__ void store4(const Ref &r, int e, const u64 *v) const { st4(r.row + e, v); }
+    __device__ __forceinline__ void load4(const Ref &r, int e, u64 *v) const { ld4(r.row + e, v); }
+    __device__ __forceinline__ void store(const Ref &r, int e, u64 v) const { r.row[e] = v; }
+};
+
+static int ntt_group_job(const ckks_ctx *ctx, uint64_t *const *x, const int *batch, const int *limb_begin,
+                         const int *limbs, int groups, GroupJob *job)
+{
+    CKKS_TRY(check_ctx(ctx));
+    if (groups < 0 || groups > kMaxNttGroups) return set_error(CKKS_EINVAL, "need 0 <= groups <= 8");
+    if (groups > 0 && (!x || !batch || !limb_begin || !limbs)) return set_error(CKKS_EINVAL, "null group array");
+    long long total = 0;
+    int n = 0;
+    for (int g = 0; g < groups; ++g) {
+        CKKS_TRY(check_limbs(ctx, limb_begin[g], limbs[g]));
+        if (batch[g] < 0) return set_error(CKKS_EINVAL, "negative batch");
+        if ((long long)batch[g] * limbs[g] == 0) continue;
+        CKKS_TRY(check_ptr(x[g], "x[g]"));
+        job->x[n] = x[g];
+        job->limbs[n] = limbs[g];
+        job->batch[n] = batch[g];
+        job->begin[n] = limb_begin[g];
+        job->start[n] = (int)total;
+        total += (long long)batch[g] * limbs[g];
+        if (total > (1LL << 30)) return set_error(CKKS_EUNSUPPORTED, "too many limbs");
+        ++n;
+    }
+    for (int g = n; g <= kMaxNttGroups; ++g) job->start[g] = (int)total;
+    job->groups = n;
+    job->count = (int)total;
+    if (total == 0) return 1;
+    CKKS_TRY(set_device(ctx));
+    return CKKS_OK;
+}
+
+extern "C" int ckks_ntt_fwd_group(const ckks_ctx *ctx, uint64_t *const *x, const int *batch,
+                                  const int *limb_begin, const int *limbs, int groups, ckks_stream_t stream)
+{
+    GroupJob j{};
+    int rc = ntt_group_job(ctx, x, batch, limb_begin, limbs, groups, &j);
+    if (rc != CKKS_OK) return rc > 0 ? CKKS_OK : rc;
+    return launch_ntt_fwd(j, ctx->t, (cudaStream_t)stream);
+}
+
+extern "C" int ckks_ntt_inv_group(const ckks_ctx *ctx, uint64_t *const *x, const int *batch,
+                                  const int *limb_begin, const int *limbs, int groups, ckks_stream_t stream)
+{
+    GroupJob j{};
+    int rc = ntt_group_job(ctx, x, batch, limb_begin, limbs, groups, &j);
+    if (rc != CKKS_OK) return rc > 0 ? CKKS_OK : rc;
+    return launch_ntt_inv(j, ctx->t, (cudaStream_t)stream);
+}
+
 extern "C" int ckks_pointwise(const ckks_ctx *ctx, int op, const uint64_t *a, const uint64_t *b,
                               uint64_t *out, int batch, int limb_begin, int limbs,
                               ckks_stream_t stream)

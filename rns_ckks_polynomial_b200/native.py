@@ -28,6 +28,10 @@ SIGNATURES = {
     "ckks_workspace_bytes": (C.c_size_t, [_vp, C.c_int, C.c_int, C.c_int]),
     "ckks_ntt_fwd": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_ntt_inv": (C.c_int, [_vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
+    "ckks_ntt_fwd_group": (C.c_int, [_vp, C.POINTER(_vp), C.POINTER(C.c_int), C.POINTER(C.c_int),
+                                     C.POINTER(C.c_int), C.c_int, _vp]),
+    "ckks_ntt_inv_group": (C.c_int, [_vp, C.POINTER(_vp), C.POINTER(C.c_int), C.POINTER(C.c_int),
+                                     C.POINTER(C.c_int), C.c_int, _vp]),
     "ckks_pointwise": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_pointwise_scalar": (C.c_int, [_vp, C.c_int, _vp, _vp, _vp, C.c_int, C.c_int, C.c_int, _vp]),
     "ckks_add_const_c0": (C.c_int, [_vp, _vp, _vp, C.c_int, _vp]),

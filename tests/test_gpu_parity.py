@@ -102,6 +102,29 @@ def test_ntt_full_sweep_2100(orc):
     assert torch.equal(x, a)
 
 
+def test_ntt_group_matches_single_launches(orc):
+    """One grouped launch over tensors of 3, 112, 512 and 5 limbs (different batches, one at an odd
+    limb_begin, one empty) gives every tensor the oracle's forward transform, and the grouped
+    inverse brings them back; more than 8 groups is rejected."""
+    ctx = context(2100, 60, 60)
+    shapes = [(16, 3, 0), (4, 112, 0), (2, 512, 40), (3, 5, 2155), (0, 7, 0)]
+    arrs = [_res((b, l, N), np.array(ctx.mods[s0:s0 + l], dtype=np.uint64), 700 + i) if b else
+            np.zeros((0, l, N), dtype=np.uint64) for i, (b, l, s0) in enumerate(shapes)]
+    xs = [dev(a) for a in arrs]
+    begins = [s0 for _, _, s0 in shapes]
+    ctx.ntt_fwd_group(xs, begins)
+    for (b, l, s0), a, x in zip(shapes, arrs, xs):
+        want = orc.ntt_fwd(a, np.array(ctx.mods[s0:s0 + l], dtype=np.uint64)) if b else a
+        assert_bits_equal(host(x), want, "grouped ntt_fwd %d x %d at %d" % (b, l, s0))
+    ctx.ntt_inv_group(xs, begins)
+    for a, x in zip(arrs, xs):
+        assert_bits_equal(host(x), a, "grouped round trip")
+    lib = native.lib()
+    ptrs = (C.c_void_p * 9)(*([xs[0].data_ptr()] * 9))
+    ints = (C.c_int * 9)(*([1] * 9))
+    assert lib.ckks_ntt_fwd_group(ctx._h, ptrs, ints, (C.c_int * 9)(*([0] * 9)), ints, 9, None) == -1
+
+
 def test_ntt_empty_and_errors():
     ctx = context(4, 1, 1)
     e = torch.empty((0, 4, N), dtype=torch.int64, device="cuda")
