@@ -23,9 +23,11 @@
 //    384..511, two 32-bit columns per source;
 //  - accumulator P_u takes columns 32 u .. 32 u + 31.
 // Warp roles (20 warps, so that 96 registers fit), synchronised by mbarriers only:
-//  - 4 MMA warps (one elected lane each) own planes {2k, 2k+1}: for tile i they wait until its data
-//    is staged and the epilogue has read their plane group (P_0..P_3 or P_4..P_7) of tile i - 1,
-//    issue the ceil(S / 4) K-steps of both planes and commit once;
+//  - 4 MMA warps (one elected lane each) own planes {k, k + 4}: for tile i each waits until its
+//    data is staged, then per plane group g (P_0..P_3, then P_4..P_7) until the epilogue has read
+//    group g of tile i - 1, issues the ceil(S / 4) K-steps of its plane in that group and commits.
+//    All four warps issue group 0 before group 1, so group 0 completes half-way through the tile
+//    and the epilogue reads it while group 1 runs;
 //  - 16 epilogue / staging warps: for tile i they read plane group 0 as soon as it completes and
 //    release it (the next tile's products into it can start) and fold it to the low 50 bits of each
 //    sum; read and release group 1 as soon as it completes, rebuild each (< 2^83) sum, reduce it
@@ -63,7 +65,7 @@ constexpr int kFSmemDelta = kFSmemY + 16 * kFEpiThreads * 8;  // 32 target delta
 constexpr int kFSmemBar = kFSmemDelta + 32 * 4;
 constexpr int kFSmemBytes = kFSmemBar + 256;
 
-enum { kFBarMma = 0, kFBarFree = 4, kFBarFull = 6, kFBarDrain = 8, kFNumBars = 9 };
+enum { kFBarMma = 0, kFBarFree = 2, kFBarFull = 4, kFBarDrain = 6, kFNumBars = 7 };
 static_assert(kFSmemBar + 8 * kFNumBars + 4 <= kFSmemBytes, "shared-memory layout");
 static_assert(kFSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -94,6 +96,13 @@ __device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, u64 bde
            "r"(0));
 }
 
+// True in exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+    return pred != 0;
+}
 __device__ __forceinline__ void fcommit(uint64_t *bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -260,7 +269,7 @@ __device__ __forceinline__ void fld4x4(uint32_t taddr, uint32_t (&r)[4][4])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Barriers: kFBarMma + k (k < 4) completes when MMA warp k's planes 2k, 2k+1 of a tile are done;
+// Barriers: kFBarMma + g (g < 2) completes when the four commits of plane group g of a tile are in;
 // kFBarFree + g (g < 2) when the epilogue has read plane group g (planes 4g .. 4g+3) of a tile;
 // kFBarFull + b when tensor-memory data buffer b is staged; kFBarDrain when every issued product
 // is done.
@@ -289,7 +298,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
-        for (int k = 0; k < 4; ++k) fbar_init(bar + kFBarMma + k, 1);
+        for (int k = 0; k < 2; ++k) fbar_init(bar + kFBarMma + k, 4);
         fbar_init(bar + kFBarFree + 0, kFEpiThreads);
         fbar_init(bar + kFBarFree + 1, kFEpiThreads);
         fbar_init(bar + kFBarFull + 0, kFEpiThreads);
@@ -316,27 +325,28 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
 
     if (warp >= kFMmaWarp0) {
         // ------------------------------------------------ MMA issue (one elected lane per warp)
-        const int issuer = warp - kFMmaWarp0;  // planes 2 issuer, 2 issuer + 1
+        const int issuer = warp - kFMmaWarp0;  // planes issuer (group 0) and issuer + 4 (group 1)
         const u64 bdesc0 = fsmem_desc(smem_u32(sm));
-        const int grp = issuer >> 1;  // plane group read back together by the epilogue
         for (int i = 0; i < ntiles && ok; ++i) {
             const int buf = i & 1;
             ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFull + buf, (i >> 1) & 1));
-            if (ok && i > 0) ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFree + grp, (i - 1) & 1));
-            if (!ok) break;
-            ffence_after();
-            if (lane == 0) {
-                const uint32_t ta = tmem + kFAcol + buf * 128;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int u = 2 * issuer + h;
-                    const u64 bd = bdesc0 + (((size_t)u * kFPlaneBytes) >> 4);
-                    for (int ks = 0; ks < nks; ++ks)
-                        mma_ts(tmem + u * kFN, ta + ks * 8, bd + ((ks * 256) >> 4), ks > 0 ? 1u : 0u);
+            const uint32_t ta = tmem + kFAcol + buf * 128;
+            for (int g = 0; g < 2 && ok; ++g) {
+                if (i > 0) ok = __all_sync(0xffffffffu, fbar_wait(bar + kFBarFree + g, (i - 1) & 1));
+                if (!ok) break;
+                ffence_after();
+                const int u = issuer + 4 * g;
+                const uint32_t td = tmem + u * kFN;
+                const u64 bd = bdesc0 + (((size_t)u * kFPlaneBytes) >> 4);
+                // Every operand is warp-uniform and one lane is elected by elect.sync: the products
+                // then issue back to back, where a lane-divergent issue cost about 120 cycles each.
+                if (elect_one()) {
+                    mma_ts(td, ta, bd, 0u);
+                    for (int ks = 1; ks < nks; ++ks) mma_ts(td, ta + ks * 8, bd + ks * 16, 1u);
+                    fcommit(bar + kFBarMma + g);
                 }
-                fcommit(bar + kFBarMma + issuer);
+                __syncwarp();
             }
-            __syncwarp();
         }
         // every product issued here has completed before tensor memory is freed (bounded)
         if (lane == 0) fcommit(bar + kFBarDrain);
@@ -400,7 +410,6 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         for (int i = 0; i < ntiles && ok; ++i) {
             // plane group 0 (P_0 .. P_3): the low 50 bits of each sum
             ok = fbar_wait(bar + kFBarMma + 0, i & 1) && ok;
-            ok = fbar_wait(bar + kFBarMma + 1, i & 1) && ok;
             ok = __all_sync(0xffffffffu, ok);  // warp-uniform: the loads below are warp-collective
             ffence_after();
             u64 g0[8];
@@ -415,8 +424,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             fbar_arrive(bar + kFBarFree + 0);
             // plane group 1 (P_4 .. P_7), released as soon as it is read: the next tile's products
             // into both groups then run while this tile's outputs are finished
-            ok = fbar_wait(bar + kFBarMma + 2, i & 1) && ok;
-            ok = fbar_wait(bar + kFBarMma + 3, i & 1) && ok;
+            ok = fbar_wait(bar + kFBarMma + 1, i & 1) && ok;
             ok = __all_sync(0xffffffffu, ok);
             ffence_after();
             uint32_t r1[4][8];
