@@ -13,9 +13,10 @@
 //  - the 15 accumulators P_d take TMEM columns 32 d .. 32 d + 31, in two groups: X = P_0..P_7
 //    (36 plane pairs) and Y = P_8..P_14 (28 pairs);
 //  - the y bytes of a tile are staged in one of two shared-memory buffers, two tiles ahead.
-// Every tcgen05.mma costs a fixed issue time of a few dozen SM cycles up to N = 64, so the tile is as
-// wide as the 15 accumulators allow (15 x 32 of the 512 columns), and four warps issue: separate
-// issuing threads overlap their issue costs.
+// With both operands in shared memory a tcgen05.mma reads its whole A tile (128 x 32 bytes) and
+// N x 32 bytes of B per K-step, at about 128 bytes per SM cycle: about 40 cycles at N = 32 against
+// 16 cycles of arithmetic, so the tile is as wide as the 15 accumulators allow (15 x 32 of the 512
+// columns), and four warps issue.
 // Warp roles: 16 epilogue warps and 4 MMA warps, synchronised by mbarriers only.
 //  - MMA warps (one elected lane each) own disjoint sets of accumulators: two split group X (P_d sets
 //    {0, 1, 6, 7} and {2, 3, 4, 5}, 18 plane pairs each), two split group Y ({8, 11, 12} and
@@ -104,6 +105,15 @@ __device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity)
 }
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+// True in exactly one lane of the (converged) warp.  The MMA warps issue from this lane with every
+// operand computed warp-wide, so the operands stay warp-uniform and the products issue back to back.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+    return pred != 0;
+}
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // The products of the y tile at `bdesc` into the accumulators P_d whose bit d is set in kMask.  The
@@ -339,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) conv_tc_kernel(TcJobs jobs, const
             if (ok && i > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar + (y_issuer ? kBarFreeY : kBarFreeX), (i - 1) & 1));
             if (!ok) break;
             fence_after();
-            if (lane == 0) {
+            if (elect_one()) {
                 // P_d sets of 18, 18, 14 and 14 plane pairs
                 if (issuer == 0) issue_set<(1 << 0) | (1 << 1) | (1 << 6) | (1 << 7)>(tmem, adesc, bdesc, two_k);
                 if (issuer == 1) issue_set<(1 << 2) | (1 << 3) | (1 << 4) | (1 << 5)>(tmem, adesc, bdesc, two_k);
@@ -450,7 +460,7 @@ int launch(const ckks_ctx *ctx, TcJobs j, int tbs, int jobs, cudaStream_t s)
 
 // ---------------------------------------------------------------- tensor-pipe microbenchmark
 // Back-to-back tcgen05.mma (kind::i8, M = 128, K = 32, both operands in shared memory) from one
-// thread per CTA, one CTA per SM: the fixed cost per MMA at a given N (the conversion's own tile is
+// elected thread per CTA (warp-uniform operands), one CTA per SM: the fixed cost per MMA at a given N (the conversion's own tile is
 // N = 32) and the dense int8 rate (N = 256).  Operand values do not matter; the products accumulate
 // into one TMEM region.
 constexpr int kBenchSmem = kTM * kKP + 256 * kKP + 64;  // A 8 KiB, B up to 16 KiB, barrier, slot
@@ -477,20 +487,23 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, int *err)
     __syncthreads();
     fence_after();
     const uint32_t tmem = *tslot;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
         constexpr uint32_t idesc = (2u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
         const u64 ad = smem_desc(smem_u32(sm)), bd = smem_desc(smem_u32(sm + kTM * kKP));
-        for (int r = 0; r < iters; r += 8) {
+        if (elect_one()) {
+            for (int r = 0; r < iters; r += 8) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                asm volatile(
-                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                    "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
-                    :: "r"(tmem), "l"(ad + ((k & 1) * 256 >> 4)), "l"(bd + ((k & 1) * 256 >> 4)), "r"(idesc),
-                       "r"(k | r), "r"(0), "r"(0), "r"(0), "r"(0));
+                for (int k = 0; k < 8; ++k)
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+                        :: "r"(tmem), "l"(ad + ((k & 1) * 256 >> 4)), "l"(bd + ((k & 1) * 256 >> 4)), "r"(idesc),
+                           "r"(k | r), "r"(0), "r"(0), "r"(0), "r"(0));
+            }
+            commit(bar);
+            if (!mbar_wait(bar, 0)) atomicExch(err, 1);
         }
-        commit(bar);
-        if (!mbar_wait(bar, 0)) atomicExch(err, 1);
+        __syncwarp();
     }
     fence_before();
     __syncthreads();
