@@ -268,8 +268,10 @@ int ckks_modup_noalloc(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *dig
  * evaluation key, which the EncryptedLLM GPU article (section 2.5) sizes at
  * hundreds of MB to several GB and names, with the rotation it serves, as
  * the under-rated cost of encrypted inference.  Sums over any number of
- * digits are exact (reduced once per 256 digits).  CKKS_EINVAL for a null
- * pointer, a pointer that is not 16-byte aligned or an even galois. */
+ * digits are exact (reduced once per 256 digits, or folded once per 8 when
+ * every prime is 2^60 - delta with delta < 2^32).  Digit and key words must
+ * be residues, below their prime.  CKKS_EINVAL for a null pointer, a pointer
+ * that is not 16-byte aligned or an even galois. */
 int ckks_key_inner(const ckks_ctx *ctx, const uint64_t *digits, const uint64_t *key,
                    uint32_t galois, uint64_t *acc, int batch, ckks_stream_t stream);
 

@@ -775,13 +775,33 @@ def test_extreme_residues_rescale(orc, lp1):
     assert_bits_equal(host(ctx.rescale(dev(ct))), orc.rescale(ct, q), "rescale extremes, %d limbs" % lp1)
 
 
-def test_key_inner_more_than_256_digits():
+def _top_general_primes(orc, count):
+    """Primes q = 1 mod 2n just below 2^60 - 2^32: close enough to 2^60 that 260 (q - 1)^2 passes
+    2^128, yet not of the 2^60 - delta (delta < 2^32) form."""
+    out, c = [], ((1 << 60) - (1 << 32)) // (2 * N) * (2 * N) + 1
+    while len(out) < count:
+        if orc.is_prime(c):
+            out.append(c)
+        c -= 2 * N
+    return out
+
+
+@pytest.mark.parametrize("form", ["special", "general"])
+def test_key_inner_more_than_256_digits(orc, form):
     """260 single-prime digits (L = 260, alpha = 1): with every digit word and
-    key word at q - 1 the exact sum 260 (q - 1)^2 passes 2^128, so the kernel
-    must reduce between blocks of digits.  Each output word is the closed
-    form 260 (q - 1)^2 = 260 mod q."""
+    key word at q - 1 the exact sum 260 (q - 1)^2 passes 2^128.  Primes of the
+    2^60 - delta form take the split sums (three 64-bit partial sums, folded
+    every 8 digits: this input drives each of them to its largest value);
+    other primes take 128-bit sums, which must be reduced between blocks of
+    256 digits.  Each output word is the closed form 260 (q - 1)^2 = 260 mod q."""
+    from rns_ckks_polynomial_b200 import Context
     L, K = 260, 1
-    ctx = context(L, K, 1)
+    if form == "special":
+        ctx = context(L, K, 1)
+    else:
+        mods_l = _top_general_primes(orc, L + K)
+        assert all((1 << 60) - q >= (1 << 32) and 260 * (q - 1) ** 2 >= 1 << 128 for q in mods_l)
+        ctx = Context(mods_l[:L], mods_l[L:], 1)
     mods = torch.tensor(np.array(ctx.mods, dtype=np.uint64).view(np.int64), device="cuda")
     LK = L + K
     top = (mods - 1).view(1, 1, LK, 1)
