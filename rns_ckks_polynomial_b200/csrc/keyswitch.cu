@@ -28,6 +28,7 @@
 
 #include "internal.cuh"
 #include "ntt.cuh"
+#include "split.cuh"
 
 namespace ckks {
 
@@ -265,36 +266,7 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 constexpr int kKiB = 4;       // ciphertexts per thread
 constexpr int kKiThreads = 128;
 constexpr int kKiFold = 256;  // digits summed exactly in 128 bits between reductions
-constexpr int kKiSplitFold = 8;  // digits between folds of the split accumulators
 constexpr int kKiMinBlocks = 4;
-
-// Split form (every prime 2^60 - delta, delta < 2^32, and every operand below 2^60): with
-// a = a1 2^30 + a0 and b = b1 2^30 + b0 (halves below 2^30),
-//     a b = a1 b1 2^60 + (a1 b0 + a0 b1) 2^30 + a0 b0,
-// each partial product below 2^60, so one 32 x 32 -> 64-bit multiply-add adds it into one of three
-// 64-bit sums (s2, s1, s0) without any carry handling.  Every kKiSplitFold digits the sums are
-// folded back below their bounds: s1 moves into s2 and s0, s0's bits from 2^60 up into s2, and s2's
-// bits from 2^60 up (its 2^120 part) come back as (s2 >> 60) delta, since 2^60 = delta (mod q).
-// Bounds: after a fold s0 < 2^60, s1 = 0, s2 < 2^60 + 2^36; a block of 8 digits adds below 8 2^60 to
-// s0 and s2 and below 16 2^60 to s1, all below 2^64.
-__device__ __forceinline__ u32 lo30(u64 a) { return (u32)a & 0x3FFFFFFFu; }
-__device__ __forceinline__ u32 hi30(u64 a) { return __funnelshift_r((u32)a, (u32)(a >> 32), 30); }
-__device__ __forceinline__ void madw(u64 &acc, u32 a, u32 b)
-{
-    asm("mad.wide.u32 %0, %1, %2, %0;" : "+l"(acc) : "r"(a), "r"(b));
-}
-__device__ __forceinline__ void split_fold(u64 &s0, u64 &s1, u64 &s2, u32 delta)
-{
-    constexpr u64 kM60 = (1ull << 60) - 1;
-    s2 += s1 >> 30;
-    s0 += (s1 & 0x3FFFFFFFull) << 30;
-    s1 = 0;
-    s2 += s0 >> 60;
-    s0 &= kM60;
-    u64 f = s2 & kM60;
-    madw(f, (u32)(s2 >> 60), delta);
-    s2 = f;
-}
 
 template <bool kSplit>
 __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
@@ -327,8 +299,8 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
 #pragma unroll
             for (int b = 0; b < kKiB; ++b) s0[c][b] = s1[c][b] = s2[c][b] = 0;
         const u32 delta = (u32)pc.delta;
-        for (int j0 = 0; j0 < T.dnum; j0 += kKiSplitFold) {
-            const int j1 = min(T.dnum, j0 + kKiSplitFold);
+        for (int j0 = 0; j0 < T.dnum; j0 += kSplitFold) {
+            const int j1 = min(T.dnum, j0 + kSplitFold);
 #pragma unroll 4
             for (int j = j0; j < j1; ++j) {
                 const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
@@ -341,12 +313,7 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
                 for (int b = 0; b < kKiB; ++b) {
                     const u32 d0 = lo30(d[b]), d1 = hi30(d[b]);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        madw(s2[c][b], d1, k1[c]);
-                        madw(s1[c][b], d1, k0[c]);
-                        madw(s1[c][b], d0, k1[c]);
-                        madw(s0[c][b], d0, k0[c]);
-                    }
+                    for (int c = 0; c < 2; ++c) split_mac(s0[c][b], s1[c][b], s2[c][b], d0, d1, k0[c], k1[c]);
                 }
             }
 #pragma unroll
@@ -358,48 +325,47 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
         for (int b = 0; b < kKiB; ++b) {
             if (b < nb) {
                 u64 *o = acc + ((size_t)(r * per_key + b0 + b) * 2 * T.LK + t) * kN + k;
-                // s2 2^60 + s0 with s0 < 2^60: the words of the 128-bit value are (s2 >> 4, s2 << 60 | s0)
-                o[0] = reduce128(s2[0][b] >> 4, (s2[0][b] << 60) | s0[0][b], pc);
-                o[LKn] = reduce128(s2[1][b] >> 4, (s2[1][b] << 60) | s0[1][b], pc);
+                o[0] = split_reduce(s0[0][b], s2[0][b], pc);
+                o[LKn] = split_reduce(s0[1][b], s2[1][b], pc);
             }
         }
-        return;
-    }
-    u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
+    } else {
+        u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
 #pragma unroll
-    for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
-    // 256 products below 2^120 plus a folded value below 2^60 stay below
-    // 2^128: past 256 digits the sums are reduced once per block of 256
-    for (int j0 = 0; j0 < T.dnum; j0 += kKiFold) {
-        if (j0 > 0) {
+        for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
+        // 256 products below 2^120 plus a folded value below 2^60 stay below
+        // 2^128: past 256 digits the sums are reduced once per block of 256
+        for (int j0 = 0; j0 < T.dnum; j0 += kKiFold) {
+            if (j0 > 0) {
 #pragma unroll
-            for (int b = 0; b < kKiB; ++b) {
-                l0[b] = reduce128(h0[b], l0[b], pc);
-                l1[b] = reduce128(h1[b], l1[b], pc);
-                h0[b] = h1[b] = 0;
+                for (int b = 0; b < kKiB; ++b) {
+                    l0[b] = reduce128(h0[b], l0[b], pc);
+                    l1[b] = reduce128(h1[b], l1[b], pc);
+                    h0[b] = h1[b] = 0;
+                }
             }
-        }
-        const int j1 = min(T.dnum, j0 + kKiFold);
+            const int j1 = min(T.dnum, j0 + kKiFold);
 #pragma unroll 4
-        for (int j = j0; j < j1; ++j) {
-            const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
-            const u64 *dj = dg + (size_t)j * LKn;
-            u64 d[kKiB];
+            for (int j = j0; j < j1; ++j) {
+                const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
+                const u64 *dj = dg + (size_t)j * LKn;
+                u64 d[kKiB];
 #pragma unroll
-            for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
+                for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
 #pragma unroll
-            for (int b = 0; b < kKiB; ++b) {
-                mac128(h0[b], l0[b], d[b], kb);
-                mac128(h1[b], l1[b], d[b], ka);
+                for (int b = 0; b < kKiB; ++b) {
+                    mac128(h0[b], l0[b], d[b], kb);
+                    mac128(h1[b], l1[b], d[b], ka);
+                }
             }
         }
-    }
 #pragma unroll
-    for (int b = 0; b < kKiB; ++b) {
-        if (b < nb) {
-            u64 *o = acc + ((size_t)(r * per_key + b0 + b) * 2 * T.LK + t) * kN + k;
-            o[0] = reduce128(h0[b], l0[b], pc);
-            o[LKn] = reduce128(h1[b], l1[b], pc);
+        for (int b = 0; b < kKiB; ++b) {
+            if (b < nb) {
+                u64 *o = acc + ((size_t)(r * per_key + b0 + b) * 2 * T.LK + t) * kN + k;
+                o[0] = reduce128(h0[b], l0[b], pc);
+                o[LKn] = reduce128(h1[b], l1[b], pc);
+            }
         }
     }
 }
