@@ -74,7 +74,8 @@ enum ckks_op {
     CKKS_OP_BSGS = 7,
     CKKS_OP_ROTATE_UNHOISTED = 8,
     CKKS_OP_MODRAISE = 9,       /* aux: l, the input's prime count */
-    CKKS_OP_CONJ_EXTRACT = 10
+    CKKS_OP_CONJ_EXTRACT = 10,
+    CKKS_OP_ROTATE_STREAMED = 11  /* aux: number of keys */
 };
 
 /* Pointwise operation codes for ckks_pointwise. */
@@ -169,7 +170,7 @@ int ckks_ctx_set_key_chain(ckks_ctx *ctx, int key_L);
 int ckks_ctx_params(const ckks_ctx *ctx, int *L, int *K, int *alpha, int *dnum, int *n);
 
 /* Bytes of workspace that `op` needs for `batch` inputs.  aux: number of keys
- * for CKKS_OP_ROTATE, input limb count (level + 1) for CKKS_OP_RESCALE,
+ * for CKKS_OP_ROTATE and CKKS_OP_ROTATE_STREAMED, input limb count (level + 1) for CKKS_OP_RESCALE,
  * bb * 1000 + gg for CKKS_OP_BSGS, ignored otherwise.  Returns 0 for an
  * unknown op or a null context. */
 size_t ckks_workspace_bytes(const ckks_ctx *ctx, int op, int batch, int aux);
@@ -322,6 +323,25 @@ int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *
 int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
                           const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
                           ckks_stream_t stream);
+
+/* a8 with ModUp, NTT and the key inner product fused by streaming: the same
+ * hoisted rotations as ckks_rotate, word for word, without the extended
+ * digits [batch][dnum][L+K][n] ever existing as a whole (1.24 GB per
+ * ciphertext at 2100 + 60 primes, alpha = 60; the boot-level rotation
+ * dominates the boot: Kestrel engine write-up, section 5.3 profile).  The
+ * primes are cut into windows of at most 20, each inside one digit's range
+ * or inside the special primes; per window the int8 tensor-core conversion
+ * (folded form) writes every digit's limbs at the window's primes into one
+ * buffer of batch * dnum * 20 limbs (the window's own digit gets the input's
+ * limbs), the forward NTT runs over it and the key inner product consumes
+ * it.  ModDown then runs as in ckks_rotate.  The first call builds the
+ * windows' conversion tables (one 128 KiB block per window and digit).
+ * Arguments, layouts and errors as ckks_rotate, plus CKKS_EUNSUPPORTED when
+ * alpha or K exceeds 64.  Each chunk of 64 keys repeats the windows' work.
+ * ws: ckks_workspace_bytes(CKKS_OP_ROTATE_STREAMED, batch, nkeys). */
+int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
+                         const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
+                         ckks_stream_t stream);
 
 /* ---------------------------------------------------------------- a10: rescale */
 

@@ -18,6 +18,7 @@ PW = {"mul": 0, "add": 1, "sub": 2}
 OP_MODUP, OP_MODDOWN, OP_KEYSWITCH, OP_ROTATE, OP_RESCALE, OP_MRR, OP_BSGS = 1, 2, 3, 4, 5, 6, 7
 OP_ROTATE_UNHOISTED = 8
 OP_MODRAISE, OP_CONJ_EXTRACT = 9, 10
+OP_ROTATE_STREAMED = 11
 
 
 def primes(count, n=N):
@@ -250,6 +251,22 @@ class Context:
         ws, wp = self._ws(ws, OP_ROTATE, B, nk)
         check("ckks_rotate", lib().ckks_rotate(self._h, _ptr(ct, "ct"), kp, gp, nk, _ptr(out, "out"),
                                                B, wp, _stream(ct)))
+        return out
+
+    def rotate_streamed(self, ct, keys, galois, out=None, ws=None):
+        """The hoisted rotations of rotate(), word for word, with ModUp -> NTT -> inner product
+        streamed over windows of at most 20 primes (no [B][dnum][L+K][n] digit tensor)."""
+        B = ct.shape[0]
+        nk = len(keys)
+        _ptr(ct, "ct", (B, 2, self.L, self.n))
+        kp = (C.c_void_p * max(1, nk))(*[_ptr(k, "key", self._kshape).value
+                                        for k in keys])
+        gp = (C.c_uint32 * max(1, nk))(*[int(g) for g in galois])
+        out = self._empty(nk, B, 2, self.L, self.n) if out is None else out
+        ws, wp = self._ws(ws, OP_ROTATE_STREAMED, B, nk)
+        check("ckks_rotate_streamed",
+              lib().ckks_rotate_streamed(self._h, _ptr(ct, "ct"), kp, gp, nk, _ptr(out, "out"), B, wp,
+                                         _stream(ct)))
         return out
 
     def rotate_unhoisted(self, ct, keys, galois, out=None, ws=None):

@@ -86,6 +86,15 @@ struct ckks_ctx {
     // host copies of the conversion matrices, for the folded tables built on first use
     std::vector<u64> up_mat_host, dn_mat_host;
     bool fold_built = false;
+    // Prime windows of the streamed rotation (built on first use, conv_fold.cu): window w covers
+    // primes t0 .. t0 + n - 1, all inside digit `own`'s range, or all special primes (own = -1);
+    // fold_win holds one folded block per (window, digit) for the digits that convert into it.
+    struct Window {
+        int t0, n, own;
+    };
+    std::vector<Window> windows;
+    const uint8_t *fold_win = nullptr;  // [windows][dnum][8][32][512]
+    bool win_built = false;
 };
 
 namespace ckks {

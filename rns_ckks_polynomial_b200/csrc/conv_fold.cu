@@ -172,7 +172,9 @@ __device__ __forceinline__ void fst32(uint32_t taddr, const u64 (&v)[16])
 }
 
 // Job geometry (kind 0: ModUp over (ciphertext, digit), the ciphertext fastest in the grid so the
-// CTAs that share a digit's F block run together; kind 1: ModDown over (job, component)).
+// CTAs that share a digit's F block run together; kind 1: ModDown over (job, component); kind 2:
+// ModUp of one prime window (primes w0 .. w0 + wn - 1) over (ciphertext, digit), into the window
+// buffer [batch][dnum][wbuf][n]; the window's own digit (wown) has no conversion).
 struct FoldJobs {
     int kind;
     const u64 *y;
@@ -180,6 +182,7 @@ struct FoldJobs {
     const uint8_t *fpl;   // F blocks
     int L, LK, alpha, dnum, K, tb_per_digit, batch;
     int csplit;
+    int win, w0, wn, wown, wbuf;  // kind 2
     __device__ __forceinline__ void geometry(int z, int &S, int &T, int &lo, const u64 *&ybase,
                                              const uint8_t *&fbase, int &zrow) const
     {
@@ -191,6 +194,14 @@ struct FoldJobs {
             ybase = y + ((size_t)b * L + lo) * kN;
             fbase = fpl + (size_t)jd * tb_per_digit * kFBlock;
             zrow = b * dnum + jd;
+        } else if (kind == 2) {
+            const int b = z % batch, jd = z / batch;
+            lo = jd * alpha;
+            S = min(alpha, L - lo);
+            T = jd == wown ? 0 : wn;
+            ybase = y + ((size_t)b * L + lo) * kN;
+            fbase = fpl + ((size_t)win * dnum + jd) * kFBlock;
+            zrow = b * dnum + jd;
         } else {
             lo = 0;
             S = K;
@@ -200,13 +211,17 @@ struct FoldJobs {
             zrow = z;
         }
     }
+    // the prime of target ti, and its row in the output block of job zrow
     __device__ __forceinline__ int prime(int ti, int lo, int S) const
     {
-        return kind == 0 ? (ti < lo ? ti : ti + S) : ti;
+        return kind == 0 ? (ti < lo ? ti : ti + S) : kind == 2 ? w0 + ti : ti;
     }
+    __device__ __forceinline__ int orow(int ti, int lo, int S) const { return kind == 2 ? ti : prime(ti, lo, S); }
     __device__ __forceinline__ u64 *row(int zrow, int t) const
     {
-        return kind == 0 ? out + ((size_t)zrow * LK + t) * kN : out + ((size_t)zrow * L + t) * kN;
+        return kind == 0   ? out + ((size_t)zrow * LK + t) * kN
+               : kind == 2 ? out + ((size_t)zrow * wbuf + t) * kN
+                           : out + ((size_t)zrow * L + t) * kN;
     }
 };
 
@@ -404,7 +419,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const int ti = tb * kFN + part * 8 + c;
-            toff[c] = ti < T ? jobs.prime(ti, lo, S) * kN + cbase + m : -1;
+            toff[c] = ti < T ? jobs.orow(ti, lo, S) * kN + cbase + m : -1;
         }
         const uint32_t tcol = tmem + lane_base + part * 8;
         for (int i = 0; i < ntiles && ok; ++i) {
@@ -459,27 +474,34 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
 // Host: the F blocks of a (targets x sources) matrix given by `at(ti, s)` over target primes
 // `prime(ti)`, one block of 32 targets after another, each in the shared-memory layout:
 // plane u, row r (target 32 tb + r), byte k' = 8 s + v holds byte u of 2^(8v) at(ti, s) mod q.
+// One block of 32 targets: targets ti0 .. ti0 + 31 (those below T) of F = 2^(8v) M mod q_t, at(ti, s)
+// giving M[s][target ti] and prime(ti) its prime index.
+template <class F, class P>
+void build_fold_block(uint8_t *blk, int ti0, int T, int S, const std::vector<u64> &mods, F at, P prime)
+{
+    for (int r = 0; r < kFN; ++r) {
+        const int ti = ti0 + r;
+        if (ti >= T) continue;
+        const u64 q = mods[prime(ti)];
+        for (int s = 0; s < S; ++s) {
+            u64 f = at(ti, s) % q;
+            for (int v = 0; v < 8; ++v) {
+                const int k = 8 * s + v;
+                for (int u = 0; u < kFPlanes; ++u)
+                    blk[(size_t)u * kFPlaneBytes + fcm_off(r, k)] = (uint8_t)(f >> (8 * u));
+                f = host_mulmod(f, 256 % q, q);
+            }
+        }
+    }
+}
+
 template <class F, class P>
 void build_fold(std::vector<uint8_t> &dst, size_t base, int T, int S, const std::vector<u64> &mods, F at,
                 P prime)
 {
     const int tbs = (T + kFN - 1) / kFN;
     parallel_for(tbs, [&](int tb) {
-        for (int r = 0; r < kFN; ++r) {
-            const int ti = tb * kFN + r;
-            if (ti >= T) continue;
-            const u64 q = mods[prime(ti)];
-            for (int s = 0; s < S; ++s) {
-                u64 f = at(ti, s) % q;
-                for (int v = 0; v < 8; ++v) {
-                    const int k = 8 * s + v;
-                    for (int u = 0; u < kFPlanes; ++u)
-                        dst[base + (size_t)tb * kFBlock + (size_t)u * kFPlaneBytes + fcm_off(r, k)] =
-                            (uint8_t)(f >> (8 * u));
-                    f = host_mulmod(f, 256 % q, q);
-                }
-            }
-        }
+        build_fold_block(dst.data() + base + (size_t)tb * kFBlock, tb * kFN, T, S, mods, at, prime);
     });
 }
 
@@ -557,6 +579,67 @@ static int ensure_fold_tables(ckks_ctx *ctx)
     CKKS_TRY(build_fold_tables(ctx));
     ctx->fold_built = true;
     return CKKS_OK;
+}
+
+// Windows of at most kWinMax primes: each digit's range and the special primes, each cut into
+// near-equal pieces.
+static void make_windows(const ckks_ctx *ctx, std::vector<ckks_ctx::Window> &out)
+{
+    auto split = [&](int a, int b, int own) {
+        const int len = b - a;
+        if (len <= 0) return;
+        const int cnt = (len + kWinMax - 1) / kWinMax;
+        for (int i = 0; i < cnt; ++i) {
+            const int s0 = a + (int)((long)len * i / cnt), s1 = a + (int)((long)len * (i + 1) / cnt);
+            out.push_back({s0, s1 - s0, own});
+        }
+    };
+    for (int j = 0; j < ctx->dnum; ++j) split(j * ctx->alpha, std::min(ctx->L, (j + 1) * ctx->alpha), j);
+    split(ctx->L, ctx->L + ctx->K, -1);
+}
+
+// The windows and their folded blocks: block (w, j) holds digit j's conversion into window w's
+// primes (none for the window's own digit), built once per context on the first streamed call.
+static int ensure_window_tables(ckks_ctx *ctx)
+{
+    CKKS_TRY(ensure_fold_tables(ctx));
+    std::lock_guard<std::mutex> lock(ctx->mu);
+    if (ctx->win_built) return CKKS_OK;
+    std::vector<ckks_ctx::Window> win;
+    make_windows(ctx, win);
+    const int nw = (int)win.size(), dnum = ctx->dnum, L = ctx->L, LK = L + ctx->K, alpha = ctx->alpha;
+    const std::vector<u64> &up_mat = ctx->up_mat_host;
+    std::vector<uint8_t> h((size_t)nw * dnum * kFBlock, 0);
+    parallel_for(nw * dnum, [&](int idx) {
+        const int w = idx / dnum, j = idx - w * dnum;
+        const ckks_ctx::Window wd = win[w];
+        if (wd.own == j) return;
+        const int S = std::min(alpha, L - j * alpha);
+        build_fold_block(h.data() + (size_t)idx * kFBlock, 0, wd.n, S, ctx->mods,
+                         [&](int ti, int s2) { return up_mat[((size_t)j * alpha + s2) * LK + wd.t0 + ti]; },
+                         [&](int ti) { return wd.t0 + ti; });
+    });
+    CKKS_TRY(upload_fold(ctx, h, &ctx->fold_win));
+    ctx->windows = std::move(win);
+    ctx->win_built = true;
+    return CKKS_OK;
+}
+
+int stream_windows(ckks_ctx *ctx, const std::vector<ckks_ctx::Window> **out)
+{
+    CKKS_TRY(ensure_window_tables(ctx));
+    *out = &ctx->windows;
+    return CKKS_OK;
+}
+
+int launch_conv_fold_window(ckks_ctx *ctx, const u64 *y, u64 *buf, int batch, int w, cudaStream_t s)
+{
+    CKKS_TRY(ensure_window_tables(ctx));
+    const Tables &T = ctx->t;
+    const ckks_ctx::Window wd = ctx->windows[w];
+    FoldJobs j{2, y, buf, ctx->fold_win, T.L, T.LK, T.alpha, T.dnum, T.K, 0, batch, 1,
+               w, wd.t0, wd.n, wd.own, kWinMax};
+    return launch_fold(ctx, j, 1, batch * T.dnum, s);
 }
 
 int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s)

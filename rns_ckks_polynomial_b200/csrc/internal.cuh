@@ -38,6 +38,11 @@ constexpr int kTcMinSources = 7;  // CKKS_CONV_AUTO: more sources (8 or more) us
 enum ConvKind { kConvInteger = 0, kConvTensor = 1, kConvFolded = 2 };
 ConvKind conv_kind(const ckks_ctx *ctx, int sources);
 int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
+// streamed rotation: prime windows of at most kWinMax primes (built with their folded blocks on
+// first use) and the conversion of y into window w's buffer [batch][dnum][kWinMax][n]
+constexpr int kWinMax = 20;
+int stream_windows(ckks_ctx *ctx, const std::vector<ckks_ctx::Window> **out);
+int launch_conv_fold_window(ckks_ctx *ctx, const u64 *y, u64 *buf, int batch, int w, cudaStream_t s);
 int launch_conv_fold_down(ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);
 int build_tc_tables(ckks_ctx *ctx, const std::vector<u64> &up_mat, const std::vector<u64> &dn_mat);
 int launch_conv_tc_up(const ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
@@ -54,6 +59,7 @@ void free_raise_tables(ckks_ctx *ctx);
 size_t modraise_ws_bytes(const ckks_ctx *ctx, int batch, int l);
 size_t conj_extract_ws_bytes(const ckks_ctx *ctx, int batch);
 size_t rotate_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys);
+size_t rotate_streamed_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys);
 
 // ---- sizes of internal stages (bytes)
 size_t modup_ws_bytes(const ckks_ctx *ctx, int batch);
@@ -73,6 +79,15 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 // hoisted (digits shared by all keys) and digit set z otherwise.
 int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, int per_key,
                     bool hoisted, u64 *acc, int jobs, cudaStream_t s);
+// The same over a digit view: digit j of ciphertext b at prime t is read at digits + b ct_stride
+// + j j_stride + (t - t_lo) n, for the primes t_lo .. t_lo + nt - 1 only (acc rows of the other
+// primes are left as they are).
+struct DigitView {
+    size_t ct_stride, j_stride;
+    int t_lo, nt;
+};
+int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, int per_key,
+                    bool hoisted, u64 *acc, int jobs, cudaStream_t s, const DigitView &dv);
 
 // What ModDown adds to its output after the P^-1 scaling.
 //  kind 0: nothing.

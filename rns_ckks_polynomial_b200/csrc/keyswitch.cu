@@ -168,7 +168,7 @@ struct UpInttJob {
         Ref r;
         r.src = in + off;
         r.src2 = kProduct ? in2 + off : nullptr;
-        r.copy = digits + (((size_t)b * dnum + i / alpha) * LK + i) * kN;
+        r.copy = digits ? digits + (((size_t)b * dnum + i / alpha) * LK + i) * kN : nullptr;
         r.yrow = y + ((size_t)b * L + i) * kN;
         r.h = hatinv[i];
         r.q = pc[i].q;
@@ -185,7 +185,7 @@ struct UpInttJob {
 #pragma unroll
             for (int k = 0; k < 4; ++k) v[k] = mulmod(v[k], w[k], c);
         }
-        st4(r.copy + e, v);
+        if (r.copy) st4(r.copy + e, v);
     }
     __device__ __forceinline__ void store(const Ref &r, int e, u64 v) const
     {
@@ -218,6 +218,27 @@ struct UpNttJob {
             jd = r - (t - L) * dnum;
         }
         return {digits + (((size_t)b * dnum + jd) * LK + t) * kN, t};
+    }
+    __device__ __forceinline__ u64 load(const Ref &r, int e) const { return r.row[e]; }
+    __device__ __forceinline__ void store4(const Ref &r, int e, const u64 *v) const { st4(r.row + e, v); }
+};
+
+// Forward NTT of one window's converted limbs: buf[b][j][tw][n] for every digit j but the window's
+// own (whose limbs are copies of the input, already in the NTT domain), prime t0 + tw.  Jobs run
+// ciphertext fastest, then digit, so consecutive jobs share a prime.
+struct WinNttJob {
+    u64 *buf;
+    int wbuf, t0, n, own, dnum, batch, count;
+    struct Ref {
+        u64 *row;
+        int prime;
+    };
+    __device__ __forceinline__ Ref ref(int j) const
+    {
+        const int b = j % batch, ndig = own >= 0 ? dnum - 1 : dnum;
+        const int r = j / batch, jj = r % ndig, tw = r / ndig;
+        const int jd = own >= 0 && jj >= own ? jj + 1 : jj;
+        return {buf + (((size_t)b * dnum + jd) * wbuf + tw) * kN, t0 + tw};
     }
     __device__ __forceinline__ u64 load(const Ref &r, int e) const { return r.row[e]; }
     __device__ __forceinline__ void store4(const Ref &r, int e, const u64 *v) const { st4(r.row + e, v); }
@@ -271,7 +292,7 @@ constexpr int kKiMinBlocks = 4;
 template <bool kSplit>
 __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
                                                         int per_key, int nkeys, int hoisted,
-                                                        u64 *__restrict__ acc, Tables T)
+                                                        u64 *__restrict__ acc, Tables T, DigitView dv)
 {
     const int nchunks = (per_key + kKiB - 1) / kKiB;
     int id = blockIdx.x;
@@ -280,14 +301,14 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
     const int r = id % nkeys;
     id /= nkeys;
     const int chunk = id % nchunks;
-    const int t = id / nchunks;
+    const int t = dv.t_lo + id / nchunks;
     const int b0 = chunk * kKiB, nb = min(kKiB, per_key - b0);
     const int k = tile * kKiThreads + threadIdx.x;
     const u32 g = kl.galois[r];
     const int src = g == 1u ? k : (int)galois_src((u32)k, g);
     const size_t LKn = (size_t)T.LK * kN;
-    const size_t bstride = (size_t)T.dnum * LKn;  // between the digit sets of consecutive ciphertexts
-    const u64 *dg = digits + (size_t)(hoisted ? b0 : r * per_key + b0) * bstride + (size_t)t * kN + src;
+    const size_t bstride = dv.ct_stride;  // between the digit sets of consecutive ciphertexts
+    const u64 *dg = digits + (size_t)(hoisted ? b0 : r * per_key + b0) * bstride + (size_t)(t - dv.t_lo) * kN + src;
     const size_t kLKn = (size_t)T.key_LK * kN;  // key rows per (digit, component)
     const int kt = t < T.L ? t : t - T.L + T.key_L;
     const u64 *kp = kl.key[r] + (size_t)kt * kN + k;
@@ -305,7 +326,7 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
             for (int j = j0; j < j1; ++j) {
                 const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
                 const u32 k0[2] = {lo30(kb), lo30(ka)}, k1[2] = {hi30(kb), hi30(ka)};
-                const u64 *dj = dg + (size_t)j * LKn;
+                const u64 *dj = dg + (size_t)j * dv.j_stride;
                 u64 d[kKiB];
 #pragma unroll
                 for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
@@ -348,7 +369,7 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
 #pragma unroll 4
             for (int j = j0; j < j1; ++j) {
                 const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
-                const u64 *dj = dg + (size_t)j * LKn;
+                const u64 *dj = dg + (size_t)j * dv.j_stride;
                 u64 d[kKiB];
 #pragma unroll
                 for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
@@ -371,19 +392,29 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
 }
 
 int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, int per_key,
-                    bool hoisted, u64 *acc, int jobs, cudaStream_t s)
+                    bool hoisted, u64 *acc, int jobs, cudaStream_t s, const DigitView &dv)
 {
-    if (jobs <= 0) return CKKS_OK;
+    if (jobs <= 0 || dv.nt <= 0) return CKKS_OK;
     const Tables &T = ctx->t;
     const int nkeys = jobs / per_key;
-    const size_t blocks = (size_t)(kN / kKiThreads) * nkeys * ((per_key + kKiB - 1) / kKiB) * T.LK;
+    const size_t blocks = (size_t)(kN / kKiThreads) * nkeys * ((per_key + kKiB - 1) / kKiB) * dv.nt;
     if (blocks > 0x7fffffffull) return set_error(CKKS_EUNSUPPORTED, "key inner product grid too large");
     if (T.special)
-        key_inner_kernel<true><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T);
+        key_inner_kernel<true><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0,
+                                                                       acc, T, dv);
     else
-        key_inner_kernel<false><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T);
+        key_inner_kernel<false><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0,
+                                                                        acc, T, dv);
     CKKS_CHECK_LAUNCH("key_inner_kernel");
     return CKKS_OK;
+}
+
+int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, int per_key,
+                    bool hoisted, u64 *acc, int jobs, cudaStream_t s)
+{
+    const Tables &T = ctx->t;
+    const DigitView dv{(size_t)T.dnum * T.LK * kN, (size_t)T.LK * kN, 0, T.LK};
+    return key_inner_stage(ctx, digits, kl, per_key, hoisted, acc, jobs, s, dv);
 }
 
 // ---------------------------------------------------------------- ModDown
@@ -564,11 +595,23 @@ size_t rotate_ws(const ckks_ctx *ctx, int batch, int nkeys)
            std::max(modup_ws_bytes(ctx, batch), moddown_ws_bytes(ctx, chunk * batch));
 }
 
+// ModUp's sources y, one window of digits, the accumulators of a key chunk and ModDown's scratch.
+size_t rotate_streamed_ws(const ckks_ctx *ctx, int batch, int nkeys)
+{
+    const int chunk = std::min(std::max(nkeys, 1), kMaxKeys);
+    return limbs_bytes((size_t)batch * ctx->L) + limbs_bytes((size_t)batch * ctx->dnum * kWinMax) +
+           limbs_bytes((size_t)chunk * batch * 2 * (ctx->L + ctx->K)) + moddown_ws_bytes(ctx, chunk * batch);
+}
+
 }  // namespace
 
 namespace ckks {
 size_t keyswitch_ws_bytes(const ckks_ctx *ctx, int batch) { return keyswitch_ws(ctx, batch); }
 size_t rotate_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys) { return rotate_ws(ctx, batch, nkeys); }
+size_t rotate_streamed_ws_bytes(const ckks_ctx *ctx, int batch, int nkeys)
+{
+    return rotate_streamed_ws(ctx, batch, nkeys);
+}
 }  // namespace ckks
 
 extern "C" int ckks_modup(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int batch,
@@ -690,6 +733,83 @@ extern "C" int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64
         CKKS_TRY(key_inner_stage(ctx, digits, kl, batch, true, acc, nk * batch, s));
         CKKS_TRY(moddown_stage(ctx, acc, out + (size_t)r0 * batch * ct_elems, nk * batch, ex,
                                scratch, s));
+    }
+    return CKKS_OK;
+}
+
+// The rotation of ckks_rotate with ModUp -> NTT -> inner product streamed over windows of at most
+// kWinMax primes: per window, the folded conversion writes every digit's limbs at the window's
+// primes into one window buffer (the window's own digit gets the input's limbs), the forward NTT
+// runs over it and the key inner product consumes it, so the extended digits never exist as a
+// whole.  ModDown then runs as in ckks_rotate.
+extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
+                                    const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
+                                    ckks_stream_t stream)
+{
+    CKKS_TRY(check_ctx(ctx));
+    CKKS_TRY(check_batch(batch));
+    if (nkeys < 0) return set_error(CKKS_EINVAL, "negative key count");
+    if (batch == 0 || nkeys == 0) return CKKS_OK;
+    if (!keys || !galois) return set_error(CKKS_EINVAL, "null key or galois array");
+    for (int r = 0; r < nkeys; ++r) {
+        CKKS_TRY(check_ptr(keys[r], "keys[r]"));
+        if ((galois[r] & 1u) == 0) return set_error(CKKS_EINVAL, "galois element must be odd");
+    }
+    if ((size_t)nkeys * batch > 32767) return set_error(CKKS_EUNSUPPORTED, "nkeys * batch above 32767");
+    if (ctx->alpha > 64 || ctx->K > 64) return set_error(CKKS_EUNSUPPORTED, "more than 64 sources per conversion");
+    CKKS_TRY(check_ptr(ct, "ct"));
+    CKKS_TRY(check_ptr(out, "out"));
+    CKKS_TRY(set_device(ctx));
+    ckks_ctx *mctx = const_cast<ckks_ctx *>(ctx);
+    const std::vector<ckks_ctx::Window> *wins = nullptr;
+    CKKS_TRY(stream_windows(mctx, &wins));
+    void *w;
+    CKKS_TRY(resolve_ws(mctx, ws, rotate_streamed_ws(ctx, batch, nkeys), &w));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const Tables &T = ctx->t;
+    const int L = ctx->L, LK = L + ctx->K, dnum = ctx->dnum;
+    const size_t ct_elems = (size_t)2 * L * kN;
+    const int chunk = std::min(nkeys, kMaxKeys);
+    Carve c(w);
+    u64 *y = c.take<u64>((size_t)batch * L * kN);
+    u64 *buf = c.take<u64>((size_t)batch * dnum * kWinMax * kN);
+    u64 *acc = c.take<u64>((size_t)chunk * batch * 2 * LK * kN);
+    void *scratch = c.base + c.off;
+    // ModUp's sources: y = INTT(c1) times [(Q_j/q_i)^-1]
+    const u64 *c1 = ct + (size_t)L * kN;
+    UpInttJob<false> ij{c1, nullptr, ct_elems, nullptr, y, T.up_hatinv, T.pc, L, LK, T.alpha, dnum, batch,
+                        L * batch};
+    CKKS_TRY(launch_ntt_inv(ij, T, s));
+    for (int r0 = 0; r0 < nkeys; r0 += chunk) {
+        const int nk = std::min(chunk, nkeys - r0);
+        KeyList kl{};
+        DownExtra ex;
+        ex.kind = 1;
+        ex.ct = ct;
+        ex.ct_bstride = ct_elems;
+        ex.ct_mod = batch;
+        ex.per = batch;
+        for (int r = 0; r < nk; ++r) {
+            kl.key[r] = keys[r0 + r];
+            kl.galois[r] = ex.gal[r] = galois[r0 + r] & (2u * kN - 1u);
+        }
+        for (int wi = 0; wi < (int)wins->size(); ++wi) {
+            const ckks_ctx::Window wd = (*wins)[wi];
+            CKKS_TRY(launch_conv_fold_window(mctx, y, buf, batch, wi, s));
+            if (wd.own >= 0) {
+                cudaError_t e = cudaMemcpy2DAsync(buf + (size_t)wd.own * kWinMax * kN,
+                                                  (size_t)dnum * kWinMax * kN * sizeof(u64), c1 + (size_t)wd.t0 * kN,
+                                                  ct_elems * sizeof(u64), (size_t)wd.n * kN * sizeof(u64), batch,
+                                                  cudaMemcpyDeviceToDevice, s);
+                if (e != cudaSuccess) return cuda_status(e, "cudaMemcpy2DAsync(window digit copy)");
+            }
+            WinNttJob nj{buf, kWinMax, wd.t0, wd.n, wd.own, dnum, batch,
+                         batch * (wd.own >= 0 ? dnum - 1 : dnum) * wd.n};
+            CKKS_TRY(launch_ntt_fwd(nj, T, s));
+            const DigitView dv{(size_t)dnum * kWinMax * kN, (size_t)kWinMax * kN, wd.t0, wd.n};
+            CKKS_TRY(key_inner_stage(ctx, buf, kl, batch, true, acc, nk * batch, s, dv));
+        }
+        CKKS_TRY(moddown_stage(ctx, acc, out + (size_t)r0 * batch * ct_elems, nk * batch, ex, scratch, s));
     }
     return CKKS_OK;
 }

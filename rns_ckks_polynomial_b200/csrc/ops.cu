@@ -285,6 +285,7 @@ extern "C" size_t ckks_workspace_bytes(const ckks_ctx *ctx, int op, int batch, i
     case CKKS_OP_MODDOWN: return moddown_ws_bytes(ctx, batch);
     case CKKS_OP_KEYSWITCH: return keyswitch_ws_bytes(ctx, batch);
     case CKKS_OP_ROTATE: return rotate_ws_bytes(ctx, batch, aux);
+    case CKKS_OP_ROTATE_STREAMED: return rotate_streamed_ws_bytes(ctx, batch, aux);
     case CKKS_OP_ROTATE_UNHOISTED: return rotate_unhoisted_ws(ctx, batch);
     case CKKS_OP_MODRAISE: return aux >= 1 ? modraise_ws_bytes(ctx, batch, aux) : 0;
     case CKKS_OP_CONJ_EXTRACT: return conj_extract_ws_bytes(ctx, batch);

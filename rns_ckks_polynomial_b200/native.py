@@ -49,6 +49,8 @@ SIGNATURES = {
                               C.c_int, _vp, _vp]),
     "ckks_rotate_unhoisted": (C.c_int, [_vp, _vp, C.POINTER(_vp), C.POINTER(C.c_uint32), C.c_int, _vp,
                               C.c_int, _vp, _vp]),
+    "ckks_rotate_streamed": (C.c_int, [_vp, _vp, C.POINTER(_vp), C.POINTER(C.c_uint32), C.c_int, _vp,
+                             C.c_int, _vp, _vp]),
     "ckks_rescale": (C.c_int, [_vp, _vp, _vp, C.c_int, C.c_int, _vp, _vp]),
     "ckks_mul_relin_rescale": (C.c_int, [_vp, _vp, _vp, _vp, _vp, C.c_int, _vp, _vp]),
     "ckks_bsgs_lintrans": (C.c_int, [_vp, _vp, _vp, C.POINTER(_vp), C.POINTER(_vp), C.c_int,
