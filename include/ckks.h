@@ -329,10 +329,10 @@ int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_
  * digits [batch][dnum][L+K][n] ever existing as a whole (1.24 GB per
  * ciphertext at 2100 + 60 primes, alpha = 60; the boot-level rotation
  * dominates the boot: Kestrel engine write-up, section 5.3 profile).  The
- * primes are cut into windows of at most 20, each inside one digit's range
+ * primes are cut into windows of at most 30, each inside one digit's range
  * or inside the special primes; per window the int8 tensor-core conversion
  * (folded form) writes every digit's limbs at the window's primes into one
- * buffer of batch * dnum * 20 limbs (the window's own digit gets the input's
+ * buffer of batch * dnum * 30 limbs (the window's own digit gets the input's
  * limbs), the forward NTT runs over it and the key inner product consumes
  * it.  ModDown then runs as in ckks_rotate.  The first call builds the
  * windows' conversion tables (one 128 KiB block per window and digit).

@@ -523,7 +523,12 @@ int launch_fold(const ckks_ctx *ctx, FoldJobs j, int tbs, int jobs, cudaStream_t
 {
     if (jobs <= 0) return CKKS_OK;
     const long ctas = (long)tbs * jobs;
-    j.csplit = ctas >= 148 * 4 ? 1 : ctas >= 148 * 2 ? 2 : 4;  // 16, 8 or 4 tiles per run
+    // 16, 8 or 4 tiles per run; a window's conversion (kind 2) keeps whole runs down to one wave,
+    // since every CTA pays the table load and the pipeline fill once
+    if (j.kind == 2)
+        j.csplit = ctas >= 148 ? 1 : ctas >= 74 ? 2 : 4;
+    else
+        j.csplit = ctas >= 148 * 4 ? 1 : ctas >= 148 * 2 ? 2 : 4;
     const dim3 grid(tbs * j.csplit, jobs);
     if (ctx->t.tc_special)
         conv_fold_kernel<true><<<grid, kFThreads, kFSmemBytes, s>>>(j, ctx->t.pc, ctx->tc_err);
