@@ -535,7 +535,7 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
             ctx.device_status()
         if "boot_rotation_streamed" in entries:
             # the same rotations with ModUp -> NTT -> inner product streamed over windows of at most
-            # 30 primes, without the [B][dnum][L+K][n] digit tensor (bit-identical output); the first
+            # 60 primes, without the [B][dnum][L+K][n] digit tensor (bit-identical output); the first
             # call builds the windows' conversion tables, outside the timing
             ws_s = torch.empty(ctx.workspace_bytes(11, B, R), dtype=torch.uint8, device=dev)
             ctx.rotate_streamed(ct, keys, gal, out=res, ws=ws_s)
@@ -544,8 +544,9 @@ def run_keyswitch(dev, hbm_peak, ipeak, B=8, R=4, entries=KS_ENTRIES, refresh_ba
             e = ks_entry(B * R, ms, work_rotation(2100, 60, 60, B, R), hbm_peak, rates, clk)
             e["workspace_bytes"] = int(ws_s.numel())
             e["hoisted_workspace_bytes"] = int(ws.numel())
-            e["note"] = ("ModUp -> NTT -> key inner product per window of at most 30 primes (folded "
-                         "conversion, window buffer of B x 35 x 30 limbs); ModDown as in the hoisted call")
+            e["note"] = ("ModUp -> NTT -> key inner product per window of at most 60 primes (folded "
+                         "conversion, two window buffers of B x 35 x 60 limbs on two streams); ModDown "
+                         "as in the hoisted call")
             out["boot_rotation_L2100_streamed"] = e
             ctx.device_status()
             del ws_s

@@ -329,13 +329,15 @@ int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_
  * digits [batch][dnum][L+K][n] ever existing as a whole (1.24 GB per
  * ciphertext at 2100 + 60 primes, alpha = 60; the boot-level rotation
  * dominates the boot: Kestrel engine write-up, section 5.3 profile).  The
- * primes are cut into windows of at most 30, each inside one digit's range
+ * primes are cut into windows of at most 60, each inside one digit's range
  * or inside the special primes; per window the int8 tensor-core conversion
  * (folded form) writes every digit's limbs at the window's primes into one
- * buffer of batch * dnum * 30 limbs (the window's own digit gets the input's
+ * buffer of batch * dnum * 60 limbs (the window's own digit gets the input's
  * limbs), the forward NTT runs over it and the key inner product consumes
- * it.  ModDown then runs as in ckks_rotate.  The first call builds the
- * windows' conversion tables (one 128 KiB block per window and digit).
+ * it; consecutive windows alternate between the caller's stream and a second
+ * stream (one stream while the caller's is being captured into a graph).
+ * ModDown then runs as in ckks_rotate.  The first call builds the windows'
+ * conversion tables (two 128 KiB blocks of 32 targets per window and digit).
  * Arguments, layouts and errors as ckks_rotate, plus CKKS_EUNSUPPORTED when
  * alpha or K exceeds 64.  Each chunk of 64 keys repeats the windows' work.
  * ws: ckks_workspace_bytes(CKKS_OP_ROTATE_STREAMED, batch, nkeys). */

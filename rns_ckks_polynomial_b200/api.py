@@ -255,7 +255,7 @@ class Context:
 
     def rotate_streamed(self, ct, keys, galois, out=None, ws=None):
         """The hoisted rotations of rotate(), word for word, with ModUp -> NTT -> inner product
-        streamed over windows of at most 30 primes (no [B][dnum][L+K][n] digit tensor)."""
+        streamed over windows of at most 60 primes (no [B][dnum][L+K][n] digit tensor)."""
         B = ct.shape[0]
         nk = len(keys)
         _ptr(ct, "ct", (B, 2, self.L, self.n))

@@ -93,7 +93,7 @@ struct ckks_ctx {
         int t0, n, own;
     };
     std::vector<Window> windows;
-    const uint8_t *fold_win = nullptr;  // [windows][dnum][8][32][512]
+    const uint8_t *fold_win = nullptr;  // [windows][dnum][blocks of 32 targets][8][32][512]
     bool win_built = false;
 };
 

@@ -50,6 +50,7 @@ namespace {
 
 constexpr int kFM = 128;                          // coefficients per tile (MMA M, TMEM lanes)
 constexpr int kFN = 32;                           // targets per CTA (MMA N)
+constexpr int kWinBlocks = (kWinMax + kFN - 1) / kFN;  // target blocks per streamed window
 constexpr int kFKP = 512;                         // K' extent in bytes: 64 sources x 8 bytes
 constexpr int kFPlanes = 8;
 constexpr int kFPlaneBytes = kFN * kFKP;          // 16 KiB
@@ -173,8 +174,9 @@ __device__ __forceinline__ void fst32(uint32_t taddr, const u64 (&v)[16])
 
 // Job geometry (kind 0: ModUp over (ciphertext, digit), the ciphertext fastest in the grid so the
 // CTAs that share a digit's F block run together; kind 1: ModDown over (job, component); kind 2:
-// ModUp of one prime window (primes w0 .. w0 + wn - 1) over (ciphertext, digit), into the window
-// buffer [batch][dnum][wbuf][n]; the window's own digit (wown) has no conversion).
+// ModUp of one prime window (primes w0 .. w0 + wn - 1, in tb_per_digit blocks of 32) over
+// (ciphertext, digit), into the window buffer [batch][dnum][wbuf][n]; the window's own digit (wown)
+// has no conversion).
 struct FoldJobs {
     int kind;
     const u64 *y;
@@ -200,7 +202,7 @@ struct FoldJobs {
             S = min(alpha, L - lo);
             T = jd == wown ? 0 : wn;
             ybase = y + ((size_t)b * L + lo) * kN;
-            fbase = fpl + ((size_t)win * dnum + jd) * kFBlock;
+            fbase = fpl + ((size_t)win * dnum + jd) * tb_per_digit * kFBlock;
             zrow = b * dnum + jd;
         } else {
             lo = 0;
@@ -603,8 +605,9 @@ static void make_windows(const ckks_ctx *ctx, std::vector<ckks_ctx::Window> &out
     split(ctx->L, ctx->L + ctx->K, -1);
 }
 
-// The windows and their folded blocks: block (w, j) holds digit j's conversion into window w's
-// primes (none for the window's own digit), built once per context on the first streamed call.
+// The windows and their folded blocks: blocks (w, j, 0 .. kWinBlocks - 1) hold digit j's conversion
+// into window w's primes (none for the window's own digit), built once per context on the first
+// streamed call.
 static int ensure_window_tables(ckks_ctx *ctx)
 {
     CKKS_TRY(ensure_fold_tables(ctx));
@@ -614,13 +617,13 @@ static int ensure_window_tables(ckks_ctx *ctx)
     make_windows(ctx, win);
     const int nw = (int)win.size(), dnum = ctx->dnum, L = ctx->L, LK = L + ctx->K, alpha = ctx->alpha;
     const std::vector<u64> &up_mat = ctx->up_mat_host;
-    std::vector<uint8_t> h((size_t)nw * dnum * kFBlock, 0);
-    parallel_for(nw * dnum, [&](int idx) {
-        const int w = idx / dnum, j = idx - w * dnum;
+    std::vector<uint8_t> h((size_t)nw * dnum * kWinBlocks * kFBlock, 0);
+    parallel_for(nw * dnum * kWinBlocks, [&](int idx) {
+        const int tb = idx % kWinBlocks, wj = idx / kWinBlocks, w = wj / dnum, j = wj - w * dnum;
         const ckks_ctx::Window wd = win[w];
         if (wd.own == j) return;
         const int S = std::min(alpha, L - j * alpha);
-        build_fold_block(h.data() + (size_t)idx * kFBlock, 0, wd.n, S, ctx->mods,
+        build_fold_block(h.data() + (size_t)idx * kFBlock, tb * kFN, wd.n, S, ctx->mods,
                          [&](int ti, int s2) { return up_mat[((size_t)j * alpha + s2) * LK + wd.t0 + ti]; },
                          [&](int ti) { return wd.t0 + ti; });
     });
@@ -642,9 +645,9 @@ int launch_conv_fold_window(ckks_ctx *ctx, const u64 *y, u64 *buf, int batch, in
     CKKS_TRY(ensure_window_tables(ctx));
     const Tables &T = ctx->t;
     const ckks_ctx::Window wd = ctx->windows[w];
-    FoldJobs j{2, y, buf, ctx->fold_win, T.L, T.LK, T.alpha, T.dnum, T.K, 0, batch, 1,
+    FoldJobs j{2, y, buf, ctx->fold_win, T.L, T.LK, T.alpha, T.dnum, T.K, kWinBlocks, batch, 1,
                w, wd.t0, wd.n, wd.own, kWinMax};
-    return launch_fold(ctx, j, 1, batch * T.dnum, s);
+    return launch_fold(ctx, j, (wd.n + kFN - 1) / kFN, batch * T.dnum, s);
 }
 
 int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s)

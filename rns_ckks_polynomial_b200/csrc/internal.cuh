@@ -40,7 +40,7 @@ ConvKind conv_kind(const ckks_ctx *ctx, int sources);
 int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
 // streamed rotation: prime windows of at most kWinMax primes (built with their folded blocks on
 // first use) and the conversion of y into window w's buffer [batch][dnum][kWinMax][n]
-constexpr int kWinMax = 30;
+constexpr int kWinMax = 60;
 int stream_windows(ckks_ctx *ctx, const std::vector<ckks_ctx::Window> **out);
 int launch_conv_fold_window(ckks_ctx *ctx, const u64 *y, u64 *buf, int batch, int w, cudaStream_t s);
 int launch_conv_fold_down(ckks_ctx *ctx, const u64 *zsrc, u64 *cv, int jobs2, cudaStream_t s);

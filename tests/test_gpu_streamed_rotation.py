@@ -1,4 +1,4 @@
-"""The streamed rotation (ModUp -> NTT -> key inner product over windows of at most 30 primes, no
+"""The streamed rotation (ModUp -> NTT -> key inner product over windows of at most 60 primes, no
 [B][dnum][L+K][n] digit tensor) against the oracle's hoisted rotation and, word for word, against
 the library's own hoisted rotation (which keeps the whole digit tensor)."""
 import numpy as np
@@ -30,9 +30,9 @@ def _res(shape, mods, stream):
 
 
 # (4, 1, 1): one-prime digits and windows; (20, 3, 7): a ragged last digit (7 + 7 + 6);
-# (112, 8, 8): the layer chain; (70, 33, 33): windows of 17 and 16 primes, a 4-prime last digit;
-# (130, 64, 64): 64-source conversions, windows of 22 and 21 primes; (120, 30, 30): windows of
-# exactly 30 primes, one per digit and one for the special primes.
+# (112, 8, 8): the layer chain; (70, 33, 33): 33-prime windows (two blocks of targets), a 4-prime
+# last digit; (130, 64, 64): 64-source conversions, two 32-prime windows per digit; (120, 30, 30):
+# one 30-prime window per digit and one for the special primes.
 @pytest.mark.parametrize("L,K,alpha", [(4, 1, 1), (20, 3, 7), (112, 8, 8), (70, 33, 33), (130, 64, 64),
                                        (120, 30, 30)])
 def test_streamed_rotation_matches_oracle(orc, L, K, alpha):
@@ -54,7 +54,7 @@ def test_streamed_rotation_matches_oracle(orc, L, K, alpha):
 def test_streamed_rotation_boot_size_equals_hoisted():
     """2100 + 60 primes, alpha = 60, 8 ciphertexts x 4 Galois keys (config 5): every word equals
     the hoisted rotation's, which its own test checks against the oracle; the streamed call's
-    workspace lacks the 9.9 GB digit tensor and holds two 138 MB windows of it instead."""
+    workspace lacks the 9.9 GB digit tensor and holds two 275 MB windows of it instead."""
     ctx = context(2100, 60, 60)
     mods = np.array(ctx.mods, dtype=np.uint64)
     gal = [galois_for_rotation(k) for k in (1, 2, 4, 8)]
@@ -68,7 +68,7 @@ def test_streamed_rotation_boot_size_equals_hoisted():
     # the hoisted call holds the digit tensor (and ModUp's sources inside ModDown's larger scratch);
     # the streamed one holds ModUp's sources and two windows of digits (one per stream) instead
     limb = N * 8
-    digits, sources, window = 8 * 35 * 2160 * limb, 8 * 2100 * limb, 8 * 35 * 30 * limb
+    digits, sources, window = 8 * 35 * 2160 * limb, 8 * 2100 * limb, 8 * 35 * 60 * limb
     ws_h = ctx.workspace_bytes(OP_ROTATE, 8, 4)
     ws_s = ctx.workspace_bytes(OP_ROTATE_STREAMED, 8, 4)
     assert ws_h - ws_s == digits - sources - 2 * window, (ws_h, ws_s)
