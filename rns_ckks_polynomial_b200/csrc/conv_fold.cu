@@ -148,6 +148,12 @@ __device__ __forceinline__ void fcp8(void *dst, const void *src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+// The same for 16 bytes, through L2 only (a table block is read once per CTA).
+__device__ __forceinline__ void fcp16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ void fcp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void fcp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
@@ -323,10 +329,43 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         fbar_init(bar + kFBarDrain, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    // Epilogue / staging threads: thread (quad, part) owns coefficient m = 32 quad + lane of a tile
+    // and sources s0 .. s0 + 15.  Each copies its 16 words of a tile into its own shared-memory
+    // slots one tile ahead, so the words are waiting when the tensor-memory buffer frees up, and no
+    // register or other thread is involved while they travel.
+    const int quad = warp & 3, part = warp >> 2;
+    const int m = quad * 32 + lane, s0 = part * 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    u64 *slot = reinterpret_cast<u64 *>(sm + kFSmemY) + tid;  // word k at slot[k * 512]
+    const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + m;
+    const bool full16 = s0 + 16 <= S;  // warp-uniform: all 16 of this thread's sources exist
+    auto issue = [&](int t) {
+        const u64 *src = ysrc + t * kFM;
+        if (full16) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) fcp8(slot + k * kFEpiThreads, src + (size_t)k * kN);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (s0 + k < S) fcp8(slot + k * kFEpiThreads, src + (size_t)k * kN);
+        }
+        fcp_commit();
+    };
     if (warp < kFEpiWarps) {
+        // tile 0's words and the table block travel together: only the K' chunks the products read,
+        // 2 nks chunks of 16 bytes in each 8-row group of each plane (the table is zero past 8 S, so
+        // the last K-step's padding comes in as zeros)
+        issue(0);
         const uint4 *src = reinterpret_cast<const uint4 *>(fbase + (size_t)tb * kFBlock);
         uint4 *dst = reinterpret_cast<uint4 *>(sm);
-        for (int i = tid; i < kFBlock / 16; i += kFEpiThreads) dst[i] = __ldg(src + i);
+        const int nkc = 2 * nks, per_group = 8 * nkc;  // 16-byte words per 8-row group
+        for (int i = tid; i < kFPlanes * (kFN / 8) * per_group; i += kFEpiThreads) {
+            const int ug = i / per_group, w = i - ug * per_group;
+            const int off = ug * (kFSbo / 16) + w;  // chunk w / 8, word w % 8 of group ug
+            fcp16(dst + off, src + off);
+        }
+        fcp_commit();
+        fcp_wait_all();
         if (tid < kFN) {
             const int ti = tb * kFN + tid;
             const PrimeConst &p = pc[ti < T ? jobs.prime(ti, lo, S) : 0];
@@ -371,27 +410,6 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
         ok = fbar_wait(bar + kFBarDrain, 0) && ok;
     } else {
         // ------------------------------------------------ epilogue and staging
-        const int quad = warp & 3, part = warp >> 2;
-        const int m = quad * 32 + lane, s0 = part * 16;
-        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        // Each thread copies its 16 words of a tile (coefficient m, sources s0 .. s0 + 15) into its
-        // own shared-memory slots one tile ahead, so the words are waiting when the tensor-memory
-        // buffer frees up, and no register or other thread is involved while they travel.
-        u64 *slot = reinterpret_cast<u64 *>(sm + kFSmemY) + tid;  // word k at slot[k * 512]
-        const u64 *ysrc = ybase + (size_t)s0 * kN + cbase + m;
-        const bool full16 = s0 + 16 <= S;  // warp-uniform: all 16 of this thread's sources exist
-        auto issue = [&](int t) {
-            const u64 *src = ysrc + t * kFM;
-            if (full16) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) fcp8(slot + k * kFEpiThreads, src + (size_t)k * kN);
-            } else {
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    if (s0 + k < S) fcp8(slot + k * kFEpiThreads, src + (size_t)k * kN);
-            }
-            fcp_commit();
-        };
         // tile t's words: own slots -> tensor-memory buffer t & 1 (the caller knows it is free); the
         // copies of tile t + 1 then start into the same slots
         auto stage = [&](int t) -> bool {
@@ -411,8 +429,7 @@ __global__ void __launch_bounds__(kFThreads, 1) conv_fold_kernel(FoldJobs jobs, 
             if (t + 1 < ntiles) issue(t + 1);
             return true;
         };
-        issue(0);
-        ok = stage(0);
+        ok = stage(0);  // tile 0's copies were issued with the table block
         if (ok && ntiles > 1) ok = stage(1);
         // the eight targets of this thread, tb * 32 + part * 8 + c: element offset of its output word
         // in tile 0 from the job's first output row (-1 for a target past the end)
