@@ -95,3 +95,55 @@ def test_streamed_rotation_errors():
     with pytest.raises(CkksError) as e:
         ctx.rotate_streamed(ct, [key], [4])
     assert e.value.code == -1
+
+
+def test_streamed_rotation_in_a_cuda_graph():
+    """Captured into a CUDA graph the call keeps every window on the capturing stream (one lane,
+    one window buffer); replays give the hoisted rotation's words."""
+    L, K, alpha = 20, 3, 7
+    ctx = context(L, K, alpha)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    dnum = (L + alpha - 1) // alpha
+    ct = dev(_res((2, 2, L, N), mods[:L], 300))
+    keys = [dev(_res((dnum, 2, L + K, N), mods, 301 + r)) for r in range(3)]
+    gal = [5, 25, 4095]
+    want = ctx.rotate(ct, keys, gal)
+    out = torch.empty_like(want)
+    ws = torch.empty(ctx.workspace_bytes(OP_ROTATE_STREAMED, 2, 3), dtype=torch.uint8, device="cuda")
+    ctx.rotate_streamed(ct, keys, gal, out=out, ws=ws)  # tables built outside the capture
+    torch.cuda.synchronize()
+    out.zero_()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            ctx.rotate_streamed(ct, keys, gal, out=out, ws=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, want)
+    ctx.device_status()
+    del g
+
+
+def test_streamed_rotation_more_than_64_keys(orc):
+    """66 keys: the call works through them in chunks of 64, each repeating the windows' work;
+    every output equals the hoisted rotation's, and two of them the oracle's."""
+    L, K, alpha = 4, 1, 1
+    ctx = context(L, K, alpha)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    ct_h = _res((1, 2, L, N), mods[:L], 400)
+    keys_h = [_res((L, 2, L + K, N), mods, 401 + r) for r in range(66)]
+    gal = [galois_for_rotation(r + 1) for r in range(66)]
+    ct = dev(ct_h)
+    keys = [dev(k) for k in keys_h]
+    out = ctx.rotate_streamed(ct, keys, gal)
+    ctx.device_status()
+    assert torch.equal(out, ctx.rotate(ct, keys, gal))
+    pick = [0, 65]
+    want = orc.rotate(ct_h, [keys_h[r] for r in pick], np.array([gal[r] for r in pick], dtype=np.uint64),
+                      mods, L, K, alpha)
+    assert_bits_equal(host(out[pick]), want, "keys 0 and 65")
