@@ -338,8 +338,8 @@ int ckks_rotate_unhoisted(const ckks_ctx *ctx, const uint64_t *ct, const uint64_
  * stream (one stream while the caller's is being captured into a graph).
  * ModDown then runs as in ckks_rotate.  The first call builds the windows'
  * conversion tables (two 128 KiB blocks of 32 targets per window and digit).
- * Arguments, layouts and errors as ckks_rotate, plus CKKS_EUNSUPPORTED when
- * alpha or K exceeds 64.  Each chunk of 64 keys repeats the windows' work.
+ * Arguments, layouts and errors as ckks_rotate.  Each chunk of 64 keys
+ * repeats the windows' work.
  * ws: ckks_workspace_bytes(CKKS_OP_ROTATE_STREAMED, batch, nkeys). */
 int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
                          const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,

@@ -595,11 +595,14 @@ size_t rotate_ws(const ckks_ctx *ctx, int batch, int nkeys)
            std::max(modup_ws_bytes(ctx, batch), moddown_ws_bytes(ctx, chunk * batch));
 }
 
-// ModUp's sources y, two window buffers, the accumulators of a key chunk and ModDown's scratch.
+constexpr int kLanes = 2;  // streams the windows of a streamed rotation alternate between
+
+// ModUp's sources y, one window buffer per lane, the accumulators of a key chunk and ModDown's
+// scratch.
 size_t rotate_streamed_ws(const ckks_ctx *ctx, int batch, int nkeys)
 {
     const int chunk = std::min(std::max(nkeys, 1), kMaxKeys);
-    return limbs_bytes((size_t)batch * ctx->L) + 2 * limbs_bytes((size_t)batch * ctx->dnum * kWinMax) +
+    return limbs_bytes((size_t)batch * ctx->L) + kLanes * limbs_bytes((size_t)batch * ctx->dnum * kWinMax) +
            limbs_bytes((size_t)chunk * batch * 2 * (ctx->L + ctx->K)) + moddown_ws_bytes(ctx, chunk * batch);
 }
 
@@ -741,9 +744,9 @@ extern "C" int ckks_rotate(const ckks_ctx *ctx, const uint64_t *ct, const uint64
 // kWinMax primes: per window, the folded conversion writes every digit's limbs at the window's
 // primes into a window buffer (the window's own digit gets the input's limbs), the forward NTT runs
 // over it and the key inner product consumes it, so the extended digits never exist as a whole.
-// Consecutive windows alternate between the caller's stream and a second stream, each with its own
-// buffer (they write disjoint accumulator rows and only read y), so one window's launches fill the
-// other's partial waves.  ModDown then runs as in ckks_rotate.
+// Consecutive windows go round kLanes streams (the caller's and kLanes - 1 of its own), each with
+// its own buffer (they write disjoint accumulator rows and only read y), so one window's launches
+// fill the others' partial waves.  ModDown then runs as in ckks_rotate.
 extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, const uint64_t *const *keys,
                                     const uint32_t *galois, int nkeys, uint64_t *out, int batch, void *ws,
                                     ckks_stream_t stream)
@@ -758,7 +761,6 @@ extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, con
         if ((galois[r] & 1u) == 0) return set_error(CKKS_EINVAL, "galois element must be odd");
     }
     if ((size_t)nkeys * batch > 32767) return set_error(CKKS_EUNSUPPORTED, "nkeys * batch above 32767");
-    if (ctx->alpha > 64 || ctx->K > 64) return set_error(CKKS_EUNSUPPORTED, "more than 64 sources per conversion");
     CKKS_TRY(check_ptr(ct, "ct"));
     CKKS_TRY(check_ptr(out, "out"));
     CKKS_TRY(set_device(ctx));
@@ -774,34 +776,34 @@ extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, con
     const int chunk = std::min(nkeys, kMaxKeys);
     Carve c(w);
     u64 *y = c.take<u64>((size_t)batch * L * kN);
-    u64 *bufs[2];
+    u64 *bufs[kLanes];
     for (u64 *&bp : bufs) bp = c.take<u64>((size_t)batch * dnum * kWinMax * kN);
     u64 *acc = c.take<u64>((size_t)chunk * batch * 2 * LK * kN);
     void *scratch = c.base + c.off;
-    // the second stream and the fork / join events live for this call only
-    cudaStream_t s2 = nullptr;
-    cudaEvent_t ev[2] = {nullptr, nullptr};
+    // the other lanes' streams and the fork / join events live for this call only
+    cudaStream_t lane[kLanes] = {};
+    cudaEvent_t ev[kLanes] = {};  // ev[0]: fork; ev[l]: lane l done
     struct Release {
-        cudaStream_t &st;
+        cudaStream_t *st;
         cudaEvent_t *e;
         ~Release()
         {
-            if (st) cudaStreamDestroy(st);
-            for (int i = 0; i < 2; ++i)
+            for (int i = 1; i < kLanes; ++i)
+                if (st[i]) cudaStreamDestroy(st[i]);
+            for (int i = 0; i < kLanes; ++i)
                 if (e[i]) cudaEventDestroy(e[i]);
         }
-    } release{s2, ev};
+    } release{lane, ev};
     // a stream being captured into a graph keeps every window on itself (one lane)
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     cudaError_t ce = cudaStreamIsCapturing(s, &cap);
-    const bool two = ce == cudaSuccess && cap == cudaStreamCaptureStatusNone;
+    const bool multi = ce == cudaSuccess && cap == cudaStreamCaptureStatusNone;
     if (ce != cudaSuccess) return cuda_status(ce, "cudaStreamIsCapturing");
-    if (two) {
-        ce = cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking);
-        for (int i = 0; i < 2 && ce == cudaSuccess; ++i) ce = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
-        if (ce != cudaSuccess) return cuda_status(ce, "stream/event for the streamed rotation");
-    }
-    const cudaStream_t lane[2] = {s, two ? s2 : s};
+    const int nl = multi ? kLanes : 1;
+    lane[0] = s;
+    for (int i = 1; i < nl && ce == cudaSuccess; ++i) ce = cudaStreamCreateWithFlags(&lane[i], cudaStreamNonBlocking);
+    for (int i = 0; i < nl && ce == cudaSuccess; ++i) ce = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+    if (ce != cudaSuccess) return cuda_status(ce, "stream/event for the streamed rotation");
     // ModUp's sources: y = INTT(c1) times [(Q_j/q_i)^-1]
     const u64 *c1 = ct + (size_t)L * kN;
     UpInttJob<false> ij{c1, nullptr, ct_elems, nullptr, y, T.up_hatinv, T.pc, L, LK, T.alpha, dnum, batch,
@@ -822,15 +824,15 @@ extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, con
         }
         // fork: the second lane starts once y (and, from the second key chunk on, the previous
         // ModDown's reads of acc) are done on the caller's stream
-        if (two) {
+        if (nl > 1) {
             ce = cudaEventRecord(ev[0], s);
-            if (ce == cudaSuccess) ce = cudaStreamWaitEvent(s2, ev[0], 0);
+            for (int i = 1; i < nl && ce == cudaSuccess; ++i) ce = cudaStreamWaitEvent(lane[i], ev[0], 0);
             if (ce != cudaSuccess) return cuda_status(ce, "fork of the streamed rotation");
         }
         for (int wi = 0; wi < (int)wins->size(); ++wi) {
             const ckks_ctx::Window wd = (*wins)[wi];
-            const cudaStream_t ls = lane[wi & 1];
-            u64 *buf = bufs[two ? wi & 1 : 0];
+            const cudaStream_t ls = lane[wi % nl];
+            u64 *buf = bufs[wi % nl];
             CKKS_TRY(launch_conv_fold_window(mctx, y, buf, batch, wi, ls));
             if (wd.own >= 0) {
                 cudaError_t e = cudaMemcpy2DAsync(buf + (size_t)wd.own * kWinMax * kN,
@@ -846,11 +848,11 @@ extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, con
             CKKS_TRY(key_inner_stage(ctx, buf, kl, batch, true, acc, nk * batch, ls, dv));
         }
         // join: ModDown reads every window's accumulator rows
-        if (two) {
-            ce = cudaEventRecord(ev[1], s2);
-            if (ce == cudaSuccess) ce = cudaStreamWaitEvent(s, ev[1], 0);
-            if (ce != cudaSuccess) return cuda_status(ce, "join of the streamed rotation");
+        for (int i = 1; i < nl && ce == cudaSuccess; ++i) {
+            ce = cudaEventRecord(ev[i], lane[i]);
+            if (ce == cudaSuccess) ce = cudaStreamWaitEvent(s, ev[i], 0);
         }
+        if (ce != cudaSuccess) return cuda_status(ce, "join of the streamed rotation");
         CKKS_TRY(moddown_stage(ctx, acc, out + (size_t)r0 * batch * ct_elems, nk * batch, ex, scratch, s));
     }
     return CKKS_OK;
