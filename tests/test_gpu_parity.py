@@ -403,10 +403,9 @@ def test_config4_dense_matrix_decrypts(orc):
 def test_config5_boot_rotation_full_size(orc):
     """2100 primes, alpha = 60, 60 special primes, 4 Galois keys (5^k,
     k in {1, 2, 4, 8}), 8 ciphertexts: the GPU runs all 32 key switches with
-    one hoisted ModUp per ciphertext.  The oracle recomputes ciphertexts 1
-    and 6 (one in each chunk of 4 that the key inner product groups) under
-    all four keys, 8 of the 32 key switches; the integer-pipe conversion
-    then gives the same words for all 32."""
+    one hoisted ModUp per ciphertext.  The oracle recomputes every one of the
+    32 key switches (two ciphertexts at a time, which bounds its memory); the
+    integer-pipe conversion then gives the same words for all 32."""
     p = Params(2100, 60, 60)
     ctx = ctx_for(p)
     seed = synth.config_seed(5)
@@ -418,11 +417,12 @@ def test_config5_boot_rotation_full_size(orc):
             for r in range(4)]
     out = ctx.rotate(ct, keys, gal)
     ctx.device_status()
-    pick = [1, 6]
-    want = orc.rotate(host(ct[pick]), [host(k) for k in keys], np.array(gal, dtype=np.uint64), mods,
-                      2100, 60, 60)
-    assert_bits_equal(host(out[:, pick]), want, "config 5, ciphertexts 1 and 6, all keys")
-    del want
+    keys_h = [host(k) for k in keys]
+    for pick in ([0, 1], [2, 3], [4, 5], [6, 7]):
+        want = orc.rotate(host(ct[pick]), keys_h, np.array(gal, dtype=np.uint64), mods, 2100, 60, 60)
+        assert_bits_equal(host(out[:, pick]), want, "config 5, ciphertexts %s, all keys" % pick)
+        del want
+    del keys_h
     try:
         for engine in ("integer",):
             ctx.set_conversion(engine)
