@@ -279,7 +279,8 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 // One thread per output coefficient k of one (prime t, key r) pair and a chunk of up to kKiB
 // ciphertexts b: per digit j it loads the two key words once and the chunk's gathered digit words,
 // and keeps 2 kKiB exact sums (three 64-bit partial sums each in the split form below, taken when
-// every prime is 2^60 - delta; 128-bit sums otherwise).  The 1-D grid is ordered coefficient tile fastest, then key,
+// every prime is 2^60 - delta, whose words arrive by cp.async kKiDepth digits ahead; 128-bit sums
+// otherwise).  The 1-D grid is ordered coefficient tile fastest, then key,
 // then ciphertext chunk, then prime, so the CTAs that read the same digit rows (all keys of one
 // chunk at one prime) run back to back and re-read them from L2.  The Galois permutation is the
 // gather on the digit load (it maps each aligned tile of 32 coefficients onto one, so a warp's
@@ -288,6 +289,18 @@ constexpr int kKiB = 4;       // ciphertexts per thread
 constexpr int kKiThreads = 128;
 constexpr int kKiFold = 256;  // digits summed exactly in 128 bits between reductions
 constexpr int kKiMinBlocks = 4;
+// Split form: each thread copies its 2 + kKiB words of a digit (cp.async, 8 bytes each) into its
+// own shared-memory slots kKiDepth digits ahead, so the loads in flight hold no registers
+constexpr int kKiDepth = 8;
+constexpr int kKiSlots = 2 + kKiB;
+constexpr size_t kKiSmem = (size_t)kKiDepth * kKiSlots * kKiThreads * sizeof(u64);  // 48 KiB
+
+// Asynchronous 8-byte copy from global into this thread's shared-memory slot.
+__device__ __forceinline__ void kcp8(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" :: "r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
 
 template <bool kSplit>
 __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
@@ -320,22 +333,44 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
 #pragma unroll
             for (int b = 0; b < kKiB; ++b) s0[c][b] = s1[c][b] = s2[c][b] = 0;
         const u32 delta = (u32)pc.delta;
+        // this thread's slots: word w of digit j at slot[((j % kKiDepth) kKiSlots + w) kKiThreads];
+        // words 0, 1: the key's two components, 2 + b: ciphertext b's digit word (zero past nb)
+        extern __shared__ u64 kism[];
+        u64 *const slot = kism + threadIdx.x;
+        for (int st = 0; st < kKiDepth; ++st)
+            for (int b = nb; b < kKiB; ++b) slot[(st * kKiSlots + 2 + b) * kKiThreads] = 0;
+        auto fetch = [&](int j) {  // one commit group per digit, empty past the last
+            if (j < T.dnum) {
+                u64 *sl = slot + (j % kKiDepth) * kKiSlots * kKiThreads;
+                kcp8(sl, kp + (size_t)(2 * j) * kLKn);
+                kcp8(sl + kKiThreads, kp + (size_t)(2 * j + 1) * kLKn);
+                const u64 *dj = dg + (size_t)j * dv.j_stride;
+#pragma unroll
+                for (int b = 0; b < kKiB; ++b)
+                    if (b < nb) kcp8(sl + (2 + b) * kKiThreads, dj + (size_t)b * bstride);
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+#pragma unroll
+        for (int j = 0; j < kKiDepth; ++j) fetch(j);
         for (int j0 = 0; j0 < T.dnum; j0 += kSplitFold) {
             const int j1 = min(T.dnum, j0 + kSplitFold);
-#pragma unroll 4
+#pragma unroll 2
             for (int j = j0; j < j1; ++j) {
-                const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
+                asm volatile("cp.async.wait_group %0;" :: "n"(kKiDepth - 1) : "memory");  // digit j is in
+                const u64 *sl = slot + (j % kKiDepth) * kKiSlots * kKiThreads;
+                const u64 kb = sl[0], ka = sl[kKiThreads];
                 const u32 k0[2] = {lo30(kb), lo30(ka)}, k1[2] = {hi30(kb), hi30(ka)};
-                const u64 *dj = dg + (size_t)j * dv.j_stride;
                 u64 d[kKiB];
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
+                for (int b = 0; b < kKiB; ++b) d[b] = sl[(2 + b) * kKiThreads];
 #pragma unroll
                 for (int b = 0; b < kKiB; ++b) {
                     const u32 d0 = lo30(d[b]), d1 = hi30(d[b]);
 #pragma unroll
                     for (int c = 0; c < 2; ++c) split_mac(s0[c][b], s1[c][b], s2[c][b], d0, d1, k0[c], k1[c]);
                 }
+                fetch(j + kKiDepth);  // into the slots just read: their values are consumed
             }
 #pragma unroll
             for (int c = 0; c < 2; ++c)
@@ -400,8 +435,8 @@ int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, i
     const size_t blocks = (size_t)(kN / kKiThreads) * nkeys * ((per_key + kKiB - 1) / kKiB) * dv.nt;
     if (blocks > 0x7fffffffull) return set_error(CKKS_EUNSUPPORTED, "key inner product grid too large");
     if (T.special)
-        key_inner_kernel<true><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0,
-                                                                       acc, T, dv);
+        key_inner_kernel<true><<<(unsigned)blocks, kKiThreads, kKiSmem, s>>>(digits, kl, per_key, nkeys,
+                                                                             hoisted ? 1 : 0, acc, T, dv);
     else
         key_inner_kernel<false><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0,
                                                                         acc, T, dv);
