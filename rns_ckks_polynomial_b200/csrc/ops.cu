@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(256) bsgs_inner_kernel(const u64 *__restrict__
         u64 hi[kBC], lo[kBC];
 #pragma unroll
         for (int q = 0; q < kBC; ++q) hi[q] = lo[q] = 0;
+#pragma unroll 8  // eight diagonal words in flight per thread
         for (int r = 0; r < bb; ++r) {
             const u64 dv = __ldg(d + (size_t)r * Ln);
 #pragma unroll
