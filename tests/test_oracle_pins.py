@@ -519,7 +519,7 @@ def test_bsgs_banded_matvec(orc):
 
 def test_bsgs_at_the_layer_chain_size(orc):
     """Config 4's shape: 112 + 8 primes, bb = gg = 32, 31 baby and 31 giant
-    keys (about 30 s).  M has nonzero diagonals at offsets spread over the
+    keys.  M has nonzero diagonals at offsets spread over the
     32 x 32 (giant, baby) grid, including both ends and both sides of a giant
     boundary; absent diagonals are zero plaintexts.  Decrypts (through
     q_0..q_2) to M x."""
