@@ -16,7 +16,8 @@
 // One CTA (one per SM, owning all 512 TMEM columns) converts one block of 32 targets (the MMA's N)
 // for a run of coefficient tiles of 128 (the MMA's M, the TMEM lanes):
 //  - the block's eight F planes (8 x 32 targets x 512 bytes = 128 KiB) stay in shared memory (the B
-//    operand, K-major core matrices) for the whole run;
+//    operand, K-major core matrices) for the whole run; the CTA copies only the K' chunks its
+//    products read (16-byte cp.async, issued together with tile 0's data words);
 //  - each staging thread copies its 16 words of the next data tile (cp.async, 8 bytes each) into
 //    its own shared-memory slots one tile ahead, and moves them (one coefficient per TMEM lane) into
 //    the A operand in tensor memory when a buffer frees up: double-buffered, columns 256..383 and
@@ -32,9 +33,13 @@
 //    release it (the next tile's products into it can start) and fold it to the low 50 bits of each
 //    sum; read and release group 1 as soon as it completes, rebuild each (< 2^83) sum, reduce it
 //    once and store it while the tensor cores run the next tile; then stage tile i + 2 from shared
-//    memory into the data buffer tile i used (every product of tile i is complete by then).  Warp w reads TMEM lane quadrant w & 3 (coefficients
-//    32 (w & 3) ..) and columns 8 (w >> 2) .. 8 (w >> 2) + 7 of each plane: eight targets of one
-//    coefficient; for staging it owns sources 16 (w >> 2) .. + 15.
+//    memory into the data buffer tile i used (every product of tile i is complete by then).
+//    Warp w reads TMEM lane quadrant w & 3 (coefficients 32 (w & 3) ..) and columns 8 (w >> 2) ..
+//    8 (w >> 2) + 7 of each plane: eight targets of one coefficient; for staging it owns sources
+//    16 (w >> 2) .. + 15.
+// Three job geometries: ModUp (a digit into its L + K - S other primes), ModDown (the special
+// primes into the ciphertext primes) and a window of ModUp (a digit into the primes of one window
+// of the streamed rotation, its own table layout).
 // Per output the epilogue spends 8 tensor-memory words, two folds and one reduction: for primes
 // 2^60 - delta (delta < 2^28) a funnel shift and one 32 x 32 multiply-add leave the value in
 // [0, 2q), which the forward NTT that consumes every converted limb accepts (it takes inputs below
