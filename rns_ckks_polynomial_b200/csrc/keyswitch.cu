@@ -815,7 +815,9 @@ extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, con
     for (u64 *&bp : bufs) bp = c.take<u64>((size_t)batch * dnum * kWinMax * kN);
     u64 *acc = c.take<u64>((size_t)chunk * batch * 2 * LK * kN);
     void *scratch = c.base + c.off;
-    // the other lanes' streams and the fork / join events live for this call only
+    // the other lanes' streams and the fork / join events live for this call only; on every way
+    // out (an error after the fork included) the caller's stream first waits for every lane, so no
+    // window work outlives the call's view of the workspace
     cudaStream_t lane[kLanes] = {};
     cudaEvent_t ev[kLanes] = {};  // ev[0]: fork; ev[l]: lane l done
     struct Release {
@@ -823,8 +825,11 @@ extern "C" int ckks_rotate_streamed(const ckks_ctx *ctx, const uint64_t *ct, con
         cudaEvent_t *e;
         ~Release()
         {
-            for (int i = 1; i < kLanes; ++i)
-                if (st[i]) cudaStreamDestroy(st[i]);
+            for (int i = 1; i < kLanes; ++i) {
+                if (!st[i]) continue;
+                if (e[i] && cudaEventRecord(e[i], st[i]) == cudaSuccess) cudaStreamWaitEvent(st[0], e[i], 0);
+                cudaStreamDestroy(st[i]);
+            }
             for (int i = 0; i < kLanes; ++i)
                 if (e[i]) cudaEventDestroy(e[i]);
         }
