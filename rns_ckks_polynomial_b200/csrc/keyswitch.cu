@@ -360,15 +360,15 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
                 asm volatile("cp.async.wait_group %0;" :: "n"(kKiDepth - 1) : "memory");  // digit j is in
                 const u64 *sl = slot + (j % kKiDepth) * kKiSlots * kKiThreads;
                 const u64 kb = sl[0], ka = sl[kKiThreads];
-                const u32 k0[2] = {lo30(kb), lo30(ka)}, k1[2] = {hi30(kb), hi30(ka)};
+                const Split30 kw[2] = {split30(kb), split30(ka)};
                 u64 d[kKiB];
 #pragma unroll
                 for (int b = 0; b < kKiB; ++b) d[b] = sl[(2 + b) * kKiThreads];
 #pragma unroll
                 for (int b = 0; b < kKiB; ++b) {
-                    const u32 d0 = lo30(d[b]), d1 = hi30(d[b]);
+                    const Split30 dw = split30(d[b]);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) split_mac(s0[c][b], s1[c][b], s2[c][b], d0, d1, k0[c], k1[c]);
+                    for (int c = 0; c < 2; ++c) split_mac(s0[c][b], s1[c][b], s2[c][b], dw, kw[c]);
                 }
                 fetch(j + kKiDepth);  // into the slots just read: their values are consumed
             }
