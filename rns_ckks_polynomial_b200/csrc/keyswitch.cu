@@ -276,24 +276,26 @@ int modup_stage(const ckks_ctx *ctx, const u64 *in, const u64 *in2, size_t in_bs
 }
 
 // ---------------------------------------------------------------- key inner product
-// One thread per output coefficient k of one (prime t, key r) pair and a chunk of up to kKiB
+// One thread per output coefficient k of one (prime t, key r) pair and a chunk of up to kB
 // ciphertexts b: per digit j it loads the two key words once and the chunk's gathered digit words,
-// and keeps 2 kKiB exact sums (three 64-bit partial sums each in the split form below, taken when
-// every prime is 2^60 - delta, whose words arrive by cp.async kKiDepth digits ahead; 128-bit sums
-// otherwise).  The 1-D grid is ordered coefficient tile fastest, then key,
+// and keeps 2 kB exact sums (three 64-bit partial sums each in the split form below, taken when
+// every prime is 2^60 - delta, whose words arrive by cp.async ki_depth(kB) digits ahead; 128-bit
+// sums otherwise).  The 1-D grid is ordered coefficient tile fastest, then key,
 // then ciphertext chunk, then prime, so the CTAs that read the same digit rows (all keys of one
 // chunk at one prime) run back to back and re-read them from L2.  The Galois permutation is the
 // gather on the digit load (it maps each aligned tile of 32 coefficients onto one, so a warp's
 // gathered loads stay within one 256-byte segment).
-constexpr int kKiB = 4;       // ciphertexts per thread
+constexpr int kKiB = 4;       // ciphertexts per thread: the 128-bit form, and batches below kKiBWide
+constexpr int kKiBWide = 8;   // ciphertexts per thread in the split form from 8 ciphertexts per key
 constexpr int kKiThreads = 128;
 constexpr int kKiFold = 256;  // digits summed exactly in 128 bits between reductions
-constexpr int kKiMinBlocks = 4;
-// Split form: each thread copies its 2 + kKiB words of a digit (cp.async, 8 bytes each) into its
-// own shared-memory slots kKiDepth digits ahead, so the loads in flight hold no registers
-constexpr int kKiDepth = 8;
-constexpr int kKiSlots = 2 + kKiB;
-constexpr size_t kKiSmem = (size_t)kKiDepth * kKiSlots * kKiThreads * sizeof(u64);  // 48 KiB
+// Split form: each thread copies its 2 + kB words of a digit (cp.async, 8 bytes each) into its
+// own shared-memory slots ki_depth(kB) digits ahead, so the loads in flight hold no registers.
+// Chunks of 4: 8 digits ahead, 48 KiB and 4 CTAs per SM; chunks of 8 (the key's two words split
+// once for 8 ciphertexts, more registers): 4 digits ahead, 40 KiB and 3 CTAs per SM.
+__host__ __device__ constexpr int ki_depth(int b) { return b == kKiBWide ? 4 : 8; }
+__host__ __device__ constexpr int ki_min_blocks(int b) { return b == kKiBWide ? 3 : 4; }
+constexpr size_t ki_smem(int b) { return (size_t)ki_depth(b) * (2 + b) * kKiThreads * sizeof(u64); }
 
 // Asynchronous 8-byte copy from global into this thread's shared-memory slot.
 __device__ __forceinline__ void kcp8(void *dst, const void *src)
@@ -302,12 +304,13 @@ __device__ __forceinline__ void kcp8(void *dst, const void *src)
                  : "memory");
 }
 
-template <bool kSplit>
-__global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
+template <bool kSplit, int kB>
+__global__ void __launch_bounds__(kKiThreads, ki_min_blocks(kB)) key_inner_kernel(const u64 *__restrict__ digits, KeyList kl,
                                                         int per_key, int nkeys, int hoisted,
                                                         u64 *__restrict__ acc, Tables T, DigitView dv)
 {
-    const int nchunks = (per_key + kKiB - 1) / kKiB;
+    constexpr int kDepth = ki_depth(kB), kSlots = 2 + kB;
+    const int nchunks = (per_key + kB - 1) / kB;
     int id = blockIdx.x;
     const int tile = id % (kN / kKiThreads);
     id /= kN / kKiThreads;
@@ -315,7 +318,7 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
     id /= nkeys;
     const int chunk = id % nchunks;
     const int t = dv.t_lo + id / nchunks;
-    const int b0 = chunk * kKiB, nb = min(kKiB, per_key - b0);
+    const int b0 = chunk * kB, nb = min(kB, per_key - b0);
     const int k = tile * kKiThreads + threadIdx.x;
     const u32 g = kl.galois[r];
     const int src = g == 1u ? k : (int)galois_src((u32)k, g);
@@ -327,58 +330,58 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
     const u64 *kp = kl.key[r] + (size_t)kt * kN + k;
     const PrimeConst pc = T.pc[t];
     if constexpr (kSplit) {
-        u64 s0[2][kKiB], s1[2][kKiB], s2[2][kKiB];
+        u64 s0[2][kB], s1[2][kB], s2[2][kB];
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int b = 0; b < kKiB; ++b) s0[c][b] = s1[c][b] = s2[c][b] = 0;
+            for (int b = 0; b < kB; ++b) s0[c][b] = s1[c][b] = s2[c][b] = 0;
         const u32 delta = (u32)pc.delta;
-        // this thread's slots: word w of digit j at slot[((j % kKiDepth) kKiSlots + w) kKiThreads];
+        // this thread's slots: word w of digit j at slot[((j % kDepth) kSlots + w) kKiThreads];
         // words 0, 1: the key's two components, 2 + b: ciphertext b's digit word (zero past nb)
         extern __shared__ u64 kism[];
         u64 *const slot = kism + threadIdx.x;
-        for (int st = 0; st < kKiDepth; ++st)
-            for (int b = nb; b < kKiB; ++b) slot[(st * kKiSlots + 2 + b) * kKiThreads] = 0;
+        for (int st = 0; st < kDepth; ++st)
+            for (int b = nb; b < kB; ++b) slot[(st * kSlots + 2 + b) * kKiThreads] = 0;
         auto fetch = [&](int j) {  // one commit group per digit, empty past the last
             if (j < T.dnum) {
-                u64 *sl = slot + (j % kKiDepth) * kKiSlots * kKiThreads;
+                u64 *sl = slot + (j % kDepth) * kSlots * kKiThreads;
                 kcp8(sl, kp + (size_t)(2 * j) * kLKn);
                 kcp8(sl + kKiThreads, kp + (size_t)(2 * j + 1) * kLKn);
                 const u64 *dj = dg + (size_t)j * dv.j_stride;
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b)
+                for (int b = 0; b < kB; ++b)
                     if (b < nb) kcp8(sl + (2 + b) * kKiThreads, dj + (size_t)b * bstride);
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
         };
 #pragma unroll
-        for (int j = 0; j < kKiDepth; ++j) fetch(j);
+        for (int j = 0; j < kDepth; ++j) fetch(j);
         for (int j0 = 0; j0 < T.dnum; j0 += kSplitFold) {
             const int j1 = min(T.dnum, j0 + kSplitFold);
 #pragma unroll 2
             for (int j = j0; j < j1; ++j) {
-                asm volatile("cp.async.wait_group %0;" :: "n"(kKiDepth - 1) : "memory");  // digit j is in
-                const u64 *sl = slot + (j % kKiDepth) * kKiSlots * kKiThreads;
+                asm volatile("cp.async.wait_group %0;" :: "n"(kDepth - 1) : "memory");  // digit j is in
+                const u64 *sl = slot + (j % kDepth) * kSlots * kKiThreads;
                 const u64 kb = sl[0], ka = sl[kKiThreads];
                 const Split30 kw[2] = {split30(kb), split30(ka)};
-                u64 d[kKiB];
+                u64 d[kB];
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) d[b] = sl[(2 + b) * kKiThreads];
+                for (int b = 0; b < kB; ++b) d[b] = sl[(2 + b) * kKiThreads];
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) {
+                for (int b = 0; b < kB; ++b) {
                     const Split30 dw = split30(d[b]);
 #pragma unroll
                     for (int c = 0; c < 2; ++c) split_mac(s0[c][b], s1[c][b], s2[c][b], dw, kw[c]);
                 }
-                fetch(j + kKiDepth);  // into the slots just read: their values are consumed
+                fetch(j + kDepth);  // into the slots just read: their values are consumed
             }
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) split_fold(s0[c][b], s1[c][b], s2[c][b], delta);
+                for (int b = 0; b < kB; ++b) split_fold(s0[c][b], s1[c][b], s2[c][b], delta);
         }
 #pragma unroll
-        for (int b = 0; b < kKiB; ++b) {
+        for (int b = 0; b < kB; ++b) {
             if (b < nb) {
                 u64 *o = acc + ((size_t)(r * per_key + b0 + b) * 2 * T.LK + t) * kN + k;
                 o[0] = split_reduce(s0[0][b], s2[0][b], pc);
@@ -386,15 +389,15 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
             }
         }
     } else {
-        u64 h0[kKiB], l0[kKiB], h1[kKiB], l1[kKiB];
+        u64 h0[kB], l0[kB], h1[kB], l1[kB];
 #pragma unroll
-        for (int b = 0; b < kKiB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
+        for (int b = 0; b < kB; ++b) h0[b] = l0[b] = h1[b] = l1[b] = 0;
         // 256 products below 2^120 plus a folded value below 2^60 stay below
         // 2^128: past 256 digits the sums are reduced once per block of 256
         for (int j0 = 0; j0 < T.dnum; j0 += kKiFold) {
             if (j0 > 0) {
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) {
+                for (int b = 0; b < kB; ++b) {
                     l0[b] = reduce128(h0[b], l0[b], pc);
                     l1[b] = reduce128(h1[b], l1[b], pc);
                     h0[b] = h1[b] = 0;
@@ -405,18 +408,18 @@ __global__ void __launch_bounds__(kKiThreads, kKiMinBlocks) key_inner_kernel(con
             for (int j = j0; j < j1; ++j) {
                 const u64 kb = __ldg(kp + (size_t)(2 * j) * kLKn), ka = __ldg(kp + (size_t)(2 * j + 1) * kLKn);
                 const u64 *dj = dg + (size_t)j * dv.j_stride;
-                u64 d[kKiB];
+                u64 d[kB];
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
+                for (int b = 0; b < kB; ++b) d[b] = b < nb ? __ldg(dj + (size_t)b * bstride) : 0;
 #pragma unroll
-                for (int b = 0; b < kKiB; ++b) {
+                for (int b = 0; b < kB; ++b) {
                     mac128(h0[b], l0[b], d[b], kb);
                     mac128(h1[b], l1[b], d[b], ka);
                 }
             }
         }
 #pragma unroll
-        for (int b = 0; b < kKiB; ++b) {
+        for (int b = 0; b < kB; ++b) {
             if (b < nb) {
                 u64 *o = acc + ((size_t)(r * per_key + b0 + b) * 2 * T.LK + t) * kN + k;
                 o[0] = reduce128(h0[b], l0[b], pc);
@@ -432,14 +435,19 @@ int key_inner_stage(const ckks_ctx *ctx, const u64 *digits, const KeyList &kl, i
     if (jobs <= 0 || dv.nt <= 0) return CKKS_OK;
     const Tables &T = ctx->t;
     const int nkeys = jobs / per_key;
-    const size_t blocks = (size_t)(kN / kKiThreads) * nkeys * ((per_key + kKiB - 1) / kKiB) * dv.nt;
+    const bool wide = T.special && per_key >= kKiBWide;
+    const int cb = wide ? kKiBWide : kKiB;
+    const size_t blocks = (size_t)(kN / kKiThreads) * nkeys * ((per_key + cb - 1) / cb) * dv.nt;
     if (blocks > 0x7fffffffull) return set_error(CKKS_EUNSUPPORTED, "key inner product grid too large");
-    if (T.special)
-        key_inner_kernel<true><<<(unsigned)blocks, kKiThreads, kKiSmem, s>>>(digits, kl, per_key, nkeys,
-                                                                             hoisted ? 1 : 0, acc, T, dv);
+    if (wide)
+        key_inner_kernel<true, kKiBWide><<<(unsigned)blocks, kKiThreads, ki_smem(kKiBWide), s>>>(
+            digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T, dv);
+    else if (T.special)
+        key_inner_kernel<true, kKiB><<<(unsigned)blocks, kKiThreads, ki_smem(kKiB), s>>>(
+            digits, kl, per_key, nkeys, hoisted ? 1 : 0, acc, T, dv);
     else
-        key_inner_kernel<false><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys, hoisted ? 1 : 0,
-                                                                        acc, T, dv);
+        key_inner_kernel<false, kKiB><<<(unsigned)blocks, kKiThreads, 0, s>>>(digits, kl, per_key, nkeys,
+                                                                              hoisted ? 1 : 0, acc, T, dv);
     CKKS_CHECK_LAUNCH("key_inner_kernel");
     return CKKS_OK;
 }

@@ -813,6 +813,41 @@ def test_key_inner_more_than_256_digits(orc, form):
     assert_bits_equal(acc, want, "key inner product over 260 digits")
 
 
+def test_key_inner_wide_chunks(orc):
+    """From 8 ciphertexts per key the split-form inner product gives each thread 8 ciphertexts
+    (4 digits of prefetch); below that, 4.  Ragged chunks (10 = 8 + 2 and 9 = 8 + 1 ciphertexts)
+    through the direct call, the hoisted rotation and the per-key digits of the unhoisted order,
+    bit-exact against the oracle; all-(q - 1) words over 40 one-prime digits against the closed
+    form 40 (q - 1)^2 = 40 mod q, which drives every split sum to its largest value."""
+    L, K, alpha = 20, 3, 7
+    p = Params(L, K, alpha)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    B = 10
+    dig = _res((B, p.dnum, L + K, N), mods, 700)
+    key = _res((p.dnum, 2, L + K, N), mods, 701)
+    for g in (1, 5, 4095):
+        got = host(ctx.key_inner(dev(dig), dev(key), g))
+        assert_bits_equal(got, orc.key_inner(dig, key, g, mods, L, K, alpha), "key_inner, 10 ct, g=%d" % g)
+    ctx.device_status()
+    ct = _res((B, 2, L, N), mods[:L], 702)
+    keys = [_res((p.dnum, 2, L + K, N), mods, 703 + r) for r in range(2)]
+    gal = np.array([5, 4095], dtype=np.uint64)
+    want = orc.rotate(ct, keys, gal, mods, L, K, alpha)
+    assert_bits_equal(host(ctx.rotate(dev(ct), [dev(k) for k in keys], list(gal))), want, "rotate, 10 ct")
+    want_u = orc.rotate_unhoisted(ct, keys, gal, mods, L, K, alpha)
+    assert_bits_equal(host(ctx.rotate_unhoisted(dev(ct), [dev(k) for k in keys], list(gal))), want_u,
+                      "rotate_unhoisted, 10 ct")
+    ctx.device_status()
+    ctx1 = context(40, 1, 1)
+    m1 = torch.tensor(np.array(ctx1.mods, dtype=np.uint64).view(np.int64), device="cuda")
+    top = (m1 - 1).view(1, 1, 41, 1)
+    acc = host(ctx1.key_inner(top.expand(9, 40, 41, N).contiguous(), top.expand(40, 2, 41, N).contiguous(), 5))
+    ctx1.device_status()
+    want_top = np.broadcast_to((40 % np.array(ctx1.mods, dtype=np.uint64))[None, None, :, None], (9, 2, 41, N))
+    assert_bits_equal(acc, want_top, "key inner product of all-(q - 1) words, 9 ct")
+
+
 def test_refresh_n2048_decodes_to_the_sine_form(orc):
     """The refresh as the oracle's n = 2048 pin runs it (23 + 4 primes, a
     dense ternary secret, three-level factored transforms with their encoded
