@@ -347,6 +347,26 @@ def test_bsgs_shapes(orc, bb, gg):
     assert_bits_equal(y, orc.bsgs(x, diags, baby, giant, bb, gg, mods, 5, 2, 2), "bsgs %dx%d" % (bb, gg))
 
 
+@pytest.mark.parametrize("bb,gg", [(9, 3), (33, 2)])
+def test_bsgs_extreme_residues(orc, bb, gg):
+    """Every diagonal word, key word and the words of ciphertext 0 at q - 1, ciphertext 1 alternating
+    q - 1 with 0: the inner sums over 9 baby values (split sums folded after 8 and after 1 term, 4
+    components per CTA) and 33 (2 per CTA) at their largest, bit-exact against the oracle."""
+    L, K, alpha = 5, 2, 2
+    p = Params(L, K, alpha)
+    ctx = ctx_for(p)
+    mods = np.array(ctx.mods, dtype=np.uint64)
+    ext = _extremes(mods[:L])
+    x = np.ascontiguousarray(np.stack([np.stack([ext[1], ext[1]]), np.stack([ext[2], ext[2][:, ::-1]])]))
+    top = lambda shape, m: np.ascontiguousarray(np.broadcast_to((m - 1)[:, None], shape), dtype=np.uint64)
+    diags = top((gg, bb, L, N), mods[:L])
+    key = top((p.dnum, 2, L + K, N), mods)
+    y = host(ctx.bsgs_lintrans(dev(x), dev(diags), [dev(key)] * (bb - 1), [dev(key)] * (gg - 1), bb, gg))
+    ctx.device_status()
+    want = orc.bsgs(x, diags, [key] * (bb - 1), [key] * (gg - 1), bb, gg, mods, L, K, alpha)
+    assert_bits_equal(y, want, "bsgs %dx%d, extreme words" % (bb, gg))
+
+
 def test_config4_bsgs_full_size(orc):
     """112 primes, alpha = 8, bb = gg = 32, 62 keys, 8 ciphertexts of seeded
     uniform residues: the GPU runs the batch, the oracle recomputes every
