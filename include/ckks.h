@@ -376,7 +376,9 @@ int ckks_mul_relin_rescale(const ckks_ctx *ctx, const uint64_t *a, const uint64_
  * x [batch][2][L][n], diags [gg][bb][L][n] (plaintexts in the NTT domain),
  * baby_keys: bb-1 host pointers (rotation b = 1..bb-1), giant_keys: gg-1
  * host pointers (rotation bb g, g = 1..gg-1), y [batch][2][L-1][n].
- * Requires L >= 2, bb >= 1, gg >= 1.
+ * Requires L >= 2, bb >= 1, gg >= 1.  Ciphertext, diagonal and key words must be
+ * residues, below their prime (the inner sums of up to 64 products below 2^120
+ * are then exact in 128 bits).
  * ws: ckks_workspace_bytes(CKKS_OP_BSGS, batch, bb * 1000 + gg). */
 int ckks_bsgs_lintrans(const ckks_ctx *ctx, const uint64_t *x, const uint64_t *diags,
                        const uint64_t *const *baby_keys, const uint64_t *const *giant_keys,
