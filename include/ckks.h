@@ -247,6 +247,12 @@ int ckks_modup(const ckks_ctx *ctx, const uint64_t *c_ntt, uint64_t *digits, int
  * which every GPU that loads the library holds until the process exits.
  * Limit: batch * L <= 2048.  Larger requests return CKKS_EUNSUPPORTED and
  * launch nothing.
+ * When the context converts on the folded tensor-core engine (the automatic
+ * choice from 8 primes per digit, or CKKS_CONV_FOLDED), that engine's tables
+ * are built, with cudaMalloc, by the first call that converts (ckks_modup,
+ * ckks_keyswitch, ckks_rotate and the other key-switching calls).  Until one
+ * of them has run on the context, this entry point returns CKKS_EUNSUPPORTED
+ * and launches nothing.
  * The first call on a device resolves the array's device address
  * (cudaGetSymbolAddress, once per device); make that first call before any
  * stream capture.  The address is cached for the life of the process and

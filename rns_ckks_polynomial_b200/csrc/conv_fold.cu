@@ -610,6 +610,12 @@ static int ensure_fold_tables(ckks_ctx *ctx)
     return CKKS_OK;
 }
 
+bool fold_tables_ready(const ckks_ctx *ctx)
+{
+    std::lock_guard<std::mutex> lock(const_cast<ckks_ctx *>(ctx)->mu);
+    return ctx->fold_built;
+}
+
 // Windows of at most kWinMax primes: each digit's range and the special primes, each cut into
 // near-equal pieces.
 static void make_windows(const ckks_ctx *ctx, std::vector<ckks_ctx::Window> &out)

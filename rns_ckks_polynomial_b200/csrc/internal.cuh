@@ -38,6 +38,8 @@ constexpr int kTcMinSources = 7;  // CKKS_CONV_AUTO: more sources (8 or more) us
 enum ConvKind { kConvInteger = 0, kConvTensor = 1, kConvFolded = 2 };
 ConvKind conv_kind(const ckks_ctx *ctx, int sources);
 int launch_conv_fold_up(ckks_ctx *ctx, const u64 *y, u64 *digits, int batch, cudaStream_t s);
+// whether the folded tables exist (they are built, with cudaMalloc, by the first folded conversion)
+bool fold_tables_ready(const ckks_ctx *ctx);
 // streamed rotation: prime windows of at most kWinMax primes (built with their folded blocks on
 // first use) and the conversion of y into window w's buffer [batch][dnum][kWinMax][n]
 constexpr int kWinMax = 60;

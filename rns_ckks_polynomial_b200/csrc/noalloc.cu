@@ -56,6 +56,11 @@ extern "C" int ckks_modup_noalloc(const ckks_ctx *ctx, const uint64_t *c_ntt, ui
     CKKS_TRY(check_ptr(digits, "digits"));
     if (ctx->device < 0 || ctx->device >= kMaxDevices)
         return set_error(CKKS_EUNSUPPORTED, "device index above 63");
+    // the folded conversion builds its tables on first use, which allocates: refuse until they exist
+    if (conv_kind(ctx, ctx->alpha) == kConvFolded && !fold_tables_ready(ctx))
+        return set_error(CKKS_EUNSUPPORTED,
+                         "ckks_modup_noalloc: the folded conversion tables are not built yet (make one "
+                         "converting call, e.g. ckks_modup, on this context first)");
     CKKS_TRY(set_device(ctx));
     void *scratch = nullptr;
     CKKS_TRY(scratch_address(ctx->device, &scratch));

@@ -70,3 +70,35 @@ def test_modup_noalloc_rejects_oversized_batch():
     rc = lib.ckks_modup_noalloc(ctx._h, None, None, 19, None)  # 19 * 112 > 2048 limbs
     assert rc == -2
     assert b"2048-limb" in lib.ckks_last_error()
+
+
+def test_modup_noalloc_refuses_before_the_folded_tables_exist():
+    """On a fresh context whose digits of 8 primes convert on the folded tensor-core engine, the
+    tables do not exist until a converting call builds them (with cudaMalloc). Until then the entry
+    point returns CKKS_EUNSUPPORTED, launches nothing and leaves the device's free memory as it
+    was; after one ckks_modup it gives ckks_modup's words."""
+    need_gpu()
+    import oracle
+    from rns_ckks_polynomial_b200 import Context
+    L, K, alpha, batch = 24, 8, 8, 2
+    mods = [int(x) for x in oracle.gen_primes(N, L + K)]
+    ctx = Context(mods[:L], mods[L:], alpha)  # not the shared cached context: no call has run on it
+    lib = native.lib()
+    stream = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    c = synth.uniform_residues((batch, L, N), mods[:L], synth.config_seed(9), 400, device="cuda")
+    out = torch.full((batch, ctx.dnum, L + K, N), -1, dtype=torch.int64, device="cuda")
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    rc = lib.ckks_modup_noalloc(ctx._h, C.c_void_p(c.data_ptr()), C.c_void_p(out.data_ptr()), batch, stream)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert rc == -2
+    assert b"folded conversion tables" in lib.ckks_last_error()
+    assert free_after == free_before
+    assert bool((out == -1).all()), "a refused call wrote its output"
+    ref = ctx.modup(c)
+    rc = lib.ckks_modup_noalloc(ctx._h, C.c_void_p(c.data_ptr()), C.c_void_p(out.data_ptr()), batch, stream)
+    assert rc == 0, lib.ckks_last_error()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    ctx.device_status()
