@@ -139,6 +139,36 @@ def test_ntt_empty_and_errors():
     assert rc == -1 and "aligned" in lib.ckks_last_error().decode()
 
 
+
+def test_key_switch_calls_accept_empty_inputs():
+    """An empty batch (or no keys) is a no-op for every key-switching call: each returns CKKS_OK with
+    null data pointers, so it reads, writes and launches nothing; a negative batch is CKKS_EINVAL."""
+    ctx = context(20, 3, 7)
+    lib = native.lib()
+    h, nul = ctx._h, None
+    no_keys = (C.c_void_p * 1)()
+    no_gal = (C.c_uint32 * 1)()
+    calls = {
+        "modup": lambda b: lib.ckks_modup(h, nul, nul, b, nul, nul),
+        "modup_noalloc": lambda b: lib.ckks_modup_noalloc(h, nul, nul, b, nul),
+        "key_inner": lambda b: lib.ckks_key_inner(h, nul, nul, 5, nul, b, nul),
+        "moddown": lambda b: lib.ckks_moddown(h, nul, nul, b, nul, nul),
+        "keyswitch": lambda b: lib.ckks_keyswitch(h, nul, nul, nul, b, nul, nul),
+        "rotate": lambda b: lib.ckks_rotate(h, nul, no_keys, no_gal, 1, nul, b, nul, nul),
+        "rotate_unhoisted": lambda b: lib.ckks_rotate_unhoisted(h, nul, no_keys, no_gal, 1, nul, b, nul, nul),
+        "rotate_streamed": lambda b: lib.ckks_rotate_streamed(h, nul, no_keys, no_gal, 1, nul, b, nul, nul),
+        "rescale": lambda b: lib.ckks_rescale(h, nul, nul, 20, b, nul, nul),
+        "mul_relin_rescale": lambda b: lib.ckks_mul_relin_rescale(h, nul, nul, nul, nul, b, nul, nul),
+        "bsgs_lintrans": lambda b: lib.ckks_bsgs_lintrans(h, nul, nul, None, None, 1, 1, nul, b, nul, nul),
+    }
+    for name, call in calls.items():
+        assert call(0) == 0, (name, lib.ckks_last_error())
+        assert call(-1) == -1, name
+    for fn in (lib.ckks_rotate, lib.ckks_rotate_unhoisted, lib.ckks_rotate_streamed):
+        assert fn(h, nul, no_keys, no_gal, 0, nul, 3, nul, nul) == 0  # no keys, a non-empty batch
+    torch.cuda.synchronize()
+    ctx.device_status()
+
 # ------------------------------------------------------------------ pointwise / automorphism
 @pytest.mark.parametrize("op", ["mul", "add", "sub"])
 def test_pointwise(orc, op):
