@@ -217,15 +217,19 @@ def traffic_for(kernel_key):
 def intpipe_peaks(ctx):
     """Same-run microbenchmarks over the whole GPU: Shoup multiplies/s,
     64x64->128 MACs/s and 64-bit high multiplies/s on the integer pipes, the
-    forward NTT's own butterfly (kind 5), and int8 tcgen05.mma ops/s at
+    forward NTT's own butterfly (kind 5), the key inner product's split-form
+    product (kind 6, for primes 2^60 - delta), and int8 tcgen05.mma ops/s at
     N = 256 (dense rate) and N = 32 (the basis conversion's tile), one
     issuing thread per SM."""
     out = {}
-    for kind, name in ((0, "shoup_mulmod_per_s"), (1, "mac128_per_s"), (2, "mulhi64_per_s"),
-                       (5, "ntt_butterfly_per_s")):
+    kinds = [(0, "shoup_mulmod_per_s", 2048), (1, "mac128_per_s", 2048), (2, "mulhi64_per_s", 2048),
+             (5, "ntt_butterfly_per_s", 2048)]
+    if all(q < 1 << 60 and (1 << 60) - q < 1 << 32 for q in ctx.mods):  # every prime 2^60 - delta
+        kinds.append((6, "split_mac_per_s", 256))
+    for kind, name, iters in kinds:
         best = 0.0
         for _ in range(3):
-            ms, ops = ctx.bench_intpipe(kind, 148 * 8, 2048)
+            ms, ops = ctx.bench_intpipe(kind, 148 * 8, iters)
             best = max(best, ops / (ms * 1e-3))
         out[name] = best
     for kind, name in ((3, "int8_mma_n256_ops_per_s"), (4, "int8_mma_n32_ops_per_s")):
@@ -240,7 +244,8 @@ def intpipe_peaks(ctx):
 def rates_from(ipeak):
     """Per-operation rates of the roofline model (operations per second)."""
     return {"bfly": ipeak["ntt_butterfly_per_s"], "mm": ipeak["shoup_mulmod_per_s"],
-            "mac": ipeak["mac128_per_s"], "int8_mac": ipeak["int8_mma_n256_ops_per_s"] / 2}
+            "mac": ipeak["mac128_per_s"], "int8_mac": ipeak["int8_mma_n256_ops_per_s"] / 2,
+            "kmac": ipeak.get("split_mac_per_s", ipeak["mac128_per_s"])}
 
 
 def ntt_roofline(limbs, k_ms, hbm_peak, peak_src, ipeak):
@@ -613,11 +618,12 @@ NTT_BFLY = (N // 2) * 11  # butterflies per limb transform, one modular product 
 TC_MIN_SOURCES = 8        # conversions with this many source primes run on the int8 tensor cores
 
 
-def work(bfly=0, mm=0, mac=0, conv_tc=0, bytes=0):
-    """Algorithmic work: NTT butterflies, other modular products, 64x64->128
-    multiply-adds (mac) of which conv_tc run as basis conversions on the int8
-    tensor cores, and the minimum bytes that cross HBM."""
-    return {"bfly": bfly, "mm": mm, "mac": mac, "conv_tc": conv_tc, "bytes": bytes}
+def work(bfly=0, mm=0, mac=0, conv_tc=0, kmac=0, bytes=0):
+    """Algorithmic work: NTT butterflies, other modular products, 60x60-bit
+    multiply-adds (mac), of which conv_tc run as basis conversions on the int8
+    tensor cores and kmac are the key inner product's, and the minimum bytes
+    that cross HBM."""
+    return {"bfly": bfly, "mm": mm, "mac": mac, "conv_tc": conv_tc, "kmac": kmac, "bytes": bytes}
 
 
 def work_sum(*parts, times=1):
@@ -643,7 +649,7 @@ def ks_work_keyswitch_parts(L, K, alpha, engine="auto"):
             conv_up_tc += S * (LK - S) * N
     conv_dn = 2 * K * L * N
     modup = work(bfly=(L + new_limbs) * NTT_BFLY, mm=L * N, mac=conv_up, conv_tc=conv_up_tc)
-    inner = work(mac=2 * dnum * LK * N)
+    inner = work(mac=2 * dnum * LK * N, kmac=2 * dnum * LK * N)
     moddown = work(bfly=2 * (K + L) * NTT_BFLY, mm=2 * (K + L) * N, mac=conv_dn,
                    conv_tc=conv_dn if tc and K >= TC_MIN_SOURCES else 0)
     return modup, inner, moddown
@@ -695,15 +701,18 @@ def work_bsgs(L, K, alpha, B, bb, gg):
 
 
 def model_seconds(w, rates, hbm_peak, engine_tc=True):
-    """(ALU seconds, HBM seconds) of a work dict.  With engine_tc the
-    conversions counted in conv_tc are charged as 64 int8 byte-plane
-    multiply-adds per 60-bit multiply-add at the same-run dense int8 rate;
-    otherwise every multiply-add is charged at the 128-bit MAC rate."""
-    t = w["bfly"] / rates["bfly"] + w["mm"] / rates["mm"]
+    """(ALU seconds, HBM seconds) of a work dict.  The key inner product's
+    multiply-adds (kmac) are charged at the same-run rate of its own split-form
+    product (rates["kmac"]).  With engine_tc the conversions counted in conv_tc
+    are charged as 64 int8 byte-plane multiply-adds per 60-bit multiply-add at
+    the same-run dense int8 rate; otherwise they too run at the 128-bit MAC
+    rate, as do the other multiply-adds."""
+    t = w["bfly"] / rates["bfly"] + w["mm"] / rates["mm"] + w["kmac"] / rates.get("kmac", rates["mac"])
+    rest = w["mac"] - w["kmac"]
     if engine_tc:
-        t += (w["mac"] - w["conv_tc"]) / rates["mac"] + w["conv_tc"] * 64 / rates["int8_mac"]
+        t += (rest - w["conv_tc"]) / rates["mac"] + w["conv_tc"] * 64 / rates["int8_mac"]
     else:
-        t += w["mac"] / rates["mac"]
+        t += rest / rates["mac"]
     return t, w["bytes"] / (hbm_peak * 1e9)
 
 
@@ -712,8 +721,9 @@ def ks_entry(nks, ms, w, hbm_peak, rates, clocks=None):
     its bytes at the measured HBM rate and its operations at the same-run
     rates of the engines that actually ran) / measured time.  NTT butterflies
     are charged at the kernel's own butterfly rate, other modular products at
-    the Shoup rate, multiply-adds at the 128-bit MAC rate, and conversions on
-    the tensor cores at the dense int8 rate.  integer_pipe_model_frac charges
+    the Shoup rate, the key inner product's multiply-adds at the rate of its
+    own split-form product, other multiply-adds at the 128-bit MAC rate, and
+    conversions on the tensor cores at the dense int8 rate.  integer_pipe_model_frac charges
     every multiply-add to the integer pipes instead: a model the tensor-core
     path can exceed, so it is reported, not used as the bound."""
     t = ms * 1e-3
@@ -721,6 +731,7 @@ def ks_entry(nks, ms, w, hbm_peak, rates, clocks=None):
     bound = "alu" if t_alu >= t_hbm else "hbm"
     out = {"keyswitches_per_s": nks / t, "ms_per_call": ms, "keyswitches_per_call": nks,
            "butterflies": w["bfly"], "mulmods": w["mm"], "macs": w["mac"], "macs_on_tensor_cores": w["conv_tc"],
+           "macs_key_inner": w["kmac"],
            "min_bytes": w["bytes"], "bound": bound, "roofline_frac": max(t_alu, t_hbm) / t,
            "alu_frac": t_alu / t, "hbm_frac": t_hbm / t,
            "conversion": "int8 tensor cores, folded form" if w["conv_tc"] else "integer pipes"}

@@ -469,7 +469,13 @@ int ckks_modraise(const ckks_ctx *ctx, const uint64_t *in, int l, uint64_t *out,
  * forward NTT's own butterfly (Shoup product with the three-partial-product
  * quotient, the cheap quotient-times-q for 2^60 - delta primes when every
  * prime of the context has that form, and the lazy add/sub; *ops counts
- * butterflies, one modular product each).
+ * butterflies, one modular product each); kind 6: the key inner product's
+ * split form without its loads (each iteration runs 8 words per chain, 8
+ * chains: a word split into 30-bit halves once and multiplied into the
+ * three-sum accumulators of two key words with the Karatsuba middle product,
+ * the sums folded every 8 words; *ops counts 60 x 60-bit products; only for
+ * contexts whose primes are all 2^60 - delta, else CKKS_EUNSUPPORTED;
+ * iters <= 2^26).
  * Tensor-pipe kinds (one issuing thread per CTA of 128 threads, `iters`
  * back-to-back int8 tcgen05.mma of M = 128, K = 32; *ops counts 2 M N K per
  * MMA): kind 3: N = 256 (the dense int8 rate); kind 4: N = 32 (the basis

@@ -410,7 +410,8 @@ class Context:
     def bench_intpipe(self, kind, blocks, iters):
         """(ms, ops) of the microbenchmark `kind`: 0 Shoup mulmod, 1 64x64->128
         MAC, 2 64-bit high multiply, 3 / 4 int8 tcgen05.mma at N = 256 / 32,
-        5 the forward NTT's butterfly."""
+        5 the forward NTT's butterfly, 6 the key inner product's split-form
+        product (primes 2^60 - delta only)."""
         ms, ops = C.c_double(), C.c_double()
         check("ckks_bench_intpipe",
               lib().ckks_bench_intpipe(self._h, kind, blocks, iters, C.byref(ms), C.byref(ops)))

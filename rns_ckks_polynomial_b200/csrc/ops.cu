@@ -5,6 +5,7 @@
 
 #include "internal.cuh"
 #include "ntt.cuh"
+#include "split.cuh"
 
 namespace ckks {
 
@@ -744,6 +745,43 @@ __device__ __forceinline__ void bfly_loop(u64 x[8], int iters, u64 q, u64 w, u64
     }
 }
 
+// Kind 6, the key inner product's split form without its loads, in a kernel of its own so that its
+// 48 sums do not raise the register count (and lower the occupancy) of the other kinds: per step a
+// new word per chain, split once and multiplied into the sums of two key words (the kernel's two
+// components), the sums folded every kSplitFold words.
+__global__ void splitmac_kernel(int iters, u64 q, u64 w, u64 *sink)
+{
+    u64 x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = (threadIdx.x * 8 + k + 1) * 0x9E3779B97F4A7C15ull % q;
+    const Split30 kw0 = split30(w), kw1 = split30(q - 1 - w);
+    const u32 delta = (u32)(((u64)1 << 60) - q);
+    u64 s[8][2][3];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) s[k][c][0] = s[k][c][1] = s[k][c][2] = 0;
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int u = 0; u < kSplitFold; ++u) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const Split30 d = split30(x[k] ^ (u64)(it * kSplitFold + u));  // stays below 2^60
+                split_mac(s[k][0][0], s[k][0][1], s[k][0][2], d, kw0);
+                split_mac(s[k][1][0], s[k][1][1], s[k][1][2], d, kw1);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) split_fold(s[k][c][0], s[k][c][1], s[k][c][2], delta);
+    }
+    u64 acc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc ^= s[k][0][0] ^ s[k][0][2] ^ s[k][1][0] ^ s[k][1][2];
+    if (acc == 0x1234567ull) sink[threadIdx.x] = acc;  // keeps the loop alive
+}
+
 __global__ void intpipe_kernel(int kind, int iters, u64 q, u64 w, u64 wp, int special, u64 *sink)
 {
     u64 x[8], h[8];
@@ -786,8 +824,11 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
                                   double *ops)
 {
     CKKS_TRY(check_ctx(ctx));
-    if (kind < 0 || kind > 5 || blocks < 1 || blocks > 148 * 64 || iters < 1 || !ms || !ops)
+    if (kind < 0 || kind > 6 || blocks < 1 || blocks > 148 * 64 || iters < 1 || !ms || !ops)
         return set_error(CKKS_EINVAL, "bad microbenchmark arguments");
+    if (kind == 6 && !ctx->t.special)
+        return set_error(CKKS_EUNSUPPORTED, "the split-form microbenchmark needs primes 2^60 - delta");
+    if (kind == 6 && iters > (1 << 26)) return set_error(CKKS_EINVAL, "too many iterations for kind 6");
     CKKS_TRY(set_device(ctx));
     if (kind == 3 || kind == 4) return bench_mma(ctx, kind == 3 ? 256 : 32, blocks, iters, ms, ops);
     const u64 q = ctx->mods[0];
@@ -799,9 +840,15 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
     cudaEventCreate(&a);
     cudaEventCreate(&b);
     const int special = ctx->t.special ? 1 : 0;
-    intpipe_kernel<<<blocks, 256>>>(kind, std::max(1, iters / 16), q, w, wp, special, sink);  // warm-up
+    if (kind == 6)
+        splitmac_kernel<<<blocks, 256>>>(std::max(1, iters / 16), q, w, sink);  // warm-up
+    else
+        intpipe_kernel<<<blocks, 256>>>(kind, std::max(1, iters / 16), q, w, wp, special, sink);
     cudaEventRecord(a);
-    intpipe_kernel<<<blocks, 256>>>(kind, iters, q, w, wp, special, sink);
+    if (kind == 6)
+        splitmac_kernel<<<blocks, 256>>>(iters, q, w, sink);
+    else
+        intpipe_kernel<<<blocks, 256>>>(kind, iters, q, w, wp, special, sink);
     cudaEventRecord(b);
     e = cudaEventSynchronize(b);
     float t = 0;
@@ -811,6 +858,6 @@ extern "C" int ckks_bench_intpipe(const ckks_ctx *ctx, int kind, int blocks, int
     cudaFree(sink);
     if (e != cudaSuccess) return cuda_status(e, "intpipe_kernel");
     *ms = t;
-    *ops = (double)blocks * 256.0 * iters * (kind == 5 ? 4.0 : 8.0);
+    *ops = (double)blocks * 256.0 * iters * (kind == 5 ? 4.0 : kind == 6 ? 8.0 * 2 * kSplitFold : 8.0);
     return CKKS_OK;
 }

@@ -58,6 +58,24 @@ def test_model_charges_the_engine_that_ran():
     assert e2["roofline_frac"] == pytest.approx(1.0)
 
 
+def test_key_inner_products_charged_at_their_own_rate():
+    """The key inner product's multiply-adds (kmac, part of mac) are charged at the
+    rate of its split-form product; the other multiply-adds stay at the 128-bit rate."""
+    up, inner, down = bench.ks_work_keyswitch_parts(2100, 60, 60)
+    assert inner["kmac"] == inner["mac"] == 2 * 35 * 2160 * 2048
+    assert up["kmac"] == 0 and down["kmac"] == 0
+    rates = {"bfly": 1e12, "mm": 1e12, "mac": 1e12, "int8_mac": 64e12, "kmac": 2e12}
+    w = bench.work(mac=3 * 10**12, kmac=2 * 10**12)
+    t, _ = bench.model_seconds(w, rates, 1e3)
+    assert t == pytest.approx(1.0 + 1.0)
+    assert bench.ks_entry(1, 4000.0, w, 1e3, rates)["macs_key_inner"] == 2 * 10**12
+    # without a measured split-form rate, kmac falls back to the 128-bit rate
+    del rates["kmac"]
+    assert bench.model_seconds(w, rates, 1e3)[0] == pytest.approx(3.0)
+    assert bench.rates_from({"ntt_butterfly_per_s": 1, "shoup_mulmod_per_s": 1, "mac128_per_s": 5,
+                             "int8_mma_n256_ops_per_s": 2})["kmac"] == 5
+
+
 def test_ntt_launch_bytes_and_products():
     bytes_, mm = bench.ntt_launch_work(2100)
     assert bytes_ == 33600 * 2 * 2048 * 8 + 2100 * 2048 * 16

@@ -482,19 +482,27 @@ def test_config5_boot_rotation_full_size(orc):
         ctx.set_conversion("auto")
 
 
-def test_microbenchmarks_report_counts():
+def test_microbenchmarks_report_counts(orc):
     """The roofline denominators: every kind runs, reports its own operation
-    count and leaves the device flag clear; bad kinds are rejected."""
+    count and leaves the device flag clear; bad kinds are rejected, and the
+    split-form kind 6 only runs where every prime is 2^60 - delta."""
+    from rns_ckks_polynomial_b200 import Context
     ctx = ctx_for(Params(4, 1, 1))
     for kind, blocks, iters, per in ((0, 16, 64, 256 * 8), (1, 16, 64, 256 * 8), (2, 16, 64, 256 * 8),
                                      (3, 4, 64, 2 * 128 * 256 * 32), (4, 4, 64, 2 * 128 * 32 * 32),
-                                     (5, 16, 64, 256 * 4)):
+                                     (5, 16, 64, 256 * 4), (6, 16, 8, 256 * 8 * 2 * 8)):
         ms, ops = ctx.bench_intpipe(kind, blocks, iters)
         assert ms > 0
         assert ops == blocks * iters * per
     ctx.device_status()
-    with pytest.raises(CkksError):
-        ctx.bench_intpipe(6, 1, 1)
+    with pytest.raises(CkksError) as e:
+        ctx.bench_intpipe(7, 1, 1)
+    assert e.value.code == -1
+    mods = _general_primes(orc, 5)
+    gctx = Context(mods[:4], mods[4:], 1)
+    with pytest.raises(CkksError) as e:
+        gctx.bench_intpipe(6, 1, 1)
+    assert e.value.code == -2
 
 
 def _general_primes(orc, count):
